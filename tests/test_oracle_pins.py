@@ -1,0 +1,432 @@
+"""Pins of the CPU oracle against mathematics that does not come from the oracle.
+
+Each test checks one oracle function against something independent of its code:
+values derived by hand from the documented router order (tests/golden), brute
+force over all k-subsets, exact integer arithmetic, library routines (numpy's
+stable argsort, torch's gelu/silu and matmul), a dense evaluate-every-expert
+reference, the E=1/k=1 closed form, permutation equivariance, linearity and fp64
+central finite differences.  A plausible mistake in the oracle (a dropped term, a
+wrong sign or index, a transposed operand, a wrong reduction order) fails at least
+one of them.  All tests are CPU-only and small.
+"""
+import itertools
+import json
+import os
+
+import numpy as np
+import pytest
+import torch
+import torch.nn.functional as F
+
+import oracle
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _rng(seed):
+    return np.random.default_rng(seed)
+
+
+# --------------------------------------------------------------------------
+# router logits
+# --------------------------------------------------------------------------
+def test_router_logits_documented_order_golden():
+    spec = json.load(open(os.path.join(GOLDEN, "router_order_cases.json")))
+    d, E = spec["d"], spec["E"]
+    for case in spec["cases"]:
+        x = np.zeros((1, d), np.float32)
+        w = np.ones((d, E), np.float32)
+        for i, v in case["x"].items():
+            x[0, int(i)] = v
+        for i, v in case["w"].items():
+            w[int(i), 0] = v
+        got = oracle.router_logits_f32(x, w)[0, 0]
+        assert got == np.float32(case["expected"]), (case["name"], float(got), case["expected"])
+
+
+def test_router_logits_exact_integer_indexing():
+    # small integers: every fp32 operation is exact, so the logits equal the
+    # integer dot products whatever the order -- pins the x / W_r / b indexing
+    r = _rng(1)
+    T, d, E = 7, 40, 5
+    x = r.integers(-3, 4, (T, d)).astype(np.float32)
+    w = r.integers(-3, 4, (d, E)).astype(np.float32)
+    b = r.integers(-5, 6, E).astype(np.float32)
+    want = x.astype(np.int64) @ w.astype(np.int64) + b.astype(np.int64)
+    got = oracle.router_logits_f32(x, w, b)
+    np.testing.assert_array_equal(got, want.astype(np.float32))
+    np.testing.assert_array_equal(oracle.router_logits_f64(x, w, b), want.astype(np.float64))
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_router_logits_within_fp32_error_bound(dtype):
+    # forward error bound of an fp32 dot product of length d: gamma_d * sum|x w|
+    g = torch.Generator().manual_seed(3)
+    T, d, E = 33, 256, 8
+    x = torch.randn(T, d, generator=g).to(dtype)
+    w = (torch.randn(d, E, generator=g) / 16).to(dtype)
+    l32 = oracle.router_logits_f32(x, w).astype(np.float64)
+    l64 = oracle.router_logits_f64(x, w)
+    xd, wd = x.double().numpy(), w.double().numpy()
+    np.testing.assert_allclose(l64, xd @ wd, rtol=0, atol=1e-12)
+    u = 2.0 ** -24
+    gamma = d * u / (1 - d * u)
+    bound = gamma * (np.abs(xd) @ np.abs(wd))
+    assert np.all(np.abs(l32 - l64) <= bound + 1e-30)
+
+
+# --------------------------------------------------------------------------
+# top-k and gates
+# --------------------------------------------------------------------------
+def test_topk_matches_brute_force_subsets():
+    r = _rng(2)
+    T, E, k = 60, 7, 3
+    logits = r.standard_normal((T, E)).astype(np.float32)
+    idx, gates = oracle.topk_gates(logits, k)
+    for t in range(T):
+        best = max(itertools.combinations(range(E), k),
+                   key=lambda s: sum(float(logits[t, e]) for e in s))
+        assert set(idx[t]) == set(best)
+        vals = [logits[t, e] for e in idx[t]]
+        assert all(vals[j] >= vals[j + 1] for j in range(k - 1))
+        sel = logits[t, idx[t]].astype(np.float64)
+        ex = np.exp(sel - sel.max())
+        np.testing.assert_allclose(gates[t], ex / ex.sum(), rtol=1e-15, atol=0)
+
+
+def test_topk_gates_equal_softmax_topk_renormalised():
+    r = _rng(4)
+    T, E, k = 100, 16, 4
+    logits = (3 * r.standard_normal((T, E))).astype(np.float32)
+    idx, gates = oracle.topk_gates(logits, k)
+    p = torch.softmax(torch.from_numpy(logits).double(), dim=-1)
+    top = torch.topk(p, k, dim=-1)
+    ren = top.values / top.values.sum(-1, keepdim=True)
+    assert np.array_equal(np.sort(idx, 1), np.sort(top.indices.numpy(), 1))
+    np.testing.assert_allclose(gates, ren.numpy(), rtol=1e-13, atol=1e-15)
+    np.testing.assert_allclose(gates.sum(1), 1.0, rtol=0, atol=1e-15)
+
+
+def test_topk_ties_go_to_lower_expert():
+    logits = np.array([[1.0, 2.0, 2.0, 0.5, 2.0],
+                       [0.0, 0.0, 0.0, 0.0, 0.0]], np.float32)
+    idx, gates = oracle.topk_gates(logits, 3)
+    assert idx.tolist() == [[1, 2, 4], [0, 1, 2]]
+    np.testing.assert_allclose(gates, 1.0 / 3.0, rtol=1e-15)
+
+
+# --------------------------------------------------------------------------
+# sort
+# --------------------------------------------------------------------------
+@pytest.mark.parametrize("T,k,E", [(1, 1, 1), (50, 2, 8), (300, 8, 64), (17, 4, 5)])
+def test_sort_matches_numpy_stable_argsort(T, k, E):
+    r = _rng(T * 31 + E)
+    idx = r.integers(0, E, (T, k)).astype(np.int32)
+    if E > 3:
+        idx[idx == 3] = 2  # an empty expert
+    ss, off = oracle.sort(idx, E)
+    np.testing.assert_array_equal(ss, np.argsort(idx.ravel(), kind="stable"))
+    counts = np.bincount(idx.ravel(), minlength=E)
+    np.testing.assert_array_equal(off, np.concatenate([[0], np.cumsum(counts)]))
+    # invariants: each slot once, experts non-decreasing, slots ascending per expert
+    assert sorted(ss.tolist()) == list(range(T * k))
+    e_sorted = idx.ravel()[ss]
+    assert np.all(np.diff(e_sorted) >= 0)
+    for e in range(E):
+        seg = ss[off[e]:off[e + 1]]
+        assert np.all(np.diff(seg) > 0)
+
+
+# --------------------------------------------------------------------------
+# activations
+# --------------------------------------------------------------------------
+def test_activations_against_torch_and_closed_forms():
+    z = np.concatenate([np.linspace(-8, 8, 161), [0.0, 30.0, -30.0, 1e-3, -1e-3]])
+    zt = torch.from_numpy(z).requires_grad_(True)
+    for kind, fn in [("gelu", lambda t: F.gelu(t, approximate="tanh")), ("silu", F.silu)]:
+        v, g = oracle.act(kind, z)
+        ref = fn(zt)
+        (gr,) = torch.autograd.grad(ref.sum(), zt)
+        np.testing.assert_allclose(v, ref.detach().numpy(), rtol=1e-14, atol=1e-15)
+        np.testing.assert_allclose(g, gr.numpy(), rtol=1e-12, atol=1e-14)
+        assert v[161] == 0.0                      # act(0) = 0
+        assert abs(v[162] - 30.0) < 1e-10         # ~ identity for large z
+        assert abs(v[163]) < 1e-10                # ~ 0 for very negative z
+    # derivative by central difference
+    h = 1e-6
+    for kind in ("gelu", "silu"):
+        vp, _ = oracle.act(kind, z + h)
+        vm, _ = oracle.act(kind, z - h)
+        _, g = oracle.act(kind, z)
+        np.testing.assert_allclose((vp - vm) / (2 * h), g, rtol=1e-7, atol=1e-8)
+
+
+# --------------------------------------------------------------------------
+# SMoE MLP forward
+# --------------------------------------------------------------------------
+def _tiny_mlp(seed, T, d, f, E, k, act, dtype=torch.float64):
+    g = torch.Generator().manual_seed(seed)
+    m = 2 if act == "swiglu" else 1
+    x = torch.randn(T, d, generator=g, dtype=torch.float64).to(dtype)
+    w_r = (torch.randn(d, E, generator=g, dtype=torch.float64) / d ** 0.5).to(dtype)
+    w1 = (torch.randn(E, d, m * f, generator=g, dtype=torch.float64) / d ** 0.5).to(dtype)
+    w2 = (torch.randn(E, f, d, generator=g, dtype=torch.float64) / f ** 0.5).to(dtype)
+    dy = torch.randn(T, d, generator=g, dtype=torch.float64)
+    return x, w_r, w1, w2, dy
+
+
+def _dense_masked_reference(x, w1, w2, act, idx, gates):
+    """Evaluate every expert on every token, then keep the top-k with their gates."""
+    X, W1, W2 = x.double(), w1.double(), w2.double()
+    T, E, f = X.shape[0], W1.shape[0], W2.shape[1]
+    outs = []
+    for e in range(E):
+        H = X @ W1[e]
+        A = F.gelu(H, approximate="tanh") if act == "gelu" else F.silu(H[:, :f]) * H[:, f:]
+        outs.append(A @ W2[e])
+    Y = torch.stack(outs, 1)                          # [T, E, d]
+    mask = torch.zeros(T, E, dtype=torch.float64)
+    mask.scatter_(1, torch.from_numpy(idx).long(), torch.from_numpy(gates))
+    return (mask[:, :, None] * Y).sum(1).numpy()
+
+
+@pytest.mark.parametrize("act", ["gelu", "swiglu"])
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_mlp_fwd_equals_dense_masked_reference(act, dtype):
+    x, w_r, w1, w2, _ = _tiny_mlp(5, 24, 16, 12, 6, 2, act, dtype)
+    idx, gates = oracle.route(x, w_r, None, 2)
+    out = oracle.mlp_fwd(x, w1, w2, act, idx, gates, want_ha=True)
+    ref = _dense_masked_reference(x, w1, w2, act, idx, gates)
+    np.testing.assert_allclose(out["y"], ref, rtol=1e-12, atol=1e-12)
+    # the saved pre-activation of slot (t, j) is x_t W1[e]
+    X, W1 = x.double(), w1.double()
+    for p in [0, 7, 47]:
+        t, j = divmod(p, 2)
+        np.testing.assert_allclose(out["h"][p], (X[t] @ W1[idx[t, j]]).numpy(), rtol=1e-12,
+                                   atol=1e-12)
+
+
+@pytest.mark.parametrize("act", ["gelu", "swiglu"])
+def test_mlp_single_expert_is_dense_mlp(act):
+    x, w_r, w1, w2, dy = _tiny_mlp(6, 10, 8, 6, 1, 1, act, torch.float32)
+    idx, gates = oracle.route(x, w_r, None, 1)
+    assert np.all(idx == 0) and np.all(gates == 1.0)
+    X, W1, W2 = x.double(), w1.double()[0], w2.double()[0]
+    f = W2.shape[0]
+    H = X @ W1
+    A = F.gelu(H, approximate="tanh") if act == "gelu" else F.silu(H[:, :f]) * H[:, f:]
+    np.testing.assert_allclose(oracle.mlp_fwd(x, w1, w2, act, idx, gates)["y"], (A @ W2).numpy(),
+                               rtol=1e-12, atol=1e-12)
+    full = oracle.mlp_bwd_full(x, w_r, w1, w2, act, idx, gates, dy)
+    assert np.all(full["dw_r"] == 0.0) and np.all(full["db_r"] == 0.0)
+
+
+def test_mlp_linear_in_w2():
+    x, w_r, w1, w2, _ = _tiny_mlp(7, 12, 8, 6, 4, 2, "swiglu", torch.float32)
+    idx, gates = oracle.route(x, w_r, None, 2)
+    y1 = oracle.mlp_fwd(x, w1, w2, "swiglu", idx, gates)["y"]
+    y3 = oracle.mlp_fwd(x, w1, w2 * 4, "swiglu", idx, gates)["y"]
+    np.testing.assert_allclose(y3, 4 * y1, rtol=1e-13, atol=1e-14)
+
+
+@pytest.mark.parametrize("act", ["gelu", "swiglu"])
+def test_mlp_token_permutation_equivariance(act):
+    x, w_r, w1, w2, dy = _tiny_mlp(8, 20, 8, 6, 4, 2, act, torch.float32)
+    idx, gates = oracle.route(x, w_r, None, 2)
+    perm = np.random.default_rng(0).permutation(20)
+    a = oracle.mlp_bwd_full(x, w_r, w1, w2, act, idx, gates, dy)
+    b = oracle.mlp_bwd_full(x[perm], w_r, w1, w2, act, idx[perm], gates[perm], dy[perm])
+    ya = oracle.mlp_fwd(x, w1, w2, act, idx, gates)["y"]
+    yb = oracle.mlp_fwd(x[perm], w1, w2, act, idx[perm], gates[perm])["y"]
+    np.testing.assert_allclose(yb, ya[perm], rtol=1e-14, atol=1e-14)
+    for key in ("dx", "dg"):
+        np.testing.assert_allclose(b[key], a[key][perm], rtol=1e-12, atol=1e-13)
+    for key in ("dw1", "dw2", "dw_r", "db_r"):
+        np.testing.assert_allclose(b[key], a[key], rtol=1e-11, atol=1e-12)
+
+
+# --------------------------------------------------------------------------
+# SMoE MLP backward: fp64 central finite differences through the whole layer
+# --------------------------------------------------------------------------
+def _route_with_margin(x, w_r, b, k, min_margin):
+    l = (x @ w_r + b).numpy()
+    order = np.argsort(-l, axis=1, kind="stable")
+    srt = np.take_along_axis(l, order, 1)
+    assert np.all(srt[:, k - 1] - srt[:, k] > min_margin), "pick another seed"
+    return order[:, :k].astype(np.int32)
+
+
+def _loss(x, w_r, b, w1, w2, act, idx, dy):
+    """L = <y, dY> with y from the oracle and gates = softmax of the selected logits."""
+    l = x @ w_r + b
+    sel = torch.gather(l, 1, torch.from_numpy(idx).long())
+    gates = torch.softmax(sel, dim=1)
+    y = oracle.mlp_fwd(x, w1, w2, act, idx, gates.numpy())["y"]
+    return float((y * dy.numpy()).sum())
+
+
+@pytest.mark.parametrize("act", ["gelu", "swiglu"])
+def test_mlp_backward_finite_differences(act):
+    T, d, f, E, k = 5, 8, 6, 4, 2
+    for seed in range(20, 60):
+        x, w_r, w1, w2, dy = _tiny_mlp(seed, T, d, f, E, k, act)
+        b = torch.randn(E, generator=torch.Generator().manual_seed(seed), dtype=torch.float64)
+        l = (x @ w_r + b).numpy()
+        s = np.sort(l, 1)[:, ::-1]
+        if np.all(s[:, k - 1] - s[:, k] > 1e-2):
+            break
+    idx = _route_with_margin(x, w_r, b, k, 1e-2)
+    sel = torch.gather(x @ w_r + b, 1, torch.from_numpy(idx).long())
+    gates = torch.softmax(sel, 1).numpy()
+    an = oracle.mlp_bwd_full(x, w_r, w1, w2, act, idx, gates, dy)
+    # db is not an oracle input in fp32 form here: the loss closes over b directly
+    h = 1e-6
+    params = {"x": x, "w_r": w_r, "b": b, "w1": w1, "w2": w2}
+    key_of = {"x": "dx", "w_r": "dw_r", "b": "db_r", "w1": "dw1", "w2": "dw2"}
+    for name, tensor in params.items():
+        fd = np.zeros(tensor.numel())
+        flat = tensor.view(-1)
+        for q in range(tensor.numel()):
+            old = float(flat[q])
+            flat[q] = old + h
+            lp = _loss(params["x"], params["w_r"], params["b"], params["w1"], params["w2"], act, idx, dy)
+            flat[q] = old - h
+            lm = _loss(params["x"], params["w_r"], params["b"], params["w1"], params["w2"], act, idx, dy)
+            flat[q] = old
+            fd[q] = (lp - lm) / (2 * h)
+        ref = an[key_of[name]].ravel()
+        err = np.max(np.abs(fd - ref)) / np.max(np.abs(ref))
+        assert err < 1e-6, (name, err)
+    # gate gradient: dL/dg[t,j] = <dY_t, o_{t,j}>
+    fd = np.zeros_like(gates)
+    for t in range(T):
+        for j in range(k):
+            gp, gm = gates.copy(), gates.copy()
+            gp[t, j] += h
+            gm[t, j] -= h
+            yp = oracle.mlp_fwd(x, w1, w2, act, idx, gp)["y"]
+            ym = oracle.mlp_fwd(x, w1, w2, act, idx, gm)["y"]
+            fd[t, j] = ((yp - ym) * dy.numpy()).sum() / (2 * h)
+    assert np.max(np.abs(fd - an["dg"])) / np.max(np.abs(an["dg"])) < 1e-6
+
+
+def test_mlp_backward_token_subset_and_sampled_dw_agree_with_full():
+    x, w_r, w1, w2, dy = _tiny_mlp(9, 30, 16, 12, 5, 2, "swiglu", torch.float32)
+    idx, gates = oracle.route(x, w_r, None, 2)
+    full = oracle.mlp_bwd_full(x, w_r, w1, w2, "swiglu", idx, gates, dy)
+    toks = np.array([3, 0, 29, 11], np.int32)
+    sub = oracle.mlp_bwd_tokens(x, w_r, w1, w2, "swiglu", idx, gates, dy, tokens=toks)
+    np.testing.assert_allclose(sub["dx"], full["dx"][toks], rtol=1e-13, atol=1e-14)
+    np.testing.assert_allclose(sub["dg"], full["dg"][toks], rtol=1e-13, atol=1e-14)
+    cols1 = [0, 5, 11, 12, 23]
+    rows2 = [0, 7, 11]
+    dw1c, dw2r = oracle.mlp_dw_sampled(x, w1, w2, "swiglu", idx, gates, dy, cols1, rows2)
+    np.testing.assert_allclose(dw1c, full["dw1"][:, :, cols1], rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(dw2r, full["dw2"][:, rows2, :], rtol=1e-12, atol=1e-13)
+
+
+# --------------------------------------------------------------------------
+# ParallelLinear
+# --------------------------------------------------------------------------
+def _pl_problem(seed, T, K, N, E, k, dtype=torch.float64):
+    g = torch.Generator().manual_seed(seed)
+    idx = torch.randint(0, E, (T, k), generator=g).int().numpy()
+    ss, off = oracle.sort(idx, E)
+    w = (torch.randn(E, K, N, generator=g, dtype=torch.float64) / K ** 0.5).to(dtype)
+    gates = torch.rand(T * k, generator=g, dtype=torch.float64).numpy()
+    return idx, ss, off, w, gates, g
+
+
+MODES = [  # (grouped_in, grouped_out, fan_out, combine)
+    (0, 1, "k", False),   # scatter -> group, token-shaped input read k times
+    (1, 0, 1, True),      # group -> scatter with k-way combine
+    (1, 0, 1, False),     # group -> scatter, slot-shaped output
+    (1, 1, 1, False),     # group -> group
+    (0, 0, 1, False),     # scatter -> scatter, slot-shaped input
+    (0, 0, "k", True),    # scatter -> scatter with combine, token-shaped input
+]
+
+
+@pytest.mark.parametrize("mode", MODES)
+@pytest.mark.parametrize("gated", [False, True])
+def test_pl_fwd_equals_dense_every_expert(mode, gated):
+    gi, go, fo, comb = mode
+    T, K, N, E, k = 9, 6, 5, 4, 2
+    idx, ss, off, w, gates, g = _pl_problem(11, T, K, N, E, k)
+    fan_out = k if fo == "k" else 1
+    x_rows = T * k if (gi or fan_out == 1) else T
+    x = torch.randn(x_rows, K, generator=g, dtype=torch.float64)
+    gv = gates if gated else None
+    y = oracle.pl_fwd(x, w, ss, off, fan_out, gi, go, gv, k if comb else 0)
+    # dense: every grouped row times every expert, then keep its own expert
+    e_of_row = np.repeat(np.arange(E), np.diff(off))
+    xin = x[np.arange(T * k)] if gi else x[torch.from_numpy(ss // fan_out).long()]
+    Yall = torch.einsum("sk,ekn->sen", xin, w.double())
+    v = Yall[torch.arange(T * k), torch.from_numpy(e_of_row).long()].numpy()
+    if gated:
+        v = v * gates[ss][:, None]
+    if comb:
+        ref = np.zeros((T, N))
+        for i in range(T * k):
+            ref[ss[i] // k] += v[i]
+    else:
+        ref = np.zeros((T * k, N))
+        for i in range(T * k):
+            ref[i if go else ss[i]] = v[i]
+    np.testing.assert_allclose(y, ref, rtol=1e-13, atol=1e-14)
+    # subsets of output rows agree with the full result
+    rows = [0, y.shape[0] - 1, 3]
+    np.testing.assert_allclose(oracle.pl_fwd(x, w, ss, off, fan_out, gi, go, gv, k if comb else 0,
+                                             out_rows=rows), y[rows], rtol=0, atol=0)
+
+
+@pytest.mark.parametrize("mode", MODES)
+def test_pl_backward_finite_differences(mode):
+    gi, go, fo, comb = mode
+    T, K, N, E, k = 5, 4, 3, 3, 2
+    idx, ss, off, w, gates, g = _pl_problem(12, T, K, N, E, k)
+    fan_out = k if fo == "k" else 1
+    x_rows = T * k if (gi or fan_out == 1) else T
+    x = torch.randn(x_rows, K, generator=g, dtype=torch.float64)
+    ck = k if comb else 0
+    y_rows = T if comb else T * k
+    dy = torch.randn(y_rows, N, generator=g, dtype=torch.float64)
+    an = oracle.pl_bwd(dy, x, w, ss, off, fan_out, gi, go, gates, ck, want_dg=True)
+    h = 1e-6
+
+    def loss(xx, ww, gg):
+        return float((oracle.pl_fwd(xx, ww, ss, off, fan_out, gi, go, gg, ck) * dy.numpy()).sum())
+
+    for name, tensor, key in [("x", x, "dx"), ("w", w, "dw")]:
+        fd = np.zeros(tensor.numel())
+        flat = tensor.view(-1)
+        for q in range(tensor.numel()):
+            old = float(flat[q])
+            flat[q] = old + h
+            lp = loss(x, w, gates)
+            flat[q] = old - h
+            lm = loss(x, w, gates)
+            flat[q] = old
+            fd[q] = (lp - lm) / (2 * h)
+        ref = an[key].ravel()
+        assert np.max(np.abs(fd - ref)) / np.max(np.abs(ref)) < 1e-6, name
+    fd = np.zeros(T * k)
+    for p in range(T * k):
+        gp, gm = gates.copy(), gates.copy()
+        gp[p] += h
+        gm[p] -= h
+        fd[p] = (loss(x, w, gp) - loss(x, w, gm)) / (2 * h)
+    assert np.max(np.abs(fd - an["dg"])) / np.max(np.abs(an["dg"])) < 1e-6
+
+
+def test_mlp_equals_parallel_linear_composition():
+    """The SMoE MLP is ParallelLinear(scatter->group, fan-out k), the activation,
+    then ParallelLinear(group->scatter, gated k-way combine)."""
+    x, w_r, w1, w2, dy = _tiny_mlp(13, 16, 8, 6, 4, 2, "gelu", torch.float32)
+    idx, gates = oracle.route(x, w_r, None, 2)
+    ss, off = oracle.sort(idx, 4)
+    H = oracle.pl_fwd(x, w1, ss, off, 2, 0, 1)
+    A = F.gelu(torch.from_numpy(H), approximate="tanh").numpy()
+    Y = oracle.pl_fwd(A, w2.double(), ss, off, 1, 1, 0, gates.ravel(), 2)
+    np.testing.assert_allclose(Y, oracle.mlp_fwd(x, w1, w2, "gelu", idx, gates)["y"], rtol=1e-12,
+                               atol=1e-12)
