@@ -1,0 +1,237 @@
+/*
+ * smoe.h -- C ABI of libsmoe.so: a sparse Mixture-of-Experts (SMoE) MLP and its
+ * building block ParallelLinear for NVIDIA B200 (sm_100a).
+ *
+ * The method is ScatterMoE ("Scattered Mixture-of-Experts Implementation",
+ * arXiv 2403.08245).  Its pages define the operations only in prose:
+ *   [abs]  arXiv abstract: an SMoE implementation built on ParallelLinear that
+ *          avoids padding and excessive copies of the input; extended to Mixture
+ *          of Attention.
+ *   [rev1] library page of arXiv 2403.08245, review 1 summary: ParallelLinear lets
+ *          the input and the output each be grouped or scattered, and serves both
+ *          the forward and the backward pass, without copying or padding.
+ *   [rev2] same page, review 2 summary: the scatter2scatter kernel covers
+ *          group-to-group, group-to-scatter, scatter-to-scatter and
+ *          scatter-to-group, fusing grouped GEMMs with scattered reads and writes.
+ *   [art]  tradepoint.io article "This Machine Learning Research Presents
+ *          ScatterMoE", method paragraphs: grouped matrix operations on scattered
+ *          groups; prior work needs a scatter-to-group copy of the input and pads
+ *          it; the backward pass computes the gradient of each expert.
+ *   [src]  sourcepulse.org project summary, "How It Works": expert linear
+ *          transforms are fused with the reordering operations.
+ *
+ * Conventions (all entry points):
+ *   - Row-major tensors.  Weights are [E, K, N] (K input features, N output
+ *     features): y = x W[e].  Indices are int32, gates fp32.
+ *   - dtype SMOE_BF16: x, W, activations and outputs in bf16, fp32 accumulation,
+ *     weight gradients in fp32.  SMOE_F32: everything fp32.
+ *   - Slots: token t's j-th selected expert is slot p = t*k + j.  "Scattered"
+ *     rows are in token/slot order; "grouped" rows are in expert-sorted order:
+ *     grouped row i holds slot sorted_slot[i], and expert e owns grouped rows
+ *     [expert_offsets[e], expert_offsets[e+1]).
+ *   - Pointers are device pointers unless stated otherwise; the caller owns all
+ *     memory.  The library never allocates device memory: scratch space is the
+ *     caller's workspace, sized by the *_workspace_size queries (256-byte aligned
+ *     start required).
+ *   - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default stream)
+ *     and never synchronised, except by smoe_check.
+ *   - Return value: SMOE_OK or a negative smoe_status.  Argument errors are found
+ *     on the host before any launch and leave outputs untouched; the message is
+ *     available from smoe_last_error() (thread-local).  T == 0 is a no-op.
+ *   - Data errors found on the device (an expert id outside [0, E), inconsistent
+ *     offsets) never trap: the kernel skips the bad element and records the error
+ *     in a per-device error word that smoe_check reports.
+ *   - Alignment: d, f, K and N must be multiples of 8 (16-byte rows for the
+ *     tensor-memory-accelerator copies); every tensor start 16-byte aligned.
+ *   - Several calls may run concurrently on different streams as long as they
+ *     do not share workspaces or outputs.
+ */
+#ifndef SMOE_H_
+#define SMOE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  SMOE_OK = 0,
+  SMOE_ERR_INVALID_ARG = -1, /* bad pointer, size, alignment or flag combination */
+  SMOE_ERR_UNSUPPORTED = -2, /* valid request this build does not implement (e.g. no sm_100 GPU) */
+  SMOE_ERR_CUDA = -3,        /* a CUDA runtime/driver call failed (message has the CUDA error) */
+  SMOE_ERR_DATA = -4,        /* device-detected bad index data (reported by smoe_check) */
+  SMOE_ERR_TIMEOUT = -5      /* a bounded device-side wait gave up (reported by smoe_check) */
+} smoe_status;
+
+typedef enum { SMOE_F32 = 0, SMOE_BF16 = 1 } smoe_dtype;
+
+typedef enum {
+  SMOE_ACT_GELU_TANH = 0, /* a = 0.5 h (1 + tanh(sqrt(2/pi) (h + 0.044715 h^3))) */
+  SMOE_ACT_SWIGLU = 1,    /* a = silu(h_gate) * h_up, silu(z) = z / (1 + exp(-z)) */
+  SMOE_ACT_NONE = 2
+} smoe_act;
+
+/* ---------------------------------------------------------------------------
+ * Status
+ * ------------------------------------------------------------------------ */
+
+/* Message of the last failing call on this host thread ("" if none). */
+const char* smoe_last_error(void);
+
+/* Synchronises `stream`, then reads and clears the calling device's error word.
+ * Returns SMOE_OK, SMOE_ERR_DATA, SMOE_ERR_TIMEOUT or SMOE_ERR_CUDA. */
+int smoe_check(void* stream);
+
+/* Library version string. */
+const char* smoe_version(void);
+
+/* ---------------------------------------------------------------------------
+ * Workspace queries (bytes; 0 means no workspace needed)
+ * ------------------------------------------------------------------------ */
+typedef enum {
+  SMOE_OP_SORT = 0,
+  SMOE_OP_PL_FWD = 1,
+  SMOE_OP_PL_BWD = 2,
+  SMOE_OP_MLP_FWD = 3,
+  SMOE_OP_MLP_BWD = 4
+} smoe_op;
+
+/* Upper bound of the workspace for `op` on an SMoE layer of T tokens, width d,
+ * expert width f, E experts, top-k.  For the ParallelLinear ops it bounds every
+ * flag combination with num_slots = T*k, K and N in {d, f, 2f}. */
+size_t smoe_workspace_size(int op, int T, int k, int E, int d, int f, smoe_dtype dt);
+
+/* ---------------------------------------------------------------------------
+ * Routing [abs, art: top-k SMoE layer; router definition: softmax, top-k,
+ * renormalised gates]
+ *
+ * smoe_route: logits l[t,e] = sum_i x[t,i] W_r[i,e] (+ b_r[e]) in fp32 in this
+ * documented order: lane L of a 32-lane group accumulates, in ascending i, the
+ * products for every i with i % 32 == L as acc = fmaf(x, w, acc) from +0;
+ * the 32 lane sums are combined by an xor butterfly with offsets 16, 8, 4, 2, 1;
+ * then b_r[e] is added.  The k largest logits are selected (descending; equal
+ * logits go to the lower expert id) and gates[t,j] = softmax over the k
+ * selected logits (this equals softmax over all E, top-k, renormalise).
+ *   x        [T, d] dtype          w_r [d, E] dtype        b_r [E] fp32 or NULL
+ *   topk_idx [T, k] int32 (out)    gates [T, k] fp32 (out)
+ * Requires 1 <= k <= E <= 256, k <= 16, d % 8 == 0.
+ * ------------------------------------------------------------------------ */
+int smoe_route(const void* x, const void* w_r, const float* b_r, int T, int d, int E, int k,
+               smoe_dtype dt, int32_t* topk_idx, float* gates, void* stream);
+
+/* smoe_route_bwd: gradient through the renormalised softmax of smoe_route.
+ *   dl[t,j] = gates[t,j] (dgates[t,j] - sum_i gates[t,i] dgates[t,i]) for the
+ *   selected expert e = topk_idx[t,j], 0 for unselected experts;
+ *   dw_r[i,e] = sum_t x[t,i] dl[t,e]  (fp32, fixed-order reduction, overwritten)
+ *   db_r[e]   = sum_t dl[t,e]         (fp32, overwritten; NULL to skip)
+ *   dx[t,i]  += sum_j dl[t,j] W_r[i, topk_idx[t,j]]  (dtype, accumulated into dx;
+ *                                                     NULL to skip)
+ * workspace: smoe_workspace_size(SMOE_OP_MLP_BWD, ...) suffices.               */
+int smoe_route_bwd(const void* x, const void* w_r, const int32_t* topk_idx, const float* gates,
+                   const float* dgates, int T, int d, int E, int k, smoe_dtype dt, void* dx,
+                   float* dw_r, float* db_r, void* workspace, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Reordering [src: "reordering operations"; rev1: grouped = expert-sorted]
+ *
+ * smoe_sort: stable sort of the T*k slots by expert id (ties by slot index) and
+ * the exclusive prefix sum of per-expert counts.
+ *   topk_idx [T, k] int32   sorted_slot [T*k] int32 (out)
+ *   expert_offsets [E+1] int32 (out; offsets[0] = 0, offsets[E] = T*k)
+ * Ids outside [0, E) are reported through smoe_check (SMOE_ERR_DATA) and their
+ * slots are left out (the outputs are then incomplete).
+ * ------------------------------------------------------------------------ */
+int smoe_sort(const int32_t* topk_idx, int T, int k, int E, int32_t* sorted_slot,
+              int32_t* expert_offsets, void* workspace, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * ParallelLinear [rev1, rev2, art]
+ *
+ * For every grouped row i of expert e, with p = sorted_slot[i]:
+ *   input row   : x[i]                 if grouped_in
+ *                 x[p / fan_out]       otherwise (fan_out = k for token-shaped
+ *                                      x [T, K]; 1 for slot-shaped x [T*k, K])
+ *   v           = g * x_row W[e]       g = gates[p] if gates != NULL, else 1
+ *   output      : y[i] = v             if grouped_out           (y [num_slots, N])
+ *                 y[p] = v             if scattered, combine_k == 0 (y [num_slots, N])
+ *                 y[p / combine_k] = sum of the combine_k slots' v, in slot
+ *                                      order (combine_k > 0, scattered only;
+ *                                      y [num_slots / combine_k, N])
+ * No grouped or padded copy of a scattered input is made.  The k-way combine is
+ * deterministic (no atomics).
+ *   x [x_rows, K] dtype, w [E, K, N] dtype, y dtype.
+ * ------------------------------------------------------------------------ */
+size_t parallel_linear_fwd_workspace_size(int num_slots, int K, int N, int E, int combine_k,
+                                          smoe_dtype dt);
+int parallel_linear_fwd(const void* x, int x_rows, int K, const void* w, int N, int E,
+                        const int32_t* sorted_slot, const int32_t* expert_offsets, int num_slots,
+                        int fan_out, int grouped_in, int grouped_out, const float* gates,
+                        int combine_k, void* y, smoe_dtype dt, void* workspace, size_t ws_bytes,
+                        void* stream);
+
+/* Backward of parallel_linear_fwd against dy (shaped like its y).  With
+ * G_i = dy[p / combine_k] (combine) or dy[output row of i]:
+ *   dx[input row of i] += g G_i W[e]^T   (dx [x_rows, K] dtype, overwritten; NULL to skip)
+ *   dw[e] = sum_i x_row(i)^T (g G_i)     (dw [E, K, N] fp32, overwritten, zero for an
+ *                                         empty expert; NULL to skip)
+ *   dgates[p] = <G_i, x_row(i) W[e]>     (fp32 [num_slots]; only with gates; NULL to skip)
+ * `gates` must be the forward's gates (NULL if the forward had none).         */
+size_t parallel_linear_bwd_workspace_size(int x_rows, int num_slots, int K, int N, int E,
+                                          int fan_out, int grouped_in, int grouped_out,
+                                          int has_gates, int combine_k, smoe_dtype dt);
+int parallel_linear_bwd(const void* dy, const void* x, const void* w, int x_rows, int K, int N,
+                        int E, const int32_t* sorted_slot, const int32_t* expert_offsets,
+                        int num_slots, int fan_out, int grouped_in, int grouped_out,
+                        const float* gates, int combine_k, void* dx, float* dw, float* dgates,
+                        smoe_dtype dt, void* workspace, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * SMoE MLP [abs, art: SMoE layer = top-k routing + weighted sum of expert MLPs]
+ *
+ * Forward: route, sort, H = ParallelLinear(x, W1; scatter->group, fan_out k),
+ * A = act(H), y = ParallelLinear(A, W2; group->scatter, gated k-way combine).
+ * Backward of L = <y, dy>: expert weight gradients, gate gradients, the router
+ * gradient (smoe_route_bwd) and dx.
+ * ------------------------------------------------------------------------ */
+typedef struct {
+  int T, d, f, E, k;
+  int act;   /* SMOE_ACT_GELU_TANH or SMOE_ACT_SWIGLU */
+  int dtype; /* smoe_dtype */
+} smoe_mlp_desc;
+
+typedef struct {
+  const void* x;    /* [T, d] */
+  const void* w_r;  /* [d, E] dtype (router weight) */
+  const float* b_r; /* [E] or NULL */
+  const void* w1;   /* [E, d, m*f]; SwiGLU (m = 2): columns [0,f) gate, [f,2f) up */
+  const void* w2;   /* [E, f, d] */
+  /* forward outputs, kept for the backward */
+  void* y;                 /* [T, d] */
+  int32_t* topk_idx;       /* [T, k] */
+  float* gates;            /* [T, k] */
+  int32_t* sorted_slot;    /* [T*k] */
+  int32_t* expert_offsets; /* [E+1] */
+  void* h;                 /* [T*k, m*f] grouped pre-activation */
+  void* a;                 /* [T*k, f] grouped activation */
+  /* backward inputs / outputs */
+  const void* dy; /* [T, d] */
+  void* dx;       /* [T, d] (overwritten) */
+  float* dw1;     /* [E, d, m*f] fp32 */
+  float* dw2;     /* [E, f, d] fp32 */
+  float* dw_r;    /* [d, E] fp32 */
+  float* db_r;    /* [E] fp32 or NULL */
+  float* dgates;  /* [T, k] fp32 or NULL */
+  void* workspace;
+  size_t workspace_bytes;
+} smoe_mlp_tensors;
+
+size_t smoe_mlp_workspace_size(const smoe_mlp_desc* desc, int backward);
+int smoe_mlp_fwd(const smoe_mlp_desc* desc, const smoe_mlp_tensors* t, void* stream);
+int smoe_mlp_bwd(const smoe_mlp_desc* desc, const smoe_mlp_tensors* t, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* SMOE_H_ */

@@ -479,7 +479,7 @@ extern "C" {
 
 /* R2: fp32 router logits in the CUDA route kernel's documented order.
  * For token t and expert e, lane L (0..31) of a 32-lane group accumulates the
- * products x[t,i]*W_r[i,e] for every i with (i / 8) % 32 == L, in ascending i,
+ * products x[t,i]*W_r[i,e] for every i with i % 32 == L, in ascending i,
  * as acc = fmaf(x, w, acc) from +0.  The 32 lane sums are then combined by an
  * xor butterfly: for off = 16, 8, 4, 2, 1: s[L] = s[L] + s[L ^ off].  The
  * logit is s[0] + b[e] (a single fp32 add; b == null means 0 and no add).     */
@@ -491,7 +491,7 @@ void oracle_router_logits_f32(const void* x, const void* w_r, int dt, const floa
       float s[32];
       for (int L = 0; L < 32; ++L) s[L] = 0.0f;
       for (int i = 0; i < d; ++i) {
-        const int L = (i / 8) % 32;
+        const int L = i % 32;
         float xv, wv;
         if (dt == 0) {
           xv = ((const float*)x)[(size_t)t * d + i];

@@ -40,7 +40,8 @@ def test_router_logits_documented_order_golden():
             x[0, int(i)] = v
         for i, v in case["w"].items():
             w[int(i), 0] = v
-        got = oracle.router_logits_f32(x, w)[0, 0]
+        b = None if case["b"] is None else np.array([case["b"]], np.float32)
+        got = oracle.router_logits_f32(x, w, b)[0, 0]
         assert got == np.float32(case["expected"]), (case["name"], float(got), case["expected"])
 
 
