@@ -1,0 +1,600 @@
+// api.cu -- the extern "C" entry points of libsmoe.so (declared in smoe.h):
+// argument validation (host side, before any launch), workspace layout, and the
+// composition of the kernels into ParallelLinear and the SMoE MLP.
+//
+// ParallelLinear (library page of arXiv 2403.08245, review 1 summary: input and
+// output each grouped or scattered, used for forward and backward; review 2
+// summary: group-to-group, group-to-scatter, scatter-to-scatter, scatter-to-group)
+// maps onto one grouped-M GEMM whose A rows are read grouped or gathered through
+// sorted_slot and whose output rows are written grouped or scattered; a k-way
+// combine goes through an fp32 slot-ordered buffer and a fixed-order sum.  The
+// backward (tradepoint.io article, method paragraphs: the gradient of each
+// expert) swaps the roles of the row maps for dx and runs a per-expert dW GEMM.
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "common.cuh"
+
+namespace smoe {
+int simt_tile_cols();
+int tc_tile_cols();
+}  // namespace smoe
+
+using namespace smoe;
+
+// Per-device error word of the data/timeout checks (one per device that loads
+// the library; read and cleared by smoe_check).
+__device__ unsigned g_smoe_error_word;
+
+namespace {
+
+thread_local char g_msg[512] = "";
+
+int fail(int code, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_msg, sizeof(g_msg), fmt, ap);
+  va_end(ap);
+  return code;
+}
+
+int cuda_fail(cudaError_t e, const char* where) {
+  return fail(SMOE_ERR_CUDA, "%s: %s", where, cudaGetErrorString(e));
+}
+
+#define SMOE_TRY(expr, where)                      \
+  do {                                             \
+    cudaError_t e_ = (expr);                       \
+    if (e_ != cudaSuccess) return cuda_fail(e_, where); \
+  } while (0)
+
+unsigned* error_word(cudaError_t* status) {
+  static std::mutex mu;
+  static unsigned* ptrs[128] = {};
+  int dev = 0;
+  *status = cudaGetDevice(&dev);
+  if (*status != cudaSuccess || dev < 0 || dev >= 128) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
+  if (ptrs[dev] == nullptr) {
+    *status = cudaGetSymbolAddress((void**)&ptrs[dev], g_smoe_error_word);
+    if (*status != cudaSuccess) return nullptr;
+  }
+  return ptrs[dev];
+}
+
+bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+size_t align256(size_t n) { return (n + 255) & ~(size_t)255; }
+size_t esize(smoe_dtype dt) { return dt == SMOE_BF16 ? 2 : 4; }
+bool valid_dtype(int dt) { return dt == SMOE_F32 || dt == SMOE_BF16; }
+
+// Bump allocator over the caller's workspace.
+struct Carve {
+  char* base;
+  size_t off = 0;
+  explicit Carve(void* b) : base((char*)b) {}
+  void* take(size_t bytes) {
+    void* p = base ? base + off : nullptr;
+    off += align256(bytes);
+    return p;
+  }
+};
+
+int act_tile_cols(smoe_dtype dt) { return dt == SMOE_BF16 ? tc_tile_cols() : simt_tile_cols(); }
+
+cudaError_t run_grouped(const GroupedGemm& g, smoe_dtype dt, cudaStream_t s) {
+  if (dt == SMOE_BF16) return launch_grouped_gemm_tc(g, s);
+  return launch_grouped_gemm_simt(g, dt, s);
+}
+cudaError_t run_dw(const DwGemm& g, smoe_dtype dt, cudaStream_t s) {
+  if (dt == SMOE_BF16) return launch_dw_gemm_tc(g, s);
+  return launch_dw_gemm_simt(g, dt, s);
+}
+
+int check_tc(smoe_dtype dt) {
+  if (dt == SMOE_BF16 && !tc_supported())
+    return fail(SMOE_ERR_UNSUPPORTED, "bf16 path needs an sm_100 (B200) device");
+  return SMOE_OK;
+}
+
+// ---------------------------------------------------------------------------
+// ParallelLinear workspace layout
+// ---------------------------------------------------------------------------
+struct PLFwdWs {
+  float* comb = nullptr;
+  size_t bytes = 0;
+};
+PLFwdWs pl_fwd_layout(void* ws, int num_slots, int N, int combine_k) {
+  Carve c(ws);
+  PLFwdWs l;
+  if (combine_k > 0) l.comb = (float*)c.take((size_t)num_slots * N * sizeof(float));
+  l.bytes = c.off;
+  return l;
+}
+
+struct PLBwdWs {
+  float* dx_comb = nullptr;  // [num_slots, K] fp32 when dx needs a fan-out combine
+  float* dg_part = nullptr;  // [num_slots, dg_ld]
+  void* gx = nullptr;        // [num_slots, K] dtype: gates * x rows, grouped
+  int dg_ld = 0;
+  size_t bytes = 0;
+};
+PLBwdWs pl_bwd_layout(void* ws, int num_slots, int K, int grouped_in, int fan_out, int has_gates,
+                      int want_dx, int want_dw, int want_dg, smoe_dtype dt) {
+  Carve c(ws);
+  PLBwdWs l;
+  if (want_dx && !grouped_in && fan_out > 1)
+    l.dx_comb = (float*)c.take((size_t)num_slots * K * sizeof(float));
+  if (has_gates && want_dg) {
+    l.dg_ld = cdiv(K, act_tile_cols(dt));
+    l.dg_part = (float*)c.take((size_t)num_slots * l.dg_ld * sizeof(float));
+  }
+  if (has_gates && want_dw) l.gx = c.take((size_t)num_slots * K * esize(dt));
+  l.bytes = c.off;
+  return l;
+}
+
+// ---------------------------------------------------------------------------
+// SMoE MLP workspace layout
+// ---------------------------------------------------------------------------
+struct MlpWs {
+  void* sort = nullptr;
+  float* ycomb = nullptr;   // fwd: [S, d] fp32
+  float* dg_part = nullptr; // bwd: [S, dg_ld]
+  void* dh = nullptr;       // bwd: [S, m*f] dtype (grouped dH)
+  void* ga = nullptr;       // bwd: [S, f] dtype (gates * A)
+  float* dxcomb = nullptr;  // bwd: [S, d] fp32
+  float* dl = nullptr;      // bwd: [T, k]
+  float* dg = nullptr;      // bwd: [T, k] when the caller passes no dgates
+  float* rpart = nullptr;   // bwd: router dW partials
+  int dg_ld = 0, r_chunks = 0;
+  size_t bytes = 0;
+};
+MlpWs mlp_layout(void* ws, const smoe_mlp_desc& m, int backward) {
+  Carve c(ws);
+  MlpWs l;
+  const size_t S = (size_t)m.T * m.k;
+  const smoe_dtype dt = (smoe_dtype)m.dtype;
+  l.sort = c.take(sort_workspace_bytes(m.T, m.k, m.E));
+  if (!backward) {
+    l.ycomb = (float*)c.take(S * m.d * sizeof(float));
+  } else {
+    l.dg_ld = cdiv(m.f, act_tile_cols(dt));
+    l.dg_part = (float*)c.take(S * l.dg_ld * sizeof(float));
+    l.dh = c.take(S * (size_t)(m.act == SMOE_ACT_SWIGLU ? 2 * m.f : m.f) * esize(dt));
+    l.ga = c.take(S * m.f * esize(dt));
+    l.dxcomb = (float*)c.take(S * m.d * sizeof(float));
+    l.dl = (float*)c.take(S * sizeof(float));
+    l.dg = (float*)c.take(S * sizeof(float));
+    l.r_chunks = route_dw_chunks(m.T);
+    l.rpart = (float*)c.take(((size_t)l.r_chunks * m.E * m.d + (size_t)l.r_chunks * m.E) * sizeof(float));
+  }
+  l.bytes = c.off;
+  return l;
+}
+
+int validate_mlp_desc(const smoe_mlp_desc* m) {
+  if (!m) return fail(SMOE_ERR_INVALID_ARG, "desc is NULL");
+  if (m->T < 0 || m->d <= 0 || m->f <= 0 || m->E <= 0 || m->k <= 0)
+    return fail(SMOE_ERR_INVALID_ARG, "bad sizes T=%d d=%d f=%d E=%d k=%d", m->T, m->d, m->f, m->E, m->k);
+  if (m->k > m->E || m->k > 16 || m->E > 128)
+    return fail(SMOE_ERR_INVALID_ARG, "need 1 <= k <= min(E, 16) and E <= 128 (k=%d E=%d)", m->k, m->E);
+  if (m->d % 8 || m->f % 8) return fail(SMOE_ERR_INVALID_ARG, "d and f must be multiples of 8");
+  if (!valid_dtype(m->dtype)) return fail(SMOE_ERR_INVALID_ARG, "bad dtype %d", m->dtype);
+  if (m->act != SMOE_ACT_GELU_TANH && m->act != SMOE_ACT_SWIGLU)
+    return fail(SMOE_ERR_INVALID_ARG, "act must be GELU_TANH or SWIGLU");
+  if ((long long)m->T * m->k * 2LL * m->f >= (1LL << 31) || (long long)m->T * m->d >= (1LL << 31))
+    return fail(SMOE_ERR_INVALID_ARG, "tensor too large for 32-bit row indexing");
+  return SMOE_OK;
+}
+
+#define NEED(p, name) \
+  if (!(p)) return fail(SMOE_ERR_INVALID_ARG, "%s is NULL", name)
+#define ALIGNED(p, name) \
+  if (!aligned16(p)) return fail(SMOE_ERR_INVALID_ARG, "%s is not 16-byte aligned", name)
+
+}  // namespace
+
+extern "C" {
+
+const char* smoe_last_error(void) { return g_msg; }
+
+const char* smoe_version(void) { return "smoe-b200 0.1 (sm_100a)"; }
+
+int smoe_check(void* stream) {
+  cudaError_t st;
+  SMOE_TRY(cudaStreamSynchronize((cudaStream_t)stream), "smoe_check sync");
+  unsigned* w = error_word(&st);
+  if (!w) return cuda_fail(st, "smoe_check error word");
+  unsigned v = 0;
+  SMOE_TRY(cudaMemcpy(&v, w, sizeof(v), cudaMemcpyDeviceToHost), "smoe_check read");
+  if (v != 0) {
+    const unsigned zero = 0;
+    SMOE_TRY(cudaMemcpy(w, &zero, sizeof(zero), cudaMemcpyHostToDevice), "smoe_check clear");
+  }
+  if (v & ERRBIT_TIMEOUT) return fail(SMOE_ERR_TIMEOUT, "a bounded device wait gave up");
+  if (v & ERRBIT_DATA) return fail(SMOE_ERR_DATA, "device found an index outside its range");
+  return SMOE_OK;
+}
+
+size_t smoe_workspace_size(int op, int T, int k, int E, int d, int f, smoe_dtype dt) {
+  if (T < 0 || k <= 0 || E <= 0 || d <= 0 || f <= 0) return 0;
+  const int S = T * k;
+  const int wide = (d > 2 * f ? d : 2 * f);
+  switch (op) {
+    case SMOE_OP_SORT: return sort_workspace_bytes(T, k, E);
+    case SMOE_OP_PL_FWD: return pl_fwd_layout(nullptr, S, wide, k).bytes;
+    case SMOE_OP_PL_BWD: return pl_bwd_layout(nullptr, S, wide, 0, k, 1, 1, 1, 1, dt).bytes;
+    case SMOE_OP_MLP_FWD:
+    case SMOE_OP_MLP_BWD: {
+      smoe_mlp_desc m{T, d, f, E, k, SMOE_ACT_SWIGLU, dt};
+      size_t b = mlp_layout(nullptr, m, op == SMOE_OP_MLP_BWD).bytes;
+      return b;
+    }
+    default: return 0;
+  }
+}
+
+int smoe_route(const void* x, const void* w_r, const float* b_r, int T, int d, int E, int k,
+               smoe_dtype dt, int32_t* topk_idx, float* gates, void* stream) {
+  if (T < 0 || d <= 0 || E <= 0 || k <= 0) return fail(SMOE_ERR_INVALID_ARG, "bad sizes");
+  if (k > E || k > 16 || E > 128) return fail(SMOE_ERR_INVALID_ARG, "need 1 <= k <= min(E,16), E <= 128");
+  if (d % 8) return fail(SMOE_ERR_INVALID_ARG, "d must be a multiple of 8");
+  if (!valid_dtype(dt)) return fail(SMOE_ERR_INVALID_ARG, "bad dtype");
+  if (T == 0) return SMOE_OK;
+  NEED(x, "x"); NEED(w_r, "w_r"); NEED(topk_idx, "topk_idx"); NEED(gates, "gates");
+  ALIGNED(x, "x"); ALIGNED(w_r, "w_r");
+  cudaError_t st;
+  unsigned* err = error_word(&st);
+  if (!err) return cuda_fail(st, "smoe_route");
+  SMOE_TRY(launch_route(x, w_r, b_r, T, d, E, k, dt, topk_idx, gates, err, (cudaStream_t)stream),
+           "smoe_route launch");
+  return SMOE_OK;
+}
+
+int smoe_route_bwd(const void* x, const void* w_r, const int32_t* topk_idx, const float* gates,
+                   const float* dgates, int T, int d, int E, int k, smoe_dtype dt, void* dx,
+                   float* dw_r, float* db_r, void* workspace, size_t ws_bytes, void* stream) {
+  if (T < 0 || d <= 0 || E <= 0 || k <= 0 || k > E || E > 128)
+    return fail(SMOE_ERR_INVALID_ARG, "bad sizes");
+  if (d % 8) return fail(SMOE_ERR_INVALID_ARG, "d must be a multiple of 8");
+  if (!valid_dtype(dt)) return fail(SMOE_ERR_INVALID_ARG, "bad dtype");
+  NEED(x, "x"); NEED(w_r, "w_r"); NEED(topk_idx, "topk_idx"); NEED(gates, "gates");
+  NEED(dgates, "dgates"); NEED(dw_r, "dw_r");
+  const int chunks = route_dw_chunks(T);
+  Carve c(workspace);
+  float* dl = (float*)c.take((size_t)T * k * sizeof(float));
+  float* part = (float*)c.take(((size_t)chunks * E * d + (size_t)chunks * E) * sizeof(float));
+  if (T > 0 && (!workspace || ws_bytes < c.off))
+    return fail(SMOE_ERR_INVALID_ARG, "workspace too small (%zu < %zu)", ws_bytes, c.off);
+  if (T == 0) {
+    cudaStream_t s = (cudaStream_t)stream;
+    SMOE_TRY(cudaMemsetAsync(dw_r, 0, (size_t)d * E * sizeof(float), s), "route_bwd zero");
+    if (db_r) SMOE_TRY(cudaMemsetAsync(db_r, 0, (size_t)E * sizeof(float), s), "route_bwd zero");
+    return SMOE_OK;
+  }
+  cudaStream_t s = (cudaStream_t)stream;
+  SMOE_TRY(launch_route_dl(gates, dgates, T, k, dl, s), "route_dl");
+  SMOE_TRY(launch_route_dw(x, topk_idx, dl, T, d, E, k, dt, part, chunks, dw_r, db_r, s), "route_dw");
+  if (dx) SMOE_TRY(launch_route_dx(dl, topk_idx, w_r, T, d, E, k, dt, dx, s), "route_dx");
+  return SMOE_OK;
+}
+
+int smoe_sort(const int32_t* topk_idx, int T, int k, int E, int32_t* sorted_slot,
+              int32_t* expert_offsets, void* workspace, size_t ws_bytes, void* stream) {
+  if (T < 0 || k <= 0 || E <= 0 || E > 1024) return fail(SMOE_ERR_INVALID_ARG, "bad sizes (E <= 1024)");
+  NEED(expert_offsets, "expert_offsets");
+  cudaStream_t s = (cudaStream_t)stream;
+  if (T == 0) {
+    SMOE_TRY(cudaMemsetAsync(expert_offsets, 0, (size_t)(E + 1) * sizeof(int32_t), s), "sort zero");
+    return SMOE_OK;
+  }
+  NEED(topk_idx, "topk_idx"); NEED(sorted_slot, "sorted_slot");
+  const size_t need = sort_workspace_bytes(T, k, E);
+  if (!workspace || ws_bytes < need)
+    return fail(SMOE_ERR_INVALID_ARG, "workspace too small (%zu < %zu)", ws_bytes, need);
+  cudaError_t st;
+  unsigned* err = error_word(&st);
+  if (!err) return cuda_fail(st, "smoe_sort");
+  SMOE_TRY(launch_sort(topk_idx, T, k, E, sorted_slot, expert_offsets, workspace, err, s), "smoe_sort");
+  return SMOE_OK;
+}
+
+// ---------------------------------------------------------------------------
+// ParallelLinear
+// ---------------------------------------------------------------------------
+static int validate_pl(const void* x, int x_rows, int K, const void* w, int N, int E,
+                       const int32_t* sorted_slot, const int32_t* offsets, int num_slots,
+                       int fan_out, int grouped_in, int grouped_out, int combine_k, int dt) {
+  if (num_slots < 0 || x_rows < 0 || K <= 0 || N <= 0 || E <= 0)
+    return fail(SMOE_ERR_INVALID_ARG, "bad sizes");
+  if (K % 8 || N % 8) return fail(SMOE_ERR_INVALID_ARG, "K and N must be multiples of 8");
+  if (!valid_dtype(dt)) return fail(SMOE_ERR_INVALID_ARG, "bad dtype");
+  if (fan_out < 1 || combine_k < 0) return fail(SMOE_ERR_INVALID_ARG, "fan_out >= 1, combine_k >= 0");
+  if (combine_k > 0 && (grouped_out || num_slots % combine_k))
+    return fail(SMOE_ERR_INVALID_ARG, "combine needs a scattered output and num_slots %% combine_k == 0");
+  if (grouped_in && x_rows != num_slots)
+    return fail(SMOE_ERR_INVALID_ARG, "grouped input needs x_rows == num_slots");
+  if (!grouped_in && (long long)x_rows * fan_out < num_slots)
+    return fail(SMOE_ERR_INVALID_ARG, "x_rows * fan_out < num_slots");
+  if ((long long)num_slots * (K > N ? K : N) >= (1LL << 31))
+    return fail(SMOE_ERR_INVALID_ARG, "tensor too large for 32-bit row indexing");
+  if (num_slots == 0) return SMOE_OK;
+  NEED(x, "x"); NEED(w, "w"); NEED(sorted_slot, "sorted_slot"); NEED(offsets, "expert_offsets");
+  ALIGNED(x, "x"); ALIGNED(w, "w");
+  return SMOE_OK;
+}
+
+size_t parallel_linear_fwd_workspace_size(int num_slots, int K, int N, int E, int combine_k,
+                                          smoe_dtype dt) {
+  (void)K; (void)E; (void)dt;
+  if (num_slots <= 0 || N <= 0) return 0;
+  return pl_fwd_layout(nullptr, num_slots, N, combine_k).bytes;
+}
+
+int parallel_linear_fwd(const void* x, int x_rows, int K, const void* w, int N, int E,
+                        const int32_t* sorted_slot, const int32_t* expert_offsets, int num_slots,
+                        int fan_out, int grouped_in, int grouped_out, const float* gates,
+                        int combine_k, void* y, smoe_dtype dt, void* workspace, size_t ws_bytes,
+                        void* stream) {
+  int rc = validate_pl(x, x_rows, K, w, N, E, sorted_slot, expert_offsets, num_slots, fan_out,
+                       grouped_in, grouped_out, combine_k, dt);
+  if (rc != SMOE_OK) return rc;
+  if (num_slots == 0) return SMOE_OK;
+  NEED(y, "y"); ALIGNED(y, "y");
+  PLFwdWs l = pl_fwd_layout(workspace, num_slots, N, combine_k);
+  if (l.bytes > 0 && (!workspace || ws_bytes < l.bytes))
+    return fail(SMOE_ERR_INVALID_ARG, "workspace too small (%zu < %zu)", ws_bytes, l.bytes);
+  if ((rc = check_tc(dt)) != SMOE_OK) return rc;
+  cudaError_t st;
+  unsigned* err = error_word(&st);
+  if (!err) return cuda_fail(st, "parallel_linear_fwd");
+  cudaStream_t s = (cudaStream_t)stream;
+  GroupedGemm g;
+  g.E = E; g.num_rows = num_slots; g.offsets = expert_offsets; g.sorted_slot = sorted_slot;
+  g.K = K; g.a = x; g.lda = K; g.a_rows = x_rows;
+  g.a_mode = grouped_in ? ROWS_GROUPED : ROWS_GATHER; g.a_fan_out = fan_out;
+  g.b = w; g.b_kn = 1; g.NW = N; g.n_out = N;
+  g.epi = EPI_STORE; g.gates = gates; g.err = err;
+  if (combine_k > 0) {
+    g.out_mode = ROWS_GATHER; g.out = l.comb; g.ldo = N; g.out_f32 = 1;
+  } else {
+    g.out_mode = grouped_out ? ROWS_GROUPED : ROWS_GATHER; g.out = y; g.ldo = N;
+    g.out_f32 = dt == SMOE_F32;
+  }
+  SMOE_TRY(run_grouped(g, dt, s), "parallel_linear_fwd gemm");
+  if (combine_k > 0)
+    SMOE_TRY(launch_combine(l.comb, num_slots / combine_k, combine_k, N, y, dt, nullptr, nullptr,
+                            nullptr, 0, s), "parallel_linear_fwd combine");
+  return SMOE_OK;
+}
+
+size_t parallel_linear_bwd_workspace_size(int x_rows, int num_slots, int K, int N, int E,
+                                          int fan_out, int grouped_in, int grouped_out,
+                                          int has_gates, int combine_k, smoe_dtype dt) {
+  (void)x_rows; (void)N; (void)E; (void)grouped_out; (void)combine_k;
+  if (num_slots <= 0 || K <= 0) return 0;
+  return pl_bwd_layout(nullptr, num_slots, K, grouped_in, fan_out, has_gates, 1, 1, 1, dt).bytes;
+}
+
+int parallel_linear_bwd(const void* dy, const void* x, const void* w, int x_rows, int K, int N,
+                        int E, const int32_t* sorted_slot, const int32_t* expert_offsets,
+                        int num_slots, int fan_out, int grouped_in, int grouped_out,
+                        const float* gates, int combine_k, void* dx, float* dw, float* dgates,
+                        smoe_dtype dt, void* workspace, size_t ws_bytes, void* stream) {
+  int rc = validate_pl(x, x_rows, K, w, N, E, sorted_slot, expert_offsets, num_slots, fan_out,
+                       grouped_in, grouped_out, combine_k, dt);
+  if (rc != SMOE_OK) return rc;
+  if (dgates && !gates) return fail(SMOE_ERR_INVALID_ARG, "dgates needs the forward's gates");
+  cudaStream_t s = (cudaStream_t)stream;
+  if (num_slots == 0) {
+    if (dw) SMOE_TRY(cudaMemsetAsync(dw, 0, (size_t)E * K * N * sizeof(float), s), "pl_bwd zero dw");
+    if (dx && x_rows > 0) SMOE_TRY(cudaMemsetAsync(dx, 0, (size_t)x_rows * K * esize(dt), s), "pl_bwd zero dx");
+    return SMOE_OK;
+  }
+  NEED(dy, "dy"); ALIGNED(dy, "dy");
+  if (dx) ALIGNED(dx, "dx");
+  const int has_g = gates != nullptr;
+  PLBwdWs l = pl_bwd_layout(workspace, num_slots, K, grouped_in, fan_out, has_g, dx != nullptr,
+                            dw != nullptr, dgates != nullptr, dt);
+  if (l.bytes > 0 && (!workspace || ws_bytes < l.bytes))
+    return fail(SMOE_ERR_INVALID_ARG, "workspace too small (%zu < %zu)", ws_bytes, l.bytes);
+  if ((rc = check_tc(dt)) != SMOE_OK) return rc;
+  cudaError_t st;
+  unsigned* err = error_word(&st);
+  if (!err) return cuda_fail(st, "parallel_linear_bwd");
+
+  // rows of dy feeding grouped row i
+  const int g_mode = combine_k > 0 ? ROWS_GATHER : (grouped_out ? ROWS_GROUPED : ROWS_GATHER);
+  const int g_fan = combine_k > 0 ? combine_k : 1;
+  const int x_mode = grouped_in ? ROWS_GROUPED : ROWS_GATHER;
+  // where dx rows go
+  const bool dx_comb = !grouped_in && fan_out > 1;
+
+  const bool need_gemm = dx != nullptr || dgates != nullptr;
+  if (need_gemm) {
+    GroupedGemm g;
+    g.E = E; g.num_rows = num_slots; g.offsets = expert_offsets; g.sorted_slot = sorted_slot;
+    g.K = N; g.a = dy; g.lda = N; g.a_mode = g_mode; g.a_fan_out = g_fan;
+    g.a_rows = combine_k > 0 ? num_slots / combine_k : num_slots;
+    g.b = w; g.b_kn = 0; g.NW = K; g.n_out = K;
+    g.gates = gates; g.err = err;
+    g.out_mode = grouped_in ? ROWS_GROUPED : ROWS_GATHER;
+    if (dx_comb) { g.out = l.dx_comb; g.ldo = K; g.out_f32 = 1; }
+    else { g.out = dx; g.ldo = K; g.out_f32 = dt == SMOE_F32; }
+    if (has_g) {
+      g.epi = EPI_ACT_BWD; g.act = SMOE_ACT_NONE;
+      g.aux_a = x; g.ld_aux_a = K; g.aux_a_mode = x_mode; g.aux_a_fan_out = fan_out;
+      g.out2 = dw ? l.gx : nullptr; g.ldo2 = K;
+      g.dg_partial = l.dg_part; g.dg_ld = l.dg_ld;
+      if (!dgates) { g.dg_partial = nullptr; }
+    } else {
+      g.epi = EPI_STORE;
+    }
+    if (!dx) g.out = nullptr;
+    SMOE_TRY(run_grouped(g, dt, s), "parallel_linear_bwd dx gemm");
+    if (dgates)
+      SMOE_TRY(launch_dg_reduce(l.dg_part, l.dg_ld, cdiv(K, act_tile_cols(dt)), sorted_slot,
+                                num_slots, dgates, s), "parallel_linear_bwd dg");
+    if (dx && dx_comb)
+      SMOE_TRY(launch_combine(l.dx_comb, x_rows, fan_out, K, dx, dt, nullptr, nullptr, nullptr, 0, s),
+               "parallel_linear_bwd dx combine");
+  }
+  if (dw) {
+    if (has_g && !need_gemm)
+      SMOE_TRY(launch_gather_scale(x, K, x_mode, fan_out, sorted_slot, gates, num_slots, K, l.gx,
+                                   dt, s), "parallel_linear_bwd gather");
+    DwGemm g;
+    g.E = E; g.num_rows = num_slots; g.offsets = expert_offsets; g.sorted_slot = sorted_slot;
+    g.M = K; g.N = N;
+    if (has_g) { g.a = l.gx; g.lda = K; g.a_mode = ROWS_GROUPED; g.a_fan_out = 1; g.a_rows = num_slots; }
+    else { g.a = x; g.lda = K; g.a_mode = x_mode; g.a_fan_out = fan_out; g.a_rows = x_rows; }
+    g.b = dy; g.ldb = N; g.b_mode = g_mode; g.b_fan_out = g_fan;
+    g.b_rows = combine_k > 0 ? num_slots / combine_k : num_slots;
+    g.dw = dw; g.err = err;
+    SMOE_TRY(run_dw(g, dt, s), "parallel_linear_bwd dw gemm");
+  }
+  return SMOE_OK;
+}
+
+// ---------------------------------------------------------------------------
+// SMoE MLP
+// ---------------------------------------------------------------------------
+size_t smoe_mlp_workspace_size(const smoe_mlp_desc* desc, int backward) {
+  if (validate_mlp_desc(desc) != SMOE_OK) return 0;
+  return mlp_layout(nullptr, *desc, backward).bytes;
+}
+
+int smoe_mlp_fwd(const smoe_mlp_desc* desc, const smoe_mlp_tensors* t, void* stream) {
+  int rc = validate_mlp_desc(desc);
+  if (rc != SMOE_OK) return rc;
+  NEED(t, "tensors");
+  const smoe_mlp_desc& m = *desc;
+  if (m.T == 0) return SMOE_OK;
+  NEED(t->x, "x"); NEED(t->w_r, "w_r"); NEED(t->w1, "w1"); NEED(t->w2, "w2"); NEED(t->y, "y");
+  NEED(t->topk_idx, "topk_idx"); NEED(t->gates, "gates"); NEED(t->sorted_slot, "sorted_slot");
+  NEED(t->expert_offsets, "expert_offsets"); NEED(t->h, "h"); NEED(t->a, "a");
+  ALIGNED(t->x, "x"); ALIGNED(t->w_r, "w_r"); ALIGNED(t->w1, "w1"); ALIGNED(t->w2, "w2");
+  ALIGNED(t->y, "y"); ALIGNED(t->h, "h"); ALIGNED(t->a, "a");
+  MlpWs l = mlp_layout(t->workspace, m, 0);
+  if (!t->workspace || t->workspace_bytes < l.bytes)
+    return fail(SMOE_ERR_INVALID_ARG, "workspace too small (%zu < %zu)", t->workspace_bytes, l.bytes);
+  if (((uintptr_t)t->workspace & 255u) != 0) return fail(SMOE_ERR_INVALID_ARG, "workspace not 256-byte aligned");
+  const smoe_dtype dt = (smoe_dtype)m.dtype;
+  if ((rc = check_tc(dt)) != SMOE_OK) return rc;
+  cudaError_t st;
+  unsigned* err = error_word(&st);
+  if (!err) return cuda_fail(st, "smoe_mlp_fwd");
+  cudaStream_t s = (cudaStream_t)stream;
+  const int S = m.T * m.k;
+  const int mf = m.act == SMOE_ACT_SWIGLU ? 2 * m.f : m.f;
+
+  SMOE_TRY(launch_route(t->x, t->w_r, t->b_r, m.T, m.d, m.E, m.k, dt, t->topk_idx, t->gates, err, s), "route");
+  SMOE_TRY(launch_sort(t->topk_idx, m.T, m.k, m.E, t->sorted_slot, t->expert_offsets, l.sort, err, s), "sort");
+  {  // H = x[gathered] W1, A = act(H)   (scatter -> group, fan-out k)
+    GroupedGemm g;
+    g.E = m.E; g.num_rows = S; g.offsets = t->expert_offsets; g.sorted_slot = t->sorted_slot;
+    g.K = m.d; g.a = t->x; g.lda = m.d; g.a_rows = m.T; g.a_mode = ROWS_GATHER; g.a_fan_out = m.k;
+    g.b = t->w1; g.b_kn = 1; g.NW = mf; g.n_out = m.f;
+    g.epi = EPI_ACT_FWD; g.act = m.act;
+    g.out_mode = ROWS_GROUPED; g.out = t->h; g.ldo = mf; g.out_f32 = 0;
+    g.out2 = t->a; g.ldo2 = m.f; g.err = err;
+    SMOE_TRY(run_grouped(g, dt, s), "mlp fwd gemm1");
+  }
+  {  // y = sum_j g * (A W2)   (group -> scatter, gated, k-way combine)
+    GroupedGemm g;
+    g.E = m.E; g.num_rows = S; g.offsets = t->expert_offsets; g.sorted_slot = t->sorted_slot;
+    g.K = m.f; g.a = t->a; g.lda = m.f; g.a_rows = S; g.a_mode = ROWS_GROUPED;
+    g.b = t->w2; g.b_kn = 1; g.NW = m.d; g.n_out = m.d;
+    g.epi = EPI_STORE; g.gates = t->gates;
+    g.out_mode = ROWS_GATHER; g.out = l.ycomb; g.ldo = m.d; g.out_f32 = 1; g.err = err;
+    SMOE_TRY(run_grouped(g, dt, s), "mlp fwd gemm2");
+  }
+  SMOE_TRY(launch_combine(l.ycomb, m.T, m.k, m.d, t->y, dt, nullptr, nullptr, nullptr, 0, s), "mlp fwd combine");
+  return SMOE_OK;
+}
+
+int smoe_mlp_bwd(const smoe_mlp_desc* desc, const smoe_mlp_tensors* t, void* stream) {
+  int rc = validate_mlp_desc(desc);
+  if (rc != SMOE_OK) return rc;
+  NEED(t, "tensors");
+  const smoe_mlp_desc& m = *desc;
+  const smoe_dtype dt = (smoe_dtype)m.dtype;
+  const int mf = m.act == SMOE_ACT_SWIGLU ? 2 * m.f : m.f;
+  NEED(t->dw1, "dw1"); NEED(t->dw2, "dw2"); NEED(t->dw_r, "dw_r");
+  cudaStream_t s = (cudaStream_t)stream;
+  if (m.T == 0) {
+    SMOE_TRY(cudaMemsetAsync(t->dw1, 0, (size_t)m.E * m.d * mf * 4, s), "zero");
+    SMOE_TRY(cudaMemsetAsync(t->dw2, 0, (size_t)m.E * m.f * m.d * 4, s), "zero");
+    SMOE_TRY(cudaMemsetAsync(t->dw_r, 0, (size_t)m.d * m.E * 4, s), "zero");
+    if (t->db_r) SMOE_TRY(cudaMemsetAsync(t->db_r, 0, (size_t)m.E * 4, s), "zero");
+    return SMOE_OK;
+  }
+  NEED(t->x, "x"); NEED(t->w_r, "w_r"); NEED(t->w1, "w1"); NEED(t->w2, "w2");
+  NEED(t->topk_idx, "topk_idx"); NEED(t->gates, "gates"); NEED(t->sorted_slot, "sorted_slot");
+  NEED(t->expert_offsets, "expert_offsets"); NEED(t->h, "h"); NEED(t->a, "a");
+  NEED(t->dy, "dy"); NEED(t->dx, "dx");
+  ALIGNED(t->dy, "dy"); ALIGNED(t->dx, "dx"); ALIGNED(t->h, "h"); ALIGNED(t->a, "a");
+  MlpWs l = mlp_layout(t->workspace, m, 1);
+  if (!t->workspace || t->workspace_bytes < l.bytes)
+    return fail(SMOE_ERR_INVALID_ARG, "workspace too small (%zu < %zu)", t->workspace_bytes, l.bytes);
+  if (((uintptr_t)t->workspace & 255u) != 0) return fail(SMOE_ERR_INVALID_ARG, "workspace not 256-byte aligned");
+  if ((rc = check_tc(dt)) != SMOE_OK) return rc;
+  cudaError_t st;
+  unsigned* err = error_word(&st);
+  if (!err) return cuda_fail(st, "smoe_mlp_bwd");
+  const int S = m.T * m.k;
+  float* dg = t->dgates ? t->dgates : l.dg;
+
+  {  // dA' = dy[gathered] W2^T; fused: dg partials, gA = g A, dH = g dA' act'(H)
+    GroupedGemm g;
+    g.E = m.E; g.num_rows = S; g.offsets = t->expert_offsets; g.sorted_slot = t->sorted_slot;
+    g.K = m.d; g.a = t->dy; g.lda = m.d; g.a_rows = m.T; g.a_mode = ROWS_GATHER; g.a_fan_out = m.k;
+    g.b = t->w2; g.b_kn = 0; g.NW = m.f; g.n_out = m.f;
+    g.epi = EPI_ACT_BWD; g.act = m.act; g.gates = t->gates;
+    g.aux_a = t->a; g.ld_aux_a = m.f; g.aux_a_mode = ROWS_GROUPED; g.aux_a_fan_out = 1;
+    g.aux_h = t->h; g.ld_aux_h = mf;
+    g.out_mode = ROWS_GROUPED; g.out = l.dh; g.ldo = mf; g.out_f32 = dt == SMOE_F32;
+    g.out2 = l.ga; g.ldo2 = m.f;
+    g.dg_partial = l.dg_part; g.dg_ld = l.dg_ld; g.err = err;
+    SMOE_TRY(run_grouped(g, dt, s), "mlp bwd gemm dA");
+  }
+  SMOE_TRY(launch_dg_reduce(l.dg_part, l.dg_ld, l.dg_ld, t->sorted_slot, S, dg, s), "mlp bwd dg");
+  SMOE_TRY(launch_route_dl(t->gates, dg, m.T, m.k, l.dl, s), "mlp bwd dl");
+  {  // dW2[e] = sum_i (g A)_i^T dy[t_i]
+    DwGemm g;
+    g.E = m.E; g.num_rows = S; g.offsets = t->expert_offsets; g.sorted_slot = t->sorted_slot;
+    g.M = m.f; g.N = m.d;
+    g.a = l.ga; g.lda = m.f; g.a_rows = S; g.a_mode = ROWS_GROUPED; g.a_fan_out = 1;
+    g.b = t->dy; g.ldb = m.d; g.b_rows = m.T; g.b_mode = ROWS_GATHER; g.b_fan_out = m.k;
+    g.dw = t->dw2; g.err = err;
+    SMOE_TRY(run_dw(g, dt, s), "mlp bwd dW2");
+  }
+  {  // dW1[e] = sum_i x[t_i]^T dH_i
+    DwGemm g;
+    g.E = m.E; g.num_rows = S; g.offsets = t->expert_offsets; g.sorted_slot = t->sorted_slot;
+    g.M = m.d; g.N = mf;
+    g.a = t->x; g.lda = m.d; g.a_rows = m.T; g.a_mode = ROWS_GATHER; g.a_fan_out = m.k;
+    g.b = l.dh; g.ldb = mf; g.b_rows = S; g.b_mode = ROWS_GROUPED; g.b_fan_out = 1;
+    g.dw = t->dw1; g.err = err;
+    SMOE_TRY(run_dw(g, dt, s), "mlp bwd dW1");
+  }
+  {  // per-slot dx rows: dH_i W1[e]^T  (group -> scatter, fp32, slot order)
+    GroupedGemm g;
+    g.E = m.E; g.num_rows = S; g.offsets = t->expert_offsets; g.sorted_slot = t->sorted_slot;
+    g.K = mf; g.a = l.dh; g.lda = mf; g.a_rows = S; g.a_mode = ROWS_GROUPED;
+    g.b = t->w1; g.b_kn = 0; g.NW = m.d; g.n_out = m.d;
+    g.epi = EPI_STORE;
+    g.out_mode = ROWS_GATHER; g.out = l.dxcomb; g.ldo = m.d; g.out_f32 = 1; g.err = err;
+    SMOE_TRY(run_grouped(g, dt, s), "mlp bwd gemm dx");
+  }
+  // dx[t] = sum_j rows + router term sum_j dl W_r[:, e_j]
+  SMOE_TRY(launch_combine(l.dxcomb, m.T, m.k, m.d, t->dx, dt, l.dl, t->topk_idx, t->w_r, m.E, s),
+           "mlp bwd dx combine");
+  SMOE_TRY(launch_route_dw(t->x, t->topk_idx, l.dl, m.T, m.d, m.E, m.k, dt, l.rpart, l.r_chunks,
+                           t->dw_r, t->db_r, s), "mlp bwd router dW");
+  return SMOE_OK;
+}
+
+}  // extern "C"

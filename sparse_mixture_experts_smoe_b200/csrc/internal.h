@@ -1,0 +1,115 @@
+// internal.h -- host-side declarations shared by the translation units of
+// libsmoe.so: argument blocks of the grouped GEMMs and the kernel launchers.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+
+#include <cuda_runtime.h>
+
+#include "smoe.h"
+
+namespace smoe {
+
+// Bits of the per-device error word (see smoe_check).
+enum : unsigned { ERRBIT_DATA = 1u, ERRBIT_TIMEOUT = 2u };
+
+// How grouped row i finds its source row in a row-indexed operand:
+//   ROWS_GROUPED: row i;  ROWS_GATHER: row sorted_slot[i] / fan_out.
+enum RowMode : int { ROWS_GROUPED = 0, ROWS_GATHER = 1 };
+
+// Epilogues of the grouped-M GEMM.
+enum EpiMode : int {
+  EPI_STORE = 0,    // out[row] = g * acc                       (g = gates[p] or 1)
+  EPI_ACT_FWD = 1,  // out = H = acc (pre-activation), out2 = A = act(H)
+  EPI_ACT_BWD = 2   // acc = dA'; dg partial <dA', aux_a>; out2 = g * aux_a; out = g dA' act'(H)
+};
+
+// Grouped-M GEMM: for every expert e and grouped row i in [offsets[e], offsets[e+1]):
+//   acc[i, n] = sum_k A[src(i), k] * B_e[k, n]
+// B_e is W[e] ([K, NW], b_kn = 1) or W[e]^T (W[e] is [NW, K], b_kn = 0).
+// For SwiGLU EPI_ACT_FWD the logical output column c uses B columns c (gate) and
+// n_out + c (up).
+struct GroupedGemm {
+  int E = 0;
+  int num_rows = 0;
+  const int32_t* offsets = nullptr;      // [E+1]
+  const int32_t* sorted_slot = nullptr;  // [num_rows]
+  int K = 0;
+  const void* a = nullptr;
+  int lda = 0, a_rows = 0, a_mode = ROWS_GROUPED, a_fan_out = 1;
+  const void* b = nullptr;
+  int b_kn = 1, NW = 0;
+  int epi = EPI_STORE, act = SMOE_ACT_NONE;
+  int n_out = 0;
+  int out_mode = ROWS_GROUPED;  // ROWS_GROUPED: row i; ROWS_GATHER: row p (fan-out 1)
+  void* out = nullptr;
+  int ldo = 0, out_f32 = 0;
+  void* out2 = nullptr;  // ACT_FWD: A [rows, n_out]; ACT_BWD: g*aux_a grouped (nullable)
+  int ldo2 = 0;
+  const float* gates = nullptr;  // per slot, nullable
+  const void* aux_a = nullptr;   // ACT_BWD: rows dotted with dA' (A, or the forward input)
+  int ld_aux_a = 0, aux_a_mode = ROWS_GROUPED, aux_a_fan_out = 1;
+  const void* aux_h = nullptr;  // ACT_BWD: H grouped
+  int ld_aux_h = 0;
+  float* dg_partial = nullptr;  // ACT_BWD: [num_rows, dg_ld], column = N tile index
+  int dg_ld = 0;
+  unsigned* err = nullptr;
+};
+
+// Per-expert weight gradient: dW[e][m, n] = sum_{i in slice(e)} A[src_a(i), m] * B[src_b(i), n]
+struct DwGemm {
+  int E = 0;
+  int num_rows = 0;
+  const int32_t* offsets = nullptr;
+  const int32_t* sorted_slot = nullptr;
+  int M = 0, N = 0;
+  const void* a = nullptr;
+  int lda = 0, a_rows = 0, a_mode = ROWS_GROUPED, a_fan_out = 1;
+  const void* b = nullptr;
+  int ldb = 0, b_rows = 0, b_mode = ROWS_GROUPED, b_fan_out = 1;
+  float* dw = nullptr;  // [E, M, N]
+  unsigned* err = nullptr;
+};
+
+// Column-tile width that the ACT_BWD dg partials are laid out in, per dtype.
+int dg_tile_cols(smoe_dtype dt);
+
+// ---- launchers (return a cudaError_t from the launch) ----------------------
+cudaError_t launch_route(const void* x, const void* w_r, const float* b_r, int T, int d, int E,
+                         int k, smoe_dtype dt, int32_t* idx, float* gates, unsigned* err,
+                         cudaStream_t s);
+cudaError_t launch_route_dl(const float* gates, const float* dgates, int T, int k, float* dl,
+                            cudaStream_t s);
+cudaError_t launch_route_dw(const void* x, const int32_t* idx, const float* dl, int T, int d,
+                            int E, int k, smoe_dtype dt, float* partial, int n_chunks,
+                            float* dw_r, float* db_r, cudaStream_t s);
+int route_dw_chunks(int T);
+cudaError_t launch_route_dx(const float* dl, const int32_t* idx, const void* w_r, int T, int d,
+                            int E, int k, smoe_dtype dt, void* dx, cudaStream_t s);
+
+size_t sort_workspace_bytes(int T, int k, int E);
+cudaError_t launch_sort(const int32_t* idx, int T, int k, int E, int32_t* sorted_slot,
+                        int32_t* offsets, void* ws, unsigned* err, cudaStream_t s);
+
+// out[t] = sum_{j<ck} ws[t*ck + j] (+ sum_j dl[t*ck+j] * W_r[:, idx[t*ck+j]] if dl)
+cudaError_t launch_combine(const float* ws, int T, int ck, int N, void* out, smoe_dtype out_dt,
+                           const float* dl, const int32_t* idx, const void* w_r, int E,
+                           cudaStream_t s);
+// dg[sorted_slot[i]] = sum_{c < n_tiles} partial[i*ld + c]
+cudaError_t launch_dg_reduce(const float* partial, int ld, int n_tiles, const int32_t* sorted_slot,
+                             int num_rows, float* dg, cudaStream_t s);
+// out[i] = gates[sorted_slot[i]] * src[row(i)]  (grouped rows, dtype)
+cudaError_t launch_gather_scale(const void* src, int ld_src, int mode, int fan_out,
+                                const int32_t* sorted_slot, const float* gates, int num_rows,
+                                int cols, void* out, smoe_dtype dt, cudaStream_t s);
+
+cudaError_t launch_grouped_gemm_simt(const GroupedGemm& g, smoe_dtype dt, cudaStream_t s);
+cudaError_t launch_dw_gemm_simt(const DwGemm& g, smoe_dtype dt, cudaStream_t s);
+
+// tcgen05 / TMEM path (bf16 only); *_supported() checks the device once.
+bool tc_supported();
+cudaError_t launch_grouped_gemm_tc(const GroupedGemm& g, cudaStream_t s);
+cudaError_t launch_dw_gemm_tc(const DwGemm& g, cudaStream_t s);
+
+}  // namespace smoe

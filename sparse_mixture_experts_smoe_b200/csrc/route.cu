@@ -1,0 +1,301 @@
+// route.cu -- router of the SMoE layer: logits, top-k selection, renormalised
+// gates (smoe_route), and the router backward (smoe_route_bwd).
+//
+// The pages define the layer as top-k routing with a gate-weighted sum of expert
+// MLPs (arXiv abstract; tradepoint.io article, method paragraphs); the router
+// itself is softmax, top-k, renormalise.  The top-k decision is an integer result
+// taken from fp32 logits, so the logits are accumulated in one documented order
+// (see smoe_route in smoe.h) that a CPU restatement can reproduce bit for bit:
+// lane L of a warp owns every input feature i with i % 32 == L, accumulates its
+// products in ascending i with fmaf, and the 32 lane sums meet in an xor
+// butterfly (16, 8, 4, 2, 1) before the bias is added.
+//
+// Work split: a warp handles TM tokens; a block of 8 warps stages CH rows of W_r
+// in shared memory as fp32 with a row stride = 4 (mod 32) words, so the eight
+// lanes of a 128-bit shared load phase read eight different bank groups.
+#include "common.cuh"
+
+namespace smoe {
+namespace {
+
+constexpr int kRouteWarps = 8;
+
+__host__ __device__ constexpr int route_row_stride(int emax) {
+  // smallest stride >= emax with stride % 32 == 4 (floats)
+  return emax + ((4 - emax % 32) + 32) % 32;
+}
+
+template <typename T, int EMAX, int TM, int CH>
+__global__ void __launch_bounds__(kRouteWarps * 32)
+route_kernel(const T* __restrict__ x, const T* __restrict__ w_r, const float* __restrict__ b_r,
+             int T_, int d, int E, int k, int32_t* __restrict__ idx, float* __restrict__ gates,
+             unsigned* err) {
+  constexpr int STRIDE = route_row_stride(EMAX);
+  extern __shared__ float4 smem_f4[];
+  float* ws = reinterpret_cast<float*>(smem_f4);  // [CH][STRIDE]
+
+  const int lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5;
+  const int t0 = (blockIdx.x * kRouteWarps + warp) * TM;
+
+  float acc[TM][EMAX];
+#pragma unroll
+  for (int m = 0; m < TM; ++m)
+#pragma unroll
+    for (int e = 0; e < EMAX; ++e) acc[m][e] = 0.0f;
+
+  for (int i0 = 0; i0 < d; i0 += CH) {
+    __syncthreads();
+    // stage W_r[i0 : i0+CH, 0:E] as fp32, zero-padded to EMAX columns
+    for (int q = threadIdx.x; q < CH * EMAX; q += blockDim.x) {
+      const int r = q / EMAX, e = q % EMAX;
+      const int i = i0 + r;
+      ws[r * STRIDE + e] = (i < d && e < E) ? to_f(w_r[(size_t)i * E + e]) : 0.0f;
+    }
+    __syncthreads();
+#pragma unroll 1
+    for (int r = lane; r < CH; r += 32) {
+      const int i = i0 + r;
+      if (i >= d) break;
+      float xv[TM];
+#pragma unroll
+      for (int m = 0; m < TM; ++m)
+        xv[m] = (t0 + m < T_) ? to_f(x[(size_t)(t0 + m) * d + i]) : 0.0f;
+      const float4* wrow = reinterpret_cast<const float4*>(ws + r * STRIDE);
+#pragma unroll
+      for (int e4 = 0; e4 < EMAX / 4; ++e4) {
+        const float4 w4 = wrow[e4];
+#pragma unroll
+        for (int m = 0; m < TM; ++m) {
+          acc[m][4 * e4 + 0] = fmaf(xv[m], w4.x, acc[m][4 * e4 + 0]);
+          acc[m][4 * e4 + 1] = fmaf(xv[m], w4.y, acc[m][4 * e4 + 1]);
+          acc[m][4 * e4 + 2] = fmaf(xv[m], w4.z, acc[m][4 * e4 + 2]);
+          acc[m][4 * e4 + 3] = fmaf(xv[m], w4.w, acc[m][4 * e4 + 3]);
+        }
+      }
+    }
+  }
+  // xor butterfly over the 32 lanes (every lane ends with the same sums)
+#pragma unroll
+  for (int m = 0; m < TM; ++m)
+#pragma unroll
+    for (int e = 0; e < EMAX; ++e) {
+      float v = acc[m][e];
+#pragma unroll
+      for (int off = 16; off >= 1; off >>= 1) v = v + __shfl_xor_sync(0xffffffffu, v, off);
+      acc[m][e] = v;
+    }
+
+#pragma unroll
+  for (int m = 0; m < TM; ++m) {
+    const int t = t0 + m;
+    if (t >= T_) break;
+    float l[EMAX];
+#pragma unroll
+    for (int e = 0; e < EMAX; ++e) l[e] = (b_r != nullptr && e < E) ? acc[m][e] + b_r[e] : acc[m][e];
+    // top-k: descending, ties to the lower expert id
+    unsigned long long taken0 = 0ull, taken1 = 0ull;  // EMAX <= 128
+    float sel[16];
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      if (j >= k) break;
+      int best = -1;
+      float bestv = 0.0f;
+#pragma unroll
+      for (int e = 0; e < EMAX; ++e) {
+        if (e >= E) break;
+        const bool tk = e < 64 ? ((taken0 >> e) & 1ull) : ((taken1 >> (e - 64)) & 1ull);
+        if (!tk && (best < 0 || l[e] > bestv)) {
+          best = e;
+          bestv = l[e];
+        }
+      }
+      if (best < 0) {  // only NaN logits left: take the lowest free id, flag the data
+#pragma unroll
+        for (int e = EMAX - 1; e >= 0; --e) {
+          if (e >= E) continue;
+          const bool tk = e < 64 ? ((taken0 >> e) & 1ull) : ((taken1 >> (e - 64)) & 1ull);
+          if (!tk) { best = e; bestv = l[e]; }
+        }
+        if (lane == 0) report_error(err, ERRBIT_DATA);
+      }
+      if (best < 64) taken0 |= 1ull << best; else taken1 |= 1ull << (best - 64);
+      sel[j] = bestv;
+      if (lane == 0) idx[(size_t)t * k + j] = best;
+    }
+    // gates: softmax over the selected logits (sel[0] is the maximum)
+    float z = 0.0f;
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      if (j >= k) break;
+      z += expf(sel[j] - sel[0]);
+    }
+    if (lane == 0) {
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        if (j >= k) break;
+        gates[(size_t)t * k + j] = expf(sel[j] - sel[0]) / z;
+      }
+    }
+  }
+}
+
+template <typename T, int EMAX, int TM>
+cudaError_t launch_route_t(const void* x, const void* w_r, const float* b_r, int T_, int d, int E,
+                           int k, int32_t* idx, float* gates, unsigned* err, cudaStream_t s) {
+  constexpr int CH = EMAX <= 64 ? 256 : 128;
+  const size_t smem = (size_t)CH * route_row_stride(EMAX) * sizeof(float);
+  auto kern = route_kernel<T, EMAX, TM, CH>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  const int blocks = cdiv(T_, kRouteWarps * TM);
+  kern<<<blocks, kRouteWarps * 32, smem, s>>>((const T*)x, (const T*)w_r, b_r, T_, d, E, k, idx,
+                                              gates, err);
+  return cudaGetLastError();
+}
+
+template <typename T>
+cudaError_t launch_route_dt(const void* x, const void* w_r, const float* b_r, int T_, int d, int E,
+                            int k, int32_t* idx, float* gates, unsigned* err, cudaStream_t s) {
+  if (E <= 8) return launch_route_t<T, 8, 4>(x, w_r, b_r, T_, d, E, k, idx, gates, err, s);
+  if (E <= 16) return launch_route_t<T, 16, 4>(x, w_r, b_r, T_, d, E, k, idx, gates, err, s);
+  if (E <= 32) return launch_route_t<T, 32, 4>(x, w_r, b_r, T_, d, E, k, idx, gates, err, s);
+  if (E <= 64) return launch_route_t<T, 64, 2>(x, w_r, b_r, T_, d, E, k, idx, gates, err, s);
+  return launch_route_t<T, 128, 1>(x, w_r, b_r, T_, d, E, k, idx, gates, err, s);
+}
+
+// dl[t,j] = g_j (dg_j - sum_i g_i dg_i)
+__global__ void route_dl_kernel(const float* __restrict__ gates, const float* __restrict__ dgates,
+                                int T_, int k, float* __restrict__ dl) {
+  const int t = blockIdx.x * blockDim.x + threadIdx.x;
+  if (t >= T_) return;
+  float s = 0.0f;
+  for (int j = 0; j < k; ++j) s = fmaf(gates[(size_t)t * k + j], dgates[(size_t)t * k + j], s);
+  for (int j = 0; j < k; ++j)
+    dl[(size_t)t * k + j] = gates[(size_t)t * k + j] * (dgates[(size_t)t * k + j] - s);
+}
+
+constexpr int kDwTokens = 256;  // tokens per partial-sum chunk
+constexpr int kDwCols = 256;    // feature columns per block (= threads)
+
+// partial[c][e][i] = sum_{t in chunk c} x[t,i] dl[t,e];  dbp[c][e] = sum_t dl[t,e]
+template <typename T>
+__global__ void __launch_bounds__(kDwCols)
+route_dw_partial_kernel(const T* __restrict__ x, const int32_t* __restrict__ idx,
+                        const float* __restrict__ dl, int T_, int d, int E, int k,
+                        float* __restrict__ partial, float* __restrict__ dbp) {
+  extern __shared__ float acc_s[];  // [E][kDwCols]
+  const int c = blockIdx.x;
+  const int i = blockIdx.y * kDwCols + threadIdx.x;
+  for (int e = 0; e < E; ++e) acc_s[e * kDwCols + threadIdx.x] = 0.0f;
+  const int t_end = min(T_, (c + 1) * kDwTokens);
+  for (int t = c * kDwTokens; t < t_end; ++t) {
+    const float xv = i < d ? to_f(x[(size_t)t * d + i]) : 0.0f;
+    for (int j = 0; j < k; ++j) {
+      const int e = idx[(size_t)t * k + j];
+      if (e < 0 || e >= E) continue;
+      float& a = acc_s[e * kDwCols + threadIdx.x];
+      a = fmaf(xv, dl[(size_t)t * k + j], a);
+    }
+  }
+  if (i < d)
+    for (int e = 0; e < E; ++e) partial[((size_t)c * E + e) * d + i] = acc_s[e * kDwCols + threadIdx.x];
+  if (blockIdx.y == 0 && threadIdx.x == 0) {
+    for (int e = 0; e < E; ++e) acc_s[e * kDwCols] = 0.0f;
+    for (int t = c * kDwTokens; t < t_end; ++t)
+      for (int j = 0; j < k; ++j) {
+        const int e = idx[(size_t)t * k + j];
+        if (e >= 0 && e < E) acc_s[e * kDwCols] += dl[(size_t)t * k + j];
+      }
+    for (int e = 0; e < E; ++e) dbp[(size_t)c * E + e] = acc_s[e * kDwCols];
+  }
+}
+
+// dw_r[i][e] = sum_c partial[c][e][i] (ascending c); db[e] = sum_c dbp[c][e]
+__global__ void route_dw_reduce_kernel(const float* __restrict__ partial,
+                                       const float* __restrict__ dbp, int n_chunks, int d, int E,
+                                       float* __restrict__ dw_r, float* __restrict__ db_r) {
+  const int q = blockIdx.x * blockDim.x + threadIdx.x;  // q = e * d + i
+  if (q < d * E) {
+    const int e = q / d, i = q % d;
+    float s = 0.0f;
+    for (int c = 0; c < n_chunks; ++c) s += partial[((size_t)c * E + e) * d + i];
+    dw_r[(size_t)i * E + e] = s;
+  }
+  if (db_r != nullptr && q < E) {
+    float s = 0.0f;
+    for (int c = 0; c < n_chunks; ++c) s += dbp[(size_t)c * E + q];
+    db_r[q] = s;
+  }
+}
+
+// dx[t,i] += sum_j dl[t,j] W_r[i, idx[t,j]]
+template <typename T>
+__global__ void route_dx_kernel(const float* __restrict__ dl, const int32_t* __restrict__ idx,
+                                const T* __restrict__ w_r, int T_, int d, int E, int k,
+                                T* __restrict__ dx) {
+  const size_t q = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (q >= (size_t)T_ * d) return;
+  const int t = (int)(q / d), i = (int)(q % d);
+  float s = to_f(dx[q]);
+  for (int j = 0; j < k; ++j) {
+    const int e = idx[(size_t)t * k + j];
+    if (e >= 0 && e < E) s = fmaf(dl[(size_t)t * k + j], to_f(w_r[(size_t)i * E + e]), s);
+  }
+  dx[q] = from_f<T>(s);
+}
+
+}  // namespace
+
+cudaError_t launch_route(const void* x, const void* w_r, const float* b_r, int T_, int d, int E,
+                         int k, smoe_dtype dt, int32_t* idx, float* gates, unsigned* err,
+                         cudaStream_t s) {
+  if (dt == SMOE_BF16) return launch_route_dt<bf16>(x, w_r, b_r, T_, d, E, k, idx, gates, err, s);
+  return launch_route_dt<float>(x, w_r, b_r, T_, d, E, k, idx, gates, err, s);
+}
+
+cudaError_t launch_route_dl(const float* gates, const float* dgates, int T_, int k, float* dl,
+                            cudaStream_t s) {
+  route_dl_kernel<<<cdiv(T_, 256), 256, 0, s>>>(gates, dgates, T_, k, dl);
+  return cudaGetLastError();
+}
+
+int route_dw_chunks(int T_) { return cdiv(T_, kDwTokens); }
+
+cudaError_t launch_route_dw(const void* x, const int32_t* idx, const float* dl, int T_, int d,
+                            int E, int k, smoe_dtype dt, float* partial, int n_chunks,
+                            float* dw_r, float* db_r, cudaStream_t s) {
+  float* dbp = partial + (size_t)n_chunks * E * d;
+  const size_t smem = (size_t)E * kDwCols * sizeof(float);
+  dim3 grid(n_chunks, cdiv(d, kDwCols));
+  if (dt == SMOE_BF16) {
+    cudaError_t e = cudaFuncSetAttribute(route_dw_partial_kernel<bf16>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    route_dw_partial_kernel<bf16><<<grid, kDwCols, smem, s>>>((const bf16*)x, idx, dl, T_, d, E,
+                                                              k, partial, dbp);
+  } else {
+    cudaError_t e = cudaFuncSetAttribute(route_dw_partial_kernel<float>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    route_dw_partial_kernel<float><<<grid, kDwCols, smem, s>>>((const float*)x, idx, dl, T_, d, E,
+                                                               k, partial, dbp);
+  }
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  route_dw_reduce_kernel<<<cdiv(d * E, 256), 256, 0, s>>>(partial, dbp, n_chunks, d, E, dw_r, db_r);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_route_dx(const float* dl, const int32_t* idx, const void* w_r, int T_, int d,
+                            int E, int k, smoe_dtype dt, void* dx, cudaStream_t s) {
+  const size_t n = (size_t)T_ * d;
+  const unsigned blocks = (unsigned)((n + 255) / 256);
+  if (dt == SMOE_BF16)
+    route_dx_kernel<bf16><<<blocks, 256, 0, s>>>(dl, idx, (const bf16*)w_r, T_, d, E, k, (bf16*)dx);
+  else
+    route_dx_kernel<float><<<blocks, 256, 0, s>>>(dl, idx, (const float*)w_r, T_, d, E, k, (float*)dx);
+  return cudaGetLastError();
+}
+
+}  // namespace smoe

@@ -1,0 +1,157 @@
+// sort.cu -- the reordering step (smoe_sort): a stable counting sort of the
+// T*k slots by expert id, and the per-expert offsets.
+//
+// The pages name "reordering operations" fused into ParallelLinear (sourcepulse.org
+// summary, "How It Works") and call the expert-sorted layout "grouped" (library
+// page of arXiv 2403.08245, review 1 summary).  Three launches:
+//   1. count:   each block histograms a chunk of kSortChunk slots (shared-memory
+//               atomics; counts are order-free).
+//   2. scan:    one block turns the [blocks][E] counts into per-block bases
+//               (expert-major, block-minor) and the exclusive offsets.
+//   3. scatter: each block walks its chunk in rounds of 256 slots in slot order;
+//               within a round, __match_any_sync gives each lane its rank among
+//               same-expert lanes of its warp, and per-warp counts are scanned
+//               across warps, so equal ids keep ascending slot order (stable).
+#include "common.cuh"
+
+namespace smoe {
+namespace {
+
+constexpr int kSortThreads = 256;
+constexpr int kSortChunk = 4096;
+constexpr int kSortMaxE = 1024;
+
+__global__ void __launch_bounds__(kSortThreads)
+sort_count_kernel(const int32_t* __restrict__ idx, int S, int E, int32_t* __restrict__ counts,
+                  unsigned* err) {
+  __shared__ int hist[kSortMaxE];
+  for (int e = threadIdx.x; e < E; e += blockDim.x) hist[e] = 0;
+  __syncthreads();
+  const int base = blockIdx.x * kSortChunk;
+  const int end = min(S, base + kSortChunk);
+  bool bad = false;
+  for (int p = base + threadIdx.x; p < end; p += blockDim.x) {
+    const int e = idx[p];
+    if (e >= 0 && e < E) atomicAdd(&hist[e], 1);
+    else bad = true;
+  }
+  if (bad) report_error(err, ERRBIT_DATA);
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x) counts[(size_t)blockIdx.x * E + e] = hist[e];
+}
+
+// counts[b][e] -> base[b][e] = offsets[e] + sum_{b' < b} counts[b'][e] (in place)
+__global__ void __launch_bounds__(kSortThreads)
+sort_scan_kernel(int32_t* __restrict__ counts, int n_blocks, int E, int32_t* __restrict__ offsets) {
+  __shared__ int tot[kSortMaxE];
+  __shared__ int warp_sums[kSortThreads / 32];
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    int s = 0;
+    for (int b = 0; b < n_blocks; ++b) s += counts[(size_t)b * E + e];
+    tot[e] = s;
+  }
+  __syncthreads();
+  // exclusive scan of tot[0..E) in chunks of blockDim.x
+  int carry = 0;
+  for (int e0 = 0; e0 < E; e0 += blockDim.x) {
+    const int e = e0 + threadIdx.x;
+    const int v = e < E ? tot[e] : 0;
+    int incl = v;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int o = __shfl_up_sync(0xffffffffu, incl, off);
+      if (lane >= off) incl += o;
+    }
+    if (lane == 31) warp_sums[warp] = incl;
+    __syncthreads();
+    int wpre = 0;
+    for (int w = 0; w < warp; ++w) wpre += warp_sums[w];
+    int chunk_total = 0;
+    for (int w = 0; w < kSortThreads / 32; ++w) chunk_total += warp_sums[w];
+    const int excl = carry + wpre + incl - v;
+    __syncthreads();
+    if (e < E) {
+      offsets[e] = excl;
+      int run = excl;
+      for (int b = 0; b < n_blocks; ++b) {
+        const int c = counts[(size_t)b * E + e];
+        counts[(size_t)b * E + e] = run;
+        run += c;
+      }
+    }
+    carry += chunk_total;
+  }
+  if (threadIdx.x == 0) offsets[E] = carry;
+}
+
+__global__ void __launch_bounds__(kSortThreads)
+sort_scatter_kernel(const int32_t* __restrict__ idx, int S, int E,
+                    const int32_t* __restrict__ base, int32_t* __restrict__ sorted_slot) {
+  __shared__ int run[kSortMaxE];                    // running position per expert
+  __shared__ int wcnt[kSortThreads / 32][kSortMaxE / 4 + 1];  // per-warp counts, per round
+  // wcnt holds up to kSortMaxE/4 experts per pass; larger E loops in passes below
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  for (int e = threadIdx.x; e < E; e += blockDim.x) run[e] = base[(size_t)blockIdx.x * E + e];
+  __syncthreads();
+  const int chunk0 = blockIdx.x * kSortChunk;
+  const int chunk_end = min(S, chunk0 + kSortChunk);
+  constexpr int kPass = kSortMaxE / 4;
+  for (int r0 = chunk0; r0 < chunk_end; r0 += kSortThreads) {
+    const int p = r0 + threadIdx.x;
+    int e = p < chunk_end ? idx[p] : -1;
+    if (e >= E) e = -1;
+    const unsigned same = __match_any_sync(0xffffffffu, e);
+    const int rank = __popc(same & ((1u << lane) - 1u));
+    const bool leader = rank == 0;
+    int pos = -1;
+    for (int e0 = 0; e0 < E; e0 += kPass) {  // experts [e0, e0 + kPass) per pass
+      const int ne = min(kPass, E - e0);
+      for (int q = threadIdx.x; q < (kSortThreads / 32) * ne; q += blockDim.x)
+        wcnt[q / ne][q % ne] = 0;
+      __syncthreads();
+      const bool mine = e >= e0 && e < e0 + ne;
+      if (mine && leader) wcnt[warp][e - e0] = __popc(same);
+      __syncthreads();
+      // exclusive scan over warps per expert, starting at the running position
+      for (int q = threadIdx.x; q < ne; q += blockDim.x) {
+        int acc = run[e0 + q];
+        for (int w = 0; w < kSortThreads / 32; ++w) {
+          const int c = wcnt[w][q];
+          wcnt[w][q] = acc;
+          acc += c;
+        }
+        run[e0 + q] = acc;
+      }
+      __syncthreads();
+      if (mine) pos = wcnt[warp][e - e0] + rank;
+      __syncthreads();
+    }
+    if (e >= 0 && pos >= 0) sorted_slot[pos] = p;
+  }
+}
+
+}  // namespace
+
+size_t sort_workspace_bytes(int T_, int k, int E) {
+  const size_t S = (size_t)T_ * k;
+  const size_t nb = (S + kSortChunk - 1) / kSortChunk;
+  return nb * (size_t)E * sizeof(int32_t);
+}
+
+cudaError_t launch_sort(const int32_t* idx, int T_, int k, int E, int32_t* sorted_slot,
+                        int32_t* offsets, void* ws, unsigned* err, cudaStream_t s) {
+  const int S = T_ * k;
+  const int nb = cdiv(S, kSortChunk);
+  int32_t* counts = (int32_t*)ws;
+  sort_count_kernel<<<nb, kSortThreads, 0, s>>>(idx, S, E, counts, err);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  sort_scan_kernel<<<1, kSortThreads, 0, s>>>(counts, nb, E, offsets);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  sort_scatter_kernel<<<nb, kSortThreads, 0, s>>>(idx, S, E, counts, sorted_slot);
+  return cudaGetLastError();
+}
+
+}  // namespace smoe

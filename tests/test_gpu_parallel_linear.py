@@ -1,0 +1,96 @@
+"""GPU parity of parallel_linear_fwd / parallel_linear_bwd against the CPU oracle
+in every grouped/scattered combination, gated and ungated, fp32 and bf16, on
+shapes that span several tiles with ragged tails and an empty expert."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import sparse_mixture_experts_smoe_b200 as smoe
+
+from ._util import TOL, assert_close
+
+pytestmark = pytest.mark.gpu
+
+MODES = {  # name: (grouped_in, grouped_out, fan_out is k?, combine?)
+    "scatter2group_fanout": (0, 1, True, False),
+    "group2scatter_combine": (1, 0, False, True),
+    "group2scatter": (1, 0, False, False),
+    "group2group": (1, 1, False, False),
+    "scatter2scatter": (0, 0, False, False),
+    "scatter2scatter_fanout_combine": (0, 0, True, True),
+}
+
+SHAPES = {torch.float32: dict(T=150, k=2, K=136, N=72, E=5),
+          torch.bfloat16: dict(T=300, k=2, K=264, N=392, E=5)}
+
+
+def _problem(dtype, mode, gated, seed=0):
+    sh = SHAPES[dtype]
+    T, k, K, N, E = sh["T"], sh["k"], sh["K"], sh["N"], sh["E"]
+    gi, go, fo_k, comb = MODES[mode]
+    g = torch.Generator(device="cuda").manual_seed(seed)
+    idx = torch.randint(0, E, (T, k), generator=g, device="cuda", dtype=torch.int32)
+    idx[idx == 3] = 1                      # expert 3 is empty
+    idx[: T // 3] = torch.where(idx[: T // 3] == 0, 4, idx[: T // 3])  # skew the sizes
+    ss, off = smoe.smoe_sort(idx, E)
+    fan_out = k if fo_k else 1
+    x_rows = T * k if (gi or fan_out == 1) else T
+    x = torch.randn(x_rows, K, generator=g, device="cuda").to(dtype)
+    w = (torch.randn(E, K, N, generator=g, device="cuda") / K ** 0.5).to(dtype)
+    gates = torch.rand(T * k, generator=g, device="cuda") if gated else None
+    ck = k if comb else 0
+    y_rows = T if comb else T * k
+    dy = torch.randn(y_rows, N, generator=g, device="cuda").to(dtype)
+    return dict(idx=idx, ss=ss, off=off, x=x, w=w, gates=gates, fan_out=fan_out, gi=gi, go=go,
+                ck=ck, dy=dy)
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("mode", list(MODES))
+@pytest.mark.parametrize("gated", [False, True])
+def test_parallel_linear_fwd_bwd(dtype, mode, gated):
+    P = _problem(dtype, mode, gated)
+    y = smoe.parallel_linear_fwd(P["x"], P["w"], P["ss"], P["off"], P["fan_out"], P["gi"], P["go"],
+                                 P["gates"], P["ck"])
+    dx, dw, dg = smoe.parallel_linear_bwd(P["dy"], P["x"], P["w"], P["ss"], P["off"], P["fan_out"],
+                                          P["gi"], P["go"], P["gates"], P["ck"], want_dgates=gated)
+    torch.cuda.synchronize()
+    assert smoe.smoe_check() == 0
+    ss, off = P["ss"].cpu().numpy(), P["off"].cpu().numpy()
+    gts = None if P["gates"] is None else P["gates"].cpu().double().numpy()
+    ref_y = oracle.pl_fwd(P["x"].cpu(), P["w"].cpu(), ss, off, P["fan_out"], P["gi"], P["go"], gts,
+                          P["ck"])
+    assert_close("y", y, ref_y, dtype)
+    ref = oracle.pl_bwd(P["dy"].cpu(), P["x"].cpu(), P["w"].cpu(), ss, off, P["fan_out"], P["gi"],
+                        P["go"], gts, P["ck"], want_dg=gated)
+    assert_close("dx", dx, ref["dx"], dtype)
+    assert_close("dw", dw, ref["dw"], dtype)
+    assert np.all(dw[3].cpu().numpy() == 0.0)      # the empty expert's gradient is written as 0
+    if gated:
+        assert_close("dgates", dg, ref["dg"], dtype)
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_parallel_linear_bwd_dw_only_gated(dtype):
+    """dw alone with gates takes the gather-and-scale route instead of the dx GEMM."""
+    P = _problem(dtype, "group2scatter_combine", True, seed=3)
+    _, dw, _ = smoe.parallel_linear_bwd(P["dy"], P["x"], P["w"], P["ss"], P["off"], P["fan_out"],
+                                        P["gi"], P["go"], P["gates"], P["ck"], want_dx=False)
+    ref = oracle.pl_bwd(P["dy"].cpu(), P["x"].cpu(), P["w"].cpu(), P["ss"].cpu().numpy(),
+                        P["off"].cpu().numpy(), P["fan_out"], P["gi"], P["go"],
+                        P["gates"].cpu().double().numpy(), P["ck"], want_dx=False)
+    assert_close("dw", dw, ref["dw"], dtype)
+
+
+def test_parallel_linear_is_deterministic():
+    P = _problem(torch.bfloat16, "scatter2scatter_fanout_combine", True, seed=5)
+    outs = []
+    for _ in range(2):
+        y = smoe.parallel_linear_fwd(P["x"], P["w"], P["ss"], P["off"], P["fan_out"], P["gi"],
+                                     P["go"], P["gates"], P["ck"])
+        r = smoe.parallel_linear_bwd(P["dy"], P["x"], P["w"], P["ss"], P["off"], P["fan_out"],
+                                     P["gi"], P["go"], P["gates"], P["ck"], want_dgates=True)
+        outs.append([y] + list(r))
+    for a, b in zip(*outs):
+        assert torch.equal(a, b)
