@@ -1,0 +1,401 @@
+"""Benchmark of the SMoE MLP forward + backward (one B200 per process).
+
+A step is one pass of the whole path over one batch of synthetic tokens:
+router (logits, top-k, gates), reorder (sort), the six expert GEMMs (H = x W1 with
+the activation, y = A W2 gated and combined, dA' = dy W2^T with the gate-gradient
+and activation-backward epilogue, dW2, dW1, dx = dH W1^T combined), the router
+backward and every weight gradient written in full.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+Under torchrun (N > 1) every rank runs its own replica on its GPU (the path has
+no exchange step of its own): the timed region is bracketed by a barrier and a
+device synchronisation, and the elapsed time is the maximum over ranks.
+Rank 0 prints one JSON line.
+
+--impl reference times the CPU oracle (the plain fp64 restatement of the method)
+on the host cores, on bounded samples of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+from sparse_mixture_experts_smoe_b200.inputs import WORKLOADS, make_mlp_inputs, mlp_flops  # noqa: E402
+
+METRIC = "SMoE MLP fwd+bwd tokens/s on 1 B200; % of dense BF16 tensor peak"
+DEFAULT_WORKLOAD = "mixtral_bf16_swiglu"
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained", d["bf16_tflops"]),
+                "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+# ---------------------------------------------------------------------------
+# distributed plumbing (replicas only)
+# ---------------------------------------------------------------------------
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if torch.cuda.is_available():
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(value: float, world: int) -> float:
+    if world == 1:
+        return value
+    import torch.distributed as dist
+    dev = torch.device("cuda") if dist.get_backend() == "nccl" else torch.device("cpu")
+    t = torch.tensor([value], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------------------
+# clocks sampled during the timed region
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self):
+        self.lines, self.proc, self.thread = [], None, None
+
+    def start(self):
+        cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "200"]
+        try:
+            uuid = str(torch.cuda.get_device_properties(torch.cuda.current_device()).uuid)
+            cmd += ["-i", uuid if uuid.startswith("GPU-") else "GPU-" + uuid]
+        except Exception:
+            pass
+        try:
+            self.proc = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        if self.thread:
+            self.thread.join(timeout=2)
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 7:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx.append(float(parts[1]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[3:7]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+# per-kernel algorithmic work (FLOPs for the GEMMs, bytes for the rest)
+# ---------------------------------------------------------------------------
+def kernel_work(cfg):
+    T, d, f, E, k = cfg["T"], cfg["d"], cfg["f"], cfg["E"], cfg["k"]
+    S = T * k
+    mf = 2 * f if cfg["act"] == "swiglu" else f
+    b = 2  # bf16 bytes
+    flops = {
+        "gemm.fwd_up": 2.0 * S * d * mf, "gemm.fwd_down": 2.0 * S * f * d,
+        "gemm.bwd_dA": 2.0 * S * d * f, "gemm.bwd_dW2": 2.0 * S * f * d,
+        "gemm.bwd_dW1": 2.0 * S * d * mf, "gemm.bwd_dx": 2.0 * S * mf * d,
+    }
+    bytes_ = {
+        "route": T * d * b + d * E * b + S * 8,
+        "sort": 2 * S * 4 + S * 4 + (E + 1) * 4,
+        "combine.y": S * d * 4 + T * d * b,
+        "combine.dx": S * d * 4 + T * d * b + S * 8,
+        "dg_reduce": S * 4 * max(1, math.ceil(f / 256)) + S * 8,
+        "route_dl": S * 12,
+        "route_dw": T * d * b + S * 8 + d * E * 4,
+    }
+    return flops, bytes_
+
+
+# ---------------------------------------------------------------------------
+# the oracle as a CPU baseline (bounded samples)
+# ---------------------------------------------------------------------------
+def oracle_step(c, cfg, n_tok):
+    import oracle
+    x = c["x"][:n_tok]
+    dy = c["dy"][:n_tok]
+    idx, gates = oracle.route(x, c["w_r"], c["b_r"], cfg["k"])
+    oracle.mlp_fwd(x, c["w1"], c["w2"], cfg["act"], idx, gates)
+    oracle.mlp_bwd_full(x, c["w_r"], c["w1"], c["w2"], cfg["act"], idx, gates, dy)
+
+
+def oracle_baseline(cfg, budget_s=12.0, seed=0):
+    """tokens/s of the oracle's full fwd+bwd on a token sample sized to ~budget_s."""
+    inp = make_mlp_inputs(cfg, seed=seed, device="cpu")
+    c = {k: v for k, v in inp.items()}
+    n = 1
+    while True:  # grow the sample until it takes about budget_s
+        t0 = time.perf_counter()
+        oracle_step(c, cfg, n)
+        dt = time.perf_counter() - t0
+        if dt >= budget_s / 2 or n >= cfg["T"]:
+            break
+        n = min(cfg["T"], 2 * n)
+    cores = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count()
+    return {"value": n / dt, "unit": "tokens/s", "cores": int(os.environ.get("OMP_NUM_THREADS", cores)),
+            "kind": "oracle",
+            "sample": f"{n} of the {cfg['T']} tokens: routing, forward and full backward "
+                      f"(dx, gate and router gradients, every expert weight gradient) in fp64 "
+                      f"plain loops, {dt:.1f} s"}
+
+
+def run_reference(args, world, rank):
+    cfg = WORKLOADS[args.workload]
+    if rank != 0:
+        return
+    inp = make_mlp_inputs(cfg, seed=0, device="cpu")
+    # size each step to ~3 s of oracle work (fixed costs make per-token time non-linear)
+    n = 1
+    while True:
+        t0 = time.perf_counter()
+        oracle_step(inp, cfg, n)
+        if time.perf_counter() - t0 >= 1.5 or n >= cfg["T"]:
+            break
+        n = min(cfg["T"], 2 * n)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle_step(inp, cfg, n)
+    el = time.perf_counter() - t0
+    value = n * args.steps / el
+    cores = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count()
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 * el / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": {"workload": args.workload, "T": cfg["T"], "d": cfg["d"],
+                                        "f": cfg["f"], "E": cfg["E"], "k": cfg["k"],
+                                        "act": cfg["act"], "tokens_per_step": n},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                         "sample": f"{n} tokens per step of the {cfg['T']}-token workload"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------------------
+# our path
+# ---------------------------------------------------------------------------
+def run_ours(args, world, rank):
+    import sparse_mixture_experts_smoe_b200 as smoe
+    cfg = WORKLOADS[args.workload]
+    if cfg["kind"] != "mlp":
+        raise SystemExit("the benchmark step is the SMoE MLP; pick an mlp workload")
+    dev = torch.device("cuda", torch.cuda.current_device())
+    dt = torch.bfloat16 if cfg["dtype"] == "bf16" else torch.float32
+    inp = make_mlp_inputs(cfg, seed=rank, device=dev)
+    st = smoe.SMoEMLPState(cfg["T"], cfg["d"], cfg["f"], cfg["E"], cfg["k"], cfg["act"], dt, dev)
+    params = (inp["x"], inp["w_r"], inp["b_r"], inp["w1"], inp["w2"])
+    stream = torch.cuda.current_stream()
+
+    def step(x=None, dy=None):
+        p = params if x is None else (x,) + params[1:]
+        smoe.smoe_mlp_fwd(st, *p)
+        smoe.smoe_mlp_bwd(st, *p, inp["dy"] if dy is None else dy)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    assert smoe.smoe_check() == 0, smoe.lib().smoe_last_error()
+
+    # ---- timed region: device events, max over ranks; clocks sampled meanwhile ----
+    clocks = ClockSampler()
+    clocks.start()
+    smoe.smoe_profile_begin(64 * (args.steps + 1))
+    barrier(world)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    prof = smoe.smoe_profile_end()
+    clk = clocks.stop()
+    ms = max_over_ranks(e0.elapsed_time(e1), world) / args.steps
+    assert smoe.smoe_check() == 0, smoe.lib().smoe_last_error()
+
+    # ---- forward alone (reported beside the metric) ----
+    barrier(world)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(args.steps):
+        smoe.smoe_mlp_fwd(st, *params)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms_fwd = max_over_ranks(e0.elapsed_time(e1), world) / args.steps
+
+    # ---- end to end through the public API with host buffers ----
+    x_h = inp["x"].cpu().pin_memory()
+    dy_h = inp["dy"].cpu().pin_memory()
+    y_h = torch.empty(st.y.shape, dtype=st.y.dtype).pin_memory()
+    x_d, dy_d = torch.empty_like(inp["x"]), torch.empty_like(inp["dy"])
+    barrier(world)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(args.steps):
+        x_d.copy_(x_h, non_blocking=True)
+        dy_d.copy_(dy_h, non_blocking=True)
+        step(x_d, dy_d)
+        y_h.copy_(st.y, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms_e2e = max_over_ranks(e0.elapsed_time(e1), world) / args.steps
+    h2d = x_h.numel() * x_h.element_size() + dy_h.numel() * dy_h.element_size()
+    d2h = y_h.numel() * y_h.element_size()
+
+    peaks = load_peaks()
+    fl = mlp_flops(cfg)
+    tokens = cfg["T"] * world
+    value = tokens / (ms / 1e3)
+    tflops = fl["fwd_bwd"] / (ms / 1e3) / 1e12
+    flops_k, bytes_k = kernel_work(cfg)
+    kernels = {}
+    for name, (cnt, tot) in prof.items():
+        per_launch_ms = tot / max(1, cnt) if tot > 0 else None
+        ent = {"launches": cnt, "ms_total": round(tot, 4),
+               "ms_per_launch": None if per_launch_ms is None else round(per_launch_ms, 4)}
+        if name in flops_k and per_launch_ms:
+            ent["tflops"] = round(flops_k[name] / (per_launch_ms / 1e3) / 1e12, 1)
+        elif name in bytes_k and per_launch_ms:
+            ent["gbs"] = round(bytes_k[name] / (per_launch_ms / 1e3) / 1e9, 1)
+        kernels[name] = ent
+    launches = sum(c for c, _ in prof.values())
+    # dominant kernel: largest share of the timed region
+    dom = max(prof.items(), key=lambda kv: kv[1][1])[0] if prof else None
+    roofline = None
+    if dom is not None:
+        cnt, tot = prof[dom]
+        per = tot / cnt / 1e3
+        if dom in flops_k:
+            ach = flops_k[dom] / per / 1e12
+            roofline = {"kernel": dom, "bound": "tensor", "achieved": round(ach, 1),
+                         "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s",
+                         "frac": round(ach / peaks["bf16_tflops_sustained"], 4),
+                         "peak_kind": f"bf16 sustained, {peaks['source']}",
+                         "frac_of_burst_peak": round(ach / peaks["bf16_tflops"], 4),
+                         "traffic": None}
+        else:
+            ach = bytes_k.get(dom, 0) / per / 1e9
+            roofline = {"kernel": dom, "bound": "hbm", "achieved": round(ach, 1),
+                        "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                        "frac": round(ach / peaks["hbm_gbs"], 4), "traffic": None}
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = oracle_baseline(cfg)
+    line = {
+        "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if dt == torch.bfloat16 else "f32",
+        "data": "synthetic",
+        "config": {"workload": args.workload, "T": cfg["T"], "d": cfg["d"], "f": cfg["f"],
+                   "E": cfg["E"], "k": cfg["k"], "act": cfg["act"], "parallelism": f"replicas x{world}",
+                   "l2": "inputs larger than L2 (x 134 MB, weights 2.8 GB), no flush"},
+        "tflops_fwd_bwd": round(tflops, 1),
+        "frac_of_bf16_peak": {"burst": round(tflops / peaks["bf16_tflops"], 4),
+                              "sustained": round(tflops / peaks["bf16_tflops_sustained"], 4),
+                              "peaks": peaks["source"]},
+        "fwd": {"tokens_per_s": round(tokens / (ms_fwd / 1e3), 1), "ms_per_step": round(ms_fwd, 4),
+                "tflops": round(fl["fwd"] / (ms_fwd / 1e3) / 1e12, 1)},
+        "e2e": {"value": round(tokens / (ms_e2e / 1e3), 1), "unit": "tokens/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "ms_per_step": round(ms_e2e, 4)},
+        "gpu_launches": launches,
+        "roofline": roofline,
+        "kernels": kernels,
+        "clocks": clk,
+        "cpu_baseline": cpu,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    world, rank, _ = dist_setup()
+    try:
+        if args.impl == "reference":
+            run_reference(args, world, rank)
+        else:
+            run_ours(args, world, rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -231,6 +231,21 @@ size_t smoe_mlp_workspace_size(const smoe_mlp_desc* desc, int backward);
 int smoe_mlp_fwd(const smoe_mlp_desc* desc, const smoe_mlp_tensors* t, void* stream);
 int smoe_mlp_bwd(const smoe_mlp_desc* desc, const smoe_mlp_tensors* t, void* stream);
 
+/* ---------------------------------------------------------------------------
+ * Instrumentation (the pages have no counterpart; used by the benchmark).
+ *
+ * smoe_profile_begin: from now on, every kernel launch this library makes from
+ * the calling process is bracketed by a pair of CUDA events recorded on the
+ * launching stream (at most max_launches brackets; later ones are not timed
+ * but still counted).  Events are created here, not per launch.
+ * smoe_profile_end: synchronises the recorded events, aggregates per kernel
+ * name, stops recording.  smoe_profile_entry then returns, for entry i < the
+ * returned count, the kernel name, its launch count and total milliseconds.
+ * ------------------------------------------------------------------------ */
+int smoe_profile_begin(int max_launches);
+int smoe_profile_end(void);
+int smoe_profile_entry(int i, const char** name, int* launches, double* total_ms);
+
 #ifdef __cplusplus
 }
 #endif

@@ -82,6 +82,10 @@ def lib():
     L.smoe_mlp_workspace_size.argtypes = [ctypes.POINTER(MlpDesc), _c_int]
     L.smoe_mlp_fwd.argtypes = [ctypes.POINTER(MlpDesc), ctypes.POINTER(MlpTensors), _vp]
     L.smoe_mlp_bwd.argtypes = [ctypes.POINTER(MlpDesc), ctypes.POINTER(MlpTensors), _vp]
+    L.smoe_profile_begin.argtypes = [_c_int]
+    L.smoe_profile_end.argtypes = []
+    L.smoe_profile_entry.argtypes = [_c_int, ctypes.POINTER(ctypes.c_char_p),
+                                     ctypes.POINTER(_c_int), ctypes.POINTER(ctypes.c_double)]
     _lib = L
     return L
 
@@ -128,6 +132,25 @@ def _workspace(nbytes: int, device) -> torch.Tensor:
 def smoe_check(stream=None) -> int:
     """Synchronise and return the device error status (0 = OK)."""
     return lib().smoe_check(_stream(stream))
+
+
+def smoe_profile_begin(max_launches: int = 4096):
+    """Start bracketing every library kernel launch with CUDA events."""
+    _check(lib().smoe_profile_begin(max_launches))
+
+
+def smoe_profile_end() -> dict:
+    """Stop recording; {kernel name: (launches, total ms)} since smoe_profile_begin."""
+    L = lib()
+    n = L.smoe_profile_end()
+    if n < 0:
+        _check(n)
+    out = {}
+    for i in range(n):
+        name, cnt, ms = ctypes.c_char_p(), _c_int(), ctypes.c_double()
+        _check(L.smoe_profile_entry(i, ctypes.byref(name), ctypes.byref(cnt), ctypes.byref(ms)))
+        out[name.value.decode()] = (cnt.value, ms.value)
+    return out
 
 
 def smoe_version() -> str:

@@ -13,7 +13,10 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <map>
 #include <mutex>
+#include <string>
+#include <vector>
 
 #include "common.cuh"
 
@@ -49,6 +52,48 @@ int cuda_fail(cudaError_t e, const char* where) {
     cudaError_t e_ = (expr);                       \
     if (e_ != cudaSuccess) return cuda_fail(e_, where); \
   } while (0)
+
+// ---------------------------------------------------------------------------
+// Launch instrumentation (smoe_profile_*): CUDA event pairs around each launch.
+// ---------------------------------------------------------------------------
+struct Profiler {
+  std::mutex mu;
+  bool on = false;
+  std::vector<cudaEvent_t> ev;                   // 2 per bracket
+  std::vector<std::pair<const char*, int>> rec;  // name, kernels in the bracket
+  int used = 0;
+  std::map<std::string, int> untimed;            // launches past max_launches
+  std::vector<std::string> names;
+  std::vector<int> counts;
+  std::vector<double> ms;
+};
+Profiler& profiler() {
+  static Profiler p;
+  return p;
+}
+
+struct ProfScope {
+  int slot = -1;
+  cudaStream_t s;
+  ProfScope(const char* name, int nk, cudaStream_t st) : s(st) {
+    Profiler& p = profiler();
+    if (!p.on) return;
+    std::lock_guard<std::mutex> lock(p.mu);
+    if (p.used < (int)p.rec.size()) {
+      slot = p.used++;
+      p.rec[slot] = {name, nk};
+      cudaEventRecord(p.ev[2 * slot], s);
+    } else {
+      p.untimed[name] += nk;
+    }
+  }
+  ~ProfScope() {
+    if (slot >= 0) cudaEventRecord(profiler().ev[2 * slot + 1], s);
+  }
+};
+#define SMOE_PROF_CAT2(a, b) a##b
+#define SMOE_PROF_CAT(a, b) SMOE_PROF_CAT2(a, b)
+#define PROF(name, nk) ProfScope SMOE_PROF_CAT(prof_scope_, __LINE__)(name, nk, s)
 
 unsigned* error_word(cudaError_t* status) {
   static std::mutex mu;
@@ -218,6 +263,54 @@ int smoe_check(void* stream) {
   return SMOE_OK;
 }
 
+int smoe_profile_begin(int max_launches) {
+  Profiler& p = profiler();
+  std::lock_guard<std::mutex> lock(p.mu);
+  if (max_launches < 0) return fail(SMOE_ERR_INVALID_ARG, "max_launches < 0");
+  for (cudaEvent_t e : p.ev) cudaEventDestroy(e);
+  p.ev.assign(2 * (size_t)max_launches, nullptr);
+  for (auto& e : p.ev) SMOE_TRY(cudaEventCreate(&e), "smoe_profile_begin");
+  p.rec.assign(max_launches, {nullptr, 0});
+  p.used = 0;
+  p.untimed.clear();
+  p.names.clear(); p.counts.clear(); p.ms.clear();
+  p.on = true;
+  return SMOE_OK;
+}
+
+int smoe_profile_end(void) {
+  Profiler& p = profiler();
+  std::lock_guard<std::mutex> lock(p.mu);
+  p.on = false;
+  std::map<std::string, std::pair<int, double>> agg;
+  for (int i = 0; i < p.used; ++i) {
+    SMOE_TRY(cudaEventSynchronize(p.ev[2 * i + 1]), "smoe_profile_end");
+    float t = 0.0f;
+    SMOE_TRY(cudaEventElapsedTime(&t, p.ev[2 * i], p.ev[2 * i + 1]), "smoe_profile_end");
+    auto& a = agg[p.rec[i].first];
+    a.first += p.rec[i].second;
+    a.second += t;
+  }
+  for (auto& kv : p.untimed) agg[kv.first].first += kv.second;
+  p.names.clear(); p.counts.clear(); p.ms.clear();
+  for (auto& kv : agg) {
+    p.names.push_back(kv.first);
+    p.counts.push_back(kv.second.first);
+    p.ms.push_back(kv.second.second);
+  }
+  return (int)p.names.size();
+}
+
+int smoe_profile_entry(int i, const char** name, int* launches, double* total_ms) {
+  Profiler& p = profiler();
+  std::lock_guard<std::mutex> lock(p.mu);
+  if (i < 0 || i >= (int)p.names.size()) return fail(SMOE_ERR_INVALID_ARG, "no entry %d", i);
+  if (name) *name = p.names[i].c_str();
+  if (launches) *launches = p.counts[i];
+  if (total_ms) *total_ms = p.ms[i];
+  return SMOE_OK;
+}
+
 size_t smoe_workspace_size(int op, int T, int k, int E, int d, int f, smoe_dtype dt) {
   if (T < 0 || k <= 0 || E <= 0 || d <= 0 || f <= 0) return 0;
   const int S = T * k;
@@ -248,8 +341,9 @@ int smoe_route(const void* x, const void* w_r, const float* b_r, int T, int d, i
   cudaError_t st;
   unsigned* err = error_word(&st);
   if (!err) return cuda_fail(st, "smoe_route");
-  SMOE_TRY(launch_route(x, w_r, b_r, T, d, E, k, dt, topk_idx, gates, err, (cudaStream_t)stream),
-           "smoe_route launch");
+  cudaStream_t s = (cudaStream_t)stream;
+  { PROF("route", 1);
+  SMOE_TRY(launch_route(x, w_r, b_r, T, d, E, k, dt, topk_idx, gates, err, s), "smoe_route launch"); }
   return SMOE_OK;
 }
 
@@ -275,9 +369,9 @@ int smoe_route_bwd(const void* x, const void* w_r, const int32_t* topk_idx, cons
     return SMOE_OK;
   }
   cudaStream_t s = (cudaStream_t)stream;
-  SMOE_TRY(launch_route_dl(gates, dgates, T, k, dl, s), "route_dl");
-  SMOE_TRY(launch_route_dw(x, topk_idx, dl, T, d, E, k, dt, part, chunks, dw_r, db_r, s), "route_dw");
-  if (dx) SMOE_TRY(launch_route_dx(dl, topk_idx, w_r, T, d, E, k, dt, dx, s), "route_dx");
+  { PROF("route_dl", 1); SMOE_TRY(launch_route_dl(gates, dgates, T, k, dl, s), "route_dl"); }
+  { PROF("route_dw", 2); SMOE_TRY(launch_route_dw(x, topk_idx, dl, T, d, E, k, dt, part, chunks, dw_r, db_r, s), "route_dw"); }
+  if (dx) { PROF("route_dx", 1); SMOE_TRY(launch_route_dx(dl, topk_idx, w_r, T, d, E, k, dt, dx, s), "route_dx"); }
   return SMOE_OK;
 }
 
@@ -297,7 +391,7 @@ int smoe_sort(const int32_t* topk_idx, int T, int k, int E, int32_t* sorted_slot
   cudaError_t st;
   unsigned* err = error_word(&st);
   if (!err) return cuda_fail(st, "smoe_sort");
-  SMOE_TRY(launch_sort(topk_idx, T, k, E, sorted_slot, expert_offsets, workspace, err, s), "smoe_sort");
+  { PROF("sort", 3); SMOE_TRY(launch_sort(topk_idx, T, k, E, sorted_slot, expert_offsets, workspace, err, s), "smoe_sort"); }
   return SMOE_OK;
 }
 
@@ -363,10 +457,12 @@ int parallel_linear_fwd(const void* x, int x_rows, int K, const void* w, int N, 
     g.out_mode = grouped_out ? ROWS_GROUPED : ROWS_GATHER; g.out = y; g.ldo = N;
     g.out_f32 = dt == SMOE_F32;
   }
-  SMOE_TRY(run_grouped(g, dt, s), "parallel_linear_fwd gemm");
-  if (combine_k > 0)
+  { PROF("pl.gemm_fwd", 1); SMOE_TRY(run_grouped(g, dt, s), "parallel_linear_fwd gemm"); }
+  if (combine_k > 0) {
+    PROF("pl.combine", 1);
     SMOE_TRY(launch_combine(l.comb, num_slots / combine_k, combine_k, N, y, dt, nullptr, nullptr,
                             nullptr, 0, s), "parallel_linear_fwd combine");
+  }
   return SMOE_OK;
 }
 
@@ -433,18 +529,24 @@ int parallel_linear_bwd(const void* dy, const void* x, const void* w, int x_rows
       g.epi = EPI_STORE;
     }
     if (!dx) g.out = nullptr;
-    SMOE_TRY(run_grouped(g, dt, s), "parallel_linear_bwd dx gemm");
-    if (dgates)
+    { PROF("pl.gemm_dx", 1); SMOE_TRY(run_grouped(g, dt, s), "parallel_linear_bwd dx gemm"); }
+    if (dgates) {
+      PROF("pl.dg_reduce", 1);
       SMOE_TRY(launch_dg_reduce(l.dg_part, l.dg_ld, cdiv(K, act_tile_cols(dt)), sorted_slot,
                                 num_slots, dgates, s), "parallel_linear_bwd dg");
-    if (dx && dx_comb)
+    }
+    if (dx && dx_comb) {
+      PROF("pl.combine_dx", 1);
       SMOE_TRY(launch_combine(l.dx_comb, x_rows, fan_out, K, dx, dt, nullptr, nullptr, nullptr, 0, s),
                "parallel_linear_bwd dx combine");
+    }
   }
   if (dw) {
-    if (has_g && !need_gemm)
+    if (has_g && !need_gemm) {
+      PROF("pl.gather", 1);
       SMOE_TRY(launch_gather_scale(x, K, x_mode, fan_out, sorted_slot, gates, num_slots, K, l.gx,
                                    dt, s), "parallel_linear_bwd gather");
+    }
     DwGemm g;
     g.E = E; g.num_rows = num_slots; g.offsets = expert_offsets; g.sorted_slot = sorted_slot;
     g.M = K; g.N = N;
@@ -453,7 +555,7 @@ int parallel_linear_bwd(const void* dy, const void* x, const void* w, int x_rows
     g.b = dy; g.ldb = N; g.b_mode = g_mode; g.b_fan_out = g_fan;
     g.b_rows = combine_k > 0 ? num_slots / combine_k : num_slots;
     g.dw = dw; g.err = err;
-    SMOE_TRY(run_dw(g, dt, s), "parallel_linear_bwd dw gemm");
+    { PROF("pl.gemm_dw", 1); SMOE_TRY(run_dw(g, dt, s), "parallel_linear_bwd dw gemm"); }
   }
   return SMOE_OK;
 }
@@ -490,8 +592,8 @@ int smoe_mlp_fwd(const smoe_mlp_desc* desc, const smoe_mlp_tensors* t, void* str
   const int S = m.T * m.k;
   const int mf = m.act == SMOE_ACT_SWIGLU ? 2 * m.f : m.f;
 
-  SMOE_TRY(launch_route(t->x, t->w_r, t->b_r, m.T, m.d, m.E, m.k, dt, t->topk_idx, t->gates, err, s), "route");
-  SMOE_TRY(launch_sort(t->topk_idx, m.T, m.k, m.E, t->sorted_slot, t->expert_offsets, l.sort, err, s), "sort");
+  { PROF("route", 1); SMOE_TRY(launch_route(t->x, t->w_r, t->b_r, m.T, m.d, m.E, m.k, dt, t->topk_idx, t->gates, err, s), "route"); }
+  { PROF("sort", 3); SMOE_TRY(launch_sort(t->topk_idx, m.T, m.k, m.E, t->sorted_slot, t->expert_offsets, l.sort, err, s), "sort"); }
   {  // H = x[gathered] W1, A = act(H)   (scatter -> group, fan-out k)
     GroupedGemm g;
     g.E = m.E; g.num_rows = S; g.offsets = t->expert_offsets; g.sorted_slot = t->sorted_slot;
@@ -500,7 +602,7 @@ int smoe_mlp_fwd(const smoe_mlp_desc* desc, const smoe_mlp_tensors* t, void* str
     g.epi = EPI_ACT_FWD; g.act = m.act;
     g.out_mode = ROWS_GROUPED; g.out = t->h; g.ldo = mf; g.out_f32 = 0;
     g.out2 = t->a; g.ldo2 = m.f; g.err = err;
-    SMOE_TRY(run_grouped(g, dt, s), "mlp fwd gemm1");
+    { PROF("gemm.fwd_up", 1); SMOE_TRY(run_grouped(g, dt, s), "mlp fwd gemm1"); }
   }
   {  // y = sum_j g * (A W2)   (group -> scatter, gated, k-way combine)
     GroupedGemm g;
@@ -509,9 +611,9 @@ int smoe_mlp_fwd(const smoe_mlp_desc* desc, const smoe_mlp_tensors* t, void* str
     g.b = t->w2; g.b_kn = 1; g.NW = m.d; g.n_out = m.d;
     g.epi = EPI_STORE; g.gates = t->gates;
     g.out_mode = ROWS_GATHER; g.out = l.ycomb; g.ldo = m.d; g.out_f32 = 1; g.err = err;
-    SMOE_TRY(run_grouped(g, dt, s), "mlp fwd gemm2");
+    { PROF("gemm.fwd_down", 1); SMOE_TRY(run_grouped(g, dt, s), "mlp fwd gemm2"); }
   }
-  SMOE_TRY(launch_combine(l.ycomb, m.T, m.k, m.d, t->y, dt, nullptr, nullptr, nullptr, 0, s), "mlp fwd combine");
+  { PROF("combine.y", 1); SMOE_TRY(launch_combine(l.ycomb, m.T, m.k, m.d, t->y, dt, nullptr, nullptr, nullptr, 0, s), "mlp fwd combine"); }
   return SMOE_OK;
 }
 
@@ -558,10 +660,10 @@ int smoe_mlp_bwd(const smoe_mlp_desc* desc, const smoe_mlp_tensors* t, void* str
     g.out_mode = ROWS_GROUPED; g.out = l.dh; g.ldo = mf; g.out_f32 = dt == SMOE_F32;
     g.out2 = l.ga; g.ldo2 = m.f;
     g.dg_partial = l.dg_part; g.dg_ld = l.dg_ld; g.err = err;
-    SMOE_TRY(run_grouped(g, dt, s), "mlp bwd gemm dA");
+    { PROF("gemm.bwd_dA", 1); SMOE_TRY(run_grouped(g, dt, s), "mlp bwd gemm dA"); }
   }
-  SMOE_TRY(launch_dg_reduce(l.dg_part, l.dg_ld, l.dg_ld, t->sorted_slot, S, dg, s), "mlp bwd dg");
-  SMOE_TRY(launch_route_dl(t->gates, dg, m.T, m.k, l.dl, s), "mlp bwd dl");
+  { PROF("dg_reduce", 1); SMOE_TRY(launch_dg_reduce(l.dg_part, l.dg_ld, l.dg_ld, t->sorted_slot, S, dg, s), "mlp bwd dg"); }
+  { PROF("route_dl", 1); SMOE_TRY(launch_route_dl(t->gates, dg, m.T, m.k, l.dl, s), "mlp bwd dl"); }
   {  // dW2[e] = sum_i (g A)_i^T dy[t_i]
     DwGemm g;
     g.E = m.E; g.num_rows = S; g.offsets = t->expert_offsets; g.sorted_slot = t->sorted_slot;
@@ -569,7 +671,7 @@ int smoe_mlp_bwd(const smoe_mlp_desc* desc, const smoe_mlp_tensors* t, void* str
     g.a = l.ga; g.lda = m.f; g.a_rows = S; g.a_mode = ROWS_GROUPED; g.a_fan_out = 1;
     g.b = t->dy; g.ldb = m.d; g.b_rows = m.T; g.b_mode = ROWS_GATHER; g.b_fan_out = m.k;
     g.dw = t->dw2; g.err = err;
-    SMOE_TRY(run_dw(g, dt, s), "mlp bwd dW2");
+    { PROF("gemm.bwd_dW2", 1); SMOE_TRY(run_dw(g, dt, s), "mlp bwd dW2"); }
   }
   {  // dW1[e] = sum_i x[t_i]^T dH_i
     DwGemm g;
@@ -578,7 +680,7 @@ int smoe_mlp_bwd(const smoe_mlp_desc* desc, const smoe_mlp_tensors* t, void* str
     g.a = t->x; g.lda = m.d; g.a_rows = m.T; g.a_mode = ROWS_GATHER; g.a_fan_out = m.k;
     g.b = l.dh; g.ldb = mf; g.b_rows = S; g.b_mode = ROWS_GROUPED; g.b_fan_out = 1;
     g.dw = t->dw1; g.err = err;
-    SMOE_TRY(run_dw(g, dt, s), "mlp bwd dW1");
+    { PROF("gemm.bwd_dW1", 1); SMOE_TRY(run_dw(g, dt, s), "mlp bwd dW1"); }
   }
   {  // per-slot dx rows: dH_i W1[e]^T  (group -> scatter, fp32, slot order)
     GroupedGemm g;
@@ -587,13 +689,15 @@ int smoe_mlp_bwd(const smoe_mlp_desc* desc, const smoe_mlp_tensors* t, void* str
     g.b = t->w1; g.b_kn = 0; g.NW = m.d; g.n_out = m.d;
     g.epi = EPI_STORE;
     g.out_mode = ROWS_GATHER; g.out = l.dxcomb; g.ldo = m.d; g.out_f32 = 1; g.err = err;
-    SMOE_TRY(run_grouped(g, dt, s), "mlp bwd gemm dx");
+    { PROF("gemm.bwd_dx", 1); SMOE_TRY(run_grouped(g, dt, s), "mlp bwd gemm dx"); }
   }
   // dx[t] = sum_j rows + router term sum_j dl W_r[:, e_j]
+  { PROF("combine.dx", 1);
   SMOE_TRY(launch_combine(l.dxcomb, m.T, m.k, m.d, t->dx, dt, l.dl, t->topk_idx, t->w_r, m.E, s),
-           "mlp bwd dx combine");
+           "mlp bwd dx combine"); }
+  { PROF("route_dw", 2);
   SMOE_TRY(launch_route_dw(t->x, t->topk_idx, l.dl, m.T, m.d, m.E, m.k, dt, l.rpart, l.r_chunks,
-                           t->dw_r, t->db_r, s), "mlp bwd router dW");
+                           t->dw_r, t->db_r, s), "mlp bwd router dW"); }
   return SMOE_OK;
 }
 
