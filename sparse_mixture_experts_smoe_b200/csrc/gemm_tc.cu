@@ -8,10 +8,13 @@
 // padded copy of the input.  Here every tile belongs to one expert's contiguous
 // slice of the expert-sorted slot list:
 //   * grouped operands (rows already in expert order) arrive by 2-D/3-D TMA tiles;
-//   * scattered operands (token rows) arrive by TMA gather4: each instruction
-//     fetches four arbitrary 128-byte row segments, so a 128-row tile is 32
-//     gather4 copies issued by the 32 lanes of the producer warp, straight from
-//     the token-ordered tensor;
+//   * scattered operands (token rows) are gathered straight from the
+//     token-ordered tensor by four producer warps with 16-byte cp.async copies
+//     (eight threads per 128-byte row segment, written in the 128-byte swizzle
+//     the tensor core reads; rows past the slice are zero-filled).  TMA gather4
+//     was measured first and moved about 10 bytes per cycle per SM, too slow to
+//     feed the tensor core; the load/store path sustains the 48 KB per 512-cycle
+//     stage;
 //   * weights arrive as 3-D TMA tiles of W[e] ([E, K, N]: MN-major operand) or of
 //     W[e]^T (K-major operand) -- out-of-range rows/columns read as zero.
 // Both operands are staged in 128-byte-swizzled shared memory and consumed by
@@ -21,14 +24,15 @@
 // expert offsets (expert-major, then N tile, then M tile, so the CTAs of one wave
 // share the expert's input rows in L2).  Warp roles: warp 0 = TMA producer,
 // warp 1 = MMA issuer and tensor-memory owner, warps 4-7 = epilogue (thread r owns
-// accumulator row r).  Two 256-column fp32 accumulators in tensor memory let the
+// accumulator row r), warps 8-11 = row gather of a scattered operand.  Two 256-column fp32 accumulators in tensor memory let the
 // epilogue of one tile overlap the main loop of the next.  Epilogues: scaled
 // store (gate), activation forward (H and A = gelu(H) or silu(Hg) * Hu), and the
 // activation backward (gate gradient partial <dA', A>, g*A, dH = g dA' act'(H)).
 //
 // dW kernel: tile (e, m, n) of dW[e] = sum over the expert's rows r of
 // A[r, m] * B[r, n]; the reduction runs over the slice rows, so both operands are
-// MN-major 64-row slabs; rows past the slice end are zeroed in shared memory.
+// MN-major 64-row slabs; rows past the slice end are zero-filled (gathered
+// operand) or zeroed in shared memory before the last MMA of the tile.
 //
 // Every mbarrier wait is bounded (2 s of %globaltimer); on expiry the kernel sets
 // the timeout bit of the error word, stops issuing work and frees its tensor
@@ -44,7 +48,9 @@ constexpr int BM = 128;           // rows per tile (MMA M)
 constexpr int BK = 64;            // K per stage: one 128-byte swizzle row of bf16
 constexpr int BN = 256;           // MMA N
 constexpr int STAGES = 4;
-constexpr int kThreads = 256;
+constexpr int kThreads = 384;        // 12 warps
+constexpr int kGatherWarp0 = 8;       // warps 8-11 gather scattered rows
+constexpr int kGatherThreads = 128;
 constexpr uint32_t kTmemCols = 512;  // two BN-column fp32 accumulators
 constexpr int A_BYTES = BM * BK * 2;  // 16 KB
 constexpr int B_BYTES = BN * BK * 2;  // 32 KB
@@ -88,7 +94,7 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 // Bounded wait: false once the CTA has aborted or after kWaitNs (then it aborts).
-__device__ __noinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
                                        unsigned* err) {
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = global_ns();
@@ -118,14 +124,20 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, u
       "l"((uint64_t)map), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2)
       : "memory");
 }
-// Four rows (r0..r3) of 64 bf16 starting at column c0 -> four consecutive 128-byte rows.
-__device__ __forceinline__ void tma_gather4(void* dst, const CUtensorMap* map, uint64_t* bar,
-                                            int c0, int r0, int r1, int r2, int r3) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(smem_u32(dst)),
-      "l"((uint64_t)map), "r"(smem_u32(bar)), "r"(c0), "r"(r0), "r"(r1), "r"(r2), "r"(r3)
-      : "memory");
+// 16-byte asynchronous copy global -> shared through L2 only; src_bytes = 0
+// writes zeros without reading the source.
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes)
+               : "memory");
+}
+// Arrive on `bar` once this thread's earlier cp.async copies have landed (the
+// barrier's expected count includes this arrival).
+__device__ __forceinline__ void cp_async_arrive(uint64_t* bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+// Byte offset of 16-byte chunk c of row r inside 128-byte-swizzled 1024-byte atoms.
+__device__ __forceinline__ uint32_t sw128_off(int r, int c) {
+  return (uint32_t)(r * 128 + ((c ^ (r & 7)) << 4));
 }
 __device__ __forceinline__ void fence_proxy_async() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -269,11 +281,11 @@ __device__ __forceinline__ Tile map_tile(const SharedCtl& c, int E, int nN, int 
 
 // Setup common to both kernels: barriers, tensor memory, offsets (validated).
 __device__ __forceinline__ void setup(SharedCtl& c, const int32_t* offsets, int E, int num_rows,
-                                      unsigned* err) {
+                                      unsigned* err, bool gather) {
   const int warp = threadIdx.x >> 5;
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
-      mbar_init(&c.full[s], 1);
+      mbar_init(&c.full[s], 1 + (gather ? kGatherThreads : 0));
       mbar_init(&c.empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
@@ -326,39 +338,25 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
   SharedCtl& c = *reinterpret_cast<SharedCtl*>(sB + STAGES * B_BYTES);
   volatile int* abort_flag = &c.abort_flag;
 
-  setup(c, g.offsets, g.E, g.num_rows, g.err);
+  setup(c, g.offsets, g.E, g.num_rows, g.err, A_GATHER);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int total = c.total_mtiles * nN;
   const int nK = cdiv(g.K, BK);
   constexpr int BNo = SWIGLU_FWD ? BN / 2 : BN;  // logical output columns per tile
 
   if (warp == 0) {
-    // ---------------- TMA producer ----------------
+    // ---------------- TMA producer (weights; A too when grouped) ----------------
     int stage = 0;
     uint32_t phase = 0;
     for (int L = blockIdx.x; L < total; L += gridDim.x) {
       const Tile t = map_tile(c, g.E, nN, L);
-      int rows[4] = {0, 0, 0, 0};
-      if (A_GATHER) {
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const int i = min(t.row0 + 4 * lane + q, t.row_end - 1);
-          rows[q] = g.sorted_slot[i] / g.a_fan_out;
-        }
-      }
       for (int kb = 0; kb < nK; ++kb) {
         if (!mbar_wait(&c.empty[stage], phase ^ 1, abort_flag, g.err)) goto producer_done;
-        if (lane == 0) mbar_expect_tx(&c.full[stage], A_BYTES + B_BYTES);
-        __syncwarp();
-        uint8_t* a_dst = sA + stage * A_BYTES;
-        uint8_t* b_dst = sB + stage * B_BYTES;
-        if (A_GATHER) {
-          tma_gather4(a_dst + lane * 512, &tmA, &c.full[stage], kb * BK, rows[0], rows[1], rows[2],
-                      rows[3]);
-        } else if (lane == 0) {
-          tma_load_2d(a_dst, &tmA, &c.full[stage], kb * BK, t.row0);
-        }
         if (lane == 0) {
+          uint8_t* a_dst = sA + stage * A_BYTES;
+          uint8_t* b_dst = sB + stage * B_BYTES;
+          mbar_expect_tx(&c.full[stage], B_BYTES + (A_GATHER ? 0 : A_BYTES));
+          if (!A_GATHER) tma_load_2d(a_dst, &tmA, &c.full[stage], kb * BK, t.row0);
           if (B_KMAJOR) {
             tma_load_3d(b_dst, &tmB, &c.full[stage], kb * BK, t.nb * BN, t.e);
           } else {
@@ -373,10 +371,54 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
             }
           }
         }
+        __syncwarp();
         if (++stage == STAGES) { stage = 0; phase ^= 1; }
       }
     }
   producer_done:;
+  } else if (A_GATHER && warp >= kGatherWarp0) {
+    // ---------------- row gather of the scattered A operand ----------------
+    // thread t copies 16-byte chunk (t % 8) of tile rows t/8 + 16 j, j = 0..7,
+    // into the 128-byte-swizzled K-major layout; rows past the expert's slice
+    // and columns past K are zero-filled.
+    const int t = threadIdx.x - kGatherWarp0 * 32;
+    const int cc = t & 7, r0 = t >> 3;
+    const bf16* A = reinterpret_cast<const bf16*>(g.a);
+    int stage = 0;
+    uint32_t phase = 0;
+    for (int L = blockIdx.x; L < total; L += gridDim.x) {
+      const Tile tl = map_tile(c, g.E, nN, L);
+      const bf16* src[8];
+      uint32_t ok_rows = 0;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const int i = tl.row0 + r0 + 16 * j;
+        src[j] = A;
+        if (i < tl.row_end) {
+          const int p = g.sorted_slot[i];
+          const int xr = p / g.a_fan_out;
+          if (p >= 0 && xr < g.a_rows) {
+            src[j] = A + (size_t)xr * g.lda + 8 * cc;
+            ok_rows |= 1u << j;
+          } else {
+            report_error(g.err, ERRBIT_DATA);
+          }
+        }
+      }
+      for (int kb = 0; kb < nK; ++kb) {
+        if (!mbar_wait(&c.empty[stage], phase ^ 1, abort_flag, g.err)) goto gather_done;
+        const uint32_t a_dst = smem_u32(sA + stage * A_BYTES);
+        const bool col_ok = kb * BK + 8 * cc < g.K;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const bool ok = col_ok && ((ok_rows >> j) & 1u);
+          cp_async16(a_dst + sw128_off(r0 + 16 * j, cc), ok ? src[j] + kb * BK : A, ok ? 16u : 0u);
+        }
+        cp_async_arrive(&c.full[stage]);
+        if (++stage == STAGES) { stage = 0; phase ^= 1; }
+      }
+    }
+  gather_done:;
   } else if (warp == 1) {
     // ---------------- MMA issuer ----------------
     if (lane == 0) {
@@ -394,6 +436,7 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
         for (int kb = 0; kb < nK; ++kb) {
           if (!mbar_wait(&c.full[stage], phase, abort_flag, g.err)) { ok = false; break; }
           tc_fence_after();
+          if (A_GATHER) fence_proxy_async();  // rows written by cp.async, read by the tensor core
           const uint32_t a_addr = smem_u32(sA + stage * A_BYTES);
           const uint32_t b_addr = smem_u32(sB + stage * B_BYTES);
 #pragma unroll
@@ -410,7 +453,7 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
       }
     }
     __syncwarp();
-  } else if (warp >= 4) {
+  } else if (warp >= 4 && warp < 8) {  // warps 2-3 (and 8-11 without a gather) idle
     // ---------------- epilogue ----------------
     const int q = warp - 4;  // tensor-memory lane quadrant
     const int r = q * 32 + lane;
@@ -437,9 +480,71 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
 #pragma unroll 1
       for (int c0 = 0; c0 < BNo; c0 += 32) {
         float v[32], u[32];
+        const int n0 = t.nb * BNo + c0;
+        if (g.epi == EPI_ACT_BWD) {
+          // issue every global load of the chunk first, then read the accumulator
+          uint4 ra[4], rg[4], ru[4];
+          const bool swi = g.act == SMOE_ACT_SWIGLU;
+          const bool need_h = g.out != nullptr && g.act != SMOE_ACT_NONE;
+#pragma unroll
+          for (int j8 = 0; j8 < 4; ++j8) {
+            const int n = n0 + 8 * j8;
+            const bool in = p_ok && n < g.n_out;
+            ra[j8] = in ? __ldg(reinterpret_cast<const uint4*>(AUXA + (size_t)arow * g.ld_aux_a + n)) : make_uint4(0, 0, 0, 0);
+            rg[j8] = (in && need_h) ? __ldg(reinterpret_cast<const uint4*>(AUXH + (size_t)i * g.ld_aux_h + n)) : make_uint4(0, 0, 0, 0);
+            ru[j8] = (in && need_h && swi) ? __ldg(reinterpret_cast<const uint4*>(AUXH + (size_t)i * g.ld_aux_h + g.n_out + n)) : make_uint4(0, 0, 0, 0);
+          }
+          tmem_ld32(trow + c0, v);
+          if (!p_ok) continue;
+#pragma unroll
+          for (int j8 = 0; j8 < 4; ++j8) {
+            const int n = n0 + 8 * j8;
+            if (n >= g.n_out) break;
+            const float* vv = v + 8 * j8;
+            float a8[8], ga[8], dh[8], du[8], hg[8], hu[8];
+            unpack8(ra[j8], a8);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              dg_acc = fmaf(vv[j], a8[j], dg_acc);
+              ga[j] = gate * a8[j];
+            }
+            if (g.out2)
+              *reinterpret_cast<uint4*>(reinterpret_cast<bf16*>(g.out2) + (size_t)i * g.ldo2 + n) = pack8(ga);
+            if (!g.out) continue;
+            if (swi) {
+              unpack8(rg[j8], hg);
+              unpack8(ru[j8], hu);
+#pragma unroll
+              for (int j = 0; j < 8; ++j) {
+                const float da = gate * vv[j];
+                dh[j] = da * hu[j] * silu_grad_f(hg[j]);
+                du[j] = da * silu_f(hg[j]);
+              }
+              bf16* O = reinterpret_cast<bf16*>(g.out) + (size_t)orow * g.ldo;
+              *reinterpret_cast<uint4*>(O + n) = pack8(dh);
+              *reinterpret_cast<uint4*>(O + g.n_out + n) = pack8(du);
+            } else {
+              if (g.act == SMOE_ACT_GELU_TANH) {
+                unpack8(rg[j8], hg);
+#pragma unroll
+                for (int j = 0; j < 8; ++j) dh[j] = gate * vv[j] * gelu_tanh_grad_f(hg[j]);
+              } else {
+#pragma unroll
+                for (int j = 0; j < 8; ++j) dh[j] = gate * vv[j];
+              }
+              if (g.out_f32) {
+                float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(g.out) + (size_t)orow * g.ldo + n);
+                dst[0] = make_float4(dh[0], dh[1], dh[2], dh[3]);
+                dst[1] = make_float4(dh[4], dh[5], dh[6], dh[7]);
+              } else {
+                *reinterpret_cast<uint4*>(reinterpret_cast<bf16*>(g.out) + (size_t)orow * g.ldo + n) = pack8(dh);
+              }
+            }
+          }
+          continue;
+        }
         tmem_ld32(trow + c0, v);
         if (SWIGLU_FWD) tmem_ld32(trow + BNo + c0, u);
-        const int n0 = t.nb * BNo + c0;
         if (!p_ok) continue;
 #pragma unroll
         for (int j8 = 0; j8 < 4; ++j8) {
@@ -457,7 +562,7 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
             } else {
               *reinterpret_cast<uint4*>(reinterpret_cast<bf16*>(g.out) + (size_t)orow * g.ldo + n) = pack8(o);
             }
-          } else if (g.epi == EPI_ACT_FWD) {
+          } else {  // EPI_ACT_FWD
             float a8[8];
             if (SWIGLU_FWD) {
               float* uu = u + 8 * j8;
@@ -472,50 +577,6 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
               *reinterpret_cast<uint4*>(reinterpret_cast<bf16*>(g.out) + (size_t)orow * g.ldo + n) = pack8(vv);
             }
             *reinterpret_cast<uint4*>(reinterpret_cast<bf16*>(g.out2) + (size_t)orow * g.ldo2 + n) = pack8(a8);
-          } else {  // EPI_ACT_BWD: vv = dA'
-            float a8[8];
-            unpack8(*reinterpret_cast<const uint4*>(AUXA + (size_t)arow * g.ld_aux_a + n), a8);
-            float ga[8], dh[8];
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-              dg_acc = fmaf(vv[j], a8[j], dg_acc);
-              ga[j] = gate * a8[j];
-            }
-            if (g.out2)
-              *reinterpret_cast<uint4*>(reinterpret_cast<bf16*>(g.out2) + (size_t)i * g.ldo2 + n) = pack8(ga);
-            if (g.out) {
-              if (g.act == SMOE_ACT_SWIGLU) {
-                float hg[8], hu[8], du[8];
-                unpack8(*reinterpret_cast<const uint4*>(AUXH + (size_t)i * g.ld_aux_h + n), hg);
-                unpack8(*reinterpret_cast<const uint4*>(AUXH + (size_t)i * g.ld_aux_h + g.n_out + n), hu);
-#pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                  const float da = gate * vv[j];
-                  dh[j] = da * hu[j] * silu_grad_f(hg[j]);
-                  du[j] = da * silu_f(hg[j]);
-                }
-                bf16* O = reinterpret_cast<bf16*>(g.out) + (size_t)orow * g.ldo;
-                *reinterpret_cast<uint4*>(O + n) = pack8(dh);
-                *reinterpret_cast<uint4*>(O + g.n_out + n) = pack8(du);
-              } else {
-                if (g.act == SMOE_ACT_GELU_TANH) {
-                  float h8[8];
-                  unpack8(*reinterpret_cast<const uint4*>(AUXH + (size_t)i * g.ld_aux_h + n), h8);
-#pragma unroll
-                  for (int j = 0; j < 8; ++j) dh[j] = gate * vv[j] * gelu_tanh_grad_f(h8[j]);
-                } else {
-#pragma unroll
-                  for (int j = 0; j < 8; ++j) dh[j] = gate * vv[j];
-                }
-                if (g.out_f32) {
-                  float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(g.out) + (size_t)orow * g.ldo + n);
-                  dst[0] = make_float4(dh[0], dh[1], dh[2], dh[3]);
-                  dst[1] = make_float4(dh[4], dh[5], dh[6], dh[7]);
-                } else {
-                  *reinterpret_cast<uint4*>(reinterpret_cast<bf16*>(g.out) + (size_t)orow * g.ldo + n) = pack8(dh);
-                }
-              }
-            }
           }
         }
       }
@@ -532,6 +593,43 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
 // ---------------------------------------------------------------------------
 // dW kernel
 // ---------------------------------------------------------------------------
+// Gather of NS 64-column slabs of BK scattered rows (the MN-major operand of the
+// dW product) with cp.async: thread t copies chunk (t % 8NS) of rows
+// t / 8NS + (128 / 8NS) j.  The slot indices of a stage are loaded one stage
+// ahead (slab_rows) so the index latency overlaps the previous stage's copies;
+// rows past the slice and columns past `ncols` are zero-filled.
+template <int NS>
+struct SlabGather {
+  static constexpr int CPR = 8 * NS;
+  static constexpr int RSTEP = kGatherThreads / CPR;
+  static constexpr int NR = BK / RSTEP;
+  int p[NR];  // slot of each of this thread's rows, -1 past the slice
+
+  __device__ __forceinline__ void load(const int32_t* sorted_slot, int rk, int valid, int t) {
+#pragma unroll
+    for (int j = 0; j < NR; ++j) {
+      const int row = t / CPR + RSTEP * j;
+      p[j] = row < valid ? __ldg(sorted_slot + rk + row) : -1;
+    }
+  }
+  __device__ __forceinline__ void issue(uint32_t dst, const bf16* base, int ld, int col0, int ncols,
+                                        int fan_out, int src_rows, int t, unsigned* err) const {
+    const int cg = t % CPR, slab = cg >> 3, cc = cg & 7;
+    const int col = col0 + 64 * slab + 8 * cc;
+    const bool col_ok = col < ncols;
+#pragma unroll
+    for (int j = 0; j < NR; ++j) {
+      const int row = t / CPR + RSTEP * j;
+      const int sr = p[j] >= 0 ? p[j] / fan_out : -1;
+      const bool in_range = sr < src_rows;
+      if (p[j] >= 0 && !in_range) report_error(err, ERRBIT_DATA);
+      const bool ok = col_ok && p[j] >= 0 && in_range;
+      cp_async16(dst + slab * 8192 + sw128_off(row, cc), ok ? base + (size_t)sr * ld + col : base,
+                 ok ? 16u : 0u);
+    }
+  }
+};
+
 template <bool A_GATHER, bool B_GATHER>
 __global__ void __launch_bounds__(kThreads, 1)
 dw_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
@@ -543,7 +641,7 @@ dw_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
   SharedCtl& c = *reinterpret_cast<SharedCtl*>(sB + STAGES * B_BYTES);
   volatile int* abort_flag = &c.abort_flag;
 
-  setup(c, g.offsets, g.E, g.num_rows, g.err);
+  setup(c, g.offsets, g.E, g.num_rows, g.err, A_GATHER || B_GATHER);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const bool offsets_ok = c.total_mtiles > 0 || g.num_rows == 0;
   const int total = offsets_ok ? g.E * nM * nN : 0;
@@ -556,6 +654,7 @@ dw_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
   };
 
   if (warp == 0) {
+    // ---------------- TMA producer of the grouped operand(s) ----------------
     int stage = 0;
     uint32_t phase = 0;
     for (int L = blockIdx.x; L < total; L += gridDim.x) {
@@ -565,49 +664,65 @@ dw_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
       const int nK = cdiv(r_end - r_begin, BK);
       for (int kb = 0; kb < nK; ++kb) {
         if (!mbar_wait(&c.empty[stage], phase ^ 1, abort_flag, g.err)) goto producer_done;
-        if (lane == 0) mbar_expect_tx(&c.full[stage], A_BYTES + B_BYTES);
+        if (lane == 0) {
+          uint8_t* a_dst = sA + stage * A_BYTES;
+          uint8_t* b_dst = sB + stage * B_BYTES;
+          const int rk = r_begin + kb * BK;
+          mbar_expect_tx(&c.full[stage], (A_GATHER ? 0 : A_BYTES) + (B_GATHER ? 0 : B_BYTES));
+          if (!A_GATHER) {  // 64 rows x 128 M-columns: two 64-column slabs of 8 KB
+            tma_load_2d(a_dst, &tmA, &c.full[stage], mb * BM, rk);
+            tma_load_2d(a_dst + 8192, &tmA, &c.full[stage], mb * BM + 64, rk);
+          }
+          if (!B_GATHER) {  // 64 rows x 256 N-columns: four slabs
+#pragma unroll
+            for (int slab = 0; slab < 4; ++slab)
+              tma_load_2d(b_dst + slab * 8192, &tmB, &c.full[stage], nb * BN + 64 * slab, rk);
+          }
+        }
         __syncwarp();
-        uint8_t* a_dst = sA + stage * A_BYTES;
-        uint8_t* b_dst = sB + stage * B_BYTES;
-        const int rk = r_begin + kb * BK;
-        // A: 64 rows x 128 M-columns (two 64-column slabs of 8 KB)
-        if (A_GATHER) {
-          const int slab = lane >> 4, j = lane & 15;
-          int rr[4];
-#pragma unroll
-          for (int qq = 0; qq < 4; ++qq) {
-            const int rrow = min(rk + 4 * j + qq, r_end - 1);
-            rr[qq] = g.sorted_slot[rrow] / g.a_fan_out;
-          }
-          tma_gather4(a_dst + slab * 8192 + j * 512, &tmA, &c.full[stage], mb * BM + 64 * slab,
-                      rr[0], rr[1], rr[2], rr[3]);
-        } else if (lane == 0) {
-          tma_load_2d(a_dst, &tmA, &c.full[stage], mb * BM, rk);
-          tma_load_2d(a_dst + 8192, &tmA, &c.full[stage], mb * BM + 64, rk);
-        }
-        // B: 64 rows x 256 N-columns (four slabs)
-        if (B_GATHER) {
-#pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            const int slab = 2 * h + (lane >> 4), j = lane & 15;
-            int rr[4];
-#pragma unroll
-            for (int qq = 0; qq < 4; ++qq) {
-              const int rrow = min(rk + 4 * j + qq, r_end - 1);
-              rr[qq] = g.sorted_slot[rrow] / g.b_fan_out;
-            }
-            tma_gather4(b_dst + slab * 8192 + j * 512, &tmB, &c.full[stage], nb * BN + 64 * slab,
-                        rr[0], rr[1], rr[2], rr[3]);
-          }
-        } else if (lane == 0) {
-#pragma unroll
-          for (int slab = 0; slab < 4; ++slab)
-            tma_load_2d(b_dst + slab * 8192, &tmB, &c.full[stage], nb * BN + 64 * slab, rk);
-        }
         if (++stage == STAGES) { stage = 0; phase ^= 1; }
       }
     }
   producer_done:;
+  } else if ((A_GATHER || B_GATHER) && warp >= kGatherWarp0) {
+    // ---------------- cp.async gather of the scattered operand(s) ----------------
+    const int t = threadIdx.x - kGatherWarp0 * 32;
+    SlabGather<2> ga0, ga1;  // ping-pong: one buffer in use, the other loading
+    SlabGather<4> gb0, gb1;
+    int stage = 0;
+    uint32_t phase = 0;
+    for (int L = blockIdx.x; L < total; L += gridDim.x) {
+      int e, mb, nb;
+      coords(L, e, mb, nb);
+      const int r_begin = c.off[e], r_end = c.off[e + 1];
+      const int nK = cdiv(r_end - r_begin, BK);
+      if (nK == 0) continue;
+      if (A_GATHER) ga0.load(g.sorted_slot, r_begin, min(BK, r_end - r_begin), t);
+      if (B_GATHER) gb0.load(g.sorted_slot, r_begin, min(BK, r_end - r_begin), t);
+      auto step = [&](SlabGather<2>& ca, SlabGather<4>& cb, SlabGather<2>& na, SlabGather<4>& nbuf,
+                      int kb) -> bool {
+        if (kb + 1 < nK) {  // indices of the next stage, consumed one step later
+          const int rn = r_begin + (kb + 1) * BK;
+          if (A_GATHER) na.load(g.sorted_slot, rn, min(BK, r_end - rn), t);
+          if (B_GATHER) nbuf.load(g.sorted_slot, rn, min(BK, r_end - rn), t);
+        }
+        if (!mbar_wait(&c.empty[stage], phase ^ 1, abort_flag, g.err)) return false;
+        if (A_GATHER)
+          ca.issue(smem_u32(sA + stage * A_BYTES), reinterpret_cast<const bf16*>(g.a), g.lda,
+                   mb * BM, g.M, g.a_fan_out, g.a_rows, t, g.err);
+        if (B_GATHER)
+          cb.issue(smem_u32(sB + stage * B_BYTES), reinterpret_cast<const bf16*>(g.b), g.ldb,
+                   nb * BN, g.N, g.b_fan_out, g.b_rows, t, g.err);
+        cp_async_arrive(&c.full[stage]);
+        if (++stage == STAGES) { stage = 0; phase ^= 1; }
+        return true;
+      };
+      for (int kb = 0; kb < nK; kb += 2) {
+        if (!step(ga0, gb0, ga1, gb1, kb)) goto gather_done;
+        if (kb + 1 < nK && !step(ga1, gb1, ga0, gb0, kb + 1)) goto gather_done;
+      }
+    }
+  gather_done:;
   } else if (warp == 1) {
     constexpr uint32_t idesc = idesc_bf16(BM, BN, 1, 1);
     int stage = 0;
@@ -627,6 +742,7 @@ dw_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
       for (int kb = 0; kb < nK; ++kb) {
         if (!mbar_wait(&c.full[stage], phase, abort_flag, g.err)) { ok = false; break; }
         tc_fence_after();
+        if (A_GATHER || B_GATHER) fence_proxy_async();  // cp.async rows -> tensor core
         const int valid = min(BK, r_end - (r_begin + kb * BK));
         if (valid < BK) {
           // rows past the slice end hold other rows' data: zero them in both operands
@@ -660,7 +776,7 @@ dw_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
       }
       __syncwarp();
     }
-  } else if (warp >= 4) {
+  } else if (warp >= 4 && warp < 8) {  // warps 2-3 (and 8-11 without a gather) idle
     const int q = warp - 4;
     const int r = q * 32 + lane;
     int it = 0;
@@ -800,7 +916,7 @@ cudaError_t launch_grouped_gemm_tc(const GroupedGemm& g, cudaStream_t s) {
   const int nN = cdiv(g.n_out, BNo);
   const bool gather = g.a_mode == ROWS_GATHER;
   CUtensorMap ta, tb;
-  cudaError_t e = rows_map(&ta, g.a, g.K, g.a_rows, g.lda, gather ? 1 : BM);
+  cudaError_t e = rows_map(&ta, g.a, g.K, g.a_rows, g.lda, BM);  // unused when gathered
   if (e != cudaSuccess) return e;
   const bool kmaj = g.b_kn == 0;
   if (kmaj) {  // W[e] is [NW, K]: dims {K, NW, E}
@@ -834,9 +950,9 @@ cudaError_t launch_dw_gemm_tc(const DwGemm& g, cudaStream_t s) {
   const int nM = cdiv(g.M, BM), nN = cdiv(g.N, BN);
   const bool ag = g.a_mode == ROWS_GATHER, bg = g.b_mode == ROWS_GATHER;
   CUtensorMap ta, tb;
-  cudaError_t e = rows_map(&ta, g.a, g.M, g.a_rows, g.lda, ag ? 1 : BK);
+  cudaError_t e = rows_map(&ta, g.a, g.M, g.a_rows, g.lda, BK);  // unused when gathered
   if (e != cudaSuccess) return e;
-  e = rows_map(&tb, g.b, g.N, g.b_rows, g.ldb, bg ? 1 : BK);
+  e = rows_map(&tb, g.b, g.N, g.b_rows, g.ldb, BK);
   if (e != cudaSuccess) return e;
   const long long tiles = (long long)g.E * nM * nN;
   const int grid = (int)(tiles < num_sms() ? tiles : num_sms());
