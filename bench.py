@@ -243,7 +243,9 @@ def run_reference(args, world, rank):
 # ---------------------------------------------------------------------------
 def run_ours(args, world, rank):
     import sparse_mixture_experts_smoe_b200 as smoe
-    cfg = WORKLOADS[args.workload]
+    cfg = dict(WORKLOADS[args.workload])
+    if args.tokens:
+        cfg["T"] = args.tokens
     if cfg["kind"] != "mlp":
         raise SystemExit("the benchmark step is the SMoE MLP; pick an mlp workload")
     dev = torch.device("cuda", torch.cuda.current_device())
@@ -354,7 +356,7 @@ def run_ours(args, world, rank):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if dt == torch.bfloat16 else "f32",
         "data": "synthetic",
-        "config": {"workload": args.workload, "T": cfg["T"], "d": cfg["d"], "f": cfg["f"],
+        "config": {"workload": args.workload + ("" if not args.tokens else f"-T{cfg['T']}"), "T": cfg["T"], "d": cfg["d"], "f": cfg["f"],
                    "E": cfg["E"], "k": cfg["k"], "act": cfg["act"], "parallelism": f"replicas x{world}",
                    "l2": "inputs larger than L2 (x 134 MB, weights 2.8 GB), no flush"},
         "tflops_fwd_bwd": round(tflops, 1),
@@ -384,6 +386,8 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--tokens", type=int, default=0,
+                    help="override T (smaller cases for profiler captures; never a bench line)")
     args = ap.parse_args()
     world, rank, _ = dist_setup()
     try:

@@ -245,11 +245,16 @@ __device__ __forceinline__ void unpack8(uint4 u, float* v) {
 // ---------------------------------------------------------------------------
 // Shared state and tile list
 // ---------------------------------------------------------------------------
+constexpr int IDX_STAGES = 8;  // slot-index ring of the dW gathers (stages ahead)
+
 struct SharedCtl {
   uint64_t full[STAGES];
   uint64_t empty[STAGES];
   uint64_t tfull[2];
   uint64_t tempty[2];
+  uint64_t ifull[IDX_STAGES];   // index ring: written by warp 2
+  uint64_t iempty[IDX_STAGES];  // index ring: released by the 4 gather warps
+  int idx[IDX_STAGES][BK];      // slot of each row of a dW stage, -1 past the slice
   uint32_t tmem_base;
   int abort_flag;
   int total_mtiles;
@@ -291,6 +296,10 @@ __device__ __forceinline__ void setup(SharedCtl& c, const int32_t* offsets, int 
     for (int b = 0; b < 2; ++b) {
       mbar_init(&c.tfull[b], 1);
       mbar_init(&c.tempty[b], 4);
+    }
+    for (int b = 0; b < IDX_STAGES; ++b) {
+      mbar_init(&c.ifull[b], 1);
+      mbar_init(&c.iempty[b], kGatherThreads / 32);
     }
     c.abort_flag = 0;
     fence_mbar_init();
@@ -595,9 +604,10 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
 // ---------------------------------------------------------------------------
 // Gather of NS 64-column slabs of BK scattered rows (the MN-major operand of the
 // dW product) with cp.async: thread t copies chunk (t % 8NS) of rows
-// t / 8NS + (128 / 8NS) j.  The slot indices of a stage are loaded one stage
-// ahead (slab_rows) so the index latency overlaps the previous stage's copies;
-// rows past the slice and columns past `ncols` are zero-filled.
+// t / 8NS + (128 / 8NS) j.  The slot indices come from a shared-memory ring that
+// an index warp fills up to IDX_STAGES stages ahead, so no global-load latency
+// sits between a free stage and its copies; rows past the slice and columns past
+// `ncols` are zero-filled.
 template <int NS>
 struct SlabGather {
   static constexpr int CPR = 8 * NS;
@@ -605,22 +615,20 @@ struct SlabGather {
   static constexpr int NR = BK / RSTEP;
   int p[NR];  // slot of each of this thread's rows, -1 past the slice
 
-  __device__ __forceinline__ void load(const int32_t* sorted_slot, int rk, int valid, int t) {
+  __device__ __forceinline__ void load(const int* ring_stage, int t) {
 #pragma unroll
-    for (int j = 0; j < NR; ++j) {
-      const int row = t / CPR + RSTEP * j;
-      p[j] = row < valid ? __ldg(sorted_slot + rk + row) : -1;
-    }
+    for (int j = 0; j < NR; ++j) p[j] = ring_stage[t / CPR + RSTEP * j];
   }
   __device__ __forceinline__ void issue(uint32_t dst, const bf16* base, int ld, int col0, int ncols,
-                                        int fan_out, int src_rows, int t, unsigned* err) const {
+                                        int fan_out, int fan_shift, int src_rows, int t,
+                                        unsigned* err) const {
     const int cg = t % CPR, slab = cg >> 3, cc = cg & 7;
     const int col = col0 + 64 * slab + 8 * cc;
     const bool col_ok = col < ncols;
 #pragma unroll
     for (int j = 0; j < NR; ++j) {
       const int row = t / CPR + RSTEP * j;
-      const int sr = p[j] >= 0 ? p[j] / fan_out : -1;
+      const int sr = p[j] < 0 ? -1 : (fan_shift >= 0 ? (p[j] >> fan_shift) : p[j] / fan_out);
       const bool in_range = sr < src_rows;
       if (p[j] >= 0 && !in_range) report_error(err, ERRBIT_DATA);
       const bool ok = col_ok && p[j] >= 0 && in_range;
@@ -684,98 +692,125 @@ dw_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
       }
     }
   producer_done:;
-  } else if ((A_GATHER || B_GATHER) && warp >= kGatherWarp0) {
-    // ---------------- cp.async gather of the scattered operand(s) ----------------
-    const int t = threadIdx.x - kGatherWarp0 * 32;
-    SlabGather<2> ga0, ga1;  // ping-pong: one buffer in use, the other loading
-    SlabGather<4> gb0, gb1;
-    int stage = 0;
-    uint32_t phase = 0;
+  } else if ((A_GATHER || B_GATHER) && warp == 2) {
+    // ---------------- slot-index producer for the gathers ----------------
+    int istage = 0;
+    uint32_t iphase = 0;
     for (int L = blockIdx.x; L < total; L += gridDim.x) {
       int e, mb, nb;
       coords(L, e, mb, nb);
       const int r_begin = c.off[e], r_end = c.off[e + 1];
       const int nK = cdiv(r_end - r_begin, BK);
-      if (nK == 0) continue;
-      if (A_GATHER) ga0.load(g.sorted_slot, r_begin, min(BK, r_end - r_begin), t);
-      if (B_GATHER) gb0.load(g.sorted_slot, r_begin, min(BK, r_end - r_begin), t);
-      auto step = [&](SlabGather<2>& ca, SlabGather<4>& cb, SlabGather<2>& na, SlabGather<4>& nbuf,
-                      int kb) -> bool {
-        if (kb + 1 < nK) {  // indices of the next stage, consumed one step later
-          const int rn = r_begin + (kb + 1) * BK;
-          if (A_GATHER) na.load(g.sorted_slot, rn, min(BK, r_end - rn), t);
-          if (B_GATHER) nbuf.load(g.sorted_slot, rn, min(BK, r_end - rn), t);
+      for (int kb = 0; kb < nK; ++kb) {
+        if (!mbar_wait(&c.iempty[istage], iphase ^ 1, abort_flag, g.err)) goto index_done;
+        const int rk = r_begin + kb * BK;
+#pragma unroll
+        for (int q = 0; q < BK / 32; ++q) {
+          const int row = lane + 32 * q;
+          c.idx[istage][row] = rk + row < r_end ? __ldg(g.sorted_slot + rk + row) : -1;
         }
-        if (!mbar_wait(&c.empty[stage], phase ^ 1, abort_flag, g.err)) return false;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&c.ifull[istage]);
+        if (++istage == IDX_STAGES) { istage = 0; iphase ^= 1; }
+      }
+    }
+  index_done:;
+  } else if ((A_GATHER || B_GATHER) && warp >= kGatherWarp0) {
+    // ---------------- cp.async gather of the scattered operand(s) ----------------
+    const int t = threadIdx.x - kGatherWarp0 * 32;
+    const int a_shift = (g.a_fan_out & (g.a_fan_out - 1)) == 0 ? __ffs(g.a_fan_out) - 1 : -1;
+    const int b_shift = (g.b_fan_out & (g.b_fan_out - 1)) == 0 ? __ffs(g.b_fan_out) - 1 : -1;
+    SlabGather<2> ga;
+    SlabGather<4> gb;
+    int stage = 0, istage = 0;
+    uint32_t phase = 0, iphase = 0;
+    for (int L = blockIdx.x; L < total; L += gridDim.x) {
+      int e, mb, nb;
+      coords(L, e, mb, nb);
+      const int nK = cdiv(c.off[e + 1] - c.off[e], BK);
+      for (int kb = 0; kb < nK; ++kb) {
+        if (!mbar_wait(&c.ifull[istage], iphase, abort_flag, g.err)) goto gather_done;
+        if (A_GATHER) ga.load(c.idx[istage], t);
+        if (B_GATHER) gb.load(c.idx[istage], t);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&c.iempty[istage]);
+        if (++istage == IDX_STAGES) { istage = 0; iphase ^= 1; }
+        if (!mbar_wait(&c.empty[stage], phase ^ 1, abort_flag, g.err)) goto gather_done;
         if (A_GATHER)
-          ca.issue(smem_u32(sA + stage * A_BYTES), reinterpret_cast<const bf16*>(g.a), g.lda,
-                   mb * BM, g.M, g.a_fan_out, g.a_rows, t, g.err);
+          ga.issue(smem_u32(sA + stage * A_BYTES), reinterpret_cast<const bf16*>(g.a), g.lda,
+                   mb * BM, g.M, g.a_fan_out, a_shift, g.a_rows, t, g.err);
         if (B_GATHER)
-          cb.issue(smem_u32(sB + stage * B_BYTES), reinterpret_cast<const bf16*>(g.b), g.ldb,
-                   nb * BN, g.N, g.b_fan_out, g.b_rows, t, g.err);
+          gb.issue(smem_u32(sB + stage * B_BYTES), reinterpret_cast<const bf16*>(g.b), g.ldb,
+                   nb * BN, g.N, g.b_fan_out, b_shift, g.b_rows, t, g.err);
         cp_async_arrive(&c.full[stage]);
         if (++stage == STAGES) { stage = 0; phase ^= 1; }
-        return true;
-      };
-      for (int kb = 0; kb < nK; kb += 2) {
-        if (!step(ga0, gb0, ga1, gb1, kb)) goto gather_done;
-        if (kb + 1 < nK && !step(ga1, gb1, ga0, gb0, kb + 1)) goto gather_done;
       }
     }
   gather_done:;
   } else if (warp == 1) {
+    // ---------------- MMA issuer ----------------
+    // With a gathered operand its rows past the slice are zero-filled, so the
+    // other operand's rows there (finite data or zero fill) contribute nothing and
+    // one lane runs the loop.  With two grouped operands the warp zeroes the
+    // tail rows of both in shared memory first.
+    constexpr bool kGather = A_GATHER || B_GATHER;
     constexpr uint32_t idesc = idesc_bf16(BM, BN, 1, 1);
-    int stage = 0;
-    uint32_t phase = 0;
-    int it = 0;
-    for (int L = blockIdx.x; L < total; L += gridDim.x, ++it) {
-      int e, mb, nb;
-      coords(L, e, mb, nb);
-      const int r_begin = c.off[e], r_end = c.off[e + 1];
-      const int nK = cdiv(r_end - r_begin, BK);
-      const int buf = it & 1;
-      const uint32_t tph = (it >> 1) & 1;
-      if (!mbar_wait(&c.tempty[buf], tph ^ 1, abort_flag, g.err)) break;
-      tc_fence_after();
-      const uint32_t d_tmem = c.tmem_base + buf * BN;
-      bool ok = true;
-      for (int kb = 0; kb < nK; ++kb) {
-        if (!mbar_wait(&c.full[stage], phase, abort_flag, g.err)) { ok = false; break; }
+    if (!kGather || lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int it = 0;
+      for (int L = blockIdx.x; L < total; L += gridDim.x, ++it) {
+        int e, mb, nb;
+        coords(L, e, mb, nb);
+        const int r_begin = c.off[e], r_end = c.off[e + 1];
+        const int nK = cdiv(r_end - r_begin, BK);
+        const int buf = it & 1;
+        const uint32_t tph = (it >> 1) & 1;
+        if (!mbar_wait(&c.tempty[buf], tph ^ 1, abort_flag, g.err)) break;
         tc_fence_after();
-        if (A_GATHER || B_GATHER) fence_proxy_async();  // cp.async rows -> tensor core
-        const int valid = min(BK, r_end - (r_begin + kb * BK));
-        if (valid < BK) {
-          // rows past the slice end hold other rows' data: zero them in both operands
-          uint8_t* a_t = sA + stage * A_BYTES;
-          uint8_t* b_t = sB + stage * B_BYTES;
-          const int nz = (BK - valid) * 8;  // 16-byte chunks per slab
-          for (int z = lane; z < nz * 6; z += 32) {
-            const int slab = z / nz, w = z % nz;
-            uint8_t* base = slab < 2 ? a_t + slab * 8192 : b_t + (slab - 2) * 8192;
-            *reinterpret_cast<uint4*>(base + valid * 128 + w * 16) = make_uint4(0, 0, 0, 0);
+        const uint32_t d_tmem = c.tmem_base + buf * BN;
+        bool ok = true;
+        for (int kb = 0; kb < nK; ++kb) {
+          if (!mbar_wait(&c.full[stage], phase, abort_flag, g.err)) { ok = false; break; }
+          tc_fence_after();
+          if (kGather) {
+            fence_proxy_async();  // cp.async rows -> tensor core
+          } else {
+            const int valid = min(BK, r_end - (r_begin + kb * BK));
+            if (valid < BK) {  // rows past the slice end hold other rows' data
+              uint8_t* a_t = sA + stage * A_BYTES;
+              uint8_t* b_t = sB + stage * B_BYTES;
+              const int nz = (BK - valid) * 8;  // 16-byte chunks per slab
+              for (int z = lane; z < nz * 6; z += 32) {
+                const int slab = z / nz, w = z % nz;
+                uint8_t* base = slab < 2 ? a_t + slab * 8192 : b_t + (slab - 2) * 8192;
+                *reinterpret_cast<uint4*>(base + valid * 128 + w * 16) = make_uint4(0, 0, 0, 0);
+              }
+              fence_proxy_async();
+            }
+            __syncwarp();
           }
-          fence_proxy_async();
-          __syncwarp();
-        }
-        if (lane == 0) {
-          const uint32_t a_addr = smem_u32(sA + stage * A_BYTES);
-          const uint32_t b_addr = smem_u32(sB + stage * B_BYTES);
+          if (lane == 0) {
+            const uint32_t a_addr = smem_u32(sA + stage * A_BYTES);
+            const uint32_t b_addr = smem_u32(sB + stage * B_BYTES);
 #pragma unroll
-          for (int kk = 0; kk < BK / 16; ++kk)
-            umma_bf16(d_tmem, desc_mnmajor(a_addr + kk * 2048), desc_mnmajor(b_addr + kk * 2048),
-                      idesc, (kb | kk) != 0);
-          umma_commit(&c.empty[stage]);
+            for (int kk = 0; kk < BK / 16; ++kk)
+              umma_bf16(d_tmem, desc_mnmajor(a_addr + kk * 2048), desc_mnmajor(b_addr + kk * 2048),
+                        idesc, (kb | kk) != 0);
+            umma_commit(&c.empty[stage]);
+          }
+          if (!kGather) __syncwarp();
+          if (++stage == STAGES) { stage = 0; phase ^= 1; }
         }
-        __syncwarp();
-        if (++stage == STAGES) { stage = 0; phase ^= 1; }
+        if (!ok) break;
+        if (lane == 0) {
+          if (nK > 0) umma_commit(&c.tfull[buf]);
+          else mbar_arrive(&c.tfull[buf]);
+        }
+        if (!kGather) __syncwarp();
       }
-      if (!ok) break;
-      if (lane == 0) {
-        if (nK > 0) umma_commit(&c.tfull[buf]);
-        else mbar_arrive(&c.tfull[buf]);
-      }
-      __syncwarp();
     }
+    __syncwarp();
   } else if (warp >= 4 && warp < 8) {  // warps 2-3 (and 8-11 without a gather) idle
     const int q = warp - 4;
     const int r = q * 32 + lane;
