@@ -146,6 +146,27 @@ int smoe_route_bwd(const void* x, const void* w_r, const int32_t* topk_idx, cons
 int smoe_sort(const int32_t* topk_idx, int T, int k, int E, int32_t* sorted_slot,
               int32_t* expert_offsets, void* workspace, size_t ws_bytes, void* stream);
 
+/* smoe_sort_static: the same stable sort and offsets as smoe_sort, for callers
+ * that cannot allocate device memory for a workspace -- for example a runtime
+ * that plans all device memory up front and gives its kernels only their inputs
+ * and outputs, or code running while a CUDA graph is being captured, where a
+ * cudaMalloc would synchronise the device or escape the graph.  This entry point
+ * calls no allocator.  (The paper has no counterpart; it is a calling
+ * convention of this library.)
+ *   Scratch: a fixed 256 KB device array inside the library (held by every GPU
+ *   that loads the library until the process exits) stores the per-block expert
+ *   counts, so ceil(T*k / 4096) * E must be <= 65536; larger problems are
+ *   rejected with SMOE_ERR_INVALID_ARG and a message (use smoe_sort).
+ *   The first call on a device looks up the array's device address with that
+ *   device current; make that first call before any stream capture begins.
+ *   Every call rewrites all the counts it uses, so nothing has to be cleared
+ *   between calls; but all calls share the one array, so calls whose work
+ *   overlaps on the GPU (different streams without ordering) race and give
+ *   wrong results.  Serialise them (one stream, or events).
+ * Arguments, outputs and data-error reporting are those of smoe_sort.          */
+int smoe_sort_static(const int32_t* topk_idx, int T, int k, int E, int32_t* sorted_slot,
+                     int32_t* expert_offsets, void* stream);
+
 /* ---------------------------------------------------------------------------
  * ParallelLinear [rev1, rev2, art]
  *

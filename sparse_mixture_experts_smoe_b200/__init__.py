@@ -68,6 +68,7 @@ def lib():
     L.smoe_route_bwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int,
                                  _vp, _vp, _vp, _vp, _c_size, _vp]
     L.smoe_sort.argtypes = [_vp, _c_int, _c_int, _c_int, _vp, _vp, _vp, _c_size, _vp]
+    L.smoe_sort_static.argtypes = [_vp, _c_int, _c_int, _c_int, _vp, _vp, _vp]
     L.parallel_linear_fwd_workspace_size.restype = _c_size
     L.parallel_linear_fwd_workspace_size.argtypes = [_c_int] * 6
     L.parallel_linear_fwd.argtypes = [_vp, _c_int, _c_int, _vp, _c_int, _c_int, _vp, _vp, _c_int,
@@ -203,6 +204,21 @@ def smoe_sort(topk_idx, E, stream=None):
     _check(lib().smoe_sort(_ptr(topk_idx), T, k, E, _ptr(ss), _ptr(off), _ptr(ws), ws.numel(),
                            _stream(stream)))
     return ss, off
+
+
+def smoe_sort_static(topk_idx, E, sorted_slot=None, expert_offsets=None, stream=None):
+    """smoe_sort without a workspace: the library keeps the per-block counts in
+    a fixed device array of its own (for callers that cannot allocate; see
+    smoe_sort_static in smoe.h for the size limit and the no-overlap rule)."""
+    _need(topk_idx, "topk_idx", torch.int32)
+    T, k = topk_idx.shape
+    if sorted_slot is None:
+        sorted_slot = torch.empty((T * k,), dtype=torch.int32, device=topk_idx.device)
+    if expert_offsets is None:
+        expert_offsets = torch.empty((E + 1,), dtype=torch.int32, device=topk_idx.device)
+    _check(lib().smoe_sort_static(_ptr(topk_idx), T, k, E, _ptr(sorted_slot),
+                                  _ptr(expert_offsets), _stream(stream)))
+    return sorted_slot, expert_offsets
 
 
 def parallel_linear_fwd(x, w, sorted_slot, expert_offsets, fan_out, grouped_in, grouped_out,

@@ -241,6 +241,17 @@ int validate_mlp_desc(const smoe_mlp_desc* m) {
 
 }  // namespace
 
+namespace smoe {
+int api_fail(int code, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_msg, sizeof(g_msg), fmt, ap);
+  va_end(ap);
+  return code;
+}
+unsigned* api_error_word(cudaError_t* status) { return error_word(status); }
+}  // namespace smoe
+
 extern "C" {
 
 const char* smoe_last_error(void) { return g_msg; }

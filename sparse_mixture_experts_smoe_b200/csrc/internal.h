@@ -112,4 +112,10 @@ bool tc_supported();
 cudaError_t launch_grouped_gemm_tc(const GroupedGemm& g, cudaStream_t s);
 cudaError_t launch_dw_gemm_tc(const DwGemm& g, cudaStream_t s);
 
+// Error reporting shared with entry points defined outside api.cu: sets the
+// thread-local message returned by smoe_last_error and returns `code`.
+int api_fail(int code, const char* fmt, ...);
+// This device's error word (resolved once per device), or null with *status set.
+unsigned* api_error_word(cudaError_t* status);
+
 }  // namespace smoe

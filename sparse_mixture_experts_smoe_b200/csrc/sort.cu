@@ -12,6 +12,8 @@
 //               within a round, __match_any_sync gives each lane its rank among
 //               same-expert lanes of its warp, and per-warp counts are scanned
 //               across warps, so equal ids keep ascending slot order (stable).
+#include <mutex>
+
 #include "common.cuh"
 
 namespace smoe {
@@ -154,4 +156,73 @@ cudaError_t launch_sort(const int32_t* idx, int T_, int k, int E, int32_t* sorte
   return cudaGetLastError();
 }
 
+// ---------------------------------------------------------------------------
+// Allocation-free variant of the sort (smoe_sort_static in smoe.h).
+//
+// Some callers have no way to obtain device memory for a workspace: code that
+// runs inside a memory-planned inference runtime which hands kernels only their
+// inputs and outputs, or code called where cudaMalloc must not be used (for
+// example while work is being captured into a CUDA graph, where an allocation
+// would synchronise or fall outside the graph).  For them the per-block expert
+// counts live in this fixed device array instead of a caller workspace.
+// Every GPU that loads the library holds the array until the process exits.
+// ---------------------------------------------------------------------------
+constexpr int kSortStaticCounts = 1 << 16;  // int32 entries: 256 KB per device
+static __device__ __align__(256) int32_t g_sort_static_counts[kSortStaticCounts];
+
+namespace {
+// Device address of the array for the current device, resolved on the first
+// call made with that device current (the host-side symbol is only a stand-in
+// and must never be passed to a kernel).
+int32_t* sort_static_scratch(cudaError_t* status) {
+  static std::mutex mu;
+  static int32_t* ptrs[128] = {};
+  int dev = 0;
+  *status = cudaGetDevice(&dev);
+  if (*status != cudaSuccess) return nullptr;
+  if (dev < 0 || dev >= 128) {
+    *status = cudaErrorInvalidDevice;
+    return nullptr;
+  }
+  std::lock_guard<std::mutex> lock(mu);
+  if (ptrs[dev] == nullptr) {
+    int32_t* p = nullptr;
+    *status = cudaGetSymbolAddress((void**)&p, g_sort_static_counts);
+    if (*status != cudaSuccess) return nullptr;
+    ptrs[dev] = p;
+  }
+  return ptrs[dev];
+}
+}  // namespace
+
 }  // namespace smoe
+
+extern "C" int smoe_sort_static(const int32_t* topk_idx, int T, int k, int E,
+                                int32_t* sorted_slot, int32_t* expert_offsets, void* stream) {
+  using namespace smoe;
+  if (T < 0 || k <= 0 || E <= 0 || E > kSortMaxE)
+    return api_fail(SMOE_ERR_INVALID_ARG, "bad sizes (E <= %d)", kSortMaxE);
+  if (!expert_offsets) return api_fail(SMOE_ERR_INVALID_ARG, "expert_offsets is NULL");
+  const size_t need = sort_workspace_bytes(T, k, E);
+  if (need > sizeof(g_sort_static_counts))
+    return api_fail(SMOE_ERR_INVALID_ARG,
+                    "smoe_sort_static: %zu bytes of counts needed (ceil(T*k/%d) * E * 4) but the "
+                    "static scratch holds %zu; use smoe_sort with a workspace",
+                    need, kSortChunk, sizeof(g_sort_static_counts));
+  cudaStream_t s = (cudaStream_t)stream;
+  if (T == 0) {
+    const cudaError_t e = cudaMemsetAsync(expert_offsets, 0, (size_t)(E + 1) * sizeof(int32_t), s);
+    return e == cudaSuccess ? SMOE_OK
+                            : api_fail(SMOE_ERR_CUDA, "smoe_sort_static: %s", cudaGetErrorString(e));
+  }
+  if (!topk_idx || !sorted_slot) return api_fail(SMOE_ERR_INVALID_ARG, "topk_idx/sorted_slot is NULL");
+  cudaError_t st;
+  int32_t* scratch = sort_static_scratch(&st);
+  if (!scratch) return api_fail(SMOE_ERR_CUDA, "smoe_sort_static scratch: %s", cudaGetErrorString(st));
+  unsigned* err = api_error_word(&st);
+  if (!err) return api_fail(SMOE_ERR_CUDA, "smoe_sort_static error word: %s", cudaGetErrorString(st));
+  // the counts are fully rewritten by every call, so nothing needs clearing first
+  st = launch_sort(topk_idx, T, k, E, sorted_slot, expert_offsets, scratch, err, s);
+  return st == cudaSuccess ? SMOE_OK
+                           : api_fail(SMOE_ERR_CUDA, "smoe_sort_static: %s", cudaGetErrorString(st));
+}
