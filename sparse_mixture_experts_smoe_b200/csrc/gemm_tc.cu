@@ -47,7 +47,6 @@ namespace {
 constexpr int BM = 128;           // rows per tile (MMA M)
 constexpr int BK = 64;            // K per stage: one 128-byte swizzle row of bf16
 constexpr int BN = 256;           // MMA N
-constexpr int STAGES = 4;
 constexpr int kThreads = 384;        // 12 warps
 constexpr int kGatherWarp0 = 8;       // warps 8-11 gather scattered rows
 constexpr int kGatherThreads = 128;
@@ -215,6 +214,27 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int m, int n, int a_mn_major, 
          ((uint32_t)b_mn_major << 16) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(m >> 4) << 24);
 }
 
+// Activation arithmetic of the bf16 epilogues: one sigmoid per element via the
+// fast exponential and division, tanh from the hardware approximation.  Their
+// relative errors (~1e-6 and ~5e-4) sit far below bf16 rounding (3.9e-3) of the
+// stored results.
+__device__ __forceinline__ float fast_sigmoid(float z) { return __fdividef(1.0f, 1.0f + __expf(-z)); }
+__device__ __forceinline__ float fast_tanh(float x) {
+  float y;
+  asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+__device__ __forceinline__ float fast_gelu(float h) {
+  const float u = 0.7978845608028654f * fmaf(0.044715f * h, h * h, h);
+  return 0.5f * h * (1.0f + fast_tanh(u));
+}
+__device__ __forceinline__ float fast_gelu_grad(float h) {
+  const float u = 0.7978845608028654f * fmaf(0.044715f * h, h * h, h);
+  const float th = fast_tanh(u);
+  const float du = 0.7978845608028654f * fmaf(3.0f * 0.044715f, h * h, 1.0f);
+  return 0.5f * (1.0f + th) + 0.5f * h * (1.0f - th * th) * du;
+}
+
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
   return (uint8_t*)(((uintptr_t)p + 1023) & ~(uintptr_t)1023);
 }
@@ -243,23 +263,36 @@ __device__ __forceinline__ void unpack8(uint4 u, float* v) {
 }
 
 // ---------------------------------------------------------------------------
-// Shared state and tile list
+// Shared state, stage rings and the tile list
 // ---------------------------------------------------------------------------
-constexpr int IDX_STAGES = 8;  // slot-index ring of the dW gathers (stages ahead)
+// The A and B operands have separate stage rings: a gathered operand (long
+// cp.async latency) gets 6 stages of 16 KB while the TMA-fed one gets 3 of 32 KB;
+// kernels fed only by TMA use 4 + 4.  Either way the rings fill kRingBytes.
+constexpr int kMaxStages = 8;
+constexpr int IDX_STAGES = 8;            // slot-index ring of the dW gathers
+constexpr int kRingBytes = 192 * 1024;
 
 struct SharedCtl {
-  uint64_t full[STAGES];
-  uint64_t empty[STAGES];
-  uint64_t tfull[2];
-  uint64_t tempty[2];
+  uint64_t fullA[kMaxStages], emptyA[kMaxStages];
+  uint64_t fullB[kMaxStages], emptyB[kMaxStages];
+  uint64_t tfull[2], tempty[2];
   uint64_t ifull[IDX_STAGES];   // index ring: written by warp 2
   uint64_t iempty[IDX_STAGES];  // index ring: released by the 4 gather warps
-  int idx[IDX_STAGES][BK];      // slot of each row of a dW stage, -1 past the slice
+  int idx[IDX_STAGES][2][BK];   // source row per operand (A, B) of each stage row, -1 = zero
   uint32_t tmem_base;
   int abort_flag;
   int total_mtiles;
   int prefix[kMaxE + 1];  // M-tile prefix per expert
   int off[kMaxE + 1];     // expert offsets
+};
+
+// Position in a ring of n stages and the parity of the current lap.
+struct Ring {
+  int s = 0;
+  uint32_t ph = 0;
+  __device__ __forceinline__ void next(int n) {
+    if (++s == n) { s = 0; ph ^= 1; }
+  }
 };
 
 struct Tile {
@@ -285,13 +318,20 @@ __device__ __forceinline__ Tile map_tile(const SharedCtl& c, int E, int nN, int 
 }
 
 // Setup common to both kernels: barriers, tensor memory, offsets (validated).
+// a_arrivals / b_arrivals: producer arrivals per full stage (1 for TMA, the
+// gather threads' cp.async arrivals otherwise).
+template <int SA, int SB>
 __device__ __forceinline__ void setup(SharedCtl& c, const int32_t* offsets, int E, int num_rows,
-                                      unsigned* err, bool gather) {
+                                      unsigned* err, uint32_t a_arrivals, uint32_t b_arrivals) {
   const int warp = threadIdx.x >> 5;
   if (threadIdx.x == 0) {
-    for (int s = 0; s < STAGES; ++s) {
-      mbar_init(&c.full[s], 1 + (gather ? kGatherThreads : 0));
-      mbar_init(&c.empty[s], 1);
+    for (int s = 0; s < SA; ++s) {
+      mbar_init(&c.fullA[s], a_arrivals);
+      mbar_init(&c.emptyA[s], 1);
+    }
+    for (int s = 0; s < SB; ++s) {
+      mbar_init(&c.fullB[s], b_arrivals);
+      mbar_init(&c.emptyB[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&c.tfull[b], 1);
@@ -340,14 +380,19 @@ template <bool A_GATHER, bool B_KMAJOR, bool SWIGLU_FWD>
 __global__ void __launch_bounds__(kThreads, 1)
 grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
                        const __grid_constant__ CUtensorMap tmB, const GroupedGemm g, int nN) {
+  // One ring of STAGES stages holds A and B together (fullA/emptyA guard a whole
+  // stage): measured faster here than separate rings, whose second wait and
+  // commit per stage cost more than their extra depth returned.
+  constexpr int STAGES = 4;
+  static_assert(STAGES * (A_BYTES + B_BYTES) <= kRingBytes, "stage ring exceeds its budget");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
   uint8_t* sA = smem;
   uint8_t* sB = smem + STAGES * A_BYTES;
-  SharedCtl& c = *reinterpret_cast<SharedCtl*>(sB + STAGES * B_BYTES);
+  SharedCtl& c = *reinterpret_cast<SharedCtl*>(smem + kRingBytes);
   volatile int* abort_flag = &c.abort_flag;
 
-  setup(c, g.offsets, g.E, g.num_rows, g.err, A_GATHER);
+  setup<STAGES, 0>(c, g.offsets, g.E, g.num_rows, g.err, 1 + (A_GATHER ? kGatherThreads : 0), 1);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int total = c.total_mtiles * nN;
   const int nK = cdiv(g.K, BK);
@@ -355,19 +400,18 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
 
   if (warp == 0) {
     // ---------------- TMA producer (weights; A too when grouped) ----------------
-    int stage = 0;
-    uint32_t phase = 0;
-    for (int L = blockIdx.x; L < total; L += gridDim.x) {
-      const Tile t = map_tile(c, g.E, nN, L);
-      for (int kb = 0; kb < nK; ++kb) {
-        if (!mbar_wait(&c.empty[stage], phase ^ 1, abort_flag, g.err)) goto producer_done;
-        if (lane == 0) {
-          uint8_t* a_dst = sA + stage * A_BYTES;
-          uint8_t* b_dst = sB + stage * B_BYTES;
-          mbar_expect_tx(&c.full[stage], B_BYTES + (A_GATHER ? 0 : A_BYTES));
-          if (!A_GATHER) tma_load_2d(a_dst, &tmA, &c.full[stage], kb * BK, t.row0);
+    if (lane == 0) {
+      Ring r;
+      bool run = true;
+      for (int L = blockIdx.x; run && L < total; L += gridDim.x) {
+        const Tile t = map_tile(c, g.E, nN, L);
+        for (int kb = 0; kb < nK; ++kb) {
+          if (!mbar_wait(&c.emptyA[r.s], r.ph ^ 1, abort_flag, g.err)) { run = false; break; }
+          uint8_t* b_dst = sB + r.s * B_BYTES;
+          mbar_expect_tx(&c.fullA[r.s], B_BYTES + (A_GATHER ? 0 : A_BYTES));
+          if (!A_GATHER) tma_load_2d(sA + r.s * A_BYTES, &tmA, &c.fullA[r.s], kb * BK, t.row0);
           if (B_KMAJOR) {
-            tma_load_3d(b_dst, &tmB, &c.full[stage], kb * BK, t.nb * BN, t.e);
+            tma_load_3d(b_dst, &tmB, &c.fullA[r.s], kb * BK, t.nb * BN, t.e);
           } else {
 #pragma unroll
             for (int q = 0; q < BN / 64; ++q) {
@@ -376,15 +420,14 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
                 col = (q < BN / 128) ? t.nb * BNo + 64 * q : g.n_out + t.nb * BNo + 64 * (q - BN / 128);
               else
                 col = t.nb * BN + 64 * q;
-              tma_load_3d(b_dst + q * (64 * BK * 2), &tmB, &c.full[stage], col, kb * BK, t.e);
+              tma_load_3d(b_dst + q * (64 * BK * 2), &tmB, &c.fullA[r.s], col, kb * BK, t.e);
             }
           }
+          r.next(STAGES);
         }
-        __syncwarp();
-        if (++stage == STAGES) { stage = 0; phase ^= 1; }
       }
     }
-  producer_done:;
+    __syncwarp();
   } else if (A_GATHER && warp >= kGatherWarp0) {
     // ---------------- row gather of the scattered A operand ----------------
     // thread t copies 16-byte chunk (t % 8) of tile rows t/8 + 16 j, j = 0..7,
@@ -393,9 +436,9 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
     const int t = threadIdx.x - kGatherWarp0 * 32;
     const int cc = t & 7, r0 = t >> 3;
     const bf16* A = reinterpret_cast<const bf16*>(g.a);
-    int stage = 0;
-    uint32_t phase = 0;
-    for (int L = blockIdx.x; L < total; L += gridDim.x) {
+    Ring r;
+    bool run = true;
+    for (int L = blockIdx.x; run && L < total; L += gridDim.x) {
       const Tile tl = map_tile(c, g.E, nN, L);
       const bf16* src[8];
       uint32_t ok_rows = 0;
@@ -415,25 +458,23 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
         }
       }
       for (int kb = 0; kb < nK; ++kb) {
-        if (!mbar_wait(&c.empty[stage], phase ^ 1, abort_flag, g.err)) goto gather_done;
-        const uint32_t a_dst = smem_u32(sA + stage * A_BYTES);
+        if (!mbar_wait(&c.emptyA[r.s], r.ph ^ 1, abort_flag, g.err)) { run = false; break; }
+        const uint32_t a_dst = smem_u32(sA + r.s * A_BYTES);
         const bool col_ok = kb * BK + 8 * cc < g.K;
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
           const bool ok = col_ok && ((ok_rows >> j) & 1u);
           cp_async16(a_dst + sw128_off(r0 + 16 * j, cc), ok ? src[j] + kb * BK : A, ok ? 16u : 0u);
         }
-        cp_async_arrive(&c.full[stage]);
-        if (++stage == STAGES) { stage = 0; phase ^= 1; }
+        cp_async_arrive(&c.fullA[r.s]);
+        r.next(STAGES);
       }
     }
-  gather_done:;
   } else if (warp == 1) {
     // ---------------- MMA issuer ----------------
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_bf16(BM, BN, 0, B_KMAJOR ? 0 : 1);
-      int stage = 0;
-      uint32_t phase = 0;
+      Ring r;
       int it = 0;
       for (int L = blockIdx.x; L < total; L += gridDim.x, ++it) {
         const int buf = it & 1;
@@ -443,19 +484,19 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
         const uint32_t d_tmem = c.tmem_base + buf * BN;
         bool ok = true;
         for (int kb = 0; kb < nK; ++kb) {
-          if (!mbar_wait(&c.full[stage], phase, abort_flag, g.err)) { ok = false; break; }
+          if (!mbar_wait(&c.fullA[r.s], r.ph, abort_flag, g.err)) { ok = false; break; }
           tc_fence_after();
           if (A_GATHER) fence_proxy_async();  // rows written by cp.async, read by the tensor core
-          const uint32_t a_addr = smem_u32(sA + stage * A_BYTES);
-          const uint32_t b_addr = smem_u32(sB + stage * B_BYTES);
+          const uint32_t a_addr = smem_u32(sA + r.s * A_BYTES);
+          const uint32_t b_addr = smem_u32(sB + r.s * B_BYTES);
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk) {
             const uint64_t ad = desc_kmajor(a_addr + kk * 32);
             const uint64_t bd = B_KMAJOR ? desc_kmajor(b_addr + kk * 32) : desc_mnmajor(b_addr + kk * 2048);
             umma_bf16(d_tmem, ad, bd, idesc, (kb | kk) != 0);
           }
-          umma_commit(&c.empty[stage]);
-          if (++stage == STAGES) { stage = 0; phase ^= 1; }
+          umma_commit(&c.emptyA[r.s]);
+          r.next(STAGES);
         }
         if (!ok) break;
         umma_commit(&c.tfull[buf]);
@@ -526,8 +567,9 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
 #pragma unroll
               for (int j = 0; j < 8; ++j) {
                 const float da = gate * vv[j];
-                dh[j] = da * hu[j] * silu_grad_f(hg[j]);
-                du[j] = da * silu_f(hg[j]);
+                const float sg = fast_sigmoid(hg[j]);
+                dh[j] = da * hu[j] * sg * fmaf(hg[j], 1.0f - sg, 1.0f);
+                du[j] = da * hg[j] * sg;
               }
               bf16* O = reinterpret_cast<bf16*>(g.out) + (size_t)orow * g.ldo;
               *reinterpret_cast<uint4*>(O + n) = pack8(dh);
@@ -536,7 +578,7 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
               if (g.act == SMOE_ACT_GELU_TANH) {
                 unpack8(rg[j8], hg);
 #pragma unroll
-                for (int j = 0; j < 8; ++j) dh[j] = gate * vv[j] * gelu_tanh_grad_f(hg[j]);
+                for (int j = 0; j < 8; ++j) dh[j] = gate * vv[j] * fast_gelu_grad(hg[j]);
               } else {
 #pragma unroll
                 for (int j = 0; j < 8; ++j) dh[j] = gate * vv[j];
@@ -576,13 +618,13 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
             if (SWIGLU_FWD) {
               float* uu = u + 8 * j8;
 #pragma unroll
-              for (int j = 0; j < 8; ++j) a8[j] = silu_f(vv[j]) * uu[j];
+              for (int j = 0; j < 8; ++j) a8[j] = vv[j] * fast_sigmoid(vv[j]) * uu[j];
               bf16* H = reinterpret_cast<bf16*>(g.out) + (size_t)orow * g.ldo;
               *reinterpret_cast<uint4*>(H + n) = pack8(vv);
               *reinterpret_cast<uint4*>(H + g.n_out + n) = pack8(uu);
             } else {
 #pragma unroll
-              for (int j = 0; j < 8; ++j) a8[j] = gelu_tanh_f(vv[j]);
+              for (int j = 0; j < 8; ++j) a8[j] = fast_gelu(vv[j]);
               *reinterpret_cast<uint4*>(reinterpret_cast<bf16*>(g.out) + (size_t)orow * g.ldo + n) = pack8(vv);
             }
             *reinterpret_cast<uint4*>(reinterpret_cast<bf16*>(g.out2) + (size_t)orow * g.ldo2 + n) = pack8(a8);
@@ -604,52 +646,67 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
 // ---------------------------------------------------------------------------
 // Gather of NS 64-column slabs of BK scattered rows (the MN-major operand of the
 // dW product) with cp.async: thread t copies chunk (t % 8NS) of rows
-// t / 8NS + (128 / 8NS) j.  The slot indices come from a shared-memory ring that
-// an index warp fills up to IDX_STAGES stages ahead, so no global-load latency
-// sits between a free stage and its copies; rows past the slice and columns past
-// `ncols` are zero-filled.
+// t / 8NS + (128 / 8NS) j.  The source rows come from a shared-memory ring that
+// the index warp fills (slot -> row, range-checked) ahead of time; destination
+// offsets are fixed per thread, so a copy costs a shared load, one address
+// computation and the cp.async.  Rows marked -1 and columns past `ncols` are
+// zero-filled.
 template <int NS>
 struct SlabGather {
   static constexpr int CPR = 8 * NS;
   static constexpr int RSTEP = kGatherThreads / CPR;
   static constexpr int NR = BK / RSTEP;
-  int p[NR];  // slot of each of this thread's rows, -1 past the slice
+  int row0;        // first row of this thread
+  uint32_t off0;   // shared-memory offset of (row0, chunk) inside a stage
+  int chunk_col;   // column of this thread's chunk inside the tile
 
-  __device__ __forceinline__ void load(const int* ring_stage, int t) {
-#pragma unroll
-    for (int j = 0; j < NR; ++j) p[j] = ring_stage[t / CPR + RSTEP * j];
-  }
-  __device__ __forceinline__ void issue(uint32_t dst, const bf16* base, int ld, int col0, int ncols,
-                                        int fan_out, int fan_shift, int src_rows, int t,
-                                        unsigned* err) const {
+  __device__ __forceinline__ void init(int t) {
     const int cg = t % CPR, slab = cg >> 3, cc = cg & 7;
-    const int col = col0 + 64 * slab + 8 * cc;
+    row0 = t / CPR;
+    off0 = slab * 8192 + sw128_off(row0, cc);
+    chunk_col = 64 * slab + 8 * cc;
+  }
+  // rows row0 + RSTEP*j keep the same (row & 7) pattern only when RSTEP % 8 == 0;
+  // otherwise the swizzled offset is recomputed per row.
+  __device__ __forceinline__ uint32_t dst_off(int j, int t) const {
+    if (RSTEP % 8 == 0) return off0 + (uint32_t)(RSTEP * j * 128);
+    const int cg = t % CPR, slab = cg >> 3, cc = cg & 7;
+    return slab * 8192 + sw128_off(row0 + RSTEP * j, cc);
+  }
+  __device__ __forceinline__ void issue(uint32_t dst, const int* rows, const bf16* base, int ld,
+                                        int col0, int ncols, int t) const {
+    const int col = col0 + chunk_col;
     const bool col_ok = col < ncols;
+    const bf16* cbase = base + col;
 #pragma unroll
     for (int j = 0; j < NR; ++j) {
-      const int row = t / CPR + RSTEP * j;
-      const int sr = p[j] < 0 ? -1 : (fan_shift >= 0 ? (p[j] >> fan_shift) : p[j] / fan_out);
-      const bool in_range = sr < src_rows;
-      if (p[j] >= 0 && !in_range) report_error(err, ERRBIT_DATA);
-      const bool ok = col_ok && p[j] >= 0 && in_range;
-      cp_async16(dst + slab * 8192 + sw128_off(row, cc), ok ? base + (size_t)sr * ld + col : base,
-                 ok ? 16u : 0u);
+      const int sr = rows[row0 + RSTEP * j];
+      const bool ok = col_ok && sr >= 0;
+      cp_async16(dst + dst_off(j, t), ok ? cbase + (size_t)sr * ld : base, ok ? 16u : 0u);
     }
   }
 };
 
-template <bool A_GATHER, bool B_GATHER>
+// dW[e] tile (e, m-block, n-block) of D[m, n] = sum over the expert's rows r of
+// A[r, m] * B[r, n].  TRANS_OUT stores D transposed (the host swapped the
+// operands so that a gathered operand sits on the 128-wide A side); the store
+// is then coalesced across the warp (consecutive m, one n at a time).
+template <bool A_GATHER, bool B_GATHER, bool TRANS_OUT>
 __global__ void __launch_bounds__(kThreads, 1)
 dw_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                   const DwGemm g, int nM, int nN) {
+  constexpr bool kOneGather = A_GATHER && !B_GATHER;
+  constexpr int SA = kOneGather ? 6 : 4, SB = kOneGather ? 3 : 4;
+  static_assert(SA * A_BYTES + SB * B_BYTES <= kRingBytes, "stage rings exceed their budget");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
   uint8_t* sA = smem;
-  uint8_t* sB = smem + STAGES * A_BYTES;
-  SharedCtl& c = *reinterpret_cast<SharedCtl*>(sB + STAGES * B_BYTES);
+  uint8_t* sB = smem + SA * A_BYTES;
+  SharedCtl& c = *reinterpret_cast<SharedCtl*>(smem + kRingBytes);
   volatile int* abort_flag = &c.abort_flag;
 
-  setup(c, g.offsets, g.E, g.num_rows, g.err, A_GATHER || B_GATHER);
+  setup<SA, SB>(c, g.offsets, g.E, g.num_rows, g.err, A_GATHER ? kGatherThreads : 1,
+                B_GATHER ? kGatherThreads : 1);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const bool offsets_ok = c.total_mtiles > 0 || g.num_rows == 0;
   const int total = offsets_ok ? g.E * nM * nN : 0;
@@ -663,90 +720,120 @@ dw_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
 
   if (warp == 0) {
     // ---------------- TMA producer of the grouped operand(s) ----------------
-    int stage = 0;
-    uint32_t phase = 0;
-    for (int L = blockIdx.x; L < total; L += gridDim.x) {
-      int e, mb, nb;
-      coords(L, e, mb, nb);
-      const int r_begin = c.off[e], r_end = c.off[e + 1];
-      const int nK = cdiv(r_end - r_begin, BK);
-      for (int kb = 0; kb < nK; ++kb) {
-        if (!mbar_wait(&c.empty[stage], phase ^ 1, abort_flag, g.err)) goto producer_done;
-        if (lane == 0) {
-          uint8_t* a_dst = sA + stage * A_BYTES;
-          uint8_t* b_dst = sB + stage * B_BYTES;
+    if (lane == 0 && !(A_GATHER && B_GATHER)) {
+      Ring ra, rb;
+      bool run = true;
+      for (int L = blockIdx.x; run && L < total; L += gridDim.x) {
+        int e, mb, nb;
+        coords(L, e, mb, nb);
+        const int r_begin = c.off[e], r_end = c.off[e + 1];
+        const int nK = cdiv(r_end - r_begin, BK);
+        for (int kb = 0; kb < nK; ++kb) {
           const int rk = r_begin + kb * BK;
-          mbar_expect_tx(&c.full[stage], (A_GATHER ? 0 : A_BYTES) + (B_GATHER ? 0 : B_BYTES));
           if (!A_GATHER) {  // 64 rows x 128 M-columns: two 64-column slabs of 8 KB
-            tma_load_2d(a_dst, &tmA, &c.full[stage], mb * BM, rk);
-            tma_load_2d(a_dst + 8192, &tmA, &c.full[stage], mb * BM + 64, rk);
+            if (!mbar_wait(&c.emptyA[ra.s], ra.ph ^ 1, abort_flag, g.err)) { run = false; break; }
+            uint8_t* a_dst = sA + ra.s * A_BYTES;
+            mbar_expect_tx(&c.fullA[ra.s], A_BYTES);
+            tma_load_2d(a_dst, &tmA, &c.fullA[ra.s], mb * BM, rk);
+            tma_load_2d(a_dst + 8192, &tmA, &c.fullA[ra.s], mb * BM + 64, rk);
+            ra.next(SA);
           }
           if (!B_GATHER) {  // 64 rows x 256 N-columns: four slabs
+            if (!mbar_wait(&c.emptyB[rb.s], rb.ph ^ 1, abort_flag, g.err)) { run = false; break; }
+            uint8_t* b_dst = sB + rb.s * B_BYTES;
+            mbar_expect_tx(&c.fullB[rb.s], B_BYTES);
 #pragma unroll
             for (int slab = 0; slab < 4; ++slab)
-              tma_load_2d(b_dst + slab * 8192, &tmB, &c.full[stage], nb * BN + 64 * slab, rk);
+              tma_load_2d(b_dst + slab * 8192, &tmB, &c.fullB[rb.s], nb * BN + 64 * slab, rk);
+            rb.next(SB);
           }
         }
-        __syncwarp();
-        if (++stage == STAGES) { stage = 0; phase ^= 1; }
       }
     }
-  producer_done:;
+    __syncwarp();
   } else if ((A_GATHER || B_GATHER) && warp == 2) {
-    // ---------------- slot-index producer for the gathers ----------------
-    int istage = 0;
-    uint32_t iphase = 0;
-    for (int L = blockIdx.x; L < total; L += gridDim.x) {
+    // ---------------- source-row producer for the gathers ----------------
+    // Loads for kIdxBatch stages are issued together before any is written, so
+    // one global-load latency is paid per batch instead of per stage.  Each slot
+    // p becomes the source row p / fan_out (a shift for a power of two), checked
+    // against the operand's row count; -1 marks a zero row.
+    constexpr int kIdxBatch = IDX_STAGES / 2;
+    const int a_shift = (g.a_fan_out & (g.a_fan_out - 1)) == 0 ? __ffs(g.a_fan_out) - 1 : -1;
+    const int b_shift = (g.b_fan_out & (g.b_fan_out - 1)) == 0 ? __ffs(g.b_fan_out) - 1 : -1;
+    auto src_of = [&](int p, int shift, int fan, int rows) -> int {
+      if (p < 0) return -1;
+      const int r = shift >= 0 ? (p >> shift) : p / fan;
+      if (r >= rows) {
+        report_error(g.err, ERRBIT_DATA);
+        return -1;
+      }
+      return r;
+    };
+    Ring ri;
+    bool run = true;
+    for (int L = blockIdx.x; run && L < total; L += gridDim.x) {
       int e, mb, nb;
       coords(L, e, mb, nb);
       const int r_begin = c.off[e], r_end = c.off[e + 1];
       const int nK = cdiv(r_end - r_begin, BK);
-      for (int kb = 0; kb < nK; ++kb) {
-        if (!mbar_wait(&c.iempty[istage], iphase ^ 1, abort_flag, g.err)) goto index_done;
-        const int rk = r_begin + kb * BK;
+      for (int kb0 = 0; run && kb0 < nK; kb0 += kIdxBatch) {
+        int v[kIdxBatch][BK / 32];
 #pragma unroll
-        for (int q = 0; q < BK / 32; ++q) {
-          const int row = lane + 32 * q;
-          c.idx[istage][row] = rk + row < r_end ? __ldg(g.sorted_slot + rk + row) : -1;
+        for (int b = 0; b < kIdxBatch; ++b)
+#pragma unroll
+          for (int q = 0; q < BK / 32; ++q) {
+            const int r = r_begin + (kb0 + b) * BK + lane + 32 * q;
+            v[b][q] = (kb0 + b < nK && r < r_end) ? __ldg(g.sorted_slot + r) : -1;
+          }
+#pragma unroll
+        for (int b = 0; b < kIdxBatch; ++b) {
+          if (kb0 + b >= nK) break;
+          if (!mbar_wait(&c.iempty[ri.s], ri.ph ^ 1, abort_flag, g.err)) { run = false; break; }
+#pragma unroll
+          for (int q = 0; q < BK / 32; ++q) {
+            if (A_GATHER) c.idx[ri.s][0][lane + 32 * q] = src_of(v[b][q], a_shift, g.a_fan_out, g.a_rows);
+            if (B_GATHER) c.idx[ri.s][1][lane + 32 * q] = src_of(v[b][q], b_shift, g.b_fan_out, g.b_rows);
+          }
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&c.ifull[ri.s]);
+          ri.next(IDX_STAGES);
         }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&c.ifull[istage]);
-        if (++istage == IDX_STAGES) { istage = 0; iphase ^= 1; }
       }
     }
-  index_done:;
   } else if ((A_GATHER || B_GATHER) && warp >= kGatherWarp0) {
     // ---------------- cp.async gather of the scattered operand(s) ----------------
     const int t = threadIdx.x - kGatherWarp0 * 32;
-    const int a_shift = (g.a_fan_out & (g.a_fan_out - 1)) == 0 ? __ffs(g.a_fan_out) - 1 : -1;
-    const int b_shift = (g.b_fan_out & (g.b_fan_out - 1)) == 0 ? __ffs(g.b_fan_out) - 1 : -1;
     SlabGather<2> ga;
     SlabGather<4> gb;
-    int stage = 0, istage = 0;
-    uint32_t phase = 0, iphase = 0;
-    for (int L = blockIdx.x; L < total; L += gridDim.x) {
+    ga.init(t);
+    gb.init(t);
+    Ring ra, rb, ri;
+    bool run = true;
+    for (int L = blockIdx.x; run && L < total; L += gridDim.x) {
       int e, mb, nb;
       coords(L, e, mb, nb);
       const int nK = cdiv(c.off[e + 1] - c.off[e], BK);
       for (int kb = 0; kb < nK; ++kb) {
-        if (!mbar_wait(&c.ifull[istage], iphase, abort_flag, g.err)) goto gather_done;
-        if (A_GATHER) ga.load(c.idx[istage], t);
-        if (B_GATHER) gb.load(c.idx[istage], t);
+        if (!mbar_wait(&c.ifull[ri.s], ri.ph, abort_flag, g.err)) { run = false; break; }
+        if (A_GATHER) {
+          if (!mbar_wait(&c.emptyA[ra.s], ra.ph ^ 1, abort_flag, g.err)) { run = false; break; }
+          ga.issue(smem_u32(sA + ra.s * A_BYTES), c.idx[ri.s][0], reinterpret_cast<const bf16*>(g.a),
+                   g.lda, mb * BM, g.M, t);
+          cp_async_arrive(&c.fullA[ra.s]);
+          ra.next(SA);
+        }
+        if (B_GATHER) {
+          if (!mbar_wait(&c.emptyB[rb.s], rb.ph ^ 1, abort_flag, g.err)) { run = false; break; }
+          gb.issue(smem_u32(sB + rb.s * B_BYTES), c.idx[ri.s][1], reinterpret_cast<const bf16*>(g.b),
+                   g.ldb, nb * BN, g.N, t);
+          cp_async_arrive(&c.fullB[rb.s]);
+          rb.next(SB);
+        }
         __syncwarp();
-        if (lane == 0) mbar_arrive(&c.iempty[istage]);
-        if (++istage == IDX_STAGES) { istage = 0; iphase ^= 1; }
-        if (!mbar_wait(&c.empty[stage], phase ^ 1, abort_flag, g.err)) goto gather_done;
-        if (A_GATHER)
-          ga.issue(smem_u32(sA + stage * A_BYTES), reinterpret_cast<const bf16*>(g.a), g.lda,
-                   mb * BM, g.M, g.a_fan_out, a_shift, g.a_rows, t, g.err);
-        if (B_GATHER)
-          gb.issue(smem_u32(sB + stage * B_BYTES), reinterpret_cast<const bf16*>(g.b), g.ldb,
-                   nb * BN, g.N, g.b_fan_out, b_shift, g.b_rows, t, g.err);
-        cp_async_arrive(&c.full[stage]);
-        if (++stage == STAGES) { stage = 0; phase ^= 1; }
+        if (lane == 0) mbar_arrive(&c.iempty[ri.s]);  // this warp is done with the rows
+        ri.next(IDX_STAGES);
       }
     }
-  gather_done:;
   } else if (warp == 1) {
     // ---------------- MMA issuer ----------------
     // With a gathered operand its rows past the slice are zero-filled, so the
@@ -756,8 +843,7 @@ dw_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
     constexpr bool kGather = A_GATHER || B_GATHER;
     constexpr uint32_t idesc = idesc_bf16(BM, BN, 1, 1);
     if (!kGather || lane == 0) {
-      int stage = 0;
-      uint32_t phase = 0;
+      Ring ra, rb;
       int it = 0;
       for (int L = blockIdx.x; L < total; L += gridDim.x, ++it) {
         int e, mb, nb;
@@ -771,15 +857,16 @@ dw_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
         const uint32_t d_tmem = c.tmem_base + buf * BN;
         bool ok = true;
         for (int kb = 0; kb < nK; ++kb) {
-          if (!mbar_wait(&c.full[stage], phase, abort_flag, g.err)) { ok = false; break; }
+          if (!mbar_wait(&c.fullA[ra.s], ra.ph, abort_flag, g.err) ||
+              !mbar_wait(&c.fullB[rb.s], rb.ph, abort_flag, g.err)) { ok = false; break; }
           tc_fence_after();
           if (kGather) {
             fence_proxy_async();  // cp.async rows -> tensor core
           } else {
             const int valid = min(BK, r_end - (r_begin + kb * BK));
             if (valid < BK) {  // rows past the slice end hold other rows' data
-              uint8_t* a_t = sA + stage * A_BYTES;
-              uint8_t* b_t = sB + stage * B_BYTES;
+              uint8_t* a_t = sA + ra.s * A_BYTES;
+              uint8_t* b_t = sB + rb.s * B_BYTES;
               const int nz = (BK - valid) * 8;  // 16-byte chunks per slab
               for (int z = lane; z < nz * 6; z += 32) {
                 const int slab = z / nz, w = z % nz;
@@ -791,16 +878,18 @@ dw_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
             __syncwarp();
           }
           if (lane == 0) {
-            const uint32_t a_addr = smem_u32(sA + stage * A_BYTES);
-            const uint32_t b_addr = smem_u32(sB + stage * B_BYTES);
+            const uint32_t a_addr = smem_u32(sA + ra.s * A_BYTES);
+            const uint32_t b_addr = smem_u32(sB + rb.s * B_BYTES);
 #pragma unroll
             for (int kk = 0; kk < BK / 16; ++kk)
               umma_bf16(d_tmem, desc_mnmajor(a_addr + kk * 2048), desc_mnmajor(b_addr + kk * 2048),
                         idesc, (kb | kk) != 0);
-            umma_commit(&c.empty[stage]);
+            umma_commit(&c.emptyA[ra.s]);
+            umma_commit(&c.emptyB[rb.s]);
           }
           if (!kGather) __syncwarp();
-          if (++stage == STAGES) { stage = 0; phase ^= 1; }
+          ra.next(SA);
+          rb.next(SB);
         }
         if (!ok) break;
         if (lane == 0) {
@@ -811,7 +900,8 @@ dw_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
       }
     }
     __syncwarp();
-  } else if (warp >= 4 && warp < 8) {  // warps 2-3 (and 8-11 without a gather) idle
+  } else if (warp >= 4 && warp < 8) {
+    // ---------------- epilogue: one accumulator row per thread ----------------
     const int q = warp - 4;
     const int r = q * 32 + lane;
     int it = 0;
@@ -825,7 +915,6 @@ dw_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
       tc_fence_after();
       const int m = mb * BM + r;
       const uint32_t trow = c.tmem_base + ((uint32_t)(q * 32) << 16) + buf * BN;
-      float* out = g.dw + ((size_t)e * g.M + m) * g.N;
 #pragma unroll 1
       for (int c0 = 0; c0 < BN; c0 += 32) {
         float v[32];
@@ -836,11 +925,22 @@ dw_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
           for (int j = 0; j < 32; ++j) v[j] = 0.0f;
         }
         if (m >= g.M) continue;
+        if (TRANS_OUT) {  // dW[e][n][m]: lanes hold consecutive m -> 128-byte lines
+          float* out = g.dw + (size_t)e * g.N * g.M + m;
 #pragma unroll
-        for (int j4 = 0; j4 < 8; ++j4) {
-          const int n = nb * BN + c0 + 4 * j4;
-          if (n >= g.N) break;
-          *reinterpret_cast<float4*>(out + n) = make_float4(v[4 * j4], v[4 * j4 + 1], v[4 * j4 + 2], v[4 * j4 + 3]);
+          for (int j = 0; j < 32; ++j) {
+            const int n = nb * BN + c0 + j;
+            if (n < g.N) out[(size_t)n * g.M] = v[j];
+          }
+        } else {
+          float* out = g.dw + ((size_t)e * g.M + m) * g.N;
+#pragma unroll
+          for (int j4 = 0; j4 < 8; ++j4) {
+            const int n = nb * BN + c0 + 4 * j4;
+            if (n >= g.N) break;
+            *reinterpret_cast<float4*>(out + n) =
+                make_float4(v[4 * j4], v[4 * j4 + 1], v[4 * j4 + 2], v[4 * j4 + 3]);
+          }
         }
       }
       tc_fence_before();
@@ -905,7 +1005,7 @@ int num_sms() {
   return n;
 }
 
-constexpr size_t kSmemBytes = 1024 + (size_t)STAGES * (A_BYTES + B_BYTES) + sizeof(SharedCtl);
+constexpr size_t kSmemBytes = 1024 + (size_t)kRingBytes + sizeof(SharedCtl);
 
 template <typename K>
 cudaError_t prep(K kern) {
@@ -922,10 +1022,10 @@ cudaError_t launch_g(const CUtensorMap& ta, const CUtensorMap& tb, const Grouped
   return cudaGetLastError();
 }
 
-template <bool AG, bool BG>
+template <bool AG, bool BG, bool TR>
 cudaError_t launch_d(const CUtensorMap& ta, const CUtensorMap& tb, const DwGemm& g, int nM, int nN,
                      int grid, cudaStream_t s) {
-  auto kern = dw_gemm_tc_kernel<AG, BG>;
+  auto kern = dw_gemm_tc_kernel<AG, BG, TR>;
   cudaError_t e = prep(kern);
   if (e != cudaSuccess) return e;
   kern<<<grid, kThreads, kSmemBytes, s>>>(ta, tb, g, nM, nN);
@@ -980,8 +1080,17 @@ cudaError_t launch_grouped_gemm_tc(const GroupedGemm& g, cudaStream_t s) {
                 : launch_g<false, false, false>(ta, tb, g, nN, grid, s);
 }
 
-cudaError_t launch_dw_gemm_tc(const DwGemm& g, cudaStream_t s) {
-  if (g.E > kMaxE) return cudaErrorInvalidValue;
+cudaError_t launch_dw_gemm_tc(const DwGemm& g_in, cudaStream_t s) {
+  if (g_in.E > kMaxE) return cudaErrorInvalidValue;
+  // Keep a single gathered operand on the A (128-wide, 16 KB per stage) side:
+  // compute dW^T and store it transposed.
+  DwGemm g = g_in;
+  const bool trans = g_in.b_mode == ROWS_GATHER && g_in.a_mode == ROWS_GROUPED;
+  if (trans) {
+    g.M = g_in.N; g.N = g_in.M;
+    g.a = g_in.b; g.lda = g_in.ldb; g.a_rows = g_in.b_rows; g.a_mode = g_in.b_mode; g.a_fan_out = g_in.b_fan_out;
+    g.b = g_in.a; g.ldb = g_in.lda; g.b_rows = g_in.a_rows; g.b_mode = g_in.a_mode; g.b_fan_out = g_in.a_fan_out;
+  }
   const int nM = cdiv(g.M, BM), nN = cdiv(g.N, BN);
   const bool ag = g.a_mode == ROWS_GATHER, bg = g.b_mode == ROWS_GATHER;
   CUtensorMap ta, tb;
@@ -991,10 +1100,11 @@ cudaError_t launch_dw_gemm_tc(const DwGemm& g, cudaStream_t s) {
   if (e != cudaSuccess) return e;
   const long long tiles = (long long)g.E * nM * nN;
   const int grid = (int)(tiles < num_sms() ? tiles : num_sms());
-  if (ag) return bg ? launch_d<true, true>(ta, tb, g, nM, nN, grid, s)
-                    : launch_d<true, false>(ta, tb, g, nM, nN, grid, s);
-  return bg ? launch_d<false, true>(ta, tb, g, nM, nN, grid, s)
-            : launch_d<false, false>(ta, tb, g, nM, nN, grid, s);
+  if (trans) return launch_d<true, false, true>(ta, tb, g, nM, nN, grid, s);
+  if (ag) return bg ? launch_d<true, true, false>(ta, tb, g, nM, nN, grid, s)
+                    : launch_d<true, false, false>(ta, tb, g, nM, nN, grid, s);
+  return bg ? launch_d<false, true, false>(ta, tb, g, nM, nN, grid, s)
+            : launch_d<false, false, false>(ta, tb, g, nM, nN, grid, s);
 }
 
 }  // namespace smoe

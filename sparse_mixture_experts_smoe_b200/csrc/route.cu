@@ -12,7 +12,10 @@
 //
 // Work split: a warp handles TM tokens; a block of 8 warps stages CH rows of W_r
 // in shared memory as fp32 with a row stride = 4 (mod 32) words, so the eight
-// lanes of a 128-bit shared load phase read eight different bank groups.
+// lanes of a 128-bit shared load phase read eight different bank groups, and the
+// block's CH-feature slice of x with 16-byte coalesced loads (lane L then reads
+// its features L, L+32, ... from shared memory; the accumulation order above is
+// unchanged).
 #include "common.cuh"
 
 namespace smoe {
@@ -31,12 +34,15 @@ route_kernel(const T* __restrict__ x, const T* __restrict__ w_r, const float* __
              int T_, int d, int E, int k, int32_t* __restrict__ idx, float* __restrict__ gates,
              unsigned* err) {
   constexpr int STRIDE = route_row_stride(EMAX);
+  constexpr int BT = kRouteWarps * TM;  // tokens per block
   extern __shared__ float4 smem_f4[];
   float* ws = reinterpret_cast<float*>(smem_f4);  // [CH][STRIDE]
+  float* xs = ws + CH * STRIDE;                   // [BT][CH]
 
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
-  const int t0 = (blockIdx.x * kRouteWarps + warp) * TM;
+  const int tb = blockIdx.x * BT;
+  const int t0 = tb + warp * TM;
 
   float acc[TM][EMAX];
 #pragma unroll
@@ -52,15 +58,42 @@ route_kernel(const T* __restrict__ x, const T* __restrict__ w_r, const float* __
       const int i = i0 + r;
       ws[r * STRIDE + e] = (i < d && e < E) ? to_f(w_r[(size_t)i * E + e]) : 0.0f;
     }
+    // stage x[tb : tb+BT, i0 : i0+CH] as fp32 with 8-element (16-byte bf16) loads
+    for (int q = threadIdx.x; q < BT * (CH / 8); q += blockDim.x) {
+      const int m = q / (CH / 8), c8 = (q % (CH / 8)) * 8;
+      const int t = tb + m, i = i0 + c8;
+      float v[8];
+      if (t < T_ && i < d) {  // d % 8 == 0, so the 8 features are all in range
+        const T* src = x + (size_t)t * d + i;
+        if (sizeof(T) == 2) {
+          const uint4 u = *reinterpret_cast<const uint4*>(src);
+          const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+          for (int h2 = 0; h2 < 4; ++h2) {
+            const float2 f = __bfloat1622float2(h[h2]);
+            v[2 * h2] = f.x;
+            v[2 * h2 + 1] = f.y;
+          }
+        } else {
+          const float4 a = *reinterpret_cast<const float4*>(src);
+          const float4 b = *reinterpret_cast<const float4*>(src + 4);
+          v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+          v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+        }
+      } else {
+#pragma unroll
+        for (int u = 0; u < 8; ++u) v[u] = 0.0f;
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) xs[m * CH + c8 + u] = v[u];
+    }
     __syncthreads();
-#pragma unroll 1
+#pragma unroll 2
     for (int r = lane; r < CH; r += 32) {
-      const int i = i0 + r;
-      if (i >= d) break;
+      if (i0 + r >= d) break;
       float xv[TM];
 #pragma unroll
-      for (int m = 0; m < TM; ++m)
-        xv[m] = (t0 + m < T_) ? to_f(x[(size_t)(t0 + m) * d + i]) : 0.0f;
+      for (int m = 0; m < TM; ++m) xv[m] = xs[(warp * TM + m) * CH + r];
       const float4* wrow = reinterpret_cast<const float4*>(ws + r * STRIDE);
 #pragma unroll
       for (int e4 = 0; e4 < EMAX / 4; ++e4) {
@@ -144,7 +177,7 @@ template <typename T, int EMAX, int TM>
 cudaError_t launch_route_t(const void* x, const void* w_r, const float* b_r, int T_, int d, int E,
                            int k, int32_t* idx, float* gates, unsigned* err, cudaStream_t s) {
   constexpr int CH = EMAX <= 64 ? 256 : 128;
-  const size_t smem = (size_t)CH * route_row_stride(EMAX) * sizeof(float);
+  const size_t smem = ((size_t)CH * route_row_stride(EMAX) + (size_t)kRouteWarps * TM * CH) * sizeof(float);
   auto kern = route_kernel<T, EMAX, TM, CH>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
