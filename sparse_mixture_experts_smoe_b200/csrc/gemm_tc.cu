@@ -49,7 +49,9 @@ constexpr int BK = 64;            // K per stage: one 128-byte swizzle row of bf
 constexpr int BN = 256;           // MMA N
 constexpr int kThreads = 384;        // 12 warps
 constexpr int kGatherWarp0 = 8;       // warps 8-11 gather scattered rows
-constexpr int kGatherThreads = 128;
+constexpr int kGatherThreads = 128;   // grouped-M kernel: warps 8-11
+constexpr int kDwGatherThreads = 256; // dW kernel: warps 8-15 gather (more copies in flight)
+constexpr int kDwThreads = 512;
 constexpr uint32_t kTmemCols = 512;  // two BN-column fp32 accumulators
 constexpr int A_BYTES = BM * BK * 2;  // 16 KB
 constexpr int B_BYTES = BN * BK * 2;  // 32 KB
@@ -137,6 +139,9 @@ __device__ __forceinline__ void cp_async_arrive(uint64_t* bar) {
 // Byte offset of 16-byte chunk c of row r inside 128-byte-swizzled 1024-byte atoms.
 __device__ __forceinline__ uint32_t sw128_off(int r, int c) {
   return (uint32_t)(r * 128 + ((c ^ (r & 7)) << 4));
+}
+__device__ __forceinline__ void prefetch_l2(const void* p) {
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
 }
 __device__ __forceinline__ void fence_proxy_async() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -322,7 +327,8 @@ __device__ __forceinline__ Tile map_tile(const SharedCtl& c, int E, int nN, int 
 // gather threads' cp.async arrivals otherwise).
 template <int SA, int SB>
 __device__ __forceinline__ void setup(SharedCtl& c, const int32_t* offsets, int E, int num_rows,
-                                      unsigned* err, uint32_t a_arrivals, uint32_t b_arrivals) {
+                                      unsigned* err, uint32_t a_arrivals, uint32_t b_arrivals,
+                                      uint32_t gather_warps = kGatherThreads / 32) {
   const int warp = threadIdx.x >> 5;
   if (threadIdx.x == 0) {
     for (int s = 0; s < SA; ++s) {
@@ -339,7 +345,7 @@ __device__ __forceinline__ void setup(SharedCtl& c, const int32_t* offsets, int 
     }
     for (int b = 0; b < IDX_STAGES; ++b) {
       mbar_init(&c.ifull[b], 1);
-      mbar_init(&c.iempty[b], kGatherThreads / 32);
+      mbar_init(&c.iempty[b], gather_warps);
     }
     c.abort_flag = 0;
     fence_mbar_init();
@@ -513,9 +519,26 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
     for (int L = blockIdx.x; L < total; L += gridDim.x, ++it) {
       const int buf = it & 1;
       const uint32_t tph = (it >> 1) & 1;
+      const Tile t = map_tile(c, g.E, nN, L);
+      if (g.epi == EPI_ACT_BWD && t.row0 + r < t.row_end) {
+        // the rows this thread will read after the main loop: pull them into L2 now
+        const int ii = t.row0 + r;
+        const int pp = g.sorted_slot[ii];
+        const int ar = g.aux_a_mode == ROWS_GROUPED ? ii : pp / g.aux_a_fan_out;
+        if (pp >= 0 && pp < g.num_rows) {
+          const int n0 = t.nb * BNo;
+          const int nn = min(BNo, g.n_out - n0);
+          for (int cb = 0; cb < nn; cb += 64) {  // 128-byte lines of bf16
+            prefetch_l2(AUXA + (size_t)ar * g.ld_aux_a + n0 + cb);
+            if (g.act != SMOE_ACT_NONE && g.out != nullptr) {
+              prefetch_l2(AUXH + (size_t)ii * g.ld_aux_h + n0 + cb);
+              if (g.act == SMOE_ACT_SWIGLU) prefetch_l2(AUXH + (size_t)ii * g.ld_aux_h + g.n_out + n0 + cb);
+            }
+          }
+        }
+      }
       if (!mbar_wait(&c.tfull[buf], tph, abort_flag, g.err)) break;
       tc_fence_after();
-      const Tile t = map_tile(c, g.E, nN, L);
       const int i = t.row0 + r;
       const bool valid = i < t.row_end;
       const int p = valid ? g.sorted_slot[i] : 0;
@@ -654,7 +677,7 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
 template <int NS>
 struct SlabGather {
   static constexpr int CPR = 8 * NS;
-  static constexpr int RSTEP = kGatherThreads / CPR;
+  static constexpr int RSTEP = kDwGatherThreads / CPR;
   static constexpr int NR = BK / RSTEP;
   int row0;        // first row of this thread
   uint32_t off0;   // shared-memory offset of (row0, chunk) inside a stage
@@ -692,7 +715,7 @@ struct SlabGather {
 // operands so that a gathered operand sits on the 128-wide A side); the store
 // is then coalesced across the warp (consecutive m, one n at a time).
 template <bool A_GATHER, bool B_GATHER, bool TRANS_OUT>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kDwThreads, 1)
 dw_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                   const DwGemm g, int nM, int nN) {
   constexpr bool kOneGather = A_GATHER && !B_GATHER;
@@ -705,8 +728,8 @@ dw_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
   SharedCtl& c = *reinterpret_cast<SharedCtl*>(smem + kRingBytes);
   volatile int* abort_flag = &c.abort_flag;
 
-  setup<SA, SB>(c, g.offsets, g.E, g.num_rows, g.err, A_GATHER ? kGatherThreads : 1,
-                B_GATHER ? kGatherThreads : 1);
+  setup<SA, SB>(c, g.offsets, g.E, g.num_rows, g.err, A_GATHER ? kDwGatherThreads : 1,
+                B_GATHER ? kDwGatherThreads : 1, kDwGatherThreads / 32);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const bool offsets_ok = c.total_mtiles > 0 || g.num_rows == 0;
   const int total = offsets_ok ? g.E * nM * nN : 0;
@@ -1028,7 +1051,7 @@ cudaError_t launch_d(const CUtensorMap& ta, const CUtensorMap& tb, const DwGemm&
   auto kern = dw_gemm_tc_kernel<AG, BG, TR>;
   cudaError_t e = prep(kern);
   if (e != cudaSuccess) return e;
-  kern<<<grid, kThreads, kSmemBytes, s>>>(ta, tb, g, nM, nN);
+  kern<<<grid, kDwThreads, kSmemBytes, s>>>(ta, tb, g, nM, nN);
   return cudaGetLastError();
 }
 
