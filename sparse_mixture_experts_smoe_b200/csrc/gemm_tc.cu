@@ -47,11 +47,19 @@ namespace {
 constexpr int BM = 128;           // rows per tile (MMA M)
 constexpr int BK = 64;            // K per stage: one 128-byte swizzle row of bf16
 constexpr int BN = 256;           // MMA N
-constexpr int kThreads = 384;        // 12 warps
+constexpr int kThreads = 512;        // 16 warps
 constexpr int kGatherWarp0 = 8;       // warps 8-11 gather scattered rows
-constexpr int kGatherThreads = 128;   // grouped-M kernel: warps 8-11
+constexpr int kGatherThreads = 256;   // grouped-M kernel: warps 8-15
 constexpr int kDwGatherThreads = 256; // dW kernel: warps 8-15 gather (more copies in flight)
 constexpr int kDwThreads = 512;
+// Warp roles.  Grouped-M kernel: 0 TMA, 1 MMA, 2-3 idle, 4-7 epilogue, 8-15 row
+// gather.  dW kernel: 0 TMA, 1 MMA, 2 source rows, 3 idle, 4-7 epilogue, 8-15
+// row gather.  (Measured: a second epilogue warp set on 12-15 with a 4-warp
+// gather was slower than this split.)  The role ranges must not overlap:
+static_assert(kGatherWarp0 == 8 && kGatherWarp0 + kGatherThreads / 32 <= kThreads / 32,
+              "grouped-M gather warps must fit the block");
+static_assert(kGatherWarp0 + kDwGatherThreads / 32 <= kDwThreads / 32,
+              "dW gather warps must fit the block");
 constexpr uint32_t kTmemCols = 512;  // two BN-column fp32 accumulators
 constexpr int A_BYTES = BM * BK * 2;  // 16 KB
 constexpr int B_BYTES = BN * BK * 2;  // 32 KB
@@ -139,9 +147,6 @@ __device__ __forceinline__ void cp_async_arrive(uint64_t* bar) {
 // Byte offset of 16-byte chunk c of row r inside 128-byte-swizzled 1024-byte atoms.
 __device__ __forceinline__ uint32_t sw128_off(int r, int c) {
   return (uint32_t)(r * 128 + ((c ^ (r & 7)) << 4));
-}
-__device__ __forceinline__ void prefetch_l2(const void* p) {
-  asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
 }
 __device__ __forceinline__ void fence_proxy_async() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -328,7 +333,8 @@ __device__ __forceinline__ Tile map_tile(const SharedCtl& c, int E, int nN, int 
 template <int SA, int SB>
 __device__ __forceinline__ void setup(SharedCtl& c, const int32_t* offsets, int E, int num_rows,
                                       unsigned* err, uint32_t a_arrivals, uint32_t b_arrivals,
-                                      uint32_t gather_warps = kGatherThreads / 32) {
+                                      uint32_t gather_warps = kGatherThreads / 32,
+                                      uint32_t epilogue_warps = 4) {
   const int warp = threadIdx.x >> 5;
   if (threadIdx.x == 0) {
     for (int s = 0; s < SA; ++s) {
@@ -341,7 +347,7 @@ __device__ __forceinline__ void setup(SharedCtl& c, const int32_t* offsets, int 
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&c.tfull[b], 1);
-      mbar_init(&c.tempty[b], 4);
+      mbar_init(&c.tempty[b], epilogue_warps);
     }
     for (int b = 0; b < IDX_STAGES; ++b) {
       mbar_init(&c.ifull[b], 1);
@@ -372,7 +378,18 @@ __device__ __forceinline__ void setup(SharedCtl& c, const int32_t* offsets, int 
   tc_fence_after();
 }
 
+// On an abort some copies (cp.async, TMA) and tensor-core operations may still
+// be in flight: each thread retires its own cp.async copies, then the CTA waits
+// a bounded 2 ms (far above any copy or MMA latency) before freeing tensor memory
+// and exiting, so nothing lands in a CTA that has gone.
 __device__ __forceinline__ void teardown(SharedCtl& c) {
+  asm volatile("cp.async.wait_all;" ::: "memory");
+  __syncthreads();
+  if (*reinterpret_cast<volatile int*>(&c.abort_flag)) {
+    const unsigned long long t0 = global_ns();
+    while (global_ns() - t0 < 2000000ull) {
+    }
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -434,11 +451,12 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
       }
     }
     __syncwarp();
-  } else if (A_GATHER && warp >= kGatherWarp0) {
+  } else if (A_GATHER && warp >= kGatherWarp0 && warp < kGatherWarp0 + kGatherThreads / 32) {
     // ---------------- row gather of the scattered A operand ----------------
-    // thread t copies 16-byte chunk (t % 8) of tile rows t/8 + 16 j, j = 0..7,
-    // into the 128-byte-swizzled K-major layout; rows past the expert's slice
-    // and columns past K are zero-filled.
+    // thread t copies 16-byte chunk (t % 8) of tile rows t/8 + kRowStep j into
+    // the 128-byte-swizzled K-major layout; rows past the expert's slice and
+    // columns past K are zero-filled.
+    constexpr int kRowStep = kGatherThreads / 8, kRowsPer = BM / kRowStep;
     const int t = threadIdx.x - kGatherWarp0 * 32;
     const int cc = t & 7, r0 = t >> 3;
     const bf16* A = reinterpret_cast<const bf16*>(g.a);
@@ -446,11 +464,11 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
     bool run = true;
     for (int L = blockIdx.x; run && L < total; L += gridDim.x) {
       const Tile tl = map_tile(c, g.E, nN, L);
-      const bf16* src[8];
+      const bf16* src[kRowsPer];
       uint32_t ok_rows = 0;
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const int i = tl.row0 + r0 + 16 * j;
+      for (int j = 0; j < kRowsPer; ++j) {
+        const int i = tl.row0 + r0 + kRowStep * j;
         src[j] = A;
         if (i < tl.row_end) {
           const int p = g.sorted_slot[i];
@@ -468,9 +486,9 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
         const uint32_t a_dst = smem_u32(sA + r.s * A_BYTES);
         const bool col_ok = kb * BK + 8 * cc < g.K;
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
+        for (int j = 0; j < kRowsPer; ++j) {
           const bool ok = col_ok && ((ok_rows >> j) & 1u);
-          cp_async16(a_dst + sw128_off(r0 + 16 * j, cc), ok ? src[j] + kb * BK : A, ok ? 16u : 0u);
+          cp_async16(a_dst + sw128_off(r0 + kRowStep * j, cc), ok ? src[j] + kb * BK : A, ok ? 16u : 0u);
         }
         cp_async_arrive(&c.fullA[r.s]);
         r.next(STAGES);
@@ -509,7 +527,7 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
       }
     }
     __syncwarp();
-  } else if (warp >= 4 && warp < 8) {  // warps 2-3 (and 8-11 without a gather) idle
+  } else if (warp >= 4 && warp < 8) {  // warps 2-3 (and 8-15 without a gather) idle
     // ---------------- epilogue ----------------
     const int q = warp - 4;  // tensor-memory lane quadrant
     const int r = q * 32 + lane;
@@ -520,23 +538,6 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
       const int buf = it & 1;
       const uint32_t tph = (it >> 1) & 1;
       const Tile t = map_tile(c, g.E, nN, L);
-      if (g.epi == EPI_ACT_BWD && t.row0 + r < t.row_end) {
-        // the rows this thread will read after the main loop: pull them into L2 now
-        const int ii = t.row0 + r;
-        const int pp = g.sorted_slot[ii];
-        const int ar = g.aux_a_mode == ROWS_GROUPED ? ii : pp / g.aux_a_fan_out;
-        if (pp >= 0 && pp < g.num_rows) {
-          const int n0 = t.nb * BNo;
-          const int nn = min(BNo, g.n_out - n0);
-          for (int cb = 0; cb < nn; cb += 64) {  // 128-byte lines of bf16
-            prefetch_l2(AUXA + (size_t)ar * g.ld_aux_a + n0 + cb);
-            if (g.act != SMOE_ACT_NONE && g.out != nullptr) {
-              prefetch_l2(AUXH + (size_t)ii * g.ld_aux_h + n0 + cb);
-              if (g.act == SMOE_ACT_SWIGLU) prefetch_l2(AUXH + (size_t)ii * g.ld_aux_h + g.n_out + n0 + cb);
-            }
-          }
-        }
-      }
       if (!mbar_wait(&c.tfull[buf], tph, abort_flag, g.err)) break;
       tc_fence_after();
       const int i = t.row0 + r;
@@ -823,7 +824,8 @@ dw_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
         }
       }
     }
-  } else if ((A_GATHER || B_GATHER) && warp >= kGatherWarp0) {
+  } else if ((A_GATHER || B_GATHER) && warp >= kGatherWarp0 &&
+             warp < kGatherWarp0 + kDwGatherThreads / 32) {
     // ---------------- cp.async gather of the scattered operand(s) ----------------
     const int t = threadIdx.x - kGatherWarp0 * 32;
     SlabGather<2> ga;
