@@ -193,6 +193,7 @@ struct MlpWs {
   float* dl = nullptr;      // bwd: [T, k]
   float* dg = nullptr;      // bwd: [T, k] when the caller passes no dgates
   float* rpart = nullptr;   // bwd: router dW partials
+  void* wrt = nullptr;      // bwd: router weight transposed [E, d] dtype
   int dg_ld = 0, r_chunks = 0;
   size_t bytes = 0;
 };
@@ -214,6 +215,7 @@ MlpWs mlp_layout(void* ws, const smoe_mlp_desc& m, int backward) {
     l.dg = (float*)c.take(S * sizeof(float));
     l.r_chunks = route_dw_chunks(m.T);
     l.rpart = (float*)c.take(((size_t)l.r_chunks * m.E * m.d + (size_t)l.r_chunks * m.E) * sizeof(float));
+    l.wrt = c.take((size_t)m.E * m.d * esize(dt));
   }
   l.bytes = c.off;
   return l;
@@ -703,8 +705,10 @@ int smoe_mlp_bwd(const smoe_mlp_desc* desc, const smoe_mlp_tensors* t, void* str
     { PROF("gemm.bwd_dx", 1); SMOE_TRY(run_grouped(g, dt, s), "mlp bwd gemm dx"); }
   }
   // dx[t] = sum_j rows + router term sum_j dl W_r[:, e_j]
+  { PROF("transpose_wr", 1);
+  SMOE_TRY(launch_transpose_wr(t->w_r, m.d, m.E, dt, l.wrt, s), "mlp bwd router transpose"); }
   { PROF("combine.dx", 1);
-  SMOE_TRY(launch_combine(l.dxcomb, m.T, m.k, m.d, t->dx, dt, l.dl, t->topk_idx, t->w_r, m.E, s),
+  SMOE_TRY(launch_combine(l.dxcomb, m.T, m.k, m.d, t->dx, dt, l.dl, t->topk_idx, l.wrt, m.E, s),
            "mlp bwd dx combine"); }
   { PROF("route_dw", 2);
   SMOE_TRY(launch_route_dw(t->x, t->topk_idx, l.dl, m.T, m.d, m.E, m.k, dt, l.rpart, l.r_chunks,

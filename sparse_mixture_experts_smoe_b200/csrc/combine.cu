@@ -15,11 +15,13 @@
 namespace smoe {
 namespace {
 
-// One thread per 4 consecutive columns of one token.
+// One thread per 4 consecutive columns of one token.  The router term reads the
+// transposed router weight w_rt [E, N] so each selected expert contributes one
+// contiguous 4-element load.
 template <typename TO, typename TW>
 __global__ void combine_kernel(const float* __restrict__ ws, int T_, int ck, int N,
                                TO* __restrict__ out, const float* __restrict__ dl,
-                               const int32_t* __restrict__ idx, const TW* __restrict__ w_r,
+                               const int32_t* __restrict__ idx, const TW* __restrict__ w_rt,
                                int E) {
   const int n4 = N / 4;
   const size_t q = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
@@ -36,10 +38,11 @@ __global__ void combine_kernel(const float* __restrict__ ws, int T_, int ck, int
       const int e = idx[(size_t)t * ck + j];
       if (e < 0 || e >= E) continue;
       const float g = dl[(size_t)t * ck + j];
-      s.x = fmaf(g, to_f(w_r[(size_t)(c + 0) * E + e]), s.x);
-      s.y = fmaf(g, to_f(w_r[(size_t)(c + 1) * E + e]), s.y);
-      s.z = fmaf(g, to_f(w_r[(size_t)(c + 2) * E + e]), s.z);
-      s.w = fmaf(g, to_f(w_r[(size_t)(c + 3) * E + e]), s.w);
+      const TW* w = w_rt + (size_t)e * N + c;
+      s.x = fmaf(g, to_f(w[0]), s.x);
+      s.y = fmaf(g, to_f(w[1]), s.y);
+      s.z = fmaf(g, to_f(w[2]), s.z);
+      s.w = fmaf(g, to_f(w[3]), s.w);
     }
   }
   TO* o = out + (size_t)t * N + c;
@@ -47,6 +50,15 @@ __global__ void combine_kernel(const float* __restrict__ ws, int T_, int ck, int
   o[1] = from_f<TO>(s.y);
   o[2] = from_f<TO>(s.z);
   o[3] = from_f<TO>(s.w);
+}
+
+// w_rt[e][i] = w_r[i][e]
+template <typename T>
+__global__ void transpose_kernel(const T* __restrict__ w_r, int d, int E, T* __restrict__ w_rt) {
+  const int q = blockIdx.x * blockDim.x + threadIdx.x;  // q = e * d + i
+  if (q >= d * E) return;
+  const int e = q / d, i = q % d;
+  w_rt[q] = w_r[(size_t)i * E + e];
 }
 
 __global__ void dg_reduce_kernel(const float* __restrict__ partial, int ld, int n_tiles,
@@ -75,17 +87,27 @@ __global__ void gather_scale_kernel(const T* __restrict__ src, int ld_src, int m
 
 }  // namespace
 
+cudaError_t launch_transpose_wr(const void* w_r, int d, int E, smoe_dtype dt, void* w_rt,
+                                cudaStream_t s) {
+  const unsigned blocks = (unsigned)((d * E + 255) / 256);
+  if (dt == SMOE_BF16)
+    transpose_kernel<bf16><<<blocks, 256, 0, s>>>((const bf16*)w_r, d, E, (bf16*)w_rt);
+  else
+    transpose_kernel<float><<<blocks, 256, 0, s>>>((const float*)w_r, d, E, (float*)w_rt);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_combine(const float* ws, int T_, int ck, int N, void* out, smoe_dtype out_dt,
-                           const float* dl, const int32_t* idx, const void* w_r, int E,
+                           const float* dl, const int32_t* idx, const void* w_rt, int E,
                            cudaStream_t s) {
   const size_t n = (size_t)T_ * (N / 4);
   const unsigned blocks = (unsigned)((n + 255) / 256);
   if (out_dt == SMOE_BF16)
     combine_kernel<bf16, bf16><<<blocks, 256, 0, s>>>(ws, T_, ck, N, (bf16*)out, dl, idx,
-                                                      (const bf16*)w_r, E);
+                                                      (const bf16*)w_rt, E);
   else
     combine_kernel<float, float><<<blocks, 256, 0, s>>>(ws, T_, ck, N, (float*)out, dl, idx,
-                                                        (const float*)w_r, E);
+                                                        (const float*)w_rt, E);
   return cudaGetLastError();
 }
 

@@ -24,10 +24,13 @@
 // expert offsets (expert-major, then N tile, then M tile, so the CTAs of one wave
 // share the expert's input rows in L2).  Warp roles: warp 0 = TMA producer,
 // warp 1 = MMA issuer and tensor-memory owner, warps 4-7 = epilogue (thread r owns
-// accumulator row r), warps 8-11 = row gather of a scattered operand.  Two 256-column fp32 accumulators in tensor memory let the
-// epilogue of one tile overlap the main loop of the next.  Epilogues: scaled
-// store (gate), activation forward (H and A = gelu(H) or silu(Hg) * Hu), and the
-// activation backward (gate gradient partial <dA', A>, g*A, dH = g dA' act'(H)).
+// accumulator row r), warps 8-15 = row gather of a scattered operand.  Two
+// 256-column fp32 accumulators in tensor memory let the epilogue of one tile
+// overlap the main loop of the next.  Epilogues: scaled store (gate), activation
+// forward (H and A = gelu(H) or silu(Hg) * Hu), and the activation backward (gate
+// gradient partial <dA', A>, g*A, dH = g dA' act'(H)); their bf16 rows in grouped
+// order move through shared memory as 32 x 32 TMA boxes, scattered or fp32 rows
+// by per-row bulk copies.
 //
 // dW kernel: tile (e, m, n) of dW[e] = sum over the expert's rows r of
 // A[r, m] * B[r, n]; the reduction runs over the slice rows, so both operands are
@@ -48,7 +51,7 @@ constexpr int BM = 128;           // rows per tile (MMA M)
 constexpr int BK = 64;            // K per stage: one 128-byte swizzle row of bf16
 constexpr int BN = 256;           // MMA N
 constexpr int kThreads = 512;        // 16 warps
-constexpr int kGatherWarp0 = 8;       // warps 8-11 gather scattered rows
+constexpr int kGatherWarp0 = 8;       // first warp of the row gather
 constexpr int kGatherThreads = 256;   // grouped-M kernel: warps 8-15
 constexpr int kDwGatherThreads = 256; // dW kernel: warps 8-15 gather (more copies in flight)
 constexpr int kDwThreads = 512;
@@ -151,6 +154,28 @@ __device__ __forceinline__ uint32_t sw128_off(int r, int c) {
 __device__ __forceinline__ void fence_proxy_async() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
+// Bulk (non-tensor) asynchronous copies on the TMA engine, one per row segment
+// in the grouped epilogue; both addresses and the size are multiples of 16 bytes.
+__device__ __forceinline__ void bulk_s2g(void* gdst, uint32_t ssrc, uint32_t bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(gdst), "r"(ssrc),
+               "r"(bytes)
+               : "memory");
+}
+// TMA tensor store of a box from shared memory (3-D map).
+__device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, uint32_t ssrc, int c0, int c1,
+                                             int c2) {
+  asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
+                   (uint64_t)map),
+               "r"(ssrc), "r"(c0), "r"(c1), "r"(c2)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// This thread's committed bulk stores have finished reading shared memory.
+__device__ __forceinline__ void bulk_wait_read() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+// ... and have been performed.
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_before() {
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
 }
@@ -288,13 +313,39 @@ struct SharedCtl {
   uint64_t tfull[2], tempty[2];
   uint64_t ifull[IDX_STAGES];   // index ring: written by warp 2
   uint64_t iempty[IDX_STAGES];  // index ring: released by the 4 gather warps
-  int idx[IDX_STAGES][2][BK];   // source row per operand (A, B) of each stage row, -1 = zero
+  uint64_t ebar[4];             // per epilogue warp: its input boxes have landed
   uint32_t tmem_base;
   int abort_flag;
   int total_mtiles;
   int prefix[kMaxE + 1];  // M-tile prefix per expert
-  int off[kMaxE + 1];     // expert offsets
 };
+
+// Shared memory after SharedCtl, per kernel.
+// dW kernel: the expert offsets and the slot-index ring.
+struct DwExtra {
+  int idx[IDX_STAGES][2][BK];  // source row per operand (A, B) of each stage row, -1 = zero
+  int off[kMaxE + 1];          // expert offsets
+};
+// Grouped-M kernel: a staging area per epilogue warp for the output of one
+// 32-column chunk of its 32 accumulator rows, used in one of two layouts:
+//   boxed: three 2 KB boxes of 32 rows x 64 bytes in the 64-byte swizzle, each
+//          written out by one TMA tensor store (the warp's rows are consecutive
+//          rows of one expert's slice);
+//   slots: per thread a 208-byte slot of up to three 64-byte row segments (or
+//          one 128-byte fp32 one) written out by per-row bulk copies; the stride
+//          of 13 x 16 bytes keeps 8 consecutive threads' 16-byte accesses on
+//          distinct banks.
+constexpr int kSlotBytes = 208;
+constexpr int kBoxBytes = 32 * 64;
+constexpr int kWarpStaging = 32 * kSlotBytes;  // 13 x 512: boxes stay 512-byte aligned
+static_assert(3 * kBoxBytes <= kWarpStaging && kWarpStaging % 512 == 0, "staging layout");
+constexpr int kStagingBytes = 4 * kWarpStaging;
+enum : int { kBoxStores = 1, kBoxLoads = 2 };  // grouped-epilogue box modes (launch flags)
+
+constexpr size_t kCtlBytes = (sizeof(SharedCtl) + 1023) / 1024 * 1024;
+constexpr size_t kGroupedSmem = 1024 + (size_t)kRingBytes + kCtlBytes + kStagingBytes;
+constexpr size_t kDwSmem = 1024 + (size_t)kRingBytes + kCtlBytes + sizeof(DwExtra);
+static_assert(kGroupedSmem <= 232448 && kDwSmem <= 232448, "shared memory exceeds 227 KB");
 
 // Position in a ring of n stages and the parity of the current lap.
 struct Ring {
@@ -309,8 +360,10 @@ struct Tile {
   int e, mb, nb, row0, row_end;
 };
 
-// linear tile L -> (expert, M tile, N tile); expert-major, then N tile, then M tile
-__device__ __forceinline__ Tile map_tile(const SharedCtl& c, int E, int nN, int L) {
+// linear tile L -> (expert, M tile, N tile); expert-major, then N tile, then M tile.
+// `off` = the expert offsets in global memory (validated by setup).
+__device__ __forceinline__ Tile map_tile(const SharedCtl& c, const int32_t* off, int E, int nN,
+                                         int L) {
   int lo = 0, hi = E - 1;  // largest e with prefix[e] * nN <= L
   while (lo < hi) {
     const int mid = (lo + hi + 1) >> 1;
@@ -322,18 +375,19 @@ __device__ __forceinline__ Tile map_tile(const SharedCtl& c, int E, int nN, int 
   const int lp = L - c.prefix[lo] * nN;
   t.nb = lp / mt;
   t.mb = lp % mt;
-  t.row0 = c.off[lo] + t.mb * BM;
-  t.row_end = c.off[lo + 1];
+  t.row0 = __ldg(off + lo) + t.mb * BM;
+  t.row_end = __ldg(off + lo + 1);
   return t;
 }
 
-// Setup common to both kernels: barriers, tensor memory, offsets (validated).
+// Setup common to both kernels: barriers, tensor memory, offsets (validated;
+// copied to off_copy when given).
 // a_arrivals / b_arrivals: producer arrivals per full stage (1 for TMA, the
 // gather threads' cp.async arrivals otherwise).
 template <int SA, int SB>
 __device__ __forceinline__ void setup(SharedCtl& c, const int32_t* offsets, int E, int num_rows,
                                       unsigned* err, uint32_t a_arrivals, uint32_t b_arrivals,
-                                      uint32_t gather_warps = kGatherThreads / 32,
+                                      uint32_t gather_warps, int* off_copy,
                                       uint32_t epilogue_warps = 4) {
   const int warp = threadIdx.x >> 5;
   if (threadIdx.x == 0) {
@@ -353,17 +407,25 @@ __device__ __forceinline__ void setup(SharedCtl& c, const int32_t* offsets, int 
       mbar_init(&c.ifull[b], 1);
       mbar_init(&c.iempty[b], gather_warps);
     }
+    for (int b = 0; b < 4; ++b) mbar_init(&c.ebar[b], 1);
     c.abort_flag = 0;
     fence_mbar_init();
   }
   if (warp == 1) tmem_alloc(&c.tmem_base, kTmemCols);
-  for (int e = threadIdx.x; e <= E; e += blockDim.x) c.off[e] = offsets[e];
+  for (int e = threadIdx.x; e <= E; e += blockDim.x) {  // raw offsets first
+    const int o = offsets[e];
+    c.prefix[e] = o;
+    if (off_copy) off_copy[e] = o;
+  }
   __syncthreads();
-  if (threadIdx.x == 0) {
-    bool ok = c.off[0] == 0 && c.off[E] == num_rows;
+  if (threadIdx.x == 0) {  // in place: offsets -> M-tile prefix
+    bool ok = c.prefix[0] == 0 && c.prefix[E] == num_rows;
+    int prev = c.prefix[0];
     c.prefix[0] = 0;
     for (int e = 0; e < E; ++e) {
-      const int n = c.off[e + 1] - c.off[e];
+      const int cur = c.prefix[e + 1];
+      const int n = cur - prev;
+      prev = cur;
       if (n < 0) ok = false;
       c.prefix[e + 1] = c.prefix[e] + (n > 0 ? (n + BM - 1) / BM : 0);
     }
@@ -402,7 +464,12 @@ __device__ __forceinline__ void teardown(SharedCtl& c) {
 template <bool A_GATHER, bool B_KMAJOR, bool SWIGLU_FWD>
 __global__ void __launch_bounds__(kThreads, 1)
 grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
-                       const __grid_constant__ CUtensorMap tmB, const GroupedGemm g, int nN) {
+                       const __grid_constant__ CUtensorMap tmB,
+                       const __grid_constant__ CUtensorMap tmO,
+                       const __grid_constant__ CUtensorMap tmO2,
+                       const __grid_constant__ CUtensorMap tmXa,
+                       const __grid_constant__ CUtensorMap tmXh, const GroupedGemm g, int nN,
+                       int box_flags) {
   // One ring of STAGES stages holds A and B together (fullA/emptyA guard a whole
   // stage): measured faster here than separate rings, whose second wait and
   // commit per stage cost more than their extra depth returned.
@@ -415,7 +482,8 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
   SharedCtl& c = *reinterpret_cast<SharedCtl*>(smem + kRingBytes);
   volatile int* abort_flag = &c.abort_flag;
 
-  setup<STAGES, 0>(c, g.offsets, g.E, g.num_rows, g.err, 1 + (A_GATHER ? kGatherThreads : 0), 1);
+  setup<STAGES, 0>(c, g.offsets, g.E, g.num_rows, g.err, 1 + (A_GATHER ? kGatherThreads : 0), 1,
+                   kGatherThreads / 32, nullptr);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int total = c.total_mtiles * nN;
   const int nK = cdiv(g.K, BK);
@@ -427,7 +495,7 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
       Ring r;
       bool run = true;
       for (int L = blockIdx.x; run && L < total; L += gridDim.x) {
-        const Tile t = map_tile(c, g.E, nN, L);
+        const Tile t = map_tile(c, g.offsets, g.E, nN, L);
         for (int kb = 0; kb < nK; ++kb) {
           if (!mbar_wait(&c.emptyA[r.s], r.ph ^ 1, abort_flag, g.err)) { run = false; break; }
           uint8_t* b_dst = sB + r.s * B_BYTES;
@@ -463,7 +531,7 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
     Ring r;
     bool run = true;
     for (int L = blockIdx.x; run && L < total; L += gridDim.x) {
-      const Tile tl = map_tile(c, g.E, nN, L);
+      const Tile tl = map_tile(c, g.offsets, g.E, nN, L);
       const bf16* src[kRowsPer];
       uint32_t ok_rows = 0;
 #pragma unroll
@@ -529,15 +597,33 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
     __syncwarp();
   } else if (warp >= 4 && warp < 8) {  // warps 2-3 (and 8-15 without a gather) idle
     // ---------------- epilogue ----------------
+    // Thread r owns accumulator row r.  Per 32-column chunk the warp stages its
+    // rows' output segments in shared memory and hands them to the TMA engine:
+    // one tensor store per output box when its 32 rows are consecutive rows of
+    // the expert's slice (o_tma), else one bulk copy per row.  Plain stores from
+    // the tensor-memory row layout would make every 16-byte access of a warp
+    // touch 32 lines and compete with the cp.async row gathers for the same
+    // unit.  ACT_BWD's per-row inputs stay 16-byte loads issued before the
+    // accumulator read: per-row bulk loads of 64 bytes measured far slower.
     const int q = warp - 4;  // tensor-memory lane quadrant
     const int r = q * 32 + lane;
+    uint8_t* wstage = smem + kRingBytes + kCtlBytes + q * kWarpStaging;
+    uint8_t* slot = wstage + lane * kSlotBytes;
+    const uint32_t wstage_s = smem_u32(wstage), slot_s = smem_u32(slot);
+    const int sw = (lane >> 1) & 3;  // 64-byte swizzle of this thread's box row
     const bf16* AUXA = reinterpret_cast<const bf16*>(g.aux_a);
     const bf16* AUXH = reinterpret_cast<const bf16*>(g.aux_h);
+    // SwiGLU's forward instantiation has only the ACT_FWD epilogue
+    const bool act_bwd = !SWIGLU_FWD && g.epi == EPI_ACT_BWD;
+    const bool epi_store = !SWIGLU_FWD && g.epi == EPI_STORE;
+    const bool swi = g.act == SMOE_ACT_SWIGLU;
+    const bool need_h = act_bwd && g.out != nullptr && g.act != SMOE_ACT_NONE;
+    uint32_t eph = 0;  // phase of this warp's input-box barrier
     int it = 0;
     for (int L = blockIdx.x; L < total; L += gridDim.x, ++it) {
       const int buf = it & 1;
       const uint32_t tph = (it >> 1) & 1;
-      const Tile t = map_tile(c, g.E, nN, L);
+      const Tile t = map_tile(c, g.offsets, g.E, nN, L);
       if (!mbar_wait(&c.tfull[buf], tph, abort_flag, g.err)) break;
       tc_fence_after();
       const int i = t.row0 + r;
@@ -548,119 +634,205 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
       const int orow = g.out_mode == ROWS_GROUPED ? i : p;
       const float gate = (p_ok && g.gates) ? g.gates[p] : 1.0f;
       const uint32_t trow = c.tmem_base + ((uint32_t)(q * 32) << 16) + buf * BN;
+      const int wrow0 = t.row0 + q * 32;
+      const bool boxed = (box_flags & kBoxStores) && wrow0 + 32 <= t.row_end;  // warp-uniform
+      // 16-byte chunk j8 of box k in this thread's row
+      auto box_chunk = [&](int k, int j8) -> uint4* {
+        return reinterpret_cast<uint4*>(wstage + k * kBoxBytes + lane * 64 + ((j8 ^ sw) << 4));
+      };
+      // 16-byte chunk j8 of output segment k of this thread's row
+      auto chunk = [&](int k, int j8) -> uint4* {
+        return reinterpret_cast<uint4*>(boxed ? wstage + k * kBoxBytes + lane * 64 + ((j8 ^ sw) << 4)
+                                              : slot + k * 64 + 16 * j8);
+      };
       float dg_acc = 0.0f;
       int arow = 0;
-      if (g.epi == EPI_ACT_BWD && p_ok) arow = g.aux_a_mode == ROWS_GROUPED ? i : p / g.aux_a_fan_out;
+      if (act_bwd && p_ok) arow = g.aux_a_mode == ROWS_GROUPED ? i : p / g.aux_a_fan_out;
 #pragma unroll 1
       for (int c0 = 0; c0 < BNo; c0 += 32) {
-        float v[32], u[32];
         const int n0 = t.nb * BNo + c0;
-        if (g.epi == EPI_ACT_BWD) {
-          // issue every global load of the chunk first, then read the accumulator
-          uint4 ra[4], rg[4], ru[4];
-          const bool swi = g.act == SMOE_ACT_SWIGLU;
-          const bool need_h = g.out != nullptr && g.act != SMOE_ACT_NONE;
-#pragma unroll
-          for (int j8 = 0; j8 < 4; ++j8) {
-            const int n = n0 + 8 * j8;
-            const bool in = p_ok && n < g.n_out;
-            ra[j8] = in ? __ldg(reinterpret_cast<const uint4*>(AUXA + (size_t)arow * g.ld_aux_a + n)) : make_uint4(0, 0, 0, 0);
-            rg[j8] = (in && need_h) ? __ldg(reinterpret_cast<const uint4*>(AUXH + (size_t)i * g.ld_aux_h + n)) : make_uint4(0, 0, 0, 0);
-            ru[j8] = (in && need_h && swi) ? __ldg(reinterpret_cast<const uint4*>(AUXH + (size_t)i * g.ld_aux_h + g.n_out + n)) : make_uint4(0, 0, 0, 0);
+        const int ncols = min(32, g.n_out - n0);  // a multiple of 8, uniform over the warp
+        if (ncols <= 0) break;
+        const uint32_t seg = (uint32_t)ncols * 2;  // bytes of the chunk's bf16 row segment
+        float v[32], u[32];
+        uint4 ra[4], rg[4], ru[4];
+        if (act_bwd && (box_flags & kBoxLoads)) {
+          // inputs as boxes of the warp's 32 rows (rows past the slice are read
+          // but not used; rows past the tensor read as zeros)
+          bulk_wait_read();
+          __syncwarp();
+          if (lane == 0) {
+            const uint32_t nbox = 1u + (need_h ? 1u : 0u) + (need_h && swi ? 1u : 0u);
+            mbar_expect_tx(&c.ebar[q], nbox * kBoxBytes);
+            tma_load_3d(wstage, &tmXa, &c.ebar[q], n0, 0, wrow0);
+            if (need_h) {
+              tma_load_3d(wstage + kBoxBytes, &tmXh, &c.ebar[q], n0, 0, wrow0);
+              if (swi) tma_load_3d(wstage + 2 * kBoxBytes, &tmXh, &c.ebar[q], n0, 1, wrow0);
+            }
           }
           tmem_ld32(trow + c0, v);
-          if (!p_ok) continue;
+          if (!mbar_wait(&c.ebar[q], eph, abort_flag, g.err)) break;
+          eph ^= 1;
+#pragma unroll
+          for (int j8 = 0; j8 < 4; ++j8) {
+            ra[j8] = *box_chunk(0, j8);
+            rg[j8] = need_h ? *box_chunk(1, j8) : make_uint4(0, 0, 0, 0);
+            ru[j8] = (need_h && swi) ? *box_chunk(2, j8) : make_uint4(0, 0, 0, 0);
+          }
+          __syncwarp();  // every lane has read its rows before any lane writes
+        } else if (act_bwd) {  // issue the chunk's global loads before the accumulator read
 #pragma unroll
           for (int j8 = 0; j8 < 4; ++j8) {
             const int n = n0 + 8 * j8;
-            if (n >= g.n_out) break;
-            const float* vv = v + 8 * j8;
-            float a8[8], ga[8], dh[8], du[8], hg[8], hu[8];
-            unpack8(ra[j8], a8);
+            const bool in = p_ok && 8 * j8 < ncols;
+            const uint4 z = make_uint4(0, 0, 0, 0);
+            ra[j8] = in ? __ldg(reinterpret_cast<const uint4*>(AUXA + (size_t)arow * g.ld_aux_a + n)) : z;
+            rg[j8] = (in && need_h) ? __ldg(reinterpret_cast<const uint4*>(AUXH + (size_t)i * g.ld_aux_h + n)) : z;
+            ru[j8] = (in && need_h && swi)
+                         ? __ldg(reinterpret_cast<const uint4*>(AUXH + (size_t)i * g.ld_aux_h + g.n_out + n))
+                         : z;
+          }
+        }
+        if (!(act_bwd && (box_flags & kBoxLoads))) tmem_ld32(trow + c0, v);
+        if (SWIGLU_FWD) tmem_ld32(trow + BNo + c0, u);
+        bulk_wait_read();  // this thread's earlier copies have read the staging area ...
+        __syncwarp();      // ... and so have the other lanes'
+        if (p_ok) {
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-              dg_acc = fmaf(vv[j], a8[j], dg_acc);
-              ga[j] = gate * a8[j];
-            }
-            if (g.out2)
-              *reinterpret_cast<uint4*>(reinterpret_cast<bf16*>(g.out2) + (size_t)i * g.ldo2 + n) = pack8(ga);
-            if (!g.out) continue;
-            if (swi) {
-              unpack8(rg[j8], hg);
-              unpack8(ru[j8], hu);
+          for (int j8 = 0; j8 < 4; ++j8) {
+            if (8 * j8 >= ncols) break;
+            float* vv = v + 8 * j8;
+            if (act_bwd) {  // [g A | dH (gate) | dH up] or [g A | dH]
+              float a8[8], ga[8], dh[8], du[8], hg[8], hu[8];
+              unpack8(ra[j8], a8);
 #pragma unroll
               for (int j = 0; j < 8; ++j) {
-                const float da = gate * vv[j];
-                const float sg = fast_sigmoid(hg[j]);
-                dh[j] = da * hu[j] * sg * fmaf(hg[j], 1.0f - sg, 1.0f);
-                du[j] = da * hg[j] * sg;
+                dg_acc = fmaf(vv[j], a8[j], dg_acc);
+                ga[j] = gate * a8[j];
               }
-              bf16* O = reinterpret_cast<bf16*>(g.out) + (size_t)orow * g.ldo;
-              *reinterpret_cast<uint4*>(O + n) = pack8(dh);
-              *reinterpret_cast<uint4*>(O + g.n_out + n) = pack8(du);
-            } else {
-              if (g.act == SMOE_ACT_GELU_TANH) {
+              *chunk(0, j8) = pack8(ga);
+              if (!g.out) continue;
+              if (swi) {
                 unpack8(rg[j8], hg);
+                unpack8(ru[j8], hu);
 #pragma unroll
-                for (int j = 0; j < 8; ++j) dh[j] = gate * vv[j] * fast_gelu_grad(hg[j]);
+                for (int j = 0; j < 8; ++j) {
+                  const float da = gate * vv[j];
+                  const float sg = fast_sigmoid(hg[j]);
+                  dh[j] = da * hu[j] * sg * fmaf(hg[j], 1.0f - sg, 1.0f);
+                  du[j] = da * hg[j] * sg;
+                }
+                *chunk(1, j8) = pack8(dh);
+                *chunk(2, j8) = pack8(du);
               } else {
+                if (g.act == SMOE_ACT_GELU_TANH) {
+                  unpack8(rg[j8], hg);
 #pragma unroll
-                for (int j = 0; j < 8; ++j) dh[j] = gate * vv[j];
+                  for (int j = 0; j < 8; ++j) dh[j] = gate * vv[j] * fast_gelu_grad(hg[j]);
+                } else {
+#pragma unroll
+                  for (int j = 0; j < 8; ++j) dh[j] = gate * vv[j];
+                }
+                if (g.out_f32) {  // never boxed
+                  float4* dst = reinterpret_cast<float4*>(slot + 64 + 32 * j8);
+                  dst[0] = make_float4(dh[0], dh[1], dh[2], dh[3]);
+                  dst[1] = make_float4(dh[4], dh[5], dh[6], dh[7]);
+                } else {
+                  *chunk(1, j8) = pack8(dh);
+                }
               }
-              if (g.out_f32) {
-                float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(g.out) + (size_t)orow * g.ldo + n);
-                dst[0] = make_float4(dh[0], dh[1], dh[2], dh[3]);
-                dst[1] = make_float4(dh[4], dh[5], dh[6], dh[7]);
+            } else if (epi_store) {  // [g acc]
+              float o[8];
+#pragma unroll
+              for (int j = 0; j < 8; ++j) o[j] = gate * vv[j];
+              if (g.out_f32) {  // never boxed
+                float4* dst = reinterpret_cast<float4*>(slot + 32 * j8);
+                dst[0] = make_float4(o[0], o[1], o[2], o[3]);
+                dst[1] = make_float4(o[4], o[5], o[6], o[7]);
               } else {
-                *reinterpret_cast<uint4*>(reinterpret_cast<bf16*>(g.out) + (size_t)orow * g.ldo + n) = pack8(dh);
+                *chunk(0, j8) = pack8(o);
+              }
+            } else {  // EPI_ACT_FWD: [H (gate) | H up | A] or [H | A]
+              float a8[8];
+              if (SWIGLU_FWD) {
+                float* uu = u + 8 * j8;
+#pragma unroll
+                for (int j = 0; j < 8; ++j) a8[j] = vv[j] * fast_sigmoid(vv[j]) * uu[j];
+                *chunk(0, j8) = pack8(vv);
+                *chunk(1, j8) = pack8(uu);
+                *chunk(2, j8) = pack8(a8);
+              } else {
+#pragma unroll
+                for (int j = 0; j < 8; ++j) a8[j] = fast_gelu(vv[j]);
+                *chunk(0, j8) = pack8(vv);
+                *chunk(1, j8) = pack8(a8);
               }
             }
           }
-          continue;
         }
-        tmem_ld32(trow + c0, v);
-        if (SWIGLU_FWD) tmem_ld32(trow + BNo + c0, u);
-        if (!p_ok) continue;
-#pragma unroll
-        for (int j8 = 0; j8 < 4; ++j8) {
-          const int n = n0 + 8 * j8;
-          if (n >= g.n_out) break;
-          float* vv = v + 8 * j8;
-          if (g.epi == EPI_STORE) {
-            float o[8];
-#pragma unroll
-            for (int j = 0; j < 8; ++j) o[j] = gate * vv[j];
-            if (g.out_f32) {
-              float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(g.out) + (size_t)orow * g.ldo + n);
-              dst[0] = make_float4(o[0], o[1], o[2], o[3]);
-              dst[1] = make_float4(o[4], o[5], o[6], o[7]);
+        fence_proxy_async();  // the staged bytes are visible to the TMA engine
+        __syncwarp();
+        if (boxed) {
+          if (lane == 0) {
+            if (act_bwd) {
+              if (g.out2) tma_store_3d(&tmO2, wstage_s, n0, 0, wrow0);
+              if (g.out) {
+                tma_store_3d(&tmO, wstage_s + kBoxBytes, n0, 0, wrow0);
+                if (swi) tma_store_3d(&tmO, wstage_s + 2 * kBoxBytes, n0, 1, wrow0);
+              }
+            } else if (epi_store) {
+              tma_store_3d(&tmO, wstage_s, n0, 0, wrow0);
             } else {
-              *reinterpret_cast<uint4*>(reinterpret_cast<bf16*>(g.out) + (size_t)orow * g.ldo + n) = pack8(o);
+              tma_store_3d(&tmO, wstage_s, n0, 0, wrow0);
+              if (SWIGLU_FWD) {
+                tma_store_3d(&tmO, wstage_s + kBoxBytes, n0, 1, wrow0);
+                tma_store_3d(&tmO2, wstage_s + 2 * kBoxBytes, n0, 0, wrow0);
+              } else {
+                tma_store_3d(&tmO2, wstage_s + kBoxBytes, n0, 0, wrow0);
+              }
             }
-          } else {  // EPI_ACT_FWD
-            float a8[8];
-            if (SWIGLU_FWD) {
-              float* uu = u + 8 * j8;
-#pragma unroll
-              for (int j = 0; j < 8; ++j) a8[j] = vv[j] * fast_sigmoid(vv[j]) * uu[j];
-              bf16* H = reinterpret_cast<bf16*>(g.out) + (size_t)orow * g.ldo;
-              *reinterpret_cast<uint4*>(H + n) = pack8(vv);
-              *reinterpret_cast<uint4*>(H + g.n_out + n) = pack8(uu);
-            } else {
-#pragma unroll
-              for (int j = 0; j < 8; ++j) a8[j] = fast_gelu(vv[j]);
-              *reinterpret_cast<uint4*>(reinterpret_cast<bf16*>(g.out) + (size_t)orow * g.ldo + n) = pack8(vv);
-            }
-            *reinterpret_cast<uint4*>(reinterpret_cast<bf16*>(g.out2) + (size_t)orow * g.ldo2 + n) = pack8(a8);
+            bulk_commit();
           }
+        } else if (p_ok) {
+          if (act_bwd) {
+            if (g.out2) bulk_s2g(reinterpret_cast<bf16*>(g.out2) + (size_t)i * g.ldo2 + n0, slot_s, seg);
+            if (g.out) {
+              if (swi) {
+                bf16* O = reinterpret_cast<bf16*>(g.out) + (size_t)orow * g.ldo;
+                bulk_s2g(O + n0, slot_s + 64, seg);
+                bulk_s2g(O + g.n_out + n0, slot_s + 128, seg);
+              } else if (g.out_f32) {
+                bulk_s2g(reinterpret_cast<float*>(g.out) + (size_t)orow * g.ldo + n0, slot_s + 64, 2 * seg);
+              } else {
+                bulk_s2g(reinterpret_cast<bf16*>(g.out) + (size_t)orow * g.ldo + n0, slot_s + 64, seg);
+              }
+            }
+          } else if (epi_store) {
+            if (g.out_f32)
+              bulk_s2g(reinterpret_cast<float*>(g.out) + (size_t)orow * g.ldo + n0, slot_s, 2 * seg);
+            else
+              bulk_s2g(reinterpret_cast<bf16*>(g.out) + (size_t)orow * g.ldo + n0, slot_s, seg);
+          } else {
+            bf16* H = reinterpret_cast<bf16*>(g.out) + (size_t)orow * g.ldo;
+            bf16* A2 = reinterpret_cast<bf16*>(g.out2) + (size_t)orow * g.ldo2;
+            bulk_s2g(H + n0, slot_s, seg);
+            if (SWIGLU_FWD) {
+              bulk_s2g(H + g.n_out + n0, slot_s + 64, seg);
+              bulk_s2g(A2 + n0, slot_s + 128, seg);
+            } else {
+              bulk_s2g(A2 + n0, slot_s + 64, seg);
+            }
+          }
+          bulk_commit();
         }
       }
-      if (g.epi == EPI_ACT_BWD && p_ok && g.dg_partial)
+      if (act_bwd && p_ok && g.dg_partial)
         g.dg_partial[(size_t)i * g.dg_ld + t.nb] = dg_acc;
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&c.tempty[buf]);
     }
+    bulk_wait_all();
   }
   teardown(c);
 }
@@ -727,10 +899,11 @@ dw_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
   uint8_t* sA = smem;
   uint8_t* sB = smem + SA * A_BYTES;
   SharedCtl& c = *reinterpret_cast<SharedCtl*>(smem + kRingBytes);
+  DwExtra& x = *reinterpret_cast<DwExtra*>(smem + kRingBytes + kCtlBytes);
   volatile int* abort_flag = &c.abort_flag;
 
   setup<SA, SB>(c, g.offsets, g.E, g.num_rows, g.err, A_GATHER ? kDwGatherThreads : 1,
-                B_GATHER ? kDwGatherThreads : 1, kDwGatherThreads / 32);
+                B_GATHER ? kDwGatherThreads : 1, kDwGatherThreads / 32, x.off);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const bool offsets_ok = c.total_mtiles > 0 || g.num_rows == 0;
   const int total = offsets_ok ? g.E * nM * nN : 0;
@@ -750,7 +923,7 @@ dw_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
       for (int L = blockIdx.x; run && L < total; L += gridDim.x) {
         int e, mb, nb;
         coords(L, e, mb, nb);
-        const int r_begin = c.off[e], r_end = c.off[e + 1];
+        const int r_begin = x.off[e], r_end = x.off[e + 1];
         const int nK = cdiv(r_end - r_begin, BK);
         for (int kb = 0; kb < nK; ++kb) {
           const int rk = r_begin + kb * BK;
@@ -798,7 +971,7 @@ dw_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
     for (int L = blockIdx.x; run && L < total; L += gridDim.x) {
       int e, mb, nb;
       coords(L, e, mb, nb);
-      const int r_begin = c.off[e], r_end = c.off[e + 1];
+      const int r_begin = x.off[e], r_end = x.off[e + 1];
       const int nK = cdiv(r_end - r_begin, BK);
       for (int kb0 = 0; run && kb0 < nK; kb0 += kIdxBatch) {
         int v[kIdxBatch][BK / 32];
@@ -815,8 +988,8 @@ dw_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
           if (!mbar_wait(&c.iempty[ri.s], ri.ph ^ 1, abort_flag, g.err)) { run = false; break; }
 #pragma unroll
           for (int q = 0; q < BK / 32; ++q) {
-            if (A_GATHER) c.idx[ri.s][0][lane + 32 * q] = src_of(v[b][q], a_shift, g.a_fan_out, g.a_rows);
-            if (B_GATHER) c.idx[ri.s][1][lane + 32 * q] = src_of(v[b][q], b_shift, g.b_fan_out, g.b_rows);
+            if (A_GATHER) x.idx[ri.s][0][lane + 32 * q] = src_of(v[b][q], a_shift, g.a_fan_out, g.a_rows);
+            if (B_GATHER) x.idx[ri.s][1][lane + 32 * q] = src_of(v[b][q], b_shift, g.b_fan_out, g.b_rows);
           }
           __syncwarp();
           if (lane == 0) mbar_arrive(&c.ifull[ri.s]);
@@ -837,19 +1010,19 @@ dw_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
     for (int L = blockIdx.x; run && L < total; L += gridDim.x) {
       int e, mb, nb;
       coords(L, e, mb, nb);
-      const int nK = cdiv(c.off[e + 1] - c.off[e], BK);
+      const int nK = cdiv(x.off[e + 1] - x.off[e], BK);
       for (int kb = 0; kb < nK; ++kb) {
         if (!mbar_wait(&c.ifull[ri.s], ri.ph, abort_flag, g.err)) { run = false; break; }
         if (A_GATHER) {
           if (!mbar_wait(&c.emptyA[ra.s], ra.ph ^ 1, abort_flag, g.err)) { run = false; break; }
-          ga.issue(smem_u32(sA + ra.s * A_BYTES), c.idx[ri.s][0], reinterpret_cast<const bf16*>(g.a),
+          ga.issue(smem_u32(sA + ra.s * A_BYTES), x.idx[ri.s][0], reinterpret_cast<const bf16*>(g.a),
                    g.lda, mb * BM, g.M, t);
           cp_async_arrive(&c.fullA[ra.s]);
           ra.next(SA);
         }
         if (B_GATHER) {
           if (!mbar_wait(&c.emptyB[rb.s], rb.ph ^ 1, abort_flag, g.err)) { run = false; break; }
-          gb.issue(smem_u32(sB + rb.s * B_BYTES), c.idx[ri.s][1], reinterpret_cast<const bf16*>(g.b),
+          gb.issue(smem_u32(sB + rb.s * B_BYTES), x.idx[ri.s][1], reinterpret_cast<const bf16*>(g.b),
                    g.ldb, nb * BN, g.N, t);
           cp_async_arrive(&c.fullB[rb.s]);
           rb.next(SB);
@@ -873,7 +1046,7 @@ dw_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
       for (int L = blockIdx.x; L < total; L += gridDim.x, ++it) {
         int e, mb, nb;
         coords(L, e, mb, nb);
-        const int r_begin = c.off[e], r_end = c.off[e + 1];
+        const int r_begin = x.off[e], r_end = x.off[e + 1];
         const int nK = cdiv(r_end - r_begin, BK);
         const int buf = it & 1;
         const uint32_t tph = (it >> 1) & 1;
@@ -933,7 +1106,7 @@ dw_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
     for (int L = blockIdx.x; L < total; L += gridDim.x, ++it) {
       int e, mb, nb;
       coords(L, e, mb, nb);
-      const int nrows = c.off[e + 1] - c.off[e];
+      const int nrows = x.off[e + 1] - x.off[e];
       const int buf = it & 1;
       const uint32_t tph = (it >> 1) & 1;
       if (!mbar_wait(&c.tfull[buf], tph, abort_flag, g.err)) break;
@@ -996,9 +1169,10 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// bf16 tensor map of rank 2 or 3, 128-byte swizzle; dims/strides innermost first.
+// bf16 tensor map of rank 2 or 3; dims/strides innermost first.
 cudaError_t make_map(CUtensorMap* m, const void* base, int rank, const uint64_t* dims,
-                     const uint64_t* strides_bytes, const uint32_t* box) {
+                     const uint64_t* strides_bytes, const uint32_t* box,
+                     CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return cudaErrorNotSupported;
   cuuint64_t d[3], s[2];
@@ -1006,7 +1180,7 @@ cudaError_t make_map(CUtensorMap* m, const void* base, int rank, const uint64_t*
   for (int i = 0; i < rank; ++i) { d[i] = dims[i]; b[i] = box[i]; }
   for (int i = 0; i < rank - 1; ++i) s[i] = strides_bytes[i];
   CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base), d, s, b, e,
-                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
@@ -1017,6 +1191,16 @@ cudaError_t rows_map(CUtensorMap* m, const void* base, int cols, int rows, int l
   const uint64_t strides[1] = {(uint64_t)ld * 2};
   const uint32_t box[2] = {64, box_rows};
   return make_map(m, base, 2, dims, strides, box);
+}
+
+// Output map of the grouped epilogue's boxed stores: rows of [rows, ld] whose
+// first parts * n_out columns hold `parts` blocks of n_out (SwiGLU's gate and up
+// halves), as dims {n_out, parts, rows} so that a box never crosses n_out.
+cudaError_t out_map(CUtensorMap* m, const void* base, int n_out, int parts, int rows, int ld) {
+  const uint64_t dims[3] = {(uint64_t)n_out, (uint64_t)parts, (uint64_t)rows};
+  const uint64_t strides[2] = {(uint64_t)n_out * 2, (uint64_t)ld * 2};
+  const uint32_t box[3] = {32, 1, 32};
+  return make_map(m, base, 3, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_64B);
 }
 
 int num_sms() {
@@ -1030,20 +1214,23 @@ int num_sms() {
   return n;
 }
 
-constexpr size_t kSmemBytes = 1024 + (size_t)kRingBytes + sizeof(SharedCtl);
-
 template <typename K>
-cudaError_t prep(K kern) {
-  return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
+cudaError_t prep(K kern, size_t bytes) {
+  return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
 }
 
+struct EpiMaps {
+  CUtensorMap out, out2, xa, xh;
+  int flags = 0;
+};
+
 template <bool AG, bool BK_, bool SW>
-cudaError_t launch_g(const CUtensorMap& ta, const CUtensorMap& tb, const GroupedGemm& g, int nN,
-                     int grid, cudaStream_t s) {
+cudaError_t launch_g(const CUtensorMap& ta, const CUtensorMap& tb, const EpiMaps& m,
+                     const GroupedGemm& g, int nN, int grid, cudaStream_t s) {
   auto kern = grouped_gemm_tc_kernel<AG, BK_, SW>;
-  cudaError_t e = prep(kern);
+  cudaError_t e = prep(kern, kGroupedSmem);
   if (e != cudaSuccess) return e;
-  kern<<<grid, kThreads, kSmemBytes, s>>>(ta, tb, g, nN);
+  kern<<<grid, kThreads, kGroupedSmem, s>>>(ta, tb, m.out, m.out2, m.xa, m.xh, g, nN, m.flags);
   return cudaGetLastError();
 }
 
@@ -1051,9 +1238,9 @@ template <bool AG, bool BG, bool TR>
 cudaError_t launch_d(const CUtensorMap& ta, const CUtensorMap& tb, const DwGemm& g, int nM, int nN,
                      int grid, cudaStream_t s) {
   auto kern = dw_gemm_tc_kernel<AG, BG, TR>;
-  cudaError_t e = prep(kern);
+  cudaError_t e = prep(kern, kDwSmem);
   if (e != cudaSuccess) return e;
-  kern<<<grid, kDwThreads, kSmemBytes, s>>>(ta, tb, g, nM, nN);
+  kern<<<grid, kDwThreads, kDwSmem, s>>>(ta, tb, g, nM, nN);
   return cudaGetLastError();
 }
 
@@ -1091,18 +1278,30 @@ cudaError_t launch_grouped_gemm_tc(const GroupedGemm& g, cudaStream_t s) {
     e = make_map(&tb, g.b, 3, dims, str, box);
   }
   if (e != cudaSuccess) return e;
+  // Boxed (TMA tensor) epilogue stores when every output is bf16 in grouped
+  // rows; boxed ACT_BWD input loads when its inputs are in grouped rows.
+  EpiMaps m;
+  memset(&m, 0, sizeof(m));
+  const int parts = (g.act == SMOE_ACT_SWIGLU && g.epi != EPI_STORE) ? 2 : 1;
+  bool st = (g.out != nullptr || g.out2 != nullptr) &&
+            (g.out == nullptr || (!g.out_f32 && g.out_mode == ROWS_GROUPED));
+  if (st && g.out && out_map(&m.out, g.out, g.n_out, parts, g.num_rows, g.ldo) != cudaSuccess) st = false;
+  if (st && g.out2 && out_map(&m.out2, g.out2, g.n_out, 1, g.num_rows, g.ldo2) != cudaSuccess) st = false;
+  const bool need_h = g.out != nullptr && g.act != SMOE_ACT_NONE;
+  bool ld = g.epi == EPI_ACT_BWD && g.aux_a_mode == ROWS_GROUPED && !swiglu;
+  if (ld && out_map(&m.xa, g.aux_a, g.n_out, 1, g.num_rows, g.ld_aux_a) != cudaSuccess) ld = false;
+  if (ld && need_h && out_map(&m.xh, g.aux_h, g.n_out, parts, g.num_rows, g.ld_aux_h) != cudaSuccess) ld = false;
+  m.flags = (st ? kBoxStores : 0) | (ld ? kBoxLoads : 0);
   const long long tiles = (long long)(cdiv(g.num_rows, BM) + g.E) * nN;
   const int grid = (int)(tiles < num_sms() ? tiles : num_sms());
+#define SMOE_LAUNCH_G(AG, KM, SW) launch_g<AG, KM, SW>(ta, tb, m, g, nN, grid, s)
   if (gather) {
-    if (kmaj) return swiglu ? launch_g<true, true, true>(ta, tb, g, nN, grid, s)
-                            : launch_g<true, true, false>(ta, tb, g, nN, grid, s);
-    return swiglu ? launch_g<true, false, true>(ta, tb, g, nN, grid, s)
-                  : launch_g<true, false, false>(ta, tb, g, nN, grid, s);
+    if (kmaj) return swiglu ? SMOE_LAUNCH_G(true, true, true) : SMOE_LAUNCH_G(true, true, false);
+    return swiglu ? SMOE_LAUNCH_G(true, false, true) : SMOE_LAUNCH_G(true, false, false);
   }
-  if (kmaj) return swiglu ? launch_g<false, true, true>(ta, tb, g, nN, grid, s)
-                          : launch_g<false, true, false>(ta, tb, g, nN, grid, s);
-  return swiglu ? launch_g<false, false, true>(ta, tb, g, nN, grid, s)
-                : launch_g<false, false, false>(ta, tb, g, nN, grid, s);
+  if (kmaj) return swiglu ? SMOE_LAUNCH_G(false, true, true) : SMOE_LAUNCH_G(false, true, false);
+  return swiglu ? SMOE_LAUNCH_G(false, false, true) : SMOE_LAUNCH_G(false, false, false);
+#undef SMOE_LAUNCH_G
 }
 
 cudaError_t launch_dw_gemm_tc(const DwGemm& g_in, cudaStream_t s) {

@@ -72,9 +72,6 @@ struct DwGemm {
   unsigned* err = nullptr;
 };
 
-// Column-tile width that the ACT_BWD dg partials are laid out in, per dtype.
-int dg_tile_cols(smoe_dtype dt);
-
 // ---- launchers (return a cudaError_t from the launch) ----------------------
 cudaError_t launch_route(const void* x, const void* w_r, const float* b_r, int T, int d, int E,
                          int k, smoe_dtype dt, int32_t* idx, float* gates, unsigned* err,
@@ -92,10 +89,14 @@ size_t sort_workspace_bytes(int T, int k, int E);
 cudaError_t launch_sort(const int32_t* idx, int T, int k, int E, int32_t* sorted_slot,
                         int32_t* offsets, void* ws, unsigned* err, cudaStream_t s);
 
-// out[t] = sum_{j<ck} ws[t*ck + j] (+ sum_j dl[t*ck+j] * W_r[:, idx[t*ck+j]] if dl)
+// out[t] = sum_{j<ck} ws[t*ck + j] (+ sum_j dl[t*ck+j] * w_rt[idx[t*ck+j], :] if dl),
+// w_rt being the router weight transposed to [E, N]
 cudaError_t launch_combine(const float* ws, int T, int ck, int N, void* out, smoe_dtype out_dt,
-                           const float* dl, const int32_t* idx, const void* w_r, int E,
+                           const float* dl, const int32_t* idx, const void* w_rt, int E,
                            cudaStream_t s);
+// w_rt[e][i] = w_r[i][e]
+cudaError_t launch_transpose_wr(const void* w_r, int d, int E, smoe_dtype dt, void* w_rt,
+                                cudaStream_t s);
 // dg[sorted_slot[i]] = sum_{c < n_tiles} partial[i*ld + c]
 cudaError_t launch_dg_reduce(const float* partial, int ld, int n_tiles, const int32_t* sorted_slot,
                              int num_rows, float* dg, cudaStream_t s);
