@@ -136,6 +136,25 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, u
       "l"((uint64_t)map), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2)
       : "memory");
 }
+// The same loads for a CTA pair: the data lands in this CTA's shared memory and
+// the transaction bytes count on the barrier at cluster address `bar_cl`, which
+// may belong to the other CTA of the pair.
+__device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* map, uint32_t bar_cl,
+                                                 int c0, int c1) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
+      "l"((uint64_t)map), "r"(bar_cl), "r"(c0), "r"(c1)
+      : "memory");
+}
+__device__ __forceinline__ void tma_load_3d_pair(void* dst, const CUtensorMap* map, uint32_t bar_cl,
+                                                 int c0, int c1, int c2) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(smem_u32(dst)),
+      "l"((uint64_t)map), "r"(bar_cl), "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
+}
 // 16-byte asynchronous copy global -> shared through L2 only; src_bytes = 0
 // writes zeros without reading the source.
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
@@ -208,6 +227,61 @@ __device__ __forceinline__ void umma_commit(uint64_t* bar) {
           smem_u32(bar))
       : "memory");
 }
+// ---- CTA pairs: a cluster of two CTAs sharing one M = 256 MMA (cta_group::2).
+// CTA v of the pair holds rows [128 v, 128 v + 128) of A and columns
+// [N/2 v, N/2 (v + 1)) of B in its shared memory, and its 128 rows of the
+// accumulator (all N columns) in its tensor memory.
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+// Address in the cluster's shared window of the counterpart of `p` in CTA `rank`.
+__device__ __forceinline__ uint32_t peer_addr(const void* p, uint32_t rank) {
+  uint32_t a;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(a) : "r"(smem_u32(p)), "r"(rank));
+  return a;
+}
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::
+                   : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cl_addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cl_addr) : "memory");
+}
+// Relaxed remote arrive: for a relay that itself wrote nothing the other CTA
+// reads (a release at cluster scope costs a memory barrier per arrival).
+__device__ __forceinline__ void mbar_arrive_cluster_relaxed(uint32_t cl_addr) {
+  asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(cl_addr) : "memory");
+}
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t* slot, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                   smem_u32(slot)),
+               "r"(ncols)
+               : "memory");
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void umma_bf16_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                               uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// Arrive on the barrier at cluster address `cl_addr` (either CTA of the pair)
+// once this thread's earlier pair MMAs have completed.
+__device__ __forceinline__ void umma_commit_pair(uint32_t cl_addr) {
+  asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                   cl_addr)
+               : "memory");
+}
+
 // 32 consecutive fp32 columns of this thread's tensor-memory lane.
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
   uint32_t r[32];
@@ -311,6 +385,7 @@ struct SharedCtl {
   uint64_t fullA[kMaxStages], emptyA[kMaxStages];
   uint64_t fullB[kMaxStages], emptyB[kMaxStages];
   uint64_t tfull[2], tempty[2];
+  uint64_t pfull[kMaxStages];   // pair leader: the other CTA's stage s has landed
   uint64_t ifull[IDX_STAGES];   // index ring: written by warp 2
   uint64_t iempty[IDX_STAGES];  // index ring: released by the 4 gather warps
   uint64_t ebar[4];             // per epilogue warp: its input boxes have landed
@@ -341,10 +416,19 @@ constexpr int kWarpStaging = 32 * kSlotBytes;  // 13 x 512: boxes stay 512-byte 
 static_assert(3 * kBoxBytes <= kWarpStaging && kWarpStaging % 512 == 0, "staging layout");
 constexpr int kStagingBytes = 4 * kWarpStaging;
 enum : int { kBoxStores = 1, kBoxLoads = 2 };  // grouped-epilogue box modes (launch flags)
+// Grouped-M GEMMs run as CTA pairs sharing M = 256 MMAs (cta_group::2).
+#ifndef SMOE_PAIR_M
+#define SMOE_PAIR_M 0
+#endif
+constexpr bool kPairM = SMOE_PAIR_M != 0;
 
 constexpr size_t kCtlBytes = (sizeof(SharedCtl) + 1023) / 1024 * 1024;
 constexpr size_t kGroupedSmem = 1024 + (size_t)kRingBytes + kCtlBytes + kStagingBytes;
-constexpr size_t kDwSmem = 1024 + (size_t)kRingBytes + kCtlBytes + sizeof(DwExtra);
+// dW kernel: after DwExtra, one 4 KB fp32 box (32 x 32, 128-byte swizzle) per
+// epilogue warp, written out by a TMA tensor store per 32-column chunk.
+constexpr size_t kDwExtraBytes = (sizeof(DwExtra) + 1023) / 1024 * 1024;
+constexpr int kDwBoxBytes = 32 * 32 * 4;
+constexpr size_t kDwSmem = 1024 + (size_t)kRingBytes + kCtlBytes + kDwExtraBytes + 4 * kDwBoxBytes;
 static_assert(kGroupedSmem <= 232448 && kDwSmem <= 232448, "shared memory exceeds 227 KB");
 
 // Position in a ring of n stages and the parity of the current lap.
@@ -362,8 +446,10 @@ struct Tile {
 
 // linear tile L -> (expert, M tile, N tile); expert-major, then N tile, then M tile.
 // `off` = the expert offsets in global memory (validated by setup).
+// A pair's M tile spans 2 BM rows, of which CTA `rank` takes the rank-th BM.
+template <bool PAIR = false>
 __device__ __forceinline__ Tile map_tile(const SharedCtl& c, const int32_t* off, int E, int nN,
-                                         int L) {
+                                         int L, int rank = 0) {
   int lo = 0, hi = E - 1;  // largest e with prefix[e] * nN <= L
   while (lo < hi) {
     const int mid = (lo + hi + 1) >> 1;
@@ -375,7 +461,7 @@ __device__ __forceinline__ Tile map_tile(const SharedCtl& c, const int32_t* off,
   const int lp = L - c.prefix[lo] * nN;
   t.nb = lp / mt;
   t.mb = lp % mt;
-  t.row0 = __ldg(off + lo) + t.mb * BM;
+  t.row0 = __ldg(off + lo) + t.mb * (PAIR ? 2 * BM : BM) + rank * BM;
   t.row_end = __ldg(off + lo + 1);
   return t;
 }
@@ -384,7 +470,7 @@ __device__ __forceinline__ Tile map_tile(const SharedCtl& c, const int32_t* off,
 // copied to off_copy when given).
 // a_arrivals / b_arrivals: producer arrivals per full stage (1 for TMA, the
 // gather threads' cp.async arrivals otherwise).
-template <int SA, int SB>
+template <int SA, int SB, bool PAIR = false>
 __device__ __forceinline__ void setup(SharedCtl& c, const int32_t* offsets, int E, int num_rows,
                                       unsigned* err, uint32_t a_arrivals, uint32_t b_arrivals,
                                       uint32_t gather_warps, int* off_copy,
@@ -394,6 +480,7 @@ __device__ __forceinline__ void setup(SharedCtl& c, const int32_t* offsets, int 
     for (int s = 0; s < SA; ++s) {
       mbar_init(&c.fullA[s], a_arrivals);
       mbar_init(&c.emptyA[s], 1);
+      mbar_init(&c.pfull[s], 1);
     }
     for (int s = 0; s < SB; ++s) {
       mbar_init(&c.fullB[s], b_arrivals);
@@ -401,7 +488,7 @@ __device__ __forceinline__ void setup(SharedCtl& c, const int32_t* offsets, int 
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&c.tfull[b], 1);
-      mbar_init(&c.tempty[b], epilogue_warps);
+      mbar_init(&c.tempty[b], epilogue_warps * (PAIR ? 2 : 1));  // a pair's leader: both CTAs' warps
     }
     for (int b = 0; b < IDX_STAGES; ++b) {
       mbar_init(&c.ifull[b], 1);
@@ -411,7 +498,10 @@ __device__ __forceinline__ void setup(SharedCtl& c, const int32_t* offsets, int 
     c.abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 1) tmem_alloc(&c.tmem_base, kTmemCols);
+  if (warp == 1) {
+    if (PAIR) tmem_alloc_pair(&c.tmem_base, kTmemCols);
+    else tmem_alloc(&c.tmem_base, kTmemCols);
+  }
   for (int e = threadIdx.x; e <= E; e += blockDim.x) {  // raw offsets first
     const int o = offsets[e];
     c.prefix[e] = o;
@@ -427,7 +517,8 @@ __device__ __forceinline__ void setup(SharedCtl& c, const int32_t* offsets, int 
       const int n = cur - prev;
       prev = cur;
       if (n < 0) ok = false;
-      c.prefix[e + 1] = c.prefix[e] + (n > 0 ? (n + BM - 1) / BM : 0);
+      constexpr int TR = PAIR ? 2 * BM : BM;
+      c.prefix[e + 1] = c.prefix[e] + (n > 0 ? (n + TR - 1) / TR : 0);
     }
     if (!ok) {  // inconsistent offsets: do nothing rather than read out of range
       report_error(err, ERRBIT_DATA);
@@ -438,12 +529,14 @@ __device__ __forceinline__ void setup(SharedCtl& c, const int32_t* offsets, int 
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  if (PAIR) cluster_sync();  // both CTAs' barriers exist before either arrives remotely
 }
 
 // On an abort some copies (cp.async, TMA) and tensor-core operations may still
 // be in flight: each thread retires its own cp.async copies, then the CTA waits
 // a bounded 2 ms (far above any copy or MMA latency) before freeing tensor memory
 // and exiting, so nothing lands in a CTA that has gone.
+template <bool PAIR = false>
 __device__ __forceinline__ void teardown(SharedCtl& c) {
   asm volatile("cp.async.wait_all;" ::: "memory");
   __syncthreads();
@@ -455,13 +548,18 @@ __device__ __forceinline__ void teardown(SharedCtl& c) {
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if ((threadIdx.x >> 5) == 1) tmem_dealloc(c.tmem_base, kTmemCols);
+  // a pair: neither CTA leaves while the other may still arrive on its barriers
+  if (PAIR) cluster_sync();
+  if ((threadIdx.x >> 5) == 1) {
+    if (PAIR) tmem_dealloc_pair(c.tmem_base, kTmemCols);
+    else tmem_dealloc(c.tmem_base, kTmemCols);
+  }
 }
 
 // ---------------------------------------------------------------------------
 // Grouped-M kernel
 // ---------------------------------------------------------------------------
-template <bool A_GATHER, bool B_KMAJOR, bool SWIGLU_FWD>
+template <bool A_GATHER, bool B_KMAJOR, bool SWIGLU_FWD, bool PAIR>
 __global__ void __launch_bounds__(kThreads, 1)
 grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
                        const __grid_constant__ CUtensorMap tmB,
@@ -472,9 +570,12 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
                        int box_flags) {
   // One ring of STAGES stages holds A and B together (fullA/emptyA guard a whole
   // stage): measured faster here than separate rings, whose second wait and
-  // commit per stage cost more than their extra depth returned.
-  constexpr int STAGES = 4;
-  static_assert(STAGES * (A_BYTES + B_BYTES) <= kRingBytes, "stage ring exceeds its budget");
+  // commit per stage cost more than their extra depth returned.  A pair's CTA
+  // holds half of B per stage, so its ring is deeper.
+  constexpr int BSTAGE = PAIR ? B_BYTES / 2 : B_BYTES;
+  constexpr int STAGES = PAIR ? 6 : 4;
+  static_assert(STAGES * (A_BYTES + BSTAGE) <= kRingBytes, "stage ring exceeds its budget");
+  static_assert(STAGES <= kMaxStages, "too many stages");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
   uint8_t* sA = smem;
@@ -482,9 +583,17 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
   SharedCtl& c = *reinterpret_cast<SharedCtl*>(smem + kRingBytes);
   volatile int* abort_flag = &c.abort_flag;
 
-  setup<STAGES, 0>(c, g.offsets, g.E, g.num_rows, g.err, 1 + (A_GATHER ? kGatherThreads : 0), 1,
-                   kGatherThreads / 32, nullptr);
+  // a pair walks the tile list as one unit; rank 0 issues the MMAs.  Arrivals
+  // on a stage's full barrier: the producer's expect-tx and the gather threads;
+  // at a pair's rank 1 only its gather threads (relayed to the leader).
+  const int rank = PAIR ? (int)cluster_rank() : 0;
+  const uint32_t full_arrivals =
+      (rank == 0 ? 1u : 0u) + (A_GATHER ? (uint32_t)kGatherThreads : 0u);
+  setup<STAGES, 0, PAIR>(c, g.offsets, g.E, g.num_rows, g.err, full_arrivals > 0 ? full_arrivals : 1u,
+                         1, kGatherThreads / 32, nullptr);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int first = PAIR ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
+  const int stride = PAIR ? (int)(gridDim.x >> 1) : (int)gridDim.x;
   const int total = c.total_mtiles * nN;
   const int nK = cdiv(g.K, BK);
   constexpr int BNo = SWIGLU_FWD ? BN / 2 : BN;  // logical output columns per tile
@@ -494,24 +603,36 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
     if (lane == 0) {
       Ring r;
       bool run = true;
-      for (int L = blockIdx.x; run && L < total; L += gridDim.x) {
-        const Tile t = map_tile(c, g.offsets, g.E, nN, L);
+      for (int L = first; run && L < total; L += stride) {
+        const Tile t = map_tile<PAIR>(c, g.offsets, g.E, nN, L, rank);
         for (int kb = 0; kb < nK; ++kb) {
           if (!mbar_wait(&c.emptyA[r.s], r.ph ^ 1, abort_flag, g.err)) { run = false; break; }
-          uint8_t* b_dst = sB + r.s * B_BYTES;
-          mbar_expect_tx(&c.fullA[r.s], B_BYTES + (A_GATHER ? 0 : A_BYTES));
-          if (!A_GATHER) tma_load_2d(sA + r.s * A_BYTES, &tmA, &c.fullA[r.s], kb * BK, t.row0);
-          if (B_KMAJOR) {
-            tma_load_3d(b_dst, &tmB, &c.fullA[r.s], kb * BK, t.nb * BN, t.e);
+          uint8_t* b_dst = sB + r.s * BSTAGE;
+          // a pair: both CTAs' TMA bytes count on the leader's barrier, whose
+          // producer expects them all
+          const uint32_t full_cl = PAIR ? peer_addr(&c.fullA[r.s], 0) : 0u;
+          auto load2 = [&](void* dst, const CUtensorMap* m, int c0, int c1) {
+            if (PAIR) tma_load_2d_pair(dst, m, full_cl, c0, c1);
+            else tma_load_2d(dst, m, &c.fullA[r.s], c0, c1);
+          };
+          auto load3 = [&](void* dst, const CUtensorMap* m, int c0, int c1, int c2) {
+            if (PAIR) tma_load_3d_pair(dst, m, full_cl, c0, c1, c2);
+            else tma_load_3d(dst, m, &c.fullA[r.s], c0, c1, c2);
+          };
+          if (rank == 0)
+            mbar_expect_tx(&c.fullA[r.s], (PAIR ? 2 : 1) * (BSTAGE + (A_GATHER ? 0 : A_BYTES)));
+          if (!A_GATHER) load2(sA + r.s * A_BYTES, &tmA, kb * BK, t.row0);
+          if (B_KMAJOR) {  // rows of W[e] = output columns; a pair's CTA takes its half
+            load3(b_dst, &tmB, kb * BK, t.nb * BN + (PAIR ? rank * (BN / 2) : 0), t.e);
           } else {
+            // 64-column slabs; SwiGLU's tile is BNo gate columns then BNo up columns
+            // (a pair: the gate half in CTA 0, the up half in CTA 1)
 #pragma unroll
-            for (int q = 0; q < BN / 64; ++q) {
-              int col;
-              if (SWIGLU_FWD)
-                col = (q < BN / 128) ? t.nb * BNo + 64 * q : g.n_out + t.nb * BNo + 64 * (q - BN / 128);
-              else
-                col = t.nb * BN + 64 * q;
-              tma_load_3d(b_dst + q * (64 * BK * 2), &tmB, &c.fullA[r.s], col, kb * BK, t.e);
+            for (int q = 0; q < BSTAGE / (64 * BK * 2); ++q) {
+              const int lc = (PAIR ? rank * (BN / 2) : 0) + 64 * q;  // column within the B tile
+              const int col = SWIGLU_FWD ? (lc < BNo ? t.nb * BNo + lc : g.n_out + t.nb * BNo + lc - BNo)
+                                         : t.nb * BN + lc;
+              load3(b_dst + q * (64 * BK * 2), &tmB, col, kb * BK, t.e);
             }
           }
           r.next(STAGES);
@@ -530,8 +651,8 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
     const bf16* A = reinterpret_cast<const bf16*>(g.a);
     Ring r;
     bool run = true;
-    for (int L = blockIdx.x; run && L < total; L += gridDim.x) {
-      const Tile tl = map_tile(c, g.offsets, g.E, nN, L);
+    for (int L = first; run && L < total; L += stride) {
+      const Tile tl = map_tile<PAIR>(c, g.offsets, g.E, nN, L, rank);
       const bf16* src[kRowsPer];
       uint32_t ok_rows = 0;
 #pragma unroll
@@ -563,12 +684,27 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
       }
     }
   } else if (warp == 1) {
-    // ---------------- MMA issuer ----------------
-    if (lane == 0) {
-      constexpr uint32_t idesc = idesc_bf16(BM, BN, 0, B_KMAJOR ? 0 : 1);
+    // ---------------- MMA issuer (a pair: rank 0; rank 1 relays its stages) ----------------
+    if (lane == 0 && PAIR && rank == 1) {
+      // the leader's MMAs read this CTA's half of each stage: its TMA bytes count
+      // on the leader's barrier directly; its gathered rows are relayed from here
+      if (A_GATHER) {
+        Ring r;
+        bool run = true;
+        for (int L = first; run && L < total; L += stride) {
+          for (int kb = 0; kb < nK; ++kb) {
+            if (!mbar_wait(&c.fullA[r.s], r.ph, abort_flag, g.err)) { run = false; break; }
+            fence_proxy_async();  // rows written by cp.async, read by the tensor core
+            mbar_arrive_cluster_relaxed(peer_addr(&c.pfull[r.s], 0));
+            r.next(STAGES);
+          }
+        }
+      }
+    } else if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16(PAIR ? 2 * BM : BM, BN, 0, B_KMAJOR ? 0 : 1);
       Ring r;
       int it = 0;
-      for (int L = blockIdx.x; L < total; L += gridDim.x, ++it) {
+      for (int L = first; L < total; L += stride, ++it) {
         const int buf = it & 1;
         const uint32_t tph = (it >> 1) & 1;
         if (!mbar_wait(&c.tempty[buf], tph ^ 1, abort_flag, g.err)) break;
@@ -577,21 +713,33 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
         bool ok = true;
         for (int kb = 0; kb < nK; ++kb) {
           if (!mbar_wait(&c.fullA[r.s], r.ph, abort_flag, g.err)) { ok = false; break; }
+          if (PAIR && A_GATHER && !mbar_wait(&c.pfull[r.s], r.ph, abort_flag, g.err)) { ok = false; break; }
           tc_fence_after();
           if (A_GATHER) fence_proxy_async();  // rows written by cp.async, read by the tensor core
           const uint32_t a_addr = smem_u32(sA + r.s * A_BYTES);
-          const uint32_t b_addr = smem_u32(sB + r.s * B_BYTES);
+          const uint32_t b_addr = smem_u32(sB + r.s * BSTAGE);
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk) {
             const uint64_t ad = desc_kmajor(a_addr + kk * 32);
             const uint64_t bd = B_KMAJOR ? desc_kmajor(b_addr + kk * 32) : desc_mnmajor(b_addr + kk * 2048);
-            umma_bf16(d_tmem, ad, bd, idesc, (kb | kk) != 0);
+            if (PAIR) umma_bf16_pair(d_tmem, ad, bd, idesc, (kb | kk) != 0);
+            else umma_bf16(d_tmem, ad, bd, idesc, (kb | kk) != 0);
           }
-          umma_commit(&c.emptyA[r.s]);
+          if (PAIR) {  // the stage is free in both CTAs
+            umma_commit_pair(smem_u32(&c.emptyA[r.s]));
+            umma_commit_pair(peer_addr(&c.emptyA[r.s], 1));
+          } else {
+            umma_commit(&c.emptyA[r.s]);
+          }
           r.next(STAGES);
         }
         if (!ok) break;
-        umma_commit(&c.tfull[buf]);
+        if (PAIR) {
+          umma_commit_pair(smem_u32(&c.tfull[buf]));
+          umma_commit_pair(peer_addr(&c.tfull[buf], 1));
+        } else {
+          umma_commit(&c.tfull[buf]);
+        }
       }
     }
     __syncwarp();
@@ -600,11 +748,13 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
     // Thread r owns accumulator row r.  Per 32-column chunk the warp stages its
     // rows' output segments in shared memory and hands them to the TMA engine:
     // one tensor store per output box when its 32 rows are consecutive rows of
-    // the expert's slice (o_tma), else one bulk copy per row.  Plain stores from
-    // the tensor-memory row layout would make every 16-byte access of a warp
-    // touch 32 lines and compete with the cp.async row gathers for the same
-    // unit.  ACT_BWD's per-row inputs stay 16-byte loads issued before the
-    // accumulator read: per-row bulk loads of 64 bytes measured far slower.
+    // the expert's slice (kBoxStores), else one bulk copy per row.  Plain stores
+    // from the tensor-memory row layout would make every 16-byte access of a
+    // warp touch 32 lines and compete with the cp.async row gathers for the same
+    // unit.  ACT_BWD reads its A and H inputs the same way, as boxes of the
+    // warp's rows (kBoxLoads), when they are in grouped order, else by 16-byte
+    // loads issued before the accumulator read (per-row bulk loads of 64 bytes
+    // measured far slower).
     const int q = warp - 4;  // tensor-memory lane quadrant
     const int r = q * 32 + lane;
     uint8_t* wstage = smem + kRingBytes + kCtlBytes + q * kWarpStaging;
@@ -620,10 +770,10 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
     const bool need_h = act_bwd && g.out != nullptr && g.act != SMOE_ACT_NONE;
     uint32_t eph = 0;  // phase of this warp's input-box barrier
     int it = 0;
-    for (int L = blockIdx.x; L < total; L += gridDim.x, ++it) {
+    for (int L = first; L < total; L += stride, ++it) {
       const int buf = it & 1;
       const uint32_t tph = (it >> 1) & 1;
-      const Tile t = map_tile(c, g.offsets, g.E, nN, L);
+      const Tile t = map_tile<PAIR>(c, g.offsets, g.E, nN, L, rank);
       if (!mbar_wait(&c.tfull[buf], tph, abort_flag, g.err)) break;
       tc_fence_after();
       const int i = t.row0 + r;
@@ -830,11 +980,14 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
         g.dg_partial[(size_t)i * g.dg_ld + t.nb] = dg_acc;
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&c.tempty[buf]);
+      if (lane == 0) {  // the accumulator buffer is free (a pair: at the leader)
+        if (PAIR && rank == 1) mbar_arrive_cluster(peer_addr(&c.tempty[buf], 0));
+        else mbar_arrive(&c.tempty[buf]);
+      }
     }
     bulk_wait_all();
   }
-  teardown(c);
+  teardown<PAIR>(c);
 }
 
 // ---------------------------------------------------------------------------
@@ -890,7 +1043,8 @@ struct SlabGather {
 template <bool A_GATHER, bool B_GATHER, bool TRANS_OUT>
 __global__ void __launch_bounds__(kDwThreads, 1)
 dw_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                  const DwGemm g, int nM, int nN) {
+                  const __grid_constant__ CUtensorMap tmD, const DwGemm g, int nM, int nN,
+                  int d_boxed) {
   constexpr bool kOneGather = A_GATHER && !B_GATHER;
   constexpr int SA = kOneGather ? 6 : 4, SB = kOneGather ? 3 : 4;
   static_assert(SA * A_BYTES + SB * B_BYTES <= kRingBytes, "stage rings exceed their budget");
@@ -1100,8 +1254,13 @@ dw_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
     __syncwarp();
   } else if (warp >= 4 && warp < 8) {
     // ---------------- epilogue: one accumulator row per thread ----------------
+    // d_boxed: per 32-column chunk the warp writes its 32 x 32 fp32 block into a
+    // 128-byte-swizzled box (transposed for TRANS_OUT) that one TMA tensor store
+    // writes out, clipped to dW's bounds; else plain stores.
     const int q = warp - 4;
     const int r = q * 32 + lane;
+    uint8_t* box = smem + kRingBytes + kCtlBytes + kDwExtraBytes + q * kDwBoxBytes;
+    const uint32_t box_s = smem_u32(box);
     int it = 0;
     for (int L = blockIdx.x; L < total; L += gridDim.x, ++it) {
       int e, mb, nb;
@@ -1121,6 +1280,29 @@ dw_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
         } else {
 #pragma unroll
           for (int j = 0; j < 32; ++j) v[j] = 0.0f;
+        }
+        if (d_boxed) {
+          if (nb * BN + c0 >= g.N) break;  // warp-uniform
+          if (lane == 0) bulk_wait_read();  // the previous chunk's store has read the box
+          __syncwarp();
+          if (TRANS_OUT) {  // box[n][m]: row j = column n, lane = m
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              *reinterpret_cast<float*>(box + j * 128 + ((((lane >> 2) ^ (j & 7))) << 4) + ((lane & 3) << 2)) = v[j];
+          } else {  // box[m][n]: row lane = m
+#pragma unroll
+            for (int j4 = 0; j4 < 8; ++j4)
+              *reinterpret_cast<float4*>(box + lane * 128 + ((j4 ^ (lane & 7)) << 4)) =
+                  make_float4(v[4 * j4], v[4 * j4 + 1], v[4 * j4 + 2], v[4 * j4 + 3]);
+          }
+          fence_proxy_async();
+          __syncwarp();
+          if (lane == 0) {
+            if (TRANS_OUT) tma_store_3d(&tmD, box_s, mb * BM + q * 32, nb * BN + c0, e);
+            else tma_store_3d(&tmD, box_s, nb * BN + c0, mb * BM + q * 32, e);
+            bulk_commit();
+          }
+          continue;
         }
         if (m >= g.M) continue;
         if (TRANS_OUT) {  // dW[e][n][m]: lanes hold consecutive m -> 128-byte lines
@@ -1145,6 +1327,7 @@ dw_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
       __syncwarp();
       if (lane == 0) mbar_arrive(&c.tempty[buf]);
     }
+    if (lane == 0) bulk_wait_all();
   }
   teardown(c);
 }
@@ -1172,14 +1355,15 @@ EncodeTiledFn encode_fn() {
 // bf16 tensor map of rank 2 or 3; dims/strides innermost first.
 cudaError_t make_map(CUtensorMap* m, const void* base, int rank, const uint64_t* dims,
                      const uint64_t* strides_bytes, const uint32_t* box,
-                     CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B) {
+                     CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B,
+                     CUtensorMapDataType dtype = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return cudaErrorNotSupported;
   cuuint64_t d[3], s[2];
   cuuint32_t b[3], e[3] = {1, 1, 1};
   for (int i = 0; i < rank; ++i) { d[i] = dims[i]; b[i] = box[i]; }
   for (int i = 0; i < rank - 1; ++i) s[i] = strides_bytes[i];
-  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base), d, s, b, e,
+  CUresult r = fn(m, dtype, rank, const_cast<void*>(base), d, s, b, e,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
@@ -1224,23 +1408,56 @@ struct EpiMaps {
   int flags = 0;
 };
 
+// Persistent grid over `tiles` tiles: one CTA per SM, or for pairs as many
+// 2-CTA clusters as the device can hold at once (fewer than half the SMs when a
+// GPC has an odd number of free SMs; a cluster beyond that would run its whole
+// share of the tile list after the others).
 template <bool AG, bool BK_, bool SW>
 cudaError_t launch_g(const CUtensorMap& ta, const CUtensorMap& tb, const EpiMaps& m,
-                     const GroupedGemm& g, int nN, int grid, cudaStream_t s) {
-  auto kern = grouped_gemm_tc_kernel<AG, BK_, SW>;
+                     const GroupedGemm& g, int nN, long long tiles, cudaStream_t s) {
+  auto kern = grouped_gemm_tc_kernel<AG, BK_, SW, kPairM>;
   cudaError_t e = prep(kern, kGroupedSmem);
   if (e != cudaSuccess) return e;
-  kern<<<grid, kThreads, kGroupedSmem, s>>>(ta, tb, m.out, m.out2, m.xa, m.xh, g, nN, m.flags);
+  if (!kPairM) {
+    const int grid = (int)(tiles < num_sms() ? tiles : num_sms());
+    kern<<<grid, kThreads, kGroupedSmem, s>>>(ta, tb, m.out, m.out2, m.xa, m.xh, g, nN, m.flags);
+    return cudaGetLastError();
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(num_sms() & ~1), 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = kGroupedSmem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  static int max_clusters = 0;  // per instantiation
+  if (max_clusters <= 0) {
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n <= 0) {
+      (void)cudaGetLastError();
+      n = num_sms() / 2;
+    }
+    max_clusters = n;
+  }
+  const long long pairs = tiles < max_clusters ? tiles : max_clusters;
+  cfg.gridDim = dim3((unsigned)(2 * pairs), 1, 1);
+  e = cudaLaunchKernelEx(&cfg, kern, ta, tb, m.out, m.out2, m.xa, m.xh, g, nN, m.flags);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
 template <bool AG, bool BG, bool TR>
-cudaError_t launch_d(const CUtensorMap& ta, const CUtensorMap& tb, const DwGemm& g, int nM, int nN,
-                     int grid, cudaStream_t s) {
+cudaError_t launch_d(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& td,
+                     int d_boxed, const DwGemm& g, int nM, int nN, int grid, cudaStream_t s) {
   auto kern = dw_gemm_tc_kernel<AG, BG, TR>;
   cudaError_t e = prep(kern, kDwSmem);
   if (e != cudaSuccess) return e;
-  kern<<<grid, kDwThreads, kDwSmem, s>>>(ta, tb, g, nM, nN);
+  kern<<<grid, kDwThreads, kDwSmem, s>>>(ta, tb, td, g, nM, nN, d_boxed);
   return cudaGetLastError();
 }
 
@@ -1269,7 +1486,7 @@ cudaError_t launch_grouped_gemm_tc(const GroupedGemm& g, cudaStream_t s) {
   if (kmaj) {  // W[e] is [NW, K]: dims {K, NW, E}
     const uint64_t dims[3] = {(uint64_t)g.K, (uint64_t)g.NW, (uint64_t)g.E};
     const uint64_t str[2] = {(uint64_t)g.K * 2, (uint64_t)g.NW * g.K * 2};
-    const uint32_t box[3] = {64, BN, 1};
+    const uint32_t box[3] = {64, kPairM ? BN / 2 : BN, 1};
     e = make_map(&tb, g.b, 3, dims, str, box);
   } else {  // W[e] is [K, NW]: dims {NW, K, E}
     const uint64_t dims[3] = {(uint64_t)g.NW, (uint64_t)g.K, (uint64_t)g.E};
@@ -1292,9 +1509,9 @@ cudaError_t launch_grouped_gemm_tc(const GroupedGemm& g, cudaStream_t s) {
   if (ld && out_map(&m.xa, g.aux_a, g.n_out, 1, g.num_rows, g.ld_aux_a) != cudaSuccess) ld = false;
   if (ld && need_h && out_map(&m.xh, g.aux_h, g.n_out, parts, g.num_rows, g.ld_aux_h) != cudaSuccess) ld = false;
   m.flags = (st ? kBoxStores : 0) | (ld ? kBoxLoads : 0);
-  const long long tiles = (long long)(cdiv(g.num_rows, BM) + g.E) * nN;
-  const int grid = (int)(tiles < num_sms() ? tiles : num_sms());
-#define SMOE_LAUNCH_G(AG, KM, SW) launch_g<AG, KM, SW>(ta, tb, m, g, nN, grid, s)
+  const int tm = kPairM ? 2 * BM : BM;  // rows per M tile
+  const long long tiles = (long long)(cdiv(g.num_rows, tm) + g.E) * nN;
+#define SMOE_LAUNCH_G(AG, KM, SW) launch_g<AG, KM, SW>(ta, tb, m, g, nN, tiles, s)
   if (gather) {
     if (kmaj) return swiglu ? SMOE_LAUNCH_G(true, true, true) : SMOE_LAUNCH_G(true, true, false);
     return swiglu ? SMOE_LAUNCH_G(true, false, true) : SMOE_LAUNCH_G(true, false, false);
@@ -1322,13 +1539,23 @@ cudaError_t launch_dw_gemm_tc(const DwGemm& g_in, cudaStream_t s) {
   if (e != cudaSuccess) return e;
   e = rows_map(&tb, g.b, g.N, g.b_rows, g.ldb, BK);
   if (e != cudaSuccess) return e;
+  // fp32 dW as [E, rows, cols] with 32 x 32 boxes: rows = M, cols = N, or the
+  // transpose when the kernel computes dW^T
+  CUtensorMap td;
+  memset(&td, 0, sizeof(td));
+  const uint64_t rows = trans ? g.N : g.M, cols = trans ? g.M : g.N;
+  const uint64_t ddims[3] = {cols, rows, (uint64_t)g.E};
+  const uint64_t dstr[2] = {cols * 4, rows * cols * 4};
+  const uint32_t dbox[3] = {32, 32, 1};
+  const int d_boxed = make_map(&td, g.dw, 3, ddims, dstr, dbox, CU_TENSOR_MAP_SWIZZLE_128B,
+                               CU_TENSOR_MAP_DATA_TYPE_FLOAT32) == cudaSuccess;
   const long long tiles = (long long)g.E * nM * nN;
   const int grid = (int)(tiles < num_sms() ? tiles : num_sms());
-  if (trans) return launch_d<true, false, true>(ta, tb, g, nM, nN, grid, s);
-  if (ag) return bg ? launch_d<true, true, false>(ta, tb, g, nM, nN, grid, s)
-                    : launch_d<true, false, false>(ta, tb, g, nM, nN, grid, s);
-  return bg ? launch_d<false, true, false>(ta, tb, g, nM, nN, grid, s)
-            : launch_d<false, false, false>(ta, tb, g, nM, nN, grid, s);
+#define SMOE_LAUNCH_D(AG, BG, TR) launch_d<AG, BG, TR>(ta, tb, td, d_boxed, g, nM, nN, grid, s)
+  if (trans) return SMOE_LAUNCH_D(true, false, true);
+  if (ag) return bg ? SMOE_LAUNCH_D(true, true, false) : SMOE_LAUNCH_D(true, false, false);
+  return bg ? SMOE_LAUNCH_D(false, true, false) : SMOE_LAUNCH_D(false, false, false);
+#undef SMOE_LAUNCH_D
 }
 
 }  // namespace smoe
