@@ -35,9 +35,13 @@ if ROOT not in sys.path:
 import numpy as np  # noqa: E402
 import torch  # noqa: E402
 
-from sparse_mixture_experts_smoe_b200.inputs import WORKLOADS, make_mlp_inputs, mlp_flops  # noqa: E402
+from sparse_mixture_experts_smoe_b200.inputs import (  # noqa: E402
+    WORKLOADS, make_mlp_inputs, make_moa_inputs, mlp_flops)
 
 METRIC = "SMoE MLP fwd+bwd tokens/s on 1 B200; % of dense BF16 tensor peak"
+METRIC_MOA = "MoA expert projections (Wq scatter->group, Wo group->scatter + gated combine) fwd+bwd tokens/s on 1 B200"
+# NVIDIA's nominal dense (no 2:4 sparsity) bf16 tensor throughput of one B200.
+NOMINAL_DENSE_BF16_TFLOPS = 2250.0
 DEFAULT_WORKLOAD = "mixtral_bf16_swiglu"
 
 
@@ -168,6 +172,7 @@ def kernel_work(cfg):
         "dg_reduce": S * 4 * max(1, math.ceil(f / 256)) + S * 8,
         "route_dl": S * 12,
         "route_dw": T * d * b + S * 8 + d * E * 4,
+        "transpose_wr": 2 * d * E * b,
     }
     return flops, bytes_
 
@@ -184,6 +189,49 @@ def oracle_step(c, cfg, n_tok):
     oracle.mlp_bwd_full(x, c["w_r"], c["w1"], c["w2"], cfg["act"], idx, gates, dy)
 
 
+# DRAM bytes per launch measured by ncu (dram__bytes_read.sum + dram__bytes_write.sum)
+# for the workload's GEMM kernels, with the SHA-256 of the kernel source they were
+# taken on; a value whose source has changed since is not reported.
+TRAFFIC_TABLE = os.path.join(ROOT, "profiles", "dram_traffic_mixtral_bf16_swiglu.md")
+KERNEL_SOURCE = os.path.join(ROOT, "sparse_mixture_experts_smoe_b200", "csrc", "gemm_tc.cu")
+
+
+def measured_traffic(kernel: str, workload: str):
+    import hashlib
+    try:
+        with open(KERNEL_SOURCE, "rb") as fh:
+            digest = hashlib.sha256(fh.read()).hexdigest()
+        with open(TRAFFIC_TABLE) as fh:
+            rows = [ln for ln in fh if ln.startswith("|")]
+    except OSError:
+        return None
+    for ln in rows:
+        cells = [c.strip() for c in ln.strip().strip("|").split("|")]
+        # | workload | kernel | read bytes | write bytes | source sha256 | ...
+        if len(cells) >= 5 and cells[0] == workload and cells[1] == kernel and cells[4] == digest:
+            try:
+                return int(float(cells[2])) + int(float(cells[3]))
+            except ValueError:
+                return None
+    return None
+
+
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as fh:
+            for ln in fh:
+                if ln.startswith("model name"):
+                    return ln.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+def oracle_threads() -> int:
+    cores = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count()
+    return int(os.environ.get("OMP_NUM_THREADS", cores))
+
+
 def oracle_baseline(cfg, budget_s=12.0, seed=0):
     """tokens/s of the oracle's full fwd+bwd on a token sample sized to ~budget_s."""
     inp = make_mlp_inputs(cfg, seed=seed, device="cpu")
@@ -196,8 +244,7 @@ def oracle_baseline(cfg, budget_s=12.0, seed=0):
         if dt >= budget_s / 2 or n >= cfg["T"]:
             break
         n = min(cfg["T"], 2 * n)
-    cores = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count()
-    return {"value": n / dt, "unit": "tokens/s", "cores": int(os.environ.get("OMP_NUM_THREADS", cores)),
+    return {"value": n / dt, "unit": "tokens/s", "cores": oracle_threads(), "cpu": cpu_model(),
             "kind": "oracle",
             "sample": f"{n} of the {cfg['T']} tokens: routing, forward and full backward "
                       f"(dx, gate and router gradients, every expert weight gradient) in fp64 "
@@ -222,7 +269,7 @@ def run_reference(args, world, rank):
         oracle_step(inp, cfg, n)
     el = time.perf_counter() - t0
     value = n * args.steps / el
-    cores = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count()
+    cores = oracle_threads()
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 * el / args.steps,
@@ -230,7 +277,8 @@ def run_reference(args, world, rank):
         "data": "synthetic", "config": {"workload": args.workload, "T": cfg["T"], "d": cfg["d"],
                                         "f": cfg["f"], "E": cfg["E"], "k": cfg["k"],
                                         "act": cfg["act"], "tokens_per_step": n},
-        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "cpu": cpu_model(),
+                         "kind": "oracle",
                          "sample": f"{n} tokens per step of the {cfg['T']}-token workload"},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
@@ -241,13 +289,102 @@ def run_reference(args, world, rank):
 # ---------------------------------------------------------------------------
 # our path
 # ---------------------------------------------------------------------------
+def moa_oracle_baseline(cfg, budget_s=12.0, seed=0):
+    """tokens/s of the oracle's MoA projections fwd+bwd on a token sample (~budget_s)."""
+    import oracle
+    inp = make_moa_inputs(cfg, seed=seed, device="cpu")
+    k, E = cfg["k"], cfg["E"]
+    n = 8
+    while True:
+        t0 = time.perf_counter()
+        x, o, dz, dq = inp["x"][:n], inp["o"][:n * k], inp["dz"][:n], inp["dq"][:n * k]
+        idx, g = oracle.route(x, inp["w_r"], None, k)
+        ss, off = oracle.sort(idx, E)
+        oracle.pl_fwd(x, inp["wq"], ss, off, k, 0, 1)
+        oracle.pl_fwd(o, inp["wo"], ss, off, 1, 1, 0, g.ravel(), k)
+        oracle.pl_bwd(dq, x, inp["wq"], ss, off, k, 0, 1)
+        oracle.pl_bwd(dz, o, inp["wo"], ss, off, 1, 1, 0, g.ravel(), k, want_dg=True)
+        dt = time.perf_counter() - t0
+        if dt >= budget_s / 2 or n >= cfg["T"]:
+            break
+        n = min(cfg["T"], 2 * n)
+    return {"value": n / dt, "unit": "tokens/s", "cores": oracle_threads(), "cpu": cpu_model(),
+            "kind": "oracle",
+            "sample": f"{n} of the {cfg['T']} tokens: routing, sort, both projections forward "
+                      f"and backward (dx, do, dWq, dWo, gate gradients) in fp64 plain loops, {dt:.1f} s"}
+
+
+def run_moa(args, world, rank, cfg):
+    """The Mixture-of-Attention expert projections around an attention core (the core
+    itself is not part of the path): route, sort, q = x Wq[e] scatter->group (fan-out k),
+    z = sum_j g o Wo[e] group->scatter with the gated k-way combine, and both backwards
+    (dx, dWq; do, dWo, dgates)."""
+    import sparse_mixture_experts_smoe_b200 as smoe
+    dev = torch.device("cuda", torch.cuda.current_device())
+    inp = make_moa_inputs(cfg, seed=rank, device=dev)
+    T, d, E, k, h = cfg["T"], cfg["d"], cfg["E"], cfg["k"], cfg["h"]
+
+    def step():
+        idx, gates = smoe.smoe_route(inp["x"], inp["w_r"], None, k)
+        ss, off = smoe.smoe_sort(idx, E)
+        smoe.parallel_linear_fwd(inp["x"], inp["wq"], ss, off, k, 0, 1)
+        smoe.parallel_linear_fwd(inp["o"], inp["wo"], ss, off, 1, 1, 0, gates, k)
+        smoe.parallel_linear_bwd(inp["dq"], inp["x"], inp["wq"], ss, off, k, 0, 1)
+        smoe.parallel_linear_bwd(inp["dz"], inp["o"], inp["wo"], ss, off, 1, 1, 0, gates, k,
+                                 want_dgates=True)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    barrier(world)
+    clk = ClockSampler()
+    clk.start()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        step()
+    e1.record()
+    torch.cuda.synchronize()
+    clocks = clk.stop()
+    barrier(world)
+    ms = max_over_ranks(e0.elapsed_time(e1), world) / args.steps
+    if smoe.smoe_check() != 0:
+        raise SystemExit("device error word set during the MoA benchmark")
+    flops = 12.0 * T * k * d * h  # two projections, fwd + 2x bwd
+    tokens = T * world
+    tflops = flops * world / (ms / 1e3) / 1e12
+    peaks = load_peaks()
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = moa_oracle_baseline(cfg)
+    line = {
+        "metric": METRIC_MOA, "value": round(tokens / (ms / 1e3), 1), "unit": "tokens/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": args.workload, "T": T, "d": d, "E": E, "k": k, "h": h,
+                   "parallelism": f"replicas x{world}"},
+        "tflops": round(tflops, 1),
+        "frac_of_bf16_peak": {"burst": round(tflops / peaks["bf16_tflops"], 4),
+                              "sustained": round(tflops / peaks["bf16_tflops_sustained"], 4),
+                              "peaks": peaks["source"]},
+        "peak_mem_gb": round(torch.cuda.max_memory_allocated(dev) / 1e9, 2),
+        "clocks": clocks,
+        "cpu_baseline": cpu,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
 def run_ours(args, world, rank):
     import sparse_mixture_experts_smoe_b200 as smoe
     cfg = dict(WORKLOADS[args.workload])
     if args.tokens:
         cfg["T"] = args.tokens
+    if cfg["kind"] == "moa":
+        return run_moa(args, world, rank, cfg)
     if cfg["kind"] != "mlp":
-        raise SystemExit("the benchmark step is the SMoE MLP; pick an mlp workload")
+        raise SystemExit("unknown workload kind")
     dev = torch.device("cuda", torch.cuda.current_device())
     dt = torch.bfloat16 if cfg["dtype"] == "bf16" else torch.float32
     inp = make_mlp_inputs(cfg, seed=rank, device=dev)
@@ -342,7 +479,7 @@ def run_ours(args, world, rank):
                          "frac": round(ach / peaks["bf16_tflops_sustained"], 4),
                          "peak_kind": f"bf16 sustained, {peaks['source']}",
                          "frac_of_burst_peak": round(ach / peaks["bf16_tflops"], 4),
-                         "traffic": None}
+                         "traffic": None if args.tokens else measured_traffic(dom, args.workload)}
         else:
             ach = bytes_k.get(dom, 0) / per / 1e9
             roofline = {"kernel": dom, "bound": "hbm", "achieved": round(ach, 1),
@@ -362,7 +499,9 @@ def run_ours(args, world, rank):
         "tflops_fwd_bwd": round(tflops, 1),
         "frac_of_bf16_peak": {"burst": round(tflops / peaks["bf16_tflops"], 4),
                               "sustained": round(tflops / peaks["bf16_tflops_sustained"], 4),
-                              "peaks": peaks["source"]},
+                              "peaks": peaks["source"],
+                              "nominal_dense": round(tflops / NOMINAL_DENSE_BF16_TFLOPS, 4)},
+        "peak_mem_gb": round(torch.cuda.max_memory_allocated(dev) / 1e9, 2),
         "fwd": {"tokens_per_s": round(tokens / (ms_fwd / 1e3), 1), "ms_per_step": round(ms_fwd, 4),
                 "tflops": round(fl["fwd"] / (ms_fwd / 1e3) / 1e12, 1)},
         "e2e": {"value": round(tokens / (ms_e2e / 1e3), 1), "unit": "tokens/s",

@@ -1,5 +1,8 @@
 """Shared helpers of the tests: error metrics and layout mapping (no arithmetic of
 the method lives here)."""
+import json
+import os
+
 import numpy as np
 import torch
 
@@ -22,7 +25,18 @@ def rel_err(gpu, ref):
     return float(np.max(np.abs(g - r)) / den)
 
 
+def log_parity(name, err, tol):
+    """Append one measured error to the JSON-lines file named by SMOE_PARITY_LOG (if set)."""
+    path = os.environ.get("SMOE_PARITY_LOG")
+    if not path:
+        return
+    test = os.environ.get("PYTEST_CURRENT_TEST", "").split(" ")[0]
+    with open(path, "a") as fh:
+        fh.write(json.dumps({"test": test, "name": name, "err": err, "tol": tol}) + "\n")
+
+
 def assert_close(name, gpu, ref, dtype):
     err = rel_err(gpu, ref)
+    log_parity(name, err, TOL[dtype])
     assert err <= TOL[dtype], f"{name}: max rel err {err:.3e} > {TOL[dtype]:.1e}"
     return err
