@@ -213,7 +213,7 @@ MlpWs mlp_layout(void* ws, const smoe_mlp_desc& m, int backward) {
     l.dxcomb = (float*)c.take(S * m.d * sizeof(float));
     l.dl = (float*)c.take(S * sizeof(float));
     l.dg = (float*)c.take(S * sizeof(float));
-    l.r_chunks = route_dw_chunks(m.T);
+    l.r_chunks = route_dw_chunks(m.T, m.d, m.E, m.k);
     l.rpart = (float*)c.take(((size_t)l.r_chunks * m.E * m.d + (size_t)l.r_chunks * m.E) * sizeof(float));
     l.wrt = c.take((size_t)m.E * m.d * esize(dt));
   }
@@ -369,7 +369,7 @@ int smoe_route_bwd(const void* x, const void* w_r, const int32_t* topk_idx, cons
   if (!valid_dtype(dt)) return fail(SMOE_ERR_INVALID_ARG, "bad dtype");
   NEED(x, "x"); NEED(w_r, "w_r"); NEED(topk_idx, "topk_idx"); NEED(gates, "gates");
   NEED(dgates, "dgates"); NEED(dw_r, "dw_r");
-  const int chunks = route_dw_chunks(T);
+  const int chunks = route_dw_chunks(T, d, E, k);
   Carve c(workspace);
   float* dl = (float*)c.take((size_t)T * k * sizeof(float));
   float* part = (float*)c.take(((size_t)chunks * E * d + (size_t)chunks * E) * sizeof(float));

@@ -81,7 +81,8 @@ cudaError_t launch_route_dl(const float* gates, const float* dgates, int T, int 
 cudaError_t launch_route_dw(const void* x, const int32_t* idx, const float* dl, int T, int d,
                             int E, int k, smoe_dtype dt, float* partial, int n_chunks,
                             float* dw_r, float* db_r, cudaStream_t s);
-int route_dw_chunks(int T);
+// Number of token chunks of the router weight gradient's first pass (sizes its workspace).
+int route_dw_chunks(int T, int d, int E, int k);
 cudaError_t launch_route_dx(const float* dl, const int32_t* idx, const void* w_r, int T, int d,
                             int E, int k, smoe_dtype dt, void* dx, cudaStream_t s);
 

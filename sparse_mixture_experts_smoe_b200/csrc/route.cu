@@ -50,13 +50,30 @@ route_kernel(const T* __restrict__ x, const T* __restrict__ w_r, const float* __
 #pragma unroll
     for (int e = 0; e < EMAX; ++e) acc[m][e] = 0.0f;
 
+  // padding columns [E, EMAX) of the staged W_r stay zero for every chunk
+  if (E < EMAX)
+    for (int q = threadIdx.x; q < CH * (EMAX - E); q += blockDim.x)
+      ws[(q / (EMAX - E)) * STRIDE + E + q % (EMAX - E)] = 0.0f;
+  constexpr int VEC = 16 / (int)sizeof(T);  // elements per 16-byte load
   for (int i0 = 0; i0 < d; i0 += CH) {
     __syncthreads();
-    // stage W_r[i0 : i0+CH, 0:E] as fp32, zero-padded to EMAX columns
-    for (int q = threadIdx.x; q < CH * EMAX; q += blockDim.x) {
-      const int r = q / EMAX, e = q % EMAX;
-      const int i = i0 + r;
-      ws[r * STRIDE + e] = (i < d && e < E) ? to_f(w_r[(size_t)i * E + e]) : 0.0f;
+    // stage W_r[i0 : i0+CH, 0:E] as fp32: the rows are one contiguous span of
+    // (rows * E) elements, a multiple of VEC because d % 8 == 0, read with 16-byte
+    // loads several in flight per thread
+    {
+      const int rows = min(CH, d - i0);
+      const int nvec = rows * E / VEC;
+      const uint4* src = reinterpret_cast<const uint4*>(w_r + (size_t)i0 * E);
+#pragma unroll 4
+      for (int q = threadIdx.x; q < nvec; q += blockDim.x) {
+        const uint4 u = __ldg(src + q);
+        const T* vals = reinterpret_cast<const T*>(&u);
+#pragma unroll
+        for (int v = 0; v < VEC; ++v) {
+          const int flat = q * VEC + v;
+          ws[(flat / E) * STRIDE + flat % E] = to_f(vals[v]);
+        }
+      }
     }
     // stage x[tb : tb+BT, i0 : i0+CH] as fp32 with 8-element (16-byte bf16) loads
     for (int q = threadIdx.x; q < BT * (CH / 8); q += blockDim.x) {
@@ -208,40 +225,53 @@ __global__ void route_dl_kernel(const float* __restrict__ gates, const float* __
     dl[(size_t)t * k + j] = gates[(size_t)t * k + j] * (dgates[(size_t)t * k + j] - s);
 }
 
-constexpr int kDwTokens = 256;  // tokens per partial-sum chunk
-constexpr int kDwCols = 256;    // feature columns per block (= threads)
-
+// Router weight gradient in two passes with a fixed summation order: tokens are
+// split into chunks of `chunk` consecutive tokens; pass 1 sums each chunk in
+// ascending token order (per feature column and expert), pass 2 sums the chunk
+// partials in ascending chunk order.  The chunk length and the columns per block
+// depend only on (T, d, E, k) (route_dw_plan), so results do not depend on the GPU.
+//
 // partial[c][e][i] = sum_{t in chunk c} x[t,i] dl[t,e];  dbp[c][e] = sum_t dl[t,e]
 template <typename T>
-__global__ void __launch_bounds__(kDwCols)
+__global__ void __launch_bounds__(256)
 route_dw_partial_kernel(const T* __restrict__ x, const int32_t* __restrict__ idx,
-                        const float* __restrict__ dl, int T_, int d, int E, int k,
+                        const float* __restrict__ dl, int T_, int d, int E, int k, int chunk,
                         float* __restrict__ partial, float* __restrict__ dbp) {
-  extern __shared__ float acc_s[];  // [E][kDwCols]
+  extern __shared__ float sm[];
+  const int cols = blockDim.x;
+  float* acc_s = sm;                                        // [E][cols]
+  int* idx_s = reinterpret_cast<int*>(acc_s + (size_t)E * cols);  // [chunk * k]
+  float* dl_s = reinterpret_cast<float*>(idx_s + chunk * k);      // [chunk * k]
   const int c = blockIdx.x;
-  const int i = blockIdx.y * kDwCols + threadIdx.x;
-  for (int e = 0; e < E; ++e) acc_s[e * kDwCols + threadIdx.x] = 0.0f;
-  const int t_end = min(T_, (c + 1) * kDwTokens);
-  for (int t = c * kDwTokens; t < t_end; ++t) {
-    const float xv = i < d ? to_f(x[(size_t)t * d + i]) : 0.0f;
+  const int i = blockIdx.y * cols + threadIdx.x;
+  const int t0 = c * chunk;
+  const int nt = min(T_, t0 + chunk) - t0;
+  for (int e = 0; e < E; ++e) acc_s[e * cols + threadIdx.x] = 0.0f;
+  for (int q = threadIdx.x; q < nt * k; q += cols) {  // the chunk's routing, once per block
+    idx_s[q] = idx[(size_t)t0 * k + q];
+    dl_s[q] = dl[(size_t)t0 * k + q];
+  }
+  __syncthreads();
+  const T* xp = x + (size_t)t0 * d + i;
+#pragma unroll 4
+  for (int t = 0; t < nt; ++t) {
+    const float xv = i < d ? to_f(xp[(size_t)t * d]) : 0.0f;
     for (int j = 0; j < k; ++j) {
-      const int e = idx[(size_t)t * k + j];
+      const int e = idx_s[t * k + j];
       if (e < 0 || e >= E) continue;
-      float& a = acc_s[e * kDwCols + threadIdx.x];
-      a = fmaf(xv, dl[(size_t)t * k + j], a);
+      float& a = acc_s[e * cols + threadIdx.x];
+      a = fmaf(xv, dl_s[t * k + j], a);
     }
   }
   if (i < d)
-    for (int e = 0; e < E; ++e) partial[((size_t)c * E + e) * d + i] = acc_s[e * kDwCols + threadIdx.x];
-  if (blockIdx.y == 0 && threadIdx.x == 0) {
-    for (int e = 0; e < E; ++e) acc_s[e * kDwCols] = 0.0f;
-    for (int t = c * kDwTokens; t < t_end; ++t)
-      for (int j = 0; j < k; ++j) {
-        const int e = idx[(size_t)t * k + j];
-        if (e >= 0 && e < E) acc_s[e * kDwCols] += dl[(size_t)t * k + j];
-      }
-    for (int e = 0; e < E; ++e) dbp[(size_t)c * E + e] = acc_s[e * kDwCols];
-  }
+    for (int e = 0; e < E; ++e) partial[((size_t)c * E + e) * d + i] = acc_s[e * cols + threadIdx.x];
+  if (blockIdx.y == 0)
+    for (int e = threadIdx.x; e < E; e += cols) {  // bias: one expert per thread
+      float sb = 0.0f;
+      for (int q = 0; q < nt * k; ++q)
+        if (idx_s[q] == e) sb += dl_s[q];
+      dbp[(size_t)c * E + e] = sb;
+    }
 }
 
 // dw_r[i][e] = sum_c partial[c][e][i] (ascending c); db[e] = sum_c dbp[c][e]
@@ -293,26 +323,49 @@ cudaError_t launch_route_dl(const float* gates, const float* dgates, int T_, int
   return cudaGetLastError();
 }
 
-int route_dw_chunks(int T_) { return cdiv(T_, kDwTokens); }
+namespace {
+struct DwPlan {
+  int chunk, cols, n_chunks;
+};
+// Columns per block: accumulators of E experts fit in 64 KB of shared memory.
+// Tokens per chunk: halved from 256 until the grid has two blocks per SM of a
+// 148-SM B200 (a fixed count, so the summation order is the same on any GPU),
+// and at most 2048 routing slots per chunk.
+DwPlan route_dw_plan(int T_, int d, int E, int k) {
+  DwPlan p;
+  p.cols = 256;
+  while (p.cols > 32 && (size_t)E * p.cols * sizeof(float) > 64 * 1024) p.cols >>= 1;
+  const int col_blocks = cdiv(d, p.cols);
+  p.chunk = 256;
+  while (p.chunk > 16 && (long long)cdiv(T_, p.chunk) * col_blocks < 2 * 148) p.chunk >>= 1;
+  while (p.chunk > 1 && p.chunk * k > 2048) p.chunk >>= 1;
+  p.n_chunks = cdiv(T_ > 0 ? T_ : 1, p.chunk);
+  return p;
+}
+}  // namespace
+
+int route_dw_chunks(int T_, int d, int E, int k) { return route_dw_plan(T_, d, E, k).n_chunks; }
 
 cudaError_t launch_route_dw(const void* x, const int32_t* idx, const float* dl, int T_, int d,
                             int E, int k, smoe_dtype dt, float* partial, int n_chunks,
                             float* dw_r, float* db_r, cudaStream_t s) {
+  const DwPlan p = route_dw_plan(T_, d, E, k);
+  if (p.n_chunks != n_chunks) return cudaErrorInvalidValue;  // workspace laid out for another plan
   float* dbp = partial + (size_t)n_chunks * E * d;
-  const size_t smem = (size_t)E * kDwCols * sizeof(float);
-  dim3 grid(n_chunks, cdiv(d, kDwCols));
+  const size_t smem = (size_t)E * p.cols * sizeof(float) + (size_t)p.chunk * k * 8;
+  dim3 grid(n_chunks, cdiv(d, p.cols));
   if (dt == SMOE_BF16) {
     cudaError_t e = cudaFuncSetAttribute(route_dw_partial_kernel<bf16>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    route_dw_partial_kernel<bf16><<<grid, kDwCols, smem, s>>>((const bf16*)x, idx, dl, T_, d, E,
-                                                              k, partial, dbp);
+    route_dw_partial_kernel<bf16><<<grid, p.cols, smem, s>>>((const bf16*)x, idx, dl, T_, d, E,
+                                                             k, p.chunk, partial, dbp);
   } else {
     cudaError_t e = cudaFuncSetAttribute(route_dw_partial_kernel<float>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    route_dw_partial_kernel<float><<<grid, kDwCols, smem, s>>>((const float*)x, idx, dl, T_, d, E,
-                                                               k, partial, dbp);
+    route_dw_partial_kernel<float><<<grid, p.cols, smem, s>>>((const float*)x, idx, dl, T_, d, E,
+                                                              k, p.chunk, partial, dbp);
   }
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
