@@ -376,6 +376,74 @@ def run_moa(args, world, rank, cfg):
         print(json.dumps(line), flush=True)
 
 
+# ---------------------------------------------------------------------------
+# granularity / sparsity sweeps of the SMoE MLP (one JSON line per configuration;
+# not the benchmark's contract line)
+# ---------------------------------------------------------------------------
+SWEEP_T, SWEEP_D = 16384, 2048
+SWEEPS = {
+    # E*f and k*f constant: the same parameters and FLOPs per token, finer experts
+    "granularity": [(8, 1, 4096), (16, 2, 2048), (32, 4, 1024), (64, 8, 512), (128, 16, 256)],
+    # E and f fixed, more experts per token
+    "sparsity": [(64, 1, 512), (64, 2, 512), (64, 4, 512), (64, 8, 512)],
+    # the same kernels as one dense SwiGLU MLP (E = 1, k = 1: every gate is exactly 1)
+    "dense": [(1, 1, 4096)],
+}
+
+
+def run_sweep(args, world, rank):
+    import sparse_mixture_experts_smoe_b200 as smoe
+    dev = torch.device("cuda", torch.cuda.current_device())
+    peaks = load_peaks()
+    names = list(SWEEPS) if args.sweep == "all" else [args.sweep]
+    for name in names:
+        for (E, k, f) in SWEEPS[name]:
+            cfg = dict(kind="mlp", T=SWEEP_T, d=SWEEP_D, f=f, E=E, k=k, act="swiglu", dtype="bf16")
+            torch.cuda.empty_cache()
+            torch.cuda.reset_peak_memory_stats(dev)
+            inp = make_mlp_inputs(cfg, seed=rank, device=dev)
+            st = smoe.SMoEMLPState(SWEEP_T, SWEEP_D, f, E, k, "swiglu", torch.bfloat16, dev)
+            p = (inp["x"], inp["w_r"], inp["b_r"], inp["w1"], inp["w2"])
+
+            def fwd():
+                smoe.smoe_mlp_fwd(st, *p)
+
+            def fwd_bwd():
+                smoe.smoe_mlp_fwd(st, *p)
+                smoe.smoe_mlp_bwd(st, *p, inp["dy"])
+
+            def timed(fn):
+                for _ in range(args.warmup):
+                    fn()
+                torch.cuda.synchronize()
+                barrier(world)
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record()
+                for _ in range(args.steps):
+                    fn()
+                e1.record()
+                torch.cuda.synchronize()
+                barrier(world)
+                return max_over_ranks(e0.elapsed_time(e1), world) / args.steps
+
+            ms = timed(fwd_bwd)
+            ms_f = timed(fwd)
+            if smoe.smoe_check() != 0:
+                raise SystemExit(f"device error word set in sweep {name} E={E} k={k}")
+            fl = mlp_flops(cfg)
+            tf = fl["fwd_bwd"] / (ms / 1e3) / 1e12
+            line = {"sweep": name, "E": E, "k": k, "f": f, "T": SWEEP_T, "d": SWEEP_D, "act": "swiglu",
+                    "dtype": "bf16", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+                    "ms_fwd_bwd": round(ms, 4), "tokens_per_s": round(SWEEP_T * world / (ms / 1e3), 1),
+                    "tflops": round(tf, 1), "frac_of_burst": round(tf / peaks["bf16_tflops"], 4),
+                    "ms_fwd": round(ms_f, 4),
+                    "tflops_fwd": round(fl["fwd"] / (ms_f / 1e3) / 1e12, 1),
+                    "peak_mem_gb": round(torch.cuda.max_memory_allocated(dev) / 1e9, 2)}
+            if rank == 0:
+                print(json.dumps(line), flush=True)
+            del st, inp, p
+
+
 def run_ours(args, world, rank):
     import sparse_mixture_experts_smoe_b200 as smoe
     cfg = dict(WORKLOADS[args.workload])
@@ -525,6 +593,8 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--sweep", choices=["granularity", "sparsity", "dense", "all"], default=None,
+                    help="time the SMoE MLP over a set of (E, k, f) shapes instead of the benchmark line")
     ap.add_argument("--tokens", type=int, default=0,
                     help="override T (smaller cases for profiler captures; never a bench line)")
     args = ap.parse_args()
@@ -532,6 +602,8 @@ def main():
     try:
         if args.impl == "reference":
             run_reference(args, world, rank)
+        elif args.sweep:
+            run_sweep(args, world, rank)
         else:
             run_ours(args, world, rank)
     finally:

@@ -84,6 +84,10 @@ REDUCED = {
     "swiglu_f32": dict(kind="mlp", T=200, d=72, f=136, E=4, k=2, dtype="f32", act="swiglu"),
     "single_expert_bf16": dict(kind="mlp", T=130, d=128, f=136, E=1, k=1, dtype="bf16",
                                act="gelu"),
+    # shapes the granularity and sparsity sweeps reach: 128 experts with k = 16, top-1
+    "e128_k16_bf16": dict(kind="mlp", T=96, d=136, f=72, E=128, k=16, dtype="bf16",
+                          act="swiglu"),
+    "top1_bf16": dict(kind="mlp", T=200, d=136, f=136, E=32, k=1, dtype="bf16", act="swiglu"),
 }
 
 
