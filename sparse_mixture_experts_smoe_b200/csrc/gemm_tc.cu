@@ -895,10 +895,11 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
               float o[8];
 #pragma unroll
               for (int j = 0; j < 8; ++j) o[j] = gate * vv[j];
-              if (g.out_f32) {  // never boxed
-                float4* dst = reinterpret_cast<float4*>(slot + 32 * j8);
-                dst[0] = make_float4(o[0], o[1], o[2], o[3]);
-                dst[1] = make_float4(o[4], o[5], o[6], o[7]);
+              if (g.out_f32) {  // a 32 x 32 fp32 box in the 128-byte swizzle, row = lane
+                float4* d0 = reinterpret_cast<float4*>(wstage + lane * 128 + (((2 * j8) ^ (lane & 7)) << 4));
+                float4* d1 = reinterpret_cast<float4*>(wstage + lane * 128 + (((2 * j8 + 1) ^ (lane & 7)) << 4));
+                *d0 = make_float4(o[0], o[1], o[2], o[3]);
+                *d1 = make_float4(o[4], o[5], o[6], o[7]);
               } else {
                 *chunk(0, j8) = pack8(o);
               }
@@ -958,10 +959,7 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
               }
             }
           } else if (epi_store) {
-            if (g.out_f32)
-              bulk_s2g(reinterpret_cast<float*>(g.out) + (size_t)orow * g.ldo + n0, slot_s, 2 * seg);
-            else
-              bulk_s2g(reinterpret_cast<bf16*>(g.out) + (size_t)orow * g.ldo + n0, slot_s, seg);
+            if (!g.out_f32) bulk_s2g(reinterpret_cast<bf16*>(g.out) + (size_t)orow * g.ldo + n0, slot_s, seg);
           } else {
             bf16* H = reinterpret_cast<bf16*>(g.out) + (size_t)orow * g.ldo;
             bf16* A2 = reinterpret_cast<bf16*>(g.out2) + (size_t)orow * g.ldo2;
@@ -974,6 +972,21 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
             }
           }
           bulk_commit();
+        }
+        if (epi_store && g.out_f32) {
+          // fp32 rows in token order (the k-way combine's slot rows): from the box,
+          // 8 lanes per 128-byte row segment, 4 rows per warp store; per-row bulk
+          // copies of 128 bytes would be one TMA operation per row per chunk
+#pragma unroll
+          for (int it2 = 0; it2 < 8; ++it2) {
+            const int rr = it2 * 4 + (lane >> 3), c4 = lane & 7;
+            const int orow_r = __shfl_sync(0xffffffffu, orow, rr);
+            const int ok_r = __shfl_sync(0xffffffffu, p_ok ? 1 : 0, rr);
+            if (ok_r && 4 * c4 < ncols) {
+              const float4 val = *reinterpret_cast<const float4*>(wstage + rr * 128 + ((c4 ^ (rr & 7)) << 4));
+              *reinterpret_cast<float4*>(reinterpret_cast<float*>(g.out) + (size_t)orow_r * g.ldo + n0 + 4 * c4) = val;
+            }
+          }
         }
       }
       if (act_bwd && p_ok && g.dg_partial)
