@@ -28,7 +28,9 @@ __host__ __device__ constexpr int route_row_stride(int emax) {
   return emax + ((4 - emax % 32) + 32) % 32;
 }
 
-template <typename T, int EMAX, int TM, int CH>
+// FULL: E == EMAX (the staged W_r rows need no padding and the index arithmetic
+// of the staging divides by a constant).
+template <typename T, int EMAX, int TM, int CH, bool FULL>
 __global__ void __launch_bounds__(kRouteWarps * 32)
 route_kernel(const T* __restrict__ x, const T* __restrict__ w_r, const float* __restrict__ b_r,
              int T_, int d, int E, int k, int32_t* __restrict__ idx, float* __restrict__ gates,
@@ -50,8 +52,9 @@ route_kernel(const T* __restrict__ x, const T* __restrict__ w_r, const float* __
 #pragma unroll
     for (int e = 0; e < EMAX; ++e) acc[m][e] = 0.0f;
 
+  const int ecols = FULL ? EMAX : E;
   // padding columns [E, EMAX) of the staged W_r stay zero for every chunk
-  if (E < EMAX)
+  if (!FULL && E < EMAX)
     for (int q = threadIdx.x; q < CH * (EMAX - E); q += blockDim.x)
       ws[(q / (EMAX - E)) * STRIDE + E + q % (EMAX - E)] = 0.0f;
   constexpr int VEC = 16 / (int)sizeof(T);  // elements per 16-byte load
@@ -62,7 +65,7 @@ route_kernel(const T* __restrict__ x, const T* __restrict__ w_r, const float* __
     // loads several in flight per thread
     {
       const int rows = min(CH, d - i0);
-      const int nvec = rows * E / VEC;
+      const int nvec = rows * ecols / VEC;
       const uint4* src = reinterpret_cast<const uint4*>(w_r + (size_t)i0 * E);
 #pragma unroll 4
       for (int q = threadIdx.x; q < nvec; q += blockDim.x) {
@@ -71,7 +74,7 @@ route_kernel(const T* __restrict__ x, const T* __restrict__ w_r, const float* __
 #pragma unroll
         for (int v = 0; v < VEC; ++v) {
           const int flat = q * VEC + v;
-          ws[(flat / E) * STRIDE + flat % E] = to_f(vals[v]);
+          ws[(flat / ecols) * STRIDE + flat % ecols] = to_f(vals[v]);
         }
       }
     }
@@ -136,42 +139,78 @@ route_kernel(const T* __restrict__ x, const T* __restrict__ w_r, const float* __
       acc[m][e] = v;
     }
 
+  // Top-k per token, warp-parallel: lane L holds the logits of experts
+  // e = L + 32 j (j < NC).  Each round reproduces the sequential scan "start at the
+  // first free expert, replace on a strictly greater logit": if the first free
+  // expert's logit is NaN it is taken, else the largest free non-NaN logit, the
+  // lower expert id on ties.
+  constexpr int NC = EMAX >= 32 ? EMAX / 32 : 1;
+  constexpr int kNone = 0x7fffffff;
 #pragma unroll
   for (int m = 0; m < TM; ++m) {
     const int t = t0 + m;
     if (t >= T_) break;
-    float l[EMAX];
+    float lv[NC];
+    unsigned fr = 0u;  // bit j: expert lane + 32 j is free
 #pragma unroll
-    for (int e = 0; e < EMAX; ++e) l[e] = (b_r != nullptr && e < E) ? acc[m][e] + b_r[e] : acc[m][e];
-    // top-k: descending, ties to the lower expert id
-    unsigned long long taken0 = 0ull, taken1 = 0ull;  // EMAX <= 128
+    for (int j = 0; j < NC; ++j) {
+      const int e = lane + 32 * j;
+      float a = 0.0f;
+#pragma unroll
+      for (int ee = 0; ee < EMAX; ++ee)
+        if (ee == e) a = acc[m][ee];
+      lv[j] = (e < E && b_r != nullptr) ? a + b_r[e] : a;
+      if (e < E && e < EMAX) fr |= 1u << j;
+    }
     float sel[16];
 #pragma unroll
-    for (int j = 0; j < 16; ++j) {
-      if (j >= k) break;
-      int best = -1;
-      float bestv = 0.0f;
+    for (int jj = 0; jj < 16; ++jj) {
+      if (jj >= k) break;
+      // first free expert and its logit
+      int ff = kNone;
 #pragma unroll
-      for (int e = 0; e < EMAX; ++e) {
-        if (e >= E) break;
-        const bool tk = e < 64 ? ((taken0 >> e) & 1ull) : ((taken1 >> (e - 64)) & 1ull);
-        if (!tk && (best < 0 || l[e] > bestv)) {
-          best = e;
-          bestv = l[e];
-        }
-      }
-      if (best < 0) {  // only NaN logits left: take the lowest free id, flag the data
+      for (int j = NC - 1; j >= 0; --j)
+        if ((fr >> j) & 1u) ff = lane + 32 * j;
 #pragma unroll
-        for (int e = EMAX - 1; e >= 0; --e) {
-          if (e >= E) continue;
-          const bool tk = e < 64 ? ((taken0 >> e) & 1ull) : ((taken1 >> (e - 64)) & 1ull);
-          if (!tk) { best = e; bestv = l[e]; }
+      for (int off = 16; off >= 1; off >>= 1) ff = min(ff, __shfl_xor_sync(0xffffffffu, ff, off));
+      float vff = 0.0f;
+#pragma unroll
+      for (int j = 0; j < NC; ++j)
+        if (ff == lane + 32 * j) vff = lv[j];
+      vff = __shfl_sync(0xffffffffu, vff, ff & 31);
+      int win;
+      float wv;
+      if (vff != vff) {  // NaN at the first free expert: the scan keeps it
+        win = ff;
+        wv = vff;
+      } else {
+        float bv = 0.0f;
+        int bi = kNone;
+#pragma unroll
+        for (int j = 0; j < NC; ++j) {
+          const float v = lv[j];
+          if (((fr >> j) & 1u) && v == v && (bi == kNone || v > bv)) {
+            bv = v;
+            bi = lane + 32 * j;
+          }
         }
-        if (lane == 0) report_error(err, ERRBIT_DATA);
+#pragma unroll
+        for (int off = 16; off >= 1; off >>= 1) {
+          const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
+          const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
+          if (oi != kNone && (bi == kNone || ov > bv || (ov == bv && oi < bi))) {
+            bv = ov;
+            bi = oi;
+          }
+        }
+        win = bi;  // a non-NaN free logit exists: the first free one is one
+        wv = bv;
       }
-      if (best < 64) taken0 |= 1ull << best; else taken1 |= 1ull << (best - 64);
-      sel[j] = bestv;
-      if (lane == 0) idx[(size_t)t * k + j] = best;
+#pragma unroll
+      for (int j = 0; j < NC; ++j)
+        if (win == lane + 32 * j) fr &= ~(1u << j);
+      sel[jj] = wv;
+      if (lane == 0) idx[(size_t)t * k + jj] = win;
     }
     // gates: softmax over the selected logits (sel[0] is the maximum)
     float z = 0.0f;
@@ -195,7 +234,7 @@ cudaError_t launch_route_t(const void* x, const void* w_r, const float* b_r, int
                            int k, int32_t* idx, float* gates, unsigned* err, cudaStream_t s) {
   constexpr int CH = EMAX <= 64 ? 256 : 128;
   const size_t smem = ((size_t)CH * route_row_stride(EMAX) + (size_t)kRouteWarps * TM * CH) * sizeof(float);
-  auto kern = route_kernel<T, EMAX, TM, CH>;
+  auto kern = E == EMAX ? route_kernel<T, EMAX, TM, CH, true> : route_kernel<T, EMAX, TM, CH, false>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   const int blocks = cdiv(T_, kRouteWarps * TM);

@@ -85,6 +85,30 @@ def test_route_ties_go_to_lower_expert():
     np.testing.assert_allclose(gates.cpu().numpy(), 1.0 / 3.0, rtol=1e-6)
 
 
+@pytest.mark.parametrize("E,k", [(64, 6), (128, 9)])
+def test_route_ties_and_nan_follow_the_scan(E, k):
+    """Logits equal to the bias (x = 0): a five-way tie spread over lanes and slots
+    goes to the lower ids; a NaN logit is taken only when it is the first free
+    expert (the scan starts there and a comparison with NaN never replaces it),
+    and is skipped anywhere else -- as in the oracle's scan."""
+    T, d = 6, 64
+    x = torch.zeros(T, d, device="cuda", dtype=torch.bfloat16)
+    w_r = torch.randn(d, E, device="cuda").to(torch.bfloat16)
+    b = torch.zeros(E)
+    b[[3, 40, 35, 8, E - 1]] = 1.0
+    b[[17, 50]] = 2.0
+    nan_first, nan_later = b.clone(), b.clone()
+    nan_first[0] = float("nan")
+    nan_later[40] = float("nan")
+    for bias in (b, nan_first, nan_later):
+        idx, gates = smoe.smoe_route(x, w_r, bias.cuda(), k)
+        torch.cuda.synchronize()
+        ref_idx, ref_g = oracle.route(x.cpu(), w_r.cpu(), bias, k)
+        np.testing.assert_array_equal(idx.cpu().numpy(), ref_idx)
+        np.testing.assert_allclose(gates.cpu().numpy(), ref_g, rtol=2e-6, equal_nan=True)
+    assert idx.cpu().tolist()[0][:4] == [17, 50, 3, 8]
+
+
 @pytest.mark.parametrize("T,k,E,pattern", [
     (1, 1, 1, "uniform"),
     (5000, 2, 8, "uniform"),        # several 4096-slot chunks plus a ragged tail
