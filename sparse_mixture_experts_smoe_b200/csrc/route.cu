@@ -270,45 +270,113 @@ __global__ void route_dl_kernel(const float* __restrict__ gates, const float* __
 // partials in ascending chunk order.  The chunk length and the columns per block
 // depend only on (T, d, E, k) (route_dw_plan), so results do not depend on the GPU.
 //
+// Pass 1 per block (chunk c, 8 feature columns per thread): the chunk's routing
+// goes to shared memory as one compact list per expert, in token order (one
+// thread per expert builds its list); then each thread sums, expert by expert,
+// x[t, i:i+8] * dl over the expert's list in registers, reading the x rows with
+// 16-byte loads several in flight -- the same additions in the same order as
+// accumulating token by token.
+//
 // partial[c][e][i] = sum_{t in chunk c} x[t,i] dl[t,e];  dbp[c][e] = sum_t dl[t,e]
+constexpr int kDwThreads = 128;
+constexpr int kDwColsPerThread = 8;
+
 template <typename T>
-__global__ void __launch_bounds__(256)
+__device__ __forceinline__ void load8(const T* p, float* v) {
+  if (sizeof(T) == 2) {
+    const uint4 u = __ldg(reinterpret_cast<const uint4*>(p));
+    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float2 f = __bfloat1622float2(h[q]);
+      v[2 * q] = f.x;
+      v[2 * q + 1] = f.y;
+    }
+  } else {
+    const float4 a = __ldg(reinterpret_cast<const float4*>(p));
+    const float4 b = __ldg(reinterpret_cast<const float4*>(p) + 1);
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+    v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+  }
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kDwThreads)
 route_dw_partial_kernel(const T* __restrict__ x, const int32_t* __restrict__ idx,
                         const float* __restrict__ dl, int T_, int d, int E, int k, int chunk,
                         float* __restrict__ partial, float* __restrict__ dbp) {
-  extern __shared__ float sm[];
-  const int cols = blockDim.x;
-  float* acc_s = sm;                                        // [E][cols]
-  int* idx_s = reinterpret_cast<int*>(acc_s + (size_t)E * cols);  // [chunk * k]
-  float* dl_s = reinterpret_cast<float*>(idx_s + chunk * k);      // [chunk * k]
+  extern __shared__ float4 sm4[];
+  const int ns = chunk * k;                               // routing slots per chunk
+  int* idx_s = reinterpret_cast<int*>(sm4);               // [ns]
+  float* dl_s = reinterpret_cast<float*>(idx_s + ns);     // [ns]
+  int* lst_t = reinterpret_cast<int*>(dl_s + ns);         // [ns] token of each entry
+  float* lst_v = reinterpret_cast<float*>(lst_t + ns);    // [ns] its dl
+  int* off = reinterpret_cast<int*>(lst_v + ns);          // [E + 1]
   const int c = blockIdx.x;
-  const int i = blockIdx.y * cols + threadIdx.x;
+  const int i = (blockIdx.y * kDwThreads + threadIdx.x) * kDwColsPerThread;
   const int t0 = c * chunk;
   const int nt = min(T_, t0 + chunk) - t0;
-  for (int e = 0; e < E; ++e) acc_s[e * cols + threadIdx.x] = 0.0f;
-  for (int q = threadIdx.x; q < nt * k; q += cols) {  // the chunk's routing, once per block
+  for (int q = threadIdx.x; q < nt * k; q += kDwThreads) {
     idx_s[q] = idx[(size_t)t0 * k + q];
     dl_s[q] = dl[(size_t)t0 * k + q];
   }
   __syncthreads();
-  const T* xp = x + (size_t)t0 * d + i;
-#pragma unroll 4
-  for (int t = 0; t < nt; ++t) {
-    const float xv = i < d ? to_f(xp[(size_t)t * d]) : 0.0f;
-    for (int j = 0; j < k; ++j) {
-      const int e = idx_s[t * k + j];
-      if (e < 0 || e >= E) continue;
-      float& a = acc_s[e * cols + threadIdx.x];
-      a = fmaf(xv, dl_s[t * k + j], a);
+  for (int e = threadIdx.x; e < E; e += kDwThreads) {  // list lengths (a token's experts are distinct)
+    int n = 0;
+    for (int q = 0; q < nt * k; ++q) n += idx_s[q] == e;
+    off[e + 1] = n;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    off[0] = 0;
+    for (int e = 0; e < E; ++e) off[e + 1] += off[e];
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += kDwThreads) {
+    int pos = off[e];
+    for (int q = 0; q < nt * k; ++q)
+      if (idx_s[q] == e) {
+        lst_t[pos] = q / k;
+        lst_v[pos] = dl_s[q];
+        ++pos;
+      }
+  }
+  __syncthreads();
+  if (i < d) {
+    const T* xc = x + (size_t)t0 * d + i;
+    for (int e = 0; e < E; ++e) {
+      float a[kDwColsPerThread];
+#pragma unroll
+      for (int j = 0; j < kDwColsPerThread; ++j) a[j] = 0.0f;
+      int u = off[e];
+      const int u1 = off[e + 1];
+      for (; u + 4 <= u1; u += 4) {  // four rows in flight, summed in list order
+        float v[4][kDwColsPerThread];
+#pragma unroll
+        for (int r = 0; r < 4; ++r) load8(xc + (size_t)lst_t[u + r] * d, v[r]);
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+          const float g = lst_v[u + r];
+#pragma unroll
+          for (int j = 0; j < kDwColsPerThread; ++j) a[j] = fmaf(v[r][j], g, a[j]);
+        }
+      }
+      for (; u < u1; ++u) {
+        float v[kDwColsPerThread];
+        load8(xc + (size_t)lst_t[u] * d, v);
+        const float g = lst_v[u];
+#pragma unroll
+        for (int j = 0; j < kDwColsPerThread; ++j) a[j] = fmaf(v[j], g, a[j]);
+      }
+      float4* dst = reinterpret_cast<float4*>(partial + ((size_t)c * E + e) * d + i);
+      dst[0] = make_float4(a[0], a[1], a[2], a[3]);
+      dst[1] = make_float4(a[4], a[5], a[6], a[7]);
     }
   }
-  if (i < d)
-    for (int e = 0; e < E; ++e) partial[((size_t)c * E + e) * d + i] = acc_s[e * cols + threadIdx.x];
   if (blockIdx.y == 0)
-    for (int e = threadIdx.x; e < E; e += cols) {  // bias: one expert per thread
+    for (int e = threadIdx.x; e < E; e += kDwThreads) {  // bias: one expert per thread, token order
       float sb = 0.0f;
-      for (int q = 0; q < nt * k; ++q)
-        if (idx_s[q] == e) sb += dl_s[q];
+      for (int u = off[e]; u < off[e + 1]; ++u) sb += lst_v[u];
       dbp[(size_t)c * E + e] = sb;
     }
 }
@@ -320,8 +388,19 @@ __global__ void route_dw_reduce_kernel(const float* __restrict__ partial,
   const int q = blockIdx.x * blockDim.x + threadIdx.x;  // q = e * d + i
   if (q < d * E) {
     const int e = q / d, i = q % d;
+    // ascending chunk order; the loads are independent, so several are in flight
+    const float* pp = partial + (size_t)e * d + i;
+    const size_t step = (size_t)E * d;
     float s = 0.0f;
-    for (int c = 0; c < n_chunks; ++c) s += partial[((size_t)c * E + e) * d + i];
+    int c = 0;
+    for (; c + 8 <= n_chunks; c += 8) {
+      float v[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) v[u] = __ldg(pp + (size_t)(c + u) * step);
+#pragma unroll
+      for (int u = 0; u < 8; ++u) s += v[u];
+    }
+    for (; c < n_chunks; ++c) s += __ldg(pp + (size_t)c * step);
     dw_r[(size_t)i * E + e] = s;
   }
   if (db_r != nullptr && q < E) {
@@ -364,21 +443,19 @@ cudaError_t launch_route_dl(const float* gates, const float* dgates, int T_, int
 
 namespace {
 struct DwPlan {
-  int chunk, cols, n_chunks;
+  int chunk, n_chunks;
 };
-// Columns per block: accumulators of E experts fit in 64 KB of shared memory.
-// Tokens per chunk: halved from 256 until the grid has two blocks per SM of a
-// 148-SM B200 (a fixed count, so the summation order is the same on any GPU),
-// and at most 2048 routing slots per chunk.
+// 8 feature columns per thread, 1024 per block.  Tokens per chunk: halved from 256
+// until the grid has two blocks per SM of a 148-SM B200 (a fixed count, so the
+// summation order is the same on any GPU) and at most 4096 routing slots.
 DwPlan route_dw_plan(int T_, int d, int E, int k) {
   DwPlan p;
-  p.cols = 256;
-  while (p.cols > 32 && (size_t)E * p.cols * sizeof(float) > 64 * 1024) p.cols >>= 1;
-  const int col_blocks = cdiv(d, p.cols);
+  const int col_blocks = cdiv(d, kDwThreads * kDwColsPerThread);
   p.chunk = 256;
   while (p.chunk > 16 && (long long)cdiv(T_, p.chunk) * col_blocks < 2 * 148) p.chunk >>= 1;
-  while (p.chunk > 1 && p.chunk * k > 2048) p.chunk >>= 1;
+  while (p.chunk > 1 && p.chunk * k > 4096) p.chunk >>= 1;
   p.n_chunks = cdiv(T_ > 0 ? T_ : 1, p.chunk);
+  (void)E;
   return p;
 }
 }  // namespace
@@ -391,20 +468,20 @@ cudaError_t launch_route_dw(const void* x, const int32_t* idx, const float* dl, 
   const DwPlan p = route_dw_plan(T_, d, E, k);
   if (p.n_chunks != n_chunks) return cudaErrorInvalidValue;  // workspace laid out for another plan
   float* dbp = partial + (size_t)n_chunks * E * d;
-  const size_t smem = (size_t)E * p.cols * sizeof(float) + (size_t)p.chunk * k * 8;
-  dim3 grid(n_chunks, cdiv(d, p.cols));
+  const size_t smem = (size_t)p.chunk * k * 16 + (size_t)(E + 1) * 4;
+  dim3 grid(n_chunks, cdiv(d, kDwThreads * kDwColsPerThread));
   if (dt == SMOE_BF16) {
     cudaError_t e = cudaFuncSetAttribute(route_dw_partial_kernel<bf16>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    route_dw_partial_kernel<bf16><<<grid, p.cols, smem, s>>>((const bf16*)x, idx, dl, T_, d, E,
-                                                             k, p.chunk, partial, dbp);
+    route_dw_partial_kernel<bf16><<<grid, kDwThreads, smem, s>>>((const bf16*)x, idx, dl, T_, d, E,
+                                                                 k, p.chunk, partial, dbp);
   } else {
     cudaError_t e = cudaFuncSetAttribute(route_dw_partial_kernel<float>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    route_dw_partial_kernel<float><<<grid, p.cols, smem, s>>>((const float*)x, idx, dl, T_, d, E,
-                                                              k, p.chunk, partial, dbp);
+    route_dw_partial_kernel<float><<<grid, kDwThreads, smem, s>>>((const float*)x, idx, dl, T_, d, E,
+                                                                  k, p.chunk, partial, dbp);
   }
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
