@@ -570,6 +570,7 @@ def run_ours(args, world, rank):
                               "peaks": peaks["source"],
                               "nominal_dense": round(tflops / NOMINAL_DENSE_BF16_TFLOPS, 4)},
         "peak_mem_gb": round(torch.cuda.max_memory_allocated(dev) / 1e9, 2),
+        "expert_rows": (st.expert_offsets[1:] - st.expert_offsets[:-1]).cpu().tolist(),
         "fwd": {"tokens_per_s": round(tokens / (ms_fwd / 1e3), 1), "ms_per_step": round(ms_fwd, 4),
                 "tflops": round(fl["fwd"] / (ms_fwd / 1e3) / 1e12, 1)},
         "e2e": {"value": round(tokens / (ms_e2e / 1e3), 1), "unit": "tokens/s",

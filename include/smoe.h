@@ -167,6 +167,18 @@ int smoe_sort(const int32_t* topk_idx, int T, int k, int E, int32_t* sorted_slot
 int smoe_sort_static(const int32_t* topk_idx, int T, int k, int E, int32_t* sorted_slot,
                      int32_t* expert_offsets, void* stream);
 
+/* smoe_selftest_wait_timeout: a check of the failure path (no counterpart on the
+ * pages).  Launches one small kernel whose thread waits, through the same bounded
+ * wait that every pipeline barrier of the GEMM kernels uses, on a barrier that
+ * nothing completes.  After limit_us microseconds (0 < limit_us <= 1e6) the wait
+ * gives up and records the timeout in the device error word, exactly as a stalled
+ * GEMM pipeline would; the next smoe_check on the stream returns SMOE_ERR_TIMEOUT
+ * and clears the word.  Nothing faults and nothing hangs: a caller or a test can
+ * confirm that a device-side stall becomes an error status on the host.
+ * Returns SMOE_OK once the kernel is launched, SMOE_ERR_INVALID_ARG for a limit
+ * out of range, SMOE_ERR_CUDA for a launch error. */
+int smoe_selftest_wait_timeout(int limit_us, void* stream);
+
 /* ---------------------------------------------------------------------------
  * ParallelLinear [rev1, rev2, art]
  *

@@ -69,6 +69,7 @@ def lib():
                                  _vp, _vp, _vp, _vp, _c_size, _vp]
     L.smoe_sort.argtypes = [_vp, _c_int, _c_int, _c_int, _vp, _vp, _vp, _c_size, _vp]
     L.smoe_sort_static.argtypes = [_vp, _c_int, _c_int, _c_int, _vp, _vp, _vp]
+    L.smoe_selftest_wait_timeout.argtypes = [_c_int, _vp]
     L.parallel_linear_fwd_workspace_size.restype = _c_size
     L.parallel_linear_fwd_workspace_size.argtypes = [_c_int] * 6
     L.parallel_linear_fwd.argtypes = [_vp, _c_int, _c_int, _vp, _c_int, _c_int, _vp, _vp, _c_int,
@@ -204,6 +205,12 @@ def smoe_sort(topk_idx, E, stream=None):
     _check(lib().smoe_sort(_ptr(topk_idx), T, k, E, _ptr(ss), _ptr(off), _ptr(ws), ws.numel(),
                            _stream(stream)))
     return ss, off
+
+
+def smoe_selftest_wait_timeout(limit_us: int, stream=None):
+    """Run the library's bounded device wait on a barrier nothing completes; the
+    next smoe_check returns SMOE_ERR_TIMEOUT (see smoe.h)."""
+    _check(lib().smoe_selftest_wait_timeout(int(limit_us), _stream(stream)))
 
 
 def smoe_sort_static(topk_idx, E, sorted_slot=None, expert_offsets=None, stream=None):

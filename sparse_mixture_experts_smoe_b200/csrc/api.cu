@@ -18,9 +18,17 @@
 #include <string>
 #include <vector>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "common.cuh"
 
 namespace smoe {
+
+// NVTX range around each entry point (a no-op unless a tool is attached).
+struct NvtxScope {
+  explicit NvtxScope(const char* name) { nvtxRangePushA(name); }
+  ~NvtxScope() { nvtxRangePop(); }
+};
 int simt_tile_cols();
 int tc_tile_cols();
 }  // namespace smoe
@@ -344,6 +352,7 @@ size_t smoe_workspace_size(int op, int T, int k, int E, int d, int f, smoe_dtype
 
 int smoe_route(const void* x, const void* w_r, const float* b_r, int T, int d, int E, int k,
                smoe_dtype dt, int32_t* topk_idx, float* gates, void* stream) {
+  smoe::NvtxScope nvtx_scope("smoe_route");
   if (T < 0 || d <= 0 || E <= 0 || k <= 0) return fail(SMOE_ERR_INVALID_ARG, "bad sizes");
   if (k > E || k > 16 || E > 128) return fail(SMOE_ERR_INVALID_ARG, "need 1 <= k <= min(E,16), E <= 128");
   if (d % 8) return fail(SMOE_ERR_INVALID_ARG, "d must be a multiple of 8");
@@ -363,6 +372,7 @@ int smoe_route(const void* x, const void* w_r, const float* b_r, int T, int d, i
 int smoe_route_bwd(const void* x, const void* w_r, const int32_t* topk_idx, const float* gates,
                    const float* dgates, int T, int d, int E, int k, smoe_dtype dt, void* dx,
                    float* dw_r, float* db_r, void* workspace, size_t ws_bytes, void* stream) {
+  smoe::NvtxScope nvtx_scope("smoe_route_bwd");
   if (T < 0 || d <= 0 || E <= 0 || k <= 0 || k > E || E > 128)
     return fail(SMOE_ERR_INVALID_ARG, "bad sizes");
   if (d % 8) return fail(SMOE_ERR_INVALID_ARG, "d must be a multiple of 8");
@@ -390,6 +400,7 @@ int smoe_route_bwd(const void* x, const void* w_r, const int32_t* topk_idx, cons
 
 int smoe_sort(const int32_t* topk_idx, int T, int k, int E, int32_t* sorted_slot,
               int32_t* expert_offsets, void* workspace, size_t ws_bytes, void* stream) {
+  smoe::NvtxScope nvtx_scope("smoe_sort");
   if (T < 0 || k <= 0 || E <= 0 || E > 1024) return fail(SMOE_ERR_INVALID_ARG, "bad sizes (E <= 1024)");
   NEED(expert_offsets, "expert_offsets");
   cudaStream_t s = (cudaStream_t)stream;
@@ -445,6 +456,7 @@ int parallel_linear_fwd(const void* x, int x_rows, int K, const void* w, int N, 
                         int fan_out, int grouped_in, int grouped_out, const float* gates,
                         int combine_k, void* y, smoe_dtype dt, void* workspace, size_t ws_bytes,
                         void* stream) {
+  smoe::NvtxScope nvtx_scope("parallel_linear_fwd");
   int rc = validate_pl(x, x_rows, K, w, N, E, sorted_slot, expert_offsets, num_slots, fan_out,
                        grouped_in, grouped_out, combine_k, dt);
   if (rc != SMOE_OK) return rc;
@@ -492,6 +504,7 @@ int parallel_linear_bwd(const void* dy, const void* x, const void* w, int x_rows
                         int num_slots, int fan_out, int grouped_in, int grouped_out,
                         const float* gates, int combine_k, void* dx, float* dw, float* dgates,
                         smoe_dtype dt, void* workspace, size_t ws_bytes, void* stream) {
+  smoe::NvtxScope nvtx_scope("parallel_linear_bwd");
   int rc = validate_pl(x, x_rows, K, w, N, E, sorted_slot, expert_offsets, num_slots, fan_out,
                        grouped_in, grouped_out, combine_k, dt);
   if (rc != SMOE_OK) return rc;
@@ -582,6 +595,7 @@ size_t smoe_mlp_workspace_size(const smoe_mlp_desc* desc, int backward) {
 }
 
 int smoe_mlp_fwd(const smoe_mlp_desc* desc, const smoe_mlp_tensors* t, void* stream) {
+  smoe::NvtxScope nvtx_scope("smoe_mlp_fwd");
   int rc = validate_mlp_desc(desc);
   if (rc != SMOE_OK) return rc;
   NEED(t, "tensors");
@@ -631,6 +645,7 @@ int smoe_mlp_fwd(const smoe_mlp_desc* desc, const smoe_mlp_tensors* t, void* str
 }
 
 int smoe_mlp_bwd(const smoe_mlp_desc* desc, const smoe_mlp_tensors* t, void* stream) {
+  smoe::NvtxScope nvtx_scope("smoe_mlp_bwd");
   int rc = validate_mlp_desc(desc);
   if (rc != SMOE_OK) return rc;
   NEED(t, "tensors");

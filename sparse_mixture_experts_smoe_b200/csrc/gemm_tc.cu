@@ -105,15 +105,15 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
-// Bounded wait: false once the CTA has aborted or after kWaitNs (then it aborts).
+// Bounded wait: false once the CTA has aborted or after limit_ns (then it aborts).
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
-                                       unsigned* err) {
+                                       unsigned* err, unsigned long long limit_ns = kWaitNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = global_ns();
   for (;;) {
     if (mbar_try_wait(bar, parity)) return true;
     if (*abort_flag) return false;
-    if (global_ns() - t0 > kWaitNs) {
+    if (global_ns() - t0 > limit_ns) {
       *abort_flag = 1;
       report_error(err, ERRBIT_TIMEOUT);
       return false;
@@ -1346,6 +1346,22 @@ dw_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
 }
 
 // ---------------------------------------------------------------------------
+// Self-test of the failure path: the bounded wait on a barrier that nothing
+// completes gives up after limit_ns and records the timeout.
+// ---------------------------------------------------------------------------
+__global__ void wait_timeout_selftest_kernel(unsigned long long limit_ns, unsigned* err) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) (void)mbar_wait(&bar, 0, &abort_flag, err, limit_ns);
+}
+
+// ---------------------------------------------------------------------------
 // Host side: tensor maps and launches
 // ---------------------------------------------------------------------------
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
@@ -1572,3 +1588,16 @@ cudaError_t launch_dw_gemm_tc(const DwGemm& g_in, cudaStream_t s) {
 }
 
 }  // namespace smoe
+
+extern "C" int smoe_selftest_wait_timeout(int limit_us, void* stream) {
+  using namespace smoe;
+  if (limit_us <= 0 || limit_us > 1000000)
+    return api_fail(SMOE_ERR_INVALID_ARG, "limit_us must be in (0, 1e6]");
+  cudaError_t st;
+  unsigned* err = api_error_word(&st);
+  if (!err) return api_fail(SMOE_ERR_CUDA, "smoe_selftest_wait_timeout: %s", cudaGetErrorString(st));
+  wait_timeout_selftest_kernel<<<1, 32, 0, (cudaStream_t)stream>>>(1000ull * (unsigned long long)limit_us, err);
+  st = cudaGetLastError();
+  return st == cudaSuccess ? SMOE_OK
+                           : api_fail(SMOE_ERR_CUDA, "smoe_selftest_wait_timeout: %s", cudaGetErrorString(st));
+}

@@ -136,3 +136,16 @@ def test_sort_reports_out_of_range_ids():
     smoe.smoe_sort(idx, 8)
     assert smoe.smoe_check() == -4       # SMOE_ERR_DATA
     assert smoe.smoe_check() == 0        # the word is cleared once read
+
+
+def test_device_wait_timeout_becomes_host_error():
+    """A bounded device wait on a barrier nothing completes gives up, and the host
+    sees SMOE_ERR_TIMEOUT from smoe_check; the word is then clear and the library
+    keeps working (the failure path without a fault or a hang)."""
+    smoe.smoe_selftest_wait_timeout(20000)  # 20 ms
+    assert smoe.smoe_check() == -5  # SMOE_ERR_TIMEOUT
+    assert b"bounded device wait" in smoe.lib().smoe_last_error()
+    assert smoe.smoe_check() == 0
+    x = torch.randn(64, 128, device="cuda").to(torch.bfloat16)
+    w_r = (torch.randn(128, 8, device="cuda") / 128 ** 0.5).to(torch.bfloat16)
+    _check_route(x, w_r, None, 2)
