@@ -115,3 +115,24 @@ def test_workspace_queries_are_consistent():
             assert bwd > fwd
             assert L.smoe_workspace_size(3, T, k, E, d, f, dt) == fwd
             assert L.smoe_workspace_size(4, T, k, E, d, f, dt) == bwd
+
+
+def test_workspaces_hold_no_copy_of_token_rows():
+    """The library never allocates, so a grouped or padded copy of x or dY would have
+    to live in its workspace.  Mixtral-shaped sizes: the forward workspace is exactly
+    the sort counts plus one fp32 [T*k, d] buffer (the k-way combine's slot rows);
+    what the backward needs beyond its documented large buffers (dH, gA and the fp32
+    dx slot rows) is far smaller than one bf16 [T*k, d] copy."""
+    import ctypes
+    import sparse_mixture_experts_smoe_b200 as smoe
+    T, d, f, E, k = 16384, 4096, 14336, 8, 2
+    S = T * k
+    L = smoe.lib()
+    a256 = lambda n: (n + 255) // 256 * 256  # noqa: E731
+    sort = L.smoe_workspace_size(0, T, k, E, d, f, 1)
+    desc = smoe.MlpDesc(T, d, f, E, k, smoe.ACT["swiglu"], smoe.BF16)
+    fwd = L.smoe_mlp_workspace_size(ctypes.byref(desc), 0)
+    bwd = L.smoe_mlp_workspace_size(ctypes.byref(desc), 1)
+    assert fwd == a256(sort) + a256(S * d * 4)
+    big = a256(S * 2 * f * 2) + a256(S * f * 2) + a256(S * d * 4)
+    assert bwd - big < S * d * 2 // 4

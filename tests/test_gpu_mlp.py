@@ -201,3 +201,24 @@ def test_moa_projections_full_size_sampled():
     assert_close("do", do[L(rows_i)], ro["dx"], bf)
     assert_close("dWo", dwo[:, :, L(cols_o)], ro["dw"], bf)
     assert_close("dgates", dgt[L(slots)], ro["dg"], bf)
+
+
+def test_library_allocates_nothing():
+    """With the caller's buffers in place, a forward and backward step allocates no
+    device memory at all (the library only uses the caller's workspace)."""
+    cfg = REDUCED["swiglu_bf16"]
+    inp = make_mlp_inputs(cfg, seed=2, device="cuda")
+    st = smoe.SMoEMLPState(cfg["T"], cfg["d"], cfg["f"], cfg["E"], cfg["k"], cfg["act"],
+                           torch.bfloat16, "cuda")
+    p = (inp["x"], inp["w_r"], inp["b_r"], inp["w1"], inp["w2"])
+    smoe.smoe_mlp_fwd(st, *p)
+    smoe.smoe_mlp_bwd(st, *p, inp["dy"])
+    torch.cuda.synchronize()
+    torch.cuda.reset_peak_memory_stats()
+    before = torch.cuda.memory_allocated()
+    for _ in range(2):
+        smoe.smoe_mlp_fwd(st, *p)
+        smoe.smoe_mlp_bwd(st, *p, inp["dy"])
+    torch.cuda.synchronize()
+    assert torch.cuda.max_memory_allocated() == before
+    assert smoe.smoe_check() == 0

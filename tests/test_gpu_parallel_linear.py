@@ -94,3 +94,62 @@ def test_parallel_linear_is_deterministic():
         outs.append([y] + list(r))
     for a, b in zip(*outs):
         assert torch.equal(a, b)
+
+
+SLICES = [0, 1, 127, 128, 129, 255, 256, 257]  # rows per expert: empty, one row, tile edges
+
+
+def _sized_problem(dtype, mode, gated, sizes, seed=0):
+    """k = 1 routing with exactly sizes[e] rows for expert e (shuffled over tokens)."""
+    K, N = (264, 392) if dtype == torch.bfloat16 else (136, 72)
+    E, T, k = len(sizes), sum(sizes), 1
+    gi, go, fo_k, comb = MODES[mode]
+    g = torch.Generator(device="cuda").manual_seed(seed)
+    ids = torch.cat([torch.full((n,), e, dtype=torch.int32) for e, n in enumerate(sizes)])
+    perm = torch.randperm(T, generator=torch.Generator().manual_seed(seed))
+    idx = ids[perm].reshape(T, k).cuda()
+    ss, off = smoe.smoe_sort(idx, E)
+    assert off.cpu().tolist() == np.concatenate([[0], np.cumsum(sizes)]).tolist()
+    x = torch.randn(T, K, generator=g, device="cuda").to(dtype)
+    w = (torch.randn(E, K, N, generator=g, device="cuda") / K ** 0.5).to(dtype)
+    gates = torch.rand(T, generator=g, device="cuda") if gated else None
+    dy = torch.randn(T, N, generator=g, device="cuda").to(dtype)
+    return dict(ss=ss, off=off, x=x, w=w, gates=gates, fan_out=1, gi=gi, go=go,
+                ck=k if comb else 0, dy=dy)
+
+
+def _check_problem(P, dtype, gated):
+    y = smoe.parallel_linear_fwd(P["x"], P["w"], P["ss"], P["off"], P["fan_out"], P["gi"], P["go"],
+                                 P["gates"], P["ck"])
+    dx, dw, dg = smoe.parallel_linear_bwd(P["dy"], P["x"], P["w"], P["ss"], P["off"], P["fan_out"],
+                                          P["gi"], P["go"], P["gates"], P["ck"], want_dgates=gated)
+    torch.cuda.synchronize()
+    assert smoe.smoe_check() == 0
+    ss, off = P["ss"].cpu().numpy(), P["off"].cpu().numpy()
+    gts = None if P["gates"] is None else P["gates"].cpu().double().numpy()
+    assert_close("y", y, oracle.pl_fwd(P["x"].cpu(), P["w"].cpu(), ss, off, P["fan_out"], P["gi"],
+                                       P["go"], gts, P["ck"]), dtype)
+    ref = oracle.pl_bwd(P["dy"].cpu(), P["x"].cpu(), P["w"].cpu(), ss, off, P["fan_out"], P["gi"],
+                        P["go"], gts, P["ck"], want_dg=gated)
+    assert_close("dx", dx, ref["dx"], dtype)
+    assert_close("dw", dw, ref["dw"], dtype)
+    if gated:
+        assert_close("dgates", dg, ref["dg"], dtype)
+    return dw
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("mode", list(MODES))
+@pytest.mark.parametrize("gated", [False, True])
+def test_parallel_linear_tile_boundaries(dtype, mode, gated):
+    """Expert slices of 0, 1, 127, 128, 129, 255, 256 and 257 rows: empty experts,
+    one-row tiles, exact tiles, one row past a tile (ragged warps and the per-row
+    store path next to the boxed one)."""
+    dw = _check_problem(_sized_problem(dtype, mode, gated, SLICES), dtype, gated)
+    assert np.all(dw[0].cpu().numpy() == 0.0)
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_parallel_linear_all_tokens_to_one_expert(dtype):
+    dw = _check_problem(_sized_problem(dtype, "scatter2group_fanout", True, [0, 0, 300, 0]), dtype, True)
+    assert np.all(dw[[0, 1, 3]].cpu().numpy() == 0.0)
