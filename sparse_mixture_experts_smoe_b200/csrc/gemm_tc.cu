@@ -1433,7 +1433,7 @@ cudaError_t prep(K kern, size_t bytes) {
 }
 
 struct EpiMaps {
-  CUtensorMap out, out2, xa, xh;
+  CUtensorMap out{}, out2{}, xa{}, xh{};  // zero: unused maps are passed but never read
   int flags = 0;
 };
 
@@ -1527,7 +1527,6 @@ cudaError_t launch_grouped_gemm_tc(const GroupedGemm& g, cudaStream_t s) {
   // Boxed (TMA tensor) epilogue stores when every output is bf16 in grouped
   // rows; boxed ACT_BWD input loads when its inputs are in grouped rows.
   EpiMaps m;
-  memset(&m, 0, sizeof(m));
   const int parts = (g.act == SMOE_ACT_SWIGLU && g.epi != EPI_STORE) ? 2 : 1;
   bool st = (g.out != nullptr || g.out2 != nullptr) &&
             (g.out == nullptr || (!g.out_f32 && g.out_mode == ROWS_GROUPED));
