@@ -155,19 +155,24 @@ int check_tc(smoe_dtype dt) {
 // ParallelLinear workspace layout
 // ---------------------------------------------------------------------------
 struct PLFwdWs {
-  float* comb = nullptr;
+  float* comb = nullptr;   // [num_slots, N] fp32 slot rows, grouped order
+  int32_t* inv = nullptr;  // [num_slots] grouped row of each slot
   size_t bytes = 0;
 };
 PLFwdWs pl_fwd_layout(void* ws, int num_slots, int N, int combine_k) {
   Carve c(ws);
   PLFwdWs l;
-  if (combine_k > 0) l.comb = (float*)c.take((size_t)num_slots * N * sizeof(float));
+  if (combine_k > 0) {
+    l.comb = (float*)c.take((size_t)num_slots * N * sizeof(float));
+    l.inv = (int32_t*)c.take((size_t)num_slots * sizeof(int32_t));
+  }
   l.bytes = c.off;
   return l;
 }
 
 struct PLBwdWs {
-  float* dx_comb = nullptr;  // [num_slots, K] fp32 when dx needs a fan-out combine
+  float* dx_comb = nullptr;  // [num_slots, K] fp32 when dx needs a fan-out combine (grouped order)
+  int32_t* inv = nullptr;    // [num_slots] grouped row of each slot, with dx_comb
   float* dg_part = nullptr;  // [num_slots, dg_ld]
   void* gx = nullptr;        // [num_slots, K] dtype: gates * x rows, grouped
   int dg_ld = 0;
@@ -177,8 +182,10 @@ PLBwdWs pl_bwd_layout(void* ws, int num_slots, int K, int grouped_in, int fan_ou
                       int want_dx, int want_dw, int want_dg, smoe_dtype dt) {
   Carve c(ws);
   PLBwdWs l;
-  if (want_dx && !grouped_in && fan_out > 1)
+  if (want_dx && !grouped_in && fan_out > 1) {
     l.dx_comb = (float*)c.take((size_t)num_slots * K * sizeof(float));
+    l.inv = (int32_t*)c.take((size_t)num_slots * sizeof(int32_t));
+  }
   if (has_gates && want_dg) {
     l.dg_ld = cdiv(K, act_tile_cols(dt));
     l.dg_part = (float*)c.take((size_t)num_slots * l.dg_ld * sizeof(float));
@@ -193,11 +200,12 @@ PLBwdWs pl_bwd_layout(void* ws, int num_slots, int K, int grouped_in, int fan_ou
 // ---------------------------------------------------------------------------
 struct MlpWs {
   void* sort = nullptr;
-  float* ycomb = nullptr;   // fwd: [S, d] fp32
+  float* ycomb = nullptr;   // fwd: [S, d] fp32 slot rows, grouped order
   float* dg_part = nullptr; // bwd: [S, dg_ld]
   void* dh = nullptr;       // bwd: [S, m*f] dtype (grouped dH)
   void* ga = nullptr;       // bwd: [S, f] dtype (gates * A)
-  float* dxcomb = nullptr;  // bwd: [S, d] fp32
+  float* dxcomb = nullptr;  // bwd: [S, d] fp32 slot rows, grouped order
+  int32_t* inv = nullptr;   // fwd and bwd: [S] grouped row of each slot
   float* dl = nullptr;      // bwd: [T, k]
   float* dg = nullptr;      // bwd: [T, k] when the caller passes no dgates
   float* rpart = nullptr;   // bwd: router dW partials
@@ -211,6 +219,7 @@ MlpWs mlp_layout(void* ws, const smoe_mlp_desc& m, int backward) {
   const size_t S = (size_t)m.T * m.k;
   const smoe_dtype dt = (smoe_dtype)m.dtype;
   l.sort = c.take(sort_workspace_bytes(m.T, m.k, m.E));
+  l.inv = (int32_t*)c.take(S * sizeof(int32_t));
   if (!backward) {
     l.ycomb = (float*)c.take(S * m.d * sizeof(float));
   } else {
@@ -477,16 +486,17 @@ int parallel_linear_fwd(const void* x, int x_rows, int K, const void* w, int N, 
   g.b = w; g.b_kn = 1; g.NW = N; g.n_out = N;
   g.epi = EPI_STORE; g.gates = gates; g.err = err;
   if (combine_k > 0) {
-    g.out_mode = ROWS_GATHER; g.out = l.comb; g.ldo = N; g.out_f32 = 1;
+    g.out_mode = ROWS_GROUPED; g.out = l.comb; g.ldo = N; g.out_f32 = 1;
   } else {
     g.out_mode = grouped_out ? ROWS_GROUPED : ROWS_GATHER; g.out = y; g.ldo = N;
     g.out_f32 = dt == SMOE_F32;
   }
   { PROF("pl.gemm_fwd", 1); SMOE_TRY(run_grouped(g, dt, s), "parallel_linear_fwd gemm"); }
   if (combine_k > 0) {
+    { PROF("pl.invert", 1); SMOE_TRY(launch_invert(sorted_slot, num_slots, l.inv, s), "parallel_linear_fwd invert"); }
     PROF("pl.combine", 1);
-    SMOE_TRY(launch_combine(l.comb, num_slots / combine_k, combine_k, N, y, dt, nullptr, nullptr,
-                            nullptr, 0, s), "parallel_linear_fwd combine");
+    SMOE_TRY(launch_combine(l.comb, l.inv, num_slots / combine_k, combine_k, N, y, dt, nullptr,
+                            nullptr, nullptr, 0, s), "parallel_linear_fwd combine");
   }
   return SMOE_OK;
 }
@@ -543,7 +553,7 @@ int parallel_linear_bwd(const void* dy, const void* x, const void* w, int x_rows
     g.b = w; g.b_kn = 0; g.NW = K; g.n_out = K;
     g.gates = gates; g.err = err;
     g.out_mode = grouped_in ? ROWS_GROUPED : ROWS_GATHER;
-    if (dx_comb) { g.out = l.dx_comb; g.ldo = K; g.out_f32 = 1; }
+    if (dx_comb) { g.out_mode = ROWS_GROUPED; g.out = l.dx_comb; g.ldo = K; g.out_f32 = 1; }
     else { g.out = dx; g.ldo = K; g.out_f32 = dt == SMOE_F32; }
     if (has_g) {
       g.epi = EPI_ACT_BWD; g.act = SMOE_ACT_NONE;
@@ -559,12 +569,14 @@ int parallel_linear_bwd(const void* dy, const void* x, const void* w, int x_rows
     if (dgates) {
       PROF("pl.dg_reduce", 1);
       SMOE_TRY(launch_dg_reduce(l.dg_part, l.dg_ld, cdiv(K, act_tile_cols(dt)), sorted_slot,
-                                num_slots, dgates, s), "parallel_linear_bwd dg");
+                                num_slots, dgates, s, dx && dx_comb ? l.inv : nullptr),
+               "parallel_linear_bwd dg");
     }
     if (dx && dx_comb) {
+      if (!dgates) { PROF("pl.invert", 1); SMOE_TRY(launch_invert(sorted_slot, num_slots, l.inv, s), "parallel_linear_bwd invert"); }
       PROF("pl.combine_dx", 1);
-      SMOE_TRY(launch_combine(l.dx_comb, x_rows, fan_out, K, dx, dt, nullptr, nullptr, nullptr, 0, s),
-               "parallel_linear_bwd dx combine");
+      SMOE_TRY(launch_combine(l.dx_comb, l.inv, x_rows, fan_out, K, dx, dt, nullptr, nullptr,
+                              nullptr, 0, s), "parallel_linear_bwd dx combine");
     }
   }
   if (dw) {
@@ -620,7 +632,7 @@ int smoe_mlp_fwd(const smoe_mlp_desc* desc, const smoe_mlp_tensors* t, void* str
   const int mf = m.act == SMOE_ACT_SWIGLU ? 2 * m.f : m.f;
 
   { PROF("route", 1); SMOE_TRY(launch_route(t->x, t->w_r, t->b_r, m.T, m.d, m.E, m.k, dt, t->topk_idx, t->gates, err, s), "route"); }
-  { PROF("sort", 3); SMOE_TRY(launch_sort(t->topk_idx, m.T, m.k, m.E, t->sorted_slot, t->expert_offsets, l.sort, err, s), "sort"); }
+  { PROF("sort", 3); SMOE_TRY(launch_sort(t->topk_idx, m.T, m.k, m.E, t->sorted_slot, t->expert_offsets, l.sort, err, s, l.inv), "sort"); }
   {  // H = x[gathered] W1, A = act(H)   (scatter -> group, fan-out k)
     GroupedGemm g;
     g.E = m.E; g.num_rows = S; g.offsets = t->expert_offsets; g.sorted_slot = t->sorted_slot;
@@ -631,16 +643,16 @@ int smoe_mlp_fwd(const smoe_mlp_desc* desc, const smoe_mlp_tensors* t, void* str
     g.out2 = t->a; g.ldo2 = m.f; g.err = err;
     { PROF("gemm.fwd_up", 1); SMOE_TRY(run_grouped(g, dt, s), "mlp fwd gemm1"); }
   }
-  {  // y = sum_j g * (A W2)   (group -> scatter, gated, k-way combine)
+  {  // y = sum_j g * (A W2)   (group -> group in fp32, gated; the k-way combine scatters)
     GroupedGemm g;
     g.E = m.E; g.num_rows = S; g.offsets = t->expert_offsets; g.sorted_slot = t->sorted_slot;
     g.K = m.f; g.a = t->a; g.lda = m.f; g.a_rows = S; g.a_mode = ROWS_GROUPED;
     g.b = t->w2; g.b_kn = 1; g.NW = m.d; g.n_out = m.d;
     g.epi = EPI_STORE; g.gates = t->gates;
-    g.out_mode = ROWS_GATHER; g.out = l.ycomb; g.ldo = m.d; g.out_f32 = 1; g.err = err;
+    g.out_mode = ROWS_GROUPED; g.out = l.ycomb; g.ldo = m.d; g.out_f32 = 1; g.err = err;
     { PROF("gemm.fwd_down", 1); SMOE_TRY(run_grouped(g, dt, s), "mlp fwd gemm2"); }
   }
-  { PROF("combine.y", 1); SMOE_TRY(launch_combine(l.ycomb, m.T, m.k, m.d, t->y, dt, nullptr, nullptr, nullptr, 0, s), "mlp fwd combine"); }
+  { PROF("combine.y", 1); SMOE_TRY(launch_combine(l.ycomb, l.inv, m.T, m.k, m.d, t->y, dt, nullptr, nullptr, nullptr, 0, s), "mlp fwd combine"); }
   return SMOE_OK;
 }
 
@@ -690,7 +702,7 @@ int smoe_mlp_bwd(const smoe_mlp_desc* desc, const smoe_mlp_tensors* t, void* str
     g.dg_partial = l.dg_part; g.dg_ld = l.dg_ld; g.err = err;
     { PROF("gemm.bwd_dA", 1); SMOE_TRY(run_grouped(g, dt, s), "mlp bwd gemm dA"); }
   }
-  { PROF("dg_reduce", 1); SMOE_TRY(launch_dg_reduce(l.dg_part, l.dg_ld, l.dg_ld, t->sorted_slot, S, dg, s), "mlp bwd dg"); }
+  { PROF("dg_reduce", 1); SMOE_TRY(launch_dg_reduce(l.dg_part, l.dg_ld, l.dg_ld, t->sorted_slot, S, dg, s, l.inv), "mlp bwd dg"); }
   { PROF("route_dl", 1); SMOE_TRY(launch_route_dl(t->gates, dg, m.T, m.k, l.dl, s), "mlp bwd dl"); }
   {  // dW2[e] = sum_i (g A)_i^T dy[t_i]
     DwGemm g;
@@ -710,20 +722,20 @@ int smoe_mlp_bwd(const smoe_mlp_desc* desc, const smoe_mlp_tensors* t, void* str
     g.dw = t->dw1; g.err = err;
     { PROF("gemm.bwd_dW1", 1); SMOE_TRY(run_dw(g, dt, s), "mlp bwd dW1"); }
   }
-  {  // per-slot dx rows: dH_i W1[e]^T  (group -> scatter, fp32, slot order)
+  {  // per-slot dx rows: dH_i W1[e]^T  (group -> group, fp32; the combine scatters)
     GroupedGemm g;
     g.E = m.E; g.num_rows = S; g.offsets = t->expert_offsets; g.sorted_slot = t->sorted_slot;
     g.K = mf; g.a = l.dh; g.lda = mf; g.a_rows = S; g.a_mode = ROWS_GROUPED;
     g.b = t->w1; g.b_kn = 0; g.NW = m.d; g.n_out = m.d;
     g.epi = EPI_STORE;
-    g.out_mode = ROWS_GATHER; g.out = l.dxcomb; g.ldo = m.d; g.out_f32 = 1; g.err = err;
+    g.out_mode = ROWS_GROUPED; g.out = l.dxcomb; g.ldo = m.d; g.out_f32 = 1; g.err = err;
     { PROF("gemm.bwd_dx", 1); SMOE_TRY(run_grouped(g, dt, s), "mlp bwd gemm dx"); }
   }
   // dx[t] = sum_j rows + router term sum_j dl W_r[:, e_j]
   { PROF("transpose_wr", 1);
   SMOE_TRY(launch_transpose_wr(t->w_r, m.d, m.E, dt, l.wrt, s), "mlp bwd router transpose"); }
   { PROF("combine.dx", 1);
-  SMOE_TRY(launch_combine(l.dxcomb, m.T, m.k, m.d, t->dx, dt, l.dl, t->topk_idx, l.wrt, m.E, s),
+  SMOE_TRY(launch_combine(l.dxcomb, l.inv, m.T, m.k, m.d, t->dx, dt, l.dl, t->topk_idx, l.wrt, m.E, s),
            "mlp bwd dx combine"); }
   { PROF("route_dw", 2);
   SMOE_TRY(launch_route_dw(t->x, t->topk_idx, l.dl, m.T, m.d, m.E, m.k, dt, l.rpart, l.r_chunks,

@@ -6,50 +6,97 @@
 //
 // The k slots of a token are owned by k different experts, so their products
 // come from different CTAs; summing them with atomics would make the result
-// depend on scheduling.  Instead the GEMM epilogue stores each slot's row at
-// row p = t*k + j of an fp32 buffer, and this pass sums the k rows of each token
-// in ascending j (group-to-scatter with combine, library page of arXiv 2403.08245,
+// depend on scheduling.  Instead the GEMM epilogue stores each slot's row in an
+// fp32 buffer, in grouped order (row i of slot p = sorted_slot[i], so that whole
+// warps of rows leave as TMA boxes), and this pass sums the k rows of each token
+// in ascending j, finding slot p's row through the inverse permutation
+// inv[p] = i (group-to-scatter with combine, library page of arXiv 2403.08245,
 // review 2 summary).
 #include "common.cuh"
 
 namespace smoe {
 namespace {
 
-// One thread per 4 consecutive columns of one token.  The router term reads the
-// transposed router weight w_rt [E, N] so each selected expert contributes one
-// contiguous 4-element load.
+// Each thread owns kCombV float4 columns of one token, u + v*U for v < kCombV
+// (U threads per token, so every v is a coalesced sweep of the row).  The slot
+// rows sit at grouped positions, so their indices come first; the thread then has
+// kCombV independent 16-byte loads in flight per slot instead of one load behind
+// a dependent index load.  The router term reads the transposed router weight
+// w_rt [E, N] so each selected expert contributes contiguous loads.
+constexpr int kCombV = 4;
+
+// four consecutive elements as one 8- or 16-byte access
+__device__ __forceinline__ float4 load4(const float* p) { return __ldg(reinterpret_cast<const float4*>(p)); }
+__device__ __forceinline__ float4 load4(const bf16* p) {
+  const uint2 r = __ldg(reinterpret_cast<const uint2*>(p));
+  const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&r.x));
+  const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&r.y));
+  return make_float4(a.x, a.y, b.x, b.y);
+}
+__device__ __forceinline__ void store4(float* p, float4 v) { *reinterpret_cast<float4*>(p) = v; }
+__device__ __forceinline__ void store4(bf16* p, float4 v) {
+  __nv_bfloat162 a = __floats2bfloat162_rn(v.x, v.y), b = __floats2bfloat162_rn(v.z, v.w);
+  uint2 r;
+  r.x = *reinterpret_cast<uint32_t*>(&a);
+  r.y = *reinterpret_cast<uint32_t*>(&b);
+  *reinterpret_cast<uint2*>(p) = r;
+}
+
 template <typename TO, typename TW>
-__global__ void combine_kernel(const float* __restrict__ ws, int T_, int ck, int N,
-                               TO* __restrict__ out, const float* __restrict__ dl,
-                               const int32_t* __restrict__ idx, const TW* __restrict__ w_rt,
-                               int E) {
+__global__ void __launch_bounds__(256)
+combine_kernel(const float* __restrict__ ws, const int32_t* __restrict__ inv, int T_, int ck,
+               int N, TO* __restrict__ out, const float* __restrict__ dl,
+               const int32_t* __restrict__ idx, const TW* __restrict__ w_rt, int E) {
   const int n4 = N / 4;
+  const int U = (n4 + kCombV - 1) / kCombV;
   const size_t q = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (q >= (size_t)T_ * n4) return;
-  const int t = (int)(q / n4);
-  const int c = (int)(q % n4) * 4;
-  float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (q >= (size_t)T_ * U) return;
+  const int t = (int)(q / U);
+  const int u = (int)(q % U);
+  const int S = T_ * ck;
+  float4 acc[kCombV];
+#pragma unroll
+  for (int v = 0; v < kCombV; ++v) acc[v] = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 2
   for (int j = 0; j < ck; ++j) {
-    const float4 v = *reinterpret_cast<const float4*>(ws + ((size_t)t * ck + j) * N + c);
-    s.x += v.x; s.y += v.y; s.z += v.z; s.w += v.w;
+    const int p = t * ck + j;
+    const int row = inv ? __ldg(inv + p) : p;
+    if (row < 0 || row >= S) continue;  // not a permutation: a data error flagged upstream
+    const float4* src = reinterpret_cast<const float4*>(ws + (size_t)row * N);
+    float4 x[kCombV];
+#pragma unroll
+    for (int v = 0; v < kCombV; ++v) {
+      const int c4 = u + v * U;
+      x[v] = c4 < n4 ? __ldg(src + c4) : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+    for (int v = 0; v < kCombV; ++v) {
+      acc[v].x += x[v].x; acc[v].y += x[v].y; acc[v].z += x[v].z; acc[v].w += x[v].w;
+    }
   }
   if (dl != nullptr) {
     for (int j = 0; j < ck; ++j) {
       const int e = idx[(size_t)t * ck + j];
       if (e < 0 || e >= E) continue;
       const float g = dl[(size_t)t * ck + j];
-      const TW* w = w_rt + (size_t)e * N + c;
-      s.x = fmaf(g, to_f(w[0]), s.x);
-      s.y = fmaf(g, to_f(w[1]), s.y);
-      s.z = fmaf(g, to_f(w[2]), s.z);
-      s.w = fmaf(g, to_f(w[3]), s.w);
+#pragma unroll
+      for (int v = 0; v < kCombV; ++v) {
+        const int c4 = u + v * U;
+        if (c4 >= n4) continue;
+        const float4 w = load4(w_rt + (size_t)e * N + 4 * c4);
+        acc[v].x = fmaf(g, w.x, acc[v].x);
+        acc[v].y = fmaf(g, w.y, acc[v].y);
+        acc[v].z = fmaf(g, w.z, acc[v].z);
+        acc[v].w = fmaf(g, w.w, acc[v].w);
+      }
     }
   }
-  TO* o = out + (size_t)t * N + c;
-  o[0] = from_f<TO>(s.x);
-  o[1] = from_f<TO>(s.y);
-  o[2] = from_f<TO>(s.z);
-  o[3] = from_f<TO>(s.w);
+#pragma unroll
+  for (int v = 0; v < kCombV; ++v) {
+    const int c4 = u + v * U;
+    if (c4 >= n4) continue;
+    store4(out + (size_t)t * N + 4 * c4, acc[v]);
+  }
 }
 
 // w_rt[e][i] = w_r[i][e]
@@ -63,12 +110,23 @@ __global__ void transpose_kernel(const T* __restrict__ w_r, int d, int E, T* __r
 
 __global__ void dg_reduce_kernel(const float* __restrict__ partial, int ld, int n_tiles,
                                  const int32_t* __restrict__ sorted_slot, int num_rows,
-                                 float* __restrict__ dg) {
+                                 float* __restrict__ dg, int32_t* __restrict__ inv) {
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= num_rows) return;
   float s = 0.0f;
   for (int c = 0; c < n_tiles; ++c) s += partial[(size_t)i * ld + c];
-  dg[sorted_slot[i]] = s;
+  const int p = sorted_slot[i];
+  if (p < 0 || p >= num_rows) return;  // reported by the GEMM that read it
+  dg[p] = s;
+  if (inv) inv[p] = i;
+}
+
+__global__ void invert_kernel(const int32_t* __restrict__ sorted_slot, int num_rows,
+                              int32_t* __restrict__ inv) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= num_rows) return;
+  const int p = sorted_slot[i];
+  if (p >= 0 && p < num_rows) inv[p] = i;
 }
 
 template <typename T>
@@ -97,24 +155,29 @@ cudaError_t launch_transpose_wr(const void* w_r, int d, int E, smoe_dtype dt, vo
   return cudaGetLastError();
 }
 
-cudaError_t launch_combine(const float* ws, int T_, int ck, int N, void* out, smoe_dtype out_dt,
-                           const float* dl, const int32_t* idx, const void* w_rt, int E,
-                           cudaStream_t s) {
-  const size_t n = (size_t)T_ * (N / 4);
+cudaError_t launch_combine(const float* ws, const int32_t* inv, int T_, int ck, int N, void* out,
+                           smoe_dtype out_dt, const float* dl, const int32_t* idx,
+                           const void* w_rt, int E, cudaStream_t s) {
+  const size_t n = (size_t)T_ * cdiv(N / 4, kCombV);
   const unsigned blocks = (unsigned)((n + 255) / 256);
   if (out_dt == SMOE_BF16)
-    combine_kernel<bf16, bf16><<<blocks, 256, 0, s>>>(ws, T_, ck, N, (bf16*)out, dl, idx,
+    combine_kernel<bf16, bf16><<<blocks, 256, 0, s>>>(ws, inv, T_, ck, N, (bf16*)out, dl, idx,
                                                       (const bf16*)w_rt, E);
   else
-    combine_kernel<float, float><<<blocks, 256, 0, s>>>(ws, T_, ck, N, (float*)out, dl, idx,
+    combine_kernel<float, float><<<blocks, 256, 0, s>>>(ws, inv, T_, ck, N, (float*)out, dl, idx,
                                                         (const float*)w_rt, E);
   return cudaGetLastError();
 }
 
+cudaError_t launch_invert(const int32_t* sorted_slot, int num_rows, int32_t* inv, cudaStream_t s) {
+  invert_kernel<<<cdiv(num_rows, 256), 256, 0, s>>>(sorted_slot, num_rows, inv);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_dg_reduce(const float* partial, int ld, int n_tiles, const int32_t* sorted_slot,
-                             int num_rows, float* dg, cudaStream_t s) {
+                             int num_rows, float* dg, cudaStream_t s, int32_t* inv) {
   dg_reduce_kernel<<<cdiv(num_rows, 256), 256, 0, s>>>(partial, ld, n_tiles, sorted_slot,
-                                                       num_rows, dg);
+                                                       num_rows, dg, inv);
   return cudaGetLastError();
 }
 

@@ -87,20 +87,25 @@ cudaError_t launch_route_dx(const float* dl, const int32_t* idx, const void* w_r
                             int E, int k, smoe_dtype dt, void* dx, cudaStream_t s);
 
 size_t sort_workspace_bytes(int T, int k, int E);
+// inv (nullable): also write inv[sorted_slot[i]] = i
 cudaError_t launch_sort(const int32_t* idx, int T, int k, int E, int32_t* sorted_slot,
-                        int32_t* offsets, void* ws, unsigned* err, cudaStream_t s);
+                        int32_t* offsets, void* ws, unsigned* err, cudaStream_t s,
+                        int32_t* inv = nullptr);
 
-// out[t] = sum_{j<ck} ws[t*ck + j] (+ sum_j dl[t*ck+j] * w_rt[idx[t*ck+j], :] if dl),
-// w_rt being the router weight transposed to [E, N]
-cudaError_t launch_combine(const float* ws, int T, int ck, int N, void* out, smoe_dtype out_dt,
-                           const float* dl, const int32_t* idx, const void* w_rt, int E,
-                           cudaStream_t s);
+// out[t] = sum_{j<ck} ws[row(t*ck + j)] (+ sum_j dl[t*ck+j] * w_rt[idx[t*ck+j], :] if dl),
+// w_rt being the router weight transposed to [E, N]; row(p) = inv[p] (the slot's
+// grouped row) or p when inv is null
+cudaError_t launch_combine(const float* ws, const int32_t* inv, int T, int ck, int N, void* out,
+                           smoe_dtype out_dt, const float* dl, const int32_t* idx,
+                           const void* w_rt, int E, cudaStream_t s);
+// inv[sorted_slot[i]] = i for i < num_rows
+cudaError_t launch_invert(const int32_t* sorted_slot, int num_rows, int32_t* inv, cudaStream_t s);
 // w_rt[e][i] = w_r[i][e]
 cudaError_t launch_transpose_wr(const void* w_r, int d, int E, smoe_dtype dt, void* w_rt,
                                 cudaStream_t s);
-// dg[sorted_slot[i]] = sum_{c < n_tiles} partial[i*ld + c]
+// dg[sorted_slot[i]] = sum_{c < n_tiles} partial[i*ld + c]; inv (nullable) as launch_invert
 cudaError_t launch_dg_reduce(const float* partial, int ld, int n_tiles, const int32_t* sorted_slot,
-                             int num_rows, float* dg, cudaStream_t s);
+                             int num_rows, float* dg, cudaStream_t s, int32_t* inv = nullptr);
 // out[i] = gates[sorted_slot[i]] * src[row(i)]  (grouped rows, dtype)
 cudaError_t launch_gather_scale(const void* src, int ld_src, int mode, int fan_out,
                                 const int32_t* sorted_slot, const float* gates, int num_rows,

@@ -89,7 +89,8 @@ sort_scan_kernel(int32_t* __restrict__ counts, int n_blocks, int E, int32_t* __r
 
 __global__ void __launch_bounds__(kSortThreads)
 sort_scatter_kernel(const int32_t* __restrict__ idx, int S, int E,
-                    const int32_t* __restrict__ base, int32_t* __restrict__ sorted_slot) {
+                    const int32_t* __restrict__ base, int32_t* __restrict__ sorted_slot,
+                    int32_t* __restrict__ inv) {
   __shared__ int run[kSortMaxE];                    // running position per expert
   __shared__ int wcnt[kSortThreads / 32][kSortMaxE / 4 + 1];  // per-warp counts, per round
   // wcnt holds up to kSortMaxE/4 experts per pass; larger E loops in passes below
@@ -129,7 +130,10 @@ sort_scatter_kernel(const int32_t* __restrict__ idx, int S, int E,
       if (mine) pos = wcnt[warp][e - e0] + rank;
       __syncthreads();
     }
-    if (e >= 0 && pos >= 0) sorted_slot[pos] = p;
+    if (e >= 0 && pos >= 0) {
+      sorted_slot[pos] = p;
+      if (inv) inv[p] = pos;
+    }
   }
 }
 
@@ -142,7 +146,7 @@ size_t sort_workspace_bytes(int T_, int k, int E) {
 }
 
 cudaError_t launch_sort(const int32_t* idx, int T_, int k, int E, int32_t* sorted_slot,
-                        int32_t* offsets, void* ws, unsigned* err, cudaStream_t s) {
+                        int32_t* offsets, void* ws, unsigned* err, cudaStream_t s, int32_t* inv) {
   const int S = T_ * k;
   const int nb = cdiv(S, kSortChunk);
   int32_t* counts = (int32_t*)ws;
@@ -152,7 +156,7 @@ cudaError_t launch_sort(const int32_t* idx, int T_, int k, int E, int32_t* sorte
   sort_scan_kernel<<<1, kSortThreads, 0, s>>>(counts, nb, E, offsets);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  sort_scatter_kernel<<<nb, kSortThreads, 0, s>>>(idx, S, E, counts, sorted_slot);
+  sort_scatter_kernel<<<nb, kSortThreads, 0, s>>>(idx, S, E, counts, sorted_slot, inv);
   return cudaGetLastError();
 }
 

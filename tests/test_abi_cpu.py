@@ -120,8 +120,8 @@ def test_workspace_queries_are_consistent():
 def test_workspaces_hold_no_copy_of_token_rows():
     """The library never allocates, so a grouped or padded copy of x or dY would have
     to live in its workspace.  Mixtral-shaped sizes: the forward workspace is exactly
-    the sort counts plus one fp32 [T*k, d] buffer (the k-way combine's slot rows);
-    what the backward needs beyond its documented large buffers (dH, gA and the fp32
+    the sort counts, one int32 per slot (its grouped row) and one fp32 [T*k, d]
+    buffer (the k-way combine's slot rows); what the backward needs beyond its documented large buffers (dH, gA and the fp32
     dx slot rows) is far smaller than one bf16 [T*k, d] copy."""
     import ctypes
     import sparse_mixture_experts_smoe_b200 as smoe
@@ -133,6 +133,6 @@ def test_workspaces_hold_no_copy_of_token_rows():
     desc = smoe.MlpDesc(T, d, f, E, k, smoe.ACT["swiglu"], smoe.BF16)
     fwd = L.smoe_mlp_workspace_size(ctypes.byref(desc), 0)
     bwd = L.smoe_mlp_workspace_size(ctypes.byref(desc), 1)
-    assert fwd == a256(sort) + a256(S * d * 4)
+    assert fwd == a256(sort) + a256(S * 4) + a256(S * d * 4)
     big = a256(S * 2 * f * 2) + a256(S * f * 2) + a256(S * d * 4)
     assert bwd - big < S * d * 2 // 4
