@@ -95,7 +95,8 @@ typedef enum {
   SMOE_OP_PL_FWD = 1,
   SMOE_OP_PL_BWD = 2,
   SMOE_OP_MLP_FWD = 3,
-  SMOE_OP_MLP_BWD = 4
+  SMOE_OP_MLP_BWD = 4,
+  SMOE_OP_ROUTE_BWD = 5
 } smoe_op;
 
 /* Upper bound of the workspace for `op` on an SMoE layer of T tokens, width d,
@@ -124,11 +125,14 @@ int smoe_route(const void* x, const void* w_r, const float* b_r, int T, int d, i
 /* smoe_route_bwd: gradient through the renormalised softmax of smoe_route.
  *   dl[t,j] = gates[t,j] (dgates[t,j] - sum_i gates[t,i] dgates[t,i]) for the
  *   selected expert e = topk_idx[t,j], 0 for unselected experts;
- *   dw_r[i,e] = sum_t x[t,i] dl[t,e]  (fp32, fixed-order reduction, overwritten)
+ *   dw_r[i,e] = sum_t x[t,i] dl[t,e]  (fp32, overwritten; summed in token order in
+ *                                      runs of 128 expert-sorted slots, the runs
+ *                                      then in order: fixed by T, k, E and routing)
  *   db_r[e]   = sum_t dl[t,e]         (fp32, overwritten; NULL to skip)
  *   dx[t,i]  += sum_j dl[t,j] W_r[i, topk_idx[t,j]]  (dtype, accumulated into dx;
  *                                                     NULL to skip)
- * workspace: smoe_workspace_size(SMOE_OP_MLP_BWD, ...) suffices.               */
+ * workspace: smoe_workspace_size(SMOE_OP_ROUTE_BWD, ...) bytes (no more than the
+ * SMOE_OP_MLP_BWD size of the same shape).                                    */
 int smoe_route_bwd(const void* x, const void* w_r, const int32_t* topk_idx, const float* gates,
                    const float* dgates, int T, int d, int E, int k, smoe_dtype dt, void* dx,
                    float* dw_r, float* db_r, void* workspace, size_t ws_bytes, void* stream);

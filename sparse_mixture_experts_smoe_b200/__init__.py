@@ -23,7 +23,7 @@ _lib = None
 SMOE_OK = 0
 F32, BF16 = 0, 1
 ACT = {"gelu": 0, "swiglu": 1, "none": 2}
-OP = {"sort": 0, "pl_fwd": 1, "pl_bwd": 2, "mlp_fwd": 3, "mlp_bwd": 4}
+OP = {"sort": 0, "pl_fwd": 1, "pl_bwd": 2, "mlp_fwd": 3, "mlp_bwd": 4, "route_bwd": 5}
 
 _c_int, _c_size, _vp = ctypes.c_int, ctypes.c_size_t, ctypes.c_void_p
 
@@ -189,7 +189,7 @@ def smoe_route_bwd(x, w_r, topk_idx, gates, dgates, dx=None, want_db=True, strea
         _need(t, n)
     dw_r = torch.empty((d, E), dtype=torch.float32, device=x.device)
     db_r = torch.empty((E,), dtype=torch.float32, device=x.device) if want_db else None
-    ws = _workspace(smoe_workspace_size("mlp_bwd", T, k, E, d, 8, x.dtype), x.device)
+    ws = _workspace(smoe_workspace_size("route_bwd", T, k, E, d, 8, x.dtype), x.device)
     _check(lib().smoe_route_bwd(_ptr(x), _ptr(w_r), _ptr(topk_idx), _ptr(gates), _ptr(dgates), T,
                                 d, E, k, _dt(x), _ptr(dx), _ptr(dw_r), _ptr(db_r), _ptr(ws),
                                 ws.numel(), _stream(stream)))

@@ -196,6 +196,30 @@ PLBwdWs pl_bwd_layout(void* ws, int num_slots, int K, int grouped_in, int fan_ou
 }
 
 // ---------------------------------------------------------------------------
+// Router backward workspace layout
+// ---------------------------------------------------------------------------
+struct RouteBwdWs {
+  float* dl = nullptr;           // [T, k]
+  void* sort = nullptr;          // the expert sort's scratch
+  int32_t* sorted_slot = nullptr;  // [T * k]
+  int32_t* offsets = nullptr;    // [E + 1]
+  float* part = nullptr;         // route_dw_runs * (d + 1)
+  size_t bytes = 0;
+};
+RouteBwdWs route_bwd_layout(void* ws, int T, int d, int E, int k) {
+  Carve c(ws);
+  RouteBwdWs l;
+  const size_t S = (size_t)T * k;
+  l.dl = (float*)c.take(S * sizeof(float));
+  l.sort = c.take(sort_workspace_bytes(T, k, E));
+  l.sorted_slot = (int32_t*)c.take(S * sizeof(int32_t));
+  l.offsets = (int32_t*)c.take((size_t)(E + 1) * sizeof(int32_t));
+  l.part = (float*)c.take((size_t)route_dw_runs((int)S, E) * (d + 1) * sizeof(float));
+  l.bytes = c.off;
+  return l;
+}
+
+// ---------------------------------------------------------------------------
 // SMoE MLP workspace layout
 // ---------------------------------------------------------------------------
 struct MlpWs {
@@ -210,7 +234,7 @@ struct MlpWs {
   float* dg = nullptr;      // bwd: [T, k] when the caller passes no dgates
   float* rpart = nullptr;   // bwd: router dW partials
   void* wrt = nullptr;      // bwd: router weight transposed [E, d] dtype
-  int dg_ld = 0, r_chunks = 0;
+  int dg_ld = 0, r_runs = 0;
   size_t bytes = 0;
 };
 MlpWs mlp_layout(void* ws, const smoe_mlp_desc& m, int backward) {
@@ -230,8 +254,8 @@ MlpWs mlp_layout(void* ws, const smoe_mlp_desc& m, int backward) {
     l.dxcomb = (float*)c.take(S * m.d * sizeof(float));
     l.dl = (float*)c.take(S * sizeof(float));
     l.dg = (float*)c.take(S * sizeof(float));
-    l.r_chunks = route_dw_chunks(m.T, m.d, m.E, m.k);
-    l.rpart = (float*)c.take(((size_t)l.r_chunks * m.E * m.d + (size_t)l.r_chunks * m.E) * sizeof(float));
+    l.r_runs = route_dw_runs((int)S, m.E);
+    l.rpart = (float*)c.take((size_t)l.r_runs * (m.d + 1) * sizeof(float));
     l.wrt = c.take((size_t)m.E * m.d * esize(dt));
   }
   l.bytes = c.off;
@@ -349,6 +373,7 @@ size_t smoe_workspace_size(int op, int T, int k, int E, int d, int f, smoe_dtype
     case SMOE_OP_SORT: return sort_workspace_bytes(T, k, E);
     case SMOE_OP_PL_FWD: return pl_fwd_layout(nullptr, S, wide, k).bytes;
     case SMOE_OP_PL_BWD: return pl_bwd_layout(nullptr, S, wide, 0, k, 1, 1, 1, 1, dt).bytes;
+    case SMOE_OP_ROUTE_BWD: return route_bwd_layout(nullptr, T, d, E, k).bytes;
     case SMOE_OP_MLP_FWD:
     case SMOE_OP_MLP_BWD: {
       smoe_mlp_desc m{T, d, f, E, k, SMOE_ACT_SWIGLU, dt};
@@ -388,22 +413,24 @@ int smoe_route_bwd(const void* x, const void* w_r, const int32_t* topk_idx, cons
   if (!valid_dtype(dt)) return fail(SMOE_ERR_INVALID_ARG, "bad dtype");
   NEED(x, "x"); NEED(w_r, "w_r"); NEED(topk_idx, "topk_idx"); NEED(gates, "gates");
   NEED(dgates, "dgates"); NEED(dw_r, "dw_r");
-  const int chunks = route_dw_chunks(T, d, E, k);
-  Carve c(workspace);
-  float* dl = (float*)c.take((size_t)T * k * sizeof(float));
-  float* part = (float*)c.take(((size_t)chunks * E * d + (size_t)chunks * E) * sizeof(float));
-  if (T > 0 && (!workspace || ws_bytes < c.off))
-    return fail(SMOE_ERR_INVALID_ARG, "workspace too small (%zu < %zu)", ws_bytes, c.off);
+  const RouteBwdWs l = route_bwd_layout(workspace, T, d, E, k);
+  if (T > 0 && (!workspace || ws_bytes < l.bytes))
+    return fail(SMOE_ERR_INVALID_ARG, "workspace too small (%zu < %zu)", ws_bytes, l.bytes);
   if (T == 0) {
     cudaStream_t s = (cudaStream_t)stream;
     SMOE_TRY(cudaMemsetAsync(dw_r, 0, (size_t)d * E * sizeof(float), s), "route_bwd zero");
     if (db_r) SMOE_TRY(cudaMemsetAsync(db_r, 0, (size_t)E * sizeof(float), s), "route_bwd zero");
     return SMOE_OK;
   }
+  cudaError_t st;
+  unsigned* err = error_word(&st);
+  if (!err) return cuda_fail(st, "smoe_route_bwd");
   cudaStream_t s = (cudaStream_t)stream;
-  { PROF("route_dl", 1); SMOE_TRY(launch_route_dl(gates, dgates, T, k, dl, s), "route_dl"); }
-  { PROF("route_dw", 2); SMOE_TRY(launch_route_dw(x, topk_idx, dl, T, d, E, k, dt, part, chunks, dw_r, db_r, s), "route_dw"); }
-  if (dx) { PROF("route_dx", 1); SMOE_TRY(launch_route_dx(dl, topk_idx, w_r, T, d, E, k, dt, dx, s), "route_dx"); }
+  { PROF("route_dl", 1); SMOE_TRY(launch_route_dl(gates, dgates, T, k, l.dl, s), "route_dl"); }
+  // the weight gradient walks the slots in grouped order
+  { PROF("sort", 3); SMOE_TRY(launch_sort(topk_idx, T, k, E, l.sorted_slot, l.offsets, l.sort, err, s), "route_bwd sort"); }
+  { PROF("route_dw", 2); SMOE_TRY(launch_route_dw(x, topk_idx, l.sorted_slot, l.offsets, l.dl, T, d, E, k, dt, l.part, dw_r, db_r, s), "route_dw"); }
+  if (dx) { PROF("route_dx", 1); SMOE_TRY(launch_route_dx(l.dl, topk_idx, w_r, T, d, E, k, dt, dx, s), "route_dx"); }
   return SMOE_OK;
 }
 
@@ -738,7 +765,8 @@ int smoe_mlp_bwd(const smoe_mlp_desc* desc, const smoe_mlp_tensors* t, void* str
   SMOE_TRY(launch_combine(l.dxcomb, l.inv, m.T, m.k, m.d, t->dx, dt, l.dl, t->topk_idx, l.wrt, m.E, s),
            "mlp bwd dx combine"); }
   { PROF("route_dw", 2);
-  SMOE_TRY(launch_route_dw(t->x, t->topk_idx, l.dl, m.T, m.d, m.E, m.k, dt, l.rpart, l.r_chunks,
+  SMOE_TRY(launch_route_dw(t->x, t->topk_idx, t->sorted_slot, t->expert_offsets, l.dl, m.T, m.d,
+                           m.E, m.k, dt, l.rpart,
                            t->dw_r, t->db_r, s), "mlp bwd router dW"); }
   return SMOE_OK;
 }

@@ -117,6 +117,19 @@ def test_workspace_queries_are_consistent():
             assert L.smoe_workspace_size(4, T, k, E, d, f, dt) == bwd
 
 
+@pytest.mark.parametrize("T,k,E,d", [(1, 1, 1, 8), (1, 1, 128, 8), (3, 2, 128, 8), (37, 3, 3, 40),
+                                     (256, 2, 8, 128), (16384, 8, 64, 2048), (16384, 2, 8, 4096)])
+def test_router_backward_fits_the_mlp_backward_workspace(T, k, E, d):
+    """smoe_route_bwd's header promises that the MLP backward's workspace size covers
+    it (its sort, slot order, dl and the weight gradient's run partials)."""
+    L = smoe.lib()
+    for dt in (0, 1):
+        rb = L.smoe_workspace_size(5, T, k, E, d, 8, dt)
+        assert 0 < rb <= L.smoe_workspace_size(4, T, k, E, d, 8, dt)
+        # run partials: (T*k / 128 + E) rows of d + 1 floats, nothing per (token, expert)
+        assert rb < T * k * 16 + ((T * k + 127) // 128 + E) * (d + 1) * 4 + 4096 + 256 * 8
+
+
 def test_workspaces_hold_no_copy_of_token_rows():
     """The library never allocates, so a grouped or padded copy of x or dY would have
     to live in its workspace.  Mixtral-shaped sizes: the forward workspace is exactly
