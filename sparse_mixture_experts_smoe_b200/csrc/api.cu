@@ -155,15 +155,15 @@ int check_tc(smoe_dtype dt) {
 // ParallelLinear workspace layout
 // ---------------------------------------------------------------------------
 struct PLFwdWs {
-  float* comb = nullptr;   // [num_slots, N] fp32 slot rows, grouped order
+  void* comb = nullptr;    // [num_slots, N] slot rows (dtype), grouped order
   int32_t* inv = nullptr;  // [num_slots] grouped row of each slot
   size_t bytes = 0;
 };
-PLFwdWs pl_fwd_layout(void* ws, int num_slots, int N, int combine_k) {
+PLFwdWs pl_fwd_layout(void* ws, int num_slots, int N, int combine_k, smoe_dtype dt) {
   Carve c(ws);
   PLFwdWs l;
   if (combine_k > 0) {
-    l.comb = (float*)c.take((size_t)num_slots * N * sizeof(float));
+    l.comb = c.take((size_t)num_slots * N * esize(dt));
     l.inv = (int32_t*)c.take((size_t)num_slots * sizeof(int32_t));
   }
   l.bytes = c.off;
@@ -171,7 +171,7 @@ PLFwdWs pl_fwd_layout(void* ws, int num_slots, int N, int combine_k) {
 }
 
 struct PLBwdWs {
-  float* dx_comb = nullptr;  // [num_slots, K] fp32 when dx needs a fan-out combine (grouped order)
+  void* dx_comb = nullptr;   // [num_slots, K] dtype when dx needs a fan-out combine (grouped order)
   int32_t* inv = nullptr;    // [num_slots] grouped row of each slot, with dx_comb
   float* dg_part = nullptr;  // [num_slots, dg_ld]
   void* gx = nullptr;        // [num_slots, K] dtype: gates * x rows, grouped
@@ -183,7 +183,7 @@ PLBwdWs pl_bwd_layout(void* ws, int num_slots, int K, int grouped_in, int fan_ou
   Carve c(ws);
   PLBwdWs l;
   if (want_dx && !grouped_in && fan_out > 1) {
-    l.dx_comb = (float*)c.take((size_t)num_slots * K * sizeof(float));
+    l.dx_comb = c.take((size_t)num_slots * K * esize(dt));
     l.inv = (int32_t*)c.take((size_t)num_slots * sizeof(int32_t));
   }
   if (has_gates && want_dg) {
@@ -224,11 +224,11 @@ RouteBwdWs route_bwd_layout(void* ws, int T, int d, int E, int k) {
 // ---------------------------------------------------------------------------
 struct MlpWs {
   void* sort = nullptr;
-  float* ycomb = nullptr;   // fwd: [S, d] fp32 slot rows, grouped order
+  void* ycomb = nullptr;    // fwd: [S, d] slot rows (dtype), grouped order
   float* dg_part = nullptr; // bwd: [S, dg_ld]
   void* dh = nullptr;       // bwd: [S, m*f] dtype (grouped dH)
   void* ga = nullptr;       // bwd: [S, f] dtype (gates * A)
-  float* dxcomb = nullptr;  // bwd: [S, d] fp32 slot rows, grouped order
+  void* dxcomb = nullptr;   // bwd: [S, d] slot rows (dtype), grouped order
   int32_t* inv = nullptr;   // fwd and bwd: [S] grouped row of each slot
   float* dl = nullptr;      // bwd: [T, k]
   float* dg = nullptr;      // bwd: [T, k] when the caller passes no dgates
@@ -245,13 +245,13 @@ MlpWs mlp_layout(void* ws, const smoe_mlp_desc& m, int backward) {
   l.sort = c.take(sort_workspace_bytes(m.T, m.k, m.E));
   l.inv = (int32_t*)c.take(S * sizeof(int32_t));
   if (!backward) {
-    l.ycomb = (float*)c.take(S * m.d * sizeof(float));
+    l.ycomb = c.take(S * m.d * esize(dt));
   } else {
     l.dg_ld = cdiv(m.f, act_tile_cols(dt));
     l.dg_part = (float*)c.take(S * l.dg_ld * sizeof(float));
     l.dh = c.take(S * (size_t)(m.act == SMOE_ACT_SWIGLU ? 2 * m.f : m.f) * esize(dt));
     l.ga = c.take(S * m.f * esize(dt));
-    l.dxcomb = (float*)c.take(S * m.d * sizeof(float));
+    l.dxcomb = c.take(S * m.d * esize(dt));
     l.dl = (float*)c.take(S * sizeof(float));
     l.dg = (float*)c.take(S * sizeof(float));
     l.r_runs = route_dw_runs((int)S, m.E);
@@ -371,7 +371,7 @@ size_t smoe_workspace_size(int op, int T, int k, int E, int d, int f, smoe_dtype
   const int wide = (d > 2 * f ? d : 2 * f);
   switch (op) {
     case SMOE_OP_SORT: return sort_workspace_bytes(T, k, E);
-    case SMOE_OP_PL_FWD: return pl_fwd_layout(nullptr, S, wide, k).bytes;
+    case SMOE_OP_PL_FWD: return pl_fwd_layout(nullptr, S, wide, k, dt).bytes;
     case SMOE_OP_PL_BWD: return pl_bwd_layout(nullptr, S, wide, 0, k, 1, 1, 1, 1, dt).bytes;
     case SMOE_OP_ROUTE_BWD: return route_bwd_layout(nullptr, T, d, E, k).bytes;
     case SMOE_OP_MLP_FWD:
@@ -482,9 +482,9 @@ static int validate_pl(const void* x, int x_rows, int K, const void* w, int N, i
 
 size_t parallel_linear_fwd_workspace_size(int num_slots, int K, int N, int E, int combine_k,
                                           smoe_dtype dt) {
-  (void)K; (void)E; (void)dt;
+  (void)K; (void)E;
   if (num_slots <= 0 || N <= 0) return 0;
-  return pl_fwd_layout(nullptr, num_slots, N, combine_k).bytes;
+  return pl_fwd_layout(nullptr, num_slots, N, combine_k, dt).bytes;
 }
 
 int parallel_linear_fwd(const void* x, int x_rows, int K, const void* w, int N, int E,
@@ -498,7 +498,7 @@ int parallel_linear_fwd(const void* x, int x_rows, int K, const void* w, int N, 
   if (rc != SMOE_OK) return rc;
   if (num_slots == 0) return SMOE_OK;
   NEED(y, "y"); ALIGNED(y, "y");
-  PLFwdWs l = pl_fwd_layout(workspace, num_slots, N, combine_k);
+  PLFwdWs l = pl_fwd_layout(workspace, num_slots, N, combine_k, dt);
   if (l.bytes > 0 && (!workspace || ws_bytes < l.bytes))
     return fail(SMOE_ERR_INVALID_ARG, "workspace too small (%zu < %zu)", ws_bytes, l.bytes);
   if ((rc = check_tc(dt)) != SMOE_OK) return rc;
@@ -513,7 +513,7 @@ int parallel_linear_fwd(const void* x, int x_rows, int K, const void* w, int N, 
   g.b = w; g.b_kn = 1; g.NW = N; g.n_out = N;
   g.epi = EPI_STORE; g.gates = gates; g.err = err;
   if (combine_k > 0) {
-    g.out_mode = ROWS_GROUPED; g.out = l.comb; g.ldo = N; g.out_f32 = 1;
+    g.out_mode = ROWS_GROUPED; g.out = l.comb; g.ldo = N; g.out_f32 = dt == SMOE_F32;
   } else {
     g.out_mode = grouped_out ? ROWS_GROUPED : ROWS_GATHER; g.out = y; g.ldo = N;
     g.out_f32 = dt == SMOE_F32;
@@ -580,7 +580,7 @@ int parallel_linear_bwd(const void* dy, const void* x, const void* w, int x_rows
     g.b = w; g.b_kn = 0; g.NW = K; g.n_out = K;
     g.gates = gates; g.err = err;
     g.out_mode = grouped_in ? ROWS_GROUPED : ROWS_GATHER;
-    if (dx_comb) { g.out_mode = ROWS_GROUPED; g.out = l.dx_comb; g.ldo = K; g.out_f32 = 1; }
+    if (dx_comb) { g.out_mode = ROWS_GROUPED; g.out = l.dx_comb; g.ldo = K; g.out_f32 = dt == SMOE_F32; }
     else { g.out = dx; g.ldo = K; g.out_f32 = dt == SMOE_F32; }
     if (has_g) {
       g.epi = EPI_ACT_BWD; g.act = SMOE_ACT_NONE;
@@ -676,7 +676,7 @@ int smoe_mlp_fwd(const smoe_mlp_desc* desc, const smoe_mlp_tensors* t, void* str
     g.K = m.f; g.a = t->a; g.lda = m.f; g.a_rows = S; g.a_mode = ROWS_GROUPED;
     g.b = t->w2; g.b_kn = 1; g.NW = m.d; g.n_out = m.d;
     g.epi = EPI_STORE; g.gates = t->gates;
-    g.out_mode = ROWS_GROUPED; g.out = l.ycomb; g.ldo = m.d; g.out_f32 = 1; g.err = err;
+    g.out_mode = ROWS_GROUPED; g.out = l.ycomb; g.ldo = m.d; g.out_f32 = dt == SMOE_F32; g.err = err;
     { PROF("gemm.fwd_down", 1); SMOE_TRY(run_grouped(g, dt, s), "mlp fwd gemm2"); }
   }
   { PROF("combine.y", 1); SMOE_TRY(launch_combine(l.ycomb, l.inv, m.T, m.k, m.d, t->y, dt, nullptr, nullptr, nullptr, 0, s), "mlp fwd combine"); }
@@ -755,7 +755,7 @@ int smoe_mlp_bwd(const smoe_mlp_desc* desc, const smoe_mlp_tensors* t, void* str
     g.K = mf; g.a = l.dh; g.lda = mf; g.a_rows = S; g.a_mode = ROWS_GROUPED;
     g.b = t->w1; g.b_kn = 0; g.NW = m.d; g.n_out = m.d;
     g.epi = EPI_STORE;
-    g.out_mode = ROWS_GROUPED; g.out = l.dxcomb; g.ldo = m.d; g.out_f32 = 1; g.err = err;
+    g.out_mode = ROWS_GROUPED; g.out = l.dxcomb; g.ldo = m.d; g.out_f32 = dt == SMOE_F32; g.err = err;
     { PROF("gemm.bwd_dx", 1); SMOE_TRY(run_grouped(g, dt, s), "mlp bwd gemm dx"); }
   }
   // dx[t] = sum_j rows + router term sum_j dl W_r[:, e_j]

@@ -6,12 +6,14 @@
 //
 // The k slots of a token are owned by k different experts, so their products
 // come from different CTAs; summing them with atomics would make the result
-// depend on scheduling.  Instead the GEMM epilogue stores each slot's row in an
-// fp32 buffer, in grouped order (row i of slot p = sorted_slot[i], so that whole
-// warps of rows leave as TMA boxes), and this pass sums the k rows of each token
-// in ascending j, finding slot p's row through the inverse permutation
-// inv[p] = i (group-to-scatter with combine, library page of arXiv 2403.08245,
-// review 2 summary).
+// depend on scheduling.  Instead the GEMM epilogue stores each slot's row, already
+// multiplied by its gate, in a buffer of the layer's dtype (the slot outputs are
+// materialised in the compute type before the gate-weighted sum, as the library
+// does it), in grouped order (row i of slot p = sorted_slot[i], so that whole warps
+// of rows leave as TMA boxes); this pass sums the k rows of each token in fp32 in
+// ascending j, finding slot p's row through the inverse permutation inv[p] = i
+// (group-to-scatter with combine, library page of arXiv 2403.08245, review 2
+// summary).
 #include "common.cuh"
 
 namespace smoe {
@@ -42,11 +44,11 @@ __device__ __forceinline__ void store4(bf16* p, float4 v) {
   *reinterpret_cast<uint2*>(p) = r;
 }
 
-template <typename TO, typename TW>
+template <typename T>
 __global__ void __launch_bounds__(256)
-combine_kernel(const float* __restrict__ ws, const int32_t* __restrict__ inv, int T_, int ck,
-               int N, TO* __restrict__ out, const float* __restrict__ dl,
-               const int32_t* __restrict__ idx, const TW* __restrict__ w_rt, int E) {
+combine_kernel(const T* __restrict__ ws, const int32_t* __restrict__ inv, int T_, int ck,
+               int N, T* __restrict__ out, const float* __restrict__ dl,
+               const int32_t* __restrict__ idx, const T* __restrict__ w_rt, int E) {
   const int n4 = N / 4;
   const int U = (n4 + kCombV - 1) / kCombV;
   const size_t q = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
@@ -62,12 +64,12 @@ combine_kernel(const float* __restrict__ ws, const int32_t* __restrict__ inv, in
     const int p = t * ck + j;
     const int row = inv ? __ldg(inv + p) : p;
     if (row < 0 || row >= S) continue;  // not a permutation: a data error flagged upstream
-    const float4* src = reinterpret_cast<const float4*>(ws + (size_t)row * N);
+    const T* src = ws + (size_t)row * N;
     float4 x[kCombV];
 #pragma unroll
     for (int v = 0; v < kCombV; ++v) {
       const int c4 = u + v * U;
-      x[v] = c4 < n4 ? __ldg(src + c4) : make_float4(0.f, 0.f, 0.f, 0.f);
+      x[v] = c4 < n4 ? load4(src + 4 * c4) : make_float4(0.f, 0.f, 0.f, 0.f);
     }
 #pragma unroll
     for (int v = 0; v < kCombV; ++v) {
@@ -155,17 +157,17 @@ cudaError_t launch_transpose_wr(const void* w_r, int d, int E, smoe_dtype dt, vo
   return cudaGetLastError();
 }
 
-cudaError_t launch_combine(const float* ws, const int32_t* inv, int T_, int ck, int N, void* out,
-                           smoe_dtype out_dt, const float* dl, const int32_t* idx,
-                           const void* w_rt, int E, cudaStream_t s) {
+cudaError_t launch_combine(const void* ws, const int32_t* inv, int T_, int ck, int N, void* out,
+                           smoe_dtype dt, const float* dl, const int32_t* idx, const void* w_rt,
+                           int E, cudaStream_t s) {
   const size_t n = (size_t)T_ * cdiv(N / 4, kCombV);
   const unsigned blocks = (unsigned)((n + 255) / 256);
-  if (out_dt == SMOE_BF16)
-    combine_kernel<bf16, bf16><<<blocks, 256, 0, s>>>(ws, inv, T_, ck, N, (bf16*)out, dl, idx,
-                                                      (const bf16*)w_rt, E);
+  if (dt == SMOE_BF16)
+    combine_kernel<bf16><<<blocks, 256, 0, s>>>((const bf16*)ws, inv, T_, ck, N, (bf16*)out, dl,
+                                                idx, (const bf16*)w_rt, E);
   else
-    combine_kernel<float, float><<<blocks, 256, 0, s>>>(ws, inv, T_, ck, N, (float*)out, dl, idx,
-                                                        (const float*)w_rt, E);
+    combine_kernel<float><<<blocks, 256, 0, s>>>((const float*)ws, inv, T_, ck, N, (float*)out, dl,
+                                                 idx, (const float*)w_rt, E);
   return cudaGetLastError();
 }
 

@@ -96,11 +96,11 @@ cudaError_t launch_sort(const int32_t* idx, int T, int k, int E, int32_t* sorted
                         int32_t* inv = nullptr);
 
 // out[t] = sum_{j<ck} ws[row(t*ck + j)] (+ sum_j dl[t*ck+j] * w_rt[idx[t*ck+j], :] if dl),
-// w_rt being the router weight transposed to [E, N]; row(p) = inv[p] (the slot's
-// grouped row) or p when inv is null
-cudaError_t launch_combine(const float* ws, const int32_t* inv, int T, int ck, int N, void* out,
-                           smoe_dtype out_dt, const float* dl, const int32_t* idx,
-                           const void* w_rt, int E, cudaStream_t s);
+// summed in fp32; ws, out and w_rt (the router weight transposed to [E, N]) in dtype
+// dt; row(p) = inv[p] (the slot's grouped row) or p when inv is null
+cudaError_t launch_combine(const void* ws, const int32_t* inv, int T, int ck, int N, void* out,
+                           smoe_dtype dt, const float* dl, const int32_t* idx, const void* w_rt,
+                           int E, cudaStream_t s);
 // inv[sorted_slot[i]] = i for i < num_rows
 cudaError_t launch_invert(const int32_t* sorted_slot, int num_rows, int32_t* inv, cudaStream_t s);
 // w_rt[e][i] = w_r[i][e]

@@ -109,9 +109,10 @@ def test_workspace_queries_are_consistent():
             desc = smoe.MlpDesc(T, d, f, E, k, 1, dt)
             fwd = L.smoe_mlp_workspace_size(ctypes.byref(desc), 0)
             bwd = L.smoe_mlp_workspace_size(ctypes.byref(desc), 1)
-            # forward: sort counts + one fp32 [T*k, d] combine buffer, nothing the size of a
-            # grouped copy of x in its own dtype is needed beyond that
-            assert fwd >= T * k * d * 4 and fwd < T * k * d * 4 + (1 << 20)
+            # forward: sort counts + one [T*k, d] combine buffer of the layer's dtype,
+            # nothing the size of a grouped copy of x is needed beyond that
+            es = 4 if dt == 0 else 2
+            assert fwd >= T * k * d * es and fwd < T * k * d * es + (1 << 20)
             assert bwd > fwd
             assert L.smoe_workspace_size(3, T, k, E, d, f, dt) == fwd
             assert L.smoe_workspace_size(4, T, k, E, d, f, dt) == bwd
@@ -133,9 +134,10 @@ def test_router_backward_fits_the_mlp_backward_workspace(T, k, E, d):
 def test_workspaces_hold_no_copy_of_token_rows():
     """The library never allocates, so a grouped or padded copy of x or dY would have
     to live in its workspace.  Mixtral-shaped sizes: the forward workspace is exactly
-    the sort counts, one int32 per slot (its grouped row) and one fp32 [T*k, d]
-    buffer (the k-way combine's slot rows); what the backward needs beyond its documented large buffers (dH, gA and the fp32
-    dx slot rows) is far smaller than one bf16 [T*k, d] copy."""
+    the sort counts, one int32 per slot (its grouped row) and one bf16 [T*k, d]
+    buffer (the k-way combine's gated slot rows); what the backward needs beyond its
+    documented large buffers (dH, gA and the dx slot rows) is far smaller than
+    another bf16 [T*k, d] copy."""
     import ctypes
     import sparse_mixture_experts_smoe_b200 as smoe
     T, d, f, E, k = 16384, 4096, 14336, 8, 2
@@ -146,6 +148,6 @@ def test_workspaces_hold_no_copy_of_token_rows():
     desc = smoe.MlpDesc(T, d, f, E, k, smoe.ACT["swiglu"], smoe.BF16)
     fwd = L.smoe_mlp_workspace_size(ctypes.byref(desc), 0)
     bwd = L.smoe_mlp_workspace_size(ctypes.byref(desc), 1)
-    assert fwd == a256(sort) + a256(S * 4) + a256(S * d * 4)
-    big = a256(S * 2 * f * 2) + a256(S * f * 2) + a256(S * d * 4)
+    assert fwd == a256(sort) + a256(S * 4) + a256(S * d * 2)
+    big = a256(S * 2 * f * 2) + a256(S * f * 2) + a256(S * d * 2)
     assert bwd - big < S * d * 2 // 4
