@@ -410,14 +410,10 @@ struct DwExtra {
 //          one 128-byte fp32 one) written out by per-row bulk copies; the stride
 //          of 13 x 16 bytes keeps 8 consecutive threads' 16-byte accesses on
 //          distinct banks.
-// EPI_STORE with fp32 output instead writes one 4 KB box of 32 rows x 128 bytes
-// in the 128-byte swizzle at the area's first 1024-byte boundary (offset 0 or
-// 512), stored by one TMA tensor store when boxed, else row by row from it.
 constexpr int kSlotBytes = 208;
 constexpr int kBoxBytes = 32 * 64;
 constexpr int kWarpStaging = 32 * kSlotBytes;  // 13 x 512: boxes stay 512-byte aligned
 static_assert(3 * kBoxBytes <= kWarpStaging && kWarpStaging % 512 == 0, "staging layout");
-static_assert(512 + 32 * 128 <= kWarpStaging, "fp32 box fits after alignment");
 constexpr int kStagingBytes = 4 * kWarpStaging;
 enum : int { kBoxStores = 1, kBoxLoads = 2 };  // grouped-epilogue box modes (launch flags)
 // Grouped-M GEMMs run as CTA pairs sharing M = 256 MMAs (cta_group::2).
@@ -747,7 +743,9 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
       }
     }
     __syncwarp();
-  } else if (warp >= 4 && warp < 8) {  // warps 2-3 (and 8-15 without a gather) idle
+  } else if ((warp >= 4 && warp < 8) ||
+             (!A_GATHER && !SWIGLU_FWD && g.epi == EPI_STORE && warp >= 8 && warp < 12)) {
+    // warps 2-3 idle, and 8-15 without a gather except as below
     // ---------------- epilogue ----------------
     // Thread r owns accumulator row r.  Per 32-column chunk the warp stages its
     // rows' output segments in shared memory and hands them to the TMA engine:
@@ -759,15 +757,18 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
     // warp's rows (kBoxLoads), when they are in grouped order, else by 16-byte
     // loads issued before the accumulator read (per-row bulk loads of 64 bytes
     // measured far slower).
-    const int q = warp - 4;  // tensor-memory lane quadrant
+    // Without a gather, EPI_STORE runs two epilogue groups, warps 4-7 on the tiles
+    // of accumulator buffer 0 and warps 8-11 on those of buffer 1, so that two
+    // tiles drain at once (a short-K product's epilogue is longer than its MMAs).
+    // A group stages in box `grp` of its quadrant's area; a warp whose rows leave
+    // the slice stores them directly.
+    const bool two = !A_GATHER && !SWIGLU_FWD && g.epi == EPI_STORE;
+    const int grp = warp >= 8 ? 1 : 0;
+    const int q = warp & 3;  // tensor-memory lane quadrant
     const int r = q * 32 + lane;
     uint8_t* wstage = smem + kRingBytes + kCtlBytes + q * kWarpStaging;
     uint8_t* slot = wstage + lane * kSlotBytes;
     const uint32_t wstage_s = smem_u32(wstage), slot_s = smem_u32(slot);
-    // the fp32 output box (32 rows x 128 bytes, 128-byte swizzle) starts on the
-    // first 1024-byte boundary of the warp's staging area
-    const uint32_t fbox_s = (wstage_s + 1023u) & ~1023u;
-    uint8_t* fbox = wstage + (fbox_s - wstage_s);
     const int sw = (lane >> 1) & 3;  // 64-byte swizzle of this thread's box row
     const bf16* AUXA = reinterpret_cast<const bf16*>(g.aux_a);
     const bf16* AUXH = reinterpret_cast<const bf16*>(g.aux_h);
@@ -780,6 +781,7 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
     int it = 0;
     for (int L = first; L < total; L += stride, ++it) {
       const int buf = it & 1;
+      if (two && buf != grp) continue;  // the other group's tile
       const uint32_t tph = (it >> 1) & 1;
       const Tile t = map_tile<PAIR>(c, g.offsets, g.E, nN, L, rank);
       if (!mbar_wait(&c.tfull[buf], tph, abort_flag, g.err)) break;
@@ -794,13 +796,15 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
       const uint32_t trow = c.tmem_base + ((uint32_t)(q * 32) << 16) + buf * BN;
       const int wrow0 = t.row0 + q * 32;
       const bool boxed = (box_flags & kBoxStores) && wrow0 + 32 <= t.row_end;  // warp-uniform
+      const bool direct = two && !boxed;  // warp-uniform: plain stores from registers
+      const int kb = two ? grp : 0;       // first box of this warp's outputs
       // 16-byte chunk j8 of box k in this thread's row
       auto box_chunk = [&](int k, int j8) -> uint4* {
         return reinterpret_cast<uint4*>(wstage + k * kBoxBytes + lane * 64 + ((j8 ^ sw) << 4));
       };
       // 16-byte chunk j8 of output segment k of this thread's row
       auto chunk = [&](int k, int j8) -> uint4* {
-        return reinterpret_cast<uint4*>(boxed ? wstage + k * kBoxBytes + lane * 64 + ((j8 ^ sw) << 4)
+        return reinterpret_cast<uint4*>(boxed ? wstage + (k + kb) * kBoxBytes + lane * 64 + ((j8 ^ sw) << 4)
                                               : slot + k * 64 + 16 * j8);
       };
       float dg_acc = 0.0f;
@@ -891,26 +895,16 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
 #pragma unroll
                   for (int j = 0; j < 8; ++j) dh[j] = gate * vv[j];
                 }
-                if (g.out_f32) {  // never boxed
-                  float4* dst = reinterpret_cast<float4*>(slot + 64 + 32 * j8);
-                  dst[0] = make_float4(dh[0], dh[1], dh[2], dh[3]);
-                  dst[1] = make_float4(dh[4], dh[5], dh[6], dh[7]);
-                } else {
-                  *chunk(1, j8) = pack8(dh);
-                }
+                *chunk(1, j8) = pack8(dh);
               }
             } else if (epi_store) {  // [g acc]
               float o[8];
 #pragma unroll
               for (int j = 0; j < 8; ++j) o[j] = gate * vv[j];
-              if (g.out_f32) {  // a 32 x 32 fp32 box in the 128-byte swizzle, row = lane
-                float4* d0 = reinterpret_cast<float4*>(fbox + lane * 128 + (((2 * j8) ^ (lane & 7)) << 4));
-                float4* d1 = reinterpret_cast<float4*>(fbox + lane * 128 + (((2 * j8 + 1) ^ (lane & 7)) << 4));
-                *d0 = make_float4(o[0], o[1], o[2], o[3]);
-                *d1 = make_float4(o[4], o[5], o[6], o[7]);
-              } else {
+              if (direct)
+                *reinterpret_cast<uint4*>(reinterpret_cast<bf16*>(g.out) + (size_t)orow * g.ldo + n0 + 8 * j8) = pack8(o);
+              else
                 *chunk(0, j8) = pack8(o);
-              }
             } else {  // EPI_ACT_FWD: [H (gate) | H up | A] or [H | A]
               float a8[8];
               if (SWIGLU_FWD) {
@@ -940,7 +934,7 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
                 if (swi) tma_store_3d(&tmO, wstage_s + 2 * kBoxBytes, n0, 1, wrow0);
               }
             } else if (epi_store) {
-              tma_store_3d(&tmO, g.out_f32 ? fbox_s : wstage_s, n0, 0, wrow0);
+              tma_store_3d(&tmO, wstage_s + kb * kBoxBytes, n0, 0, wrow0);
             } else {
               tma_store_3d(&tmO, wstage_s, n0, 0, wrow0);
               if (SWIGLU_FWD) {
@@ -952,7 +946,7 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
             }
             bulk_commit();
           }
-        } else if (p_ok) {
+        } else if (p_ok && !direct) {
           if (act_bwd) {
             if (g.out2) bulk_s2g(reinterpret_cast<bf16*>(g.out2) + (size_t)i * g.ldo2 + n0, slot_s, seg);
             if (g.out) {
@@ -960,14 +954,12 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
                 bf16* O = reinterpret_cast<bf16*>(g.out) + (size_t)orow * g.ldo;
                 bulk_s2g(O + n0, slot_s + 64, seg);
                 bulk_s2g(O + g.n_out + n0, slot_s + 128, seg);
-              } else if (g.out_f32) {
-                bulk_s2g(reinterpret_cast<float*>(g.out) + (size_t)orow * g.ldo + n0, slot_s + 64, 2 * seg);
               } else {
                 bulk_s2g(reinterpret_cast<bf16*>(g.out) + (size_t)orow * g.ldo + n0, slot_s + 64, seg);
               }
             }
           } else if (epi_store) {
-            if (!g.out_f32) bulk_s2g(reinterpret_cast<bf16*>(g.out) + (size_t)orow * g.ldo + n0, slot_s, seg);
+            bulk_s2g(reinterpret_cast<bf16*>(g.out) + (size_t)orow * g.ldo + n0, slot_s, seg);
           } else {
             bf16* H = reinterpret_cast<bf16*>(g.out) + (size_t)orow * g.ldo;
             bf16* A2 = reinterpret_cast<bf16*>(g.out2) + (size_t)orow * g.ldo2;
@@ -980,22 +972,6 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
             }
           }
           bulk_commit();
-        }
-        if (epi_store && g.out_f32 && !boxed) {
-          // fp32 rows of a warp that is not wholly inside the slice, or in token
-          // order: from the box, 8 lanes per 128-byte row segment, 4 rows per warp
-          // store; per-row bulk copies of 128 bytes would be one TMA operation per
-          // row per chunk
-#pragma unroll
-          for (int it2 = 0; it2 < 8; ++it2) {
-            const int rr = it2 * 4 + (lane >> 3), c4 = lane & 7;
-            const int orow_r = __shfl_sync(0xffffffffu, orow, rr);
-            const int ok_r = __shfl_sync(0xffffffffu, p_ok ? 1 : 0, rr);
-            if (ok_r && 4 * c4 < ncols) {
-              const float4 val = *reinterpret_cast<const float4*>(fbox + rr * 128 + ((c4 ^ (rr & 7)) << 4));
-              *reinterpret_cast<float4*>(reinterpret_cast<float*>(g.out) + (size_t)orow_r * g.ldo + n0 + 4 * c4) = val;
-            }
-          }
         }
       }
       if (act_bwd && p_ok && g.dg_partial)
@@ -1425,16 +1401,6 @@ cudaError_t out_map(CUtensorMap* m, const void* base, int n_out, int parts, int 
   return make_map(m, base, 3, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_64B);
 }
 
-// fp32 variant for EPI_STORE: dims {n_out, 1, rows}, box 32 x 32 in the 128-byte
-// swizzle (the layout the epilogue writes its fp32 box in).
-cudaError_t out_map_f32(CUtensorMap* m, const void* base, int n_out, int rows, int ld) {
-  const uint64_t dims[3] = {(uint64_t)n_out, 1, (uint64_t)rows};
-  const uint64_t strides[2] = {(uint64_t)n_out * 4, (uint64_t)ld * 4};
-  const uint32_t box[3] = {32, 1, 32};
-  return make_map(m, base, 3, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B,
-                  CU_TENSOR_MAP_DATA_TYPE_FLOAT32);
-}
-
 int num_sms() {
   static int n = 0;
   if (n == 0) {
@@ -1523,6 +1489,7 @@ int tc_tile_cols() { return BN; }
 cudaError_t launch_grouped_gemm_tc(const GroupedGemm& g, cudaStream_t s) {
   if (g.num_rows == 0) return cudaSuccess;
   if (g.E > kMaxE) return cudaErrorInvalidValue;
+  if (g.out_f32) return cudaErrorInvalidValue;  // every output of this path is bf16
   const bool swiglu = g.epi == EPI_ACT_FWD && g.act == SMOE_ACT_SWIGLU;
   const int BNo = swiglu ? BN / 2 : BN;
   const int nN = cdiv(g.n_out, BNo);
@@ -1543,19 +1510,13 @@ cudaError_t launch_grouped_gemm_tc(const GroupedGemm& g, cudaStream_t s) {
     e = make_map(&tb, g.b, 3, dims, str, box);
   }
   if (e != cudaSuccess) return e;
-  // Boxed (TMA tensor) epilogue stores when every output is in grouped rows and
-  // bf16, or fp32 from EPI_STORE; boxed ACT_BWD input loads when its inputs are
-  // in grouped rows.
+  // Boxed (TMA tensor) epilogue stores when every output is in grouped rows;
+  // boxed ACT_BWD input loads when its inputs are in grouped rows.
   EpiMaps m;
   const int parts = (g.act == SMOE_ACT_SWIGLU && g.epi != EPI_STORE) ? 2 : 1;
   bool st = (g.out != nullptr || g.out2 != nullptr) &&
-            (g.out == nullptr ||
-             (g.out_mode == ROWS_GROUPED && (!g.out_f32 || g.epi == EPI_STORE)));
-  if (st && g.out) {
-    const cudaError_t me = g.out_f32 ? out_map_f32(&m.out, g.out, g.n_out, g.num_rows, g.ldo)
-                                     : out_map(&m.out, g.out, g.n_out, parts, g.num_rows, g.ldo);
-    if (me != cudaSuccess) st = false;
-  }
+            (g.out == nullptr || g.out_mode == ROWS_GROUPED);
+  if (st && g.out && out_map(&m.out, g.out, g.n_out, parts, g.num_rows, g.ldo) != cudaSuccess) st = false;
   if (st && g.out2 && out_map(&m.out2, g.out2, g.n_out, 1, g.num_rows, g.ldo2) != cudaSuccess) st = false;
   const bool need_h = g.out != nullptr && g.act != SMOE_ACT_NONE;
   bool ld = g.epi == EPI_ACT_BWD && g.aux_a_mode == ROWS_GROUPED && !swiglu;
