@@ -19,62 +19,89 @@
 namespace smoe {
 namespace {
 
-// Each thread owns kCombV float4 columns of one token, u + v*U for v < kCombV
-// (U threads per token, so every v is a coalesced sweep of the row).  The slot
-// rows sit at grouped positions, so their indices come first; the thread then has
-// kCombV independent 16-byte loads in flight per slot instead of one load behind
-// a dependent index load.  The router term reads the transposed router weight
-// w_rt [E, N] so each selected expert contributes contiguous loads.
+// Each thread owns kCombV 16-byte vectors of one token's row (VE = 8 bf16 or 4 fp32
+// elements each), vector u + v*U for v < kCombV (U threads per token, so every v is
+// a coalesced sweep of the row).  The slot rows sit at grouped positions, so their
+// index comes first; the thread then has kCombV independent 16-byte loads in flight
+// per slot instead of one load behind a dependent index load.  The router term
+// reads the transposed router weight w_rt [E, N] so each selected expert
+// contributes contiguous loads.
 constexpr int kCombV = 4;
 
-// four consecutive elements as one 8- or 16-byte access
-__device__ __forceinline__ float4 load4(const float* p) { return __ldg(reinterpret_cast<const float4*>(p)); }
-__device__ __forceinline__ float4 load4(const bf16* p) {
-  const uint2 r = __ldg(reinterpret_cast<const uint2*>(p));
-  const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&r.x));
-  const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&r.y));
-  return make_float4(a.x, a.y, b.x, b.y);
-}
-__device__ __forceinline__ void store4(float* p, float4 v) { *reinterpret_cast<float4*>(p) = v; }
-__device__ __forceinline__ void store4(bf16* p, float4 v) {
-  __nv_bfloat162 a = __floats2bfloat162_rn(v.x, v.y), b = __floats2bfloat162_rn(v.z, v.w);
-  uint2 r;
-  r.x = *reinterpret_cast<uint32_t*>(&a);
-  r.y = *reinterpret_cast<uint32_t*>(&b);
-  *reinterpret_cast<uint2*>(p) = r;
-}
+template <typename T>
+struct Vec16 {
+  static constexpr int VE = 16 / (int)sizeof(T);
+  float f[VE];
+  __device__ __forceinline__ void zero() {
+#pragma unroll
+    for (int i = 0; i < VE; ++i) f[i] = 0.f;
+  }
+  __device__ __forceinline__ void load(const T* p) {
+    const uint4 u = __ldg(reinterpret_cast<const uint4*>(p));
+    if constexpr (sizeof(T) == 2) {
+      const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float2 a = __bfloat1622float2(h[i]);
+        f[2 * i] = a.x;
+        f[2 * i + 1] = a.y;
+      }
+    } else {
+      f[0] = __uint_as_float(u.x); f[1] = __uint_as_float(u.y);
+      f[2] = __uint_as_float(u.z); f[3] = __uint_as_float(u.w);
+    }
+  }
+  __device__ __forceinline__ void store(T* p) const {
+    uint4 u;
+    if constexpr (sizeof(T) == 2) {
+      uint32_t* w = reinterpret_cast<uint32_t*>(&u);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        __nv_bfloat162 h = __floats2bfloat162_rn(f[2 * i], f[2 * i + 1]);
+        w[i] = *reinterpret_cast<uint32_t*>(&h);
+      }
+    } else {
+      u = make_uint4(__float_as_uint(f[0]), __float_as_uint(f[1]), __float_as_uint(f[2]),
+                     __float_as_uint(f[3]));
+    }
+    *reinterpret_cast<uint4*>(p) = u;
+  }
+};
 
 template <typename T>
 __global__ void __launch_bounds__(256)
 combine_kernel(const T* __restrict__ ws, const int32_t* __restrict__ inv, int T_, int ck,
                int N, T* __restrict__ out, const float* __restrict__ dl,
                const int32_t* __restrict__ idx, const T* __restrict__ w_rt, int E) {
-  const int n4 = N / 4;
-  const int U = (n4 + kCombV - 1) / kCombV;
+  using V = Vec16<T>;
+  constexpr int VE = V::VE;
+  const int nv = N / VE;  // N % 8 == 0
+  const int U = (nv + kCombV - 1) / kCombV;
   const size_t q = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (q >= (size_t)T_ * U) return;
   const int t = (int)(q / U);
   const int u = (int)(q % U);
   const int S = T_ * ck;
-  float4 acc[kCombV];
+  V acc[kCombV];
 #pragma unroll
-  for (int v = 0; v < kCombV; ++v) acc[v] = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int v = 0; v < kCombV; ++v) acc[v].zero();
 #pragma unroll 2
   for (int j = 0; j < ck; ++j) {
     const int p = t * ck + j;
     const int row = inv ? __ldg(inv + p) : p;
     if (row < 0 || row >= S) continue;  // not a permutation: a data error flagged upstream
     const T* src = ws + (size_t)row * N;
-    float4 x[kCombV];
+    V x[kCombV];
 #pragma unroll
     for (int v = 0; v < kCombV; ++v) {
-      const int c4 = u + v * U;
-      x[v] = c4 < n4 ? load4(src + 4 * c4) : make_float4(0.f, 0.f, 0.f, 0.f);
+      const int cv = u + v * U;
+      if (cv < nv) x[v].load(src + VE * cv);
+      else x[v].zero();
     }
 #pragma unroll
-    for (int v = 0; v < kCombV; ++v) {
-      acc[v].x += x[v].x; acc[v].y += x[v].y; acc[v].z += x[v].z; acc[v].w += x[v].w;
-    }
+    for (int v = 0; v < kCombV; ++v)
+#pragma unroll
+      for (int i = 0; i < VE; ++i) acc[v].f[i] += x[v].f[i];
   }
   if (dl != nullptr) {
     for (int j = 0; j < ck; ++j) {
@@ -83,21 +110,19 @@ combine_kernel(const T* __restrict__ ws, const int32_t* __restrict__ inv, int T_
       const float g = dl[(size_t)t * ck + j];
 #pragma unroll
       for (int v = 0; v < kCombV; ++v) {
-        const int c4 = u + v * U;
-        if (c4 >= n4) continue;
-        const float4 w = load4(w_rt + (size_t)e * N + 4 * c4);
-        acc[v].x = fmaf(g, w.x, acc[v].x);
-        acc[v].y = fmaf(g, w.y, acc[v].y);
-        acc[v].z = fmaf(g, w.z, acc[v].z);
-        acc[v].w = fmaf(g, w.w, acc[v].w);
+        const int cv = u + v * U;
+        if (cv >= nv) continue;
+        V w;
+        w.load(w_rt + (size_t)e * N + VE * cv);
+#pragma unroll
+        for (int i = 0; i < VE; ++i) acc[v].f[i] = fmaf(g, w.f[i], acc[v].f[i]);
       }
     }
   }
 #pragma unroll
   for (int v = 0; v < kCombV; ++v) {
-    const int c4 = u + v * U;
-    if (c4 >= n4) continue;
-    store4(out + (size_t)t * N + 4 * c4, acc[v]);
+    const int cv = u + v * U;
+    if (cv < nv) acc[v].store(out + (size_t)t * N + VE * cv);
   }
 }
 
@@ -160,7 +185,8 @@ cudaError_t launch_transpose_wr(const void* w_r, int d, int E, smoe_dtype dt, vo
 cudaError_t launch_combine(const void* ws, const int32_t* inv, int T_, int ck, int N, void* out,
                            smoe_dtype dt, const float* dl, const int32_t* idx, const void* w_rt,
                            int E, cudaStream_t s) {
-  const size_t n = (size_t)T_ * cdiv(N / 4, kCombV);
+  const int ve = dt == SMOE_BF16 ? 8 : 4;
+  const size_t n = (size_t)T_ * cdiv(N / ve, kCombV);
   const unsigned blocks = (unsigned)((n + 255) / 256);
   if (dt == SMOE_BF16)
     combine_kernel<bf16><<<blocks, 256, 0, s>>>((const bf16*)ws, inv, T_, ck, N, (bf16*)out, dl,
