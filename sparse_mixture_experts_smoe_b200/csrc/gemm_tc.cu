@@ -400,6 +400,7 @@ struct SharedCtl {
 struct DwExtra {
   int idx[IDX_STAGES][2][BK];  // source row per operand (A, B) of each stage row, -1 = zero
   int off[kMaxE + 1];          // expert offsets
+  short order[kMaxE];          // experts by descending row count (ties: lower id)
 };
 // Grouped-M kernel: a staging area per epilogue warp for the output of one
 // 32-column chunk of its 32 accumulator rows, used in one of two layouts:
@@ -1059,9 +1060,32 @@ dw_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const bool offsets_ok = c.total_mtiles > 0 || g.num_rows == 0;
   const int total = offsets_ok ? g.E * nM * nN : 0;
+  // A tile's work grows with its expert's rows, and routing can be very uneven, so
+  // the tile list runs over the experts from the most rows to the fewest and the
+  // CTAs take it in rounds of gridDim.x tiles, alternately forward and backward
+  // (every role of the CTA derives the same sequence).  Experts beyond 256 keep
+  // their order.
+  if (g.E <= 256) {
+    for (int e = threadIdx.x; e < g.E; e += blockDim.x) {
+      const int n = x.off[e + 1] - x.off[e];
+      int rank = 0;
+      for (int f = 0; f < g.E; ++f) {
+        const int m = x.off[f + 1] - x.off[f];
+        rank += (m > n) || (m == n && f < e);
+      }
+      x.order[rank] = (short)e;
+    }
+  } else {
+    for (int e = threadIdx.x; e < g.E; e += blockDim.x) x.order[e] = (short)e;
+  }
+  __syncthreads();
+  auto tile_of = [&](int j) {  // this CTA's j-th tile
+    const int P = (int)gridDim.x, b = (int)blockIdx.x;
+    return j * P + ((j & 1) ? P - 1 - b : b);
+  };
   // tile L -> (e, nb, mb), mb fastest
   auto coords = [&](int L, int& e, int& mb, int& nb) {
-    e = L / (nM * nN);
+    e = x.order[L / (nM * nN)];
     const int rem = L % (nM * nN);
     nb = rem / nM;
     mb = rem % nM;
@@ -1072,7 +1096,7 @@ dw_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
     if (lane == 0 && !(A_GATHER && B_GATHER)) {
       Ring ra, rb;
       bool run = true;
-      for (int L = blockIdx.x; run && L < total; L += gridDim.x) {
+      for (int jt = 0, L = tile_of(0); run && L < total; L = tile_of(++jt)) {
         int e, mb, nb;
         coords(L, e, mb, nb);
         const int r_begin = x.off[e], r_end = x.off[e + 1];
@@ -1120,7 +1144,7 @@ dw_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
     };
     Ring ri;
     bool run = true;
-    for (int L = blockIdx.x; run && L < total; L += gridDim.x) {
+    for (int jt = 0, L = tile_of(0); run && L < total; L = tile_of(++jt)) {
       int e, mb, nb;
       coords(L, e, mb, nb);
       const int r_begin = x.off[e], r_end = x.off[e + 1];
@@ -1159,7 +1183,7 @@ dw_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
     gb.init(t);
     Ring ra, rb, ri;
     bool run = true;
-    for (int L = blockIdx.x; run && L < total; L += gridDim.x) {
+    for (int jt = 0, L = tile_of(0); run && L < total; L = tile_of(++jt)) {
       int e, mb, nb;
       coords(L, e, mb, nb);
       const int nK = cdiv(x.off[e + 1] - x.off[e], BK);
@@ -1195,7 +1219,7 @@ dw_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
     if (!kGather || lane == 0) {
       Ring ra, rb;
       int it = 0;
-      for (int L = blockIdx.x; L < total; L += gridDim.x, ++it) {
+      for (int jt = 0, L = tile_of(0); L < total; L = tile_of(++jt), ++it) {
         int e, mb, nb;
         coords(L, e, mb, nb);
         const int r_begin = x.off[e], r_end = x.off[e + 1];
@@ -1260,7 +1284,7 @@ dw_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
     uint8_t* box = smem + kRingBytes + kCtlBytes + kDwExtraBytes + q * kDwBoxBytes;
     const uint32_t box_s = smem_u32(box);
     int it = 0;
-    for (int L = blockIdx.x; L < total; L += gridDim.x, ++it) {
+    for (int jt = 0, L = tile_of(0); L < total; L = tile_of(++jt), ++it) {
       int e, mb, nb;
       coords(L, e, mb, nb);
       const int nrows = x.off[e + 1] - x.off[e];
