@@ -158,7 +158,7 @@ def kernel_work(cfg):
     T, d, f, E, k = cfg["T"], cfg["d"], cfg["f"], cfg["E"], cfg["k"]
     S = T * k
     mf = 2 * f if cfg["act"] == "swiglu" else f
-    b = 2  # bf16 bytes
+    b = 4 if cfg.get("dtype") == "f32" else 2  # bytes per element of the layer's dtype
     flops = {
         "gemm.fwd_up": 2.0 * S * d * mf, "gemm.fwd_down": 2.0 * S * f * d,
         "gemm.bwd_dA": 2.0 * S * d * f, "gemm.bwd_dW2": 2.0 * S * f * d,
@@ -167,8 +167,9 @@ def kernel_work(cfg):
     bytes_ = {
         "route": T * d * b + d * E * b + S * 8,
         "sort": 2 * S * 4 + S * 4 + (E + 1) * 4,
-        "combine.y": S * d * 4 + T * d * b,
-        "combine.dx": S * d * 4 + T * d * b + S * 8,
+        # slot rows in the layer dtype (+ one int32 grouped row per slot), output rows
+        "combine.y": S * d * b + S * 4 + T * d * b,
+        "combine.dx": S * d * b + S * 4 + T * d * b + S * 8,
         "dg_reduce": S * 4 * max(1, math.ceil(f / 256)) + S * 8,
         "route_dl": S * 12,
         "route_dw": T * d * b + S * 8 + d * E * 4,
