@@ -392,8 +392,59 @@ SWEEPS = {
 }
 
 
+# small-T forward (inference) on the Mixtral-shaped layer: with a handful of rows per
+# expert the forward reads each used expert's weights once, so the bound is HBM
+DECODE_T = [1, 8, 64, 512]
+
+
+def run_decode(args, world, rank):
+    import sparse_mixture_experts_smoe_b200 as smoe
+    dev = torch.device("cuda", torch.cuda.current_device())
+    peaks = load_peaks()
+    base = WORKLOADS[DEFAULT_WORKLOAD]
+    for T in DECODE_T:
+        cfg = dict(base, T=T)
+        d, f, E, k = cfg["d"], cfg["f"], cfg["E"], cfg["k"]
+        torch.cuda.empty_cache()
+        inp = make_mlp_inputs(cfg, seed=rank, device=dev, with_dy=False)
+        st = smoe.SMoEMLPState(T, d, f, E, k, cfg["act"], torch.bfloat16, dev, with_grad=False)
+        p = (inp["x"], inp["w_r"], inp["b_r"], inp["w1"], inp["w2"])
+        for _ in range(args.warmup):
+            smoe.smoe_mlp_fwd(st, *p)
+        torch.cuda.synchronize()
+        barrier(world)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(args.steps):
+            smoe.smoe_mlp_fwd(st, *p)
+        e1.record()
+        torch.cuda.synchronize()
+        barrier(world)
+        ms = max_over_ranks(e0.elapsed_time(e1), world) / args.steps
+        if smoe.smoe_check() != 0:
+            raise SystemExit(f"device error word set in decode T={T}")
+        rows = (st.expert_offsets[1:] - st.expert_offsets[:-1]).cpu()
+        used = int((rows > 0).sum())
+        mf = 2 * f if cfg["act"] == "swiglu" else f
+        wbytes = used * (d * mf + f * d) * 2  # weights of the experts that received rows
+        gbs = wbytes / (ms / 1e3) / 1e9
+        line = {"sweep": "decode", "T": T, "d": d, "f": f, "E": E, "k": k, "act": cfg["act"],
+                "dtype": "bf16", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+                "ms_fwd": round(ms, 4), "tokens_per_s": round(T * world / (ms / 1e3), 1),
+                "experts_used": used, "weight_bytes": wbytes,
+                "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"],
+                             "unit": "GB/s", "frac": round(gbs / peaks["hbm_gbs"], 4),
+                             "traffic": None},
+                "l2": "weights larger than L2, no flush"}
+        if rank == 0:
+            print(json.dumps(line), flush=True)
+        del st, inp, p
+
+
 def run_sweep(args, world, rank):
     import sparse_mixture_experts_smoe_b200 as smoe
+    if args.sweep == "decode":
+        return run_decode(args, world, rank)
     dev = torch.device("cuda", torch.cuda.current_device())
     peaks = load_peaks()
     names = list(SWEEPS) if args.sweep == "all" else [args.sweep]
@@ -629,7 +680,7 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--sweep", choices=["granularity", "sparsity", "dense", "all"], default=None,
+    ap.add_argument("--sweep", choices=["granularity", "sparsity", "dense", "decode", "all"], default=None,
                     help="time the SMoE MLP over a set of (E, k, f) shapes instead of the benchmark line")
     ap.add_argument("--tokens", type=int, default=0,
                     help="override T (smaller cases for profiler captures; never a bench line)")

@@ -88,6 +88,9 @@ REDUCED = {
     "e128_k16_bf16": dict(kind="mlp", T=96, d=136, f=72, E=128, k=16, dtype="bf16",
                           act="swiglu"),
     "top1_bf16": dict(kind="mlp", T=200, d=136, f=136, E=32, k=1, dtype="bf16", act="swiglu"),
+    # decode-sized batches: a few rows per tile, most experts empty
+    "decode_t1_bf16": dict(kind="mlp", T=1, d=264, f=392, E=8, k=2, dtype="bf16", act="swiglu"),
+    "decode_t5_bf16": dict(kind="mlp", T=5, d=264, f=392, E=8, k=2, dtype="bf16", act="swiglu"),
 }
 
 
@@ -98,6 +101,25 @@ def test_mlp_reduced_full(name):
     if cfg["E"] == 1:      # closed form: gates are exactly 1 and the router gradient vanishes
         assert torch.all(st.gates == 1.0)
         assert torch.all(st.dw_r == 0.0)
+
+
+@pytest.mark.parametrize("T", [1, 8])
+def test_decode_forward_mixtral_shape(T):
+    """The small-T forward the decode sweep times (Mixtral-shaped layer, T tokens):
+    routing bit for bit, every element of y, H and A."""
+    cfg = dict(WORKLOADS["mixtral_bf16_swiglu"], T=T)
+    inp = make_mlp_inputs(cfg, seed=3, device="cuda", with_dy=False)
+    st = smoe.SMoEMLPState(T, cfg["d"], cfg["f"], cfg["E"], cfg["k"], cfg["act"], torch.bfloat16,
+                           "cuda", with_grad=False)
+    smoe.smoe_mlp_fwd(st, inp["x"], inp["w_r"], inp["b_r"], inp["w1"], inp["w2"])
+    torch.cuda.synchronize()
+    assert smoe.smoe_check() == 0
+    c = _cpu(inp)
+    idx, gates, ss = _check_routing(cfg, st, c)
+    fwd = oracle.mlp_fwd(c["x"], c["w1"], c["w2"], cfg["act"], idx, gates, want_ha=True)
+    assert_close("y", st.y, fwd["y"], torch.bfloat16)
+    assert_close("h", st.h, fwd["h"][ss], torch.bfloat16)
+    assert_close("a", st.a, fwd["a"][ss], torch.bfloat16)
 
 
 def test_mlp_is_deterministic():
