@@ -24,13 +24,14 @@
 // expert offsets (expert-major, then N tile, then M tile, so the CTAs of one wave
 // share the expert's input rows in L2).  Warp roles: warp 0 = TMA producer,
 // warp 1 = MMA issuer and tensor-memory owner, warps 4-7 = epilogue (thread r owns
-// accumulator row r), warps 8-15 = row gather of a scattered operand.  Two
+// accumulator row r), warps 8-15 = row gather of a scattered operand (without a
+// gather, warps 8-11 are a second epilogue group for the scaled store).  Two
 // 256-column fp32 accumulators in tensor memory let the epilogue of one tile
 // overlap the main loop of the next.  Epilogues: scaled store (gate), activation
 // forward (H and A = gelu(H) or silu(Hg) * Hu), and the activation backward (gate
 // gradient partial <dA', A>, g*A, dH = g dA' act'(H)); their bf16 rows in grouped
-// order move through shared memory as 32 x 32 TMA boxes, scattered or fp32 rows
-// by per-row bulk copies.
+// order move through shared memory as 32 x 32 TMA boxes, scattered rows by
+// per-row bulk copies.
 //
 // dW kernel: tile (e, m, n) of dW[e] = sum over the expert's rows r of
 // A[r, m] * B[r, n]; the reduction runs over the slice rows, so both operands are
@@ -56,7 +57,7 @@ constexpr int kGatherThreads = 256;   // grouped-M kernel: warps 8-15
 constexpr int kDwGatherThreads = 256; // dW kernel: warps 8-15 gather (more copies in flight)
 constexpr int kDwThreads = 512;
 // Warp roles.  Grouped-M kernel: 0 TMA, 1 MMA, 2-3 idle, 4-7 epilogue, 8-15 row
-// gather.  dW kernel: 0 TMA, 1 MMA, 2 source rows, 3 idle, 4-7 epilogue, 8-15
+// gather (without a gather: 8-11 second epilogue group for EPI_STORE).  dW kernel: 0 TMA, 1 MMA, 2 source rows, 3 idle, 4-7 epilogue, 8-15
 // row gather.  (Measured: a second epilogue warp set on 12-15 with a 4-warp
 // gather was slower than this split.)  The role ranges must not overlap:
 static_assert(kGatherWarp0 == 8 && kGatherWarp0 + kGatherThreads / 32 <= kThreads / 32,
@@ -1064,8 +1065,8 @@ dw_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
   // A tile's work grows with its expert's rows, and routing can be very uneven, so
   // the tile list runs over the experts from the most rows to the fewest and the
   // CTAs take it in rounds of gridDim.x tiles, alternately forward and backward
-  // (every role of the CTA derives the same sequence).  Experts beyond 256 keep
-  // their order.
+  // (every role of the CTA derives the same sequence).  With more than 256
+  // experts the tiles keep the expert index order.
   if (g.E <= 256) {
     for (int e = threadIdx.x; e < g.E; e += blockDim.x) {
       const int n = x.off[e + 1] - x.off[e];

@@ -10,12 +10,15 @@
 // products in ascending i with fmaf, and the 32 lane sums meet in an xor
 // butterfly (16, 8, 4, 2, 1) before the bias is added.
 //
-// Work split: a warp handles TM tokens; a block of 8 warps stages CH rows of W_r
-// in shared memory as fp32 with a row stride = 4 (mod 32) words, so the eight
-// lanes of a 128-bit shared load phase read eight different bank groups, and the
-// block's CH-feature slice of x with 16-byte coalesced loads (lane L then reads
-// its features L, L+32, ... from shared memory; the accumulation order above is
-// unchanged).
+// Two kernels compute these sums.  route_tiled_kernel (E * sizeof(T) a multiple
+// of 16 bytes) blocks the (token, expert) tile over the warps and registers and
+// streams W_r and x through a cp.async pipeline (see its comment).  route_kernel
+// serves the other shapes: a warp handles TM tokens; a block of 8 warps stages CH
+// rows of W_r in shared memory as fp32 with a row stride = 4 (mod 32) words, so
+// the eight lanes of a 128-bit shared load phase read eight different bank
+// groups, and the block's CH-feature slice of x with 16-byte coalesced loads
+// (lane L then reads its features L, L+32, ... from shared memory; the
+// accumulation order above is unchanged).
 #include "common.cuh"
 
 namespace smoe {
