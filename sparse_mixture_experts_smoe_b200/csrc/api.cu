@@ -428,7 +428,7 @@ int smoe_route_bwd(const void* x, const void* w_r, const int32_t* topk_idx, cons
   cudaStream_t s = (cudaStream_t)stream;
   { PROF("route_dl", 1); SMOE_TRY(launch_route_dl(gates, dgates, T, k, l.dl, s), "route_dl"); }
   // the weight gradient walks the slots in grouped order
-  { PROF("sort", 3); SMOE_TRY(launch_sort(topk_idx, T, k, E, l.sorted_slot, l.offsets, l.sort, err, s), "route_bwd sort"); }
+  { PROF("sort", sort_launches(T, k, E)); SMOE_TRY(launch_sort(topk_idx, T, k, E, l.sorted_slot, l.offsets, l.sort, err, s), "route_bwd sort"); }
   { PROF("route_dw", 2); SMOE_TRY(launch_route_dw(x, topk_idx, l.sorted_slot, l.offsets, l.dl, T, d, E, k, dt, l.part, dw_r, db_r, s), "route_dw"); }
   if (dx) { PROF("route_dx", 1); SMOE_TRY(launch_route_dx(l.dl, topk_idx, w_r, T, d, E, k, dt, dx, s), "route_dx"); }
   return SMOE_OK;
@@ -451,7 +451,7 @@ int smoe_sort(const int32_t* topk_idx, int T, int k, int E, int32_t* sorted_slot
   cudaError_t st;
   unsigned* err = error_word(&st);
   if (!err) return cuda_fail(st, "smoe_sort");
-  { PROF("sort", 3); SMOE_TRY(launch_sort(topk_idx, T, k, E, sorted_slot, expert_offsets, workspace, err, s), "smoe_sort"); }
+  { PROF("sort", sort_launches(T, k, E)); SMOE_TRY(launch_sort(topk_idx, T, k, E, sorted_slot, expert_offsets, workspace, err, s), "smoe_sort"); }
   return SMOE_OK;
 }
 
@@ -659,7 +659,7 @@ int smoe_mlp_fwd(const smoe_mlp_desc* desc, const smoe_mlp_tensors* t, void* str
   const int mf = m.act == SMOE_ACT_SWIGLU ? 2 * m.f : m.f;
 
   { PROF("route", 1); SMOE_TRY(launch_route(t->x, t->w_r, t->b_r, m.T, m.d, m.E, m.k, dt, t->topk_idx, t->gates, err, s), "route"); }
-  { PROF("sort", 3); SMOE_TRY(launch_sort(t->topk_idx, m.T, m.k, m.E, t->sorted_slot, t->expert_offsets, l.sort, err, s, l.inv), "sort"); }
+  { PROF("sort", sort_launches(m.T, m.k, m.E)); SMOE_TRY(launch_sort(t->topk_idx, m.T, m.k, m.E, t->sorted_slot, t->expert_offsets, l.sort, err, s, l.inv), "sort"); }
   {  // H = x[gathered] W1, A = act(H)   (scatter -> group, fan-out k)
     GroupedGemm g;
     g.E = m.E; g.num_rows = S; g.offsets = t->expert_offsets; g.sorted_slot = t->sorted_slot;

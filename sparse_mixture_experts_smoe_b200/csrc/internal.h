@@ -90,6 +90,8 @@ cudaError_t launch_route_dx(const float* dl, const int32_t* idx, const void* w_r
                             int E, int k, smoe_dtype dt, void* dx, cudaStream_t s);
 
 size_t sort_workspace_bytes(int T, int k, int E);
+// kernel launches of launch_sort for this shape (1 for a single-block sort, else 3)
+int sort_launches(int T, int k, int E);
 // inv (nullable): also write inv[sorted_slot[i]] = i
 cudaError_t launch_sort(const int32_t* idx, int T, int k, int E, int32_t* sorted_slot,
                         int32_t* offsets, void* ws, unsigned* err, cudaStream_t s,

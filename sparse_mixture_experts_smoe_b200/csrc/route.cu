@@ -464,9 +464,55 @@ cudaError_t launch_route_t(const void* x, const void* w_r, const float* b_r, int
   return cudaGetLastError();
 }
 
+// ---------------------------------------------------------------------------
+// Router for a few tokens (decode).  With T tokens there are only 32 * E * T
+// lane chains, too few to fill a pipeline of feature chunks, so each chain gets
+// its own thread: one block per token, warp w takes experts w, w + 16, ...; lane L
+// accumulates x[t, i] * W_r[i, e] over i = L (mod 32) in ascending i with fmaf
+// (several loads in flight), then the xor butterfly 16, 8, 4, 2, 1 and + b: the
+// documented order, so the logits are the same bits as the other kernels'.
+constexpr int kChainWarps = 16;
+constexpr int kChainMaxT = 64;
+
+template <typename T>
+__global__ void __launch_bounds__(kChainWarps * 32)
+route_chain_kernel(const T* __restrict__ x, const T* __restrict__ w_r,
+                   const float* __restrict__ b_r, int d, int E, int k,
+                   int32_t* __restrict__ idx, float* __restrict__ gates) {
+  __shared__ float logit[128];
+  const int t = blockIdx.x;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const T* xt = x + (size_t)t * d;
+  for (int e = warp; e < E; e += kChainWarps) {
+    float acc = 0.0f;
+#pragma unroll 8
+    for (int i = lane; i < d; i += 32) acc = fmaf(to_f(xt[i]), to_f(w_r[(size_t)i * E + e]), acc);
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) acc = acc + __shfl_xor_sync(0xffffffffu, acc, off);
+    if (lane == 0) logit[e] = b_r != nullptr ? acc + b_r[e] : acc;
+  }
+  __syncthreads();
+  if (warp == 0) {
+    float lv[4];
+    unsigned fr = 0u;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int e = lane + 32 * j;
+      lv[j] = e < E ? logit[e] : 0.0f;
+      if (e < E) fr |= 1u << j;
+    }
+    select_topk<4>(lv, fr, k, lane, idx + (size_t)t * k, gates + (size_t)t * k);
+  }
+}
+
 template <typename T>
 cudaError_t launch_route_dt(const void* x, const void* w_r, const float* b_r, int T_, int d, int E,
                             int k, int32_t* idx, float* gates, unsigned* err, cudaStream_t s) {
+  if (T_ <= kChainMaxT) {
+    route_chain_kernel<T><<<T_, kChainWarps * 32, 0, s>>>((const T*)x, (const T*)w_r, b_r, d, E, k,
+                                                          idx, gates);
+    return cudaGetLastError();
+  }
   // Tiles of 64 accumulators per lane (two blocks per SM) measured faster than
   // 128 (one block per SM) on the 64-expert router: the shorter per-lane work
   // hides the shared-memory and conversion latencies better.

@@ -3,7 +3,8 @@
 //
 // The pages name "reordering operations" fused into ParallelLinear (sourcepulse.org
 // summary, "How It Works") and call the expert-sorted layout "grouped" (library
-// page of arXiv 2403.08245, review 1 summary).  Three launches:
+// page of arXiv 2403.08245, review 1 summary).  Three launches (one, sort_small_kernel,
+// when the slots fit one chunk and E <= 128):
 //   1. count:   each block histograms a chunk of kSortChunk slots (shared-memory
 //               atomics; counts are order-free).
 //   2. scan:    one block turns the [blocks][E] counts into per-block bases
@@ -87,18 +88,18 @@ sort_scan_kernel(int32_t* __restrict__ counts, int n_blocks, int E, int32_t* __r
   if (threadIdx.x == 0) offsets[E] = carry;
 }
 
-__global__ void __launch_bounds__(kSortThreads)
-sort_scatter_kernel(const int32_t* __restrict__ idx, int S, int E,
-                    const int32_t* __restrict__ base, int32_t* __restrict__ sorted_slot,
-                    int32_t* __restrict__ inv) {
-  __shared__ int run[kSortMaxE];                    // running position per expert
-  __shared__ int wcnt[kSortThreads / 32][kSortMaxE / 4 + 1];  // per-warp counts, per round
+// Stable placement of the slots [chunk0, chunk_end) given each expert's running
+// position run[e] (shared memory, advanced in place): rounds of kSortThreads slots
+// in slot order; __match_any_sync ranks each lane among same-expert lanes of its
+// warp, and per-warp counts are scanned across warps, so equal ids keep ascending
+// slot order.
+__device__ __forceinline__ void scatter_chunk(const int32_t* __restrict__ idx, int E, int chunk0,
+                                              int chunk_end, int* run,
+                                              int (*wcnt)[kSortMaxE / 4 + 1],
+                                              int32_t* __restrict__ sorted_slot,
+                                              int32_t* __restrict__ inv) {
   // wcnt holds up to kSortMaxE/4 experts per pass; larger E loops in passes below
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  for (int e = threadIdx.x; e < E; e += blockDim.x) run[e] = base[(size_t)blockIdx.x * E + e];
-  __syncthreads();
-  const int chunk0 = blockIdx.x * kSortChunk;
-  const int chunk_end = min(S, chunk0 + kSortChunk);
   constexpr int kPass = kSortMaxE / 4;
   for (int r0 = chunk0; r0 < chunk_end; r0 += kSortThreads) {
     const int p = r0 + threadIdx.x;
@@ -137,6 +138,51 @@ sort_scatter_kernel(const int32_t* __restrict__ idx, int S, int E,
   }
 }
 
+__global__ void __launch_bounds__(kSortThreads)
+sort_scatter_kernel(const int32_t* __restrict__ idx, int S, int E,
+                    const int32_t* __restrict__ base, int32_t* __restrict__ sorted_slot,
+                    int32_t* __restrict__ inv) {
+  __shared__ int run[kSortMaxE];                              // running position per expert
+  __shared__ int wcnt[kSortThreads / 32][kSortMaxE / 4 + 1];  // per-warp counts, per round
+  for (int e = threadIdx.x; e < E; e += blockDim.x) run[e] = base[(size_t)blockIdx.x * E + e];
+  __syncthreads();
+  const int chunk0 = blockIdx.x * kSortChunk;
+  scatter_chunk(idx, E, chunk0, min(S, chunk0 + kSortChunk), run, wcnt, sorted_slot, inv);
+}
+
+// The three steps in one block, for at most one chunk of slots and kSortSmallE
+// experts (a decode-sized batch): one launch instead of three.
+constexpr int kSortSmallE = 128;
+
+__global__ void __launch_bounds__(kSortThreads)
+sort_small_kernel(const int32_t* __restrict__ idx, int S, int E, int32_t* __restrict__ sorted_slot,
+                  int32_t* __restrict__ offsets, int32_t* __restrict__ inv, unsigned* err) {
+  __shared__ int run[kSortMaxE];
+  __shared__ int wcnt[kSortThreads / 32][kSortMaxE / 4 + 1];
+  for (int e = threadIdx.x; e < E; e += blockDim.x) run[e] = 0;
+  __syncthreads();
+  bool bad = false;
+  for (int p = threadIdx.x; p < S; p += blockDim.x) {
+    const int e = idx[p];
+    if (e >= 0 && e < E) atomicAdd(&run[e], 1);
+    else bad = true;
+  }
+  if (bad) report_error(err, ERRBIT_DATA);
+  __syncthreads();
+  if (threadIdx.x == 0) {  // exclusive prefix sum (E <= kSortSmallE)
+    int acc = 0;
+    for (int e = 0; e < E; ++e) {
+      const int c = run[e];
+      run[e] = acc;
+      offsets[e] = acc;
+      acc += c;
+    }
+    offsets[E] = acc;
+  }
+  __syncthreads();
+  scatter_chunk(idx, E, 0, S, run, wcnt, sorted_slot, inv);
+}
+
 }  // namespace
 
 size_t sort_workspace_bytes(int T_, int k, int E) {
@@ -145,9 +191,17 @@ size_t sort_workspace_bytes(int T_, int k, int E) {
   return nb * (size_t)E * sizeof(int32_t);
 }
 
+int sort_launches(int T_, int k, int E) {
+  return (T_ * k <= kSortChunk && E <= kSortSmallE) ? 1 : 3;
+}
+
 cudaError_t launch_sort(const int32_t* idx, int T_, int k, int E, int32_t* sorted_slot,
                         int32_t* offsets, void* ws, unsigned* err, cudaStream_t s, int32_t* inv) {
   const int S = T_ * k;
+  if (sort_launches(T_, k, E) == 1) {
+    sort_small_kernel<<<1, kSortThreads, 0, s>>>(idx, S, E, sorted_slot, offsets, inv, err);
+    return cudaGetLastError();
+  }
   const int nb = cdiv(S, kSortChunk);
   int32_t* counts = (int32_t*)ws;
   sort_count_kernel<<<nb, kSortThreads, 0, s>>>(idx, S, E, counts, err);
