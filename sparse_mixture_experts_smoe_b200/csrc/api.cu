@@ -225,6 +225,8 @@ RouteBwdWs route_bwd_layout(void* ws, int T, int d, int E, int k) {
 struct MlpWs {
   void* sort = nullptr;
   void* ycomb = nullptr;    // fwd: [S, d] slot rows (dtype), grouped order
+  float* kpart = nullptr;   // fwd: [ksplit, S, d] fp32 split-K partials of the down projection
+  int ksplit = 1;
   float* dg_part = nullptr; // bwd: [S, dg_ld]
   void* dh = nullptr;       // bwd: [S, m*f] dtype (grouped dH)
   void* ga = nullptr;       // bwd: [S, f] dtype (gates * A)
@@ -246,6 +248,9 @@ MlpWs mlp_layout(void* ws, const smoe_mlp_desc& m, int backward) {
   l.inv = (int32_t*)c.take(S * sizeof(int32_t));
   if (!backward) {
     l.ycomb = c.take(S * m.d * esize(dt));
+    // a decode-sized batch splits the down projection's K (tensor-core path only)
+    l.ksplit = dt == SMOE_BF16 ? grouped_ksplit((int)S, m.E, m.d, m.f) : 1;
+    if (l.ksplit > 1) l.kpart = (float*)c.take((size_t)l.ksplit * S * m.d * sizeof(float));
   } else {
     l.dg_ld = cdiv(m.f, act_tile_cols(dt));
     l.dg_part = (float*)c.take(S * l.dg_ld * sizeof(float));
@@ -677,7 +682,13 @@ int smoe_mlp_fwd(const smoe_mlp_desc* desc, const smoe_mlp_tensors* t, void* str
     g.b = t->w2; g.b_kn = 1; g.NW = m.d; g.n_out = m.d;
     g.epi = EPI_STORE; g.gates = t->gates;
     g.out_mode = ROWS_GROUPED; g.out = l.ycomb; g.ldo = m.d; g.out_f32 = dt == SMOE_F32; g.err = err;
+    g.ksplit = l.ksplit; g.partial = l.kpart;
     { PROF("gemm.fwd_down", 1); SMOE_TRY(run_grouped(g, dt, s), "mlp fwd gemm2"); }
+    if (l.ksplit > 1) {
+      PROF("splitk_reduce", 1);
+      SMOE_TRY(launch_splitk_reduce(l.kpart, l.ksplit, S, m.d, t->sorted_slot, t->gates, l.ycomb,
+                                    m.d, s), "mlp fwd split-K reduce");
+    }
   }
   { PROF("combine.y", 1); SMOE_TRY(launch_combine(l.ycomb, l.inv, m.T, m.k, m.d, t->y, dt, nullptr, nullptr, nullptr, 0, s), "mlp fwd combine"); }
   return SMOE_OK;

@@ -170,7 +170,39 @@ __global__ void gather_scale_kernel(const T* __restrict__ src, int ld_src, int m
   out[q] = from_f<T>(g * to_f(src[(size_t)r * ld_src + c]));
 }
 
+// out[i, c..c+3] = g * sum_s partial[s, i, c..c+3], one thread per 4 columns of a row
+__global__ void splitk_reduce_kernel(const float* __restrict__ partial, int ks, int num_rows,
+                                     int n_out, const int32_t* __restrict__ sorted_slot,
+                                     const float* __restrict__ gates, bf16* __restrict__ out,
+                                     int ldo) {
+  const int n4 = n_out / 4;
+  const size_t q = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (q >= (size_t)num_rows * n4) return;
+  const int i = (int)(q / n4), c = (int)(q % n4) * 4;
+  float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int sp = 0; sp < ks; ++sp) {
+    const float4 v = __ldg(reinterpret_cast<const float4*>(partial + ((size_t)sp * num_rows + i) * n_out + c));
+    a.x += v.x; a.y += v.y; a.z += v.z; a.w += v.w;
+  }
+  const int p = sorted_slot[i];
+  const float g = (gates != nullptr && p >= 0 && p < num_rows) ? gates[p] : 1.0f;
+  __nv_bfloat162 lo = __floats2bfloat162_rn(g * a.x, g * a.y), hi = __floats2bfloat162_rn(g * a.z, g * a.w);
+  uint2 r;
+  r.x = *reinterpret_cast<uint32_t*>(&lo);
+  r.y = *reinterpret_cast<uint32_t*>(&hi);
+  *reinterpret_cast<uint2*>(out + (size_t)i * ldo + c) = r;
+}
+
 }  // namespace
+
+cudaError_t launch_splitk_reduce(const float* partial, int ksplit, int num_rows, int n_out,
+                                 const int32_t* sorted_slot, const float* gates, void* out,
+                                 int ldo, cudaStream_t s) {
+  const size_t n = (size_t)num_rows * (n_out / 4);
+  splitk_reduce_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(partial, ksplit, num_rows, n_out,
+                                                                    sorted_slot, gates, (bf16*)out, ldo);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_transpose_wr(const void* w_r, int d, int E, smoe_dtype dt, void* w_rt,
                                 cudaStream_t s) {

@@ -561,7 +561,7 @@ __device__ __forceinline__ void teardown(SharedCtl& c) {
 // ---------------------------------------------------------------------------
 // Grouped-M kernel
 // ---------------------------------------------------------------------------
-template <bool A_GATHER, bool B_KMAJOR, bool SWIGLU_FWD, bool PAIR>
+template <bool A_GATHER, bool B_KMAJOR, bool SWIGLU_FWD, bool PAIR, bool SPLITK = false>
 __global__ void __launch_bounds__(kThreads, 1)
 grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
                        const __grid_constant__ CUtensorMap tmB,
@@ -596,8 +596,14 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int first = PAIR ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
   const int stride = PAIR ? (int)(gridDim.x >> 1) : (int)gridDim.x;
-  const int total = c.total_mtiles * nN;
   const int nK = cdiv(g.K, BK);
+  // Split K (a product with too few tiles to fill the GPU, as at decode sizes):
+  // work item L is K-blocks [kb_lo(L), kb_hi(L)) of tile L / ks, and the epilogue
+  // stores the raw fp32 sum to its split's partial buffer (reduced afterwards).
+  const int ks = SPLITK ? g.ksplit : 1;  // 1 (folded away) in every other instantiation
+  const int total = c.total_mtiles * nN * ks;
+  auto kb_lo = [&](int L) { return (L % ks) * nK / ks; };
+  auto kb_hi = [&](int L) { return (L % ks + 1) * nK / ks; };
   constexpr int BNo = SWIGLU_FWD ? BN / 2 : BN;  // logical output columns per tile
 
   if (warp == 0) {
@@ -606,8 +612,8 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
       Ring r;
       bool run = true;
       for (int L = first; run && L < total; L += stride) {
-        const Tile t = map_tile<PAIR>(c, g.offsets, g.E, nN, L, rank);
-        for (int kb = 0; kb < nK; ++kb) {
+        const Tile t = map_tile<PAIR>(c, g.offsets, g.E, nN, L / ks, rank);
+        for (int kb = kb_lo(L), kb_end = kb_hi(L); kb < kb_end; ++kb) {
           if (!mbar_wait(&c.emptyA[r.s], r.ph ^ 1, abort_flag, g.err)) { run = false; break; }
           uint8_t* b_dst = sB + r.s * BSTAGE;
           // a pair: both CTAs' TMA bytes count on the leader's barrier, whose
@@ -654,7 +660,7 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
     Ring r;
     bool run = true;
     for (int L = first; run && L < total; L += stride) {
-      const Tile tl = map_tile<PAIR>(c, g.offsets, g.E, nN, L, rank);
+      const Tile tl = map_tile<PAIR>(c, g.offsets, g.E, nN, L / ks, rank);
       const bf16* src[kRowsPer];
       uint32_t ok_rows = 0;
 #pragma unroll
@@ -672,7 +678,7 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
           }
         }
       }
-      for (int kb = 0; kb < nK; ++kb) {
+      for (int kb = kb_lo(L), kb_end = kb_hi(L); kb < kb_end; ++kb) {
         if (!mbar_wait(&c.emptyA[r.s], r.ph ^ 1, abort_flag, g.err)) { run = false; break; }
         const uint32_t a_dst = smem_u32(sA + r.s * A_BYTES);
         const bool col_ok = kb * BK + 8 * cc < g.K;
@@ -694,7 +700,7 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
         Ring r;
         bool run = true;
         for (int L = first; run && L < total; L += stride) {
-          for (int kb = 0; kb < nK; ++kb) {
+          for (int kb = kb_lo(L), kb_end = kb_hi(L); kb < kb_end; ++kb) {
             if (!mbar_wait(&c.fullA[r.s], r.ph, abort_flag, g.err)) { run = false; break; }
             fence_proxy_async();  // rows written by cp.async, read by the tensor core
             mbar_arrive_cluster_relaxed(peer_addr(&c.pfull[r.s], 0));
@@ -712,8 +718,9 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
         if (!mbar_wait(&c.tempty[buf], tph ^ 1, abort_flag, g.err)) break;
         tc_fence_after();
         const uint32_t d_tmem = c.tmem_base + buf * BN;
+        const int kb0 = kb_lo(L);
         bool ok = true;
-        for (int kb = 0; kb < nK; ++kb) {
+        for (int kb = kb_lo(L), kb_end = kb_hi(L); kb < kb_end; ++kb) {
           if (!mbar_wait(&c.fullA[r.s], r.ph, abort_flag, g.err)) { ok = false; break; }
           if (PAIR && A_GATHER && !mbar_wait(&c.pfull[r.s], r.ph, abort_flag, g.err)) { ok = false; break; }
           tc_fence_after();
@@ -724,8 +731,8 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
           for (int kk = 0; kk < BK / 16; ++kk) {
             const uint64_t ad = desc_kmajor(a_addr + kk * 32);
             const uint64_t bd = B_KMAJOR ? desc_kmajor(b_addr + kk * 32) : desc_mnmajor(b_addr + kk * 2048);
-            if (PAIR) umma_bf16_pair(d_tmem, ad, bd, idesc, (kb | kk) != 0);
-            else umma_bf16(d_tmem, ad, bd, idesc, (kb | kk) != 0);
+            if (PAIR) umma_bf16_pair(d_tmem, ad, bd, idesc, ((kb - kb0) | kk) != 0);
+            else umma_bf16(d_tmem, ad, bd, idesc, ((kb - kb0) | kk) != 0);
           }
           if (PAIR) {  // the stage is free in both CTAs
             umma_commit_pair(smem_u32(&c.emptyA[r.s]));
@@ -785,7 +792,7 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
       const int buf = it & 1;
       if (two && buf != grp) continue;  // the other group's tile
       const uint32_t tph = (it >> 1) & 1;
-      const Tile t = map_tile<PAIR>(c, g.offsets, g.E, nN, L, rank);
+      const Tile t = map_tile<PAIR>(c, g.offsets, g.E, nN, L / ks, rank);
       if (!mbar_wait(&c.tfull[buf], tph, abort_flag, g.err)) break;
       tc_fence_after();
       const int i = t.row0 + r;
@@ -858,6 +865,17 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
           }
         }
         if (!(act_bwd && (box_flags & kBoxLoads))) tmem_ld32(trow + c0, v);
+        if (SPLITK) {  // split K: this split's raw fp32 sums
+          if (valid) {
+            float4* dst = reinterpret_cast<float4*>(
+                g.partial + ((size_t)(L % ks) * g.num_rows + i) * g.n_out + n0);
+#pragma unroll
+            for (int q4 = 0; q4 < 8; ++q4)
+              if (4 * q4 < ncols)
+                dst[q4] = make_float4(v[4 * q4], v[4 * q4 + 1], v[4 * q4 + 2], v[4 * q4 + 3]);
+          }
+          continue;
+        }
         if (SWIGLU_FWD) tmem_ld32(trow + BNo + c0, u);
         bulk_wait_read();  // this thread's earlier copies have read the staging area ...
         __syncwarp();      // ... and so have the other lanes'
@@ -1452,10 +1470,10 @@ struct EpiMaps {
 // 2-CTA clusters as the device can hold at once (fewer than half the SMs when a
 // GPC has an odd number of free SMs; a cluster beyond that would run its whole
 // share of the tile list after the others).
-template <bool AG, bool BK_, bool SW>
+template <bool AG, bool BK_, bool SW, bool SPLIT = false>
 cudaError_t launch_g(const CUtensorMap& ta, const CUtensorMap& tb, const EpiMaps& m,
                      const GroupedGemm& g, int nN, long long tiles, cudaStream_t s) {
-  auto kern = grouped_gemm_tc_kernel<AG, BK_, SW, kPairM>;
+  auto kern = grouped_gemm_tc_kernel<AG, BK_, SW, kPairM, SPLIT>;
   cudaError_t e = prep(kern, kGroupedSmem);
   if (e != cudaSuccess) return e;
   if (!kPairM) {
@@ -1512,10 +1530,26 @@ bool tc_supported() {
 
 int tc_tile_cols() { return BN; }
 
+int grouped_ksplit(int num_rows, int E, int n_out, int K) {
+  constexpr long long kSms = 148;  // a fixed count, so the split (and the workspace) is the same on any GPU
+  const long long tiles = (long long)(cdiv(num_rows, BM) + (E < num_rows ? E : num_rows)) * cdiv(n_out, BN);
+  if (tiles <= 0 || tiles * 2 > kSms) return 1;
+  int ks = (int)((kSms + tiles - 1) / tiles);
+  if (ks > 8) ks = 8;
+  const int most = cdiv(K, BK) / 4;  // at least four K-blocks per split
+  if (ks > most) ks = most;
+  return ks > 1 ? ks : 1;
+}
+
 cudaError_t launch_grouped_gemm_tc(const GroupedGemm& g, cudaStream_t s) {
   if (g.num_rows == 0) return cudaSuccess;
   if (g.E > kMaxE) return cudaErrorInvalidValue;
   if (g.out_f32) return cudaErrorInvalidValue;  // every output of this path is bf16
+  if (g.ksplit > 1) {  // split K: the plain-store epilogue of a TMA-fed single-CTA product
+    if (g.a_mode != ROWS_GROUPED || g.epi != EPI_STORE || kPairM || g.partial == nullptr ||
+        g.ksplit > cdiv(g.K, BK))
+      return cudaErrorInvalidValue;
+  }
   const bool swiglu = g.epi == EPI_ACT_FWD && g.act == SMOE_ACT_SWIGLU;
   const int BNo = swiglu ? BN / 2 : BN;
   const int nN = cdiv(g.n_out, BNo);
@@ -1550,7 +1584,11 @@ cudaError_t launch_grouped_gemm_tc(const GroupedGemm& g, cudaStream_t s) {
   if (ld && need_h && out_map(&m.xh, g.aux_h, g.n_out, parts, g.num_rows, g.ld_aux_h) != cudaSuccess) ld = false;
   m.flags = (st ? kBoxStores : 0) | (ld ? kBoxLoads : 0);
   const int tm = kPairM ? 2 * BM : BM;  // rows per M tile
-  const long long tiles = (long long)(cdiv(g.num_rows, tm) + g.E) * nN;
+  const long long tiles = (long long)(cdiv(g.num_rows, tm) + g.E) * nN * (g.ksplit > 1 ? g.ksplit : 1);
+  if (g.ksplit > 1) {  // grouped A, plain store (checked above)
+    if (kmaj) return launch_g<false, true, false, true>(ta, tb, m, g, nN, tiles, s);
+    return launch_g<false, false, false, true>(ta, tb, m, g, nN, tiles, s);
+  }
 #define SMOE_LAUNCH_G(AG, KM, SW) launch_g<AG, KM, SW>(ta, tb, m, g, nN, tiles, s)
   if (gather) {
     if (kmaj) return swiglu ? SMOE_LAUNCH_G(true, true, true) : SMOE_LAUNCH_G(true, true, false);

@@ -54,6 +54,11 @@ struct GroupedGemm {
   int ld_aux_h = 0;
   float* dg_partial = nullptr;  // ACT_BWD: [num_rows, dg_ld], column = N tile index
   int dg_ld = 0;
+  // split K (EPI_STORE, grouped A, tensor-core path): ksplit > 1 writes each split's
+  // raw fp32 sums to partial [ksplit, num_rows, n_out]; launch_splitk_reduce then
+  // applies the gates and stores out
+  int ksplit = 1;
+  float* partial = nullptr;
   unsigned* err = nullptr;
 };
 
@@ -115,6 +120,16 @@ cudaError_t launch_dg_reduce(const float* partial, int ld, int n_tiles, const in
 cudaError_t launch_gather_scale(const void* src, int ld_src, int mode, int fan_out,
                                 const int32_t* sorted_slot, const float* gates, int num_rows,
                                 int cols, void* out, smoe_dtype dt, cudaStream_t s);
+
+// out[i, :] = gates[sorted_slot[i]] * sum_{s < ksplit} partial[s, i, :] (ascending s),
+// grouped rows, bf16; the epilogue of a split-K grouped product
+cudaError_t launch_splitk_reduce(const float* partial, int ksplit, int num_rows, int n_out,
+                                 const int32_t* sorted_slot, const float* gates, void* out,
+                                 int ldo, cudaStream_t s);
+// Splits of K for a grouped product of num_rows rows over E experts with n_out
+// output columns and K-dimension K: > 1 only when even the most tiles it can have
+// would leave most SMs idle (decode-sized batches).
+int grouped_ksplit(int num_rows, int E, int n_out, int K);
 
 cudaError_t launch_grouped_gemm_simt(const GroupedGemm& g, smoe_dtype dt, cudaStream_t s);
 cudaError_t launch_dw_gemm_simt(const DwGemm& g, smoe_dtype dt, cudaStream_t s);

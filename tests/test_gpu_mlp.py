@@ -91,6 +91,9 @@ REDUCED = {
     # decode-sized batches: a few rows per tile, most experts empty
     "decode_t1_bf16": dict(kind="mlp", T=1, d=264, f=392, E=8, k=2, dtype="bf16", act="swiglu"),
     "decode_t5_bf16": dict(kind="mlp", T=5, d=264, f=392, E=8, k=2, dtype="bf16", act="swiglu"),
+    # few enough tiles that the down projection splits its K (4 splits, ragged last K-block)
+    "decode_t2_splitk_bf16": dict(kind="mlp", T=2, d=264, f=1000, E=8, k=2, dtype="bf16",
+                                  act="swiglu"),
 }
 
 
