@@ -151,3 +151,22 @@ def test_workspaces_hold_no_copy_of_token_rows():
     assert fwd == a256(sort) + a256(S * 4) + a256(S * d * 2)
     big = a256(S * 2 * f * 2) + a256(S * f * 2) + a256(S * d * 2)
     assert bwd - big < S * d * 2 // 4
+
+
+def test_decode_workspace_holds_the_split_k_partials():
+    """A one-token Mixtral-shaped forward splits the down projection's K four ways (2
+    experts x 16 N tiles cannot fill 148 SMs): its workspace is the sort counts, the
+    grouped row of each slot, the bf16 slot rows and 4 fp32 partial copies of them.
+    From 8 tokens on, the tiles can fill the GPU and no partials are reserved."""
+    import ctypes
+    import sparse_mixture_experts_smoe_b200 as smoe
+    L = smoe.lib()
+    a256 = lambda n: (n + 255) // 256 * 256  # noqa: E731
+    d, f, E, k = 4096, 14336, 8, 2
+    for T, splits in ((1, 4), (8, 1)):
+        S = T * k
+        desc = smoe.MlpDesc(T, d, f, E, k, smoe.ACT["swiglu"], smoe.BF16)
+        fwd = L.smoe_mlp_workspace_size(ctypes.byref(desc), 0)
+        sort = L.smoe_workspace_size(0, T, k, E, d, f, 1)
+        part = a256(splits * S * d * 4) if splits > 1 else 0
+        assert fwd == a256(sort) + a256(S * 4) + a256(S * d * 2) + part
