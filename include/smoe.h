@@ -126,8 +126,8 @@ int smoe_route(const void* x, const void* w_r, const float* b_r, int T, int d, i
  *   dl[t,j] = gates[t,j] (dgates[t,j] - sum_i gates[t,i] dgates[t,i]) for the
  *   selected expert e = topk_idx[t,j], 0 for unselected experts;
  *   dw_r[i,e] = sum_t x[t,i] dl[t,e]  (fp32, overwritten; summed in token order in
- *                                      runs of 128 expert-sorted slots, the runs
- *                                      then in order: fixed by T, k, E and routing)
+ *                                      runs of 32-128 expert-sorted slots, the runs
+ *                                      then in order: fixed by T, k, d, E, routing)
  *   db_r[e]   = sum_t dl[t,e]         (fp32, overwritten; NULL to skip)
  *   dx[t,i]  += sum_j dl[t,j] W_r[i, topk_idx[t,j]]  (dtype, accumulated into dx;
  *                                                     NULL to skip)
@@ -197,7 +197,8 @@ int smoe_selftest_wait_timeout(int limit_us, void* stream);
  *                                      order (combine_k > 0, scattered only;
  *                                      y [num_slots / combine_k, N])
  * No grouped or padded copy of a scattered input is made.  The k-way combine is
- * deterministic (no atomics).
+ * deterministic (no atomics): each slot's (gated) v is rounded to dtype, as the
+ * library materialises per-slot outputs, and the combine_k values are summed in fp32.
  *   x [x_rows, K] dtype, w [E, K, N] dtype, y dtype.
  * ------------------------------------------------------------------------ */
 size_t parallel_linear_fwd_workspace_size(int num_slots, int K, int N, int E, int combine_k,

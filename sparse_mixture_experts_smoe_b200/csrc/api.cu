@@ -214,7 +214,7 @@ RouteBwdWs route_bwd_layout(void* ws, int T, int d, int E, int k) {
   l.sort = c.take(sort_workspace_bytes(T, k, E));
   l.sorted_slot = (int32_t*)c.take(S * sizeof(int32_t));
   l.offsets = (int32_t*)c.take((size_t)(E + 1) * sizeof(int32_t));
-  l.part = (float*)c.take((size_t)route_dw_runs((int)S, E) * (d + 1) * sizeof(float));
+  l.part = (float*)c.take((size_t)route_dw_runs((int)S, E, d) * (d + 1) * sizeof(float));
   l.bytes = c.off;
   return l;
 }
@@ -259,7 +259,7 @@ MlpWs mlp_layout(void* ws, const smoe_mlp_desc& m, int backward) {
     l.dxcomb = c.take(S * m.d * esize(dt));
     l.dl = (float*)c.take(S * sizeof(float));
     l.dg = (float*)c.take(S * sizeof(float));
-    l.r_runs = route_dw_runs((int)S, m.E);
+    l.r_runs = route_dw_runs((int)S, m.E, m.d);
     l.rpart = (float*)c.take((size_t)l.r_runs * (m.d + 1) * sizeof(float));
     l.wrt = c.take((size_t)m.E * m.d * esize(dt));
   }

@@ -84,13 +84,13 @@ cudaError_t launch_route(const void* x, const void* w_r, const float* b_r, int T
 cudaError_t launch_route_dl(const float* gates, const float* dgates, int T, int k, float* dl,
                             cudaStream_t s);
 // Router weight gradient from the slots in grouped order (sorted_slot, offsets of
-// the expert sort of idx).  partial: route_dw_runs(T*k, E) * (d + 1) floats.
+// the expert sort of idx).  partial: route_dw_runs(T*k, E, d) * (d + 1) floats.
 cudaError_t launch_route_dw(const void* x, const int32_t* idx, const int32_t* sorted_slot,
                             const int32_t* offsets, const float* dl, int T, int d, int E, int k,
                             smoe_dtype dt, float* partial, float* dw_r, float* db_r,
                             cudaStream_t s);
 // Rows of the router weight gradient's partial sums (sizes its workspace).
-int route_dw_runs(int S, int E);
+int route_dw_runs(int S, int E, int d);
 cudaError_t launch_route_dx(const float* dl, const int32_t* idx, const void* w_r, int T, int d,
                             int E, int k, smoe_dtype dt, void* dx, cudaStream_t s);
 

@@ -543,35 +543,48 @@ __global__ void route_dl_kernel(const float* __restrict__ gates, const float* __
 
 // Router weight gradient, dw_r[i, e] = sum_t x[t, i] dl[t, e], over the slots in
 // grouped order (sorted by expert, token order within an expert).  The grouped
-// rows are cut into segments of kRunRows; a warp walks one segment for one slab
+// rows are cut into segments of R rows; a warp walks one segment for one slab
 // of columns, accumulating the current expert's sum in registers, and writes one
 // partial row per (segment w, expert e) run it meets.  Along the grouped order the
 // expert never decreases, so w + e numbers the runs without collisions
-// (S / kRunRows + E rows).  A second pass sums, for each expert, the runs of the
+// (S / R + E rows).  A second pass sums, for each expert, the runs of the
 // segments its slice covers in ascending w.  The order of every addition depends
 // only on (T, k, E) and the routing, not on the GPU.  x is read once per slot,
 // mostly from L2 (k reads of each token row).
-constexpr int kRunRows = 128;
-constexpr int kDwLoads = 2;  // 16-byte x loads per lane per row
+// R (128, 64 or 32 rows) and the slab width (2 or 1 16-byte loads per lane and row)
+// follow from (S, d) alone -- the largest that still gives two blocks per SM of a
+// 148-SM B200 -- so the order of the additions is fixed by the shape.
+struct DwPlan {
+  int rows, loads;
+};
+DwPlan dw_plan(int S, int d) {
+  const int cands[4][2] = {{128, 2}, {64, 2}, {32, 2}, {32, 1}};
+  for (const auto& c : cands) {
+    const long long blocks = (long long)cdiv(cdiv(S > 0 ? S : 1, c[0]), 8) * cdiv(d, 32 * c[1] * 8);
+    if (blocks >= 2 * 148) return {c[0], c[1]};
+  }
+  return {32, 1};
+}
 
-template <typename T>
+template <typename T, int LOADS>
 struct DwSlab {
   static constexpr int VPL = 16 / (int)sizeof(T);       // elements per 16-byte load
-  static constexpr int COLS = 32 * kDwLoads * VPL;       // slab width: 512 bf16 / 256 fp32
+  static constexpr int COLS = 32 * LOADS * VPL;          // slab width
 };
 
-template <typename T>
+template <typename T, int LOADS>
 __global__ void __launch_bounds__(256)
 route_dw_run_kernel(const T* __restrict__ x, const int32_t* __restrict__ idx,
                     const int32_t* __restrict__ sorted_slot, const float* __restrict__ dl, int S,
-                    int d, int E, int k, float* __restrict__ part, float* __restrict__ partb) {
-  constexpr int VPL = DwSlab<T>::VPL, NA = kDwLoads * VPL;
+                    int d, int E, int k, int R, float* __restrict__ part,
+                    float* __restrict__ partb) {
+  constexpr int VPL = DwSlab<T, LOADS>::VPL, NA = LOADS * VPL;
   const int lane = threadIdx.x & 31;
   const int w = blockIdx.x * 8 + (threadIdx.x >> 5);  // segment
-  const int r0 = w * kRunRows;
+  const int r0 = w * R;
   if (r0 >= S) return;
-  const int r1 = min(S, r0 + kRunRows);
-  const int c0 = blockIdx.y * DwSlab<T>::COLS + lane * VPL;  // column of load u: c0 + 32 u VPL
+  const int r1 = min(S, r0 + R);
+  const int c0 = blockIdx.y * DwSlab<T, LOADS>::COLS + lane * VPL;  // column of load u: c0 + 32 u VPL
   float2 acc[NA / 2];
 #pragma unroll
   for (int a = 0; a < NA / 2; ++a) acc[a] = make_float2(0.f, 0.f);
@@ -581,7 +594,7 @@ route_dw_run_kernel(const T* __restrict__ x, const int32_t* __restrict__ idx,
     if (cur < 0) return;
     float* dst = part + (size_t)(w + cur) * d;
 #pragma unroll
-    for (int u = 0; u < kDwLoads; ++u) {
+    for (int u = 0; u < LOADS; ++u) {
       const int col = c0 + u * 32 * VPL;
       if (col >= d) continue;
 #pragma unroll
@@ -605,7 +618,7 @@ route_dw_run_kernel(const T* __restrict__ x, const int32_t* __restrict__ idx,
       }
     }
     for (int j = 0; j < n; j += 4) {
-      uint4 xv[4][kDwLoads];
+      uint4 xv[4][LOADS];
       int ej[4];
       float gj[4];
 #pragma unroll
@@ -616,7 +629,7 @@ route_dw_run_kernel(const T* __restrict__ x, const int32_t* __restrict__ idx,
         gj[q] = __shfl_sync(0xffffffffu, g, jj);
         ej[q] = jj < n ? e_q : -1;
 #pragma unroll
-        for (int u = 0; u < kDwLoads; ++u) {
+        for (int u = 0; u < LOADS; ++u) {
           const int col = c0 + u * 32 * VPL;
           xv[q][u] = (ej[q] >= 0 && col < d)
                          ? __ldg(reinterpret_cast<const uint4*>(x + (size_t)t_q * d + col))
@@ -635,7 +648,7 @@ route_dw_run_kernel(const T* __restrict__ x, const int32_t* __restrict__ idx,
         }
         const float2 g2 = make_float2(gj[q], gj[q]);
 #pragma unroll
-        for (int u = 0; u < kDwLoads; ++u) {
+        for (int u = 0; u < LOADS; ++u) {
           float xf[VPL];
           cvt16(xv[q][u], xf, T());
 #pragma unroll
@@ -652,7 +665,7 @@ route_dw_run_kernel(const T* __restrict__ x, const int32_t* __restrict__ idx,
 // dw_r[i][e] = sum over the segments w covering expert e's rows (ascending) of
 // part[w + e][i]; db_r[e] likewise from partb
 __global__ void route_dw_sum_kernel(const float* __restrict__ part, const float* __restrict__ partb,
-                                    const int32_t* __restrict__ offsets, int S, int d, int E,
+                                    const int32_t* __restrict__ offsets, int S, int d, int E, int R,
                                     float* __restrict__ dw_r, float* __restrict__ db_r) {
   const int q = blockIdx.x * blockDim.x + threadIdx.x;  // q = e * d + i
   if (q >= d * E) return;
@@ -660,8 +673,8 @@ __global__ void route_dw_sum_kernel(const float* __restrict__ part, const float*
   const int lo = min(max(offsets[e], 0), S), hi = min(max(offsets[e + 1], lo), S);
   float s = 0.f, sb = 0.f;
   if (hi > lo) {
-    const int w1 = (hi - 1) / kRunRows;
-    for (int w = lo / kRunRows; w <= w1; ++w) {
+    const int w1 = (hi - 1) / R;
+    for (int w = lo / R; w <= w1; ++w) {
       s += __ldg(part + (size_t)(w + e) * d + i);
       if (i == 0) sb += partb[w + e];
     }
@@ -701,26 +714,40 @@ cudaError_t launch_route_dl(const float* gates, const float* dgates, int T_, int
   return cudaGetLastError();
 }
 
-int route_dw_runs(int S, int E) { return cdiv(S > 0 ? S : 1, kRunRows) + E; }
+int route_dw_runs(int S, int E, int d) { return cdiv(S > 0 ? S : 1, dw_plan(S, d).rows) + E; }
 
 cudaError_t launch_route_dw(const void* x, const int32_t* idx, const int32_t* sorted_slot,
                             const int32_t* offsets, const float* dl, int T_, int d, int E, int k,
                             smoe_dtype dt, float* part, float* dw_r, float* db_r, cudaStream_t s) {
   const int S = T_ * k;
-  const int nseg = cdiv(S, kRunRows);
-  float* partb = part + (size_t)route_dw_runs(S, E) * d;
+  const DwPlan pl = dw_plan(S, d);
+  const int nseg = cdiv(S, pl.rows);
+  float* partb = part + (size_t)route_dw_runs(S, E, d) * d;
   if (dt == SMOE_BF16) {
-    dim3 grid(cdiv(nseg, 8), cdiv(d, DwSlab<bf16>::COLS));
-    route_dw_run_kernel<bf16><<<grid, 256, 0, s>>>((const bf16*)x, idx, sorted_slot, dl, S, d, E, k,
-                                                    part, partb);
+    if (pl.loads == 2) {
+      dim3 grid(cdiv(nseg, 8), cdiv(d, DwSlab<bf16, 2>::COLS));
+      route_dw_run_kernel<bf16, 2><<<grid, 256, 0, s>>>((const bf16*)x, idx, sorted_slot, dl, S, d, E, k,
+                                                        pl.rows, part, partb);
+    } else {
+      dim3 grid(cdiv(nseg, 8), cdiv(d, DwSlab<bf16, 1>::COLS));
+      route_dw_run_kernel<bf16, 1><<<grid, 256, 0, s>>>((const bf16*)x, idx, sorted_slot, dl, S, d, E, k,
+                                                        pl.rows, part, partb);
+    }
   } else {
-    dim3 grid(cdiv(nseg, 8), cdiv(d, DwSlab<float>::COLS));
-    route_dw_run_kernel<float><<<grid, 256, 0, s>>>((const float*)x, idx, sorted_slot, dl, S, d, E,
-                                                     k, part, partb);
+    if (pl.loads == 2) {
+      dim3 grid(cdiv(nseg, 8), cdiv(d, DwSlab<float, 2>::COLS));
+      route_dw_run_kernel<float, 2><<<grid, 256, 0, s>>>((const float*)x, idx, sorted_slot, dl, S, d,
+                                                         E, k, pl.rows, part, partb);
+    } else {
+      dim3 grid(cdiv(nseg, 8), cdiv(d, DwSlab<float, 1>::COLS));
+      route_dw_run_kernel<float, 1><<<grid, 256, 0, s>>>((const float*)x, idx, sorted_slot, dl, S, d,
+                                                         E, k, pl.rows, part, partb);
+    }
   }
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  route_dw_sum_kernel<<<cdiv(d * E, 256), 256, 0, s>>>(part, partb, offsets, S, d, E, dw_r, db_r);
+  route_dw_sum_kernel<<<cdiv(d * E, 256), 256, 0, s>>>(part, partb, offsets, S, d, E, pl.rows, dw_r,
+                                                       db_r);
   return cudaGetLastError();
 }
 
