@@ -65,6 +65,10 @@ static_assert(kGatherWarp0 == 8 && kGatherWarp0 + kGatherThreads / 32 <= kThread
 static_assert(kGatherWarp0 + kDwGatherThreads / 32 <= kDwThreads / 32,
               "dW gather warps must fit the block");
 constexpr uint32_t kTmemCols = 512;  // two BN-column fp32 accumulators
+// Gathered products with K up to this (except SwiGLU's forward) use the short-K layout
+// of the grouped kernel (4 gather warps, two epilogue groups, 3 stages); longer ones
+// keep 8 gather warps.
+constexpr int kShortK = 2048;
 constexpr int A_BYTES = BM * BK * 2;  // 16 KB
 constexpr int B_BYTES = BN * BK * 2;  // 32 KB
 constexpr int kMaxE = 1024;
@@ -389,7 +393,7 @@ struct SharedCtl {
   uint64_t pfull[kMaxStages];   // pair leader: the other CTA's stage s has landed
   uint64_t ifull[IDX_STAGES];   // index ring: written by warp 2
   uint64_t iempty[IDX_STAGES];  // index ring: released by the 4 gather warps
-  uint64_t ebar[4];             // per epilogue warp: its input boxes have landed
+  uint64_t ebar[8];             // per epilogue warp: its input boxes have landed
   uint32_t tmem_base;
   int abort_flag;
   int total_mtiles;
@@ -496,7 +500,7 @@ __device__ __forceinline__ void setup(SharedCtl& c, const int32_t* offsets, int 
       mbar_init(&c.ifull[b], 1);
       mbar_init(&c.iempty[b], gather_warps);
     }
-    for (int b = 0; b < 4; ++b) mbar_init(&c.ebar[b], 1);
+    for (int b = 0; b < 8; ++b) mbar_init(&c.ebar[b], 1);
     c.abort_flag = 0;
     fence_mbar_init();
   }
@@ -561,7 +565,8 @@ __device__ __forceinline__ void teardown(SharedCtl& c) {
 // ---------------------------------------------------------------------------
 // Grouped-M kernel
 // ---------------------------------------------------------------------------
-template <bool A_GATHER, bool B_KMAJOR, bool SWIGLU_FWD, bool PAIR, bool SPLITK = false>
+template <bool A_GATHER, bool B_KMAJOR, bool SWIGLU_FWD, bool PAIR, bool SPLITK = false,
+          bool SHORTK = false>
 __global__ void __launch_bounds__(kThreads, 1)
 grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
                        const __grid_constant__ CUtensorMap tmB,
@@ -573,9 +578,15 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
   // One ring of STAGES stages holds A and B together (fullA/emptyA guard a whole
   // stage): measured faster here than separate rings, whose second wait and
   // commit per stage cost more than their extra depth returned.  A pair's CTA
-  // holds half of B per stage, so its ring is deeper.
+  // holds half of B per stage, so its ring is deeper.  SHORTK (a gathered product
+  // with a short K): 3 stages, half the gather warps (8-11), and warps 12-15 as a
+  // second epilogue group staging in the ring space the fourth stage leaves free.
   constexpr int BSTAGE = PAIR ? B_BYTES / 2 : B_BYTES;
-  constexpr int STAGES = PAIR ? 6 : 4;
+  constexpr int STAGES = PAIR ? 6 : (SHORTK ? 3 : 4);
+  constexpr int GTHREADS = SHORTK ? kGatherThreads / 2 : kGatherThreads;  // gather threads
+  static_assert(!SHORTK || (A_GATHER && !PAIR &&
+                            STAGES * (A_BYTES + BSTAGE) + 4 * kWarpStaging <= kRingBytes),
+                "short-K layout");
   static_assert(STAGES * (A_BYTES + BSTAGE) <= kRingBytes, "stage ring exceeds its budget");
   static_assert(STAGES <= kMaxStages, "too many stages");
   extern __shared__ uint8_t smem_raw[];
@@ -590,9 +601,9 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
   // at a pair's rank 1 only its gather threads (relayed to the leader).
   const int rank = PAIR ? (int)cluster_rank() : 0;
   const uint32_t full_arrivals =
-      (rank == 0 ? 1u : 0u) + (A_GATHER ? (uint32_t)kGatherThreads : 0u);
+      (rank == 0 ? 1u : 0u) + (A_GATHER ? (uint32_t)GTHREADS : 0u);
   setup<STAGES, 0, PAIR>(c, g.offsets, g.E, g.num_rows, g.err, full_arrivals > 0 ? full_arrivals : 1u,
-                         1, kGatherThreads / 32, nullptr);
+                         1, GTHREADS / 32, nullptr);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int first = PAIR ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
   const int stride = PAIR ? (int)(gridDim.x >> 1) : (int)gridDim.x;
@@ -648,12 +659,12 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
       }
     }
     __syncwarp();
-  } else if (A_GATHER && warp >= kGatherWarp0 && warp < kGatherWarp0 + kGatherThreads / 32) {
+  } else if (A_GATHER && warp >= kGatherWarp0 && warp < kGatherWarp0 + GTHREADS / 32) {
     // ---------------- row gather of the scattered A operand ----------------
     // thread t copies 16-byte chunk (t % 8) of tile rows t/8 + kRowStep j into
     // the 128-byte-swizzled K-major layout; rows past the expert's slice and
     // columns past K are zero-filled.
-    constexpr int kRowStep = kGatherThreads / 8, kRowsPer = BM / kRowStep;
+    constexpr int kRowStep = GTHREADS / 8, kRowsPer = BM / kRowStep;
     const int t = threadIdx.x - kGatherWarp0 * 32;
     const int cc = t & 7, r0 = t >> 3;
     const bf16* A = reinterpret_cast<const bf16*>(g.a);
@@ -753,7 +764,8 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
     }
     __syncwarp();
   } else if ((warp >= 4 && warp < 8) ||
-             (!A_GATHER && !SWIGLU_FWD && g.epi == EPI_STORE && warp >= 8 && warp < 12)) {
+             (!A_GATHER && !SWIGLU_FWD && g.epi == EPI_STORE && warp >= 8 && warp < 12) ||
+             (SHORTK && warp >= 12 && warp < 16)) {
     // warps 2-3 idle, and 8-15 without a gather except as below
     // ---------------- epilogue ----------------
     // Thread r owns accumulator row r.  Per 32-column chunk the warp stages its
@@ -771,11 +783,17 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
     // tiles drain at once (a short-K product's epilogue is longer than its MMAs).
     // A group stages in box `grp` of its quadrant's area; a warp whose rows leave
     // the slice stores them directly.
-    const bool two = !A_GATHER && !SWIGLU_FWD && g.epi == EPI_STORE;
+    // SHORTK: the same split of tiles by accumulator buffer for every epilogue, warps
+    // 12-15 with staging areas of their own (so ragged rows use their slots).
+    const bool shared_area = !A_GATHER && !SWIGLU_FWD && g.epi == EPI_STORE;
+    const bool two = shared_area || SHORTK;
     const int grp = warp >= 8 ? 1 : 0;
     const int q = warp & 3;  // tensor-memory lane quadrant
     const int r = q * 32 + lane;
-    uint8_t* wstage = smem + kRingBytes + kCtlBytes + q * kWarpStaging;
+    uint8_t* wstage = (SHORTK && grp == 1)
+                          ? smem + STAGES * (A_BYTES + BSTAGE) + q * kWarpStaging
+                          : smem + kRingBytes + kCtlBytes + q * kWarpStaging;
+    uint64_t* ebar = &c.ebar[grp * 4 + q];
     uint8_t* slot = wstage + lane * kSlotBytes;
     const uint32_t wstage_s = smem_u32(wstage), slot_s = smem_u32(slot);
     const int sw = (lane >> 1) & 3;  // 64-byte swizzle of this thread's box row
@@ -805,8 +823,8 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
       const uint32_t trow = c.tmem_base + ((uint32_t)(q * 32) << 16) + buf * BN;
       const int wrow0 = t.row0 + q * 32;
       const bool boxed = (box_flags & kBoxStores) && wrow0 + 32 <= t.row_end;  // warp-uniform
-      const bool direct = two && !boxed;  // warp-uniform: plain stores from registers
-      const int kb = two ? grp : 0;       // first box of this warp's outputs
+      const bool direct = shared_area && !boxed;  // warp-uniform: plain stores from registers
+      const int kb = shared_area ? grp : 0;       // first box of this warp's outputs
       // 16-byte chunk j8 of box k in this thread's row
       auto box_chunk = [&](int k, int j8) -> uint4* {
         return reinterpret_cast<uint4*>(wstage + k * kBoxBytes + lane * 64 + ((j8 ^ sw) << 4));
@@ -834,15 +852,15 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
           __syncwarp();
           if (lane == 0) {
             const uint32_t nbox = 1u + (need_h ? 1u : 0u) + (need_h && swi ? 1u : 0u);
-            mbar_expect_tx(&c.ebar[q], nbox * kBoxBytes);
-            tma_load_3d(wstage, &tmXa, &c.ebar[q], n0, 0, wrow0);
+            mbar_expect_tx(ebar, nbox * kBoxBytes);
+            tma_load_3d(wstage, &tmXa, ebar, n0, 0, wrow0);
             if (need_h) {
-              tma_load_3d(wstage + kBoxBytes, &tmXh, &c.ebar[q], n0, 0, wrow0);
-              if (swi) tma_load_3d(wstage + 2 * kBoxBytes, &tmXh, &c.ebar[q], n0, 1, wrow0);
+              tma_load_3d(wstage + kBoxBytes, &tmXh, ebar, n0, 0, wrow0);
+              if (swi) tma_load_3d(wstage + 2 * kBoxBytes, &tmXh, ebar, n0, 1, wrow0);
             }
           }
           tmem_ld32(trow + c0, v);
-          if (!mbar_wait(&c.ebar[q], eph, abort_flag, g.err)) break;
+          if (!mbar_wait(ebar, eph, abort_flag, g.err)) break;
           eph ^= 1;
 #pragma unroll
           for (int j8 = 0; j8 < 4; ++j8) {
@@ -1470,10 +1488,10 @@ struct EpiMaps {
 // 2-CTA clusters as the device can hold at once (fewer than half the SMs when a
 // GPC has an odd number of free SMs; a cluster beyond that would run its whole
 // share of the tile list after the others).
-template <bool AG, bool BK_, bool SW, bool SPLIT = false>
+template <bool AG, bool BK_, bool SW, bool SPLIT = false, bool SHORT = false>
 cudaError_t launch_g(const CUtensorMap& ta, const CUtensorMap& tb, const EpiMaps& m,
                      const GroupedGemm& g, int nN, long long tiles, cudaStream_t s) {
-  auto kern = grouped_gemm_tc_kernel<AG, BK_, SW, kPairM, SPLIT>;
+  auto kern = grouped_gemm_tc_kernel<AG, BK_, SW, kPairM, SPLIT, SHORT>;
   cudaError_t e = prep(kern, kGroupedSmem);
   if (e != cudaSuccess) return e;
   if (!kPairM) {
@@ -1590,6 +1608,14 @@ cudaError_t launch_grouped_gemm_tc(const GroupedGemm& g, cudaStream_t s) {
     return launch_g<false, false, false, true>(ta, tb, m, g, nN, tiles, s);
   }
 #define SMOE_LAUNCH_G(AG, KM, SW) launch_g<AG, KM, SW>(ta, tb, m, g, nN, tiles, s)
+  // A gathered product with a short K has little main loop per tile to hide its
+  // epilogue behind: half the gather warps become a second epilogue group.  Not for
+  // SwiGLU's forward, whose epilogue (half-width tiles) is short and whose gather
+  // then sets the pace (measured slower with 4 gather warps).
+  if (gather && !swiglu && !kPairM && g.K <= kShortK) {
+    if (kmaj) return launch_g<true, true, false, false, true>(ta, tb, m, g, nN, tiles, s);
+    return launch_g<true, false, false, false, true>(ta, tb, m, g, nN, tiles, s);
+  }
   if (gather) {
     if (kmaj) return swiglu ? SMOE_LAUNCH_G(true, true, true) : SMOE_LAUNCH_G(true, true, false);
     return swiglu ? SMOE_LAUNCH_G(true, false, true) : SMOE_LAUNCH_G(true, false, false);
