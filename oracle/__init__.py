@@ -170,6 +170,27 @@ def sort(topk_idx, E):
     return ss, off
 
 
+def route_bwd(x, w_r, topk_idx, gates, dgates):
+    """Router backward alone (R5): {"dl": [T,k], "dx": [T,d] (the router's share of
+    dx), "dw_r": [d,E], "db_r": [E]}, all fp64, for gate gradients ``dgates``."""
+    lib = _load()
+    xs, dt = _stored(x)
+    ws, dtw = _stored(w_r)
+    assert dt == dtw and dt in (0, 1, 2)
+    T, d = xs.shape
+    E = ws.shape[1]
+    idx = _i32(topk_idx)
+    k = idx.shape[1]
+    g = _f64(gates)
+    dg = _f64(dgates)
+    assert g.shape == (T, k) and dg.shape == (T, k)
+    out = {"dl": np.empty((T, k)), "dx": np.empty((T, d)), "dw_r": np.empty((d, E)),
+           "db_r": np.empty(E)}
+    lib.oracle_route_bwd(_p(xs), _p(ws), dt, T, d, E, k, _p(idx), _p(g), _p(dg), _p(out["dl"]),
+                         _p(out["dx"]), _p(out["dw_r"]), _p(out["db_r"]))
+    return out
+
+
 def act(kind, z):
     """(value, derivative) of gelu(tanh) (kind 'gelu') or silu (kind 'silu')."""
     lib = _load()

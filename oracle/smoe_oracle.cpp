@@ -612,6 +612,43 @@ void oracle_mlp_dw_sampled(const void* x, int dtx, const void* w1, const void* w
                           gates, dy, cols1, n_c1, rows2, n_r2, dw1_cols, dw2_rows));
 }
 
+/* R5, the router part alone (what smoe_route_bwd computes): given the routing
+ * (idx, gates) and the gate gradients dg [T,k] (fp64), the logit gradients
+ * dl [T,k] of the selected experts through the renormalised softmax, then
+ *   dx_r[t,i]  = sum_j dl[t,j] W_r[i, idx[t,j]]        (the router's share of dx)
+ *   dw_r[i,e]  = sum over slots (t,j) with idx = e of x[t,i] dl[t,j]
+ *   db_r[e]    = sum over the same slots of dl[t,j]
+ * Slots are taken in ascending order.  dx_r [T,d], dw_r [d,E], db_r [E], dl [T,k]. */
+void oracle_route_bwd(const void* x, const void* w_r, int dt, int T, int d, int E, int k,
+                      const int32_t* idx, const double* gates, const double* dg, double* dl,
+                      double* dx_r, double* dw_r, double* db_r) {
+#pragma omp parallel for schedule(static)
+  for (int t = 0; t < T; ++t) {
+    router_dlogits(gates + (size_t)t * k, dg + (size_t)t * k, k, dl + (size_t)t * k);
+    double* dxt = dx_r + (size_t)t * d;
+    for (int i = 0; i < d; ++i) dxt[i] = 0.0;
+    for (int j = 0; j < k; ++j) {
+      const int e = idx[(size_t)t * k + j];
+      const double v = dl[(size_t)t * k + j];
+      for (int i = 0; i < d; ++i) dxt[i] += v * load_any(w_r, dt, (size_t)i * E + e);
+    }
+  }
+  /* one thread per expert column: each sums its slots in ascending order */
+#pragma omp parallel for schedule(dynamic, 1)
+  for (int e = 0; e < E; ++e) {
+    double b = 0.0;
+    for (int i = 0; i < d; ++i) dw_r[(size_t)i * E + e] = 0.0;
+    for (int p = 0; p < T * k; ++p) {
+      if (idx[p] != e) continue;
+      const int t = p / k;
+      const double v = dl[p];
+      b += v;
+      for (int i = 0; i < d; ++i) dw_r[(size_t)i * E + e] += load_any(x, dt, (size_t)t * d + i) * v;
+    }
+    db_r[e] = b;
+  }
+}
+
 /* R6 forward.  gates: fp64 per slot (nullable).  out_rows (nullable): the rows
  * of y to compute (grouped row, slot or token, by mode); y: [n_out, N].      */
 void oracle_pl_fwd(const void* x, int dtx, const void* w, int dtw, int K, int N, int E,

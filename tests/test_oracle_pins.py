@@ -311,6 +311,63 @@ def test_mlp_backward_finite_differences(act):
     assert np.max(np.abs(fd - an["dg"])) / np.max(np.abs(an["dg"])) < 1e-6
 
 
+def test_route_bwd_finite_differences():
+    """The router backward alone: L = sum_{t,j} dg[t,j] * g[t,j](x W_r + b), the gates
+    the softmax over each token's (fixed) selected logits.  Central differences of L
+    in x, W_r and b against the oracle's dx, dW_r and db; a repeated expert index
+    across tokens and an expert nobody picks are both present."""
+    T, d, E, k = 7, 9, 5, 3
+    g = torch.Generator().manual_seed(41)
+    x = torch.randn(T, d, generator=g, dtype=torch.float64)
+    w_r = torch.randn(d, E, generator=g, dtype=torch.float64)
+    b = torch.randn(E, generator=g, dtype=torch.float64)
+    b[E - 1] = -50.0  # never selected: its dW_r column and db entry are exactly zero
+    dg = torch.randn(T, k, generator=g, dtype=torch.float64).numpy()
+    idx = _route_with_margin(x, w_r, b, k, 1e-3)
+    gates = torch.softmax(torch.gather(x @ w_r + b, 1, torch.from_numpy(idx).long()), 1).numpy()
+    an = oracle.route_bwd(x, w_r, idx, gates, dg)
+
+    def loss(xv, wv, bv):
+        sel = torch.gather(xv @ wv + bv, 1, torch.from_numpy(idx).long())
+        return float((torch.softmax(sel, 1).numpy() * dg).sum())
+
+    h = 1e-6
+    params = {"x": x, "w_r": w_r, "b": b}
+    key_of = {"x": "dx", "w_r": "dw_r", "b": "db_r"}
+    for name, tensor in params.items():
+        flat = tensor.view(-1)
+        fd = np.zeros(tensor.numel())
+        for q in range(tensor.numel()):
+            old = float(flat[q])
+            flat[q] = old + h
+            lp = loss(x, w_r, b)
+            flat[q] = old - h
+            lm = loss(x, w_r, b)
+            flat[q] = old
+            fd[q] = (lp - lm) / (2 * h)
+        ref = an[key_of[name]].ravel()
+        assert np.max(np.abs(fd - ref)) / np.max(np.abs(ref)) < 1e-6, name
+    assert np.all(an["dw_r"][:, E - 1] == 0.0) and an["db_r"][E - 1] == 0.0
+    # the logit gradients of a token sum to zero (its gates sum to one)
+    assert np.max(np.abs(an["dl"].sum(1))) < 1e-12
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_route_bwd_agrees_with_the_mlp_backward(dtype):
+    """Fed the MLP backward's own gate gradients, the standalone router backward
+    gives the MLP's dW_r and db, and its dx is the MLP's dx minus the expert path."""
+    x, w_r, w1, w2, dy = _tiny_mlp(12, 40, 24, 16, 6, 2, "swiglu", dtype)
+    idx, gates = oracle.route(x, w_r, None, 2)
+    full = oracle.mlp_bwd_full(x, w_r, w1, w2, "swiglu", idx, gates, dy)
+    r = oracle.route_bwd(x, w_r, idx, gates, full["dg"])
+    np.testing.assert_allclose(r["dw_r"], full["dw_r"], rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(r["db_r"], full["db_r"], rtol=1e-12, atol=1e-13)
+    # the expert path alone: the MLP backward of a router whose weights are zero
+    # (dx_expert does not depend on W_r once idx and gates are fixed)
+    no_router = oracle.mlp_bwd_full(x, torch.zeros_like(w_r), w1, w2, "swiglu", idx, gates, dy)
+    np.testing.assert_allclose(r["dx"] + no_router["dx"], full["dx"], rtol=1e-11, atol=1e-12)
+
+
 def test_mlp_backward_token_subset_and_sampled_dw_agree_with_full():
     x, w_r, w1, w2, dy = _tiny_mlp(9, 30, 16, 12, 5, 2, "swiglu", torch.float32)
     idx, gates = oracle.route(x, w_r, None, 2)
