@@ -45,6 +45,13 @@
  *     tensor-memory-accelerator copies); every tensor start 16-byte aligned.
  *   - Several calls may run concurrently on different streams as long as they
  *     do not share workspaces or outputs.
+ *   - Size limits (checked on the host, SMOE_ERR_INVALID_ARG beyond them):
+ *       routed entry points (smoe_route, smoe_route_bwd, smoe_mlp_*):
+ *         1 <= k <= min(E, SMOE_MAX_TOPK), E <= SMOE_MAX_ROUTED_EXPERTS;
+ *       sort and ParallelLinear (smoe_sort, smoe_sort_static,
+ *         parallel_linear_*): E <= SMOE_MAX_EXPERTS;
+ *       everywhere: T * k (the slot count) <= INT32_MAX, and every [rows, cols]
+ *         tensor the call touches has fewer than 2^31 elements.
  */
 #ifndef SMOE_H_
 #define SMOE_H_
@@ -66,6 +73,10 @@ typedef enum {
 } smoe_status;
 
 typedef enum { SMOE_F32 = 0, SMOE_BF16 = 1 } smoe_dtype;
+
+#define SMOE_MAX_ROUTED_EXPERTS 128 /* E for the router and the MLP */
+#define SMOE_MAX_TOPK 16            /* k for the router and the MLP */
+#define SMOE_MAX_EXPERTS 1024       /* E for the sort and ParallelLinear */
 
 typedef enum {
   SMOE_ACT_GELU_TANH = 0, /* a = 0.5 h (1 + tanh(sqrt(2/pi) (h + 0.044715 h^3))) */
@@ -117,7 +128,7 @@ size_t smoe_workspace_size(int op, int T, int k, int E, int d, int f, smoe_dtype
  * selected logits (this equals softmax over all E, top-k, renormalise).
  *   x        [T, d] dtype          w_r [d, E] dtype        b_r [E] fp32 or NULL
  *   topk_idx [T, k] int32 (out)    gates [T, k] fp32 (out)
- * Requires 1 <= k <= E <= 256, k <= 16, d % 8 == 0.
+ * Requires 1 <= k <= min(E, 16), E <= 128, d % 8 == 0.
  * ------------------------------------------------------------------------ */
 int smoe_route(const void* x, const void* w_r, const float* b_r, int T, int d, int E, int k,
                smoe_dtype dt, int32_t* topk_idx, float* gates, void* stream);
@@ -132,7 +143,8 @@ int smoe_route(const void* x, const void* w_r, const float* b_r, int T, int d, i
  *   dx[t,i]  += sum_j dl[t,j] W_r[i, topk_idx[t,j]]  (dtype, accumulated into dx;
  *                                                     NULL to skip)
  * workspace: smoe_workspace_size(SMOE_OP_ROUTE_BWD, ...) bytes (no more than the
- * SMOE_OP_MLP_BWD size of the same shape).                                    */
+ * SMOE_OP_MLP_BWD size of the same shape).
+ * Requires 1 <= k <= min(E, 16), E <= 128, d % 8 == 0 (as smoe_route).       */
 int smoe_route_bwd(const void* x, const void* w_r, const int32_t* topk_idx, const float* gates,
                    const float* dgates, int T, int d, int E, int k, smoe_dtype dt, void* dx,
                    float* dw_r, float* db_r, void* workspace, size_t ws_bytes, void* stream);
@@ -145,7 +157,7 @@ int smoe_route_bwd(const void* x, const void* w_r, const int32_t* topk_idx, cons
  *   topk_idx [T, k] int32   sorted_slot [T*k] int32 (out)
  *   expert_offsets [E+1] int32 (out; offsets[0] = 0, offsets[E] = T*k)
  * Ids outside [0, E) are reported through smoe_check (SMOE_ERR_DATA) and their
- * slots are left out (the outputs are then incomplete).
+ * slots are left out (the outputs are then incomplete).  Requires 1 <= E <= 1024.
  * ------------------------------------------------------------------------ */
 int smoe_sort(const int32_t* topk_idx, int T, int k, int E, int32_t* sorted_slot,
               int32_t* expert_offsets, void* workspace, size_t ws_bytes, void* stream);
@@ -163,6 +175,9 @@ int smoe_sort(const int32_t* topk_idx, int T, int k, int E, int32_t* sorted_slot
  *   rejected with SMOE_ERR_INVALID_ARG and a message (use smoe_sort).
  *   The first call on a device looks up the array's device address with that
  *   device current; make that first call before any stream capture begins.
+ *   The address is kept for the life of the process, so the library must not
+ *   be used across a cudaDeviceReset (or any other teardown of the device's
+ *   primary context) that unloads and reloads its module.
  *   Every call rewrites all the counts it uses, so nothing has to be cleared
  *   between calls; but all calls share the one array, so calls whose work
  *   overlaps on the GPU (different streams without ordering) race and give
@@ -197,9 +212,10 @@ int smoe_selftest_wait_timeout(int limit_us, void* stream);
  *                                      order (combine_k > 0, scattered only;
  *                                      y [num_slots / combine_k, N])
  * No grouped or padded copy of a scattered input is made.  The k-way combine is
- * deterministic (no atomics): each slot's (gated) v is rounded to dtype, as the
- * library materialises per-slot outputs, and the combine_k values are summed in fp32.
- *   x [x_rows, K] dtype, w [E, K, N] dtype, y dtype.
+ * deterministic (no atomics): this library rounds each slot's (gated) v to dtype
+ * (its own choice: the pages do not say how per-slot outputs are held), then sums
+ * the combine_k values in fp32 in slot order.
+ *   x [x_rows, K] dtype, w [E, K, N] dtype, y dtype.  Requires 1 <= E <= 1024.
  * ------------------------------------------------------------------------ */
 size_t parallel_linear_fwd_workspace_size(int num_slots, int K, int N, int E, int combine_k,
                                           smoe_dtype dt);

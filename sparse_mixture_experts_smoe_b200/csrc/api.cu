@@ -7,7 +7,8 @@
 // summary: group-to-group, group-to-scatter, scatter-to-scatter, scatter-to-group)
 // maps onto one grouped-M GEMM whose A rows are read grouped or gathered through
 // sorted_slot and whose output rows are written grouped or scattered; a k-way
-// combine goes through an fp32 slot-ordered buffer and a fixed-order sum.  The
+// combine goes through a grouped-order buffer of gated slot rows in the layer's
+// dtype and a fixed-order fp32 sum per token.  The
 // backward (tradepoint.io article, method paragraphs: the gradient of each
 // expert) swaps the roles of the row maps for dx and runs a per-expert dW GEMM.
 #include <cstdarg>
@@ -118,6 +119,8 @@ unsigned* error_word(cudaError_t* status) {
 }
 
 bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+// The slot count T*k (and every slot index) fits an int32.
+bool slots_fit(int T, int k) { return (long long)T * k <= 0x7fffffffLL; }
 size_t align256(size_t n) { return (n + 255) & ~(size_t)255; }
 size_t esize(smoe_dtype dt) { return dt == SMOE_BF16 ? 2 : 4; }
 bool valid_dtype(int dt) { return dt == SMOE_F32 || dt == SMOE_BF16; }
@@ -271,8 +274,9 @@ int validate_mlp_desc(const smoe_mlp_desc* m) {
   if (!m) return fail(SMOE_ERR_INVALID_ARG, "desc is NULL");
   if (m->T < 0 || m->d <= 0 || m->f <= 0 || m->E <= 0 || m->k <= 0)
     return fail(SMOE_ERR_INVALID_ARG, "bad sizes T=%d d=%d f=%d E=%d k=%d", m->T, m->d, m->f, m->E, m->k);
-  if (m->k > m->E || m->k > 16 || m->E > 128)
-    return fail(SMOE_ERR_INVALID_ARG, "need 1 <= k <= min(E, 16) and E <= 128 (k=%d E=%d)", m->k, m->E);
+  if (m->k > m->E || m->k > SMOE_MAX_TOPK || m->E > SMOE_MAX_ROUTED_EXPERTS)
+    return fail(SMOE_ERR_INVALID_ARG, "need 1 <= k <= min(E, %d) and E <= %d (k=%d E=%d)",
+                SMOE_MAX_TOPK, SMOE_MAX_ROUTED_EXPERTS, m->k, m->E);
   if (m->d % 8 || m->f % 8) return fail(SMOE_ERR_INVALID_ARG, "d and f must be multiples of 8");
   if (!valid_dtype(m->dtype)) return fail(SMOE_ERR_INVALID_ARG, "bad dtype %d", m->dtype);
   if (m->act != SMOE_ACT_GELU_TANH && m->act != SMOE_ACT_SWIGLU)
@@ -371,7 +375,7 @@ int smoe_profile_entry(int i, const char** name, int* launches, double* total_ms
 }
 
 size_t smoe_workspace_size(int op, int T, int k, int E, int d, int f, smoe_dtype dt) {
-  if (T < 0 || k <= 0 || E <= 0 || d <= 0 || f <= 0) return 0;
+  if (T < 0 || k <= 0 || E <= 0 || d <= 0 || f <= 0 || !slots_fit(T, k)) return 0;
   const int S = T * k;
   const int wide = (d > 2 * f ? d : 2 * f);
   switch (op) {
@@ -393,8 +397,12 @@ int smoe_route(const void* x, const void* w_r, const float* b_r, int T, int d, i
                smoe_dtype dt, int32_t* topk_idx, float* gates, void* stream) {
   smoe::NvtxScope nvtx_scope("smoe_route");
   if (T < 0 || d <= 0 || E <= 0 || k <= 0) return fail(SMOE_ERR_INVALID_ARG, "bad sizes");
-  if (k > E || k > 16 || E > 128) return fail(SMOE_ERR_INVALID_ARG, "need 1 <= k <= min(E,16), E <= 128");
+  if (k > E || k > SMOE_MAX_TOPK || E > SMOE_MAX_ROUTED_EXPERTS)
+    return fail(SMOE_ERR_INVALID_ARG, "need 1 <= k <= min(E, %d), E <= %d", SMOE_MAX_TOPK,
+                SMOE_MAX_ROUTED_EXPERTS);
   if (d % 8) return fail(SMOE_ERR_INVALID_ARG, "d must be a multiple of 8");
+  if (!slots_fit(T, k) || (long long)T * d >= (1LL << 31))
+    return fail(SMOE_ERR_INVALID_ARG, "T*k or T*d too large for 32-bit indexing");
   if (!valid_dtype(dt)) return fail(SMOE_ERR_INVALID_ARG, "bad dtype");
   if (T == 0) return SMOE_OK;
   NEED(x, "x"); NEED(w_r, "w_r"); NEED(topk_idx, "topk_idx"); NEED(gates, "gates");
@@ -412,9 +420,13 @@ int smoe_route_bwd(const void* x, const void* w_r, const int32_t* topk_idx, cons
                    const float* dgates, int T, int d, int E, int k, smoe_dtype dt, void* dx,
                    float* dw_r, float* db_r, void* workspace, size_t ws_bytes, void* stream) {
   smoe::NvtxScope nvtx_scope("smoe_route_bwd");
-  if (T < 0 || d <= 0 || E <= 0 || k <= 0 || k > E || E > 128)
-    return fail(SMOE_ERR_INVALID_ARG, "bad sizes");
+  if (T < 0 || d <= 0 || E <= 0 || k <= 0 || k > E || k > SMOE_MAX_TOPK ||
+      E > SMOE_MAX_ROUTED_EXPERTS)
+    return fail(SMOE_ERR_INVALID_ARG, "bad sizes (need 1 <= k <= min(E, %d), E <= %d)",
+                SMOE_MAX_TOPK, SMOE_MAX_ROUTED_EXPERTS);
   if (d % 8) return fail(SMOE_ERR_INVALID_ARG, "d must be a multiple of 8");
+  if (!slots_fit(T, k) || (long long)T * d >= (1LL << 31))
+    return fail(SMOE_ERR_INVALID_ARG, "T*k or T*d too large for 32-bit indexing");
   if (!valid_dtype(dt)) return fail(SMOE_ERR_INVALID_ARG, "bad dtype");
   NEED(x, "x"); NEED(w_r, "w_r"); NEED(topk_idx, "topk_idx"); NEED(gates, "gates");
   NEED(dgates, "dgates"); NEED(dw_r, "dw_r");
@@ -442,7 +454,9 @@ int smoe_route_bwd(const void* x, const void* w_r, const int32_t* topk_idx, cons
 int smoe_sort(const int32_t* topk_idx, int T, int k, int E, int32_t* sorted_slot,
               int32_t* expert_offsets, void* workspace, size_t ws_bytes, void* stream) {
   smoe::NvtxScope nvtx_scope("smoe_sort");
-  if (T < 0 || k <= 0 || E <= 0 || E > 1024) return fail(SMOE_ERR_INVALID_ARG, "bad sizes (E <= 1024)");
+  if (T < 0 || k <= 0 || E <= 0 || E > SMOE_MAX_EXPERTS)
+    return fail(SMOE_ERR_INVALID_ARG, "bad sizes (E <= %d)", SMOE_MAX_EXPERTS);
+  if (!slots_fit(T, k)) return fail(SMOE_ERR_INVALID_ARG, "T*k too large for 32-bit indexing");
   NEED(expert_offsets, "expert_offsets");
   cudaStream_t s = (cudaStream_t)stream;
   if (T == 0) {
@@ -468,6 +482,7 @@ static int validate_pl(const void* x, int x_rows, int K, const void* w, int N, i
                        int fan_out, int grouped_in, int grouped_out, int combine_k, int dt) {
   if (num_slots < 0 || x_rows < 0 || K <= 0 || N <= 0 || E <= 0)
     return fail(SMOE_ERR_INVALID_ARG, "bad sizes");
+  if (E > SMOE_MAX_EXPERTS) return fail(SMOE_ERR_INVALID_ARG, "E <= %d", SMOE_MAX_EXPERTS);
   if (K % 8 || N % 8) return fail(SMOE_ERR_INVALID_ARG, "K and N must be multiples of 8");
   if (!valid_dtype(dt)) return fail(SMOE_ERR_INVALID_ARG, "bad dtype");
   if (fan_out < 1 || combine_k < 0) return fail(SMOE_ERR_INVALID_ARG, "fan_out >= 1, combine_k >= 0");
@@ -477,7 +492,8 @@ static int validate_pl(const void* x, int x_rows, int K, const void* w, int N, i
     return fail(SMOE_ERR_INVALID_ARG, "grouped input needs x_rows == num_slots");
   if (!grouped_in && (long long)x_rows * fan_out < num_slots)
     return fail(SMOE_ERR_INVALID_ARG, "x_rows * fan_out < num_slots");
-  if ((long long)num_slots * (K > N ? K : N) >= (1LL << 31))
+  if ((long long)num_slots * (K > N ? K : N) >= (1LL << 31) ||
+      (long long)x_rows * K >= (1LL << 31))
     return fail(SMOE_ERR_INVALID_ARG, "tensor too large for 32-bit row indexing");
   if (num_slots == 0) return SMOE_OK;
   NEED(x, "x"); NEED(w, "w"); NEED(sorted_slot, "sorted_slot"); NEED(offsets, "expert_offsets");

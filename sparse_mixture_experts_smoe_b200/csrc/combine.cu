@@ -1,15 +1,16 @@
 // combine.cu -- bandwidth-bound helpers around the grouped GEMMs:
-//   * the deterministic k-way combine of a slot-ordered fp32 buffer into token rows
-//     (optionally adding the router's term dl W_r^T of the backward),
+//   * the deterministic k-way combine of a grouped-order buffer of gated slot rows
+//     (in the layer's dtype) into token rows, summed in fp32 (optionally adding the
+//     router's term dl W_r^T of the backward),
 //   * the fixed-order reduction of per-column-tile gate-gradient partials,
 //   * a gated gather of rows into grouped order.
 //
 // The k slots of a token are owned by k different experts, so their products
 // come from different CTAs; summing them with atomics would make the result
 // depend on scheduling.  Instead the GEMM epilogue stores each slot's row, already
-// multiplied by its gate, in a buffer of the layer's dtype (the slot outputs are
-// materialised in the compute type before the gate-weighted sum, as the library
-// does it), in grouped order (row i of slot p = sorted_slot[i], so that whole warps
+// multiplied by its gate, in a buffer of the layer's dtype (this library's choice:
+// the pages do not say in what precision per-slot outputs are held before the
+// gate-weighted sum), in grouped order (row i of slot p = sorted_slot[i], so that whole warps
 // of rows leave as TMA boxes); this pass sums the k rows of each token in fp32 in
 // ascending j, finding slot p's row through the inverse permutation inv[p] = i
 // (group-to-scatter with combine, library page of arXiv 2403.08245, review 2

@@ -260,6 +260,8 @@ extern "C" int smoe_sort_static(const int32_t* topk_idx, int T, int k, int E,
   using namespace smoe;
   if (T < 0 || k <= 0 || E <= 0 || E > kSortMaxE)
     return api_fail(SMOE_ERR_INVALID_ARG, "bad sizes (E <= %d)", kSortMaxE);
+  if ((long long)T * k > 0x7fffffffLL)
+    return api_fail(SMOE_ERR_INVALID_ARG, "T*k too large for 32-bit indexing");
   if (!expert_offsets) return api_fail(SMOE_ERR_INVALID_ARG, "expert_offsets is NULL");
   const size_t need = sort_workspace_bytes(T, k, E);
   if (need > sizeof(g_sort_static_counts))

@@ -15,6 +15,7 @@ deviation, then rounded to the storage dtype (bf16 round-to-nearest-even).
   W1 ~ N(0, 1/d)          [E, d, m*f]      (m = 2 for SwiGLU: gate | up columns)
   W2 ~ N(0, 1/f)          [E, f, d]
   dY ~ N(0, 1)            [T, d]           (upstream gradient)
+  dgates ~ N(0, 1)        [T, k] fp32      (router backward on its own)
   b_r                     [E] fp32, zero except the skewed workload (below)
 
 Skewed workload: experts get ranks r = 1..E from a seeded permutation;
@@ -44,7 +45,7 @@ WORKLOADS = {
 }
 
 _STREAM = {"x": 1, "w_r": 2, "w1": 3, "w2": 4, "dy": 5, "perm": 6, "wq": 7, "wo": 8, "o": 9,
-           "dz": 10, "dq": 11}
+           "dz": 10, "dq": 11, "dg": 12}
 
 
 def torch_dtype(name: str) -> torch.dtype:
@@ -90,6 +91,22 @@ def make_mlp_inputs(cfg: dict, seed: int = 0, device="cpu", with_dy: bool = True
         out["b_r"] = None
     if with_dy:
         out["dy"] = _randn((T, d), 1.0, "dy", seed, device, dt)
+    return out
+
+
+def make_router_inputs(cfg: dict, seed: int = 0, device="cpu") -> dict:
+    """Router-only inputs of a workload: x, W_r and b_r as in ``make_mlp_inputs``
+    (same streams, so the same values), plus upstream gate gradients
+    dgates ~ N(0, 1) [T, k] in fp32 for the router backward on its own."""
+    T, d, E, k = cfg["T"], cfg["d"], cfg["E"], cfg["k"]
+    dt = torch_dtype(cfg["dtype"])
+    out = {
+        "x": _randn((T, d), 1.0, "x", seed, device, dt),
+        "w_r": _randn((d, E), 1.0 / math.sqrt(d), "w_r", seed, device, dt),
+        "b_r": (zipf_bias(E, cfg["zipf_s"], cfg["n_empty"], seed).to(device)
+                if "zipf_s" in cfg else None),
+        "dgates": _randn((T, k), 1.0, "dg", seed, device, torch.float32),
+    }
     return out
 
 

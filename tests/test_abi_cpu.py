@@ -171,3 +171,52 @@ def test_decode_workspace_holds_the_split_k_partials():
         sort = L.smoe_workspace_size(0, T, k, E, d, f, 1)
         part = a256(splits * S * d * 4) if splits > 1 else 0
         assert fwd == a256(sort) + a256(S * 4) + a256(S * d * 2) + part
+
+
+def test_limits_are_stated_and_enforced_per_entry_point():
+    """Each entry point's size limit (smoe.h): the largest allowed value passes host
+    validation (T == 0, so nothing runs), the next one is refused before any launch."""
+    L = smoe.lib()
+    hdr = open(os.path.join(ROOT, "include", "smoe.h")).read()
+    lim = {n: int(re.search(r"#define %s (\d+)" % n, hdr).group(1))
+           for n in ("SMOE_MAX_ROUTED_EXPERTS", "SMOE_MAX_TOPK", "SMOE_MAX_EXPERTS")}
+    Er, Kmax, Emax = lim["SMOE_MAX_ROUTED_EXPERTS"], lim["SMOE_MAX_TOPK"], lim["SMOE_MAX_EXPERTS"]
+    # router: E and k
+    assert L.smoe_route(None, None, None, 0, 8, Er, Kmax, 1, None, None, None) == 0
+    assert L.smoe_route(None, None, None, 0, 8, Er + 1, 2, 1, None, None, None) == -1
+    assert L.smoe_route(None, None, None, 0, 8, Er, Kmax + 1, 1, None, None, None) == -1
+    # router backward: same limits (T == 0 with valid sizes only zeroes the outputs,
+    # which needs a device, so the boundary is checked on the refusals)
+    args = (FAKE, FAKE, FAKE, FAKE, FAKE, 4, 8)
+    assert L.smoe_route_bwd(*args, Er + 1, 2, 1, None, FAKE, None, FAKE, 1 << 20, None) == -1
+    assert L.smoe_route_bwd(*args, Er, Kmax + 1, 1, None, FAKE, None, FAKE, 1 << 20, None) == -1
+    # the MLP: E and k, through its workspace query (0 = refused)
+    ok = smoe.MlpDesc(16, 64, 64, Er, Kmax, 1, 1)
+    assert L.smoe_mlp_workspace_size(ctypes.byref(ok), 1) > 0
+    for bad in (smoe.MlpDesc(16, 64, 64, Er + 1, 2, 1, 1), smoe.MlpDesc(16, 64, 64, Er, Kmax + 1, 1, 1)):
+        assert L.smoe_mlp_workspace_size(ctypes.byref(bad), 1) == 0
+        assert L.smoe_mlp_fwd(ctypes.byref(bad), ctypes.byref(smoe.MlpTensors()), None) == -1
+    # sort and the allocation-free sort: E
+    assert L.smoe_sort(FAKE, 4, 2, Emax + 1, FAKE, FAKE, FAKE, 1 << 20, None) == -1
+    assert L.smoe_sort_static(FAKE, 4, 2, Emax + 1, FAKE, FAKE, None) == -1
+    assert L.smoe_sort(FAKE, 4, 2, Emax, FAKE, FAKE, None, 0, None) == -1  # passes E, fails on ws
+    assert b"workspace" in L.smoe_last_error()
+    # ParallelLinear: E (the empty problem with E at the limit is a no-op)
+    pl = lambda E, S: L.parallel_linear_fwd(FAKE, S, 16, FAKE, 16, E, FAKE, FAKE, S, 1, 1, 1,  # noqa: E731
+                                            None, 0, FAKE, 1, None, 0, None)
+    assert pl(Emax, 0) == 0
+    assert pl(Emax + 1, 0) == -1
+
+
+def test_slot_count_overflow_is_refused():
+    """T*k beyond int32 is refused on the host by every entry point that takes T and k."""
+    L = smoe.lib()
+    T, k = (1 << 30), 4
+    assert L.smoe_route(FAKE, FAKE, None, T, 8, 8, k, 1, FAKE, FAKE, None) == -1
+    assert L.smoe_sort(FAKE, T, k, 8, FAKE, FAKE, FAKE, 1 << 20, None) == -1
+    assert L.smoe_sort_static(FAKE, T, k, 8, FAKE, FAKE, None) == -1
+    assert L.smoe_route_bwd(FAKE, FAKE, FAKE, FAKE, FAKE, T, 8, 8, k, 1, None, FAKE, None, FAKE,
+                            1 << 20, None) == -1
+    assert L.smoe_workspace_size(0, T, k, 8, 8, 8, 1) == 0
+    d = smoe.MlpDesc(T, 64, 64, 8, k, 1, 1)
+    assert L.smoe_mlp_workspace_size(ctypes.byref(d), 0) == 0
