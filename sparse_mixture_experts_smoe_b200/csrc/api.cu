@@ -12,6 +12,7 @@
 // backward (tradepoint.io article, method paragraphs: the gradient of each
 // expert) swaps the roles of the row maps for dx and runs a per-expert dW GEMM.
 #include <cstdarg>
+#include <cstdlib>
 #include <cstdio>
 #include <cstring>
 #include <map>
@@ -177,12 +178,13 @@ struct PLBwdWs {
   void* dx_comb = nullptr;   // [num_slots, K] dtype when dx needs a fan-out combine (grouped order)
   int32_t* inv = nullptr;    // [num_slots] grouped row of each slot, with dx_comb
   float* dg_part = nullptr;  // [num_slots, dg_ld]
-  void* gx = nullptr;        // [num_slots, K] dtype: gates * x rows, grouped
   int dg_ld = 0;
   size_t bytes = 0;
 };
+// No term here holds x: with gates, dW's gate multiplies x's rows inside the dW
+// kernel as they are gathered.
 PLBwdWs pl_bwd_layout(void* ws, int num_slots, int K, int grouped_in, int fan_out, int has_gates,
-                      int want_dx, int want_dw, int want_dg, smoe_dtype dt) {
+                      int want_dx, int want_dg, smoe_dtype dt) {
   Carve c(ws);
   PLBwdWs l;
   if (want_dx && !grouped_in && fan_out > 1) {
@@ -193,7 +195,6 @@ PLBwdWs pl_bwd_layout(void* ws, int num_slots, int K, int grouped_in, int fan_ou
     l.dg_ld = cdiv(K, act_tile_cols(dt));
     l.dg_part = (float*)c.take((size_t)num_slots * l.dg_ld * sizeof(float));
   }
-  if (has_gates && want_dw) l.gx = c.take((size_t)num_slots * K * esize(dt));
   l.bytes = c.off;
   return l;
 }
@@ -232,7 +233,7 @@ struct MlpWs {
   int ksplit = 1;
   float* dg_part = nullptr; // bwd: [S, dg_ld]
   void* dh = nullptr;       // bwd: [S, m*f] dtype (grouped dH)
-  void* ga = nullptr;       // bwd: [S, f] dtype (gates * A)
+  void* ga = nullptr;       // bwd: [S, f] dtype (gates * A), only when dW2 reads a gated copy
   void* dxcomb = nullptr;   // bwd: [S, d] slot rows (dtype), grouped order
   int32_t* inv = nullptr;   // fwd and bwd: [S] grouped row of each slot
   float* dl = nullptr;      // bwd: [T, k]
@@ -242,6 +243,18 @@ struct MlpWs {
   int dg_ld = 0, r_runs = 0;
   size_t bytes = 0;
 };
+// dW2 = sum_i (g A_i)^T dY_t: the gate either multiplies dY's gathered rows inside
+// the dW kernel (default) or A in the dA' epilogue, which then writes g*A
+// (SMOE_MLP_GA=1 in the environment; read once).
+bool mlp_dw2_reads_ga() {
+  static int v = -1;
+  if (v < 0) {
+    const char* env = getenv("SMOE_MLP_GA");
+    v = (env != nullptr && env[0] == '1') ? 1 : 0;
+  }
+  return v == 1;
+}
+
 MlpWs mlp_layout(void* ws, const smoe_mlp_desc& m, int backward) {
   Carve c(ws);
   MlpWs l;
@@ -258,7 +271,7 @@ MlpWs mlp_layout(void* ws, const smoe_mlp_desc& m, int backward) {
     l.dg_ld = cdiv(m.f, act_tile_cols(dt));
     l.dg_part = (float*)c.take(S * l.dg_ld * sizeof(float));
     l.dh = c.take(S * (size_t)(m.act == SMOE_ACT_SWIGLU ? 2 * m.f : m.f) * esize(dt));
-    l.ga = c.take(S * m.f * esize(dt));
+    if (mlp_dw2_reads_ga()) l.ga = c.take(S * m.f * esize(dt));
     l.dxcomb = c.take(S * m.d * esize(dt));
     l.dl = (float*)c.take(S * sizeof(float));
     l.dg = (float*)c.take(S * sizeof(float));
@@ -381,7 +394,7 @@ size_t smoe_workspace_size(int op, int T, int k, int E, int d, int f, smoe_dtype
   switch (op) {
     case SMOE_OP_SORT: return sort_workspace_bytes(T, k, E);
     case SMOE_OP_PL_FWD: return pl_fwd_layout(nullptr, S, wide, k, dt).bytes;
-    case SMOE_OP_PL_BWD: return pl_bwd_layout(nullptr, S, wide, 0, k, 1, 1, 1, 1, dt).bytes;
+    case SMOE_OP_PL_BWD: return pl_bwd_layout(nullptr, S, wide, 0, k, 1, 1, 1, dt).bytes;
     case SMOE_OP_ROUTE_BWD: return route_bwd_layout(nullptr, T, d, E, k).bytes;
     case SMOE_OP_MLP_FWD:
     case SMOE_OP_MLP_BWD: {
@@ -554,7 +567,7 @@ size_t parallel_linear_bwd_workspace_size(int x_rows, int num_slots, int K, int 
                                           int has_gates, int combine_k, smoe_dtype dt) {
   (void)x_rows; (void)N; (void)E; (void)grouped_out; (void)combine_k;
   if (num_slots <= 0 || K <= 0) return 0;
-  return pl_bwd_layout(nullptr, num_slots, K, grouped_in, fan_out, has_gates, 1, 1, 1, dt).bytes;
+  return pl_bwd_layout(nullptr, num_slots, K, grouped_in, fan_out, has_gates, 1, 1, dt).bytes;
 }
 
 int parallel_linear_bwd(const void* dy, const void* x, const void* w, int x_rows, int K, int N,
@@ -577,7 +590,7 @@ int parallel_linear_bwd(const void* dy, const void* x, const void* w, int x_rows
   if (dx) ALIGNED(dx, "dx");
   const int has_g = gates != nullptr;
   PLBwdWs l = pl_bwd_layout(workspace, num_slots, K, grouped_in, fan_out, has_g, dx != nullptr,
-                            dw != nullptr, dgates != nullptr, dt);
+                            dgates != nullptr, dt);
   if (l.bytes > 0 && (!workspace || ws_bytes < l.bytes))
     return fail(SMOE_ERR_INVALID_ARG, "workspace too small (%zu < %zu)", ws_bytes, l.bytes);
   if ((rc = check_tc(dt)) != SMOE_OK) return rc;
@@ -603,10 +616,10 @@ int parallel_linear_bwd(const void* dy, const void* x, const void* w, int x_rows
     g.out_mode = grouped_in ? ROWS_GROUPED : ROWS_GATHER;
     if (dx_comb) { g.out_mode = ROWS_GROUPED; g.out = l.dx_comb; g.ldo = K; g.out_f32 = dt == SMOE_F32; }
     else { g.out = dx; g.ldo = K; g.out_f32 = dt == SMOE_F32; }
-    if (has_g) {
+    if (has_g) {  // dx rows g * dA'; gate-gradient partials <dA', x row>
       g.epi = EPI_ACT_BWD; g.act = SMOE_ACT_NONE;
       g.aux_a = x; g.ld_aux_a = K; g.aux_a_mode = x_mode; g.aux_a_fan_out = fan_out;
-      g.out2 = dw ? l.gx : nullptr; g.ldo2 = K;
+      g.out2 = nullptr;
       g.dg_partial = l.dg_part; g.dg_ld = l.dg_ld;
       if (!dgates) { g.dg_partial = nullptr; }
     } else {
@@ -627,19 +640,14 @@ int parallel_linear_bwd(const void* dy, const void* x, const void* w, int x_rows
                               nullptr, 0, s), "parallel_linear_bwd dx combine");
     }
   }
-  if (dw) {
-    if (has_g && !need_gemm) {
-      PROF("pl.gather", 1);
-      SMOE_TRY(launch_gather_scale(x, K, x_mode, fan_out, sorted_slot, gates, num_slots, K, l.gx,
-                                   dt, s), "parallel_linear_bwd gather");
-    }
+  if (dw) {  // dW[e] = sum_i (g x_row(i))^T G_i: the gate is applied inside the dW kernel
     DwGemm g;
     g.E = E; g.num_rows = num_slots; g.offsets = expert_offsets; g.sorted_slot = sorted_slot;
     g.M = K; g.N = N;
-    if (has_g) { g.a = l.gx; g.lda = K; g.a_mode = ROWS_GROUPED; g.a_fan_out = 1; g.a_rows = num_slots; }
-    else { g.a = x; g.lda = K; g.a_mode = x_mode; g.a_fan_out = fan_out; g.a_rows = x_rows; }
+    g.a = x; g.lda = K; g.a_mode = x_mode; g.a_fan_out = fan_out; g.a_rows = x_rows;
     g.b = dy; g.ldb = N; g.b_mode = g_mode; g.b_fan_out = g_fan;
     g.b_rows = combine_k > 0 ? num_slots / combine_k : num_slots;
+    g.row_gates = gates;
     g.dw = dw; g.err = err;
     { PROF("pl.gemm_dw", 1); SMOE_TRY(run_dw(g, dt, s), "parallel_linear_bwd dw gemm"); }
   }
@@ -752,7 +760,7 @@ int smoe_mlp_bwd(const smoe_mlp_desc* desc, const smoe_mlp_tensors* t, void* str
     g.aux_a = t->a; g.ld_aux_a = m.f; g.aux_a_mode = ROWS_GROUPED; g.aux_a_fan_out = 1;
     g.aux_h = t->h; g.ld_aux_h = mf;
     g.out_mode = ROWS_GROUPED; g.out = l.dh; g.ldo = mf; g.out_f32 = dt == SMOE_F32;
-    g.out2 = l.ga; g.ldo2 = m.f;
+    g.out2 = l.ga; g.ldo2 = m.f;  // null unless dW2 reads a gated copy of A
     g.dg_partial = l.dg_part; g.dg_ld = l.dg_ld; g.err = err;
     { PROF("gemm.bwd_dA", 1); SMOE_TRY(run_grouped(g, dt, s), "mlp bwd gemm dA"); }
   }
@@ -762,7 +770,13 @@ int smoe_mlp_bwd(const smoe_mlp_desc* desc, const smoe_mlp_tensors* t, void* str
     DwGemm g;
     g.E = m.E; g.num_rows = S; g.offsets = t->expert_offsets; g.sorted_slot = t->sorted_slot;
     g.M = m.f; g.N = m.d;
-    g.a = l.ga; g.lda = m.f; g.a_rows = S; g.a_mode = ROWS_GROUPED; g.a_fan_out = 1;
+    if (l.ga) {
+      g.a = l.ga;
+    } else {
+      g.a = t->a;
+      g.row_gates = t->gates;
+    }
+    g.lda = m.f; g.a_rows = S; g.a_mode = ROWS_GROUPED; g.a_fan_out = 1;
     g.b = t->dy; g.ldb = m.d; g.b_rows = m.T; g.b_mode = ROWS_GATHER; g.b_fan_out = m.k;
     g.dw = t->dw2; g.err = err;
     { PROF("gemm.bwd_dW2", 1); SMOE_TRY(run_dw(g, dt, s), "mlp bwd dW2"); }

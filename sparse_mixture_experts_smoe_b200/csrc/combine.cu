@@ -3,7 +3,7 @@
 //     (in the layer's dtype) into token rows, summed in fp32 (optionally adding the
 //     router's term dl W_r^T of the backward),
 //   * the fixed-order reduction of per-column-tile gate-gradient partials,
-//   * a gated gather of rows into grouped order.
+//   * the fixed-order reduction of split-K partials (decode-sized batches).
 //
 // The k slots of a token are owned by k different experts, so their products
 // come from different CTAs; summing them with atomics would make the result
@@ -157,20 +157,6 @@ __global__ void invert_kernel(const int32_t* __restrict__ sorted_slot, int num_r
   if (p >= 0 && p < num_rows) inv[p] = i;
 }
 
-template <typename T>
-__global__ void gather_scale_kernel(const T* __restrict__ src, int ld_src, int mode, int fan_out,
-                                    const int32_t* __restrict__ sorted_slot,
-                                    const float* __restrict__ gates, int num_rows, int cols,
-                                    T* __restrict__ out) {
-  const size_t q = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (q >= (size_t)num_rows * cols) return;
-  const int i = (int)(q / cols), c = (int)(q % cols);
-  const int p = sorted_slot[i];
-  const int r = mode == ROWS_GROUPED ? i : p / fan_out;
-  const float g = gates ? gates[p] : 1.0f;
-  out[q] = from_f<T>(g * to_f(src[(size_t)r * ld_src + c]));
-}
-
 // out[i, c..c+3] = g * sum_s partial[s, i, c..c+3], one thread per 4 columns of a row
 __global__ void splitk_reduce_kernel(const float* __restrict__ partial, int ks, int num_rows,
                                      int n_out, const int32_t* __restrict__ sorted_slot,
@@ -239,21 +225,6 @@ cudaError_t launch_dg_reduce(const float* partial, int ld, int n_tiles, const in
                              int num_rows, float* dg, cudaStream_t s, int32_t* inv) {
   dg_reduce_kernel<<<cdiv(num_rows, 256), 256, 0, s>>>(partial, ld, n_tiles, sorted_slot,
                                                        num_rows, dg, inv);
-  return cudaGetLastError();
-}
-
-cudaError_t launch_gather_scale(const void* src, int ld_src, int mode, int fan_out,
-                                const int32_t* sorted_slot, const float* gates, int num_rows,
-                                int cols, void* out, smoe_dtype dt, cudaStream_t s) {
-  const size_t n = (size_t)num_rows * cols;
-  const unsigned blocks = (unsigned)((n + 255) / 256);
-  if (dt == SMOE_BF16)
-    gather_scale_kernel<bf16><<<blocks, 256, 0, s>>>((const bf16*)src, ld_src, mode, fan_out,
-                                                     sorted_slot, gates, num_rows, cols, (bf16*)out);
-  else
-    gather_scale_kernel<float><<<blocks, 256, 0, s>>>((const float*)src, ld_src, mode, fan_out,
-                                                      sorted_slot, gates, num_rows, cols,
-                                                      (float*)out);
   return cudaGetLastError();
 }
 

@@ -203,7 +203,10 @@ __global__ void __launch_bounds__(kThreads) dw_gemm_simt_kernel(DwGemm g) {
       const int r = r0 + kk;
       float va = 0.0f, vb = 0.0f;
       if (r < r_end) {
-        if (m0 + m < g.M) va = to_f(A[(size_t)src_row(g.a_mode, r, g.sorted_slot, g.a_fan_out) * g.lda + m0 + m]);
+        if (m0 + m < g.M) {
+          va = to_f(A[(size_t)src_row(g.a_mode, r, g.sorted_slot, g.a_fan_out) * g.lda + m0 + m]);
+          if (g.row_gates) va *= g.row_gates[g.sorted_slot[r]];
+        }
         if (n0 + m < g.N) vb = to_f(B[(size_t)src_row(g.b_mode, r, g.sorted_slot, g.b_fan_out) * g.ldb + n0 + m]);
       }
       As[kk][m] = va;

@@ -43,6 +43,8 @@
 // memory before returning.
 #include <cuda.h>
 
+#include <cstdlib>
+
 #include "common.cuh"
 
 namespace smoe {
@@ -404,6 +406,7 @@ struct SharedCtl {
 // dW kernel: the expert offsets and the slot-index ring.
 struct DwExtra {
   int idx[IDX_STAGES][2][BK];  // source row per operand (A, B) of each stage row, -1 = zero
+  float gsc[IDX_STAGES][BK];   // gate of each stage row (gated A rows only)
   int off[kMaxE + 1];          // expert offsets
   short order[kMaxE];          // experts by descending row count (ties: lower id)
 };
@@ -1070,13 +1073,268 @@ struct SlabGather {
       cp_async16(dst + dst_off(j, t), ok ? cbase + (size_t)sr * ld : base, ok ? 16u : 0u);
     }
   }
+  // This thread's gates of a stage (one per row it copies), from the index ring.
+  __device__ __forceinline__ void load_gates(const float* gsc, float* g) const {
+#pragma unroll
+    for (int j = 0; j < NR; ++j) g[j] = gsc[row0 + RSTEP * j];
+  }
+  // Multiplies the chunks this thread copied into `stage` (already landed) by
+  // their rows' gates: bf16 value times fp32 gate, rounded once to bf16.
+  __device__ __forceinline__ void scale(uint8_t* stage, const float* g, int t) const {
+#pragma unroll
+    for (int j = 0; j < NR; ++j) {
+      uint4* p = reinterpret_cast<uint4*>(stage + dst_off(j, t));
+      float v[8];
+      unpack8(*p, v);
+#pragma unroll
+      for (int q = 0; q < 8; ++q) v[q] *= g[j];
+      *p = pack8(v);
+    }
+  }
 };
+
+// Gated gather of the A operand with deferred hand-over.  The gate multiplies the
+// copied bytes in shared memory, so a stage can only be handed to the tensor core
+// once this thread's copies of it have landed: each thread keeps its last kDefer
+// stages in flight (one cp.async group per stage) and, after issuing a stage,
+// waits for the group kDefer stages older, scales that stage's rows, makes the
+// writes visible to the tensor core's (async) proxy and arrives on its full
+// barrier.  kDefer < the ring depth, so the thread never waits on a stage that
+// can only be freed by the hand-over it is holding back.
+constexpr int kDefer = 2;
+struct GatePending {
+  int stage[kDefer + 1];
+  bool live[kDefer + 1];
+  float g[kDefer + 1][SlabGather<2>::NR];
+  __device__ __forceinline__ void init() {
+#pragma unroll
+    for (int i = 0; i <= kDefer; ++i) live[i] = false;
+  }
+};
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait_group() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+// After the copies of `stage_idx` were issued (gates g_new): commit them as one
+// group, then hand over the stage issued kDefer steps ago, if any.
+__device__ __forceinline__ void gated_push(GatePending& q, const SlabGather<2>& ga, int t, int stage_idx,
+                                           const float* g_new, uint8_t* ring, int stage_bytes,
+                                           uint64_t* full) {
+  cp_async_commit();
+  q.stage[kDefer] = stage_idx;
+  q.live[kDefer] = true;
+#pragma unroll
+  for (int j = 0; j < SlabGather<2>::NR; ++j) q.g[kDefer][j] = g_new[j];
+  if (q.live[0]) {
+    cp_async_wait_group<kDefer>();
+    ga.scale(ring + q.stage[0] * stage_bytes, q.g[0], t);
+    fence_proxy_async();
+    mbar_arrive(&full[q.stage[0]]);
+  }
+#pragma unroll
+  for (int i = 0; i < kDefer; ++i) {
+    q.stage[i] = q.stage[i + 1];
+    q.live[i] = q.live[i + 1];
+#pragma unroll
+    for (int j = 0; j < SlabGather<2>::NR; ++j) q.g[i][j] = q.g[i + 1][j];
+  }
+  q.live[kDefer] = false;
+}
+// Hands over every stage still held back (end of the work list).
+__device__ __forceinline__ void gated_drain(GatePending& q, const SlabGather<2>& ga, int t, uint8_t* ring,
+                                            int stage_bytes, uint64_t* full) {
+  cp_async_wait_group<0>();
+#pragma unroll
+  for (int i = 0; i < kDefer; ++i) {
+    if (!q.live[i]) continue;
+    ga.scale(ring + q.stage[i] * stage_bytes, q.g[i], t);
+    fence_proxy_async();
+    mbar_arrive(&full[q.stage[i]]);
+    q.live[i] = false;
+  }
+}
+
+// The tile list of the dW kernels: a tile's work grows with its expert's rows, and
+// routing can be very uneven, so the list runs over the experts from the most rows
+// to the fewest and the P workers (CTAs, or CTA pairs) take it in rounds of P
+// tiles, alternately forward and backward (every role derives the same sequence).
+// Tile L -> (e, nb, mb), mb fastest.
+struct DwTiles {
+  int P, w;    // workers and this worker's index
+  int nM, nN;  // M and N tiles per expert
+  int total;
+  __device__ __forceinline__ int tile(int j) const { return j * P + ((j & 1) ? P - 1 - w : w); }
+  __device__ __forceinline__ void coords(const DwExtra& x, int L, int& e, int& mb, int& nb) const {
+    e = x.order[L / (nM * nN)];
+    const int rem = L % (nM * nN);
+    nb = rem / nM;
+    mb = rem % nM;
+  }
+};
+
+// Experts by descending row count (ties: lower id); with more than 256 experts
+// the tiles keep the expert index order.  Ends with a block barrier.
+__device__ __forceinline__ void dw_expert_order(DwExtra& x, int E) {
+  if (E <= 256) {
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+      const int n = x.off[e + 1] - x.off[e];
+      int rank = 0;
+      for (int f = 0; f < E; ++f) {
+        const int m = x.off[f + 1] - x.off[f];
+        rank += (m > n) || (m == n && f < e);
+      }
+      x.order[rank] = (short)e;
+    }
+  } else {
+    for (int e = threadIdx.x; e < E; e += blockDim.x) x.order[e] = (short)e;
+  }
+  __syncthreads();
+}
+
+// Source-row producer of the dW gathers (one warp).  Loads for kIdxBatch stages
+// are issued together before any is written, so one global-load latency is paid
+// per batch instead of per stage.  Each slot p becomes the source row p / fan_out
+// (a shift for a power of two), checked against the operand's row count; -1 marks
+// a zero row.  A_SCALE: the slot's gate goes beside it, and a grouped A (gathered
+// row by row) takes grouped row r itself.
+template <bool A_GATHER, bool B_GATHER, bool A_SCALE>
+__device__ __forceinline__ void dw_index_producer(SharedCtl& c, DwExtra& x, const DwGemm& g,
+                                                  const DwTiles& tl, volatile int* abort_flag, int lane) {
+  constexpr int kIdxBatch = IDX_STAGES / 2;
+  const int a_shift = (g.a_fan_out & (g.a_fan_out - 1)) == 0 ? __ffs(g.a_fan_out) - 1 : -1;
+  const int b_shift = (g.b_fan_out & (g.b_fan_out - 1)) == 0 ? __ffs(g.b_fan_out) - 1 : -1;
+  auto src_of = [&](int p, int shift, int fan, int rows) -> int {
+    if (p < 0) return -1;
+    const int r = shift >= 0 ? (p >> shift) : p / fan;
+    if (r >= rows) {
+      report_error(g.err, ERRBIT_DATA);
+      return -1;
+    }
+    return r;
+  };
+  const bool a_ident = g.a_mode == ROWS_GROUPED;
+  Ring ri;
+  bool run = true;
+  for (int jt = 0, L = tl.tile(0); run && L < tl.total; L = tl.tile(++jt)) {
+    int e, mb, nb;
+    tl.coords(x, L, e, mb, nb);
+    const int r_begin = x.off[e], r_end = x.off[e + 1];
+    const int nK = cdiv(r_end - r_begin, BK);
+    for (int kb0 = 0; run && kb0 < nK; kb0 += kIdxBatch) {
+      int v[kIdxBatch][BK / 32];
+      float gv[kIdxBatch][BK / 32];
+#pragma unroll
+      for (int b = 0; b < kIdxBatch; ++b)
+#pragma unroll
+        for (int q = 0; q < BK / 32; ++q) {
+          const int r = r_begin + (kb0 + b) * BK + lane + 32 * q;
+          v[b][q] = (kb0 + b < nK && r < r_end) ? __ldg(g.sorted_slot + r) : -1;
+          gv[b][q] = 0.0f;
+        }
+      if (A_SCALE) {  // the gates of those slots (a second dependent load per batch)
+#pragma unroll
+        for (int b = 0; b < kIdxBatch; ++b)
+#pragma unroll
+          for (int q = 0; q < BK / 32; ++q) {
+            const int p = v[b][q];
+            if (p >= 0 && p < g.num_rows) gv[b][q] = __ldg(g.row_gates + p);
+          }
+      }
+#pragma unroll
+      for (int b = 0; b < kIdxBatch; ++b) {
+        if (kb0 + b >= nK) break;
+        if (!mbar_wait(&c.iempty[ri.s], ri.ph ^ 1, abort_flag, g.err)) { run = false; break; }
+#pragma unroll
+        for (int q = 0; q < BK / 32; ++q) {
+          const int r = r_begin + (kb0 + b) * BK + lane + 32 * q;
+          if (A_GATHER) {
+            int a_src;
+            if (A_SCALE && a_ident) a_src = (v[b][q] < 0 || r >= g.a_rows) ? -1 : r;
+            else a_src = src_of(v[b][q], a_shift, g.a_fan_out, g.a_rows);
+            x.idx[ri.s][0][lane + 32 * q] = a_src;
+          }
+          if (A_SCALE) x.gsc[ri.s][lane + 32 * q] = gv[b][q];
+          if (B_GATHER) x.idx[ri.s][1][lane + 32 * q] = src_of(v[b][q], b_shift, g.b_fan_out, g.b_rows);
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&c.ifull[ri.s]);
+        ri.next(IDX_STAGES);
+      }
+    }
+  }
+}
+
+// Epilogue of a dW tile: this warp's 32 accumulator rows (M = m0 + 32 q + lane)
+// times the tile's BN columns (from n0), from tensor memory (zeros when the
+// expert has no rows).  d_boxed: per 32-column chunk the warp writes its 32 x 32
+// fp32 block into a 128-byte-swizzled box (transposed for TRANS_OUT) that one TMA
+// tensor store writes out, clipped to dW's bounds; else plain stores.
+template <bool TRANS_OUT>
+__device__ __forceinline__ void dw_store_tile(const DwGemm& g, const CUtensorMap* tmD, int d_boxed,
+                                              uint8_t* box, uint32_t box_s, uint32_t trow,
+                                              bool has_rows, int e, int m0, int n0, int q, int lane) {
+  const int m = m0 + q * 32 + lane;
+#pragma unroll 1
+  for (int c0 = 0; c0 < BN; c0 += 32) {
+    float v[32];
+    if (has_rows) {
+      tmem_ld32(trow + c0, v);
+    } else {
+#pragma unroll
+      for (int j = 0; j < 32; ++j) v[j] = 0.0f;
+    }
+    if (d_boxed) {
+      if (n0 + c0 >= g.N) break;  // warp-uniform
+      if (lane == 0) bulk_wait_read();  // the previous chunk's store has read the box
+      __syncwarp();
+      if (TRANS_OUT) {  // box[n][m]: row j = column n, lane = m
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+          *reinterpret_cast<float*>(box + j * 128 + ((((lane >> 2) ^ (j & 7))) << 4) + ((lane & 3) << 2)) = v[j];
+      } else {  // box[m][n]: row lane = m
+#pragma unroll
+        for (int j4 = 0; j4 < 8; ++j4)
+          *reinterpret_cast<float4*>(box + lane * 128 + ((j4 ^ (lane & 7)) << 4)) =
+              make_float4(v[4 * j4], v[4 * j4 + 1], v[4 * j4 + 2], v[4 * j4 + 3]);
+      }
+      fence_proxy_async();
+      __syncwarp();
+      if (lane == 0) {
+        if (TRANS_OUT) tma_store_3d(tmD, box_s, m0 + q * 32, n0 + c0, e);
+        else tma_store_3d(tmD, box_s, n0 + c0, m0 + q * 32, e);
+        bulk_commit();
+      }
+      continue;
+    }
+    if (m >= g.M) continue;
+    if (TRANS_OUT) {  // dW[e][n][m]: lanes hold consecutive m -> 128-byte lines
+      float* out = g.dw + (size_t)e * g.N * g.M + m;
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        const int n = n0 + c0 + j;
+        if (n < g.N) out[(size_t)n * g.M] = v[j];
+      }
+    } else {
+      float* out = g.dw + ((size_t)e * g.M + m) * g.N;
+#pragma unroll
+      for (int j4 = 0; j4 < 8; ++j4) {
+        const int n = n0 + c0 + 4 * j4;
+        if (n >= g.N) break;
+        *reinterpret_cast<float4*>(out + n) =
+            make_float4(v[4 * j4], v[4 * j4 + 1], v[4 * j4 + 2], v[4 * j4 + 3]);
+      }
+    }
+  }
+}
 
 // dW[e] tile (e, m-block, n-block) of D[m, n] = sum over the expert's rows r of
 // A[r, m] * B[r, n].  TRANS_OUT stores D transposed (the host swapped the
 // operands so that a gathered operand sits on the 128-wide A side); the store
 // is then coalesced across the warp (consecutive m, one n at a time).
-template <bool A_GATHER, bool B_GATHER, bool TRANS_OUT>
+// A_SCALE: A is gathered (through sorted_slot, or row by row when it is grouped)
+// and each of its rows is multiplied by the gate of its slot on the way in.
+template <bool A_GATHER, bool B_GATHER, bool TRANS_OUT, bool A_SCALE = false>
 __global__ void __launch_bounds__(kDwThreads, 1)
 dw_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                   const __grid_constant__ CUtensorMap tmD, const DwGemm g, int nM, int nN,
@@ -1085,6 +1343,7 @@ dw_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
   // at the cost of a 3-stage B ring measured about 1% slower
   constexpr int SA = 4, SB = 4;
   static_assert(SA * A_BYTES + SB * B_BYTES <= kRingBytes, "stage rings exceed their budget");
+  static_assert(!A_SCALE || (A_GATHER && kDefer < SA), "gated rows are gathered, deferred < ring");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
   uint8_t* sA = smem;
@@ -1097,46 +1356,22 @@ dw_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
                 B_GATHER ? kDwGatherThreads : 1, kDwGatherThreads / 32, x.off);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const bool offsets_ok = c.total_mtiles > 0 || g.num_rows == 0;
-  const int total = offsets_ok ? g.E * nM * nN : 0;
-  // A tile's work grows with its expert's rows, and routing can be very uneven, so
-  // the tile list runs over the experts from the most rows to the fewest and the
-  // CTAs take it in rounds of gridDim.x tiles, alternately forward and backward
-  // (every role of the CTA derives the same sequence).  With more than 256
-  // experts the tiles keep the expert index order.
-  if (g.E <= 256) {
-    for (int e = threadIdx.x; e < g.E; e += blockDim.x) {
-      const int n = x.off[e + 1] - x.off[e];
-      int rank = 0;
-      for (int f = 0; f < g.E; ++f) {
-        const int m = x.off[f + 1] - x.off[f];
-        rank += (m > n) || (m == n && f < e);
-      }
-      x.order[rank] = (short)e;
-    }
-  } else {
-    for (int e = threadIdx.x; e < g.E; e += blockDim.x) x.order[e] = (short)e;
-  }
-  __syncthreads();
-  auto tile_of = [&](int j) {  // this CTA's j-th tile
-    const int P = (int)gridDim.x, b = (int)blockIdx.x;
-    return j * P + ((j & 1) ? P - 1 - b : b);
-  };
-  // tile L -> (e, nb, mb), mb fastest
-  auto coords = [&](int L, int& e, int& mb, int& nb) {
-    e = x.order[L / (nM * nN)];
-    const int rem = L % (nM * nN);
-    nb = rem / nM;
-    mb = rem % nM;
-  };
+  DwTiles tl;
+  tl.P = (int)gridDim.x;
+  tl.w = (int)blockIdx.x;
+  tl.nM = nM;
+  tl.nN = nN;
+  tl.total = offsets_ok ? g.E * nM * nN : 0;
+  dw_expert_order(x, g.E);
 
   if (warp == 0) {
     // ---------------- TMA producer of the grouped operand(s) ----------------
     if (lane == 0 && !(A_GATHER && B_GATHER)) {
       Ring ra, rb;
       bool run = true;
-      for (int jt = 0, L = tile_of(0); run && L < total; L = tile_of(++jt)) {
+      for (int jt = 0, L = tl.tile(0); run && L < tl.total; L = tl.tile(++jt)) {
         int e, mb, nb;
-        coords(L, e, mb, nb);
+        tl.coords(x, L, e, mb, nb);
         const int r_begin = x.off[e], r_end = x.off[e + 1];
         const int nK = cdiv(r_end - r_begin, BK);
         for (int kb = 0; kb < nK; ++kb) {
@@ -1164,53 +1399,7 @@ dw_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
     __syncwarp();
   } else if ((A_GATHER || B_GATHER) && warp == 2) {
     // ---------------- source-row producer for the gathers ----------------
-    // Loads for kIdxBatch stages are issued together before any is written, so
-    // one global-load latency is paid per batch instead of per stage.  Each slot
-    // p becomes the source row p / fan_out (a shift for a power of two), checked
-    // against the operand's row count; -1 marks a zero row.
-    constexpr int kIdxBatch = IDX_STAGES / 2;
-    const int a_shift = (g.a_fan_out & (g.a_fan_out - 1)) == 0 ? __ffs(g.a_fan_out) - 1 : -1;
-    const int b_shift = (g.b_fan_out & (g.b_fan_out - 1)) == 0 ? __ffs(g.b_fan_out) - 1 : -1;
-    auto src_of = [&](int p, int shift, int fan, int rows) -> int {
-      if (p < 0) return -1;
-      const int r = shift >= 0 ? (p >> shift) : p / fan;
-      if (r >= rows) {
-        report_error(g.err, ERRBIT_DATA);
-        return -1;
-      }
-      return r;
-    };
-    Ring ri;
-    bool run = true;
-    for (int jt = 0, L = tile_of(0); run && L < total; L = tile_of(++jt)) {
-      int e, mb, nb;
-      coords(L, e, mb, nb);
-      const int r_begin = x.off[e], r_end = x.off[e + 1];
-      const int nK = cdiv(r_end - r_begin, BK);
-      for (int kb0 = 0; run && kb0 < nK; kb0 += kIdxBatch) {
-        int v[kIdxBatch][BK / 32];
-#pragma unroll
-        for (int b = 0; b < kIdxBatch; ++b)
-#pragma unroll
-          for (int q = 0; q < BK / 32; ++q) {
-            const int r = r_begin + (kb0 + b) * BK + lane + 32 * q;
-            v[b][q] = (kb0 + b < nK && r < r_end) ? __ldg(g.sorted_slot + r) : -1;
-          }
-#pragma unroll
-        for (int b = 0; b < kIdxBatch; ++b) {
-          if (kb0 + b >= nK) break;
-          if (!mbar_wait(&c.iempty[ri.s], ri.ph ^ 1, abort_flag, g.err)) { run = false; break; }
-#pragma unroll
-          for (int q = 0; q < BK / 32; ++q) {
-            if (A_GATHER) x.idx[ri.s][0][lane + 32 * q] = src_of(v[b][q], a_shift, g.a_fan_out, g.a_rows);
-            if (B_GATHER) x.idx[ri.s][1][lane + 32 * q] = src_of(v[b][q], b_shift, g.b_fan_out, g.b_rows);
-          }
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&c.ifull[ri.s]);
-          ri.next(IDX_STAGES);
-        }
-      }
-    }
+    dw_index_producer<A_GATHER, B_GATHER, A_SCALE>(c, x, g, tl, abort_flag, lane);
   } else if ((A_GATHER || B_GATHER) && warp >= kGatherWarp0 &&
              warp < kGatherWarp0 + kDwGatherThreads / 32) {
     // ---------------- cp.async gather of the scattered operand(s) ----------------
@@ -1219,11 +1408,13 @@ dw_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
     SlabGather<4> gb;
     ga.init(t);
     gb.init(t);
+    GatePending pend;
+    pend.init();
     Ring ra, rb, ri;
     bool run = true;
-    for (int jt = 0, L = tile_of(0); run && L < total; L = tile_of(++jt)) {
+    for (int jt = 0, L = tl.tile(0); run && L < tl.total; L = tl.tile(++jt)) {
       int e, mb, nb;
-      coords(L, e, mb, nb);
+      tl.coords(x, L, e, mb, nb);
       const int nK = cdiv(x.off[e + 1] - x.off[e], BK);
       for (int kb = 0; kb < nK; ++kb) {
         if (!mbar_wait(&c.ifull[ri.s], ri.ph, abort_flag, g.err)) { run = false; break; }
@@ -1231,7 +1422,13 @@ dw_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
           if (!mbar_wait(&c.emptyA[ra.s], ra.ph ^ 1, abort_flag, g.err)) { run = false; break; }
           ga.issue(smem_u32(sA + ra.s * A_BYTES), x.idx[ri.s][0], reinterpret_cast<const bf16*>(g.a),
                    g.lda, mb * BM, g.M, t);
-          cp_async_arrive(&c.fullA[ra.s]);
+          if (A_SCALE) {
+            float gn[SlabGather<2>::NR];
+            ga.load_gates(x.gsc[ri.s], gn);
+            gated_push(pend, ga, t, ra.s, gn, sA, A_BYTES, c.fullA);
+          } else {
+            cp_async_arrive(&c.fullA[ra.s]);
+          }
           ra.next(SA);
         }
         if (B_GATHER) {
@@ -1246,6 +1443,7 @@ dw_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
         ri.next(IDX_STAGES);
       }
     }
+    if (A_SCALE && run) gated_drain(pend, ga, t, sA, A_BYTES, c.fullA);
   } else if (warp == 1) {
     // ---------------- MMA issuer ----------------
     // With a gathered operand its rows past the slice are zero-filled, so the
@@ -1257,9 +1455,9 @@ dw_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
     if (!kGather || lane == 0) {
       Ring ra, rb;
       int it = 0;
-      for (int jt = 0, L = tile_of(0); L < total; L = tile_of(++jt), ++it) {
+      for (int jt = 0, L = tl.tile(0); L < tl.total; L = tl.tile(++jt), ++it) {
         int e, mb, nb;
-        coords(L, e, mb, nb);
+        tl.coords(x, L, e, mb, nb);
         const int r_begin = x.off[e], r_end = x.off[e + 1];
         const int nK = cdiv(r_end - r_begin, BK);
         const int buf = it & 1;
@@ -1314,75 +1512,20 @@ dw_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
     __syncwarp();
   } else if (warp >= 4 && warp < 8) {
     // ---------------- epilogue: one accumulator row per thread ----------------
-    // d_boxed: per 32-column chunk the warp writes its 32 x 32 fp32 block into a
-    // 128-byte-swizzled box (transposed for TRANS_OUT) that one TMA tensor store
-    // writes out, clipped to dW's bounds; else plain stores.
     const int q = warp - 4;
-    const int r = q * 32 + lane;
     uint8_t* box = smem + kRingBytes + kCtlBytes + kDwExtraBytes + q * kDwBoxBytes;
     const uint32_t box_s = smem_u32(box);
     int it = 0;
-    for (int jt = 0, L = tile_of(0); L < total; L = tile_of(++jt), ++it) {
+    for (int jt = 0, L = tl.tile(0); L < tl.total; L = tl.tile(++jt), ++it) {
       int e, mb, nb;
-      coords(L, e, mb, nb);
+      tl.coords(x, L, e, mb, nb);
       const int nrows = x.off[e + 1] - x.off[e];
       const int buf = it & 1;
       const uint32_t tph = (it >> 1) & 1;
       if (!mbar_wait(&c.tfull[buf], tph, abort_flag, g.err)) break;
       tc_fence_after();
-      const int m = mb * BM + r;
       const uint32_t trow = c.tmem_base + ((uint32_t)(q * 32) << 16) + buf * BN;
-#pragma unroll 1
-      for (int c0 = 0; c0 < BN; c0 += 32) {
-        float v[32];
-        if (nrows > 0) {
-          tmem_ld32(trow + c0, v);
-        } else {
-#pragma unroll
-          for (int j = 0; j < 32; ++j) v[j] = 0.0f;
-        }
-        if (d_boxed) {
-          if (nb * BN + c0 >= g.N) break;  // warp-uniform
-          if (lane == 0) bulk_wait_read();  // the previous chunk's store has read the box
-          __syncwarp();
-          if (TRANS_OUT) {  // box[n][m]: row j = column n, lane = m
-#pragma unroll
-            for (int j = 0; j < 32; ++j)
-              *reinterpret_cast<float*>(box + j * 128 + ((((lane >> 2) ^ (j & 7))) << 4) + ((lane & 3) << 2)) = v[j];
-          } else {  // box[m][n]: row lane = m
-#pragma unroll
-            for (int j4 = 0; j4 < 8; ++j4)
-              *reinterpret_cast<float4*>(box + lane * 128 + ((j4 ^ (lane & 7)) << 4)) =
-                  make_float4(v[4 * j4], v[4 * j4 + 1], v[4 * j4 + 2], v[4 * j4 + 3]);
-          }
-          fence_proxy_async();
-          __syncwarp();
-          if (lane == 0) {
-            if (TRANS_OUT) tma_store_3d(&tmD, box_s, mb * BM + q * 32, nb * BN + c0, e);
-            else tma_store_3d(&tmD, box_s, nb * BN + c0, mb * BM + q * 32, e);
-            bulk_commit();
-          }
-          continue;
-        }
-        if (m >= g.M) continue;
-        if (TRANS_OUT) {  // dW[e][n][m]: lanes hold consecutive m -> 128-byte lines
-          float* out = g.dw + (size_t)e * g.N * g.M + m;
-#pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            const int n = nb * BN + c0 + j;
-            if (n < g.N) out[(size_t)n * g.M] = v[j];
-          }
-        } else {
-          float* out = g.dw + ((size_t)e * g.M + m) * g.N;
-#pragma unroll
-          for (int j4 = 0; j4 < 8; ++j4) {
-            const int n = nb * BN + c0 + 4 * j4;
-            if (n >= g.N) break;
-            *reinterpret_cast<float4*>(out + n) =
-                make_float4(v[4 * j4], v[4 * j4 + 1], v[4 * j4 + 2], v[4 * j4 + 3]);
-          }
-        }
-      }
+      dw_store_tile<TRANS_OUT>(g, &tmD, d_boxed, box, box_s, trow, nrows > 0, e, mb * BM, nb * BN, q, lane);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&c.tempty[buf]);
@@ -1390,6 +1533,197 @@ dw_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
     if (lane == 0) bulk_wait_all();
   }
   teardown(c);
+}
+
+// ---------------------------------------------------------------------------
+// dW kernel on CTA pairs (cta_group::2)
+// ---------------------------------------------------------------------------
+// A cluster of two CTAs takes a 256 (M) x 256 (N) tile of dW[e] with M = 256
+// MMAs.  For the same 64 slice rows per stage, CTA r gathers M columns
+// [128 r, 128 r + 128) of the tile's A rows (the scattered operand, optionally
+// gated) and TMA-loads N columns [128 r, 128 r + 128) of B, so a CTA brings 32 KB
+// per K-block instead of 48 KB and its ring holds six stages instead of four:
+// about 2.5x the single-CTA kernel's look-ahead in time, which is what the
+// gather's latency needs.  Rank 0 issues the MMAs once its own stage has landed
+// (its gathered rows, plus both CTAs' TMA bytes, which count on its barrier) and
+// rank 1 has relayed that its gathered rows have landed; it commits to both
+// CTAs' empty barriers.  Each CTA's tensor memory holds its 128 rows of the
+// accumulator (all 256 columns), drained by its own epilogue warps; rank 1's
+// epilogue frees an accumulator buffer on rank 0's barrier.  No load uses
+// multicast: every CTA fetches its own bytes.
+template <bool A_SCALE, bool TRANS_OUT>
+__global__ void __launch_bounds__(kDwThreads, 1)
+dw_pair_tc_kernel(const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmD,
+                  const DwGemm g, int nMP, int nN, int d_boxed) {
+  constexpr int STAGES = 6;
+  constexpr int BH = B_BYTES / 2;  // this CTA's half of B per stage (16 KB)
+  static_assert(STAGES * (A_BYTES + BH) <= kRingBytes && STAGES <= kMaxStages && kDefer < STAGES,
+                "pair ring");
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + STAGES * A_BYTES;
+  SharedCtl& c = *reinterpret_cast<SharedCtl*>(smem + kRingBytes);
+  DwExtra& x = *reinterpret_cast<DwExtra*>(smem + kRingBytes + kCtlBytes);
+  volatile int* abort_flag = &c.abort_flag;
+  const int rank = (int)cluster_rank();
+  // a stage's full barrier: this CTA's gather threads, plus at rank 0 the
+  // producer's expect-tx for both CTAs' B halves
+  setup<STAGES, 0, true>(c, g.offsets, g.E, g.num_rows, g.err,
+                         (uint32_t)kDwGatherThreads + (rank == 0 ? 1u : 0u), 1, kDwGatherThreads / 32,
+                         x.off);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const bool offsets_ok = c.total_mtiles > 0 || g.num_rows == 0;
+  DwTiles tl;
+  tl.P = (int)(gridDim.x >> 1);
+  tl.w = (int)(blockIdx.x >> 1);
+  tl.nM = nMP;
+  tl.nN = nN;
+  tl.total = offsets_ok ? g.E * nMP * nN : 0;
+  dw_expert_order(x, g.E);
+
+  if (warp == 0) {
+    // ---------------- TMA producer: this CTA's half of the B columns ----------------
+    if (lane == 0) {
+      Ring r;
+      bool run = true;
+      for (int jt = 0, L = tl.tile(0); run && L < tl.total; L = tl.tile(++jt)) {
+        int e, mp, nb;
+        tl.coords(x, L, e, mp, nb);
+        const int r_begin = x.off[e], r_end = x.off[e + 1];
+        const int nK = cdiv(r_end - r_begin, BK);
+        for (int kb = 0; kb < nK; ++kb) {
+          if (!mbar_wait(&c.emptyA[r.s], r.ph ^ 1, abort_flag, g.err)) { run = false; break; }
+          const uint32_t full_cl = peer_addr(&c.fullA[r.s], 0);
+          if (rank == 0) mbar_expect_tx(&c.fullA[r.s], 2 * BH);
+          uint8_t* b_dst = sB + r.s * BH;
+          const int col = nb * BN + rank * (BN / 2);
+          tma_load_2d_pair(b_dst, &tmB, full_cl, col, r_begin + kb * BK);
+          tma_load_2d_pair(b_dst + 8192, &tmB, full_cl, col + 64, r_begin + kb * BK);
+          r.next(STAGES);
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 2) {
+    // ---------------- source-row producer (both CTAs build the same rows) ----------------
+    dw_index_producer<true, false, A_SCALE>(c, x, g, tl, abort_flag, lane);
+  } else if (warp >= kGatherWarp0 && warp < kGatherWarp0 + kDwGatherThreads / 32) {
+    // ---------------- cp.async gather of this CTA's 128 A columns ----------------
+    const int t = threadIdx.x - kGatherWarp0 * 32;
+    SlabGather<2> ga;
+    ga.init(t);
+    GatePending pend;
+    pend.init();
+    Ring r, ri;
+    bool run = true;
+    for (int jt = 0, L = tl.tile(0); run && L < tl.total; L = tl.tile(++jt)) {
+      int e, mp, nb;
+      tl.coords(x, L, e, mp, nb);
+      const int nK = cdiv(x.off[e + 1] - x.off[e], BK);
+      for (int kb = 0; kb < nK; ++kb) {
+        if (!mbar_wait(&c.ifull[ri.s], ri.ph, abort_flag, g.err)) { run = false; break; }
+        if (!mbar_wait(&c.emptyA[r.s], r.ph ^ 1, abort_flag, g.err)) { run = false; break; }
+        ga.issue(smem_u32(sA + r.s * A_BYTES), x.idx[ri.s][0], reinterpret_cast<const bf16*>(g.a), g.lda,
+                 mp * 2 * BM + rank * BM, g.M, t);
+        if (A_SCALE) {
+          float gn[SlabGather<2>::NR];
+          ga.load_gates(x.gsc[ri.s], gn);
+          gated_push(pend, ga, t, r.s, gn, sA, A_BYTES, c.fullA);
+        } else {
+          cp_async_arrive(&c.fullA[r.s]);
+        }
+        r.next(STAGES);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&c.iempty[ri.s]);
+        ri.next(IDX_STAGES);
+      }
+    }
+    if (A_SCALE && run) gated_drain(pend, ga, t, sA, A_BYTES, c.fullA);
+  } else if (warp == 1) {
+    if (lane == 0 && rank == 1) {
+      // ---------------- relay: this CTA's gathered rows of a stage have landed ----------------
+      Ring r;
+      bool run = true;
+      for (int jt = 0, L = tl.tile(0); run && L < tl.total; L = tl.tile(++jt)) {
+        int e, mp, nb;
+        tl.coords(x, L, e, mp, nb);
+        const int nK = cdiv(x.off[e + 1] - x.off[e], BK);
+        for (int kb = 0; kb < nK; ++kb) {
+          if (!mbar_wait(&c.fullA[r.s], r.ph, abort_flag, g.err)) { run = false; break; }
+          fence_proxy_async();  // rows written by cp.async (and the gate pass), read by the tensor core
+          mbar_arrive_cluster_relaxed(peer_addr(&c.pfull[r.s], 0));
+          r.next(STAGES);
+        }
+      }
+    } else if (lane == 0) {
+      // ---------------- MMA issuer (rank 0) ----------------
+      constexpr uint32_t idesc = idesc_bf16(2 * BM, BN, 1, 1);
+      Ring r;
+      int it = 0;
+      for (int jt = 0, L = tl.tile(0); L < tl.total; L = tl.tile(++jt), ++it) {
+        int e, mp, nb;
+        tl.coords(x, L, e, mp, nb);
+        const int nK = cdiv(x.off[e + 1] - x.off[e], BK);
+        const int buf = it & 1;
+        const uint32_t tph = (it >> 1) & 1;
+        if (!mbar_wait(&c.tempty[buf], tph ^ 1, abort_flag, g.err)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = c.tmem_base + buf * BN;
+        bool ok = true;
+        for (int kb = 0; kb < nK; ++kb) {
+          if (!mbar_wait(&c.fullA[r.s], r.ph, abort_flag, g.err) ||
+              !mbar_wait(&c.pfull[r.s], r.ph, abort_flag, g.err)) { ok = false; break; }
+          tc_fence_after();
+          fence_proxy_async();  // rows written by cp.async (and the gate pass), read by the tensor core
+          const uint32_t a_addr = smem_u32(sA + r.s * A_BYTES);
+          const uint32_t b_addr = smem_u32(sB + r.s * BH);
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk)
+            umma_bf16_pair(d_tmem, desc_mnmajor(a_addr + kk * 2048), desc_mnmajor(b_addr + kk * 2048), idesc,
+                           (kb | kk) != 0);
+          umma_commit_pair(smem_u32(&c.emptyA[r.s]));  // the stage is free in both CTAs
+          umma_commit_pair(peer_addr(&c.emptyA[r.s], 1));
+          r.next(STAGES);
+        }
+        if (!ok) break;
+        if (nK > 0) {
+          umma_commit_pair(smem_u32(&c.tfull[buf]));
+          umma_commit_pair(peer_addr(&c.tfull[buf], 1));
+        } else {  // an empty expert: both epilogues write zeros
+          mbar_arrive(&c.tfull[buf]);
+          mbar_arrive_cluster(peer_addr(&c.tfull[buf], 1));
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp >= 4 && warp < 8) {
+    // ---------------- epilogue: this CTA's 128 accumulator rows ----------------
+    const int q = warp - 4;
+    uint8_t* box = smem + kRingBytes + kCtlBytes + kDwExtraBytes + q * kDwBoxBytes;
+    const uint32_t box_s = smem_u32(box);
+    int it = 0;
+    for (int jt = 0, L = tl.tile(0); L < tl.total; L = tl.tile(++jt), ++it) {
+      int e, mp, nb;
+      tl.coords(x, L, e, mp, nb);
+      const int nrows = x.off[e + 1] - x.off[e];
+      const int buf = it & 1;
+      const uint32_t tph = (it >> 1) & 1;
+      if (!mbar_wait(&c.tfull[buf], tph, abort_flag, g.err)) break;
+      tc_fence_after();
+      const uint32_t trow = c.tmem_base + ((uint32_t)(q * 32) << 16) + buf * BN;
+      dw_store_tile<TRANS_OUT>(g, &tmD, d_boxed, box, box_s, trow, nrows > 0, e, mp * 2 * BM + rank * BM,
+                               nb * BN, q, lane);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {  // the accumulator buffer is free (counted at rank 0)
+        if (rank == 0) mbar_arrive(&c.tempty[buf]);
+        else mbar_arrive_cluster(peer_addr(&c.tempty[buf], 0));
+      }
+    }
+    if (lane == 0) bulk_wait_all();
+  }
+  teardown<true>(c);
 }
 
 // ---------------------------------------------------------------------------
@@ -1527,14 +1861,62 @@ cudaError_t launch_g(const CUtensorMap& ta, const CUtensorMap& tb, const EpiMaps
   return cudaGetLastError();
 }
 
-template <bool AG, bool BG, bool TR>
+template <bool AG, bool BG, bool TR, bool SC = false>
 cudaError_t launch_d(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& td,
                      int d_boxed, const DwGemm& g, int nM, int nN, int grid, cudaStream_t s) {
-  auto kern = dw_gemm_tc_kernel<AG, BG, TR>;
+  auto kern = dw_gemm_tc_kernel<AG, BG, TR, SC>;
   cudaError_t e = prep(kern, kDwSmem);
   if (e != cudaSuccess) return e;
   kern<<<grid, kDwThreads, kDwSmem, s>>>(ta, tb, td, g, nM, nN, d_boxed);
   return cudaGetLastError();
+}
+
+// The pair dW kernel on as many 2-CTA clusters as the device holds at once (at
+// most one per tile pair).
+template <bool SC, bool TR>
+cudaError_t launch_dp(const CUtensorMap& tb, const CUtensorMap& td, int d_boxed, const DwGemm& g,
+                      int nMP, int nN, long long tiles, cudaStream_t s) {
+  auto kern = dw_pair_tc_kernel<SC, TR>;
+  cudaError_t e = prep(kern, kDwSmem);
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(num_sms() & ~1), 1, 1);
+  cfg.blockDim = dim3(kDwThreads, 1, 1);
+  cfg.dynamicSmemBytes = kDwSmem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  static int max_clusters = 0;  // per instantiation
+  if (max_clusters <= 0) {
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n <= 0) {
+      (void)cudaGetLastError();
+      n = num_sms() / 2;
+    }
+    max_clusters = n;
+  }
+  const long long pairs = tiles < max_clusters ? tiles : max_clusters;
+  if (pairs <= 0) return cudaSuccess;
+  cfg.gridDim = dim3((unsigned)(2 * pairs), 1, 1);
+  e = cudaLaunchKernelEx(&cfg, kern, tb, td, g, nMP, nN, d_boxed);
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
+// Whether the dW products whose gathered operand is on the A side run on CTA
+// pairs (SMOE_DW_PAIR=1 in the environment; read once).
+bool dw_pair_enabled() {
+  static int v = -1;
+  if (v < 0) {
+    const char* env = getenv("SMOE_DW_PAIR");
+    v = (env != nullptr && env[0] == '1') ? 1 : 0;
+  }
+  return v == 1;
 }
 
 }  // namespace
@@ -1638,6 +2020,9 @@ cudaError_t launch_dw_gemm_tc(const DwGemm& g_in, cudaStream_t s) {
   }
   const int nM = cdiv(g.M, BM), nN = cdiv(g.N, BN);
   const bool ag = g.a_mode == ROWS_GATHER, bg = g.b_mode == ROWS_GATHER;
+  // gated rows: the gate multiplies the A operand as it is gathered (a grouped A
+  // is then gathered row by row)
+  const bool sc = g.row_gates != nullptr;
   CUtensorMap ta, tb;
   cudaError_t e = rows_map(&ta, g.a, g.M, g.a_rows, g.lda, BK);  // unused when gathered
   if (e != cudaSuccess) return e;
@@ -1653,12 +2038,26 @@ cudaError_t launch_dw_gemm_tc(const DwGemm& g_in, cudaStream_t s) {
   const uint32_t dbox[3] = {32, 32, 1};
   const int d_boxed = make_map(&td, g.dw, 3, ddims, dstr, dbox, CU_TENSOR_MAP_SWIZZLE_128B,
                                CU_TENSOR_MAP_DATA_TYPE_FLOAT32) == cudaSuccess;
+  // CTA pairs: the A operand gathered, B by TMA, and at least two 128-column
+  // halves of M
+  if (dw_pair_enabled() && (ag || sc) && !bg && g.M > BM) {
+    const int nMP = cdiv(g.M, 2 * BM);
+    const long long ptiles = (long long)g.E * nMP * nN;
+    if (sc) return trans ? launch_dp<true, true>(tb, td, d_boxed, g, nMP, nN, ptiles, s)
+                         : launch_dp<true, false>(tb, td, d_boxed, g, nMP, nN, ptiles, s);
+    return trans ? launch_dp<false, true>(tb, td, d_boxed, g, nMP, nN, ptiles, s)
+                 : launch_dp<false, false>(tb, td, d_boxed, g, nMP, nN, ptiles, s);
+  }
   const long long tiles = (long long)g.E * nM * nN;
   const int grid = (int)(tiles < num_sms() ? tiles : num_sms());
-#define SMOE_LAUNCH_D(AG, BG, TR) launch_d<AG, BG, TR>(ta, tb, td, d_boxed, g, nM, nN, grid, s)
-  if (trans) return SMOE_LAUNCH_D(true, false, true);
-  if (ag) return bg ? SMOE_LAUNCH_D(true, true, false) : SMOE_LAUNCH_D(true, false, false);
-  return bg ? SMOE_LAUNCH_D(false, true, false) : SMOE_LAUNCH_D(false, false, false);
+#define SMOE_LAUNCH_D(AG, BG, TR, SC) launch_d<AG, BG, TR, SC>(ta, tb, td, d_boxed, g, nM, nN, grid, s)
+  if (sc) {
+    if (bg) return SMOE_LAUNCH_D(true, true, false, true);
+    return trans ? SMOE_LAUNCH_D(true, false, true, true) : SMOE_LAUNCH_D(true, false, false, true);
+  }
+  if (trans) return SMOE_LAUNCH_D(true, false, true, false);
+  if (ag) return bg ? SMOE_LAUNCH_D(true, true, false, false) : SMOE_LAUNCH_D(true, false, false, false);
+  return SMOE_LAUNCH_D(false, false, false, false);
 #undef SMOE_LAUNCH_D
 }
 

@@ -74,6 +74,11 @@ struct DwGemm {
   const void* b = nullptr;
   int ldb = 0, b_rows = 0, b_mode = ROWS_GROUPED, b_fan_out = 1;
   float* dw = nullptr;  // [E, M, N]
+  // Per-slot gates multiplying each reduction row's product (row i by
+  // gates[sorted_slot[i]]), nullable: the gated ParallelLinear's
+  // dW = sum_i (g_i x_i)^T G_i without a gated copy of x.  The kernels apply the
+  // gate to whichever operand they gather.
+  const float* row_gates = nullptr;
   unsigned* err = nullptr;
 };
 
@@ -116,11 +121,6 @@ cudaError_t launch_transpose_wr(const void* w_r, int d, int E, smoe_dtype dt, vo
 // dg[sorted_slot[i]] = sum_{c < n_tiles} partial[i*ld + c]; inv (nullable) as launch_invert
 cudaError_t launch_dg_reduce(const float* partial, int ld, int n_tiles, const int32_t* sorted_slot,
                              int num_rows, float* dg, cudaStream_t s, int32_t* inv = nullptr);
-// out[i] = gates[sorted_slot[i]] * src[row(i)]  (grouped rows, dtype)
-cudaError_t launch_gather_scale(const void* src, int ld_src, int mode, int fan_out,
-                                const int32_t* sorted_slot, const float* gates, int num_rows,
-                                int cols, void* out, smoe_dtype dt, cudaStream_t s);
-
 // out[i, :] = gates[sorted_slot[i]] * sum_{s < ksplit} partial[s, i, :] (ascending s),
 // grouped rows, bf16; the epilogue of a split-K grouped product
 cudaError_t launch_splitk_reduce(const float* partial, int ksplit, int num_rows, int n_out,

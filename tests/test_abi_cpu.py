@@ -150,8 +150,10 @@ def test_workspaces_hold_no_copy_of_token_rows():
     fwd = L.smoe_mlp_workspace_size(ctypes.byref(desc), 0)
     bwd = L.smoe_mlp_workspace_size(ctypes.byref(desc), 1)
     assert fwd == a256(sort) + a256(S * 4) + a256(S * d * 2)
-    big = a256(S * 2 * f * 2) + a256(S * f * 2) + a256(S * d * 2)
-    assert bwd - big < S * d * 2 // 4
+    # backward: dH [T*k, 2f] and the dx slot rows [T*k, d] (no gated copy of A: the
+    # gates multiply dY's gathered rows inside the dW2 kernel)
+    big = a256(S * 2 * f * 2) + a256(S * d * 2)
+    assert 0 < bwd - big < S * d * 2 // 4
 
 
 def test_decode_workspace_holds_the_split_k_partials():
@@ -220,3 +222,23 @@ def test_slot_count_overflow_is_refused():
     assert L.smoe_workspace_size(0, T, k, 8, 8, 8, 1) == 0
     d = smoe.MlpDesc(T, 64, 64, 8, k, 1, 1)
     assert L.smoe_mlp_workspace_size(ctypes.byref(d), 0) == 0
+
+
+@pytest.mark.parametrize("grouped_in,fan_out", [(1, 1), (0, 4), (0, 1)])
+def test_gated_parallel_linear_backward_adds_no_copy_of_x(grouped_in, fan_out):
+    """With gates, the ParallelLinear backward's workspace grows only by the gate
+    gradient's per-column-tile partials ([num_slots, ceil(K / tile)] fp32): dW's
+    gate multiplies x's rows inside the dW kernel, so no [num_slots, K] gated or
+    grouped copy of x exists (the MoA shapes: 32768 slots, K = 2048, N = 512)."""
+    L = smoe.lib()
+    S, K, N, E = 32768, 2048, 512, 16
+    x_rows = S if (grouped_in or fan_out == 1) else S // fan_out
+    a256 = lambda n: (n + 255) // 256 * 256  # noqa: E731
+    for dt, tile in ((1, 256), (0, 64)):
+        gated = L.parallel_linear_bwd_workspace_size(x_rows, S, K, N, E, fan_out, grouped_in, 0, 1, 0, dt)
+        plain = L.parallel_linear_bwd_workspace_size(x_rows, S, K, N, E, fan_out, grouped_in, 0, 0, 0, dt)
+        assert gated - plain == a256(S * ((K + tile - 1) // tile) * 4)
+        es = 2 if dt == 1 else 4
+        # the only [num_slots, K] buffer is the dx slot rows of a fan-out combine
+        combine = a256(S * K * es) + a256(S * 4) if (not grouped_in and fan_out > 1) else 0
+        assert plain == combine

@@ -73,7 +73,8 @@ def test_parallel_linear_fwd_bwd(dtype, mode, gated):
 
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
 def test_parallel_linear_bwd_dw_only_gated(dtype):
-    """dw alone with gates takes the gather-and-scale route instead of the dx GEMM."""
+    """dw alone with gates: no dx GEMM runs, and the dW kernel applies the gates
+    to the rows it gathers (no gated copy of x)."""
     P = _problem(dtype, "group2scatter_combine", True, seed=3)
     _, dw, _ = smoe.parallel_linear_bwd(P["dy"], P["x"], P["w"], P["ss"], P["off"], P["fan_out"],
                                         P["gi"], P["go"], P["gates"], P["ck"], want_dx=False)
