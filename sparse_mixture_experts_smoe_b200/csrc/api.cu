@@ -12,7 +12,6 @@
 // backward (tradepoint.io article, method paragraphs: the gradient of each
 // expert) swaps the roles of the row maps for dx and runs a per-expert dW GEMM.
 #include <cstdarg>
-#include <cstdlib>
 #include <cstdio>
 #include <cstring>
 #include <map>
@@ -233,7 +232,7 @@ struct MlpWs {
   int ksplit = 1;
   float* dg_part = nullptr; // bwd: [S, dg_ld]
   void* dh = nullptr;       // bwd: [S, m*f] dtype (grouped dH)
-  void* ga = nullptr;       // bwd: [S, f] dtype (gates * A), only when dW2 reads a gated copy
+  void* ga = nullptr;       // bwd: [S, f] dtype (gates * A), written by the dA' epilogue for dW2
   void* dxcomb = nullptr;   // bwd: [S, d] slot rows (dtype), grouped order
   int32_t* inv = nullptr;   // fwd and bwd: [S] grouped row of each slot
   float* dl = nullptr;      // bwd: [T, k]
@@ -243,18 +242,6 @@ struct MlpWs {
   int dg_ld = 0, r_runs = 0;
   size_t bytes = 0;
 };
-// dW2 = sum_i (g A_i)^T dY_t: the gate either multiplies dY's gathered rows inside
-// the dW kernel (default) or A in the dA' epilogue, which then writes g*A
-// (SMOE_MLP_GA=1 in the environment; read once).
-bool mlp_dw2_reads_ga() {
-  static int v = -1;
-  if (v < 0) {
-    const char* env = getenv("SMOE_MLP_GA");
-    v = (env != nullptr && env[0] == '1') ? 1 : 0;
-  }
-  return v == 1;
-}
-
 MlpWs mlp_layout(void* ws, const smoe_mlp_desc& m, int backward) {
   Carve c(ws);
   MlpWs l;
@@ -271,7 +258,7 @@ MlpWs mlp_layout(void* ws, const smoe_mlp_desc& m, int backward) {
     l.dg_ld = cdiv(m.f, act_tile_cols(dt));
     l.dg_part = (float*)c.take(S * l.dg_ld * sizeof(float));
     l.dh = c.take(S * (size_t)(m.act == SMOE_ACT_SWIGLU ? 2 * m.f : m.f) * esize(dt));
-    if (mlp_dw2_reads_ga()) l.ga = c.take(S * m.f * esize(dt));
+    l.ga = c.take(S * m.f * esize(dt));
     l.dxcomb = c.take(S * m.d * esize(dt));
     l.dl = (float*)c.take(S * sizeof(float));
     l.dg = (float*)c.take(S * sizeof(float));
@@ -760,23 +747,21 @@ int smoe_mlp_bwd(const smoe_mlp_desc* desc, const smoe_mlp_tensors* t, void* str
     g.aux_a = t->a; g.ld_aux_a = m.f; g.aux_a_mode = ROWS_GROUPED; g.aux_a_fan_out = 1;
     g.aux_h = t->h; g.ld_aux_h = mf;
     g.out_mode = ROWS_GROUPED; g.out = l.dh; g.ldo = mf; g.out_f32 = dt == SMOE_F32;
-    g.out2 = l.ga; g.ldo2 = m.f;  // null unless dW2 reads a gated copy of A
+    g.out2 = l.ga; g.ldo2 = m.f;
     g.dg_partial = l.dg_part; g.dg_ld = l.dg_ld; g.err = err;
     { PROF("gemm.bwd_dA", 1); SMOE_TRY(run_grouped(g, dt, s), "mlp bwd gemm dA"); }
   }
   { PROF("dg_reduce", 1); SMOE_TRY(launch_dg_reduce(l.dg_part, l.dg_ld, l.dg_ld, t->sorted_slot, S, dg, s, l.inv), "mlp bwd dg"); }
   { PROF("route_dl", 1); SMOE_TRY(launch_route_dl(t->gates, dg, m.T, m.k, l.dl, s), "mlp bwd dl"); }
-  {  // dW2[e] = sum_i (g A)_i^T dy[t_i]
+  {  // dW2[e] = sum_i (g A)_i^T dy[t_i].  g A comes from the dA' epilogue: measured
+     // faster than multiplying dY's gathered rows by g inside the dW kernel
+     // (Mixtral-shaped step: dW2 4.5 ms against 7.6 ms, the epilogue's extra
+     // store 0.4 ms), since a gated stage can only be handed to the tensor core
+     // after its copies land, which shortens the gather's look-ahead.
     DwGemm g;
     g.E = m.E; g.num_rows = S; g.offsets = t->expert_offsets; g.sorted_slot = t->sorted_slot;
     g.M = m.f; g.N = m.d;
-    if (l.ga) {
-      g.a = l.ga;
-    } else {
-      g.a = t->a;
-      g.row_gates = t->gates;
-    }
-    g.lda = m.f; g.a_rows = S; g.a_mode = ROWS_GROUPED; g.a_fan_out = 1;
+    g.a = l.ga; g.lda = m.f; g.a_rows = S; g.a_mode = ROWS_GROUPED; g.a_fan_out = 1;
     g.b = t->dy; g.ldb = m.d; g.b_rows = m.T; g.b_mode = ROWS_GATHER; g.b_fan_out = m.k;
     g.dw = t->dw2; g.err = err;
     { PROF("gemm.bwd_dW2", 1); SMOE_TRY(run_dw(g, dt, s), "mlp bwd dW2"); }

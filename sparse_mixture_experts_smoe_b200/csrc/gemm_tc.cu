@@ -43,8 +43,6 @@
 // memory before returning.
 #include <cuda.h>
 
-#include <cstdlib>
-
 #include "common.cuh"
 
 namespace smoe {
@@ -1192,16 +1190,52 @@ __device__ __forceinline__ void dw_expert_order(DwExtra& x, int E) {
   __syncthreads();
 }
 
-// Source-row producer of the dW gathers (one warp).  Loads for kIdxBatch stages
-// are issued together before any is written, so one global-load latency is paid
-// per batch instead of per stage.  Each slot p becomes the source row p / fan_out
-// (a shift for a power of two), checked against the operand's row count; -1 marks
-// a zero row.  A_SCALE: the slot's gate goes beside it, and a grouped A (gathered
-// row by row) takes grouped row r itself.
+// Walks the (tile, K-block) stages of a dW worker's tile list in order.
+struct DwStageIt {
+  int jt, L, rb, re, nK, kb;
+  bool valid;
+  // From tile L at K-block kb (0 for a new tile): skip tiles without rows.
+  __device__ __forceinline__ void settle(const DwTiles& tl, const DwExtra& x) {
+    while (L < tl.total) {
+      int e, mb, nb;
+      tl.coords(x, L, e, mb, nb);
+      rb = x.off[e];
+      re = x.off[e + 1];
+      nK = cdiv(re - rb, BK);
+      if (kb < nK) { valid = true; return; }
+      L = tl.tile(++jt);
+      kb = 0;
+    }
+    valid = false;
+    nK = 0;
+  }
+  __device__ __forceinline__ void init(const DwTiles& tl, const DwExtra& x) {
+    jt = 0;
+    L = tl.tile(0);
+    kb = 0;
+    settle(tl, x);
+  }
+  // The tile's coordinates are derived again only when its K-blocks run out.
+  __device__ __forceinline__ void next(const DwTiles& tl, const DwExtra& x) {
+    if (++kb < nK) return;
+    L = tl.tile(++jt);
+    kb = 0;
+    settle(tl, x);
+  }
+};
+
+// Source-row producer of the dW gathers (one warp).  The slot ids of kIdxBatch
+// stages are loaded together, and those of the next batch are already in flight
+// while this batch is written to the ring, so the global-load latency overlaps
+// the wait for free ring slots instead of stalling the gathers.  Each slot p
+// becomes the source row p / fan_out (a shift for a power of two), checked
+// against the operand's row count; -1 marks a zero row.  A_SCALE: the slot's gate
+// goes beside it, and a grouped A (gathered row by row) takes grouped row r itself.
 template <bool A_GATHER, bool B_GATHER, bool A_SCALE>
 __device__ __forceinline__ void dw_index_producer(SharedCtl& c, DwExtra& x, const DwGemm& g,
                                                   const DwTiles& tl, volatile int* abort_flag, int lane) {
   constexpr int kIdxBatch = IDX_STAGES / 2;
+  constexpr int NQ = BK / 32;  // slots per lane per stage
   const int a_shift = (g.a_fan_out & (g.a_fan_out - 1)) == 0 ? __ffs(g.a_fan_out) - 1 : -1;
   const int b_shift = (g.b_fan_out & (g.b_fan_out - 1)) == 0 ? __ffs(g.b_fan_out) - 1 : -1;
   auto src_of = [&](int p, int shift, int fan, int rows) -> int {
@@ -1214,53 +1248,67 @@ __device__ __forceinline__ void dw_index_producer(SharedCtl& c, DwExtra& x, cons
     return r;
   };
   const bool a_ident = g.a_mode == ROWS_GROUPED;
+  // slot ids of the next kIdxBatch stages of `it` (-1 past a slice end)
+  auto load_batch = [&](DwStageIt& it, int (&v)[kIdxBatch][NQ], int (&r0)[kIdxBatch]) {
+#pragma unroll
+    for (int b = 0; b < kIdxBatch; ++b) {
+      r0[b] = it.valid ? it.rb + it.kb * BK : 0;
+#pragma unroll
+      for (int q = 0; q < NQ; ++q) {
+        const int r = r0[b] + lane + 32 * q;
+        v[b][q] = (it.valid && r < it.re) ? __ldg(g.sorted_slot + r) : -1;
+      }
+      if (it.valid) it.next(tl, x);
+    }
+  };
+  DwStageIt ld, wr;
+  ld.init(tl, x);
+  wr = ld;
+  int va[kIdxBatch][NQ], ra[kIdxBatch];
+  load_batch(ld, va, ra);
   Ring ri;
-  bool run = true;
-  for (int jt = 0, L = tl.tile(0); run && L < tl.total; L = tl.tile(++jt)) {
-    int e, mb, nb;
-    tl.coords(x, L, e, mb, nb);
-    const int r_begin = x.off[e], r_end = x.off[e + 1];
-    const int nK = cdiv(r_end - r_begin, BK);
-    for (int kb0 = 0; run && kb0 < nK; kb0 += kIdxBatch) {
-      int v[kIdxBatch][BK / 32];
-      float gv[kIdxBatch][BK / 32];
+  while (wr.valid) {
+    int vb[kIdxBatch][NQ], rbn[kIdxBatch];
+    load_batch(ld, vb, rbn);  // the next batch, in flight while this one is written
+    float gv[kIdxBatch][NQ];
 #pragma unroll
-      for (int b = 0; b < kIdxBatch; ++b)
+    for (int b = 0; b < kIdxBatch; ++b)
 #pragma unroll
-        for (int q = 0; q < BK / 32; ++q) {
-          const int r = r_begin + (kb0 + b) * BK + lane + 32 * q;
-          v[b][q] = (kb0 + b < nK && r < r_end) ? __ldg(g.sorted_slot + r) : -1;
-          gv[b][q] = 0.0f;
+      for (int q = 0; q < NQ; ++q) {
+        gv[b][q] = 0.0f;
+        if (A_SCALE) {
+          const int p = va[b][q];
+          if (p >= 0 && p < g.num_rows) gv[b][q] = __ldg(g.row_gates + p);
         }
-      if (A_SCALE) {  // the gates of those slots (a second dependent load per batch)
-#pragma unroll
-        for (int b = 0; b < kIdxBatch; ++b)
-#pragma unroll
-          for (int q = 0; q < BK / 32; ++q) {
-            const int p = v[b][q];
-            if (p >= 0 && p < g.num_rows) gv[b][q] = __ldg(g.row_gates + p);
-          }
       }
+    bool run = true;
 #pragma unroll
-      for (int b = 0; b < kIdxBatch; ++b) {
-        if (kb0 + b >= nK) break;
-        if (!mbar_wait(&c.iempty[ri.s], ri.ph ^ 1, abort_flag, g.err)) { run = false; break; }
+    for (int b = 0; b < kIdxBatch; ++b) {
+      if (!wr.valid) break;
+      if (!mbar_wait(&c.iempty[ri.s], ri.ph ^ 1, abort_flag, g.err)) { run = false; break; }
 #pragma unroll
-        for (int q = 0; q < BK / 32; ++q) {
-          const int r = r_begin + (kb0 + b) * BK + lane + 32 * q;
-          if (A_GATHER) {
-            int a_src;
-            if (A_SCALE && a_ident) a_src = (v[b][q] < 0 || r >= g.a_rows) ? -1 : r;
-            else a_src = src_of(v[b][q], a_shift, g.a_fan_out, g.a_rows);
-            x.idx[ri.s][0][lane + 32 * q] = a_src;
-          }
-          if (A_SCALE) x.gsc[ri.s][lane + 32 * q] = gv[b][q];
-          if (B_GATHER) x.idx[ri.s][1][lane + 32 * q] = src_of(v[b][q], b_shift, g.b_fan_out, g.b_rows);
+      for (int q = 0; q < NQ; ++q) {
+        const int r = ra[b] + lane + 32 * q;
+        if (A_GATHER) {
+          int a_src;
+          if (A_SCALE && a_ident) a_src = (va[b][q] < 0 || r >= g.a_rows) ? -1 : r;
+          else a_src = src_of(va[b][q], a_shift, g.a_fan_out, g.a_rows);
+          x.idx[ri.s][0][lane + 32 * q] = a_src;
         }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&c.ifull[ri.s]);
-        ri.next(IDX_STAGES);
+        if (A_SCALE) x.gsc[ri.s][lane + 32 * q] = gv[b][q];
+        if (B_GATHER) x.idx[ri.s][1][lane + 32 * q] = src_of(va[b][q], b_shift, g.b_fan_out, g.b_rows);
       }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&c.ifull[ri.s]);
+      ri.next(IDX_STAGES);
+      wr.next(tl, x);
+    }
+    if (!run) break;
+#pragma unroll
+    for (int b = 0; b < kIdxBatch; ++b) {
+      ra[b] = rbn[b];
+#pragma unroll
+      for (int q = 0; q < NQ; ++q) va[b][q] = vb[b][q];
     }
   }
 }
@@ -1908,17 +1956,6 @@ cudaError_t launch_dp(const CUtensorMap& tb, const CUtensorMap& td, int d_boxed,
   return cudaGetLastError();
 }
 
-// Whether the dW products whose gathered operand is on the A side run on CTA
-// pairs (SMOE_DW_PAIR=1 in the environment; read once).
-bool dw_pair_enabled() {
-  static int v = -1;
-  if (v < 0) {
-    const char* env = getenv("SMOE_DW_PAIR");
-    v = (env != nullptr && env[0] == '1') ? 1 : 0;
-  }
-  return v == 1;
-}
-
 }  // namespace
 
 bool tc_supported() {
@@ -2038,15 +2075,16 @@ cudaError_t launch_dw_gemm_tc(const DwGemm& g_in, cudaStream_t s) {
   const uint32_t dbox[3] = {32, 32, 1};
   const int d_boxed = make_map(&td, g.dw, 3, ddims, dstr, dbox, CU_TENSOR_MAP_SWIZZLE_128B,
                                CU_TENSOR_MAP_DATA_TYPE_FLOAT32) == cudaSuccess;
-  // CTA pairs: the A operand gathered, B by TMA, and at least two 128-column
-  // halves of M
-  if (dw_pair_enabled() && (ag || sc) && !bg && g.M > BM) {
+  // Gated rows with B by TMA and at least two 128-column halves of M run on CTA
+  // pairs: their six-stage rings keep more gathered stages in flight while the
+  // gate pass holds stages back (measured 9% faster than one CTA on the
+  // Mixtral-shaped dW2; without gates the pair measured the same as one CTA, so
+  // those keep the single-CTA kernel).
+  if (sc && !bg && g.M > BM) {
     const int nMP = cdiv(g.M, 2 * BM);
     const long long ptiles = (long long)g.E * nMP * nN;
-    if (sc) return trans ? launch_dp<true, true>(tb, td, d_boxed, g, nMP, nN, ptiles, s)
-                         : launch_dp<true, false>(tb, td, d_boxed, g, nMP, nN, ptiles, s);
-    return trans ? launch_dp<false, true>(tb, td, d_boxed, g, nMP, nN, ptiles, s)
-                 : launch_dp<false, false>(tb, td, d_boxed, g, nMP, nN, ptiles, s);
+    return trans ? launch_dp<true, true>(tb, td, d_boxed, g, nMP, nN, ptiles, s)
+                 : launch_dp<true, false>(tb, td, d_boxed, g, nMP, nN, ptiles, s);
   }
   const long long tiles = (long long)g.E * nM * nN;
   const int grid = (int)(tiles < num_sms() ? tiles : num_sms());

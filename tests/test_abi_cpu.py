@@ -150,9 +150,9 @@ def test_workspaces_hold_no_copy_of_token_rows():
     fwd = L.smoe_mlp_workspace_size(ctypes.byref(desc), 0)
     bwd = L.smoe_mlp_workspace_size(ctypes.byref(desc), 1)
     assert fwd == a256(sort) + a256(S * 4) + a256(S * d * 2)
-    # backward: dH [T*k, 2f] and the dx slot rows [T*k, d] (no gated copy of A: the
-    # gates multiply dY's gathered rows inside the dW2 kernel)
-    big = a256(S * 2 * f * 2) + a256(S * d * 2)
+    # backward: dH [T*k, 2f], g*A [T*k, f] (dW2's gated operand) and the dx slot
+    # rows [T*k, d]; the rest is small
+    big = a256(S * 2 * f * 2) + a256(S * f * 2) + a256(S * d * 2)
     assert 0 < bwd - big < S * d * 2 // 4
 
 

@@ -25,8 +25,8 @@ SHAPES = {torch.float32: dict(T=150, k=2, K=136, N=72, E=5),
           torch.bfloat16: dict(T=300, k=2, K=264, N=392, E=5)}
 
 
-def _problem(dtype, mode, gated, seed=0):
-    sh = SHAPES[dtype]
+def _problem(dtype, mode, gated, seed=0, shape=None):
+    sh = shape or SHAPES[dtype]
     T, k, K, N, E = sh["T"], sh["k"], sh["K"], sh["N"], sh["E"]
     gi, go, fo_k, comb = MODES[mode]
     g = torch.Generator(device="cuda").manual_seed(seed)
@@ -154,3 +154,22 @@ def test_parallel_linear_tile_boundaries(dtype, mode, gated):
 def test_parallel_linear_all_tokens_to_one_expert(dtype):
     dw = _check_problem(_sized_problem(dtype, "scatter2group_fanout", True, [0, 0, 300, 0]), dtype, True)
     assert np.all(dw[[0, 1, 3]].cpu().numpy() == 0.0)
+
+
+@pytest.mark.parametrize("mode", ["scatter2group_fanout", "group2scatter_combine", "group2group"])
+def test_parallel_linear_gated_dw_narrow(mode):
+    """Gated dW with a narrow output (K, N <= 128): the gate is applied by the
+    single-CTA dW kernel (wider products use the CTA-pair kernel), with the
+    gathered operand on either side and a grouped operand gathered row by row."""
+    P = _problem(torch.bfloat16, mode, True, seed=7, shape=dict(T=260, k=2, K=120, N=96, E=5))
+    dx, dw, dg = smoe.parallel_linear_bwd(P["dy"], P["x"], P["w"], P["ss"], P["off"], P["fan_out"],
+                                          P["gi"], P["go"], P["gates"], P["ck"], want_dgates=True)
+    torch.cuda.synchronize()
+    assert smoe.smoe_check() == 0
+    ref = oracle.pl_bwd(P["dy"].cpu(), P["x"].cpu(), P["w"].cpu(), P["ss"].cpu().numpy(),
+                        P["off"].cpu().numpy(), P["fan_out"], P["gi"], P["go"],
+                        P["gates"].cpu().double().numpy(), P["ck"], want_dg=True)
+    assert_close("dx", dx, ref["dx"], torch.bfloat16)
+    assert_close("dw", dw, ref["dw"], torch.bfloat16)
+    assert_close("dgates", dg, ref["dg"], torch.bfloat16)
+    assert np.all(dw[3].cpu().numpy() == 0.0)
