@@ -8,7 +8,7 @@ CUDA package.
 Every function takes CPU tensors or numpy arrays holding the stored values
 (float32, or bfloat16 as a torch tensor) and returns fp64 numpy arrays, except the
 integer routing outputs.  The definitions follow the ScatterMoE pages as listed
-in the header of ``smoe_oracle.cpp`` (readings R1-R6 there).
+in the header of ``smoe_oracle.cpp`` (readings R1-R7 there).
 
 Parity status: every function here is pinned by ``tests/test_oracle_pins.py``
 against independent mathematics (brute force, closed forms, library routines,
@@ -188,6 +188,41 @@ def route_bwd(x, w_r, topk_idx, gates, dgates):
            "db_r": np.empty(E)}
     lib.oracle_route_bwd(_p(xs), _p(ws), dt, T, d, E, k, _p(idx), _p(g), _p(dg), _p(out["dl"]),
                          _p(out["dx"]), _p(out["dw_r"]), _p(out["db_r"]))
+    return out
+
+
+def moa_attn(q, k, v, sorted_slot, kslots, L, heads, dout=None, q_rows=None, kv_tokens=None,
+             want_dkv=True):
+    """Mixture-of-Attention core (R7): {"o", "lse"} for grouped rows ``q_rows`` (all if
+    None); with ``dout`` also "dq" for those rows and, when ``want_dkv``, "dk", "dv"
+    for tokens ``kv_tokens`` (all if None).  All fp64."""
+    lib = _load()
+    qs, dt = _stored(q)
+    ks, dtk = _stored(k)
+    vs, dtv = _stored(v)
+    assert dt == dtk == dtv
+    ds = None
+    if dout is not None:
+        ds, dtd = _stored(dout)
+        assert dtd == dt
+    S, W = qs.shape
+    T = ks.shape[0]
+    dh = W // heads
+    ss = _i32(sorted_slot)
+    assert ss.size == S == T * kslots
+    rows = None if q_rows is None else _i32(np.asarray(q_rows, np.int32))
+    nq = S if rows is None else rows.size
+    toks = None if kv_tokens is None else _i32(np.asarray(kv_tokens, np.int32))
+    nkv = 0 if (dout is None or not want_dkv) else (T if toks is None else toks.size)
+    out = {"o": np.empty((nq, W)), "lse": np.empty((nq, heads))}
+    if dout is not None:
+        out["dq"] = np.empty((nq, W))
+        if want_dkv:
+            out["dk"] = np.empty((nkv, W))
+            out["dv"] = np.empty((nkv, W))
+    lib.oracle_moa_attn(_p(qs), _p(ks), _p(vs), _p(ds), dt, _p(ss), T, kslots, L, heads, dh,
+                        _p(rows), nq, _p(toks), nkv, _p(out["o"]), _p(out["lse"]),
+                        _p(out.get("dq")), _p(out.get("dk")), _p(out.get("dv")))
     return out
 
 

@@ -37,6 +37,9 @@
  *      (scattered); the product v = x_row W[e] goes to row i (grouped), row p
  *      (scattered), or is summed into row p / combine_k (k-way combine),
  *      multiplied by gates[p] when gates are given.
+ *   R7 Mixture-of-Attention core (see oracle_moa_attn): per-expert queries in
+ *      grouped order attend causally, within each sequence of L tokens, to keys
+ *      and values shared by all experts, head by head.
  *
  * Every input array is passed as its stored values (fp32, or bf16 bit patterns)
  * and upcast exactly to fp64.  All arithmetic below is fp64 except the fp32
@@ -646,6 +649,143 @@ void oracle_route_bwd(const void* x, const void* w_r, int dt, int T, int d, int 
       for (int i = 0; i < d; ++i) dw_r[(size_t)i * E + e] += load_any(x, dt, (size_t)t * d + i) * v;
     }
     db_r[e] = b;
+  }
+}
+
+/* R7: the Mixture-of-Attention core between the per-expert query projection and
+ * the per-expert output projection (arXiv abstract: ParallelLinear extended to
+ * Mixture of Attention; tradepoint.io article, method paragraph: MoA without
+ * additional memory costs).  Reading: the T tokens form T / L sequences of L
+ * consecutive tokens; slot p = t*kslots + j holds the query of token t for its
+ * j-th selected expert, in grouped order (row inv[p] of q and o, inv the inverse
+ * of sorted_slot); each of the `heads` heads of width dh attends causally, within
+ * the token's sequence, to the shared keys and values of that head:
+ *   s_u   = <q[inv[p], head a], k[u, head a]> / sqrt(dh)      for u in [t0, t]
+ *   o[inv[p], head a] = sum_u softmax(s)_u v[u, head a],  lse = log sum_u exp(s_u)
+ * (t0 = the first token of t's sequence).  Backward of L = <o, dout>:
+ *   P_u = exp(s_u - lse), dP_u = <dout, v_u>, D = <dout, o> = sum_u P_u dP_u,
+ *   dS_u = P_u (dP_u - D);  dq = sum_u dS_u k_u / sqrt(dh);
+ *   dk_u += dS_u q / sqrt(dh);  dv_u += P_u dout      (summed over all queries).
+ * q, dout: [T*kslots, heads*dh] grouped; k, v: [T, heads*dh] token order; all in
+ * the stored dtype dt.  q_rows (nullable = all grouped rows): rows of o, lse, dq;
+ * kv_tokens (nullable = all tokens, ignored when n_kv == 0): rows of dk, dv.
+ * dout == null: forward only.                                                */
+void oracle_moa_attn(const void* q, const void* k, const void* v, const void* dout, int dt,
+                     const int32_t* sorted_slot, int T, int kslots, int L, int heads, int dh,
+                     const int32_t* q_rows, int n_q, const int32_t* kv_tokens, int n_kv, double* o,
+                     double* lse, double* dq, double* dk, double* dv) {
+  const int S = T * kslots, W = heads * dh;
+  const double scale = 1.0 / std::sqrt((double)dh);
+  std::vector<int32_t> inv(S);
+  for (int i = 0; i < S; ++i) inv[sorted_slot[i]] = i;
+  auto Q = [&](int row, int a, int c) { return load_any(q, dt, (size_t)row * W + a * dh + c); };
+  auto Kv = [&](int u, int a, int c) { return load_any(k, dt, (size_t)u * W + a * dh + c); };
+  auto Vv = [&](int u, int a, int c) { return load_any(v, dt, (size_t)u * W + a * dh + c); };
+  auto G = [&](int row, int a, int c) { return load_any(dout, dt, (size_t)row * W + a * dh + c); };
+  /* scores of grouped row `row`, head a, over its causal window, into s; returns t0 */
+  auto scores = [&](int row, int a, std::vector<double>& s, int& t_lo, int& t_hi) {
+    const int t = sorted_slot[row] / kslots;
+    t_lo = (t / L) * L;
+    t_hi = t;
+    s.assign(t_hi - t_lo + 1, 0.0);
+    for (int u = t_lo; u <= t_hi; ++u) {
+      double acc = 0.0;
+      for (int c = 0; c < dh; ++c) acc += Q(row, a, c) * Kv(u, a, c);
+      s[u - t_lo] = acc * scale;
+    }
+  };
+  /* softmax of the window in place, returning lse */
+  auto softmax = [&](std::vector<double>& s) {
+    double m = s[0];
+    for (double x : s) m = std::max(m, x);
+    double z = 0.0;
+    for (double& x : s) { x = std::exp(x - m); z += x; }
+    for (double& x : s) x /= z;
+    return m + std::log(z);
+  };
+  const bool all_q = q_rows == nullptr;
+  const int nq = all_q ? S : n_q;
+  /* forward rows and dq */
+#pragma omp parallel for schedule(dynamic, 4)
+  for (int qi = 0; qi < nq; ++qi) {
+    const int row = all_q ? qi : q_rows[qi];
+    std::vector<double> s;
+    for (int a = 0; a < heads; ++a) {
+      int t_lo, t_hi;
+      scores(row, a, s, t_lo, t_hi);
+      const double ls = softmax(s);
+      if (lse) lse[(size_t)qi * heads + a] = ls;
+      std::vector<double> orow(dh, 0.0);
+      for (int u = t_lo; u <= t_hi; ++u)
+        for (int c = 0; c < dh; ++c) orow[c] += s[u - t_lo] * Vv(u, a, c);
+      if (o)
+        for (int c = 0; c < dh; ++c) o[(size_t)qi * W + a * dh + c] = orow[c];
+      if (dout && dq) {
+        double D = 0.0;
+        for (int c = 0; c < dh; ++c) D += G(row, a, c) * orow[c];
+        double* dqr = dq + (size_t)qi * W + a * dh;
+        for (int c = 0; c < dh; ++c) dqr[c] = 0.0;
+        for (int u = t_lo; u <= t_hi; ++u) {
+          double dP = 0.0;
+          for (int c = 0; c < dh; ++c) dP += G(row, a, c) * Vv(u, a, c);
+          const double dS = s[u - t_lo] * (dP - D);
+          for (int c = 0; c < dh; ++c) dqr[c] += dS * Kv(u, a, c) * scale;
+        }
+      }
+    }
+  }
+  if (!dout || n_kv == 0 || (!dk && !dv)) return;
+  /* dk, dv: every query of the listed tokens' sequences contributes; its lse and
+   * D = <dout, o> are computed once per (grouped row, head) */
+  const bool all_kv = kv_tokens == nullptr;
+  const int nkv = all_kv ? T : n_kv;
+  std::vector<char> need_seq((T + L - 1) / L, 0);
+  for (int ti = 0; ti < nkv; ++ti) need_seq[(all_kv ? ti : kv_tokens[ti]) / L] = 1;
+  std::vector<double> lse_all((size_t)S * heads, 0.0), D_all((size_t)S * heads, 0.0);
+#pragma omp parallel for schedule(dynamic, 4)
+  for (int row = 0; row < S; ++row) {
+    const int t = sorted_slot[row] / kslots;
+    if (!need_seq[t / L]) continue;
+    std::vector<double> s;
+    for (int a = 0; a < heads; ++a) {
+      int t_lo, t_hi;
+      scores(row, a, s, t_lo, t_hi);
+      lse_all[(size_t)row * heads + a] = softmax(s);
+      double D = 0.0;
+      for (int c = 0; c < dh; ++c) {
+        double oc = 0.0;
+        for (int u = t_lo; u <= t_hi; ++u) oc += s[u - t_lo] * Vv(u, a, c);
+        D += G(row, a, c) * oc;
+      }
+      D_all[(size_t)row * heads + a] = D;
+    }
+  }
+#pragma omp parallel for schedule(dynamic, 1)
+  for (int ti = 0; ti < nkv; ++ti) {
+    const int u = all_kv ? ti : kv_tokens[ti];
+    const int seq_end = std::min(T, (u / L + 1) * L);
+    for (int a = 0; a < heads; ++a) {
+      std::vector<double> dkr(dh, 0.0), dvr(dh, 0.0);
+      for (int t = u; t < seq_end; ++t)
+        for (int j = 0; j < kslots; ++j) {
+          const int row = inv[(size_t)t * kslots + j];
+          double sc = 0.0, dP = 0.0;
+          for (int c = 0; c < dh; ++c) {
+            sc += Q(row, a, c) * Kv(u, a, c);
+            dP += G(row, a, c) * Vv(u, a, c);
+          }
+          const double P = std::exp(sc * scale - lse_all[(size_t)row * heads + a]);
+          const double dS = P * (dP - D_all[(size_t)row * heads + a]);
+          for (int c = 0; c < dh; ++c) {
+            dkr[c] += dS * Q(row, a, c) * scale;
+            dvr[c] += P * G(row, a, c);
+          }
+        }
+      for (int c = 0; c < dh; ++c) {
+        if (dk) dk[(size_t)ti * W + a * dh + c] = dkr[c];
+        if (dv) dv[(size_t)ti * W + a * dh + c] = dvr[c];
+      }
+    }
   }
 }
 

@@ -488,3 +488,89 @@ def test_mlp_equals_parallel_linear_composition():
     Y = oracle.pl_fwd(A, w2.double(), ss, off, 1, 1, 0, gates.ravel(), 2)
     np.testing.assert_allclose(Y, oracle.mlp_fwd(x, w1, w2, "gelu", idx, gates)["y"], rtol=1e-12,
                                atol=1e-12)
+
+
+# --------------------------------------------------------------------------
+# Mixture-of-Attention core (grouped per-expert queries, shared keys/values)
+# --------------------------------------------------------------------------
+def _moa_problem(seed, T, L, kslots, E, heads, dh, dtype=torch.float64):
+    g = torch.Generator().manual_seed(seed)
+    idx = torch.stack([torch.randperm(E, generator=g)[:kslots] for _ in range(T)]).int().numpy()
+    ss, _ = oracle.sort(idx, E)
+    W = heads * dh
+    q = torch.randn(T * kslots, W, generator=g, dtype=torch.float64).to(dtype)
+    k = torch.randn(T, W, generator=g, dtype=torch.float64).to(dtype)
+    v = torch.randn(T, W, generator=g, dtype=torch.float64).to(dtype)
+    dout = torch.randn(T * kslots, W, generator=g, dtype=torch.float64).to(dtype)
+    return ss, q, k, v, dout
+
+
+def test_moa_attn_equals_torch_sdpa():
+    """Every query row against torch's scaled-dot-product attention (fp64, CPU) with
+    an explicit mask: query (t, j) sees the keys of its own sequence up to t."""
+    T, L, kslots, E, heads, dh = 12, 6, 3, 5, 2, 8
+    ss, q, k, v, _ = _moa_problem(3, T, L, kslots, E, heads, dh)
+    out = oracle.moa_attn(q, k, v, ss, kslots, L, heads)
+    S = T * kslots
+    tok = torch.from_numpy(ss.astype(np.int64)) // kslots          # token of grouped row i
+    mask = (torch.arange(T)[None, :] <= tok[:, None]) & (torch.arange(T)[None, :] // L == tok[:, None] // L)
+    qh = q.view(S, heads, dh).transpose(0, 1)                      # [heads, S, dh]
+    kh = k.view(T, heads, dh).transpose(0, 1)
+    vh = v.view(T, heads, dh).transpose(0, 1)
+    ref = F.scaled_dot_product_attention(qh, kh, vh, attn_mask=mask[None])  # [heads, S, dh]
+    ref = ref.transpose(0, 1).reshape(S, heads * dh).numpy()
+    np.testing.assert_allclose(out["o"], ref, rtol=1e-12, atol=1e-12)
+    s = torch.einsum("hid,hjd->hij", qh, kh) / dh ** 0.5
+    lse = torch.logsumexp(s.masked_fill(~mask[None], -torch.inf), dim=-1).T.numpy()
+    np.testing.assert_allclose(out["lse"], lse, rtol=1e-12, atol=1e-12)
+
+
+def test_moa_attn_backward_finite_differences():
+    T, L, kslots, E, heads, dh = 6, 3, 2, 3, 2, 4
+    ss, q, k, v, dout = _moa_problem(5, T, L, kslots, E, heads, dh)
+    an = oracle.moa_attn(q, k, v, ss, kslots, L, heads, dout=dout)
+
+    def loss():
+        return float((oracle.moa_attn(q, k, v, ss, kslots, L, heads)["o"] * dout.numpy()).sum())
+
+    h = 1e-6
+    for name, tensor, key in (("q", q, "dq"), ("k", k, "dk"), ("v", v, "dv")):
+        flat = tensor.view(-1)
+        fd = np.zeros(tensor.numel())
+        for i in range(tensor.numel()):
+            old = float(flat[i])
+            flat[i] = old + h
+            lp = loss()
+            flat[i] = old - h
+            lm = loss()
+            flat[i] = old
+            fd[i] = (lp - lm) / (2 * h)
+        ref = an[key].ravel()
+        assert np.max(np.abs(fd - ref)) / np.max(np.abs(ref)) < 1e-6, name
+
+
+def test_moa_attn_single_token_sequences_and_subsets():
+    """L = 1: every query sees only its own token, so o = v[t] exactly, lse = <q, k_t>/sqrt(dh),
+    dq = dk = 0 and dv[t] = the sum of dout over the token's k slots.  Row and token
+    subsets of a longer problem equal the full computation."""
+    T, kslots, E, heads, dh = 7, 2, 4, 2, 4
+    ss, q, k, v, dout = _moa_problem(8, T, 1, kslots, E, heads, dh)
+    out = oracle.moa_attn(q, k, v, ss, kslots, 1, heads, dout=dout)
+    tok = ss // kslots
+    np.testing.assert_array_equal(out["o"], v.numpy()[tok])
+    qh = q.numpy().reshape(-1, heads, dh)
+    kh = k.numpy().reshape(-1, heads, dh)[tok]
+    np.testing.assert_allclose(out["lse"], (qh * kh).sum(-1) / dh ** 0.5, rtol=1e-13, atol=1e-13)
+    assert np.all(out["dq"] == 0) and np.all(out["dk"] == 0)
+    dv = np.zeros((T, heads * dh))
+    np.add.at(dv, tok, dout.numpy())
+    np.testing.assert_allclose(out["dv"], dv, rtol=1e-13, atol=1e-13)
+    T, L = 16, 8
+    ss, q, k, v, dout = _moa_problem(9, T, L, kslots, E, heads, dh)
+    full = oracle.moa_attn(q, k, v, ss, kslots, L, heads, dout=dout)
+    rows, toks = np.array([0, 5, 31, 17], np.int32), np.array([15, 0, 8, 3], np.int32)
+    sub = oracle.moa_attn(q, k, v, ss, kslots, L, heads, dout=dout, q_rows=rows, kv_tokens=toks)
+    for key in ("o", "lse", "dq"):
+        np.testing.assert_allclose(sub[key], full[key][rows], rtol=1e-12, atol=1e-13)
+    for key in ("dk", "dv"):
+        np.testing.assert_allclose(sub[key], full[key][toks], rtol=1e-12, atol=1e-13)
