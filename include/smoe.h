@@ -242,6 +242,40 @@ int parallel_linear_bwd(const void* dy, const void* x, const void* w, int x_rows
                         smoe_dtype dt, void* workspace, size_t ws_bytes, void* stream);
 
 /* ---------------------------------------------------------------------------
+ * Mixture-of-Attention core [abs: ParallelLinear extended to Mixture of
+ * Attention; art, method paragraph: MoA without additional memory costs]
+ *
+ * The attention between the per-expert query projection (ParallelLinear,
+ * scatter->group, fan_out kslots) and the per-expert output projection
+ * (group->scatter with the gated k-way combine).  The pages give no formula; this
+ * library's reading: the T tokens form sequences of L consecutive tokens (the
+ * last may be shorter); keys and values are shared by all experts; slot
+ * p = t*kslots + j holds token t's query for its j-th selected expert, in grouped
+ * order (row i with sorted_slot[i] = p); for every head h of width head_dim:
+ *   o[i, h] = sum_u softmax_u(<q[i, h], k[u, h]> / sqrt(head_dim)) v[u, h]
+ * over u from the first token of t's sequence to t (causal), and
+ *   lse[i, h] = log sum_u exp(<q[i, h], k[u, h]> / sqrt(head_dim)).
+ *   q, o [T*kslots, heads*head_dim] dtype, grouped rows;  k, v [T, heads*head_dim]
+ *   dtype, token order;  lse [T*kslots, heads] fp32.  Columns of head h are
+ *   [h*head_dim, (h+1)*head_dim).
+ * No grouped copy is made: the kernels gather query rows through sorted_slot.
+ * Requires dt == SMOE_BF16 and head_dim == 128 (else SMOE_ERR_UNSUPPORTED);
+ * 1 <= kslots <= 128; L >= 1.  workspace: smoe_moa_attn_workspace_size(T, kslots,
+ * heads, backward) bytes, 256-byte aligned (the inverse of sorted_slot, and for
+ * the backward D = <dO, O> per row and head).
+ * Backward of L = <o, dout>: dq (grouped, like q), dk and dv (token order, like
+ * k and v), all overwritten, dtype; summed in a fixed order (no atomics).
+ * ------------------------------------------------------------------------ */
+size_t smoe_moa_attn_workspace_size(int T, int kslots, int heads, int backward);
+int smoe_moa_attn_fwd(const void* q, const void* k, const void* v, const int32_t* sorted_slot, int T,
+                      int L, int kslots, int heads, int head_dim, smoe_dtype dt, void* o, float* lse,
+                      void* workspace, size_t ws_bytes, void* stream);
+int smoe_moa_attn_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                      const void* dout, const int32_t* sorted_slot, int T, int L, int kslots, int heads,
+                      int head_dim, smoe_dtype dt, void* dq, void* dk, void* dv, void* workspace,
+                      size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------
  * SMoE MLP [abs, art: SMoE layer = top-k routing + weighted sum of expert MLPs]
  *
  * Forward: route, sort, H = ParallelLinear(x, W1; scatter->group, fan_out k),

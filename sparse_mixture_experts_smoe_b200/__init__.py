@@ -80,6 +80,10 @@ def lib():
     L.parallel_linear_bwd.argtypes = [_vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _vp, _vp,
                                       _c_int, _c_int, _c_int, _c_int, _vp, _c_int, _vp, _vp, _vp,
                                       _c_int, _vp, _c_size, _vp]
+    L.smoe_moa_attn_workspace_size.restype = _c_size
+    L.smoe_moa_attn_workspace_size.argtypes = [_c_int] * 4
+    L.smoe_moa_attn_fwd.argtypes = [_vp, _vp, _vp, _vp] + [_c_int] * 6 + [_vp, _vp, _vp, _c_size, _vp]
+    L.smoe_moa_attn_bwd.argtypes = [_vp] * 7 + [_c_int] * 6 + [_vp] * 4 + [_c_size, _vp]
     L.smoe_mlp_workspace_size.restype = _c_size
     L.smoe_mlp_workspace_size.argtypes = [ctypes.POINTER(MlpDesc), _c_int]
     L.smoe_mlp_fwd.argtypes = [ctypes.POINTER(MlpDesc), ctypes.POINTER(MlpTensors), _vp]
@@ -270,6 +274,40 @@ def parallel_linear_bwd(dy, x, w, sorted_slot, expert_offsets, fan_out, grouped_
                                      int(grouped_out), _ptr(gates), combine_k, _ptr(dx), _ptr(dw),
                                      _ptr(dg), _dt(x), _ptr(ws), ws.numel(), _stream(stream)))
     return dx, dw, dg
+
+
+def smoe_moa_attn_fwd(q, k, v, sorted_slot, kslots, L, heads, stream=None):
+    """Mixture-of-Attention core forward: (o [T*kslots, heads*dh] grouped like q,
+    lse [T*kslots, heads] fp32)."""
+    S, W = q.shape
+    T = k.shape[0]
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _need(t, n, q.dtype)
+    _need(sorted_slot, "sorted_slot", torch.int32, (S,))
+    o = torch.empty_like(q)
+    lse = torch.empty((S, heads), dtype=torch.float32, device=q.device)
+    ws = _workspace(lib().smoe_moa_attn_workspace_size(T, kslots, heads, 0), q.device)
+    _check(lib().smoe_moa_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(sorted_slot), T, L, kslots, heads,
+                                   W // heads, _dt(q), _ptr(o), _ptr(lse), _ptr(ws), ws.numel(),
+                                   _stream(stream)))
+    return o, lse
+
+
+def smoe_moa_attn_bwd(q, k, v, o, lse, dout, sorted_slot, kslots, L, heads, stream=None):
+    """Mixture-of-Attention core backward: (dq grouped like q, dk, dv like k, v)."""
+    S, W = q.shape
+    T = k.shape[0]
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o"), (dout, "dout")):
+        _need(t, n, q.dtype)
+    _need(lse, "lse", torch.float32, (S, heads))
+    _need(sorted_slot, "sorted_slot", torch.int32, (S,))
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ws = _workspace(lib().smoe_moa_attn_workspace_size(T, kslots, heads, 1), q.device)
+    _check(lib().smoe_moa_attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dout),
+                                   _ptr(sorted_slot), T, L, kslots, heads, W // heads, _dt(q),
+                                   _ptr(dq), _ptr(dk), _ptr(dv), _ptr(ws), ws.numel(),
+                                   _stream(stream)))
+    return dq, dk, dv
 
 
 class SMoEMLPState:

@@ -642,6 +642,87 @@ int parallel_linear_bwd(const void* dy, const void* x, const void* w, int x_rows
 }
 
 // ---------------------------------------------------------------------------
+// Mixture-of-Attention core
+// ---------------------------------------------------------------------------
+static size_t moa_ws_bytes(int T, int kslots, int heads, int backward) {
+  const size_t S = (size_t)T * kslots;
+  return align256(S * sizeof(int32_t)) + (backward ? align256(S * heads * sizeof(float)) : 0);
+}
+
+static int validate_moa(int T, int L, int kslots, int heads, int head_dim, int dt) {
+  if (T < 0 || L < 1 || kslots < 1 || kslots > 128 || heads < 1)
+    return fail(SMOE_ERR_INVALID_ARG, "bad sizes (T >= 0, L >= 1, 1 <= kslots <= 128, heads >= 1)");
+  if (!slots_fit(T, kslots) || (long long)T * kslots * heads * head_dim >= (1LL << 31))
+    return fail(SMOE_ERR_INVALID_ARG, "tensor too large for 32-bit row indexing");
+  if (!valid_dtype(dt)) return fail(SMOE_ERR_INVALID_ARG, "bad dtype");
+  if (dt != SMOE_BF16) return fail(SMOE_ERR_UNSUPPORTED, "the attention core is bf16 only");
+  if (head_dim != attn_head_dim())
+    return fail(SMOE_ERR_UNSUPPORTED, "head_dim must be %d", attn_head_dim());
+  return SMOE_OK;
+}
+
+size_t smoe_moa_attn_workspace_size(int T, int kslots, int heads, int backward) {
+  if (T < 0 || kslots < 1 || heads < 1 || !slots_fit(T, kslots)) return 0;
+  return moa_ws_bytes(T, kslots, heads, backward);
+}
+
+int smoe_moa_attn_fwd(const void* q, const void* k, const void* v, const int32_t* sorted_slot, int T,
+                      int L, int kslots, int heads, int head_dim, smoe_dtype dt, void* o, float* lse,
+                      void* workspace, size_t ws_bytes, void* stream) {
+  smoe::NvtxScope nvtx_scope("smoe_moa_attn_fwd");
+  int rc = validate_moa(T, L, kslots, heads, head_dim, dt);
+  if (rc != SMOE_OK) return rc;
+  if (T == 0) return SMOE_OK;
+  NEED(q, "q"); NEED(k, "k"); NEED(v, "v"); NEED(sorted_slot, "sorted_slot"); NEED(o, "o");
+  NEED(lse, "lse");
+  ALIGNED(q, "q"); ALIGNED(k, "k"); ALIGNED(v, "v"); ALIGNED(o, "o");
+  const size_t need = moa_ws_bytes(T, kslots, heads, 0);
+  if (!workspace || ws_bytes < need)
+    return fail(SMOE_ERR_INVALID_ARG, "workspace too small (%zu < %zu)", ws_bytes, need);
+  if ((rc = check_tc(dt)) != SMOE_OK) return rc;
+  cudaError_t st;
+  unsigned* err = error_word(&st);
+  if (!err) return cuda_fail(st, "smoe_moa_attn_fwd");
+  cudaStream_t s = (cudaStream_t)stream;
+  int32_t* inv = (int32_t*)workspace;
+  { PROF("moa.invert", 1); SMOE_TRY(launch_invert(sorted_slot, T * kslots, inv, s), "moa invert"); }
+  { PROF("moa.attn_fwd", 1);
+    SMOE_TRY(launch_moa_attn_fwd(q, k, v, inv, T, L, kslots, heads, o, lse, err, s), "moa attn fwd"); }
+  return SMOE_OK;
+}
+
+int smoe_moa_attn_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                      const void* dout, const int32_t* sorted_slot, int T, int L, int kslots, int heads,
+                      int head_dim, smoe_dtype dt, void* dq, void* dk, void* dv, void* workspace,
+                      size_t ws_bytes, void* stream) {
+  smoe::NvtxScope nvtx_scope("smoe_moa_attn_bwd");
+  int rc = validate_moa(T, L, kslots, heads, head_dim, dt);
+  if (rc != SMOE_OK) return rc;
+  if (T == 0) return SMOE_OK;
+  NEED(q, "q"); NEED(k, "k"); NEED(v, "v"); NEED(o, "o"); NEED(lse, "lse"); NEED(dout, "dout");
+  NEED(sorted_slot, "sorted_slot"); NEED(dq, "dq"); NEED(dk, "dk"); NEED(dv, "dv");
+  ALIGNED(q, "q"); ALIGNED(k, "k"); ALIGNED(v, "v"); ALIGNED(o, "o"); ALIGNED(dout, "dout");
+  ALIGNED(dq, "dq"); ALIGNED(dk, "dk"); ALIGNED(dv, "dv");
+  const size_t need = moa_ws_bytes(T, kslots, heads, 1);
+  if (!workspace || ws_bytes < need)
+    return fail(SMOE_ERR_INVALID_ARG, "workspace too small (%zu < %zu)", ws_bytes, need);
+  if (((uintptr_t)workspace & 255u) != 0) return fail(SMOE_ERR_INVALID_ARG, "workspace not 256-byte aligned");
+  if ((rc = check_tc(dt)) != SMOE_OK) return rc;
+  cudaError_t st;
+  unsigned* err = error_word(&st);
+  if (!err) return cuda_fail(st, "smoe_moa_attn_bwd");
+  cudaStream_t s = (cudaStream_t)stream;
+  const size_t S = (size_t)T * kslots;
+  int32_t* inv = (int32_t*)workspace;
+  float* dsum = (float*)((char*)workspace + align256(S * sizeof(int32_t)));
+  { PROF("moa.invert", 1); SMOE_TRY(launch_invert(sorted_slot, (int)S, inv, s), "moa invert"); }
+  { PROF("moa.attn_bwd", 4);
+    SMOE_TRY(launch_moa_attn_bwd(q, k, v, o, lse, dout, inv, T, L, kslots, heads, dq, dk, dv, dsum, err, s),
+             "moa attn bwd"); }
+  return SMOE_OK;
+}
+
+// ---------------------------------------------------------------------------
 // SMoE MLP
 // ---------------------------------------------------------------------------
 size_t smoe_mlp_workspace_size(const smoe_mlp_desc* desc, int backward) {

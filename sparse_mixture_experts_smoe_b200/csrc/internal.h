@@ -134,6 +134,18 @@ int grouped_ksplit(int num_rows, int E, int n_out, int K);
 cudaError_t launch_grouped_gemm_simt(const GroupedGemm& g, smoe_dtype dt, cudaStream_t s);
 cudaError_t launch_dw_gemm_simt(const DwGemm& g, smoe_dtype dt, cudaStream_t s);
 
+// Mixture-of-Attention core (attn_tc.cu, bf16, head width attn_head_dim()):
+// q/o/dout grouped [T*kslots, heads*128], k/v [T, heads*128], inv the grouped row
+// of each slot; lse [T*kslots, heads] fp32; dsum scratch [T*kslots, heads] fp32.
+int attn_head_dim();
+cudaError_t launch_moa_attn_fwd(const void* q, const void* k, const void* v, const int32_t* inv, int T,
+                                int L, int kslots, int heads, void* o, float* lse, unsigned* err,
+                                cudaStream_t s);
+cudaError_t launch_moa_attn_bwd(const void* q, const void* k, const void* v, const void* o,
+                                const float* lse, const void* dout, const int32_t* inv, int T, int L,
+                                int kslots, int heads, void* dq, void* dk, void* dv, float* dsum,
+                                unsigned* err, cudaStream_t s);
+
 // tcgen05 / TMEM path (bf16 only); *_supported() checks the device once.
 bool tc_supported();
 cudaError_t launch_grouped_gemm_tc(const GroupedGemm& g, cudaStream_t s);

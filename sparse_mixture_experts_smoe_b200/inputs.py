@@ -25,6 +25,9 @@ b_r[e] = -s * ln(r_e) for r_e <= E - n_empty and -1e4 otherwise, so exactly
 Mixture-of-Attention projections: x [T, d]; Wq [E, d, h] ~ N(0, 1/d);
 Wo [E, h, d] ~ N(0, 1/h); per-slot attention output o [T*k, h] ~ N(0, 1) in
 grouped order; upstream gradients dz [T, d] and dq [T*k, h] ~ N(0, 1).
+Mixture-of-Attention core: the T tokens are sequences of L = 2048 tokens; queries
+q [T*k, h] (grouped), shared keys and values k, v [T, h] and the upstream
+gradient do [T*k, h] ~ N(0, 1); h = heads * 128 with heads = 4.
 """
 from __future__ import annotations
 
@@ -41,11 +44,11 @@ WORKLOADS = {
                                 act="swiglu"),
     "finegrained_zipf_bf16_swiglu": dict(kind="mlp", T=16384, d=2048, f=512, E=64, k=8,
                                          dtype="bf16", act="swiglu", zipf_s=1.2, n_empty=4),
-    "moa_bf16": dict(kind="moa", T=8192, d=2048, E=16, k=4, h=512, dtype="bf16"),
+    "moa_bf16": dict(kind="moa", T=8192, d=2048, E=16, k=4, h=512, dtype="bf16", L=2048, heads=4),
 }
 
 _STREAM = {"x": 1, "w_r": 2, "w1": 3, "w2": 4, "dy": 5, "perm": 6, "wq": 7, "wo": 8, "o": 9,
-           "dz": 10, "dq": 11, "dg": 12}
+           "dz": 10, "dq": 11, "dg": 12, "aq": 13, "ak": 14, "av": 15, "ado": 16}
 
 
 def torch_dtype(name: str) -> torch.dtype:
@@ -123,6 +126,37 @@ def make_moa_inputs(cfg: dict, seed: int = 0, device="cpu") -> dict:
         "dz": _randn((T, d), 1.0, "dz", seed, device, dt),
         "dq": _randn((T * k, h), 1.0, "dq", seed, device, dt),
     }
+
+
+def make_moa_attn_inputs(cfg: dict, seed: int = 0, device="cpu") -> dict:
+    """Inputs of the Mixture-of-Attention core at a workload's sizes: x and W_r (the
+    router, as in ``make_moa_inputs``), per-slot queries q [T*k, h] in grouped order,
+    shared keys and values k, v [T, h] and the upstream gradient do [T*k, h], all
+    N(0, 1) in bf16 (h = heads * 128)."""
+    T, d, E, k, h = cfg["T"], cfg["d"], cfg["E"], cfg["k"], cfg["h"]
+    dt = torch_dtype(cfg["dtype"])
+    return {
+        "x": _randn((T, d), 1.0, "x", seed, device, dt),
+        "w_r": _randn((d, E), 1.0 / math.sqrt(d), "w_r", seed, device, dt),
+        "q": _randn((T * k, h), 1.0, "aq", seed, device, dt),
+        "k": _randn((T, h), 1.0, "ak", seed, device, dt),
+        "v": _randn((T, h), 1.0, "av", seed, device, dt),
+        "do": _randn((T * k, h), 1.0, "ado", seed, device, dt),
+    }
+
+
+def moa_attn_flops(cfg: dict) -> dict:
+    """Algorithmic FLOPs of the causal attention core: per head and query row, two
+    products of width 128 over its window (scores and P V), the window of query
+    token t being t - (sequence start) + 1 keys; backward = 2.5 x forward (dS K,
+    dP = dO V^T, dV, dK plus the score recomputation)."""
+    T, k, heads, L = cfg["T"], cfg["k"], cfg["heads"], cfg["L"]
+    keys = 0
+    for s0 in range(0, T, L):
+        n = min(L, T - s0)
+        keys += n * (n + 1) // 2  # sum of window lengths over the sequence's tokens
+    fwd = 2.0 * 2 * 128 * keys * k * heads
+    return {"fwd": fwd, "bwd": 2.5 * fwd, "fwd_bwd": 3.5 * fwd}
 
 
 def mlp_flops(cfg: dict) -> dict:
