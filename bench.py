@@ -36,10 +36,10 @@ import numpy as np  # noqa: E402
 import torch  # noqa: E402
 
 from sparse_mixture_experts_smoe_b200.inputs import (  # noqa: E402
-    WORKLOADS, make_mlp_inputs, make_moa_inputs, mlp_flops)
+    WORKLOADS, make_mlp_inputs, make_moa_inputs, mlp_flops, moa_attn_flops)
 
 METRIC = "SMoE MLP fwd+bwd tokens/s on 1 B200; % of dense BF16 tensor peak"
-METRIC_MOA = "MoA expert projections (Wq scatter->group, Wo group->scatter + gated combine) fwd+bwd tokens/s on 1 B200"
+METRIC_MOA = "Mixture-of-Attention layer (router, per-expert Wq/Wo, shared Wk/Wv, causal attention core) fwd+bwd tokens/s on 1 B200"
 # NVIDIA's nominal dense (no 2:4 sparsity) bf16 tensor throughput of one B200.
 NOMINAL_DENSE_BF16_TFLOPS = 2250.0
 DEFAULT_WORKLOAD = "mixtral_bf16_swiglu"
@@ -291,70 +291,136 @@ def run_reference(args, world, rank):
 # our path
 # ---------------------------------------------------------------------------
 def moa_oracle_baseline(cfg, budget_s=12.0, seed=0):
-    """tokens/s of the oracle's MoA projections fwd+bwd on a token sample (~budget_s)."""
+    """tokens/s of the oracle's Mixture-of-Attention layer fwd+bwd on a bounded sample:
+    the first n tokens of the first sequence (so their causal windows are complete)."""
     import oracle
     inp = make_moa_inputs(cfg, seed=seed, device="cpu")
-    k, E = cfg["k"], cfg["E"]
+    k, E, L, heads = cfg["k"], cfg["E"], cfg["L"], cfg["heads"]
     n = 8
     while True:
         t0 = time.perf_counter()
-        x, o, dz, dq = inp["x"][:n], inp["o"][:n * k], inp["dz"][:n], inp["dq"][:n * k]
+        x, dz = inp["x"][:n], inp["dz"][:n]
         idx, g = oracle.route(x, inp["w_r"], None, k)
         ss, off = oracle.sort(idx, E)
-        oracle.pl_fwd(x, inp["wq"], ss, off, k, 0, 1)
+        tok, one = np.arange(n, dtype=np.int32), np.array([0, n], np.int32)
+        q = oracle.pl_fwd(x, inp["wq"], ss, off, k, 0, 1)
+        kk = oracle.pl_fwd(x, inp["wk"], tok, one, 1, 1, 1)
+        v = oracle.pl_fwd(x, inp["wv"], tok, one, 1, 1, 1)
+        o = oracle.moa_attn(q, kk, v, ss, k, L, heads)["o"]
         oracle.pl_fwd(o, inp["wo"], ss, off, 1, 1, 0, g.ravel(), k)
-        oracle.pl_bwd(dq, x, inp["wq"], ss, off, k, 0, 1)
-        oracle.pl_bwd(dz, o, inp["wo"], ss, off, 1, 1, 0, g.ravel(), k, want_dg=True)
+        bo = oracle.pl_bwd(dz, o, inp["wo"], ss, off, 1, 1, 0, g.ravel(), k, want_dg=True)
+        ba = oracle.moa_attn(q, kk, v, ss, k, L, heads, dout=bo["dx"])
+        oracle.pl_bwd(ba["dq"], x, inp["wq"], ss, off, k, 0, 1)
+        oracle.pl_bwd(ba["dk"], x, inp["wk"], tok, one, 1, 1, 1)
+        oracle.pl_bwd(ba["dv"], x, inp["wv"], tok, one, 1, 1, 1)
+        oracle.route_bwd(x, inp["w_r"], idx, g, bo["dg"].reshape(n, k))
         dt = time.perf_counter() - t0
-        if dt >= budget_s / 2 or n >= cfg["T"]:
+        if dt >= budget_s / 2 or n >= min(cfg["T"], L):
             break
-        n = min(cfg["T"], 2 * n)
+        n = min(cfg["T"], L, 2 * n)
     return {"value": n / dt, "unit": "tokens/s", "cores": oracle_threads(), "cpu": cpu_model(),
             "kind": "oracle",
-            "sample": f"{n} of the {cfg['T']} tokens: routing, sort, both projections forward "
-                      f"and backward (dx, do, dWq, dWo, gate gradients) in fp64 plain loops, {dt:.1f} s"}
+            "sample": f"the first {n} of the {cfg['T']} tokens (one sequence prefix): routing, sort, "
+                      f"query/key/value/output projections, causal attention core and every "
+                      f"backward in fp64 plain loops, {dt:.1f} s"}
+
+
+def moa_kernel_work(cfg):
+    """Algorithmic work per launch of the Mixture-of-Attention layer's kernels."""
+    T, d, E, k, h = cfg["T"], cfg["d"], cfg["E"], cfg["k"], cfg["h"]
+    af = moa_attn_flops(cfg)["fwd"]  # two width-128 products per (query, key) pair
+    flops = {
+        "moa.attn_fwd": af,           # S = Q K^T, O += P V
+        "moa.attn_dq": 1.5 * af,      # S, dP = dO V^T, dQ += dS K
+        "moa.attn_dkv": 2.0 * af,     # S^T, dP^T, dV += P^T dO, dK += dS^T Q
+    }
+    bytes_ = {"moa.attn_dsum": 2 * T * k * h * 2 + T * k * cfg["heads"] * 4}
+    return flops, bytes_
 
 
 def run_moa(args, world, rank, cfg):
-    """The Mixture-of-Attention expert projections around an attention core (the core
-    itself is not part of the path): route, sort, q = x Wq[e] scatter->group (fan-out k),
-    z = sum_j g o Wo[e] group->scatter with the gated k-way combine, and both backwards
-    (dx, dWq; do, dWo, dgates)."""
+    """The whole Mixture-of-Attention layer, forward and backward: route, sort, per-expert
+    query projection (scatter->group, fan-out k), shared key and value projections
+    (one-expert ParallelLinear), the causal attention core, per-expert output projection
+    (group->scatter, gated k-way combine); backward through all of them, the router
+    included.  The layer's dx is the router's term plus three projection parts (query,
+    key, value); the step leaves the key and value parts as separate outputs (summing
+    them would be two [T, d] additions)."""
     import sparse_mixture_experts_smoe_b200 as smoe
     dev = torch.device("cuda", torch.cuda.current_device())
     inp = make_moa_inputs(cfg, seed=rank, device=dev)
-    T, d, E, k, h = cfg["T"], cfg["d"], cfg["E"], cfg["k"], cfg["h"]
+    T, d, E, k, h, L, heads = cfg["T"], cfg["d"], cfg["E"], cfg["k"], cfg["h"], cfg["L"], cfg["heads"]
+    one = torch.tensor([0, T], dtype=torch.int32, device=dev)
+    ident = torch.arange(T, dtype=torch.int32, device=dev)
+    x, w_r = inp["x"], inp["w_r"]
 
     def step():
-        idx, gates = smoe.smoe_route(inp["x"], inp["w_r"], None, k)
+        idx, gates = smoe.smoe_route(x, w_r, None, k)
         ss, off = smoe.smoe_sort(idx, E)
-        smoe.parallel_linear_fwd(inp["x"], inp["wq"], ss, off, k, 0, 1)
-        smoe.parallel_linear_fwd(inp["o"], inp["wo"], ss, off, 1, 1, 0, gates, k)
-        smoe.parallel_linear_bwd(inp["dq"], inp["x"], inp["wq"], ss, off, k, 0, 1)
-        smoe.parallel_linear_bwd(inp["dz"], inp["o"], inp["wo"], ss, off, 1, 1, 0, gates, k,
-                                 want_dgates=True)
+        q = smoe.parallel_linear_fwd(x, inp["wq"], ss, off, k, 0, 1)
+        kk = smoe.parallel_linear_fwd(x, inp["wk"], ident, one, 1, 1, 1)
+        v = smoe.parallel_linear_fwd(x, inp["wv"], ident, one, 1, 1, 1)
+        o, lse = smoe.smoe_moa_attn_fwd(q, kk, v, ss, k, L, heads)
+        smoe.parallel_linear_fwd(o, inp["wo"], ss, off, 1, 1, 0, gates, k)
+        do, _, dg = smoe.parallel_linear_bwd(inp["dz"], o, inp["wo"], ss, off, 1, 1, 0, gates, k,
+                                             want_dgates=True)
+        dq, dk, dv = smoe.smoe_moa_attn_bwd(q, kk, v, o, lse, do, ss, k, L, heads)
+        dx, _, _ = smoe.parallel_linear_bwd(dq, x, inp["wq"], ss, off, k, 0, 1)
+        smoe.parallel_linear_bwd(dk, x, inp["wk"], ident, one, 1, 1, 1)
+        smoe.parallel_linear_bwd(dv, x, inp["wv"], ident, one, 1, 1, 1)
+        smoe.smoe_route_bwd(x, w_r, idx, gates, dg.view(T, k), dx=dx)
 
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
+    assert smoe.smoe_check() == 0, smoe.lib().smoe_last_error()
+    stream = torch.cuda.current_stream()
     barrier(world)
     clk = ClockSampler()
     clk.start()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
+    torch.cuda.synchronize()
+    e0.record(stream)
     for _ in range(args.steps):
         step()
-    e1.record()
+    e1.record(stream)
     torch.cuda.synchronize()
     clocks = clk.stop()
     barrier(world)
     ms = max_over_ranks(e0.elapsed_time(e1), world) / args.steps
     if smoe.smoe_check() != 0:
         raise SystemExit("device error word set during the MoA benchmark")
-    flops = 12.0 * T * k * d * h  # two projections, fwd + 2x bwd
+    # per-kernel times: a second pass with every launch bracketed by CUDA events
+    smoe.smoe_profile_begin(64 * (args.steps + 1))
+    for _ in range(args.steps):
+        step()
+    torch.cuda.synchronize()
+    prof = smoe.smoe_profile_end()
+    proj = 3 * (2.0 * T * k * d * h + 2 * 2.0 * T * d * h + 2.0 * T * k * h * d)  # fwd + 2x bwd
+    attn = moa_attn_flops(cfg)["fwd_bwd"]
+    flops = proj + attn
     tokens = T * world
     tflops = flops * world / (ms / 1e3) / 1e12
     peaks = load_peaks()
+    fk, bk = moa_kernel_work(cfg)
+    kernels = {}
+    for name, (cnt, tot) in prof.items():
+        per = tot / max(1, cnt) if tot > 0 else None
+        ent = {"launches": cnt, "ms_total": round(tot, 4), "ms_per_launch": None if per is None else round(per, 4)}
+        if name in fk and per:
+            ent["tflops"] = round(fk[name] / (per / 1e3) / 1e12, 1)
+        elif name in bk and per:
+            ent["gbs"] = round(bk[name] / (per / 1e3) / 1e9, 1)
+        kernels[name] = ent
+    # the attention core's dominant kernel against the tensor roofline
+    att = {n: kernels[n] for n in fk if n in kernels}
+    dom = max(att.items(), key=lambda kv: kv[1]["ms_total"])[0] if att else None
+    roofline = None
+    if dom is not None and kernels[dom].get("tflops"):
+        ach = kernels[dom]["tflops"]
+        roofline = {"kernel": dom, "bound": "tensor", "achieved": ach, "peak": peaks["bf16_tflops_sustained"],
+                    "unit": "TFLOP/s", "frac": round(ach / peaks["bf16_tflops_sustained"], 4),
+                    "peak_kind": f"bf16 sustained, {peaks['source']}", "traffic": None}
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = moa_oracle_baseline(cfg)
@@ -363,13 +429,18 @@ def run_moa(args, world, rank, cfg):
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic",
-        "config": {"workload": args.workload, "T": T, "d": d, "E": E, "k": k, "h": h,
-                   "parallelism": f"replicas x{world}"},
+        "config": {"workload": args.workload, "T": T, "d": d, "E": E, "k": k, "h": h, "L": L,
+                   "heads": heads, "parallelism": f"replicas x{world}"},
         "tflops": round(tflops, 1),
+        "tflops_split": {"projections": round(proj / (ms / 1e3) / 1e12, 1),
+                         "attention_core_share_of_flops": round(attn / flops, 4)},
         "frac_of_bf16_peak": {"burst": round(tflops / peaks["bf16_tflops"], 4),
                               "sustained": round(tflops / peaks["bf16_tflops_sustained"], 4),
                               "peaks": peaks["source"]},
         "peak_mem_gb": round(torch.cuda.max_memory_allocated(dev) / 1e9, 2),
+        "gpu_launches": sum(c for c, _ in prof.values()),
+        "roofline": roofline,
+        "kernels": kernels,
         "clocks": clocks,
         "cpu_baseline": cpu,
     }

@@ -716,9 +716,13 @@ int smoe_moa_attn_bwd(const void* q, const void* k, const void* v, const void* o
   int32_t* inv = (int32_t*)workspace;
   float* dsum = (float*)((char*)workspace + align256(S * sizeof(int32_t)));
   { PROF("moa.invert", 1); SMOE_TRY(launch_invert(sorted_slot, (int)S, inv, s), "moa invert"); }
-  { PROF("moa.attn_bwd", 4);
-    SMOE_TRY(launch_moa_attn_bwd(q, k, v, o, lse, dout, inv, T, L, kslots, heads, dq, dk, dv, dsum, err, s),
-             "moa attn bwd"); }
+  { PROF("moa.attn_dsum", 1);
+    SMOE_TRY(launch_attn_dsum(dout, o, (int)S, heads, dsum, s), "moa attn dsum"); }
+  { PROF("moa.attn_dq", 1);
+    SMOE_TRY(launch_attn_dq(q, k, v, lse, dout, inv, T, L, kslots, heads, dq, dsum, err, s), "moa attn dq"); }
+  { PROF("moa.attn_dkv", 1);
+    SMOE_TRY(launch_attn_dkv(q, k, v, lse, dout, inv, T, L, kslots, heads, dk, dv, dsum, err, s),
+             "moa attn dkv"); }
   return SMOE_OK;
 }
 

@@ -724,34 +724,59 @@ cudaError_t launch_moa_attn_fwd(const void* q, const void* k, const void* v, con
   return cudaGetLastError();
 }
 
-cudaError_t launch_moa_attn_bwd(const void* q, const void* k, const void* v, const void* o,
-                                const float* lse, const void* dout, const int32_t* inv, int T, int L,
-                                int kslots, int heads, void* dq, void* dk, void* dv, float* dsum,
-                                unsigned* err, cudaStream_t s) {
+// The backward's three launches (each is bracketed on its own by the caller).
+struct AttnBwdPlan {
   CUtensorMap tk, tv;
-  cudaError_t e = kv_map(&tk, k, T, heads * kDh);
+  AttnArgs a;
+};
+static cudaError_t attn_bwd_plan(AttnBwdPlan& p, const void* q, const void* k, const void* v,
+                                 const float* lse, const void* dout, const int32_t* inv, int T, int L,
+                                 int kslots, int heads, void* dq, void* dk, void* dv, float* dsum,
+                                 unsigned* err) {
+  cudaError_t e = kv_map(&p.tk, k, T, heads * kDh);
   if (e != cudaSuccess) return e;
-  if ((e = kv_map(&tv, v, T, heads * kDh)) != cudaSuccess) return e;
-  const int S = T * kslots;
+  if ((e = kv_map(&p.tv, v, T, heads * kDh)) != cudaSuccess) return e;
+  p.a = attn_args(T, L, kslots, heads, inv, err);
+  p.a.q = (const bf16*)q;
+  p.a.dout = (const bf16*)dout;
+  p.a.lse = lse;
+  p.a.dsum = dsum;
+  p.a.dq = (bf16*)dq;
+  p.a.dk = (bf16*)dk;
+  p.a.dv = (bf16*)dv;
+  return cudaSuccess;
+}
+
+cudaError_t launch_attn_dsum(const void* dout, const void* o, int S, int heads, float* dsum, cudaStream_t s) {
   attn_dsum_kernel<<<cdiv(S, 8), 256, 0, s>>>((const bf16*)dout, (const bf16*)o, S, heads, dsum);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  AttnArgs a = attn_args(T, L, kslots, heads, inv, err);
-  a.q = (const bf16*)q;
-  a.dout = (const bf16*)dout;
-  a.lse = lse;
-  a.dsum = dsum;
-  a.dq = (bf16*)dq;
-  a.dk = (bf16*)dk;
-  a.dv = (bf16*)dv;
+  return cudaGetLastError();
+}
+
+cudaError_t launch_attn_dq(const void* q, const void* k, const void* v, const float* lse,
+                           const void* dout, const int32_t* inv, int T, int L, int kslots, int heads,
+                           void* dq, const float* dsum, unsigned* err, cudaStream_t s) {
+  AttnBwdPlan p;
+  cudaError_t e = attn_bwd_plan(p, q, k, v, lse, dout, inv, T, L, kslots, heads, dq, nullptr, nullptr,
+                                const_cast<float*>(dsum), err);
+  if (e != cudaSuccess) return e;
   if ((e = cudaFuncSetAttribute(moa_attn_dq_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 (int)kDqSmem)) != cudaSuccess)
     return e;
+  moa_attn_dq_kernel<<<p.a.heads * p.a.nseq * p.a.tiles_per_seq, kAttnThreads, kDqSmem, s>>>(p.tk, p.tv, p.a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_attn_dkv(const void* q, const void* k, const void* v, const float* lse,
+                            const void* dout, const int32_t* inv, int T, int L, int kslots, int heads,
+                            void* dk, void* dv, const float* dsum, unsigned* err, cudaStream_t s) {
+  AttnBwdPlan p;
+  cudaError_t e = attn_bwd_plan(p, q, k, v, lse, dout, inv, T, L, kslots, heads, nullptr, dk, dv,
+                                const_cast<float*>(dsum), err);
+  if (e != cudaSuccess) return e;
   if ((e = cudaFuncSetAttribute(moa_attn_dkv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 (int)kDkvSmem)) != cudaSuccess)
     return e;
-  moa_attn_dq_kernel<<<a.heads * a.nseq * a.tiles_per_seq, kAttnThreads, kDqSmem, s>>>(tk, tv, a);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  moa_attn_dkv_kernel<<<a.heads * a.nseq * a.kv_per_seq, kAttnThreads, kDkvSmem, s>>>(tk, tv, a);
+  moa_attn_dkv_kernel<<<p.a.heads * p.a.nseq * p.a.kv_per_seq, kAttnThreads, kDkvSmem, s>>>(p.tk, p.tv, p.a);
   return cudaGetLastError();
 }
 

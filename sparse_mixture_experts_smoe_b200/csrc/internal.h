@@ -141,10 +141,14 @@ int attn_head_dim();
 cudaError_t launch_moa_attn_fwd(const void* q, const void* k, const void* v, const int32_t* inv, int T,
                                 int L, int kslots, int heads, void* o, float* lse, unsigned* err,
                                 cudaStream_t s);
-cudaError_t launch_moa_attn_bwd(const void* q, const void* k, const void* v, const void* o,
-                                const float* lse, const void* dout, const int32_t* inv, int T, int L,
-                                int kslots, int heads, void* dq, void* dk, void* dv, float* dsum,
-                                unsigned* err, cudaStream_t s);
+// backward: dsum = <dO, O> first, then dq and (dk, dv) from it
+cudaError_t launch_attn_dsum(const void* dout, const void* o, int S, int heads, float* dsum, cudaStream_t s);
+cudaError_t launch_attn_dq(const void* q, const void* k, const void* v, const float* lse,
+                           const void* dout, const int32_t* inv, int T, int L, int kslots, int heads,
+                           void* dq, const float* dsum, unsigned* err, cudaStream_t s);
+cudaError_t launch_attn_dkv(const void* q, const void* k, const void* v, const float* lse,
+                            const void* dout, const int32_t* inv, int T, int L, int kslots, int heads,
+                            void* dk, void* dv, const float* dsum, unsigned* err, cudaStream_t s);
 
 // tcgen05 / TMEM path (bf16 only); *_supported() checks the device once.
 bool tc_supported();

@@ -23,7 +23,7 @@ b_r[e] = -s * ln(r_e) for r_e <= E - n_empty and -1e4 otherwise, so exactly
 ``n_empty`` experts can never be selected (k < E - n_empty).
 
 Mixture-of-Attention projections: x [T, d]; Wq [E, d, h] ~ N(0, 1/d);
-Wo [E, h, d] ~ N(0, 1/h); per-slot attention output o [T*k, h] ~ N(0, 1) in
+Wo [E, h, d] ~ N(0, 1/h); shared Wk, Wv [1, d, h] ~ N(0, 1/d); per-slot attention output o [T*k, h] ~ N(0, 1) in
 grouped order; upstream gradients dz [T, d] and dq [T*k, h] ~ N(0, 1).
 Mixture-of-Attention core: the T tokens are sequences of L = 2048 tokens; queries
 q [T*k, h] (grouped), shared keys and values k, v [T, h] and the upstream
@@ -48,7 +48,8 @@ WORKLOADS = {
 }
 
 _STREAM = {"x": 1, "w_r": 2, "w1": 3, "w2": 4, "dy": 5, "perm": 6, "wq": 7, "wo": 8, "o": 9,
-           "dz": 10, "dq": 11, "dg": 12, "aq": 13, "ak": 14, "av": 15, "ado": 16}
+           "dz": 10, "dq": 11, "dg": 12, "aq": 13, "ak": 14, "av": 15, "ado": 16, "wk": 17,
+           "wv": 18}
 
 
 def torch_dtype(name: str) -> torch.dtype:
@@ -122,6 +123,9 @@ def make_moa_inputs(cfg: dict, seed: int = 0, device="cpu") -> dict:
         "b_r": None,
         "wq": _randn((E, d, h), 1.0 / math.sqrt(d), "wq", seed, device, dt),
         "wo": _randn((E, h, d), 1.0 / math.sqrt(h), "wo", seed, device, dt),
+        # shared key and value projections of the attention core (one "expert" each)
+        "wk": _randn((1, d, h), 1.0 / math.sqrt(d), "wk", seed, device, dt),
+        "wv": _randn((1, d, h), 1.0 / math.sqrt(d), "wv", seed, device, dt),
         "o": _randn((T * k, h), 1.0, "o", seed, device, dt),
         "dz": _randn((T, d), 1.0, "dz", seed, device, dt),
         "dq": _randn((T * k, h), 1.0, "dq", seed, device, dt),
