@@ -8,7 +8,7 @@ CUDA package.
 Every function takes CPU tensors or numpy arrays holding the stored values
 (float32, or bfloat16 as a torch tensor) and returns fp64 numpy arrays, except the
 integer routing outputs.  The definitions follow the ScatterMoE pages as listed
-in the header of ``smoe_oracle.cpp`` (readings R1-R7 there).
+in the header of ``smoe_oracle.cpp`` (readings R1-R8 there).
 
 Parity status: every function here is pinned by ``tests/test_oracle_pins.py``
 against independent mathematics (brute force, closed forms, library routines,
@@ -223,6 +223,70 @@ def moa_attn(q, k, v, sorted_slot, kslots, L, heads, dout=None, q_rows=None, kv_
     lib.oracle_moa_attn(_p(qs), _p(ks), _p(vs), _p(ds), dt, _p(ss), T, kslots, L, heads, dh,
                         _p(rows), nq, _p(toks), nkv, _p(out["o"]), _p(out["lse"]),
                         _p(out.get("dq")), _p(out.get("dk")), _p(out.get("dv")))
+    return out
+
+
+def e4m3_round(v):
+    """Values rounded to the nearest e4m3 value (ties to even, saturating at 448)."""
+    lib = _load()
+    a = np.ascontiguousarray(v, dtype=np.float64).ravel()
+    out = np.empty_like(a)
+    lib.oracle_e4m3_round(_p(a), a.size, _p(out))
+    return out.reshape(np.shape(v))
+
+
+def e4m3_decode(codes):
+    lib = _load()
+    b = np.ascontiguousarray(codes, dtype=np.uint8).ravel()
+    out = np.empty(b.size)
+    lib.oracle_e4m3_decode(_p(b), b.size, _p(out))
+    return out.reshape(np.shape(codes))
+
+
+def quantize_weights_fp8(w):
+    """W [E, K, N] -> (codes uint8 [E, N, K] (K-major), scales fp32 [E, N])."""
+    lib = _load()
+    ws, dt = _stored(w)
+    E, K, N = ws.shape
+    codes = np.empty((E, N, K), np.uint8)
+    scales = np.empty((E, N), np.float32)
+    lib.oracle_quantize_weights_fp8(_p(ws), dt, E, K, N, _p(codes), _p(scales))
+    return codes, scales
+
+
+def quantize_rows_fp8(x):
+    """x [rows, cols] -> (codes uint8 [rows, cols], scales fp32 [rows])."""
+    lib = _load()
+    xs, dt = _stored(x)
+    rows, cols = xs.shape
+    codes = np.empty((rows, cols), np.uint8)
+    scales = np.empty(rows, np.float32)
+    lib.oracle_quantize_rows_fp8(_p(xs), dt, rows, cols, _p(codes), _p(scales))
+    return codes, scales
+
+
+def mlp_fwd_fp8(x, w1q, s1, w2q, s2, act_name, topk_idx, gates, tokens=None, want_a=False):
+    """FP8 forward (R8) with weights quantised by ``quantize_weights_fp8``:
+    {"y": [n_tok, d], "a": [n_tok*k, f] (bf16-rounded A, slot order) if want_a}."""
+    lib = _load()
+    xs, dtx = _stored(x)
+    T, d = xs.shape
+    E, mf, d2 = w1q.shape
+    assert d2 == d
+    f = w2q.shape[2]
+    idx = _i32(topk_idx)
+    k = idx.shape[1]
+    g = _f64(gates)
+    tok = np.arange(T, dtype=np.int32) if tokens is None else _i32(tokens)
+    n = tok.size
+    y = np.empty((n, d))
+    a = np.empty((n * k, f)) if want_a else None
+    lib.oracle_mlp_fwd_fp8(_p(xs), dtx, _p(np.ascontiguousarray(w1q)), _p(np.ascontiguousarray(s1)),
+                           _p(np.ascontiguousarray(w2q)), _p(np.ascontiguousarray(s2)), d, f, E, k,
+                           ACT[act_name], _p(idx), _p(g), _p(tok), n, _p(y), _p(a))
+    out = {"y": y}
+    if want_a:
+        out["a"] = a
     return out
 
 

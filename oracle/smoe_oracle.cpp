@@ -40,6 +40,10 @@
  *   R7 Mixture-of-Attention core (see oracle_moa_attn): per-expert queries in
  *      grouped order attend causally, within each sequence of L tokens, to keys
  *      and values shared by all experts, head by head.
+ *   R8 FP8 inference forward (see oracle_mlp_fwd_fp8): e4m3 codes with one fp32
+ *      scale per expert output column (weights) and per row (x, and A stored in
+ *      bf16 first); the quantisation decisions are taken in fp32, the products in
+ *      fp64 from the decoded codes.
  *
  * Every input array is passed as its stored values (fp32, or bf16 bit patterns)
  * and upcast exactly to fp64.  All arithmetic below is fp64 except the fp32
@@ -476,6 +480,70 @@ void pl_bwd_impl(const TD* dy, const TX* x, const TW* w, int x_rows, int K, int 
     else { typedef double TX; typedef double TW; CALL; }                      \
   } while (0)
 
+/* R8: FP8 (e4m3) inference forward (sourcepulse.org summary: inference speed).
+ * e4m3 as the OCP 8-bit floating-point format defines it: 1 sign bit, 4 exponent
+ * bits (bias 7), 3 mantissa bits; normal values (1 + m/8) 2^(e-7) for e = 1..15
+ * (except e = 15, m = 7, which is NaN), subnormal values (m/8) 2^-6; largest 448.
+ * e4m3_round: round to nearest, ties to even mantissa, saturating at +-448. */
+double e4m3_round(double x) {
+  if (x == 0.0 || std::isnan(x)) return x;
+  const double a = std::fabs(x);
+  double q;
+  if (a >= 448.0) {
+    q = 448.0;
+  } else {
+    int e = (int)std::floor(std::log2(a));
+    if (std::ldexp(1.0, e) > a) --e;          /* guard log2 rounding */
+    if (std::ldexp(1.0, e + 1) <= a) ++e;
+    const double quantum = e < -6 ? std::ldexp(1.0, -9) : std::ldexp(1.0, e - 3);
+    const double n = a / quantum;             /* exact: a power-of-two scaling */
+    double r = std::floor(n);
+    const double frac = n - r;
+    if (frac > 0.5 || (frac == 0.5 && std::fmod(r, 2.0) != 0.0)) r += 1.0;
+    q = std::min(r * quantum, 448.0);
+  }
+  return x < 0 ? -q : q;
+}
+/* bits of an e4m3 value produced by e4m3_round (finite, |v| <= 448) */
+uint8_t e4m3_bits(double v) {
+  const uint8_t s = (std::signbit(v) ? 0x80 : 0x00);
+  const double a = std::fabs(v);
+  if (a == 0.0) return s;
+  if (a < std::ldexp(1.0, -6)) return (uint8_t)(s | (uint8_t)std::lround(a / std::ldexp(1.0, -9)));
+  int e = (int)std::floor(std::log2(a));
+  if (std::ldexp(1.0, e) > a) --e;
+  if (std::ldexp(1.0, e + 1) <= a) ++e;
+  const int m = (int)std::lround((a / std::ldexp(1.0, e) - 1.0) * 8.0);
+  return (uint8_t)(s | (uint8_t)((e + 7) << 3) | (uint8_t)m);
+}
+double e4m3_value(uint8_t b) {
+  const int s = b >> 7, e = (b >> 3) & 15, m = b & 7;
+  const double v = e == 0 ? std::ldexp((double)m / 8.0, -6) : std::ldexp(1.0 + m / 8.0, e - 7);
+  return s ? -v : v;
+}
+/* Row quantisation (the kernels' decision precision, fp32): scale = fl32(amax / 448)
+ * (1 for an all-zero row), code = e4m3(fl32(v / scale)). */
+void quantize_row_fp8(const double* v, int n, uint8_t* codes, float* scale) {
+  float amax = 0.0f;
+  for (int i = 0; i < n; ++i) amax = std::max(amax, (float)std::fabs(v[i]));
+  const float s = amax > 0.0f ? amax / 448.0f : 1.0f;
+  for (int i = 0; i < n; ++i) codes[i] = e4m3_bits(e4m3_round((double)((float)v[i] / s)));
+  *scale = s;
+}
+
+/* bf16 storage of a value (round to nearest even from fp32), as the kernels store
+ * activations */
+bf16s bf16_round(double v) {
+  const float f = (float)v;
+  uint32_t u;
+  std::memcpy(&u, &f, 4);
+  const uint32_t lsb = (u >> 16) & 1u;
+  u += 0x7FFFu + lsb;
+  bf16s r;
+  r.bits = (uint16_t)(u >> 16);
+  return r;
+}
+
 }  // namespace
 
 extern "C" {
@@ -787,6 +855,82 @@ void oracle_moa_attn(const void* q, const void* k, const void* v, const void* do
       }
     }
   }
+}
+
+/* e4m3 rounding of n values (for pins) */
+void oracle_e4m3_round(const double* v, int n, double* out) {
+  for (int i = 0; i < n; ++i) out[i] = e4m3_round(v[i]);
+}
+void oracle_e4m3_decode(const uint8_t* b, int n, double* out) {
+  for (int i = 0; i < n; ++i) out[i] = e4m3_value(b[i]);
+}
+/* Weights W [E, K, N] (stored dtype dt) -> codes [E, N, K] (K-major) and one scale per
+ * (expert, output column) [E, N], over that column's K values. */
+void oracle_quantize_weights_fp8(const void* w, int dt, int E, int K, int N, uint8_t* codes,
+                                 float* scales) {
+#pragma omp parallel for schedule(static)
+  for (int en = 0; en < E * N; ++en) {
+    const int e = en / N, n = en % N;
+    std::vector<double> col(K);
+    for (int k = 0; k < K; ++k) col[k] = load_any(w, dt, ((size_t)e * K + k) * N + n);
+    quantize_row_fp8(col.data(), K, codes + (size_t)en * K, scales + en);
+  }
+}
+/* Rows of a matrix [rows, cols] (stored dtype dt) -> codes [rows, cols], scales [rows]. */
+void oracle_quantize_rows_fp8(const void* x, int dt, int rows, int cols, uint8_t* codes,
+                              float* scales) {
+#pragma omp parallel for schedule(static)
+  for (int r = 0; r < rows; ++r) {
+    std::vector<double> v(cols);
+    for (int c = 0; c < cols; ++c) v[c] = load_any(x, dt, (size_t)r * cols + c);
+    quantize_row_fp8(v.data(), cols, codes + (size_t)r * cols, scales + r);
+  }
+}
+/* FP8 forward of the listed tokens with quantised weights (codes K-major [E, N, K],
+ * scales [E, N]) from oracle_quantize_weights_fp8:
+ *   x8, sx = row quantisation of x[t];  H = (x8 . w1_8[e]) sx s1[e]  (fp64)
+ *   A = act(H), stored in bf16;  a8, sa = row quantisation of A (its f values)
+ *   o = (a8 . w2_8[e]) sa s2[e];  y_t = sum_j g[t,j] o_{t*k+j}.
+ * y [n_tok, d]; a (nullable) [n_tok*k, f] = the bf16-rounded A. */
+void oracle_mlp_fwd_fp8(const void* x, int dtx, const uint8_t* w1q, const float* s1,
+                        const uint8_t* w2q, const float* s2, int d, int f, int E, int k, int act,
+                        const int32_t* idx, const double* gates, const int32_t* tokens, int n_tok,
+                        double* y, double* a_out) {
+  const int mf = (act == ACT_SWIGLU) ? 2 * f : f;
+#pragma omp parallel for schedule(dynamic, 1)
+  for (int q = 0; q < n_tok; ++q) {
+    const int t = tokens[q];
+    std::vector<double> xv(d), h(mf), a(f);
+    std::vector<uint8_t> x8(d), a8(f);
+    float sx, sa;
+    for (int i = 0; i < d; ++i) xv[i] = load_any(x, dtx, (size_t)t * d + i);
+    quantize_row_fp8(xv.data(), d, x8.data(), &sx);
+    double* yq = y + (size_t)q * d;
+    for (int n = 0; n < d; ++n) yq[n] = 0.0;
+    for (int j = 0; j < k; ++j) {
+      const int e = idx[(size_t)t * k + j];
+      for (int n = 0; n < mf; ++n) {
+        const uint8_t* wr = w1q + ((size_t)e * mf + n) * d;
+        double acc = 0.0;
+        for (int i = 0; i < d; ++i) acc += e4m3_value(x8[i]) * e4m3_value(wr[i]);
+        h[n] = acc * (double)sx * (double)s1[(size_t)e * mf + n];
+      }
+      for (int c = 0; c < f; ++c) {
+        const double av = (act == ACT_SWIGLU) ? silu(h[c]) * h[f + c] : gelu_tanh(h[c]);
+        a[c] = (double)to_float(bf16_round(av));
+      }
+      if (a_out) std::memcpy(a_out + ((size_t)q * k + j) * f, a.data(), sizeof(double) * f);
+      quantize_row_fp8(a.data(), f, a8.data(), &sa);
+      const double g = gates[(size_t)t * k + j];
+      for (int n = 0; n < d; ++n) {
+        const uint8_t* wr = w2q + ((size_t)e * d + n) * f;
+        double acc = 0.0;
+        for (int c = 0; c < f; ++c) acc += e4m3_value(a8[c]) * e4m3_value(wr[c]);
+        yq[n] += g * acc * (double)sa * (double)s2[(size_t)e * d + n];
+      }
+    }
+  }
+  (void)E;
 }
 
 /* R6 forward.  gates: fp64 per slot (nullable).  out_rows (nullable): the rows

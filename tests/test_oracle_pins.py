@@ -574,3 +574,84 @@ def test_moa_attn_single_token_sequences_and_subsets():
         np.testing.assert_allclose(sub[key], full[key][rows], rtol=1e-12, atol=1e-13)
     for key in ("dk", "dv"):
         np.testing.assert_allclose(sub[key], full[key][toks], rtol=1e-12, atol=1e-13)
+
+
+# --------------------------------------------------------------------------
+# FP8 (e4m3) inference forward
+# --------------------------------------------------------------------------
+def test_e4m3_rounding_matches_torch_float8():
+    """Round-to-nearest-even into e4m3 against torch's float8_e4m3fn conversion, on
+    every representable magnitude, the midpoints between neighbours (ties), random
+    values over the whole range including subnormals, and saturation at 448."""
+    reps = np.unique(np.abs(torch.arange(256, dtype=torch.uint8).view(torch.float8_e4m3fn)
+                            .float().numpy().astype(np.float64)))
+    reps = reps[np.isfinite(reps)]
+    mids = (reps[1:] + reps[:-1]) / 2
+    r = _rng(5)
+    rnd = np.concatenate([r.uniform(-448, 448, 4000), r.uniform(-0.05, 0.05, 2000),
+                          np.ldexp(r.uniform(1, 2, 500), r.integers(-12, 9, 500))])
+    v = np.concatenate([reps, -reps, mids, -mids, rnd])
+    v = v[np.abs(v) <= 448]  # beyond 448 torch gives NaN; saturation is checked below
+    want = torch.from_numpy(v).to(torch.float8_e4m3fn).double().numpy()
+    np.testing.assert_array_equal(oracle.e4m3_round(v), want)
+    assert oracle.e4m3_round(np.array([449.0, 460.0, -1000.0])).tolist() == [448.0, 448.0, -448.0]
+    # codes decode back to the values (every finite code)
+    codes = np.array([c for c in range(256) if (c & 0x7F) != 0x7F], np.uint8)
+    np.testing.assert_array_equal(oracle.e4m3_decode(codes),
+                                  torch.from_numpy(codes).view(torch.float8_e4m3fn).double().numpy())
+
+
+def test_fp8_quantisation_of_rows_and_weights():
+    """Each row (or weight column) maps its largest magnitude to 448 exactly, every
+    code decodes to e4m3(fl32(v / scale)), and the weight codes are the columns'
+    codes laid out K-major."""
+    g = torch.Generator().manual_seed(6)
+    x = (torch.randn(7, 40, generator=g) * 3).to(torch.bfloat16)
+    x[3] = 0
+    codes, sc = oracle.quantize_rows_fp8(x)
+    xv = x.float().numpy()
+    amax = np.abs(xv).max(1)
+    np.testing.assert_array_equal(sc, np.where(amax > 0, (amax / np.float32(448)).astype(np.float32), 1))
+    dec = oracle.e4m3_decode(codes)
+    want = torch.from_numpy((xv / sc[:, None]).astype(np.float32)).to(torch.float8_e4m3fn).double().numpy()
+    np.testing.assert_array_equal(dec, want)
+    assert np.all(np.abs(dec).max(1)[amax > 0] == 448)
+    w = (torch.randn(3, 24, 10, generator=g) / 5).to(torch.bfloat16)
+    wc, ws = oracle.quantize_weights_fp8(w)
+    for e in range(3):
+        c2, s2 = oracle.quantize_rows_fp8(w[e].T.contiguous())
+        np.testing.assert_array_equal(wc[e], c2)
+        np.testing.assert_array_equal(ws[e], s2)
+
+
+@pytest.mark.parametrize("act", ["gelu", "swiglu"])
+def test_fp8_forward_equals_dequantised_dense_reference(act):
+    """The FP8 forward equals the dense evaluate-every-expert-and-mask reference run on
+    the dequantised codes (torch, fp64): x8 * sx and w8 * s per column, A rounded to
+    bf16 and requantised per row; and it stays close to the exact bf16 forward."""
+    T, d, f, E, k = 12, 32, 24, 4, 2
+    x, w_r, w1, w2, _ = _tiny_mlp(14, T, d, f, E, k, act, torch.bfloat16)
+    idx, gates = oracle.route(x, w_r, None, k)
+    w1q, s1 = oracle.quantize_weights_fp8(w1)
+    w2q, s2 = oracle.quantize_weights_fp8(w2)
+    out = oracle.mlp_fwd_fp8(x, w1q, s1, w2q, s2, act, idx, gates, want_a=True)
+    x8, sx = oracle.quantize_rows_fp8(x)
+    xd = torch.from_numpy(oracle.e4m3_decode(x8) * sx[:, None].astype(np.float64))
+    W1 = torch.from_numpy(oracle.e4m3_decode(w1q) * s1[:, :, None].astype(np.float64)).transpose(1, 2)
+    W2 = torch.from_numpy(oracle.e4m3_decode(w2q) * s2[:, :, None].astype(np.float64)).transpose(1, 2)
+    y = torch.zeros(T, d, dtype=torch.float64)
+    for t in range(T):
+        for j in range(k):
+            e = int(idx[t, j])
+            h = xd[t] @ W1[e]
+            a = F.gelu(h, approximate="tanh") if act == "gelu" else F.silu(h[:f]) * h[f:]
+            a = a.float().to(torch.bfloat16).double()
+            np.testing.assert_allclose(out["a"][t * k + j], a.numpy(), rtol=0, atol=0)
+            a8, sa = oracle.quantize_rows_fp8(a[None])
+            ad = torch.from_numpy(oracle.e4m3_decode(a8)[0] * np.float64(sa[0]))
+            y[t] += gates[t, j] * (ad @ W2[e])
+    np.testing.assert_allclose(out["y"], y.numpy(), rtol=1e-12, atol=1e-12)
+    # e4m3 keeps 3 mantissa bits (relative steps up to 2^-3); with 24-32 terms per
+    # product little of that averages out, so only a loose agreement is expected here
+    exact = oracle.mlp_fwd(x, w1, w2, act, idx, gates)["y"]
+    assert np.max(np.abs(out["y"] - exact)) / np.max(np.abs(exact)) < 0.25
