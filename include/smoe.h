@@ -320,6 +320,46 @@ int smoe_mlp_fwd(const smoe_mlp_desc* desc, const smoe_mlp_tensors* t, void* str
 int smoe_mlp_bwd(const smoe_mlp_desc* desc, const smoe_mlp_tensors* t, void* stream);
 
 /* ---------------------------------------------------------------------------
+ * FP8 inference forward [src: inference speed as a target of the method]
+ *
+ * The pages name inference speed but no number format; this library's FP8 path
+ * stores expert weights as e4m3 codes (OCP 8-bit float: 4 exponent bits, bias 7,
+ * 3 mantissa bits, largest value 448) and runs both expert products on
+ * tcgen05.mma kind::f8f6f4 with fp32 accumulation.  Scales are fp32: one per
+ * (expert, output column) for the weights, one per row for the activations
+ * (x per token, A per slot row after it is stored in bf16); a scale maps its
+ * row's or column's largest magnitude to 448 (scale = amax / 448 in fp32, 1 for an
+ * all-zero row), and a code is e4m3(fl32(v / scale)), rounded to nearest even.
+ *
+ * smoe_quantize_weights_fp8: W [E, K, N] bf16 -> codes [E, N, K] uint8 (K-major:
+ * row n of expert e holds column n of W[e]) and scales [E, N] fp32.  K % 16 == 0.
+ * For the MLP: W1 [E, d, m*f] -> w1q [E, m*f, d], s1 [E, m*f];
+ * W2 [E, f, d] -> w2q [E, d, f], s2 [E, d].
+ *
+ * smoe_mlp_fwd_fp8: the forward of smoe_mlp_fwd with those weights:
+ *   h = (x8 . w1q[e]) sx s1[e]  (bf16, grouped, as smoe_mlp_fwd's h),
+ *   a = act(h) (bf16), a8 = the row quantisation of a,
+ *   y_t = sum_j gates[t,j] (a8 . w2q[e]) sa s2[e].
+ * Routing, sort and the deterministic k-way combine are those of smoe_mlp_fwd.
+ * Uses desc (dtype must be SMOE_BF16; d % 16 == 0, f % 16 == 0), the routing and
+ * activation buffers of t (x, w_r, b_r, y, topk_idx, gates, sorted_slot,
+ * expert_offsets, h, a, workspace of smoe_mlp_fp8_workspace_size bytes); t->w1
+ * and t->w2 are not read.
+ * ------------------------------------------------------------------------ */
+typedef struct {
+  const uint8_t* w1q; /* [E, m*f, d] e4m3 codes */
+  const float* s1;    /* [E, m*f] */
+  const uint8_t* w2q; /* [E, d, f] e4m3 codes */
+  const float* s2;    /* [E, d] */
+} smoe_fp8_weights;
+
+int smoe_quantize_weights_fp8(const void* w, int E, int K, int N, smoe_dtype dt, uint8_t* codes,
+                              float* scales, void* stream);
+size_t smoe_mlp_fp8_workspace_size(const smoe_mlp_desc* desc);
+int smoe_mlp_fwd_fp8(const smoe_mlp_desc* desc, const smoe_mlp_tensors* t, const smoe_fp8_weights* w8,
+                     void* stream);
+
+/* ---------------------------------------------------------------------------
  * Instrumentation (the pages have no counterpart; used by the benchmark).
  *
  * smoe_profile_begin: from now on, every kernel launch this library makes from

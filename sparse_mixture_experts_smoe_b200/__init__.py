@@ -46,6 +46,10 @@ class MlpTensors(ctypes.Structure):
                [("workspace_bytes", _c_size)]
 
 
+class Fp8Weights(ctypes.Structure):
+    _fields_ = [("w1q", _vp), ("s1", _vp), ("w2q", _vp), ("s2", _vp)]
+
+
 def library_path() -> str:
     return _LIB_PATH
 
@@ -80,6 +84,11 @@ def lib():
     L.parallel_linear_bwd.argtypes = [_vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _vp, _vp,
                                       _c_int, _c_int, _c_int, _c_int, _vp, _c_int, _vp, _vp, _vp,
                                       _c_int, _vp, _c_size, _vp]
+    L.smoe_quantize_weights_fp8.argtypes = [_vp, _c_int, _c_int, _c_int, _c_int, _vp, _vp, _vp]
+    L.smoe_mlp_fp8_workspace_size.restype = _c_size
+    L.smoe_mlp_fp8_workspace_size.argtypes = [ctypes.POINTER(MlpDesc)]
+    L.smoe_mlp_fwd_fp8.argtypes = [ctypes.POINTER(MlpDesc), ctypes.POINTER(MlpTensors),
+                                   ctypes.POINTER(Fp8Weights), _vp]
     L.smoe_moa_attn_workspace_size.restype = _c_size
     L.smoe_moa_attn_workspace_size.argtypes = [_c_int] * 4
     L.smoe_moa_attn_fwd.argtypes = [_vp, _vp, _vp, _vp] + [_c_int] * 6 + [_vp, _vp, _vp, _c_size, _vp]
@@ -310,6 +319,37 @@ def smoe_moa_attn_bwd(q, k, v, o, lse, dout, sorted_slot, kslots, L, heads, stre
     return dq, dk, dv
 
 
+def smoe_quantize_weights_fp8(w, stream=None):
+    """W [E, K, N] bf16 -> (codes uint8 [E, N, K] e4m3, K-major; scales fp32 [E, N])."""
+    _need(w, "w", torch.bfloat16)
+    E, K, N = w.shape
+    codes = torch.empty((E, N, K), dtype=torch.uint8, device=w.device)
+    scales = torch.empty((E, N), dtype=torch.float32, device=w.device)
+    _check(lib().smoe_quantize_weights_fp8(_ptr(w), E, K, N, BF16, _ptr(codes), _ptr(scales),
+                                           _stream(stream)))
+    return codes, scales
+
+
+def smoe_mlp_fwd_fp8(st, x, w_r, b_r, w1q, s1, w2q, s2, stream=None):
+    """FP8 forward into the state's y, h, a and routing buffers (see smoe.h)."""
+    for t_, n in ((x, "x"), (w_r, "w_r")):
+        _need(t_, n, torch.bfloat16)
+    for t_, n in ((w1q, "w1q"), (w2q, "w2q")):
+        _need(t_, n, torch.uint8)
+    for t_, n in ((s1, "s1"), (s2, "s2")):
+        _need(t_, n, torch.float32)
+    d = st.desc
+    ws_bytes = lib().smoe_mlp_fp8_workspace_size(ctypes.byref(d))
+    if ws_bytes == 0:
+        _check(-1)
+    ws = _workspace(ws_bytes, x.device)
+    t = st.tensors(x, w_r, b_r, None, None)
+    t.workspace = ws.data_ptr()
+    t.workspace_bytes = ws.numel()
+    w8 = Fp8Weights(w1q.data_ptr(), s1.data_ptr(), w2q.data_ptr(), s2.data_ptr())
+    _check(lib().smoe_mlp_fwd_fp8(ctypes.byref(d), ctypes.byref(t), ctypes.byref(w8), _stream(stream)))
+
+
 class SMoEMLPState:
     """Buffers of one SMoE MLP layer call: parameters, saved forward outputs and
     gradients, all allocated by torch once and reused across steps."""
@@ -341,9 +381,8 @@ class SMoEMLPState:
 
     def tensors(self, x, w_r, b_r, w1, w2, dy=None) -> MlpTensors:
         t = MlpTensors()
-        t.x, t.w_r, t.b_r, t.w1, t.w2 = (x.data_ptr(), w_r.data_ptr(),
-                                         None if b_r is None else b_r.data_ptr(), w1.data_ptr(),
-                                         w2.data_ptr())
+        ptr = lambda v: None if v is None else v.data_ptr()  # noqa: E731
+        t.x, t.w_r, t.b_r, t.w1, t.w2 = ptr(x), ptr(w_r), ptr(b_r), ptr(w1), ptr(w2)
         for n in ("y", "topk_idx", "gates", "sorted_slot", "expert_offsets", "h", "a"):
             setattr(t, n, getattr(self, n).data_ptr())
         if dy is not None:

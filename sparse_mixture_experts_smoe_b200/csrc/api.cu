@@ -642,6 +642,46 @@ int parallel_linear_bwd(const void* dy, const void* x, const void* w, int x_rows
 }
 
 // ---------------------------------------------------------------------------
+// FP8 inference forward
+// ---------------------------------------------------------------------------
+struct Fp8Ws {
+  void* sort = nullptr;
+  int32_t* inv = nullptr;
+  void* ycomb = nullptr;    // [S, d] bf16 slot rows, grouped order
+  float* kpart = nullptr;   // split-K partials of the down projection
+  int ksplit = 1;
+  uint8_t* x8 = nullptr;    // [T, d] codes
+  float* sx = nullptr;      // [T]
+  uint8_t* a8 = nullptr;    // [S, f] codes (grouped rows)
+  float* sa = nullptr;      // [S]
+  size_t bytes = 0;
+};
+static Fp8Ws fp8_layout(void* ws, const smoe_mlp_desc& m) {
+  Carve c(ws);
+  Fp8Ws l;
+  const size_t S = (size_t)m.T * m.k;
+  l.sort = c.take(sort_workspace_bytes(m.T, m.k, m.E));
+  l.inv = (int32_t*)c.take(S * sizeof(int32_t));
+  l.ycomb = c.take(S * m.d * 2);
+  l.ksplit = grouped_ksplit((int)S, m.E, m.d, m.f, 1);
+  if (l.ksplit > 1) l.kpart = (float*)c.take((size_t)l.ksplit * S * m.d * sizeof(float));
+  l.x8 = (uint8_t*)c.take((size_t)m.T * m.d);
+  l.sx = (float*)c.take((size_t)m.T * sizeof(float));
+  l.a8 = (uint8_t*)c.take(S * m.f);
+  l.sa = (float*)c.take(S * sizeof(float));
+  l.bytes = c.off;
+  return l;
+}
+
+static int validate_fp8_desc(const smoe_mlp_desc* m) {
+  int rc = validate_mlp_desc(m);
+  if (rc != SMOE_OK) return rc;
+  if (m->dtype != SMOE_BF16) return fail(SMOE_ERR_UNSUPPORTED, "the FP8 forward takes bf16 activations");
+  if (m->d % 16 || m->f % 16) return fail(SMOE_ERR_INVALID_ARG, "FP8: d and f must be multiples of 16");
+  return SMOE_OK;
+}
+
+// ---------------------------------------------------------------------------
 // Mixture-of-Attention core
 // ---------------------------------------------------------------------------
 static size_t moa_ws_bytes(int T, int kslots, int heads, int backward) {
@@ -723,6 +763,84 @@ int smoe_moa_attn_bwd(const void* q, const void* k, const void* v, const void* o
   { PROF("moa.attn_dkv", 1);
     SMOE_TRY(launch_attn_dkv(q, k, v, lse, dout, inv, T, L, kslots, heads, dk, dv, dsum, err, s),
              "moa attn dkv"); }
+  return SMOE_OK;
+}
+
+int smoe_quantize_weights_fp8(const void* w, int E, int K, int N, smoe_dtype dt, uint8_t* codes,
+                              float* scales, void* stream) {
+  smoe::NvtxScope nvtx_scope("smoe_quantize_weights_fp8");
+  if (E <= 0 || K <= 0 || N <= 0) return fail(SMOE_ERR_INVALID_ARG, "bad sizes");
+  if (K % 16) return fail(SMOE_ERR_INVALID_ARG, "K must be a multiple of 16");
+  if (dt != SMOE_BF16) return fail(SMOE_ERR_UNSUPPORTED, "FP8 weights are quantised from bf16");
+  if ((long long)E * K * N >= (1LL << 40)) return fail(SMOE_ERR_INVALID_ARG, "tensor too large");
+  NEED(w, "w"); NEED(codes, "codes"); NEED(scales, "scales");
+  cudaStream_t s = (cudaStream_t)stream;
+  { PROF("fp8.quantize_w", 1);
+    SMOE_TRY(launch_quantize_weights_fp8(w, E, K, N, codes, scales, s), "quantize weights"); }
+  return SMOE_OK;
+}
+
+size_t smoe_mlp_fp8_workspace_size(const smoe_mlp_desc* desc) {
+  if (validate_fp8_desc(desc) != SMOE_OK) return 0;
+  return fp8_layout(nullptr, *desc).bytes;
+}
+
+int smoe_mlp_fwd_fp8(const smoe_mlp_desc* desc, const smoe_mlp_tensors* t, const smoe_fp8_weights* w8,
+                     void* stream) {
+  smoe::NvtxScope nvtx_scope("smoe_mlp_fwd_fp8");
+  int rc = validate_fp8_desc(desc);
+  if (rc != SMOE_OK) return rc;
+  NEED(t, "tensors"); NEED(w8, "fp8 weights");
+  const smoe_mlp_desc& m = *desc;
+  if (m.T == 0) return SMOE_OK;
+  NEED(t->x, "x"); NEED(t->w_r, "w_r"); NEED(t->y, "y"); NEED(t->topk_idx, "topk_idx");
+  NEED(t->gates, "gates"); NEED(t->sorted_slot, "sorted_slot"); NEED(t->expert_offsets, "expert_offsets");
+  NEED(t->h, "h"); NEED(t->a, "a");
+  NEED(w8->w1q, "w1q"); NEED(w8->s1, "s1"); NEED(w8->w2q, "w2q"); NEED(w8->s2, "s2");
+  ALIGNED(t->x, "x"); ALIGNED(t->w_r, "w_r"); ALIGNED(t->y, "y"); ALIGNED(t->h, "h"); ALIGNED(t->a, "a");
+  ALIGNED(w8->w1q, "w1q"); ALIGNED(w8->w2q, "w2q"); ALIGNED(w8->s1, "s1"); ALIGNED(w8->s2, "s2");
+  Fp8Ws l = fp8_layout(t->workspace, m);
+  if (!t->workspace || t->workspace_bytes < l.bytes)
+    return fail(SMOE_ERR_INVALID_ARG, "workspace too small (%zu < %zu)", t->workspace_bytes, l.bytes);
+  if (((uintptr_t)t->workspace & 255u) != 0) return fail(SMOE_ERR_INVALID_ARG, "workspace not 256-byte aligned");
+  if ((rc = check_tc(SMOE_BF16)) != SMOE_OK) return rc;
+  cudaError_t st;
+  unsigned* err = error_word(&st);
+  if (!err) return cuda_fail(st, "smoe_mlp_fwd_fp8");
+  cudaStream_t s = (cudaStream_t)stream;
+  const int S = m.T * m.k;
+  const int mf = m.act == SMOE_ACT_SWIGLU ? 2 * m.f : m.f;
+  { PROF("route", 1); SMOE_TRY(launch_route(t->x, t->w_r, t->b_r, m.T, m.d, m.E, m.k, SMOE_BF16, t->topk_idx, t->gates, err, s), "route"); }
+  { PROF("sort", sort_launches(m.T, m.k, m.E)); SMOE_TRY(launch_sort(t->topk_idx, m.T, m.k, m.E, t->sorted_slot, t->expert_offsets, l.sort, err, s, l.inv), "sort"); }
+  { PROF("fp8.quantize_x", 1); SMOE_TRY(launch_quantize_rows_fp8(t->x, m.T, m.d, l.x8, l.sx, s), "quantize x"); }
+  {  // H = (x8 W1_8[e]) sx s1, A = act(H)   (scatter -> group, fan-out k)
+    GroupedGemm g;
+    g.E = m.E; g.num_rows = S; g.offsets = t->expert_offsets; g.sorted_slot = t->sorted_slot;
+    g.K = m.d; g.a = l.x8; g.lda = m.d; g.a_rows = m.T; g.a_mode = ROWS_GATHER; g.a_fan_out = m.k;
+    g.b = w8->w1q; g.b_kn = 0; g.NW = mf; g.n_out = m.f;
+    g.epi = EPI_ACT_FWD; g.act = m.act;
+    g.out_mode = ROWS_GROUPED; g.out = t->h; g.ldo = mf; g.out2 = t->a; g.ldo2 = m.f;
+    g.fp8 = 1; g.row_scale = l.sx; g.col_scale = w8->s1; g.err = err;
+    { PROF("gemm.fwd_up_fp8", 1); SMOE_TRY(launch_grouped_gemm_tc(g, s), "fp8 gemm1"); }
+  }
+  { PROF("fp8.quantize_a", 1); SMOE_TRY(launch_quantize_rows_fp8(t->a, S, m.f, l.a8, l.sa, s), "quantize a"); }
+  {  // slot rows g (a8 W2_8[e]) sa s2   (group -> group; the k-way combine scatters)
+    GroupedGemm g;
+    g.E = m.E; g.num_rows = S; g.offsets = t->expert_offsets; g.sorted_slot = t->sorted_slot;
+    g.K = m.f; g.a = l.a8; g.lda = m.f; g.a_rows = S; g.a_mode = ROWS_GROUPED;
+    g.b = w8->w2q; g.b_kn = 0; g.NW = m.d; g.n_out = m.d;
+    g.epi = EPI_STORE; g.gates = t->gates;
+    g.out_mode = ROWS_GROUPED; g.out = l.ycomb; g.ldo = m.d;
+    g.ksplit = l.ksplit; g.partial = l.kpart;
+    g.fp8 = 1; g.row_scale = l.sa; g.col_scale = w8->s2; g.err = err;
+    { PROF("gemm.fwd_down_fp8", 1); SMOE_TRY(launch_grouped_gemm_tc(g, s), "fp8 gemm2"); }
+    if (l.ksplit > 1) {
+      PROF("splitk_reduce", 1);
+      SMOE_TRY(launch_splitk_reduce(l.kpart, l.ksplit, S, m.d, t->sorted_slot, t->gates, l.ycomb, m.d, s),
+               "fp8 split-K reduce");
+    }
+  }
+  { PROF("combine.y", 1); SMOE_TRY(launch_combine(l.ycomb, l.inv, m.T, m.k, m.d, t->y, SMOE_BF16, nullptr, nullptr, nullptr, 0, s), "fp8 combine"); }
   return SMOE_OK;
 }
 

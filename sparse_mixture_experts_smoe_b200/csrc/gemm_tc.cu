@@ -282,8 +282,12 @@ __device__ __forceinline__ void teardown(SharedCtl& c) {
 // ---------------------------------------------------------------------------
 // Grouped-M kernel
 // ---------------------------------------------------------------------------
+// F8: e4m3 operands (kind::f8f6f4, B K-major): a K-block is 128 values, i.e. the
+// same 128 bytes per row as 64 bf16 values, so rings, swizzle and descriptors are
+// unchanged; the epilogue multiplies the fp32 sums by the A row's scale and the
+// weight column's scale before it does anything else.
 template <bool A_GATHER, bool B_KMAJOR, bool SWIGLU_FWD, bool PAIR, bool SPLITK = false,
-          bool SHORTK = false>
+          bool SHORTK = false, bool F8 = false>
 __global__ void __launch_bounds__(kThreads, 1)
 grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
                        const __grid_constant__ CUtensorMap tmB,
@@ -306,6 +310,8 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
                 "short-K layout");
   static_assert(STAGES * (A_BYTES + BSTAGE) <= kRingBytes, "stage ring exceeds its budget");
   static_assert(STAGES <= kMaxStages, "too many stages");
+  static_assert(!F8 || (B_KMAJOR && !PAIR && !SHORTK), "FP8 products: K-major weights, one CTA");
+  constexpr int BKE = F8 ? 2 * BK : BK;  // K values per stage (128 bytes per row either way)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
   uint8_t* sA = smem;
@@ -324,7 +330,7 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int first = PAIR ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
   const int stride = PAIR ? (int)(gridDim.x >> 1) : (int)gridDim.x;
-  const int nK = cdiv(g.K, BK);
+  const int nK = cdiv(g.K, BKE);
   // Split K (a product with too few tiles to fill the GPU, as at decode sizes):
   // work item L is K-blocks [kb_lo(L), kb_hi(L)) of tile L / ks, and the epilogue
   // stores the raw fp32 sum to its split's partial buffer (reduced afterwards).
@@ -357,9 +363,12 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
           };
           if (rank == 0)
             mbar_expect_tx(&c.fullA[r.s], (PAIR ? 2 : 1) * (BSTAGE + (A_GATHER ? 0 : A_BYTES)));
-          if (!A_GATHER) load2(sA + r.s * A_BYTES, &tmA, kb * BK, t.row0);
-          if (B_KMAJOR) {  // rows of W[e] = output columns; a pair's CTA takes its half
-            load3(b_dst, &tmB, kb * BK, t.nb * BN + (PAIR ? rank * (BN / 2) : 0), t.e);
+          if (!A_GATHER) load2(sA + r.s * A_BYTES, &tmA, kb * BKE, t.row0);
+          if (B_KMAJOR && SWIGLU_FWD) {  // BNo gate rows, then BNo up rows of W[e]^T
+            load3(b_dst, &tmB, kb * BKE, t.nb * BNo, t.e);
+            load3(b_dst + BNo * 128, &tmB, kb * BKE, g.n_out + t.nb * BNo, t.e);
+          } else if (B_KMAJOR) {  // rows of W[e] = output columns; a pair's CTA takes its half
+            load3(b_dst, &tmB, kb * BKE, t.nb * BN + (PAIR ? rank * (BN / 2) : 0), t.e);
           } else {
             // 64-column slabs; SwiGLU's tile is BNo gate columns then BNo up columns
             // (a pair: the gate half in CTA 0, the up half in CTA 1)
@@ -381,15 +390,17 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
     // thread t copies 16-byte chunk (t % 8) of tile rows t/8 + kRowStep j into
     // the 128-byte-swizzled K-major layout; rows past the expert's slice and
     // columns past K are zero-filled.
+    // (addressed in bytes: a row is lda elements of 2 bytes, or of 1 for F8)
     constexpr int kRowStep = GTHREADS / 8, kRowsPer = BM / kRowStep;
+    constexpr int ESZ = F8 ? 1 : 2;
     const int t = threadIdx.x - kGatherWarp0 * 32;
     const int cc = t & 7, r0 = t >> 3;
-    const bf16* A = reinterpret_cast<const bf16*>(g.a);
+    const char* A = reinterpret_cast<const char*>(g.a);
     Ring r;
     bool run = true;
     for (int L = first; run && L < total; L += stride) {
       const Tile tl = map_tile<PAIR>(c, g.offsets, g.E, nN, L / ks, rank);
-      const bf16* src[kRowsPer];
+      const char* src[kRowsPer];
       uint32_t ok_rows = 0;
 #pragma unroll
       for (int j = 0; j < kRowsPer; ++j) {
@@ -399,7 +410,7 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
           const int p = g.sorted_slot[i];
           const int xr = p / g.a_fan_out;
           if (p >= 0 && xr < g.a_rows) {
-            src[j] = A + (size_t)xr * g.lda + 8 * cc;
+            src[j] = A + (size_t)xr * g.lda * ESZ + 16 * cc;
             ok_rows |= 1u << j;
           } else {
             report_error(g.err, ERRBIT_DATA);
@@ -409,11 +420,11 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
       for (int kb = kb_lo(L), kb_end = kb_hi(L); kb < kb_end; ++kb) {
         if (!mbar_wait(&c.emptyA[r.s], r.ph ^ 1, abort_flag, g.err)) { run = false; break; }
         const uint32_t a_dst = smem_u32(sA + r.s * A_BYTES);
-        const bool col_ok = kb * BK + 8 * cc < g.K;
+        const bool col_ok = kb * 128 + 16 * cc < g.K * ESZ;
 #pragma unroll
         for (int j = 0; j < kRowsPer; ++j) {
           const bool ok = col_ok && ((ok_rows >> j) & 1u);
-          cp_async16(a_dst + sw128_off(r0 + kRowStep * j, cc), ok ? src[j] + kb * BK : A, ok ? 16u : 0u);
+          cp_async16(a_dst + sw128_off(r0 + kRowStep * j, cc), ok ? src[j] + kb * 128 : A, ok ? 16u : 0u);
         }
         cp_async_arrive(&c.fullA[r.s]);
         r.next(STAGES);
@@ -437,7 +448,8 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
         }
       }
     } else if (lane == 0) {
-      constexpr uint32_t idesc = idesc_bf16(PAIR ? 2 * BM : BM, BN, 0, B_KMAJOR ? 0 : 1);
+      constexpr uint32_t idesc = F8 ? idesc_e4m3(BM, BN)
+                                    : idesc_bf16(PAIR ? 2 * BM : BM, BN, 0, B_KMAJOR ? 0 : 1);
       Ring r;
       int it = 0;
       for (int L = first; L < total; L += stride, ++it) {
@@ -460,6 +472,7 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
             const uint64_t ad = desc_kmajor(a_addr + kk * 32);
             const uint64_t bd = B_KMAJOR ? desc_kmajor(b_addr + kk * 32) : desc_mnmajor(b_addr + kk * 2048);
             if (PAIR) umma_bf16_pair(d_tmem, ad, bd, idesc, ((kb - kb0) | kk) != 0);
+            else if (F8) umma_e4m3(d_tmem, ad, bd, idesc, ((kb - kb0) | kk) != 0);
             else umma_bf16(d_tmem, ad, bd, idesc, ((kb - kb0) | kk) != 0);
           }
           if (PAIR) {  // the stage is free in both CTAs
@@ -537,6 +550,11 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
       if (valid && !p_ok) report_error(g.err, ERRBIT_DATA);
       const int orow = g.out_mode == ROWS_GROUPED ? i : p;
       const float gate = (p_ok && g.gates) ? g.gates[p] : 1.0f;
+      // F8: the scale of this row's A operand (its source row) and the weight
+      // column scales of the tile's expert
+      const float rs = (F8 && p_ok) ? (g.a_mode == ROWS_GATHER ? g.row_scale[p / g.a_fan_out] : g.row_scale[i])
+                                    : 0.0f;
+      const float* col_sc = F8 ? g.col_scale + (size_t)t.e * g.NW : nullptr;
       const uint32_t trow = c.tmem_base + ((uint32_t)(q * 32) << 16) + buf * BN;
       const int wrow0 = t.row0 + q * 32;
       const bool boxed = (box_flags & kBoxStores) && wrow0 + 32 <= t.row_end;  // warp-uniform
@@ -600,6 +618,15 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
           }
         }
         if (!(act_bwd && (box_flags & kBoxLoads))) tmem_ld32(trow + c0, v);
+        if (F8) {  // fp32 sum x (A row's scale) x (weight column's scale)
+#pragma unroll
+          for (int q4 = 0; q4 < 8; ++q4) {
+            const float4 cs = 4 * q4 < ncols ? __ldg(reinterpret_cast<const float4*>(col_sc + n0 + 4 * q4))
+                                             : make_float4(0.f, 0.f, 0.f, 0.f);
+            v[4 * q4] *= rs * cs.x; v[4 * q4 + 1] *= rs * cs.y;
+            v[4 * q4 + 2] *= rs * cs.z; v[4 * q4 + 3] *= rs * cs.w;
+          }
+        }
         if (SPLITK) {  // split K: this split's raw fp32 sums
           if (valid) {
             float4* dst = reinterpret_cast<float4*>(
@@ -612,6 +639,16 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
           continue;
         }
         if (SWIGLU_FWD) tmem_ld32(trow + BNo + c0, u);
+        if (F8 && SWIGLU_FWD) {  // the up half's columns start at n_out
+#pragma unroll
+          for (int q4 = 0; q4 < 8; ++q4) {
+            const float4 cs = 4 * q4 < ncols
+                                  ? __ldg(reinterpret_cast<const float4*>(col_sc + g.n_out + n0 + 4 * q4))
+                                  : make_float4(0.f, 0.f, 0.f, 0.f);
+            u[4 * q4] *= rs * cs.x; u[4 * q4 + 1] *= rs * cs.y;
+            u[4 * q4 + 2] *= rs * cs.z; u[4 * q4 + 3] *= rs * cs.w;
+          }
+        }
         bulk_wait_read();  // this thread's earlier copies have read the staging area ...
         __syncwarp();      // ... and so have the other lanes'
         if (p_ok) {
@@ -1541,13 +1578,14 @@ struct EpiMaps {
 // 2-CTA clusters as the device can hold at once (fewer than half the SMs when a
 // GPC has an odd number of free SMs; a cluster beyond that would run its whole
 // share of the tile list after the others).
-template <bool AG, bool BK_, bool SW, bool SPLIT = false, bool SHORT = false>
+template <bool AG, bool BK_, bool SW, bool SPLIT = false, bool SHORT = false, bool F8 = false>
 cudaError_t launch_g(const CUtensorMap& ta, const CUtensorMap& tb, const EpiMaps& m,
                      const GroupedGemm& g, int nN, long long tiles, cudaStream_t s) {
-  auto kern = grouped_gemm_tc_kernel<AG, BK_, SW, kPairM, SPLIT, SHORT>;
+  constexpr bool kPair = F8 ? false : kPairM;
+  auto kern = grouped_gemm_tc_kernel<AG, BK_, SW, kPair, SPLIT, SHORT, F8>;
   cudaError_t e = prep(kern, kGroupedSmem);
   if (e != cudaSuccess) return e;
-  if (!kPairM) {
+  if (!kPair) {
     const int grid = (int)(tiles < num_sms() ? tiles : num_sms());
     kern<<<grid, kThreads, kGroupedSmem, s>>>(ta, tb, m.out, m.out2, m.xa, m.xh, g, nN, m.flags);
     return cudaGetLastError();
@@ -1638,21 +1676,65 @@ bool tc_supported() {
 
 int tc_tile_cols() { return BN; }
 
-int grouped_ksplit(int num_rows, int E, int n_out, int K) {
+int grouped_ksplit(int num_rows, int E, int n_out, int K, int fp8) {
   constexpr long long kSms = 148;  // a fixed count, so the split (and the workspace) is the same on any GPU
   const long long tiles = (long long)(cdiv(num_rows, BM) + (E < num_rows ? E : num_rows)) * cdiv(n_out, BN);
   if (tiles <= 0 || tiles * 2 > kSms) return 1;
   int ks = (int)((kSms + tiles - 1) / tiles);
   if (ks > 8) ks = 8;
-  const int most = cdiv(K, BK) / 4;  // at least four K-blocks per split
+  const int most = cdiv(K, fp8 ? 2 * BK : BK) / 4;  // at least four K-blocks per split
   if (ks > most) ks = most;
   return ks > 1 ? ks : 1;
+}
+
+// FP8 products (e4m3 codes, K-major weights): the up projection with a row gather
+// and the activation epilogue, and the down projection (grouped rows, plain or
+// split-K store).
+cudaError_t launch_grouped_gemm_fp8(const GroupedGemm& g, cudaStream_t s) {
+  const bool swiglu = g.epi == EPI_ACT_FWD && g.act == SMOE_ACT_SWIGLU;
+  const int BNo = swiglu ? BN / 2 : BN;
+  const int nN = cdiv(g.n_out, BNo);
+  if (g.b_kn != 0 || !g.row_scale || !g.col_scale || g.epi == EPI_ACT_BWD) return cudaErrorInvalidValue;
+  if (g.K % 16 || g.ksplit > cdiv(g.K, 2 * BK)) return cudaErrorInvalidValue;
+  CUtensorMap ta, tb;
+  {  // A codes [a_rows, K] (grouped products): 128 x 128 boxes
+    const uint64_t dims[2] = {(uint64_t)g.K, (uint64_t)(g.a_rows > 0 ? g.a_rows : 1)};
+    const uint64_t str[1] = {(uint64_t)g.lda};
+    const uint32_t box[2] = {128, (uint32_t)BM};
+    cudaError_t e = make_map(&ta, g.a, 2, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B,
+                             CU_TENSOR_MAP_DATA_TYPE_UINT8);
+    if (e != cudaSuccess) return e;
+  }
+  {  // W codes [E, NW, K]: dims {K, NW, E}; SwiGLU loads its gate and up rows separately
+    const uint64_t dims[3] = {(uint64_t)g.K, (uint64_t)g.NW, (uint64_t)g.E};
+    const uint64_t str[2] = {(uint64_t)g.K, (uint64_t)g.NW * g.K};
+    const uint32_t box[3] = {128, (uint32_t)(swiglu ? BN / 2 : BN), 1};
+    cudaError_t e = make_map(&tb, g.b, 3, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B,
+                             CU_TENSOR_MAP_DATA_TYPE_UINT8);
+    if (e != cudaSuccess) return e;
+  }
+  EpiMaps m;
+  const int parts = swiglu ? 2 : 1;
+  bool st = g.out != nullptr && (g.out_mode == ROWS_GROUPED);
+  if (st && out_map(&m.out, g.out, g.n_out, parts, g.num_rows, g.ldo) != cudaSuccess) st = false;
+  if (st && g.out2 && out_map(&m.out2, g.out2, g.n_out, 1, g.num_rows, g.ldo2) != cudaSuccess) st = false;
+  m.flags = st ? kBoxStores : 0;
+  const long long tiles = (long long)(cdiv(g.num_rows, BM) + g.E) * nN * (g.ksplit > 1 ? g.ksplit : 1);
+  if (g.a_mode == ROWS_GATHER) {
+    if (g.ksplit > 1) return cudaErrorInvalidValue;
+    return swiglu ? launch_g<true, true, true, false, false, true>(ta, tb, m, g, nN, tiles, s)
+                  : launch_g<true, true, false, false, false, true>(ta, tb, m, g, nN, tiles, s);
+  }
+  if (g.epi != EPI_STORE) return cudaErrorInvalidValue;
+  if (g.ksplit > 1) return launch_g<false, true, false, true, false, true>(ta, tb, m, g, nN, tiles, s);
+  return launch_g<false, true, false, false, false, true>(ta, tb, m, g, nN, tiles, s);
 }
 
 cudaError_t launch_grouped_gemm_tc(const GroupedGemm& g, cudaStream_t s) {
   if (g.num_rows == 0) return cudaSuccess;
   if (g.E > kMaxE) return cudaErrorInvalidValue;
   if (g.out_f32) return cudaErrorInvalidValue;  // every output of this path is bf16
+  if (g.fp8) return launch_grouped_gemm_fp8(g, s);
   if (g.ksplit > 1) {  // split K: the plain-store epilogue of a TMA-fed single-CTA product
     if (g.a_mode != ROWS_GROUPED || g.epi != EPI_STORE || kPairM || g.partial == nullptr ||
         g.ksplit > cdiv(g.K, BK))
@@ -1669,7 +1751,8 @@ cudaError_t launch_grouped_gemm_tc(const GroupedGemm& g, cudaStream_t s) {
   if (kmaj) {  // W[e] is [NW, K]: dims {K, NW, E}
     const uint64_t dims[3] = {(uint64_t)g.K, (uint64_t)g.NW, (uint64_t)g.E};
     const uint64_t str[2] = {(uint64_t)g.K * 2, (uint64_t)g.NW * g.K * 2};
-    const uint32_t box[3] = {64, kPairM ? BN / 2 : BN, 1};
+    // (SwiGLU's forward loads its gate and up rows as two half-height boxes)
+    const uint32_t box[3] = {64, (uint32_t)((kPairM || swiglu) ? BN / 2 : BN), 1};
     e = make_map(&tb, g.b, 3, dims, str, box);
   } else {  // W[e] is [K, NW]: dims {NW, K, E}
     const uint64_t dims[3] = {(uint64_t)g.NW, (uint64_t)g.K, (uint64_t)g.E};

@@ -59,6 +59,11 @@ struct GroupedGemm {
   // applies the gates and stores out
   int ksplit = 1;
   float* partial = nullptr;
+  // fp8 = 1: a and b hold e4m3 codes (b K-major, b_kn = 0); the fp32 sums are
+  // multiplied by row_scale[source row of A] and col_scale[e * NW + column]
+  int fp8 = 0;
+  const float* row_scale = nullptr;
+  const float* col_scale = nullptr;
   unsigned* err = nullptr;
 };
 
@@ -129,7 +134,7 @@ cudaError_t launch_splitk_reduce(const float* partial, int ksplit, int num_rows,
 // Splits of K for a grouped product of num_rows rows over E experts with n_out
 // output columns and K-dimension K: > 1 only when even the most tiles it can have
 // would leave most SMs idle (decode-sized batches).
-int grouped_ksplit(int num_rows, int E, int n_out, int K);
+int grouped_ksplit(int num_rows, int E, int n_out, int K, int fp8 = 0);
 
 cudaError_t launch_grouped_gemm_simt(const GroupedGemm& g, smoe_dtype dt, cudaStream_t s);
 cudaError_t launch_dw_gemm_simt(const DwGemm& g, smoe_dtype dt, cudaStream_t s);
@@ -149,6 +154,13 @@ cudaError_t launch_attn_dq(const void* q, const void* k, const void* v, const fl
 cudaError_t launch_attn_dkv(const void* q, const void* k, const void* v, const float* lse,
                             const void* dout, const int32_t* inv, int T, int L, int kslots, int heads,
                             void* dk, void* dv, const float* dsum, unsigned* err, cudaStream_t s);
+
+// e4m3 quantisation (fp8.cu): rows of a bf16 [rows, cols] matrix with one scale per
+// row; weights [E, K, N] bf16 -> codes [E, N, K] with one scale per (e, column)
+cudaError_t launch_quantize_rows_fp8(const void* x, int rows, int cols, uint8_t* codes, float* scales,
+                                     cudaStream_t s);
+cudaError_t launch_quantize_weights_fp8(const void* w, int E, int K, int N, uint8_t* codes, float* scales,
+                                        cudaStream_t s);
 
 // tcgen05 / TMEM path (bf16 only); *_supported() checks the device once.
 bool tc_supported();
