@@ -509,7 +509,34 @@ def run_decode(args, world, rank):
                 "l2": "weights larger than L2, no flush"}
         if rank == 0:
             print(json.dumps(line), flush=True)
-        del st, inp, p
+        # the same forward with e4m3 expert weights (codes + per-column fp32 scales):
+        # half the weight bytes per token
+        w1q, s1 = smoe.smoe_quantize_weights_fp8(inp["w1"])
+        w2q, s2 = smoe.smoe_quantize_weights_fp8(inp["w2"])
+        q = (inp["x"], inp["w_r"], inp["b_r"], w1q, s1, w2q, s2)
+        for _ in range(args.warmup):
+            smoe.smoe_mlp_fwd_fp8(st, *q)
+        torch.cuda.synchronize()
+        barrier(world)
+        e0.record()
+        for _ in range(args.steps):
+            smoe.smoe_mlp_fwd_fp8(st, *q)
+        e1.record()
+        torch.cuda.synchronize()
+        barrier(world)
+        ms8 = max_over_ranks(e0.elapsed_time(e1), world) / args.steps
+        if smoe.smoe_check() != 0:
+            raise SystemExit(f"device error word set in FP8 decode T={T}")
+        wbytes8 = used * (d * mf + f * d) + used * (mf + d) * 4
+        gbs8 = wbytes8 / (ms8 / 1e3) / 1e9
+        line8 = dict(line, dtype="e4m3 weights, bf16 activations", ms_fwd=round(ms8, 4),
+                     tokens_per_s=round(T * world / (ms8 / 1e3), 1), weight_bytes=wbytes8,
+                     roofline={"bound": "hbm", "achieved": round(gbs8, 1), "peak": peaks["hbm_gbs"],
+                               "unit": "GB/s", "frac": round(gbs8 / peaks["hbm_gbs"], 4), "traffic": None},
+                     speedup_vs_bf16=round(ms / ms8, 3))
+        if rank == 0:
+            print(json.dumps(line8), flush=True)
+        del st, inp, p, q, w1q, w2q
 
 
 def run_sweep(args, world, rank):
