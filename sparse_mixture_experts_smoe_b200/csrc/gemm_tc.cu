@@ -51,7 +51,7 @@ constexpr int BK = 64;            // K per stage: one 128-byte swizzle row of bf
 constexpr int BN = 256;           // MMA N
 constexpr int kThreads = 512;        // 16 warps
 constexpr int kGatherWarp0 = 8;       // first warp of the row gather
-constexpr int kGatherThreads = 256;   // grouped-M kernel: warps 8-15
+constexpr int kGatherThreads = 256;   // grouped-M kernel: warps 8-15 (or 8-11, below)
 constexpr int kDwGatherThreads = 256; // dW kernel: warps 8-15 gather (more copies in flight)
 constexpr int kDwThreads = 512;
 // Warp roles.  Grouped-M kernel: 0 TMA, 1 MMA, 2-3 idle, 4-7 epilogue, 8-15 row
@@ -139,11 +139,6 @@ constexpr int kWarpStaging = 32 * kSlotBytes;  // 13 x 512: boxes stay 512-byte 
 static_assert(3 * kBoxBytes <= kWarpStaging && kWarpStaging % 512 == 0, "staging layout");
 constexpr int kStagingBytes = 4 * kWarpStaging;
 enum : int { kBoxStores = 1, kBoxLoads = 2 };  // grouped-epilogue box modes (launch flags)
-// Grouped-M GEMMs run as CTA pairs sharing M = 256 MMAs (cta_group::2).
-#ifndef SMOE_PAIR_M
-#define SMOE_PAIR_M 0
-#endif
-constexpr bool kPairM = SMOE_PAIR_M != 0;
 
 constexpr size_t kCtlBytes = (sizeof(SharedCtl) + 1023) / 1024 * 1024;
 constexpr size_t kGroupedSmem = 1024 + (size_t)kRingBytes + kCtlBytes + kStagingBytes;
@@ -287,7 +282,7 @@ __device__ __forceinline__ void teardown(SharedCtl& c) {
 // unchanged; the epilogue multiplies the fp32 sums by the A row's scale and the
 // weight column's scale before it does anything else.
 template <bool A_GATHER, bool B_KMAJOR, bool SWIGLU_FWD, bool PAIR, bool SPLITK = false,
-          bool SHORTK = false, bool F8 = false>
+          bool SHORTK = false, bool F8 = false, bool G128 = false>
 __global__ void __launch_bounds__(kThreads, 1)
 grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
                        const __grid_constant__ CUtensorMap tmB,
@@ -302,9 +297,12 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
   // holds half of B per stage, so its ring is deeper.  SHORTK (a gathered product
   // with a short K): 3 stages, half the gather warps (8-11), and warps 12-15 as a
   // second epilogue group staging in the ring space the fourth stage leaves free.
+  // G128: a long-K gathered product with 4 gather warps (8-11) instead of 8: half
+  // the per-stage barrier arrivals, measured faster on the tensor pipe.
   constexpr int BSTAGE = PAIR ? B_BYTES / 2 : B_BYTES;
   constexpr int STAGES = PAIR ? 6 : (SHORTK ? 3 : 4);
-  constexpr int GTHREADS = SHORTK ? kGatherThreads / 2 : kGatherThreads;  // gather threads
+  constexpr int GTHREADS = (SHORTK || G128) ? 128 : kGatherThreads;  // gather threads
+  static_assert(!G128 || (A_GATHER && !SHORTK), "4-warp gather of a long-K product");
   static_assert(!SHORTK || (A_GATHER && !PAIR &&
                             STAGES * (A_BYTES + BSTAGE) + 4 * kWarpStaging <= kRingBytes),
                 "short-K layout");
@@ -476,8 +474,7 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
             else umma_bf16(d_tmem, ad, bd, idesc, ((kb - kb0) | kk) != 0);
           }
           if (PAIR) {  // the stage is free in both CTAs
-            umma_commit_pair(smem_u32(&c.emptyA[r.s]));
-            umma_commit_pair(peer_addr(&c.emptyA[r.s], 1));
+            umma_commit_pair_both(&c.emptyA[r.s]);
           } else {
             umma_commit(&c.emptyA[r.s]);
           }
@@ -485,8 +482,7 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
         }
         if (!ok) break;
         if (PAIR) {
-          umma_commit_pair(smem_u32(&c.tfull[buf]));
-          umma_commit_pair(peer_addr(&c.tfull[buf], 1));
+          umma_commit_pair_both(&c.tfull[buf]);
         } else {
           umma_commit(&c.tfull[buf]);
         }
@@ -1044,7 +1040,7 @@ __device__ __forceinline__ void dw_index_producer(SharedCtl& c, DwExtra& x, cons
         const int r = ra[b] + lane + 32 * q;
         if (A_GATHER) {
           int a_src;
-          if (A_SCALE && a_ident) a_src = (va[b][q] < 0 || r >= g.a_rows) ? -1 : r;
+          if (a_ident) a_src = (va[b][q] < 0 || r >= g.a_rows) ? -1 : r;  // grouped A, gathered by row
           else a_src = src_of(va[b][q], a_shift, g.a_fan_out, g.a_rows);
           x.idx[ri.s][0][lane + 32 * q] = a_src;
         }
@@ -1483,14 +1479,12 @@ dw_pair_tc_kernel(const __grid_constant__ CUtensorMap tmB, const __grid_constant
           for (int kk = 0; kk < BK / 16; ++kk)
             umma_bf16_pair(d_tmem, desc_mnmajor(a_addr + kk * 2048), desc_mnmajor(b_addr + kk * 2048), idesc,
                            (kb | kk) != 0);
-          umma_commit_pair(smem_u32(&c.emptyA[r.s]));  // the stage is free in both CTAs
-          umma_commit_pair(peer_addr(&c.emptyA[r.s], 1));
+          umma_commit_pair_both(&c.emptyA[r.s]);  // the stage is free in both CTAs
           r.next(STAGES);
         }
         if (!ok) break;
         if (nK > 0) {
-          umma_commit_pair(smem_u32(&c.tfull[buf]));
-          umma_commit_pair(peer_addr(&c.tfull[buf], 1));
+          umma_commit_pair_both(&c.tfull[buf]);
         } else {  // an empty expert: both epilogues write zeros
           mbar_arrive(&c.tfull[buf]);
           mbar_arrive_cluster(peer_addr(&c.tfull[buf], 1));
@@ -1578,11 +1572,12 @@ struct EpiMaps {
 // 2-CTA clusters as the device can hold at once (fewer than half the SMs when a
 // GPC has an odd number of free SMs; a cluster beyond that would run its whole
 // share of the tile list after the others).
-template <bool AG, bool BK_, bool SW, bool SPLIT = false, bool SHORT = false, bool F8 = false>
+template <bool AG, bool BK_, bool SW, bool kPair = false, bool SPLIT = false, bool SHORT = false,
+          bool F8 = false, bool G128 = false>
 cudaError_t launch_g(const CUtensorMap& ta, const CUtensorMap& tb, const EpiMaps& m,
                      const GroupedGemm& g, int nN, long long tiles, cudaStream_t s) {
-  constexpr bool kPair = F8 ? false : kPairM;
-  auto kern = grouped_gemm_tc_kernel<AG, BK_, SW, kPair, SPLIT, SHORT, F8>;
+  static_assert(!kPair || !(SPLIT || SHORT || F8), "pairs: plain bf16 products");
+  auto kern = grouped_gemm_tc_kernel<AG, BK_, SW, kPair, SPLIT, SHORT, F8, G128>;
   cudaError_t e = prep(kern, kGroupedSmem);
   if (e != cudaSuccess) return e;
   if (!kPair) {
@@ -1722,12 +1717,12 @@ cudaError_t launch_grouped_gemm_fp8(const GroupedGemm& g, cudaStream_t s) {
   const long long tiles = (long long)(cdiv(g.num_rows, BM) + g.E) * nN * (g.ksplit > 1 ? g.ksplit : 1);
   if (g.a_mode == ROWS_GATHER) {
     if (g.ksplit > 1) return cudaErrorInvalidValue;
-    return swiglu ? launch_g<true, true, true, false, false, true>(ta, tb, m, g, nN, tiles, s)
-                  : launch_g<true, true, false, false, false, true>(ta, tb, m, g, nN, tiles, s);
+    return swiglu ? launch_g<true, true, true, false, false, false, true>(ta, tb, m, g, nN, tiles, s)
+                  : launch_g<true, true, false, false, false, false, true>(ta, tb, m, g, nN, tiles, s);
   }
   if (g.epi != EPI_STORE) return cudaErrorInvalidValue;
-  if (g.ksplit > 1) return launch_g<false, true, false, true, false, true>(ta, tb, m, g, nN, tiles, s);
-  return launch_g<false, true, false, false, false, true>(ta, tb, m, g, nN, tiles, s);
+  if (g.ksplit > 1) return launch_g<false, true, false, false, true, false, true>(ta, tb, m, g, nN, tiles, s);
+  return launch_g<false, true, false, false, false, false, true>(ta, tb, m, g, nN, tiles, s);
 }
 
 cudaError_t launch_grouped_gemm_tc(const GroupedGemm& g, cudaStream_t s) {
@@ -1736,14 +1731,27 @@ cudaError_t launch_grouped_gemm_tc(const GroupedGemm& g, cudaStream_t s) {
   if (g.out_f32) return cudaErrorInvalidValue;  // every output of this path is bf16
   if (g.fp8) return launch_grouped_gemm_fp8(g, s);
   if (g.ksplit > 1) {  // split K: the plain-store epilogue of a TMA-fed single-CTA product
-    if (g.a_mode != ROWS_GROUPED || g.epi != EPI_STORE || kPairM || g.partial == nullptr ||
-        g.ksplit > cdiv(g.K, BK))
+    if (g.a_mode != ROWS_GROUPED || g.epi != EPI_STORE || g.partial == nullptr || g.ksplit > cdiv(g.K, BK))
       return cudaErrorInvalidValue;
   }
   const bool swiglu = g.epi == EPI_ACT_FWD && g.act == SMOE_ACT_SWIGLU;
   const int BNo = swiglu ? BN / 2 : BN;
   const int nN = cdiv(g.n_out, BNo);
   const bool gather = g.a_mode == ROWS_GATHER;
+  // A gathered product with a short K has little main loop per tile to hide its
+  // epilogue behind: half the gather warps become a second epilogue group.  Not for
+  // SwiGLU's forward, whose epilogue (half-width tiles) is short and whose gather
+  // then sets the pace (measured slower with 4 gather warps).
+  const bool shortk = gather && !swiglu && g.K <= kShortK && g.ksplit <= 1;
+  // Long-K products over large expert slices (at least 2048 rows per expert on
+  // average, K >= 4096): TMA-fed ones and the activation-backward product run on
+  // CTA pairs (six-stage rings of 32 KB per CTA, half of B per CTA), gathered ones
+  // gather with 4 warps.  Measured on the Mixtral-shaped layer: down projection
+  // -5%, dx -8%, dA' -5%, up projection -5% (4 warps, one CTA; on pairs it was
+  // slower).  Smaller shapes keep the single-CTA kernels they were tuned with.
+  const bool big = g.ksplit <= 1 && g.K >= 4096 && (long long)g.num_rows >= 2048LL * g.E;
+  const bool pair = big && (!gather || g.epi == EPI_ACT_BWD);
+  const bool g128 = gather && !shortk && g.K >= 4096;
   CUtensorMap ta, tb;
   cudaError_t e = rows_map(&ta, g.a, g.K, g.a_rows, g.lda, BM);  // unused when gathered
   if (e != cudaSuccess) return e;
@@ -1752,7 +1760,7 @@ cudaError_t launch_grouped_gemm_tc(const GroupedGemm& g, cudaStream_t s) {
     const uint64_t dims[3] = {(uint64_t)g.K, (uint64_t)g.NW, (uint64_t)g.E};
     const uint64_t str[2] = {(uint64_t)g.K * 2, (uint64_t)g.NW * g.K * 2};
     // (SwiGLU's forward loads its gate and up rows as two half-height boxes)
-    const uint32_t box[3] = {64, (uint32_t)((kPairM || swiglu) ? BN / 2 : BN), 1};
+    const uint32_t box[3] = {64, (uint32_t)((pair || swiglu) ? BN / 2 : BN), 1};
     e = make_map(&tb, g.b, 3, dims, str, box);
   } else {  // W[e] is [K, NW]: dims {NW, K, E}
     const uint64_t dims[3] = {(uint64_t)g.NW, (uint64_t)g.K, (uint64_t)g.E};
@@ -1774,21 +1782,21 @@ cudaError_t launch_grouped_gemm_tc(const GroupedGemm& g, cudaStream_t s) {
   if (ld && out_map(&m.xa, g.aux_a, g.n_out, 1, g.num_rows, g.ld_aux_a) != cudaSuccess) ld = false;
   if (ld && need_h && out_map(&m.xh, g.aux_h, g.n_out, parts, g.num_rows, g.ld_aux_h) != cudaSuccess) ld = false;
   m.flags = (st ? kBoxStores : 0) | (ld ? kBoxLoads : 0);
-  const int tm = kPairM ? 2 * BM : BM;  // rows per M tile
+  const int tm = pair ? 2 * BM : BM;  // rows per M tile
   const long long tiles = (long long)(cdiv(g.num_rows, tm) + g.E) * nN * (g.ksplit > 1 ? g.ksplit : 1);
   if (g.ksplit > 1) {  // grouped A, plain store (checked above)
-    if (kmaj) return launch_g<false, true, false, true>(ta, tb, m, g, nN, tiles, s);
-    return launch_g<false, false, false, true>(ta, tb, m, g, nN, tiles, s);
+    if (kmaj) return launch_g<false, true, false, false, true>(ta, tb, m, g, nN, tiles, s);
+    return launch_g<false, false, false, false, true>(ta, tb, m, g, nN, tiles, s);
   }
-#define SMOE_LAUNCH_G(AG, KM, SW) launch_g<AG, KM, SW>(ta, tb, m, g, nN, tiles, s)
-  // A gathered product with a short K has little main loop per tile to hide its
-  // epilogue behind: half the gather warps become a second epilogue group.  Not for
-  // SwiGLU's forward, whose epilogue (half-width tiles) is short and whose gather
-  // then sets the pace (measured slower with 4 gather warps).
-  if (gather && !swiglu && !kPairM && g.K <= kShortK) {
-    if (kmaj) return launch_g<true, true, false, false, true>(ta, tb, m, g, nN, tiles, s);
-    return launch_g<true, false, false, false, true>(ta, tb, m, g, nN, tiles, s);
+  if (shortk) {
+    if (kmaj) return launch_g<true, true, false, false, false, true>(ta, tb, m, g, nN, tiles, s);
+    return launch_g<true, false, false, false, false, true>(ta, tb, m, g, nN, tiles, s);
   }
+#define SMOE_LAUNCH_G(AG, KM, SW)                                                              \
+  (pair ? (g128 ? launch_g<AG, KM, SW, true, false, false, false, AG>(ta, tb, m, g, nN, tiles, s)        \
+                : launch_g<AG, KM, SW, true>(ta, tb, m, g, nN, tiles, s))                               \
+        : (g128 ? launch_g<AG, KM, SW, false, false, false, false, AG>(ta, tb, m, g, nN, tiles, s)       \
+                : launch_g<AG, KM, SW, false>(ta, tb, m, g, nN, tiles, s)))
   if (gather) {
     if (kmaj) return swiglu ? SMOE_LAUNCH_G(true, true, true) : SMOE_LAUNCH_G(true, true, false);
     return swiglu ? SMOE_LAUNCH_G(true, false, true) : SMOE_LAUNCH_G(true, false, false);
@@ -1832,11 +1840,17 @@ cudaError_t launch_dw_gemm_tc(const DwGemm& g_in, cudaStream_t s) {
   // Gated rows with B by TMA and at least two 128-column halves of M run on CTA
   // pairs: their six-stage rings keep more gathered stages in flight while the
   // gate pass holds stages back (measured 9% faster than one CTA on the
-  // Mixtral-shaped dW2; without gates the pair measured the same as one CTA, so
-  // those keep the single-CTA kernel).
-  if (sc && !bg && g.M > BM) {
+  // Mixtral-shaped dW2).  Ungated products over large slices (at least 2048 rows
+  // per expert on average) do too, since the pair commits once to both CTAs
+  // (measured 2-3% faster on the Mixtral-shaped dW1 and dW2); smaller ones keep
+  // the single-CTA kernel.
+  const bool big = (long long)g.num_rows >= 2048LL * g.E;
+  if ((sc || (ag && big)) && !bg && g.M > BM) {
     const int nMP = cdiv(g.M, 2 * BM);
     const long long ptiles = (long long)g.E * nMP * nN;
+    if (!sc)
+      return trans ? launch_dp<false, true>(tb, td, d_boxed, g, nMP, nN, ptiles, s)
+                   : launch_dp<false, false>(tb, td, d_boxed, g, nMP, nN, ptiles, s);
     return trans ? launch_dp<true, true>(tb, td, d_boxed, g, nMP, nN, ptiles, s)
                  : launch_dp<true, false>(tb, td, d_boxed, g, nMP, nN, ptiles, s);
   }

@@ -227,6 +227,17 @@ __device__ __forceinline__ void umma_commit_pair(uint32_t cl_addr) {
                    cl_addr)
                : "memory");
 }
+// Arrive on the barrier at the same shared-memory offset in both CTAs of the pair
+// (CTA mask 0b11) once this thread's earlier pair MMAs have completed: one
+// multicast commit.  Two separate commits, one per CTA, measured about 9% fewer
+// MMAs per cycle on a TMA-fed pair.
+__device__ __forceinline__ void umma_commit_pair_both(uint64_t* bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+          smem_u32(bar)),
+      "h"((uint16_t)0x3)
+      : "memory");
+}
 
 // 32 consecutive fp32 columns of this thread's tensor-memory lane.
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {

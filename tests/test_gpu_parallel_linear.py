@@ -31,8 +31,9 @@ def _problem(dtype, mode, gated, seed=0, shape=None):
     gi, go, fo_k, comb = MODES[mode]
     g = torch.Generator(device="cuda").manual_seed(seed)
     idx = torch.randint(0, E, (T, k), generator=g, device="cuda", dtype=torch.int32)
-    idx[idx == 3] = 1                      # expert 3 is empty
-    idx[: T // 3] = torch.where(idx[: T // 3] == 0, 4, idx[: T // 3])  # skew the sizes
+    if E > 4:
+        idx[idx == 3] = 1                      # expert 3 is empty
+        idx[: T // 3] = torch.where(idx[: T // 3] == 0, 4, idx[: T // 3])  # skew the sizes
     ss, off = smoe.smoe_sort(idx, E)
     fan_out = k if fo_k else 1
     x_rows = T * k if (gi or fan_out == 1) else T
@@ -173,3 +174,31 @@ def test_parallel_linear_gated_dw_narrow(mode):
     assert_close("dw", dw, ref["dw"], torch.bfloat16)
     assert_close("dgates", dg, ref["dg"], torch.bfloat16)
     assert np.all(dw[3].cpu().numpy() == 0.0)
+
+
+@pytest.mark.parametrize("mode", ["group2group", "scatter2group_fanout", "group2scatter_combine"])
+def test_parallel_linear_long_k_pairs(mode):
+    """K = 4096 over slices of at least 2048 rows per expert: the TMA-fed products
+    run on CTA pairs, the gathered ones gather with 4 warps, and the dW of a
+    gathered operand runs on the pair dW kernel; every element against the oracle
+    (ragged pair tiles and a ragged N tile)."""
+    gated = mode == "group2scatter_combine"
+    P = _problem(torch.bfloat16, mode, gated, seed=5, shape=dict(T=2200, k=2, K=4096, N=264, E=2))
+    y = smoe.parallel_linear_fwd(P["x"], P["w"], P["ss"], P["off"], P["fan_out"], P["gi"], P["go"],
+                                 P["gates"], P["ck"])
+    dx, dw, dg = smoe.parallel_linear_bwd(P["dy"], P["x"], P["w"], P["ss"], P["off"], P["fan_out"],
+                                          P["gi"], P["go"], P["gates"], P["ck"], want_dgates=gated)
+    torch.cuda.synchronize()
+    assert smoe.smoe_check() == 0
+    ss, off = P["ss"].cpu().numpy(), P["off"].cpu().numpy()
+    assert np.diff(off).min() >= 2048
+    gts = None if P["gates"] is None else P["gates"].cpu().double().numpy()
+    ref_y = oracle.pl_fwd(P["x"].cpu(), P["w"].cpu(), ss, off, P["fan_out"], P["gi"], P["go"], gts,
+                          P["ck"])
+    assert_close("y", y, ref_y, torch.bfloat16)
+    ref = oracle.pl_bwd(P["dy"].cpu(), P["x"].cpu(), P["w"].cpu(), ss, off, P["fan_out"], P["gi"],
+                        P["go"], gts, P["ck"], want_dg=gated)
+    assert_close("dx", dx, ref["dx"], torch.bfloat16)
+    assert_close("dw", dw, ref["dw"], torch.bfloat16)
+    if gated:
+        assert_close("dgates", dg, ref["dg"], torch.bfloat16)
