@@ -359,6 +359,23 @@ size_t smoe_mlp_fp8_workspace_size(const smoe_mlp_desc* desc);
 int smoe_mlp_fwd_fp8(const smoe_mlp_desc* desc, const smoe_mlp_tensors* t, const smoe_fp8_weights* w8,
                      void* stream);
 
+/* smoe_set_gemm_policy: how the tensor-core GEMMs of every later call in this
+ * process choose their kernel variant (no counterpart on the pages; every policy
+ * computes the same products, bit for bit on the same GPU).
+ *   0 (default): one CTA per 128-row tile, 8 gather warps, tiles of an expert in
+ *     panels of 16 M tiles.  Measured fastest per step over 20 steps of the
+ *     Mixtral-shaped layer under the B200's 1 kW power cap.
+ *   1: long-K products (K >= 4096) over large expert slices (at least 2048 rows per
+ *     expert on average): TMA-fed ones on 2-CTA pairs sharing M = 256 MMAs,
+ *     gathered ones with 4 gather warps, and ungated weight gradients on pairs.
+ *     More MMAs per cycle (about 90% against 78% of the tensor pipe on the
+ *     TMA-fed products) and about 2.5% less time per step in short runs below the
+ *     power cap, but more DRAM traffic: over sustained steps under the cap it
+ *     measured equal or slower.
+ * Set it between calls, not while a call of this library is in flight.
+ * Returns SMOE_OK, or SMOE_ERR_INVALID_ARG for another value. */
+int smoe_set_gemm_policy(int policy);
+
 /* ---------------------------------------------------------------------------
  * Instrumentation (the pages have no counterpart; used by the benchmark).
  *

@@ -74,6 +74,7 @@ def lib():
     L.smoe_sort.argtypes = [_vp, _c_int, _c_int, _c_int, _vp, _vp, _vp, _c_size, _vp]
     L.smoe_sort_static.argtypes = [_vp, _c_int, _c_int, _c_int, _vp, _vp, _vp]
     L.smoe_selftest_wait_timeout.argtypes = [_c_int, _vp]
+    L.smoe_set_gemm_policy.argtypes = [_c_int]
     L.parallel_linear_fwd_workspace_size.restype = _c_size
     L.parallel_linear_fwd_workspace_size.argtypes = [_c_int] * 6
     L.parallel_linear_fwd.argtypes = [_vp, _c_int, _c_int, _vp, _c_int, _c_int, _vp, _vp, _c_int,
@@ -218,6 +219,13 @@ def smoe_sort(topk_idx, E, stream=None):
     _check(lib().smoe_sort(_ptr(topk_idx), T, k, E, _ptr(ss), _ptr(off), _ptr(ws), ws.numel(),
                            _stream(stream)))
     return ss, off
+
+
+def smoe_set_gemm_policy(policy: int):
+    """Kernel-selection policy of the tensor-core GEMMs for later calls (0: one
+    CTA per tile, the default; 1: CTA pairs and 4-warp gathers on long-K products
+    over large expert slices; see smoe.h)."""
+    _check(lib().smoe_set_gemm_policy(int(policy)))
 
 
 def smoe_selftest_wait_timeout(limit_us: int, stream=None):

@@ -1000,4 +1000,10 @@ int smoe_mlp_bwd(const smoe_mlp_desc* desc, const smoe_mlp_tensors* t, void* str
   return SMOE_OK;
 }
 
+int smoe_set_gemm_policy(int policy) {
+  if (policy != 0 && policy != 1) return api_fail(SMOE_ERR_INVALID_ARG, "gemm policy must be 0 or 1");
+  set_gemm_policy(policy);
+  return SMOE_OK;
+}
+
 }  // extern "C"

@@ -165,9 +165,12 @@ struct Tile {
 // linear tile L -> (expert, M tile, N tile); expert-major, then N tile, then M tile.
 // `off` = the expert offsets in global memory (validated by setup).
 // A pair's M tile spans 2 BM rows, of which CTA `rank` takes the rank-th BM.
+// Inside an expert the tiles go in panels of `pm` M tiles (the last panel may be
+// shorter): M tile fastest, then N tile, then panel, so that the tiles in flight
+// at once share fewer A rows (pm >= the expert's M tiles: one panel).
 template <bool PAIR = false>
 __device__ __forceinline__ Tile map_tile(const SharedCtl& c, const int32_t* off, int E, int nN,
-                                         int L, int rank = 0) {
+                                         int L, int rank = 0, int pm = 1 << 30) {
   int lo = 0, hi = E - 1;  // largest e with prefix[e] * nN <= L
   while (lo < hi) {
     const int mid = (lo + hi + 1) >> 1;
@@ -177,8 +180,13 @@ __device__ __forceinline__ Tile map_tile(const SharedCtl& c, const int32_t* off,
   t.e = lo;
   const int mt = c.prefix[lo + 1] - c.prefix[lo];
   const int lp = L - c.prefix[lo] * nN;
-  t.nb = lp / mt;
-  t.mb = lp % mt;
+  const int ph = pm < mt ? pm : mt;      // full panel height
+  const int pan = lp / (ph * nN);        // panel index
+  const int m0 = pan * ph;               // its first M tile
+  const int h = min(ph, mt - m0);        // its height
+  const int q = lp - pan * ph * nN;      // position inside the panel
+  t.nb = q / h;
+  t.mb = m0 + q % h;
   t.row0 = __ldg(off + lo) + t.mb * (PAIR ? 2 * BM : BM) + rank * BM;
   t.row_end = __ldg(off + lo + 1);
   return t;
@@ -344,7 +352,7 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
       Ring r;
       bool run = true;
       for (int L = first; run && L < total; L += stride) {
-        const Tile t = map_tile<PAIR>(c, g.offsets, g.E, nN, L / ks, rank);
+        const Tile t = map_tile<PAIR>(c, g.offsets, g.E, nN, L / ks, rank, g.panel_m);
         for (int kb = kb_lo(L), kb_end = kb_hi(L); kb < kb_end; ++kb) {
           if (!mbar_wait(&c.emptyA[r.s], r.ph ^ 1, abort_flag, g.err)) { run = false; break; }
           uint8_t* b_dst = sB + r.s * BSTAGE;
@@ -397,7 +405,7 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
     Ring r;
     bool run = true;
     for (int L = first; run && L < total; L += stride) {
-      const Tile tl = map_tile<PAIR>(c, g.offsets, g.E, nN, L / ks, rank);
+      const Tile tl = map_tile<PAIR>(c, g.offsets, g.E, nN, L / ks, rank, g.panel_m);
       const char* src[kRowsPer];
       uint32_t ok_rows = 0;
 #pragma unroll
@@ -536,7 +544,7 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
       const int buf = it & 1;
       if (two && buf != grp) continue;  // the other group's tile
       const uint32_t tph = (it >> 1) & 1;
-      const Tile t = map_tile<PAIR>(c, g.offsets, g.E, nN, L / ks, rank);
+      const Tile t = map_tile<PAIR>(c, g.offsets, g.E, nN, L / ks, rank, g.panel_m);
       if (!mbar_wait(&c.tfull[buf], tph, abort_flag, g.err)) break;
       tc_fence_after();
       const int i = t.row0 + r;
@@ -1662,6 +1670,12 @@ cudaError_t launch_dp(const CUtensorMap& tb, const CUtensorMap& td, int d_boxed,
 
 }  // namespace
 
+namespace {
+volatile int g_gemm_policy = 0;  // smoe_set_gemm_policy
+}  // namespace
+
+void set_gemm_policy(int policy) { g_gemm_policy = policy; }
+
 bool tc_supported() {
   int dev = 0, major = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return false;
@@ -1743,15 +1757,16 @@ cudaError_t launch_grouped_gemm_tc(const GroupedGemm& g, cudaStream_t s) {
   // SwiGLU's forward, whose epilogue (half-width tiles) is short and whose gather
   // then sets the pace (measured slower with 4 gather warps).
   const bool shortk = gather && !swiglu && g.K <= kShortK && g.ksplit <= 1;
-  // Long-K products over large expert slices (at least 2048 rows per expert on
-  // average, K >= 4096): TMA-fed ones and the activation-backward product run on
-  // CTA pairs (six-stage rings of 32 KB per CTA, half of B per CTA), gathered ones
-  // gather with 4 warps.  Measured on the Mixtral-shaped layer: down projection
-  // -5%, dx -8%, dA' -5%, up projection -5% (4 warps, one CTA; on pairs it was
-  // slower).  Smaller shapes keep the single-CTA kernels they were tuned with.
-  const bool big = g.ksplit <= 1 && g.K >= 4096 && (long long)g.num_rows >= 2048LL * g.E;
-  const bool pair = big && (!gather || g.epi == EPI_ACT_BWD);
-  const bool g128 = gather && !shortk && g.K >= 4096;
+  // Policy 1 (smoe_set_gemm_policy): long-K products over large expert slices
+  // (at least 2048 rows per expert on average, K >= 4096) run TMA-fed ones on CTA
+  // pairs (six-stage rings of 32 KB per CTA, half of B per CTA) and gather the
+  // others with 4 warps on one CTA.  Either policy walks an expert's tiles in
+  // panels of M tiles (map_tile): a wave of 148 CTAs then covers about 16 x 9
+  // tiles, whose A rows and weight columns are read by more tiles at once.
+  const bool big = g_gemm_policy == 1 && g.ksplit <= 1 && g.K >= 4096 &&
+                   (long long)g.num_rows >= 2048LL * g.E;
+  const bool pair = big && !gather;
+  const bool g128 = big && gather && !shortk;
   CUtensorMap ta, tb;
   cudaError_t e = rows_map(&ta, g.a, g.K, g.a_rows, g.lda, BM);  // unused when gathered
   if (e != cudaSuccess) return e;
@@ -1783,20 +1798,24 @@ cudaError_t launch_grouped_gemm_tc(const GroupedGemm& g, cudaStream_t s) {
   if (ld && need_h && out_map(&m.xh, g.aux_h, g.n_out, parts, g.num_rows, g.ld_aux_h) != cudaSuccess) ld = false;
   m.flags = (st ? kBoxStores : 0) | (ld ? kBoxLoads : 0);
   const int tm = pair ? 2 * BM : BM;  // rows per M tile
+  // Panels of 16 M tiles (8 on pairs): measured 33% fewer DRAM reads on the
+  // Mixtral-shaped down projection and 1.2% less time per step over 20 steps.
+  GroupedGemm gp = g;
+  gp.panel_m = pair ? 8 : 16;
   const long long tiles = (long long)(cdiv(g.num_rows, tm) + g.E) * nN * (g.ksplit > 1 ? g.ksplit : 1);
   if (g.ksplit > 1) {  // grouped A, plain store (checked above)
-    if (kmaj) return launch_g<false, true, false, false, true>(ta, tb, m, g, nN, tiles, s);
-    return launch_g<false, false, false, false, true>(ta, tb, m, g, nN, tiles, s);
+    if (kmaj) return launch_g<false, true, false, false, true>(ta, tb, m, gp, nN, tiles, s);
+    return launch_g<false, false, false, false, true>(ta, tb, m, gp, nN, tiles, s);
   }
   if (shortk) {
-    if (kmaj) return launch_g<true, true, false, false, false, true>(ta, tb, m, g, nN, tiles, s);
-    return launch_g<true, false, false, false, false, true>(ta, tb, m, g, nN, tiles, s);
+    if (kmaj) return launch_g<true, true, false, false, false, true>(ta, tb, m, gp, nN, tiles, s);
+    return launch_g<true, false, false, false, false, true>(ta, tb, m, gp, nN, tiles, s);
   }
 #define SMOE_LAUNCH_G(AG, KM, SW)                                                              \
-  (pair ? (g128 ? launch_g<AG, KM, SW, true, false, false, false, AG>(ta, tb, m, g, nN, tiles, s)        \
-                : launch_g<AG, KM, SW, true>(ta, tb, m, g, nN, tiles, s))                               \
-        : (g128 ? launch_g<AG, KM, SW, false, false, false, false, AG>(ta, tb, m, g, nN, tiles, s)       \
-                : launch_g<AG, KM, SW, false>(ta, tb, m, g, nN, tiles, s)))
+  (pair ? (g128 ? launch_g<AG, KM, SW, true, false, false, false, AG>(ta, tb, m, gp, nN, tiles, s)        \
+                : launch_g<AG, KM, SW, true>(ta, tb, m, gp, nN, tiles, s))                               \
+        : (g128 ? launch_g<AG, KM, SW, false, false, false, false, AG>(ta, tb, m, gp, nN, tiles, s)       \
+                : launch_g<AG, KM, SW, false>(ta, tb, m, gp, nN, tiles, s)))
   if (gather) {
     if (kmaj) return swiglu ? SMOE_LAUNCH_G(true, true, true) : SMOE_LAUNCH_G(true, true, false);
     return swiglu ? SMOE_LAUNCH_G(true, false, true) : SMOE_LAUNCH_G(true, false, false);
@@ -1840,11 +1859,10 @@ cudaError_t launch_dw_gemm_tc(const DwGemm& g_in, cudaStream_t s) {
   // Gated rows with B by TMA and at least two 128-column halves of M run on CTA
   // pairs: their six-stage rings keep more gathered stages in flight while the
   // gate pass holds stages back (measured 9% faster than one CTA on the
-  // Mixtral-shaped dW2).  Ungated products over large slices (at least 2048 rows
-  // per expert on average) do too, since the pair commits once to both CTAs
-  // (measured 2-3% faster on the Mixtral-shaped dW1 and dW2); smaller ones keep
-  // the single-CTA kernel.
-  const bool big = (long long)g.num_rows >= 2048LL * g.E;
+  // Mixtral-shaped dW2).  Under policy 1 ungated products over large slices (at
+  // least 2048 rows per expert on average) do too (2-3% faster on the
+  // Mixtral-shaped dW1 and dW2 in short runs below the power cap).
+  const bool big = g_gemm_policy == 1 && (long long)g.num_rows >= 2048LL * g.E;
   if ((sc || (ag && big)) && !bg && g.M > BM) {
     const int nMP = cdiv(g.M, 2 * BM);
     const long long ptiles = (long long)g.E * nMP * nN;

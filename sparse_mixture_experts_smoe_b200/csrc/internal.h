@@ -58,6 +58,7 @@ struct GroupedGemm {
   // raw fp32 sums to partial [ksplit, num_rows, n_out]; launch_splitk_reduce then
   // applies the gates and stores out
   int ksplit = 1;
+  int panel_m = 1 << 30;  // M tiles per raster panel of an expert's tile list (the tensor-core path)
   float* partial = nullptr;
   // fp8 = 1: a and b hold e4m3 codes (b K-major, b_kn = 0); the fp32 sums are
   // multiplied by row_scale[source row of A] and col_scale[e * NW + column]
@@ -164,6 +165,8 @@ cudaError_t launch_quantize_weights_fp8(const void* w, int E, int K, int N, uint
 
 // tcgen05 / TMEM path (bf16 only); *_supported() checks the device once.
 bool tc_supported();
+// Kernel-selection policy of the tensor-core GEMMs (smoe_set_gemm_policy).
+void set_gemm_policy(int policy);
 cudaError_t launch_grouped_gemm_tc(const GroupedGemm& g, cudaStream_t s);
 cudaError_t launch_dw_gemm_tc(const DwGemm& g, cudaStream_t s);
 

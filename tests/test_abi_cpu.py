@@ -242,3 +242,11 @@ def test_gated_parallel_linear_backward_adds_no_copy_of_x(grouped_in, fan_out):
         # the only [num_slots, K] buffer is the dx slot rows of a fan-out combine
         combine = a256(S * K * es) + a256(S * 4) if (not grouped_in and fan_out > 1) else 0
         assert plain == combine
+
+
+def test_gemm_policy_accepts_only_its_values():
+    L = smoe.lib()
+    assert L.smoe_set_gemm_policy(2) == -1 and b"policy" in L.smoe_last_error()
+    assert L.smoe_set_gemm_policy(-1) == -1
+    assert L.smoe_set_gemm_policy(1) == 0
+    assert L.smoe_set_gemm_policy(0) == 0

@@ -94,12 +94,21 @@ REDUCED = {
     # few enough tiles that the down projection splits its K (4 splits, ragged last K-block)
     "decode_t2_splitk_bf16": dict(kind="mlp", T=2, d=264, f=1000, E=8, k=2, dtype="bf16",
                                   act="swiglu"),
-    # K = 4096 over expert slices of 2200 rows (every token routed to both experts):
-    # the up projection gathers with 4 warps, dA' runs on CTA pairs with a 4-warp
-    # gather, dW1 and dW2 on the pair dW kernel (ragged pair tiles, a ragged N tile)
-    "long_k_pairs_bf16": dict(kind="mlp", T=2200, d=4096, f=200, E=2, k=2, dtype="bf16",
-                              act="swiglu"),
 }
+
+# K = 4096 over expert slices of 2200 rows (every token routed to both experts): under
+# GEMM policy 1 the up projection and dA' gather with 4 warps and dW1 and dW2 run on
+# the pair dW kernel (ragged pair tiles, a ragged N tile); policy 0 as a baseline
+LONG_K = dict(kind="mlp", T=2200, d=4096, f=200, E=2, k=2, dtype="bf16", act="swiglu")
+
+
+@pytest.mark.parametrize("policy", [0, 1])
+def test_mlp_long_k_policies(policy):
+    smoe.smoe_set_gemm_policy(policy)
+    try:
+        _check_full(LONG_K, make_mlp_inputs(LONG_K, seed=1, device="cuda"))
+    finally:
+        smoe.smoe_set_gemm_policy(0)
 
 
 @pytest.mark.parametrize("name", list(REDUCED))

@@ -178,17 +178,22 @@ def test_parallel_linear_gated_dw_narrow(mode):
 
 @pytest.mark.parametrize("mode", ["group2group", "scatter2group_fanout", "group2scatter_combine"])
 def test_parallel_linear_long_k_pairs(mode):
-    """K = 4096 over slices of at least 2048 rows per expert: the TMA-fed products
-    run on CTA pairs, the gathered ones gather with 4 warps, and the dW of a
-    gathered operand runs on the pair dW kernel; every element against the oracle
-    (ragged pair tiles and a ragged N tile)."""
+    """K = 4096 over slices of at least 2048 rows per expert under GEMM policy 1:
+    the TMA-fed products run on CTA pairs (tiles in panels), the gathered ones
+    gather with 4 warps, and the dW of a gathered operand runs on the pair dW
+    kernel; every element against the oracle (ragged pair tiles and a ragged N
+    tile)."""
     gated = mode == "group2scatter_combine"
     P = _problem(torch.bfloat16, mode, gated, seed=5, shape=dict(T=2200, k=2, K=4096, N=264, E=2))
-    y = smoe.parallel_linear_fwd(P["x"], P["w"], P["ss"], P["off"], P["fan_out"], P["gi"], P["go"],
-                                 P["gates"], P["ck"])
-    dx, dw, dg = smoe.parallel_linear_bwd(P["dy"], P["x"], P["w"], P["ss"], P["off"], P["fan_out"],
-                                          P["gi"], P["go"], P["gates"], P["ck"], want_dgates=gated)
-    torch.cuda.synchronize()
+    smoe.smoe_set_gemm_policy(1)
+    try:
+        y = smoe.parallel_linear_fwd(P["x"], P["w"], P["ss"], P["off"], P["fan_out"], P["gi"], P["go"],
+                                     P["gates"], P["ck"])
+        dx, dw, dg = smoe.parallel_linear_bwd(P["dy"], P["x"], P["w"], P["ss"], P["off"], P["fan_out"],
+                                              P["gi"], P["go"], P["gates"], P["ck"], want_dgates=gated)
+        torch.cuda.synchronize()
+    finally:
+        smoe.smoe_set_gemm_policy(0)
     assert smoe.smoe_check() == 0
     ss, off = P["ss"].cpu().numpy(), P["off"].cpu().numpy()
     assert np.diff(off).min() >= 2048
