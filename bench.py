@@ -539,10 +539,59 @@ def run_decode(args, world, rank):
         del st, inp, p, q, w1q, w2q
 
 
+def run_library_bar(args, world, rank):
+    """The six expert products of the Mixtral-shaped layer as dense batched products
+    with equal slices (8 experts x 4096 rows, i.e. perfectly balanced routing and
+    no gather), timed through torch.bmm (cuBLAS): a reference bar for the per-kernel
+    times of the benchmark, not part of the path.  Outputs are bf16 (the library's
+    weight gradients are fp32)."""
+    dev = torch.device("cuda", torch.cuda.current_device())
+    cfg = WORKLOADS[DEFAULT_WORKLOAD]
+    E, d, f = cfg["E"], cfg["d"], cfg["f"]
+    M = cfg["T"] * cfg["k"] // E
+    g = torch.Generator(device=dev)
+    g.manual_seed(rank)
+
+    def r(*shape):
+        return torch.randn(*shape, generator=g, device=dev, dtype=torch.bfloat16)
+
+    prods = {
+        "fwd_up": lambda: (r(E, M, d), r(E, d, 2 * f)),
+        "fwd_down": lambda: (r(E, M, f), r(E, f, d)),
+        "bwd_dA": lambda: (r(E, M, d), r(E, f, d).transpose(1, 2)),
+        "bwd_dx": lambda: (r(E, M, 2 * f), r(E, d, 2 * f).transpose(1, 2)),
+        "bwd_dW2": lambda: (r(E, M, f).transpose(1, 2), r(E, M, d)),
+        "bwd_dW1": lambda: (r(E, M, d).transpose(1, 2), r(E, M, 2 * f)),
+    }
+    for name, make in prods.items():
+        torch.cuda.empty_cache()
+        a, b = make()
+        for _ in range(args.warmup):
+            torch.bmm(a, b)
+        torch.cuda.synchronize()
+        barrier(world)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(args.steps):
+            torch.bmm(a, b)
+        e1.record()
+        torch.cuda.synchronize()
+        barrier(world)
+        ms = max_over_ranks(e0.elapsed_time(e1), world) / args.steps
+        fl = 2.0 * E * a.shape[1] * a.shape[2] * b.shape[2]
+        if rank == 0:
+            print(json.dumps({"sweep": "library", "product": name, "impl": "torch.bmm (cuBLAS), bf16 out",
+                              "shape": [E, a.shape[1], a.shape[2], b.shape[2]], "steps": args.steps,
+                              "ms": round(ms, 4), "tflops": round(fl / (ms / 1e3) / 1e12, 1)}), flush=True)
+        del a, b
+
+
 def run_sweep(args, world, rank):
     import sparse_mixture_experts_smoe_b200 as smoe
     if args.sweep == "decode":
         return run_decode(args, world, rank)
+    if args.sweep == "library":
+        return run_library_bar(args, world, rank)
     dev = torch.device("cuda", torch.cuda.current_device())
     peaks = load_peaks()
     names = list(SWEEPS) if args.sweep == "all" else [args.sweep]
@@ -794,7 +843,8 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--sweep", choices=["granularity", "sparsity", "dense", "decode", "all"], default=None,
+    ap.add_argument("--sweep", choices=["granularity", "sparsity", "dense", "decode", "library", "all"],
+                    default=None,
                     help="time the SMoE MLP over a set of (E, k, f) shapes instead of the benchmark line")
     ap.add_argument("--tokens", type=int, default=0,
                     help="override T (smaller cases for profiler captures; never a bench line)")

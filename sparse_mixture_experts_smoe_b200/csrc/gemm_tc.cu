@@ -95,16 +95,17 @@ __device__ __forceinline__ float fast_gelu_grad(float h) {
 // ---------------------------------------------------------------------------
 // Shared state, stage rings and the tile list
 // ---------------------------------------------------------------------------
-// The A and B operands have separate stage rings: a gathered operand (long
-// cp.async latency) gets 6 stages of 16 KB while the TMA-fed one gets 3 of 32 KB;
-// kernels fed only by TMA use 4 + 4.  Either way the rings fill kRingBytes.
+// The grouped-M kernel keeps both operands of a stage in one ring (4 stages of
+// 48 KB, 6 of 32 KB per CTA of a pair); the dW kernel keeps them in two rings of 4
+// stages (16 KB A + 32 KB B) that advance together.  Either way the rings fill
+// kRingBytes.
 constexpr int kMaxStages = 8;
 constexpr int IDX_STAGES = 8;            // slot-index ring of the dW gathers
 constexpr int kRingBytes = 192 * 1024;
 
 struct SharedCtl {
-  uint64_t fullA[kMaxStages], emptyA[kMaxStages];
-  uint64_t fullB[kMaxStages], emptyB[kMaxStages];
+  uint64_t fullA[kMaxStages], emptyA[kMaxStages];  // emptyA frees a stage of both rings
+  uint64_t fullB[kMaxStages];
   uint64_t tfull[2], tempty[2];
   uint64_t pfull[kMaxStages];   // pair leader: the other CTA's stage s has landed
   uint64_t ifull[IDX_STAGES];   // index ring: written by warp 2
@@ -210,7 +211,6 @@ __device__ __forceinline__ void setup(SharedCtl& c, const int32_t* offsets, int 
     }
     for (int s = 0; s < SB; ++s) {
       mbar_init(&c.fullB[s], b_arrivals);
-      mbar_init(&c.emptyB[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&c.tfull[b], 1);
@@ -1145,8 +1145,11 @@ dw_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
                   const __grid_constant__ CUtensorMap tmD, const DwGemm g, int nM, int nN,
                   int d_boxed) {
   // four stages of each operand (16 KB A + 32 KB B): a deeper A ring for the gather
-  // at the cost of a 3-stage B ring measured about 1% slower
+  // at the cost of a 3-stage B ring measured about 1% slower.  The two rings advance
+  // together, so one empty barrier per stage (emptyA) frees both: one MMA commit per
+  // stage instead of two.
   constexpr int SA = 4, SB = 4;
+  static_assert(SA == SB, "the A and B rings share their empty barriers");
   static_assert(SA * A_BYTES + SB * B_BYTES <= kRingBytes, "stage rings exceed their budget");
   static_assert(!A_SCALE || (A_GATHER && kDefer < SA), "gated rows are gathered, deferred < ring");
   extern __shared__ uint8_t smem_raw[];
@@ -1190,7 +1193,7 @@ dw_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
             ra.next(SA);
           }
           if (!B_GATHER) {  // 64 rows x 256 N-columns: four slabs
-            if (!mbar_wait(&c.emptyB[rb.s], rb.ph ^ 1, abort_flag, g.err)) { run = false; break; }
+            if (!mbar_wait(&c.emptyA[rb.s], rb.ph ^ 1, abort_flag, g.err)) { run = false; break; }
             uint8_t* b_dst = sB + rb.s * B_BYTES;
             mbar_expect_tx(&c.fullB[rb.s], B_BYTES);
 #pragma unroll
@@ -1237,7 +1240,7 @@ dw_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
           ra.next(SA);
         }
         if (B_GATHER) {
-          if (!mbar_wait(&c.emptyB[rb.s], rb.ph ^ 1, abort_flag, g.err)) { run = false; break; }
+          if (!mbar_wait(&c.emptyA[rb.s], rb.ph ^ 1, abort_flag, g.err)) { run = false; break; }
           gb.issue(smem_u32(sB + rb.s * B_BYTES), x.idx[ri.s][1], reinterpret_cast<const bf16*>(g.b),
                    g.ldb, nb * BN, g.N, t);
           cp_async_arrive(&c.fullB[rb.s]);
@@ -1299,8 +1302,7 @@ dw_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
             for (int kk = 0; kk < BK / 16; ++kk)
               umma_bf16(d_tmem, desc_mnmajor(a_addr + kk * 2048), desc_mnmajor(b_addr + kk * 2048),
                         idesc, (kb | kk) != 0);
-            umma_commit(&c.emptyA[ra.s]);
-            umma_commit(&c.emptyB[rb.s]);
+            umma_commit(&c.emptyA[ra.s]);  // frees the stage of both rings
           }
           if (!kGather) __syncwarp();
           ra.next(SA);
