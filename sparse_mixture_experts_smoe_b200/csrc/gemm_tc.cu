@@ -139,7 +139,10 @@ constexpr int kBoxBytes = 32 * 64;
 constexpr int kWarpStaging = 32 * kSlotBytes;  // 13 x 512: boxes stay 512-byte aligned
 static_assert(3 * kBoxBytes <= kWarpStaging && kWarpStaging % 512 == 0, "staging layout");
 constexpr int kStagingBytes = 4 * kWarpStaging;
-enum : int { kBoxStores = 1, kBoxLoads = 2 };  // grouped-epilogue box modes (launch flags)
+// Launch flags of the grouped kernel: epilogue box stores / box loads, and B (an
+// MN-major weight operand) through the slab view (one TMA load per run of
+// 64-column slabs instead of one per slab).
+enum : int { kBoxStores = 1, kBoxLoads = 2, kSlabB = 4 };
 
 constexpr size_t kCtlBytes = (sizeof(SharedCtl) + 1023) / 1024 * 1024;
 constexpr size_t kGroupedSmem = 1024 + (size_t)kRingBytes + kCtlBytes + kStagingBytes;
@@ -367,6 +370,10 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
             if (PAIR) tma_load_3d_pair(dst, m, full_cl, c0, c1, c2);
             else tma_load_3d(dst, m, &c.fullA[r.s], c0, c1, c2);
           };
+          auto load4 = [&](void* dst, const CUtensorMap* m, int c0, int c1, int c2, int c3) {
+            if (PAIR) tma_load_4d_pair(dst, m, full_cl, c0, c1, c2, c3);
+            else tma_load_4d(dst, m, &c.fullA[r.s], c0, c1, c2, c3);
+          };
           if (rank == 0)
             mbar_expect_tx(&c.fullA[r.s], (PAIR ? 2 : 1) * (BSTAGE + (A_GATHER ? 0 : A_BYTES)));
           if (!A_GATHER) load2(sA + r.s * A_BYTES, &tmA, kb * BKE, t.row0);
@@ -375,6 +382,17 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA,
             load3(b_dst + BNo * 128, &tmB, kb * BKE, g.n_out + t.nb * BNo, t.e);
           } else if (B_KMAJOR) {  // rows of W[e] = output columns; a pair's CTA takes its half
             load3(b_dst, &tmB, kb * BKE, t.nb * BN + (PAIR ? rank * (BN / 2) : 0), t.e);
+          } else if (box_flags & kSlabB) {
+            // slab view: one load per contiguous column run (128 columns for SwiGLU's
+            // gate and up halves and for a pair's half, else the tile's 256)
+            constexpr int kRun = (PAIR || SWIGLU_FWD) ? BN / 2 : BN;
+#pragma unroll
+            for (int q = 0; q < BSTAGE / (kRun * BK * 2); ++q) {
+              const int lc = (PAIR ? rank * (BN / 2) : 0) + kRun * q;  // column within the B tile
+              const int col = SWIGLU_FWD ? (lc < BNo ? t.nb * BNo + lc : g.n_out + t.nb * BNo + lc - BNo)
+                                         : t.nb * BN + lc;
+              load4(b_dst + q * (kRun * BK * 2), &tmB, 0, kb * BK, col / 64, t.e);
+            }
           } else {
             // 64-column slabs; SwiGLU's tile is BNo gate columns then BNo up columns
             // (a pair: the gate half in CTA 0, the up half in CTA 1)
@@ -1143,7 +1161,7 @@ template <bool A_GATHER, bool B_GATHER, bool TRANS_OUT, bool A_SCALE = false>
 __global__ void __launch_bounds__(kDwThreads, 1)
 dw_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                   const __grid_constant__ CUtensorMap tmD, const DwGemm g, int nM, int nN,
-                  int d_boxed) {
+                  int d_boxed, int slabs) {
   // four stages of each operand (16 KB A + 32 KB B): a deeper A ring for the gather
   // at the cost of a 3-stage B ring measured about 1% slower.  The two rings advance
   // together, so one empty barrier per stage (emptyA) frees both: one MMA commit per
@@ -1188,17 +1206,25 @@ dw_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
             if (!mbar_wait(&c.emptyA[ra.s], ra.ph ^ 1, abort_flag, g.err)) { run = false; break; }
             uint8_t* a_dst = sA + ra.s * A_BYTES;
             mbar_expect_tx(&c.fullA[ra.s], A_BYTES);
-            tma_load_2d(a_dst, &tmA, &c.fullA[ra.s], mb * BM, rk);
-            tma_load_2d(a_dst + 8192, &tmA, &c.fullA[ra.s], mb * BM + 64, rk);
+            if (slabs & 1) {  // slab view {64, rows, slabs}: both slabs in one load
+              tma_load_3d(a_dst, &tmA, &c.fullA[ra.s], 0, rk, mb * (BM / 64));
+            } else {
+              tma_load_2d(a_dst, &tmA, &c.fullA[ra.s], mb * BM, rk);
+              tma_load_2d(a_dst + 8192, &tmA, &c.fullA[ra.s], mb * BM + 64, rk);
+            }
             ra.next(SA);
           }
           if (!B_GATHER) {  // 64 rows x 256 N-columns: four slabs
             if (!mbar_wait(&c.emptyA[rb.s], rb.ph ^ 1, abort_flag, g.err)) { run = false; break; }
             uint8_t* b_dst = sB + rb.s * B_BYTES;
             mbar_expect_tx(&c.fullB[rb.s], B_BYTES);
+            if (slabs & 2) {  // slab view: the four slabs in one load
+              tma_load_3d(b_dst, &tmB, &c.fullB[rb.s], 0, rk, nb * (BN / 64));
+            } else {
 #pragma unroll
-            for (int slab = 0; slab < 4; ++slab)
-              tma_load_2d(b_dst + slab * 8192, &tmB, &c.fullB[rb.s], nb * BN + 64 * slab, rk);
+              for (int slab = 0; slab < 4; ++slab)
+                tma_load_2d(b_dst + slab * 8192, &tmB, &c.fullB[rb.s], nb * BN + 64 * slab, rk);
+            }
             rb.next(SB);
           }
         }
@@ -1361,7 +1387,7 @@ dw_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
 template <bool A_SCALE, bool TRANS_OUT>
 __global__ void __launch_bounds__(kDwThreads, 1)
 dw_pair_tc_kernel(const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmD,
-                  const DwGemm g, int nMP, int nN, int d_boxed) {
+                  const DwGemm g, int nMP, int nN, int d_boxed, int slabs) {
   constexpr int STAGES = 6;
   constexpr int BH = B_BYTES / 2;  // this CTA's half of B per stage (16 KB)
   static_assert(STAGES * (A_BYTES + BH) <= kRingBytes && STAGES <= kMaxStages && kDefer < STAGES,
@@ -1405,8 +1431,12 @@ dw_pair_tc_kernel(const __grid_constant__ CUtensorMap tmB, const __grid_constant
           if (rank == 0) mbar_expect_tx(&c.fullA[r.s], 2 * BH);
           uint8_t* b_dst = sB + r.s * BH;
           const int col = nb * BN + rank * (BN / 2);
-          tma_load_2d_pair(b_dst, &tmB, full_cl, col, r_begin + kb * BK);
-          tma_load_2d_pair(b_dst + 8192, &tmB, full_cl, col + 64, r_begin + kb * BK);
+          if (slabs & 2) {  // slab view: this CTA's two slabs in one load
+            tma_load_3d_pair(b_dst, &tmB, full_cl, 0, r_begin + kb * BK, col / 64);
+          } else {
+            tma_load_2d_pair(b_dst, &tmB, full_cl, col, r_begin + kb * BK);
+            tma_load_2d_pair(b_dst + 8192, &tmB, full_cl, col + 64, r_begin + kb * BK);
+          }
           r.next(STAGES);
         }
       }
@@ -1558,6 +1588,18 @@ cudaError_t rows_map(CUtensorMap* m, const void* base, int cols, int rows, int l
   return make_map(m, base, 2, dims, strides, box);
 }
 
+// Slab view of [rows, ld] bf16 rows whose first `cols` columns (a multiple of 64)
+// are used: dims {64, rows, cols / 64}, strides {ld * 2, 128}; a box is `nslab`
+// slabs of 64 columns x box_rows rows, landing slab after slab (8 KB per 64 rows).
+cudaError_t slab_map(CUtensorMap* m, const void* base, int cols, int rows, int ld, uint32_t box_rows,
+                     uint32_t nslab) {
+  if (cols % 64) return cudaErrorInvalidValue;
+  const uint64_t dims[3] = {64, (uint64_t)(rows > 0 ? rows : 1), (uint64_t)cols / 64};
+  const uint64_t strides[2] = {(uint64_t)ld * 2, 128};
+  const uint32_t box[3] = {64, box_rows, nslab};
+  return make_map(m, base, 3, dims, strides, box);
+}
+
 // Output map of the grouped epilogue's boxed stores: rows of [rows, ld] whose
 // first parts * n_out columns hold `parts` blocks of n_out (SwiGLU's gate and up
 // halves), as dims {n_out, parts, rows} so that a box never crosses n_out.
@@ -1625,19 +1667,19 @@ cudaError_t launch_g(const CUtensorMap& ta, const CUtensorMap& tb, const EpiMaps
 
 template <bool AG, bool BG, bool TR, bool SC = false>
 cudaError_t launch_d(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& td,
-                     int d_boxed, const DwGemm& g, int nM, int nN, int grid, cudaStream_t s) {
+                     int d_boxed, int slabs, const DwGemm& g, int nM, int nN, int grid, cudaStream_t s) {
   auto kern = dw_gemm_tc_kernel<AG, BG, TR, SC>;
   cudaError_t e = prep(kern, kDwSmem);
   if (e != cudaSuccess) return e;
-  kern<<<grid, kDwThreads, kDwSmem, s>>>(ta, tb, td, g, nM, nN, d_boxed);
+  kern<<<grid, kDwThreads, kDwSmem, s>>>(ta, tb, td, g, nM, nN, d_boxed, slabs);
   return cudaGetLastError();
 }
 
 // The pair dW kernel on as many 2-CTA clusters as the device holds at once (at
 // most one per tile pair).
 template <bool SC, bool TR>
-cudaError_t launch_dp(const CUtensorMap& tb, const CUtensorMap& td, int d_boxed, const DwGemm& g,
-                      int nMP, int nN, long long tiles, cudaStream_t s) {
+cudaError_t launch_dp(const CUtensorMap& tb, const CUtensorMap& td, int d_boxed, int slabs,
+                      const DwGemm& g, int nMP, int nN, long long tiles, cudaStream_t s) {
   auto kern = dw_pair_tc_kernel<SC, TR>;
   cudaError_t e = prep(kern, kDwSmem);
   if (e != cudaSuccess) return e;
@@ -1665,7 +1707,7 @@ cudaError_t launch_dp(const CUtensorMap& tb, const CUtensorMap& td, int d_boxed,
   const long long pairs = tiles < max_clusters ? tiles : max_clusters;
   if (pairs <= 0) return cudaSuccess;
   cfg.gridDim = dim3((unsigned)(2 * pairs), 1, 1);
-  e = cudaLaunchKernelEx(&cfg, kern, tb, td, g, nMP, nN, d_boxed);
+  e = cudaLaunchKernelEx(&cfg, kern, tb, td, g, nMP, nN, d_boxed, slabs);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
@@ -1773,12 +1815,20 @@ cudaError_t launch_grouped_gemm_tc(const GroupedGemm& g, cudaStream_t s) {
   cudaError_t e = rows_map(&ta, g.a, g.K, g.a_rows, g.lda, BM);  // unused when gathered
   if (e != cudaSuccess) return e;
   const bool kmaj = g.b_kn == 0;
+  // The slab view needs whole 64-column slabs (and SwiGLU's up half to start on one):
+  // it never reaches past a row, so every element it addresses is in the tensor.
+  const bool slab = !kmaj && g.NW % 64 == 0 && (!swiglu || g.n_out % 64 == 0);
   if (kmaj) {  // W[e] is [NW, K]: dims {K, NW, E}
     const uint64_t dims[3] = {(uint64_t)g.K, (uint64_t)g.NW, (uint64_t)g.E};
     const uint64_t str[2] = {(uint64_t)g.K * 2, (uint64_t)g.NW * g.K * 2};
     // (SwiGLU's forward loads its gate and up rows as two half-height boxes)
     const uint32_t box[3] = {64, (uint32_t)((pair || swiglu) ? BN / 2 : BN), 1};
     e = make_map(&tb, g.b, 3, dims, str, box);
+  } else if (slab) {  // W[e] is [K, NW] seen as slabs: dims {64, K, NW / 64, E}
+    const uint64_t dims[4] = {64, (uint64_t)g.K, (uint64_t)g.NW / 64, (uint64_t)g.E};
+    const uint64_t str[3] = {(uint64_t)g.NW * 2, 128, (uint64_t)g.K * g.NW * 2};
+    const uint32_t box[4] = {64, BK, (uint32_t)((pair || swiglu) ? 2 : 4), 1};
+    e = make_map(&tb, g.b, 4, dims, str, box);
   } else {  // W[e] is [K, NW]: dims {NW, K, E}
     const uint64_t dims[3] = {(uint64_t)g.NW, (uint64_t)g.K, (uint64_t)g.E};
     const uint64_t str[2] = {(uint64_t)g.NW * 2, (uint64_t)g.K * g.NW * 2};
@@ -1798,7 +1848,7 @@ cudaError_t launch_grouped_gemm_tc(const GroupedGemm& g, cudaStream_t s) {
   bool ld = g.epi == EPI_ACT_BWD && g.aux_a_mode == ROWS_GROUPED && !swiglu;
   if (ld && out_map(&m.xa, g.aux_a, g.n_out, 1, g.num_rows, g.ld_aux_a) != cudaSuccess) ld = false;
   if (ld && need_h && out_map(&m.xh, g.aux_h, g.n_out, parts, g.num_rows, g.ld_aux_h) != cudaSuccess) ld = false;
-  m.flags = (st ? kBoxStores : 0) | (ld ? kBoxLoads : 0);
+  m.flags = (st ? kBoxStores : 0) | (ld ? kBoxLoads : 0) | (slab ? kSlabB : 0);
   const int tm = pair ? 2 * BM : BM;  // rows per M tile
   // Panels of 16 M tiles (8 on pairs): measured 33% fewer DRAM reads on the
   // Mixtral-shaped down projection and 1.2% less time per step over 20 steps.
@@ -1843,10 +1893,19 @@ cudaError_t launch_dw_gemm_tc(const DwGemm& g_in, cudaStream_t s) {
   // gated rows: the gate multiplies the A operand as it is gathered (a grouped A
   // is then gathered row by row)
   const bool sc = g.row_gates != nullptr;
+  // A product with both operands fed by TMA and whole 64-column slabs uses the slab
+  // view {64, rows, slabs}: one load per stage and operand instead of one per slab
+  // (the view never reaches past a row).  With a gathered operand the gather sets
+  // the pace, and the Mixtral-shaped dW measured 1% slower with the slab view.
+  const bool pair_b = (sc || (ag && g_gemm_policy == 1 && (long long)g.num_rows >= 2048LL * g.E)) &&
+                      !bg && g.M > BM;  // the pair kernel below (half of B per CTA)
+  const int slabs = (!ag && !sc && !bg && g.M % 64 == 0 && g.N % 64 == 0) ? 3 : 0;
   CUtensorMap ta, tb;
-  cudaError_t e = rows_map(&ta, g.a, g.M, g.a_rows, g.lda, BK);  // unused when gathered
+  cudaError_t e = (slabs & 1) ? slab_map(&ta, g.a, g.M, g.a_rows, g.lda, BK, 2)
+                              : rows_map(&ta, g.a, g.M, g.a_rows, g.lda, BK);  // unused when gathered
   if (e != cudaSuccess) return e;
-  e = rows_map(&tb, g.b, g.N, g.b_rows, g.ldb, BK);
+  e = (slabs & 2) ? slab_map(&tb, g.b, g.N, g.b_rows, g.ldb, BK, pair_b ? 2 : 4)
+                  : rows_map(&tb, g.b, g.N, g.b_rows, g.ldb, BK);
   if (e != cudaSuccess) return e;
   // fp32 dW as [E, rows, cols] with 32 x 32 boxes: rows = M, cols = N, or the
   // transpose when the kernel computes dW^T
@@ -1864,19 +1923,18 @@ cudaError_t launch_dw_gemm_tc(const DwGemm& g_in, cudaStream_t s) {
   // Mixtral-shaped dW2).  Under policy 1 ungated products over large slices (at
   // least 2048 rows per expert on average) do too (2-3% faster on the
   // Mixtral-shaped dW1 and dW2 in short runs below the power cap).
-  const bool big = g_gemm_policy == 1 && (long long)g.num_rows >= 2048LL * g.E;
-  if ((sc || (ag && big)) && !bg && g.M > BM) {
+  if (pair_b) {
     const int nMP = cdiv(g.M, 2 * BM);
     const long long ptiles = (long long)g.E * nMP * nN;
     if (!sc)
-      return trans ? launch_dp<false, true>(tb, td, d_boxed, g, nMP, nN, ptiles, s)
-                   : launch_dp<false, false>(tb, td, d_boxed, g, nMP, nN, ptiles, s);
-    return trans ? launch_dp<true, true>(tb, td, d_boxed, g, nMP, nN, ptiles, s)
-                 : launch_dp<true, false>(tb, td, d_boxed, g, nMP, nN, ptiles, s);
+      return trans ? launch_dp<false, true>(tb, td, d_boxed, slabs, g, nMP, nN, ptiles, s)
+                   : launch_dp<false, false>(tb, td, d_boxed, slabs, g, nMP, nN, ptiles, s);
+    return trans ? launch_dp<true, true>(tb, td, d_boxed, slabs, g, nMP, nN, ptiles, s)
+                 : launch_dp<true, false>(tb, td, d_boxed, slabs, g, nMP, nN, ptiles, s);
   }
   const long long tiles = (long long)g.E * nM * nN;
   const int grid = (int)(tiles < num_sms() ? tiles : num_sms());
-#define SMOE_LAUNCH_D(AG, BG, TR, SC) launch_d<AG, BG, TR, SC>(ta, tb, td, d_boxed, g, nM, nN, grid, s)
+#define SMOE_LAUNCH_D(AG, BG, TR, SC) launch_d<AG, BG, TR, SC>(ta, tb, td, d_boxed, slabs, g, nM, nN, grid, s)
   if (sc) {
     if (bg) return SMOE_LAUNCH_D(true, true, false, true);
     return trans ? SMOE_LAUNCH_D(true, false, true, true) : SMOE_LAUNCH_D(true, false, false, true);

@@ -207,3 +207,30 @@ def test_parallel_linear_long_k_pairs(mode):
     assert_close("dw", dw, ref["dw"], torch.bfloat16)
     if gated:
         assert_close("dgates", dg, ref["dg"], torch.bfloat16)
+
+
+@pytest.mark.parametrize("mode", list(MODES))
+@pytest.mark.parametrize("gated", [False, True])
+def test_parallel_linear_slab_shapes(mode, gated):
+    """K and N multiples of 64: the MN-major weight and dW operands load through the
+    slab view (one TMA load per run of 64-column slabs); every element against the
+    oracle, with a ragged last N tile (N = 320) and an empty expert."""
+    P = _problem(torch.bfloat16, mode, gated, seed=7, shape=dict(T=300, k=2, K=256, N=320, E=5))
+    y = smoe.parallel_linear_fwd(P["x"], P["w"], P["ss"], P["off"], P["fan_out"], P["gi"], P["go"],
+                                 P["gates"], P["ck"])
+    dx, dw, dg = smoe.parallel_linear_bwd(P["dy"], P["x"], P["w"], P["ss"], P["off"], P["fan_out"],
+                                          P["gi"], P["go"], P["gates"], P["ck"], want_dgates=gated)
+    torch.cuda.synchronize()
+    assert smoe.smoe_check() == 0
+    ss, off = P["ss"].cpu().numpy(), P["off"].cpu().numpy()
+    gts = None if P["gates"] is None else P["gates"].cpu().double().numpy()
+    ref_y = oracle.pl_fwd(P["x"].cpu(), P["w"].cpu(), ss, off, P["fan_out"], P["gi"], P["go"], gts,
+                          P["ck"])
+    assert_close("y", y, ref_y, torch.bfloat16)
+    ref = oracle.pl_bwd(P["dy"].cpu(), P["x"].cpu(), P["w"].cpu(), ss, off, P["fan_out"], P["gi"],
+                        P["go"], gts, P["ck"], want_dg=gated)
+    assert_close("dx", dx, ref["dx"], torch.bfloat16)
+    assert_close("dw", dw, ref["dw"], torch.bfloat16)
+    assert np.all(dw[3].cpu().numpy() == 0.0)
+    if gated:
+        assert_close("dgates", dg, ref["dg"], torch.bfloat16)
