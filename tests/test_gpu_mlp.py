@@ -79,10 +79,10 @@ def test_tiny_fp32_gelu_full():
 REDUCED = {
     "gelu_bf16": dict(kind="mlp", T=300, d=264, f=392, E=6, k=2, dtype="bf16", act="gelu"),
     "swiglu_bf16": dict(kind="mlp", T=300, d=264, f=200, E=6, k=2, dtype="bf16", act="swiglu"),
-    # whole 64-column slabs everywhere: MN-major weights and dW operands load through
-    # the slab view (SwiGLU's last gate run crosses into the up half, a 3-slab dW2 tile)
-    "swiglu_bf16_slabs": dict(kind="mlp", T=300, d=256, f=192, E=6, k=2, dtype="bf16", act="swiglu"),
-    "gelu_bf16_slabs": dict(kind="mlp", T=300, d=320, f=448, E=5, k=2, dtype="bf16", act="gelu"),
+    # whole 64-column slabs and K = 4096 for the up projection: its MN-major weights
+    # load through the slab view (SwiGLU's last gate run crosses into the up half)
+    "swiglu_bf16_slabs": dict(kind="mlp", T=300, d=4096, f=192, E=6, k=2, dtype="bf16", act="swiglu"),
+    "gelu_bf16_slabs": dict(kind="mlp", T=300, d=4096, f=448, E=5, k=2, dtype="bf16", act="gelu"),
     "swiglu_bf16_zipf": dict(kind="mlp", T=257, d=136, f=128, E=16, k=4, dtype="bf16",
                              act="swiglu", zipf_s=1.2, n_empty=3),
     "swiglu_f32": dict(kind="mlp", T=200, d=72, f=136, E=4, k=2, dtype="f32", act="swiglu"),

@@ -212,10 +212,11 @@ def test_parallel_linear_long_k_pairs(mode):
 @pytest.mark.parametrize("mode", list(MODES))
 @pytest.mark.parametrize("gated", [False, True])
 def test_parallel_linear_slab_shapes(mode, gated):
-    """K and N multiples of 64: the MN-major weight and dW operands load through the
-    slab view (one TMA load per run of 64-column slabs); every element against the
-    oracle, with a ragged last N tile (N = 320) and an empty expert."""
-    P = _problem(torch.bfloat16, mode, gated, seed=7, shape=dict(T=300, k=2, K=256, N=320, E=5))
+    """K = 4096 and N a multiple of 64: the MN-major weights (forward) and both
+    operands of a TMA-fed dW load through the slab view (one TMA load per run of
+    64-column slabs); every element against the oracle, with a ragged last N tile
+    (N = 320) and an empty expert."""
+    P = _problem(torch.bfloat16, mode, gated, seed=7, shape=dict(T=300, k=2, K=4096, N=320, E=5))
     y = smoe.parallel_linear_fwd(P["x"], P["w"], P["ss"], P["off"], P["fan_out"], P["gi"], P["go"],
                                  P["gates"], P["ck"])
     dx, dw, dg = smoe.parallel_linear_bwd(P["dy"], P["x"], P["w"], P["ss"], P["off"], P["fan_out"],
