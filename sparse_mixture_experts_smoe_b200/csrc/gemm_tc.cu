@@ -21,8 +21,9 @@
 // tcgen05.mma (kind::f16, bf16 in, fp32 accumulate) issued by one thread.
 //
 // Grouped-M kernel (forward, dx): persistent CTAs walk a tile list built from the
-// expert offsets (expert-major, then N tile, then M tile, so the CTAs of one wave
-// share the expert's input rows in L2).  Warp roles: warp 0 = TMA producer,
+// expert offsets (expert-major; inside an expert, panels of M tiles walked M tile
+// first, then N tile, so that the CTAs of one wave share input rows and weight
+// columns in L2).  Warp roles: warp 0 = TMA producer,
 // warp 1 = MMA issuer and tensor-memory owner, warps 4-7 = epilogue (thread r owns
 // accumulator row r), warps 8-15 = row gather of a scattered operand (without a
 // gather, warps 8-11 are a second epilogue group for the scaled store).  Two
@@ -166,7 +167,7 @@ struct Tile {
   int e, mb, nb, row0, row_end;
 };
 
-// linear tile L -> (expert, M tile, N tile); expert-major, then N tile, then M tile.
+// linear tile L -> (expert, M tile, N tile); expert-major, then panel, N tile, M tile.
 // `off` = the expert offsets in global memory (validated by setup).
 // A pair's M tile spans 2 BM rows, of which CTA `rank` takes the rank-th BM.
 // Inside an expert the tiles go in panels of `pm` M tiles (the last panel may be
