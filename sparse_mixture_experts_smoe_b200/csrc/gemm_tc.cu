@@ -1820,8 +1820,8 @@ cudaError_t launch_grouped_gemm_tc(const GroupedGemm& g, cudaStream_t s) {
   // it never reaches past a row, so every element it addresses is in the tensor.
   // Used for long K only: the Mixtral-shaped down projection (K = 14336) measured 3%
   // faster with it, while the fine-grained sweep's products (K = 512-2048) measured up
-  // to 6% slower.
-  const bool slab = !kmaj && g.K >= 4096 && g.NW % 64 == 0 && (!swiglu || g.n_out % 64 == 0);
+  // to 6% slower.  Single CTAs only: CTA pairs (policy 1) keep one load per slab.
+  const bool slab = !kmaj && !pair && g.K >= 4096 && g.NW % 64 == 0 && (!swiglu || g.n_out % 64 == 0);
   if (kmaj) {  // W[e] is [NW, K]: dims {K, NW, E}
     const uint64_t dims[3] = {(uint64_t)g.K, (uint64_t)g.NW, (uint64_t)g.E};
     const uint64_t str[2] = {(uint64_t)g.K * 2, (uint64_t)g.NW * g.K * 2};
