@@ -33,3 +33,24 @@ def test_hbm_bytes_follow_the_layer_dtype():
         # combine: every slot row (layer dtype) and its grouped row index read, y written
         assert b["combine.y"] == S * d * es + S * 4 + T * d * es
         assert b["combine.dx"] == b["combine.y"] + S * 8
+
+
+def test_measured_traffic_needs_the_captured_source(tmp_path, monkeypatch):
+    """roofline.traffic comes from the committed ncu table only while the kernel source
+    is the one the counters were taken on (its SHA-256 in the row); any other source,
+    workload or kernel gives null."""
+    import hashlib
+    src = tmp_path / "gemm_tc.cu"
+    src.write_text("// kernels\n")
+    sha = hashlib.sha256(src.read_bytes()).hexdigest()
+    table = tmp_path / "traffic.md"
+    table.write_text("| workload | kernel | read bytes | write bytes | sha | algorithmic |\n|---|---|---|---|---|---|\n"
+                     f"| wl | gemm.bwd_dW1 | 5000 | 300 | {sha} | x |\n")
+    monkeypatch.setattr(bench, "KERNEL_SOURCE", str(src))
+    monkeypatch.setattr(bench, "TRAFFIC_TABLE", str(table))
+    assert bench.measured_traffic("gemm.bwd_dW1", "wl") == 5300
+    assert bench.measured_traffic("gemm.bwd_dW2", "wl") is None
+    assert bench.measured_traffic("gemm.bwd_dW1", "other") is None
+    src.write_text("// kernels, changed\n")
+    assert bench.measured_traffic("gemm.bwd_dW1", "wl") is None
+
